@@ -1,0 +1,192 @@
+"""CPU oracle of the forward MoE layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product (``combine_device_top_b200``)
+never imports it and shares no code with it.
+
+The arithmetic lives in ``mok_oracle.c`` (plain C, double precision, compiled
+with gcc); this file is ctypes marshalling plus small conveniences.  Each C
+function cites the passage of the pages it follows.
+
+Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
+against brute force, closed forms, invariants and textbook special cases.
+The MXFP8 emulation is pinned by hand-computed bytes in ``tests/golden/``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from functools import lru_cache
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRCS = [os.path.join(_HERE, "mok_oracle.c"), os.path.join(_HERE, "mxfp8_oracle.c")]
+_SO = os.path.join(_HERE, "liboracle.so")
+CFLAGS = ["-O3", "-march=x86-64-v3", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` (gcc, OpenMP) next to the sources."""
+    srcs = [s for s in _SRCS if os.path.exists(s)]
+    newest = max(os.path.getmtime(s) for s in srcs)
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < newest:
+        tmp = _SO + ".tmp"
+        subprocess.check_call(["gcc", *CFLAGS, *srcs, "-o", tmp, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+@lru_cache(maxsize=1)
+def lib():
+    L = ctypes.CDLL(build())
+    i32, vp = ctypes.c_int, ctypes.c_void_p
+    L.oracle_topk_gates.argtypes = [vp, i32, i32, i32, vp, vp]
+    L.oracle_schedule.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.oracle_gather.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+    L.oracle_expert_ffn.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+    L.oracle_combine.argtypes = [vp, vp, i32, i32, i32, vp]
+    L.oracle_moe_forward.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.oracle_num_threads.argtypes = []
+    L.oracle_set_num_threads.argtypes = [i32]
+    L.oracle_set_num_threads.restype = None
+    if hasattr(L, "oracle_mxfp8_quantize"):
+        L.oracle_mxfp8_quantize.argtypes = [vp, ctypes.c_int64, vp, vp]
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_mxfp8_expert_ffn.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    for name in ("oracle_topk_gates", "oracle_schedule", "oracle_gather", "oracle_expert_ffn",
+                 "oracle_combine", "oracle_moe_forward", "oracle_num_threads"):
+        getattr(L, name).restype = ctypes.c_int
+    if hasattr(L, "oracle_mxfp8_quantize"):
+        L.oracle_mxfp8_quantize.restype = ctypes.c_int
+        L.oracle_mxfp8_expert_ffn.restype = ctypes.c_int
+    return L
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr() if isinstance(t, torch.Tensor) else t.ctypes.data)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def _c(t: torch.Tensor, dtype) -> torch.Tensor:
+    assert t.device.type == "cpu"
+    return t.to(dtype).contiguous()
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    lib().oracle_set_num_threads(int(n))
+
+
+def topk_gates(logits: torch.Tensor, k: int):
+    """-> (topk_idx [T,k] int32, gates [T,k] fp32)."""
+    logits = _c(logits, torch.float32)
+    T, E = logits.shape
+    idx = torch.empty((T, k), dtype=torch.int32)
+    g = torch.empty((T, k), dtype=torch.float32)
+    _check(lib().oracle_topk_gates(_ptr(logits), T, E, k, _ptr(idx), _ptr(g)), "topk_gates")
+    return idx, g
+
+
+def schedule(topk_idx: torch.Tensor, E: int, R: int):
+    """-> dict(counts, offsets, src_rank, src_index, row_slot, pos) (int32)."""
+    topk_idx = _c(topk_idx, torch.int32)
+    T, k = topk_idx.shape
+    ns = T * k
+    out = dict(counts=torch.empty(E, dtype=torch.int32), offsets=torch.empty(E + 1, dtype=torch.int32),
+               src_rank=torch.empty(ns, dtype=torch.int32), src_index=torch.empty(ns, dtype=torch.int32),
+               row_slot=torch.empty(ns, dtype=torch.int32), pos=torch.empty(ns, dtype=torch.int32))
+    _check(lib().oracle_schedule(_ptr(topk_idx), T, E, k, R, *(_ptr(out[n]) for n in
+           ("counts", "offsets", "src_rank", "src_index", "row_slot", "pos"))), "schedule")
+    return out
+
+
+def plan(logits: torch.Tensor, k: int, R: int):
+    idx, g = topk_gates(logits, k)
+    p = schedule(idx, logits.shape[1], R)
+    p["topk_idx"], p["gates"] = idx, g
+    return p
+
+
+def gather(x: torch.Tensor, R: int, src_rank: torch.Tensor, src_index: torch.Tensor) -> torch.Tensor:
+    x = _c(x, torch.bfloat16)
+    T, H = x.shape
+    n = src_rank.numel()
+    rows = torch.empty((n, H), dtype=torch.bfloat16)
+    _check(lib().oracle_gather(_ptr(x), T, H, R, n, _ptr(_c(src_rank, torch.int32)),
+                               _ptr(_c(src_index, torch.int32)), _ptr(rows)), "gather")
+    return rows
+
+
+def expert_ffn(x_rows: torch.Tensor, wg: torch.Tensor, wu: torch.Tensor, wd: torch.Tensor) -> torch.Tensor:
+    """One expert's SwiGLU FFN; bf16 inputs, float64 result [n, H]."""
+    x_rows = _c(x_rows, torch.bfloat16)
+    n, H = x_rows.shape
+    I = wg.shape[1]
+    o = torch.empty((n, H), dtype=torch.float64)
+    _check(lib().oracle_expert_ffn(_ptr(x_rows), n, H, I, _ptr(_c(wg, torch.bfloat16)),
+                                   _ptr(_c(wu, torch.bfloat16)), _ptr(_c(wd, torch.bfloat16)), _ptr(o)),
+           "expert_ffn")
+    return o
+
+
+def combine(o_slot: torch.Tensor, gates: torch.Tensor) -> torch.Tensor:
+    """o_slot [T,k,H] float64, gates [T,k] -> y [T,H] float64."""
+    o_slot = _c(o_slot, torch.float64)
+    T, k, H = o_slot.shape
+    y = torch.empty((T, H), dtype=torch.float64)
+    _check(lib().oracle_combine(_ptr(o_slot), _ptr(_c(gates, torch.float32)), T, k, H, _ptr(y)), "combine")
+    return y
+
+
+def moe_forward(x, logits, wg, wu, wd, k: int, R: int):
+    """Whole layer on small inputs -> (y [T,H] float64, topk_idx, gates)."""
+    x = _c(x, torch.bfloat16)
+    logits = _c(logits, torch.float32)
+    T, H = x.shape
+    E, _, I = wg.shape
+    y = torch.empty((T, H), dtype=torch.float64)
+    idx = torch.empty((T, k), dtype=torch.int32)
+    g = torch.empty((T, k), dtype=torch.float32)
+    _check(lib().oracle_moe_forward(_ptr(x), _ptr(logits), T, H, I, E, k, R,
+                                    _ptr(_c(wg, torch.bfloat16)), _ptr(_c(wu, torch.bfloat16)),
+                                    _ptr(_c(wd, torch.bfloat16)), _ptr(y), _ptr(idx), _ptr(g)),
+           "moe_forward")
+    return y, idx, g
+
+
+def forward_tokens(cfg, x, logits, token_ids, weight_fn, k=None):
+    """y rows for a subset of tokens of a large configuration.
+
+    ``weight_fn(e)`` returns (Wg, Wu, Wd) of expert e on the host; only the
+    experts these tokens select are materialised.  Routing uses the full-T
+    oracle plan restricted to the chosen tokens (a token's selection and
+    gates depend on its own logits only).
+    """
+    k = cfg.k if k is None else k
+    token_ids = torch.as_tensor(token_ids, dtype=torch.int64)
+    idx, g = topk_gates(logits[token_ids], k)
+    n = token_ids.numel()
+    o_slot = torch.zeros((n, k, cfg.H), dtype=torch.float64)
+    xs = x[token_ids].contiguous()
+    need = {}
+    for a in range(n):
+        for j in range(k):
+            need.setdefault(int(idx[a, j]), []).append((a, j))
+    for e, uses in sorted(need.items()):
+        wg, wu, wd = weight_fn(e)
+        rows = torch.stack([xs[a] for a, _ in uses])
+        o = expert_ffn(rows, wg, wu, wd)
+        for r, (a, j) in enumerate(uses):
+            o_slot[a, j] = o[r]
+    return combine(o_slot, g), idx, g
