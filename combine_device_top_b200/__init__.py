@@ -1,0 +1,262 @@
+"""Forward Mixture-of-Kittens MoE layer on B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/mok.h`` (``libmok.so``,
+built in-tree by ``combine_device_top_b200.build``).  This module only
+marshals arguments: PyTorch provides device memory and the current CUDA
+stream, and every step of the layer runs in the library's CUDA kernels.
+There is no CPU path: if ``libmok.so`` cannot be loaded, importing the
+binding's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from functools import lru_cache
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmok.so")
+
+MOK_OK = 0
+MOK_ERR_INVALID_ARG = 1
+MOK_ERR_UNSUPPORTED = 2
+MOK_ERR_WORKSPACE = 3
+MOK_ERR_CUDA = 4
+MOK_ERR_TIMEOUT = 5
+MOK_ERR_CAPACITY = 6
+MOK_MODE_PERSISTENT = 0
+MOK_MODE_STAGED = 1
+MOK_MAX_SHARDS = 64
+
+# every entry point of include/mok.h
+EXPORTS = (
+    "mok_plan_workspace_bytes", "mok_plan", "mok_forward_workspace_bytes", "mok_moe_forward",
+    "mok_get_status", "mok_last_error_string", "mok_gather", "mok_expert_ffn_workspace_bytes",
+    "mok_expert_ffn", "mok_combine", "mok_forward_host_workspace_bytes", "mok_moe_forward_host",
+)
+
+
+class MokError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"mok error {code}: {msg}")
+        self.code = code
+
+
+class PlanT(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("R", ctypes.c_int32),
+                ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("sched_src_rank", ctypes.c_void_p), ("sched_src_index", ctypes.c_void_p),
+                ("row_slot", ctypes.c_void_p), ("pos", ctypes.c_void_p),
+                ("topk_idx", ctypes.c_void_p), ("gates", ctypes.c_void_p)]
+
+
+class FwdOpts(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("dispatch_ctas", ctypes.c_int32),
+                ("gemm_ctas", ctypes.c_int32), ("mxfp8", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("timeout_ns", ctypes.c_uint64)]
+
+
+@lru_cache(maxsize=1)
+def lib() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m combine_device_top_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    i32, sz, vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    L.mok_plan_workspace_bytes.argtypes = [i32, i32, i32]
+    L.mok_plan_workspace_bytes.restype = sz
+    L.mok_plan.argtypes = [vp, i32, i32, i32, i32, vp, sz, ctypes.POINTER(PlanT), vp]
+    L.mok_forward_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(FwdOpts)]
+    L.mok_forward_workspace_bytes.restype = sz
+    L.mok_moe_forward.argtypes = [vp, i32, i32, vp, vp, vp, ctypes.POINTER(PlanT), i32, ctypes.POINTER(FwdOpts),
+                                  vp, sz, vp, vp]
+    L.mok_get_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int)]
+    L.mok_last_error_string.argtypes = []
+    L.mok_last_error_string.restype = ctypes.c_char_p
+    L.mok_gather.argtypes = [vp, i32, ctypes.POINTER(PlanT), vp, vp]
+    L.mok_expert_ffn_workspace_bytes.argtypes = [i32, i32, i32]
+    L.mok_expert_ffn_workspace_bytes.restype = sz
+    L.mok_expert_ffn.argtypes = [vp, i32, i32, vp, vp, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
+    L.mok_combine.argtypes = [vp, i32, ctypes.POINTER(PlanT), vp, vp]
+    L.mok_forward_host_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(FwdOpts)]
+    L.mok_forward_host_workspace_bytes.restype = sz
+    L.mok_moe_forward_host.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32,
+                                       ctypes.POINTER(FwdOpts), vp, sz, vp, vp]
+    for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
+              "mok_moe_forward_host"):
+        getattr(L, n).restype = ctypes.c_int
+    return L
+
+
+def _check(rc: int) -> None:
+    if rc != MOK_OK:
+        raise MokError(rc, lib().mok_last_error_string().decode())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr_array(tensors):
+    arr = (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
+    return arr
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class Plan:
+    """Result of :func:`plan`: a C ``mok_plan_t`` plus the workspace it views."""
+    c: PlanT
+    ws: torch.Tensor
+
+    def _view(self, ptr, n, dtype):
+        # zero-copy view of a plan array (the storage is ``ws``)
+        off = ptr - self.ws.data_ptr()
+        itemsize = torch.empty((), dtype=dtype).element_size()
+        return self.ws[off:off + n * itemsize].view(dtype)
+
+    @property
+    def ns(self):
+        return self.c.T * self.c.k
+
+    def counts(self):
+        return self._view(self.c.counts, self.c.E, torch.int32)
+
+    def offsets(self):
+        return self._view(self.c.offsets, self.c.E + 1, torch.int32)
+
+    def src_rank(self):
+        return self._view(self.c.sched_src_rank, self.ns, torch.int32)
+
+    def src_index(self):
+        return self._view(self.c.sched_src_index, self.ns, torch.int32)
+
+    def row_slot(self):
+        return self._view(self.c.row_slot, self.ns, torch.int32)
+
+    def pos(self):
+        return self._view(self.c.pos, self.ns, torch.int32)
+
+    def topk_idx(self):
+        return self._view(self.c.topk_idx, self.ns, torch.int32).view(self.c.T, self.c.k)
+
+    def gates(self):
+        return self._view(self.c.gates, self.ns, torch.float32).view(self.c.T, self.c.k)
+
+
+def plan(logits: torch.Tensor, top_k: int, R: int, ws: torch.Tensor | None = None, stream=None) -> Plan:
+    """Steps 1-2: ``mok_plan`` on fp32 device logits [T, E]."""
+    assert logits.is_cuda and logits.dtype == torch.float32 and logits.is_contiguous()
+    T, E = logits.shape
+    need = lib().mok_plan_workspace_bytes(T, E, top_k)
+    if need == 0:
+        raise MokError(MOK_ERR_INVALID_ARG, "invalid plan shape")
+    if ws is None:
+        ws = _workspace(need, logits.device)
+    p = PlanT()
+    _check(lib().mok_plan(ctypes.c_void_p(logits.data_ptr()), T, E, top_k, R, ctypes.c_void_p(ws.data_ptr()),
+                          ws.numel(), ctypes.byref(p), _stream(stream)))
+    return Plan(p, ws)
+
+
+def fwd_opts(mode: int = MOK_MODE_PERSISTENT, ring_slots: int = 0, dispatch_ctas: int = 0, gemm_ctas: int = 0,
+             mxfp8: bool = False, timeout_ns: int = 0) -> FwdOpts:
+    return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), 0, timeout_ns)
+
+
+def forward_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None = None) -> int:
+    return lib().mok_forward_workspace_bytes(T, H, I, E, k, minibatch, ctypes.byref(opts) if opts else None)
+
+
+def shards(x: torch.Tensor, R: int):
+    """R contiguous row blocks of a [T, H] tensor (views, no copy)."""
+    return list(x.view(R, x.shape[0] // R, x.shape[1]).unbind(0))
+
+
+def moe_forward(x_shards, w_gate, w_up, w_down, p: Plan, minibatch: int = 2560, opts: FwdOpts | None = None,
+                y_shards=None, ws: torch.Tensor | None = None, stream=None):
+    """Steps 3-5: ``mok_moe_forward``.  Returns (y_shards, ws)."""
+    R = p.c.R
+    assert len(x_shards) == R
+    H = x_shards[0].shape[1]
+    I = w_gate.shape[-1]
+    dev = x_shards[0].device
+    if y_shards is None:
+        y_shards = [torch.empty_like(s) for s in x_shards]
+    if ws is None:
+        need = forward_workspace_bytes(p.c.T, H, I, p.c.E, p.c.k, minibatch, opts)
+        if need == 0:
+            raise MokError(MOK_ERR_INVALID_ARG, "invalid forward shape")
+        ws = _workspace(need, dev)
+    xa, ya = _ptr_array(x_shards), _ptr_array(y_shards)
+    _check(lib().mok_moe_forward(xa, H, I, ctypes.c_void_p(w_gate.data_ptr()), ctypes.c_void_p(w_up.data_ptr()),
+                                 ctypes.c_void_p(w_down.data_ptr()), ctypes.byref(p.c), minibatch,
+                                 ctypes.byref(opts) if opts else None, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                 ya, _stream(stream)))
+    return y_shards, ws
+
+
+def get_status(ws: torch.Tensor, stream=None) -> int:
+    code = ctypes.c_int(-1)
+    _check(lib().mok_get_status(ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream), ctypes.byref(code)))
+    return code.value
+
+
+def last_error() -> str:
+    return lib().mok_last_error_string().decode()
+
+
+def gather(x_shards, p: Plan, rows: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    H = x_shards[0].shape[1]
+    if rows is None:
+        rows = torch.empty((p.ns, H), dtype=torch.bfloat16, device=x_shards[0].device)
+    _check(lib().mok_gather(_ptr_array(x_shards), H, ctypes.byref(p.c), ctypes.c_void_p(rows.data_ptr()),
+                            _stream(stream)))
+    return rows
+
+
+def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
+    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] slot-indexed, ws)."""
+    H = rows.shape[1]
+    I = w_gate.shape[-1]
+    if out is None:
+        out = torch.empty((p.ns, H), dtype=torch.bfloat16, device=rows.device)
+    if ws is None:
+        ws = _workspace(lib().mok_expert_ffn_workspace_bytes(p.ns, I, p.c.E), rows.device)
+    _check(lib().mok_expert_ffn(ctypes.c_void_p(rows.data_ptr()), H, I, ctypes.c_void_p(w_gate.data_ptr()),
+                                ctypes.c_void_p(w_up.data_ptr()), ctypes.c_void_p(w_down.data_ptr()),
+                                ctypes.byref(p.c), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                ctypes.c_void_p(out.data_ptr()), _stream(stream)))
+    return out, ws
+
+
+def combine(out: torch.Tensor, p: Plan, y_shards, stream=None):
+    H = out.shape[-1]
+    _check(lib().mok_combine(ctypes.c_void_p(out.data_ptr()), H, ctypes.byref(p.c), _ptr_array(y_shards),
+                             _stream(stream)))
+    return y_shards
+
+
+def forward_host_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None = None) -> int:
+    return lib().mok_forward_host_workspace_bytes(T, H, I, E, k, minibatch, ctypes.byref(opts) if opts else None)
+
+
+def moe_forward_host(x_host: torch.Tensor, logits_host: torch.Tensor, top_k: int, R: int, w_gate, w_up, w_down,
+                     minibatch: int, opts: FwdOpts | None, ws: torch.Tensor, y_host: torch.Tensor, stream=None):
+    """End to end from host memory: ``mok_moe_forward_host``."""
+    T, H = x_host.shape
+    E = logits_host.shape[1]
+    I = w_gate.shape[-1]
+    _check(lib().mok_moe_forward_host(ctypes.c_void_p(x_host.data_ptr()), ctypes.c_void_p(logits_host.data_ptr()),
+                                      T, H, I, E, top_k, R, ctypes.c_void_p(w_gate.data_ptr()),
+                                      ctypes.c_void_p(w_up.data_ptr()), ctypes.c_void_p(w_down.data_ptr()),
+                                      minibatch, ctypes.byref(opts) if opts else None,
+                                      ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                      ctypes.c_void_p(y_host.data_ptr()), _stream(stream)))
+    return y_host

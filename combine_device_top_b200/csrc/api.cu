@@ -1,0 +1,427 @@
+// api.cu -- the C ABI declared in include/mok.h: argument validation,
+// workspace layout, tensor-map encoding and kernel launches.  No device
+// memory is allocated here; every buffer lives in a caller-provided
+// workspace.
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "mok_device.cuh"
+#include "mok_internal.h"
+
+namespace mok {
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_err = "no error";
+
+static int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+static int cuda_fail(cudaError_t e, const char* what) {
+    return fail(MOK_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define MOK_CUDA(call, what)                       \
+    do {                                           \
+        cudaError_t e_ = (call);                   \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+static int device_sms(int* dev_out) {
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (sms[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        sms[dev] = v;
+    }
+    if (dev_out) *dev_out = dev;
+    return sms[dev];
+}
+
+// ------------------------------------------------------------------ tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer, const char** err) {
+    auto enc = get_encode();
+    if (!enc) {
+        *err = "cuTensorMapEncodeTiled unavailable";
+        return false;
+    }
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *err = "cuTensorMapEncodeTiled failed";
+        return false;
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------ layouts
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct FwdLayout {
+    size_t status, counts2, chunks, mbs, counters, rows, h, out, total;
+    int max_chunks, max_mb, buf_rows, cap, minibatch, mode;
+};
+
+static const uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* o, FwdLayout* L) {
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return false;
+    const int64_t ns = (int64_t)T * k;
+    if (ns > 0x7fffffff / 2) return false;
+    FwdLayout l{};
+    l.mode = o ? o->mode : MOK_MODE_PERSISTENT;
+    if (l.mode == MOK_MODE_STAGED) {
+        l.minibatch = (int)(ns > 0 ? ns : 1);
+        l.cap = l.minibatch;
+        l.buf_rows = (int)ns;
+    } else {
+        l.minibatch = minibatch;
+        const int ring = (o && o->ring_slots > 0) ? o->ring_slots : 2 * (minibatch > 4096 ? minibatch : 4096);
+        l.cap = ring / 2;
+        l.buf_rows = ring;
+    }
+    if (l.minibatch < 1) return false;
+    l.max_mb = max_minibatches((int)ns, l.minibatch);
+    l.max_chunks = max_chunks((int)ns, E, l.max_mb);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += align256(bytes);
+        return at;
+    };
+    l.status = take(sizeof(DevStatus));
+    l.counts2 = take(sizeof(int) * 4);
+    l.chunks = take(sizeof(Chunk) * (size_t)l.max_chunks);
+    l.mbs = take(sizeof(Minibatch) * (size_t)l.max_mb);
+    l.counters = take(sizeof(int) * 4 * (size_t)l.max_mb + 256);
+    l.rows = take((size_t)l.buf_rows * H * 2);
+    l.h = take((size_t)l.buf_rows * I * 2);
+    l.out = take((size_t)ns * H * 2);
+    l.total = off;
+    *L = l;
+    return true;
+}
+
+static int check_ws(const void* ws, size_t have, size_t need) {
+    if (ws == nullptr) return fail(MOK_ERR_WORKSPACE, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOK_ERR_WORKSPACE, "workspace not 256-byte aligned");
+    if (have < need) return fail(MOK_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", have, need);
+    return MOK_OK;
+}
+
+static int check_plan(const mok_plan_t* p) {
+    if (!p) return fail(MOK_ERR_INVALID_ARG, "plan is NULL");
+    if (p->T < 0 || p->E <= 0 || p->k <= 0 || p->k > p->E || p->R <= 0 || p->R > MOK_MAX_SHARDS ||
+        (p->T > 0 && p->T % p->R))
+        return fail(MOK_ERR_INVALID_ARG, "plan holds an invalid shape");
+    if (!p->counts || !p->offsets || !p->sched_src_rank || !p->sched_src_index || !p->row_slot || !p->pos ||
+        !p->topk_idx || !p->gates)
+        return fail(MOK_ERR_INVALID_ARG, "plan has NULL views (was mok_plan called?)");
+    return MOK_OK;
+}
+
+static int check_hi(int H, int I) {
+    if (H <= 0 || I <= 0) return fail(MOK_ERR_INVALID_ARG, "H and I must be positive");
+    if (H % 128) return fail(MOK_ERR_UNSUPPORTED, "H %% 128 != 0 (H = %d)", H);
+    if (I % 64) return fail(MOK_ERR_UNSUPPORTED, "I %% 64 != 0 (I = %d)", I);
+    return MOK_OK;
+}
+
+// ------------------------------------------------------------------ pieces
+static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const void* wg, const void* wu,
+                          const void* wd, int E, const int32_t* row_slot, const Chunk* chunks, const int* counts2,
+                          void* h, void* out, DevStatus* status, uint64_t timeout_ns, cudaStream_t stream) {
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(gemm_configure(dev), "gemm configure");
+    CUtensorMap tm_wg, tm_wu, tm_wd, tm_rows, tm_h;
+    const char* err = nullptr;
+    if (!encode_tmap_2d_bf16(&tm_wg, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
+        !encode_tmap_2d_bf16(&tm_wu, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
+        !encode_tmap_2d_bf16(&tm_wd, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, &err) ||
+        !encode_tmap_2d_bf16(&tm_rows, rows, (uint64_t)H, (uint64_t)n_rows_buf, 64, 16, &err) ||
+        !encode_tmap_2d_bf16(&tm_h, h, (uint64_t)I, (uint64_t)n_rows_buf, 64, 16, &err))
+        return fail(MOK_ERR_CUDA, "tensor map: %s", err);
+    GemmShape sh{H, I, E};
+    MOK_CUDA(launch_gemm_phase(0, tm_wg, tm_wu, tm_rows, sh, chunks, counts2, h, out, row_slot, status, timeout_ns,
+                               sms, stream),
+             "gate/up GEMM launch");
+    MOK_CUDA(launch_gemm_phase(1, tm_wd, tm_wd, tm_h, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
+                               stream),
+             "down GEMM launch");
+    return MOK_OK;
+}
+
+static bool all_nonnull(const void* const* p, int n) {
+    if (!p) return false;
+    for (int i = 0; i < n; ++i)
+        if (!p[i]) return false;
+    return true;
+}
+
+}  // namespace mok
+
+using namespace mok;
+
+extern "C" {
+
+const char* mok_last_error_string(void) { return g_err.c_str(); }
+
+size_t mok_plan_workspace_bytes(int T, int E, int k) {
+    if (T < 0 || E <= 0 || E > MOK_MAX_EXPERTS || k <= 0 || k > E || k > MOK_MAX_TOPK) return 0;
+    return plan_layout(T, E, k, nullptr);
+}
+
+int mok_plan(const float* logits, int T, int E, int top_k, int R, void* ws, size_t ws_bytes, mok_plan_t* plan,
+             mok_stream_t stream) {
+    if (!plan) return fail(MOK_ERR_INVALID_ARG, "plan is NULL");
+    if (T < 0 || E <= 0 || top_k <= 0 || R <= 0) return fail(MOK_ERR_INVALID_ARG, "T, E, top_k, R out of range");
+    if (E > MOK_MAX_EXPERTS) return fail(MOK_ERR_UNSUPPORTED, "E > %d", MOK_MAX_EXPERTS);
+    if (top_k > E) return fail(MOK_ERR_INVALID_ARG, "top_k > E");
+    if (top_k > MOK_MAX_TOPK) return fail(MOK_ERR_UNSUPPORTED, "top_k > %d", MOK_MAX_TOPK);
+    if (R > MOK_MAX_SHARDS) return fail(MOK_ERR_UNSUPPORTED, "R > %d", MOK_MAX_SHARDS);
+    if (T % R) return fail(MOK_ERR_UNSUPPORTED, "T %% R != 0 (T = %d, R = %d)", T, R);
+    if ((int64_t)T * top_k > 0x3fffffff) return fail(MOK_ERR_UNSUPPORTED, "T * top_k too large");
+    if (T > 0 && !logits) return fail(MOK_ERR_INVALID_ARG, "logits is NULL");
+    PlanLayout L;
+    const size_t need = plan_layout(T, E, top_k, &L);
+    int rc = check_ws(ws, ws_bytes, need);
+    if (rc) return rc;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    plan->T = T;
+    plan->E = E;
+    plan->k = top_k;
+    plan->R = R;
+    plan->counts = reinterpret_cast<int32_t*>(base + L.counts);
+    plan->offsets = reinterpret_cast<int32_t*>(base + L.offsets);
+    plan->sched_src_rank = reinterpret_cast<int32_t*>(base + L.src_rank);
+    plan->sched_src_index = reinterpret_cast<int32_t*>(base + L.src_index);
+    plan->row_slot = reinterpret_cast<int32_t*>(base + L.row_slot);
+    plan->pos = reinterpret_cast<int32_t*>(base + L.pos);
+    plan->topk_idx = reinterpret_cast<int32_t*>(base + L.topk);
+    plan->gates = reinterpret_cast<float*>(base + L.gates);
+    if (device_sms(nullptr) <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_plan(logits, T, E, top_k, R, base, L, reinterpret_cast<cudaStream_t>(stream)), "plan launch");
+    return MOK_OK;
+}
+
+size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* opts) {
+    FwdLayout L;
+    if (!fwd_layout(T, H, I, E, k, minibatch, opts, &L)) return 0;
+    return L.total;
+}
+
+int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gate, const void* w_up,
+                    const void* w_down, const mok_plan_t* plan, int minibatch, const mok_fwd_opts* opts, void* ws,
+                    size_t ws_bytes, void* const* y_shards, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if ((rc = check_hi(H, I))) return rc;
+    const int mode = opts ? opts->mode : MOK_MODE_PERSISTENT;
+    if (mode != MOK_MODE_STAGED && mode != MOK_MODE_PERSISTENT) return fail(MOK_ERR_INVALID_ARG, "unknown mode %d", mode);
+    if (opts && opts->reserved != 0) return fail(MOK_ERR_INVALID_ARG, "opts.reserved must be 0");
+    if (opts && opts->mxfp8) return fail(MOK_ERR_UNSUPPORTED, "MXFP8 path not built");
+    if (mode == MOK_MODE_PERSISTENT && minibatch < 16) return fail(MOK_ERR_INVALID_ARG, "minibatch < 16");
+    const int T = plan->T, E = plan->E, k = plan->k, R = plan->R;
+    if (T == 0) return MOK_OK;
+    if (!all_nonnull(x_shards, R) || !all_nonnull(y_shards, R)) return fail(MOK_ERR_INVALID_ARG, "NULL shard pointer");
+    if (!w_gate || !w_up || !w_down) return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
+    FwdLayout L;
+    if (!fwd_layout(T, H, I, E, k, minibatch, opts, &L)) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
+    if (mode == MOK_MODE_PERSISTENT) {
+        if (L.cap < minibatch) return fail(MOK_ERR_INVALID_ARG, "ring_slots / 2 < minibatch");
+        return fail(MOK_ERR_UNSUPPORTED, "persistent mode not built yet");
+    }
+    if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    const uint64_t timeout = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    DevStatus* status = reinterpret_cast<DevStatus*>(base + L.status);
+    int* counts2 = reinterpret_cast<int*>(base + L.counts2);
+    Chunk* chunks = reinterpret_cast<Chunk*>(base + L.chunks);
+    Minibatch* mbs = reinterpret_cast<Minibatch*>(base + L.mbs);
+    ShardsIn xs{};
+    ShardsOut ys{};
+    for (int r = 0; r < R; ++r) {
+        xs.p[r] = x_shards[r];
+        ys.p[r] = y_shards[r];
+    }
+    const int ns = T * k;
+    MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
+    MOK_CUDA(launch_build_chunks(plan->offsets, E, ns, L.minibatch, L.cap, chunks, L.max_chunks, mbs, L.max_mb,
+                                 counts2, status, stream),
+             "work list launch");
+    MOK_CUDA(launch_gather(xs, T / R, H, plan->sched_src_rank, plan->sched_src_index, ns, base + L.rows, sms, stream),
+             "gather launch");
+    rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, chunks, counts2,
+                        base + L.h, base + L.out, status, timeout, stream);
+    if (rc) return rc;
+    MOK_CUDA(launch_combine(base + L.out, plan->gates, T, k, H, T / R, ys, sms, stream), "combine launch");
+    return MOK_OK;
+}
+
+int mok_get_status(const void* ws, size_t ws_bytes, mok_stream_t stream, int* device_code) {
+    if (!device_code) return fail(MOK_ERR_INVALID_ARG, "device_code is NULL");
+    int rc = check_ws(ws, ws_bytes, sizeof(DevStatus));
+    if (rc) return rc;
+    MOK_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream synchronize");
+    DevStatus st;
+    MOK_CUDA(cudaMemcpy(&st, ws, sizeof st, cudaMemcpyDeviceToHost), "status read");
+    *device_code = st.code;
+    if (st.code != MOK_OK)
+        fail(st.code, "device status %d (where %d, aux %d %d)", st.code, st.where, st.aux0, st.aux1);
+    return MOK_OK;
+}
+
+int mok_gather(const void* const* x_shards, int H, const mok_plan_t* plan, void* rows, mok_stream_t stream) {
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if (H <= 0 || H % 8) return fail(MOK_ERR_UNSUPPORTED, "H %% 8 != 0");
+    if (plan->T == 0) return MOK_OK;
+    if (!rows || !all_nonnull(x_shards, plan->R)) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    ShardsIn xs{};
+    for (int r = 0; r < plan->R; ++r) xs.p[r] = x_shards[r];
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_gather(xs, plan->T / plan->R, H, plan->sched_src_rank, plan->sched_src_index,
+                           plan->T * plan->k, rows, sms, reinterpret_cast<cudaStream_t>(stream)),
+             "gather launch");
+    return MOK_OK;
+}
+
+size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E) {
+    if (n_rows < 0 || I <= 0 || E <= 0) return 0;
+    const int mb = max_minibatches(n_rows, n_rows > 0 ? n_rows : 1);
+    const int mc = max_chunks(n_rows, E, mb);
+    return align256(sizeof(DevStatus)) + align256(sizeof(int) * 4) + align256(sizeof(Chunk) * (size_t)mc) +
+           align256(sizeof(Minibatch) * (size_t)mb) + align256((size_t)n_rows * I * 2);
+}
+
+int mok_expert_ffn(const void* rows, int H, int I, const void* w_gate, const void* w_up, const void* w_down,
+                   const mok_plan_t* plan, void* ws, size_t ws_bytes, void* out, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if ((rc = check_hi(H, I))) return rc;
+    const int ns = plan->T * plan->k;
+    if ((rc = check_ws(ws, ws_bytes, mok_expert_ffn_workspace_bytes(ns, I, plan->E)))) return rc;
+    if (ns == 0) return MOK_OK;
+    if (!rows || !out || !w_gate || !w_up || !w_down) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    const int mb = max_minibatches(ns, ns);
+    const int mc = max_chunks(ns, plan->E, mb);
+    size_t off = 0;
+    DevStatus* status = reinterpret_cast<DevStatus*>(base + off);
+    off += align256(sizeof(DevStatus));
+    int* counts2 = reinterpret_cast<int*>(base + off);
+    off += align256(sizeof(int) * 4);
+    Chunk* chunks = reinterpret_cast<Chunk*>(base + off);
+    off += align256(sizeof(Chunk) * (size_t)mc);
+    Minibatch* mbs = reinterpret_cast<Minibatch*>(base + off);
+    off += align256(sizeof(Minibatch) * (size_t)mb);
+    void* h = base + off;
+    MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
+    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, chunks, mc, mbs, mb, counts2, status, stream),
+             "work list launch");
+    return run_expert_ffn(rows, ns, H, I, w_gate, w_up, w_down, plan->E, plan->row_slot, chunks, counts2, h, out,
+                          status, kDefaultTimeoutNs, stream);
+}
+
+int mok_combine(const void* out, int H, const mok_plan_t* plan, void* const* y_shards, mok_stream_t stream) {
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if (H <= 0 || H % 8) return fail(MOK_ERR_UNSUPPORTED, "H %% 8 != 0");
+    if (plan->T == 0) return MOK_OK;
+    if (!out || !all_nonnull(y_shards, plan->R)) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    ShardsOut ys{};
+    for (int r = 0; r < plan->R; ++r) ys.p[r] = y_shards[r];
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_combine(out, plan->gates, plan->T, plan->k, H, plan->T / plan->R, ys, sms,
+                            reinterpret_cast<cudaStream_t>(stream)),
+             "combine launch");
+    return MOK_OK;
+}
+
+size_t mok_forward_host_workspace_bytes(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* opts) {
+    const size_t p = mok_plan_workspace_bytes(T, E, k);
+    const size_t f = mok_forward_workspace_bytes(T, H, I, E, k, minibatch, opts);
+    if (!p || !f) return 0;
+    return align256((size_t)T * H * 2) * 2 + align256((size_t)T * E * 4) + align256(p) + f;
+}
+
+int mok_moe_forward_host(const void* x_host, const float* logits_host, int T, int H, int I, int E, int top_k, int R,
+                         const void* w_gate, const void* w_up, const void* w_down, int minibatch,
+                         const mok_fwd_opts* opts, void* ws, size_t ws_bytes, void* y_host, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!x_host || !logits_host || !y_host) return fail(MOK_ERR_INVALID_ARG, "NULL host pointer");
+    if (T <= 0 || R <= 0 || R > MOK_MAX_SHARDS || T % R) return fail(MOK_ERR_INVALID_ARG, "T, R invalid");
+    const size_t need = mok_forward_host_workspace_bytes(T, H, I, E, top_k, minibatch, opts);
+    if (!need) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
+    int rc = check_ws(ws, ws_bytes, need);
+    if (rc) return rc;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    const size_t xb = (size_t)T * H * 2, lb = (size_t)T * E * 4;
+    unsigned char* x_dev = base;
+    unsigned char* y_dev = x_dev + align256(xb);
+    unsigned char* l_dev = y_dev + align256(xb);
+    unsigned char* plan_ws = l_dev + align256(lb);
+    const size_t plan_bytes = align256(mok_plan_workspace_bytes(T, E, top_k));
+    unsigned char* fwd_ws = plan_ws + plan_bytes;
+    const size_t fwd_bytes = ws_bytes - (size_t)(fwd_ws - base);
+    MOK_CUDA(cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream), "x upload");
+    MOK_CUDA(cudaMemcpyAsync(l_dev, logits_host, lb, cudaMemcpyHostToDevice, stream), "logits upload");
+    mok_plan_t plan;
+    if ((rc = mok_plan(reinterpret_cast<const float*>(l_dev), T, E, top_k, R, plan_ws, plan_bytes, &plan, stream_)))
+        return rc;
+    const void* xs[MOK_MAX_SHARDS];
+    void* ys[MOK_MAX_SHARDS];
+    const int S_r = T / R;
+    for (int r = 0; r < R; ++r) {
+        xs[r] = x_dev + (size_t)r * S_r * H * 2;
+        ys[r] = y_dev + (size_t)r * S_r * H * 2;
+    }
+    if ((rc = mok_moe_forward(xs, H, I, w_gate, w_up, w_down, &plan, minibatch, opts, fwd_ws, fwd_bytes, ys,
+                              stream_)))
+        return rc;
+    MOK_CUDA(cudaMemcpyAsync(y_host, y_dev, xb, cudaMemcpyDeviceToHost, stream), "y download");
+    MOK_CUDA(cudaStreamSynchronize(stream), "stream synchronize");
+    return MOK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,70 @@
+// mok_internal.h -- host-side declarations shared by the translation units
+// of libmok (workspace layouts and kernel launchers).  Not installed.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mok.h"
+
+namespace mok {
+
+// ---- plan workspace (byte offsets from the workspace base)
+struct PlanLayout {
+    int nb;  // route blocks
+    size_t counts, offsets, src_rank, src_index, row_slot, pos, topk, gates, blk_cnt, rank, total;
+};
+size_t plan_layout(int T, int E, int k, PlanLayout* L);
+cudaError_t launch_plan(const float* logits, int T, int E, int k, int R, unsigned char* ws, const PlanLayout& L,
+                        cudaStream_t stream);
+
+// ---- token shards as kernel parameters
+struct ShardsIn {
+    const void* p[MOK_MAX_SHARDS];
+};
+struct ShardsOut {
+    void* p[MOK_MAX_SHARDS];
+};
+
+cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, const int32_t* src_rank, const int32_t* src_index,
+                          int n_rows, void* rows, int num_sms, cudaStream_t stream);
+cudaError_t launch_combine(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
+                           int num_sms, cudaStream_t stream);
+
+// ---- work decomposition of the grouped GEMM
+// A chunk is <= 256 consecutive rows of one expert inside one minibatch.
+struct Chunk {
+    int expert, row0, rows, mb;
+};
+// A minibatch is a range of rows [row0, row1) with its chunk range.
+struct Minibatch {
+    int row0, row1, chunk0, chunk1;
+};
+constexpr int CHUNK_MAX_ROWS = 256;
+
+int max_chunks(int n_slots, int E, int n_mb);
+int max_minibatches(int n_slots, int minibatch);
+cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int minibatch, int cap, Chunk* chunks,
+                                int max_chunks, Minibatch* mbs, int max_mb, int* counts2, void* status,
+                                cudaStream_t stream);
+
+// ---- the grouped GEMM (tcgen05)
+struct GemmShape {
+    int H, I, E;
+};
+size_t gemm_smem_bytes();
+cudaError_t gemm_configure(int dev);
+// Staged grouped GEMM over every chunk: phase 0 = gate/up + SwiGLU -> h,
+// phase 1 = down -> out[row_slot].  Tensor maps are built by the caller.
+cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmB,
+                              const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out,
+                              void* out, const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
+                              cudaStream_t stream);
+
+// ---- tensor maps (driver entry point fetched at run time)
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer, const char** err);
+
+}  // namespace mok

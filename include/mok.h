@@ -1,0 +1,233 @@
+/*
+ * mok.h -- C ABI of the forward Mixture-of-Kittens (MoK) MoE layer on one
+ * B200 (sm_100a).
+ *
+ * The layer (MoK article on tahou.com, routing paragraph and the benchmark
+ * paragraph listing "scheduling, dispatch, expert FFN, combine, weighted
+ * merge"; MoK wiki summary "Mixture-of-Kittens: Cursor가 새로 공개한 NVL72용
+ * MoE 학습 메가커널", key points) runs in five steps:
+ *   1. router top-k over fp32 logits with softmax gates and a per-expert
+ *      histogram;
+ *   2. a device-built pull schedule {src_rank, src_index} per row of the
+ *      expert-major layout (no sort, no host round trip);
+ *   3. pull dispatch: a gather of token rows from R source shards into an
+ *      expert-contiguous buffer;
+ *   4. a grouped GEMM per expert with SwiGLU fused: h = silu(x Wg) * (x Wu),
+ *      o = h Wd; the result row is pushed back to its token slot;
+ *   5. the fixed-order weighted combine y[t] = sum_j g[t,j] o[t,j].
+ *
+ * Conventions for every call below:
+ *  - Every data pointer is a DEVICE pointer owned by the caller unless the
+ *    argument says "host".  The library never allocates device memory on
+ *    these paths: scratch space is a caller-provided workspace whose size
+ *    the matching *_workspace_bytes() call returns.  Workspaces must be
+ *    256-byte aligned.
+ *  - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
+ *    is the legacy default stream).  No call synchronises the host except
+ *    mok_get_status() and mok_moe_forward_host().
+ *  - Inputs are never modified.
+ *  - Return value: MOK_OK or a MOK_ERR_* code; mok_last_error_string()
+ *    gives a message for the calling thread's last failure.  Argument and
+ *    shape errors are detected on the host before anything is enqueued.
+ *  - Device-side failures (a bounded wait that gave up, a capacity bound)
+ *    are written to a status word in the forward workspace and read with
+ *    mok_get_status().
+ *  - Layouts are row-major.  bf16 is IEEE bfloat16 stored as uint16.
+ *  - Shapes: T tokens, H hidden, I expert intermediate, E experts, k top-k,
+ *    R logical source shards; shard r holds tokens [r*S_r, (r+1)*S_r),
+ *    S_r = T / R.  A "slot" is (t, j), j the rank in t's top-k list, slot
+ *    index t*k + j; N_s = T*k slots.  A "row" is a position in the
+ *    expert-major layout: rows offsets[e] .. offsets[e+1]-1 belong to
+ *    expert e, in ascending token order.
+ */
+#ifndef MOK_H
+#define MOK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mok_stream_t; /* same type as cudaStream_t */
+
+enum {
+    MOK_OK = 0,
+    MOK_ERR_INVALID_ARG = 1, /* null pointer, negative size, k > E, ...      */
+    MOK_ERR_UNSUPPORTED = 2, /* shape or alignment outside what is built     */
+    MOK_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small   */
+    MOK_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed            */
+    MOK_ERR_TIMEOUT = 5,     /* a device-side wait gave up (device status)   */
+    MOK_ERR_CAPACITY = 6     /* a device-side capacity bound was exceeded    */
+};
+
+enum { MOK_MAX_SHARDS = 64, MOK_MAX_EXPERTS = 1024, MOK_MAX_TOPK = 32 };
+
+/* ------------------------------------------------------------------------
+ * Step 1 + 2: the plan.
+ * ---------------------------------------------------------------------- */
+
+/* Views into the plan workspace, filled by mok_plan().  All device arrays. */
+typedef struct mok_plan_t {
+    int32_t T, E, k, R;
+    int32_t* counts;          /* [E]   tokens routed to expert e              */
+    int32_t* offsets;         /* [E+1] exclusive prefix sum; offsets[E]=N_s   */
+    int32_t* sched_src_rank;  /* [N_s] per row: source shard  = t / S_r       */
+    int32_t* sched_src_index; /* [N_s] per row: index in shard = t % S_r      */
+    int32_t* row_slot;        /* [N_s] per row: slot t*k + j it came from      */
+    int32_t* pos;             /* [N_s] per slot: its row                       */
+    int32_t* topk_idx;        /* [T,k] selected experts in rank order          */
+    float* gates;             /* [T,k] softmax over the k selected logits      */
+} mok_plan_t;
+
+/* Bytes of plan workspace for (T, E, k); 0 if the shape is invalid. */
+size_t mok_plan_workspace_bytes(int T, int E, int k);
+
+/*
+ * mok_plan -- router top-k, gates, histogram and pull schedule.
+ * Source: MoK article, routing paragraph (count each expert's tokens, plan
+ * where they go, lay an expert's tokens out contiguously) and pull
+ * paragraph (the destination needs only the source rank and the offset);
+ * MoK wiki summary, schedule bullet ({src_rank, src_index} built on the
+ * device, no sort, no CPU-GPU traffic).
+ *   logits  [T, E] fp32, finite (NaN compares as -inf; order then unspecified)
+ *   top_k   1 <= top_k <= min(E, MOK_MAX_TOPK);  E <= MOK_MAX_EXPERTS
+ *   R       1 <= R <= MOK_MAX_SHARDS, T % R == 0
+ *   ws      plan workspace (>= mok_plan_workspace_bytes), owned by the caller
+ *   plan    host struct receiving views into ws; valid while ws lives
+ * Selection: the k largest logits, ties to the lower expert index, listed in
+ * rank order.  Gates: g_j = exp(l_j - l_0) / sum_i exp(l_i - l_0).
+ * Counts, offsets, schedule, row_slot and pos are deterministic (a stable
+ * counting placement: ascending token inside each expert segment).
+ */
+int mok_plan(const float* logits, int T, int E, int top_k, int R,
+             void* ws, size_t ws_bytes, mok_plan_t* plan, mok_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Steps 3-5: the forward layer.
+ * ---------------------------------------------------------------------- */
+
+enum {
+    MOK_MODE_PERSISTENT = 0, /* one SM-partitioned persistent launch, ring    */
+    MOK_MODE_STAGED = 1      /* gather, gate/up GEMM, down GEMM, combine as   */
+                             /* four launches over full-size buffers          */
+};
+
+typedef struct mok_fwd_opts {
+    int32_t mode;          /* MOK_MODE_*                                        */
+    int32_t ring_slots;    /* rows of the ring token buffer (persistent mode);  */
+                           /* 0 = 2 * max(minibatch, 4096) rows                 */
+    int32_t dispatch_ctas; /* CTAs doing gather/combine in persistent mode;     */
+                           /* 0 = default (16)                                  */
+    int32_t gemm_ctas;     /* GEMM CTAs; 0 = all remaining SMs                  */
+    int32_t mxfp8;         /* 1 = MXFP8 path (weights from                      */
+                           /* mok_quantize_weights_mxfp8); 0 = bf16             */
+    int32_t reserved;      /* must be 0                                         */
+    uint64_t timeout_ns;   /* bound on every device-side wait; 0 = 2 s          */
+} mok_fwd_opts;
+
+/* Bytes of forward workspace; 0 if the shape is invalid.  opts may be NULL
+ * (defaults).  minibatch = rows per minibatch (see mok_moe_forward). */
+size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int minibatch,
+                                   const mok_fwd_opts* opts);
+
+/*
+ * mok_moe_forward -- pull dispatch, expert FFN (SwiGLU), push combine and
+ * the weighted merge.
+ * Source: MoK article, pull paragraph (forward dispatch pulls), push-combine
+ * paragraph (results are pushed back to their token's slot), megakernel and
+ * minibatch paragraphs (SM split, local counters, at least two waves per
+ * minibatch), ring-buffer paragraph (fixed-size token buffer reused once the
+ * combine has shipped a minibatch's results), benchmark paragraph (weighted
+ * merge); MoK wiki summary, key points (SM split, TMA, local counters).
+ *   x_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
+ *   H, I      hidden and intermediate sizes; H % 128 == 0, I % 64 == 0
+ *   w_gate    [E, H, I] bf16 (bf16 mode) or an MXFP8 weight pack
+ *   w_up      [E, H, I] bf16 (bf16 mode) or an MXFP8 weight pack
+ *   w_down    [E, I, H] bf16 (bf16 mode) or an MXFP8 weight pack
+ *   plan      from mok_plan() on the same stream (its workspace must live)
+ *   minibatch rows of the expert-major layout per minibatch (persistent
+ *             mode; >= 16); boundaries snap forward to expert boundaries
+ *             where the ring allows.  Ignored in staged mode.
+ *   opts      may be NULL (persistent mode, defaults)
+ *   ws        forward workspace (>= mok_forward_workspace_bytes)
+ *   y_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
+ * Arithmetic: bf16 inputs, fp32 accumulation, h stored bf16, each expert
+ * output row stored bf16 at its slot, y[t] = bf16(sum_{j<k} g[t,j] *
+ * o[t,j]) accumulated in fp32 with j ascending.  y does not depend on the
+ * mode, minibatch, ring size or R.
+ */
+int mok_moe_forward(const void* const* x_shards, int H, int I,
+                    const void* w_gate, const void* w_up, const void* w_down,
+                    const mok_plan_t* plan, int minibatch, const mok_fwd_opts* opts,
+                    void* ws, size_t ws_bytes, void* const* y_shards, mok_stream_t stream);
+
+/*
+ * mok_get_status -- synchronise `stream` and read the device status word of
+ * a forward workspace.  *device_code receives MOK_OK, MOK_ERR_TIMEOUT or
+ * MOK_ERR_CAPACITY; the return value is MOK_OK unless the read itself
+ * failed.  The status word is cleared at the start of every forward.
+ */
+int mok_get_status(const void* ws, size_t ws_bytes, mok_stream_t stream, int* device_code);
+
+/* Message for the calling thread's last non-OK return (never NULL). */
+const char* mok_last_error_string(void);
+
+/* ------------------------------------------------------------------------
+ * The steps one at a time (parity bisection and per-kernel profiling).
+ * They compute exactly what mok_moe_forward's staged mode computes.
+ * ---------------------------------------------------------------------- */
+
+/* rows[row] = x_shard[src_rank[row]][src_index[row]], row < plan->T*plan->k.
+ * rows: [N_s, H] bf16.  Source: MoK article, pull paragraph. */
+int mok_gather(const void* const* x_shards, int H, const mok_plan_t* plan,
+               void* rows, mok_stream_t stream);
+
+/* Bytes of scratch for mok_expert_ffn. */
+size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E);
+
+/* Grouped SwiGLU FFN over the expert-major rows of `plan`:
+ *   h[row]   = bf16(silu(rows[row] Wg[e]) * (rows[row] Wu[e]))   [N_s, I]
+ *   out[row_slot[row]] = bf16(h[row] Wd[e])                         [N_s, H]
+ * (e = expert of the row).  h is returned in the workspace only; `out` is
+ * slot-indexed, i.e. [T, k, H].  Source: MoK article, routing paragraph
+ * (grouped GEMM over contiguous per-expert tokens) and push-combine
+ * paragraph. */
+int mok_expert_ffn(const void* rows, int H, int I,
+                   const void* w_gate, const void* w_up, const void* w_down,
+                   const mok_plan_t* plan, void* ws, size_t ws_bytes,
+                   void* out, mok_stream_t stream);
+
+/* y[t] = bf16(sum_{j<k} gates[t,j] * float(out[t,j,:])), fp32, j ascending,
+ * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] bf16.
+ * Source: MoK article, benchmark paragraph (final weighted merge). */
+int mok_combine(const void* out, int H, const mok_plan_t* plan,
+                void* const* y_shards, mok_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * End to end from host memory (what a caller without device buffers uses).
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of workspace for mok_moe_forward_host. */
+size_t mok_forward_host_workspace_bytes(int T, int H, int I, int E, int k, int minibatch,
+                                        const mok_fwd_opts* opts);
+
+/*
+ * mok_moe_forward_host -- copies HOST x [T, H] bf16 and HOST logits [T, E]
+ * fp32 to the device, runs mok_plan and mok_moe_forward, copies y [T, H]
+ * bf16 back to HOST memory and synchronises `stream`.  Weights are device
+ * pointers as in mok_moe_forward.  Host buffers should be pinned for
+ * full copy bandwidth (pageable memory works, slower).  ws: device
+ * workspace of mok_forward_host_workspace_bytes().
+ */
+int mok_moe_forward_host(const void* x_host, const float* logits_host,
+                         int T, int H, int I, int E, int top_k, int R,
+                         const void* w_gate, const void* w_up, const void* w_down,
+                         int minibatch, const mok_fwd_opts* opts,
+                         void* ws, size_t ws_bytes, void* y_host, mok_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOK_H */

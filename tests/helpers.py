@@ -1,0 +1,78 @@
+"""Shared helpers for the parity tests (inputs from mokgen, expectations from oracle)."""
+from __future__ import annotations
+
+import math
+
+import torch
+
+import mokgen
+import oracle
+
+# Tolerances for bf16 outputs (forward layer): relative Frobenius error and
+# max abs error relative to rms(y).
+REL_FRO_BF16 = 5e-3
+MAX_ABS_BF16 = 2e-2
+GATES_ATOL = 2e-6
+
+
+def has_gpu() -> bool:
+    return torch.cuda.is_available()
+
+
+def rel_fro(a: torch.Tensor, b: torch.Tensor) -> float:
+    a, b = a.double(), b.double()
+    return (torch.linalg.norm(a - b) / torch.linalg.norm(b)).item()
+
+
+def max_abs_over_rms(a: torch.Tensor, b: torch.Tensor) -> float:
+    a, b = a.double(), b.double()
+    rms = torch.sqrt(torch.mean(b * b)).item()
+    return ((a - b).abs().max().item()) / rms
+
+
+def assert_bf16_close(got: torch.Tensor, want: torch.Tensor, what: str = ""):
+    rf, ma = rel_fro(got, want), max_abs_over_rms(got, want)
+    assert rf <= REL_FRO_BF16, f"{what}: relative Frobenius {rf:.3e} > {REL_FRO_BF16}"
+    assert ma <= MAX_ABS_BF16, f"{what}: max abs / rms {ma:.3e} > {MAX_ABS_BF16}"
+    return rf, ma
+
+
+class Case:
+    """Inputs of one configuration, on the host and on the device."""
+
+    def __init__(self, cfg: mokgen.MoEConfig, device="cuda", weights_on_host: bool = True):
+        self.cfg = cfg
+        self.x = mokgen.tokens(cfg)
+        self.logits = mokgen.router_logits(cfg, self.x)
+        self.device = device
+        if weights_on_host:
+            self.wg, self.wu, self.wd = mokgen.all_expert_weights(cfg)
+            self.dwg, self.dwu, self.dwd = (w.to(device) for w in (self.wg, self.wu, self.wd))
+        else:
+            self.wg = self.wu = self.wd = None
+            self.dwg, self.dwu, self.dwd = mokgen.upload_expert_weights(cfg, device)
+        self.dx = self.x.to(device)
+        self.dlogits = self.logits.to(device)
+
+    def weight_fn(self, e):
+        if self.wg is not None:
+            return self.wg[e], self.wu[e], self.wd[e]
+        return mokgen.expert_weights(self.cfg, e)
+
+    def x_shards(self):
+        R = self.cfg.R
+        return list(self.dx.view(R, self.cfg.T // R, self.cfg.H).unbind(0))
+
+    def oracle_y(self, token_ids=None):
+        """Oracle y (float64) on all tokens (small configs) or a subset."""
+        if token_ids is None and self.wg is not None:
+            y, _, _ = oracle.moe_forward(self.x, self.logits, self.wg, self.wu, self.wd, self.cfg.k, self.cfg.R)
+            return y
+        y, _, _ = oracle.forward_tokens(self.cfg, self.x, self.logits, token_ids, self.weight_fn)
+        return y
+
+
+def sample_tokens(T: int, n: int, seed: int = 0) -> list[int]:
+    g = torch.Generator().manual_seed(seed)
+    ids = torch.randperm(T, generator=g)[:n].tolist()
+    return sorted(set(ids + [0, T - 1]))

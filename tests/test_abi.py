@@ -1,0 +1,103 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every entry point include/mok.h declares, sizes workspaces, and rejects bad
+arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_device_top_b200 as mok
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(mok_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    L = mok.lib()
+    declared = _declared()
+    assert len(declared) >= 12
+    missing = [n for n in declared if not hasattr(L, n)]
+    assert not missing, missing
+    assert set(mok.EXPORTS) <= set(declared)
+
+
+def test_plan_workspace_sizes():
+    L = mok.lib()
+    assert L.mok_plan_workspace_bytes(8192, 384, 8) > 8192 * 8 * 4 * 7
+    assert L.mok_plan_workspace_bytes(0, 8, 2) > 0            # empty token set is valid
+    assert L.mok_plan_workspace_bytes(16, 8, 9) == 0          # k > E
+    assert L.mok_plan_workspace_bytes(16, 2048, 2) == 0       # E above the built maximum
+    assert L.mok_plan_workspace_bytes(16, 64, 33) == 0        # k above the built maximum
+
+
+def test_forward_workspace_sizes():
+    staged = mok.fwd_opts(mode=mok.MOK_MODE_STAGED)
+    s = mok.forward_workspace_bytes(8192, 7168, 2048, 384, 8, 2560, staged)
+    ns = 8192 * 8
+    assert s >= ns * 7168 * 2 * 2 + ns * 2048 * 2        # rows + out + h
+    p = mok.forward_workspace_bytes(8192, 7168, 2048, 384, 8, 2560, mok.fwd_opts(ring_slots=8192))
+    assert p < s                                          # the ring is smaller than the full buffers
+    assert mok.forward_workspace_bytes(8192, 7168, 2048, 384, 0, 2560, staged) == 0
+
+
+def _plan_call(T, E, k, R, logits=1, ws=None, nbytes=0):
+    p = mok.PlanT()
+    L = mok.lib()
+    rc = L.mok_plan(ctypes.c_void_p(logits), T, E, k, R, ctypes.c_void_p(ws), nbytes, ctypes.byref(p), None)
+    return rc, L.mok_last_error_string().decode()
+
+
+@pytest.mark.parametrize("T,E,k,R,code", [
+    (16, 8, 9, 2, mok.MOK_ERR_INVALID_ARG),      # k > E
+    (16, 8, 0, 2, mok.MOK_ERR_INVALID_ARG),      # k = 0
+    (16, 8, 2, 0, mok.MOK_ERR_INVALID_ARG),      # R = 0
+    (15, 8, 2, 2, mok.MOK_ERR_UNSUPPORTED),      # R does not divide T
+    (16, 2048, 2, 2, mok.MOK_ERR_UNSUPPORTED),   # E above the built maximum
+    (16, 8, 2, 65, mok.MOK_ERR_UNSUPPORTED),     # R above MOK_MAX_SHARDS
+])
+def test_plan_rejects_bad_shapes(T, E, k, R, code):
+    rc, msg = _plan_call(T, E, k, R)
+    assert rc == code, msg
+    assert msg
+
+
+def test_plan_rejects_missing_or_small_workspace():
+    rc, msg = _plan_call(16, 8, 2, 2, ws=0, nbytes=0)
+    assert rc == mok.MOK_ERR_WORKSPACE and "NULL" in msg
+    rc, msg = _plan_call(16, 8, 2, 2, ws=256 * 7 + 128, nbytes=1 << 20)
+    assert rc == mok.MOK_ERR_WORKSPACE and "aligned" in msg
+    rc, msg = _plan_call(16, 8, 2, 2, ws=4096, nbytes=64)
+    assert rc == mok.MOK_ERR_WORKSPACE and "small" in msg
+
+
+def test_forward_rejects_unsupported_shapes():
+    p = mok.PlanT(16, 8, 2, 2)
+    L = mok.lib()
+    arr = (ctypes.c_void_p * 2)(1, 2)
+    rc = L.mok_moe_forward(arr, 100, 256, 1, 1, 1, ctypes.byref(p), 256, None, 256, 1 << 30, arr, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG          # plan views are NULL
+    for name in ("counts", "offsets", "sched_src_rank", "sched_src_index", "row_slot", "pos", "topk_idx", "gates"):
+        setattr(p, name, 4096)
+    rc = L.mok_moe_forward(arr, 100, 256, 1, 1, 1, ctypes.byref(p), 256, None, 256, 1 << 30, arr, None)
+    assert rc == mok.MOK_ERR_UNSUPPORTED and "H" in mok.last_error()
+    rc = L.mok_moe_forward(arr, 128, 100, 1, 1, 1, ctypes.byref(p), 256, None, 256, 1 << 30, arr, None)
+    assert rc == mok.MOK_ERR_UNSUPPORTED and "I" in mok.last_error()
+    o = mok.fwd_opts(mode=7)
+    rc = L.mok_moe_forward(arr, 128, 128, 1, 1, 1, ctypes.byref(p), 256, ctypes.byref(o), 256, 1 << 30, arr, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG
+
+
+def test_get_status_argument_checks():
+    L = mok.lib()
+    rc = L.mok_get_status(None, 0, None, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG
