@@ -113,13 +113,13 @@ def algorithmic_work(cfg):
     """Algorithmic bytes / flops of one forward (one step)."""
     ns = cfg.slots
     w_bytes = cfg.E * 3 * cfg.H * cfg.I * 2
-    gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 2  # weights, rows in, h out+in, out
+    gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 4  # weights, rows in, h out+in, fp32 out
     return {
         "gemm_flops": 6.0 * cfg.H * cfg.I * ns,
         "gemm_bytes": float(gemm_bytes),
         "weight_bytes": float(w_bytes),
         "gather_bytes": float(cfg.T * cfg.H * 2 + ns * cfg.H * 2),
-        "combine_bytes": float(ns * cfg.H * 2 + ns * 4 + cfg.T * cfg.H * 2),
+        "combine_bytes": float(ns * cfg.H * 4 + ns * 4 + cfg.T * cfg.H * 2),
         "plan_bytes": float(cfg.T * cfg.E * 4 + ns * 4 * 8),
     }
 
@@ -131,7 +131,9 @@ def run_mok(args, cfg, rank, world, device):
     x = mokgen.tokens(cfg)
     logits = mokgen.router_logits(cfg, x)
     dx, dlogits = x.to(device), logits.to(device)
-    wg, wu, wd = mokgen.upload_expert_weights(cfg, device)
+    wg, wu, wd_bf16 = mokgen.upload_expert_weights(cfg, device)
+    wd = mok.prepare_w_down(wd_bf16)      # one-time weight preparation, untimed
+    del wd_bf16
     x_shards = mok.shards(dx, cfg.R)
     y = torch.empty_like(dx)
     y_shards = mok.shards(y, cfg.R)
@@ -144,7 +146,7 @@ def run_mok(args, cfg, rank, world, device):
     staged = mode == mok.MOK_MODE_STAGED
     if staged:
         rows = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
-        out = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
+        out = torch.empty((cfg.slots, cfg.H), dtype=torch.float32, device=device)
         ffn_ws = torch.empty(mok.lib().mok_expert_ffn_workspace_bytes(cfg.slots, cfg.I, cfg.E), dtype=torch.uint8,
                              device=device)
     stream = torch.cuda.current_stream()
@@ -279,8 +281,14 @@ def main():
     ap.add_argument("--minibatch", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--scale-experts", type=int, default=0,
+                    help="profiling case: E experts and T scaled by the same factor (same rows per expert)")
     args = ap.parse_args()
     cfg = mokgen.CONFIGS[args.config]
+    if args.scale_experts:
+        n = args.scale_experts
+        T = max(cfg.R, round(cfg.T * n / cfg.E / cfg.R) * cfg.R)
+        cfg = mokgen.scaled(cfg, E=n, T=T)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

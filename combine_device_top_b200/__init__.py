@@ -35,6 +35,7 @@ EXPORTS = (
     "mok_plan_workspace_bytes", "mok_plan", "mok_forward_workspace_bytes", "mok_moe_forward",
     "mok_get_status", "mok_last_error_string", "mok_gather", "mok_expert_ffn_workspace_bytes",
     "mok_expert_ffn", "mok_combine", "mok_forward_host_workspace_bytes", "mok_moe_forward_host",
+    "mok_prepare_w_down",
 )
 
 
@@ -83,8 +84,9 @@ def lib() -> ctypes.CDLL:
     L.mok_forward_host_workspace_bytes.restype = sz
     L.mok_moe_forward_host.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32,
                                        ctypes.POINTER(FwdOpts), vp, sz, vp, vp]
+    L.mok_prepare_w_down.argtypes = [vp, vp, sz, vp]
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
-              "mok_moe_forward_host"):
+              "mok_moe_forward_host", "mok_prepare_w_down"):
         getattr(L, n).restype = ctypes.c_int
     return L
 
@@ -165,6 +167,16 @@ def plan(logits: torch.Tensor, top_k: int, R: int, ws: torch.Tensor | None = Non
     return Plan(p, ws)
 
 
+def prepare_w_down(w_down: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One-time fp16 copy of a bf16 W_down [E, I, H] (``mok_prepare_w_down``)."""
+    assert w_down.is_cuda and w_down.dtype == torch.bfloat16 and w_down.is_contiguous()
+    if out is None:
+        out = torch.empty(w_down.shape, dtype=torch.float16, device=w_down.device)
+    _check(lib().mok_prepare_w_down(ctypes.c_void_p(w_down.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                    w_down.numel(), _stream(stream)))
+    return out
+
+
 def fwd_opts(mode: int = MOK_MODE_PERSISTENT, ring_slots: int = 0, dispatch_ctas: int = 0, gemm_ctas: int = 0,
              mxfp8: bool = False, timeout_ns: int = 0) -> FwdOpts:
     return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), 0, timeout_ns)
@@ -222,11 +234,12 @@ def gather(x_shards, p: Plan, rows: torch.Tensor | None = None, stream=None) -> 
 
 
 def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
-    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] slot-indexed, ws)."""
+    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] fp32 slot-indexed, ws)."""
     H = rows.shape[1]
     I = w_gate.shape[-1]
     if out is None:
-        out = torch.empty((p.ns, H), dtype=torch.bfloat16, device=rows.device)
+        out = torch.empty((p.ns, H), dtype=torch.float32, device=rows.device)
+    assert out.dtype == torch.float32
     if ws is None:
         ws = _workspace(lib().mok_expert_ffn_workspace_bytes(p.ns, I, p.c.E), rows.device)
     _check(lib().mok_expert_ffn(ctypes.c_void_p(rows.data_ptr()), H, I, ctypes.c_void_p(w_gate.data_ptr()),
@@ -237,6 +250,8 @@ def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = N
 
 
 def combine(out: torch.Tensor, p: Plan, y_shards, stream=None):
+    """y = fixed-order gate-weighted sum of the fp32 per-slot outputs."""
+    assert out.dtype == torch.float32
     H = out.shape[-1]
     _check(lib().mok_combine(ctypes.c_void_p(out.data_ptr()), H, ctypes.byref(p.c), _ptr_array(y_shards),
                              _stream(stream)))

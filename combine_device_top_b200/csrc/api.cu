@@ -65,8 +65,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                         uint32_t box_outer, const char** err) {
+bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
+                        uint32_t box_inner, uint32_t box_outer, const char** err) {
     auto enc = get_encode();
     if (!enc) {
         *err = "cuTensorMapEncodeTiled unavailable";
@@ -76,7 +76,8 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uin
     cuuint64_t strides[1] = {inner * 2};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -128,7 +129,7 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
     l.counters = take(sizeof(int) * 4 * (size_t)l.max_mb + 256);
     l.rows = take((size_t)l.buf_rows * H * 2);
     l.h = take((size_t)l.buf_rows * I * 2);
-    l.out = take((size_t)ns * H * 2);
+    l.out = take((size_t)ns * H * 4);
     l.total = off;
     *L = l;
     return true;
@@ -169,11 +170,11 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
     MOK_CUDA(gemm_configure(dev), "gemm configure");
     CUtensorMap tm_wg, tm_wu, tm_wd, tm_rows, tm_h;
     const char* err = nullptr;
-    if (!encode_tmap_2d_bf16(&tm_wg, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
-        !encode_tmap_2d_bf16(&tm_wu, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
-        !encode_tmap_2d_bf16(&tm_wd, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, &err) ||
-        !encode_tmap_2d_bf16(&tm_rows, rows, (uint64_t)H, (uint64_t)n_rows_buf, 64, 16, &err) ||
-        !encode_tmap_2d_bf16(&tm_h, h, (uint64_t)I, (uint64_t)n_rows_buf, 64, 16, &err))
+    if (!encode_tmap_2d_16b(&tm_wg, true, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
+        !encode_tmap_2d_16b(&tm_wu, true, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
+        !encode_tmap_2d_16b(&tm_wd, false, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, &err) ||
+        !encode_tmap_2d_16b(&tm_rows, true, rows, (uint64_t)H, (uint64_t)n_rows_buf, 64, 16, &err) ||
+        !encode_tmap_2d_16b(&tm_h, false, h, (uint64_t)I, (uint64_t)n_rows_buf, 64, 16, &err))
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
     GemmShape sh{H, I, E};
     MOK_CUDA(launch_gemm_phase(0, tm_wg, tm_wu, tm_rows, sh, chunks, counts2, h, out, row_slot, status, timeout_ns,
@@ -292,6 +293,21 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
                         base + L.h, base + L.out, status, timeout, stream);
     if (rc) return rc;
     MOK_CUDA(launch_combine(base + L.out, plan->gates, T, k, H, T / R, ys, sms, stream), "combine launch");
+    return MOK_OK;
+}
+
+int mok_prepare_w_down(const void* w_down_bf16, void* w_down_fp16, size_t count, mok_stream_t stream) {
+    if (count == 0) return MOK_OK;
+    if (!w_down_bf16 || !w_down_fp16) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(w_down_bf16) | reinterpret_cast<uintptr_t>(w_down_fp16)) & 15u)
+        return fail(MOK_ERR_UNSUPPORTED, "weight buffers must be 16-byte aligned");
+    const char* a = static_cast<const char*>(w_down_bf16);
+    const char* b = static_cast<const char*>(w_down_fp16);
+    if (a < b + count * 2 && b < a + count * 2) return fail(MOK_ERR_INVALID_ARG, "source and destination overlap");
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_bf16_to_fp16(w_down_bf16, w_down_fp16, count, sms, reinterpret_cast<cudaStream_t>(stream)),
+             "weight conversion launch");
     return MOK_OK;
 }
 

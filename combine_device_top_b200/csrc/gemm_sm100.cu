@@ -15,10 +15,15 @@
 //     columns of Wu (M = 128, K = H, read MN-major straight from the
 //     [E, H, I] layout), B = the chunk's token rows (K-major).  Accumulator
 //     lanes 0-63 hold gate, 64-127 up; the epilogue forms
-//     h = silu(gate) * up and stores bf16 h rows.
-//   down unit (phase 1): A = 128 columns of Wd (MN-major from [E, I, H]),
-//     B = the chunk's h rows; the epilogue stores bf16 rows to
-//     out[row_slot[row]] (the push combine).
+//     h = silu(gate) * up and stores fp16 h rows.
+//   down unit (phase 1): A = 128 columns of the fp16 copy of Wd (MN-major
+//     from [E, I, H]), B = the chunk's fp16 h rows; fp16 keeps 3 more
+//     mantissa bits of h than bf16 would, which is what keeps the largest
+//     element error of y near the floor set by rounding y itself to bf16.
+//     The epilogue stores fp32 rows to
+//     out[row_slot[row]] (the push combine).  fp32 rather than bf16: with a
+//     bf16 slot buffer the three bf16 roundings (h, o, y) put the largest
+//     element error of y above 2e-2 * rms(y) on heavy-tailed outputs.
 //
 // Roles in a CTA of 6 warps: warp 0 issues TMA loads into a 4-stage ring
 // of 48 KB stages, warp 1 allocates 512 TMEM columns and one thread of it
@@ -59,8 +64,8 @@ struct GemmParams {
     int MT;              // M tiles per chunk
     int w_rows;          // rows per expert in the A tensor map (H or I)
     int I, H;
-    __nv_bfloat16* h_out;     // phase 0: [rows, I]
-    __nv_bfloat16* out;       // phase 1: [N_s, H] slot-indexed
+    __half* h_out;            // phase 0: [rows, I] fp16
+    float* out;               // phase 1: [N_s, H] fp32, slot-indexed
     const int32_t* row_slot;  // phase 1
     DevStatus* st;
     uint64_t timeout_ns;
@@ -178,7 +183,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 unit_map(u, nch, p.MT, c, m);
                 const Chunk ck = p.chunks[c];
                 const int N = (ck.rows + 15) & ~15;
-                const uint32_t idesc = umma_idesc_bf16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0);
+                // gate/up: bf16 x bf16; down: fp16 x fp16 (fp16 W_down copy, fp16 h)
+                const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, PHASE == 0);
                 if (!mbar_wait(&tempty[tb], tph ^ 1u, p.st, p.timeout_ns, 20)) break;
                 tc_fence_after();
                 const uint32_t dt = tmem_base + (uint32_t)(tb * ACC_COLS);
@@ -255,24 +261,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                             const float u1 = epi[(64 + fq * 16 + i + 1) * EPI_LD + tok];
                             const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
                             const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                            pk[i >> 1] = pack_bf16x2(h0, h1);
+                            pk[i >> 1] = pack_half2_sat(h0, h1);
                         }
                         uint4* dst = reinterpret_cast<uint4*>(p.h_out + (size_t)(ck.row0 + col) * p.I + m * 64 + fq * 16);
                         dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     } else {
+                        // fp32 push: the combine reads these once more and rounds y once
                         const int slot = __ldg(p.row_slot + ck.row0 + col);
-                        uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)slot * p.H + m * 128 + fq * 32);
+                        float4* dst = reinterpret_cast<float4*>(p.out + (size_t)slot * p.H + m * 128 + fq * 32);
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int i = 0; i < 8; i += 2) {
-                                const float a = epi[(fq * 32 + q4 * 8 + i) * EPI_LD + tok];
-                                const float b = epi[(fq * 32 + q4 * 8 + i + 1) * EPI_LD + tok];
-                                pk[i >> 1] = pack_bf16x2(a, b);
-                            }
-                            dst[q4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const int f = fq * 32 + q4 * 4;
+                            dst[q4] = make_float4(epi[f * EPI_LD + tok], epi[(f + 1) * EPI_LD + tok],
+                                                  epi[(f + 2) * EPI_LD + tok], epi[(f + 3) * EPI_LD + tok]);
                         }
                     }
                 }
@@ -451,8 +453,8 @@ cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensor
     p.w_rows = phase == 0 ? sh.H : sh.I;
     p.I = sh.I;
     p.H = sh.H;
-    p.h_out = reinterpret_cast<__nv_bfloat16*>(h_out);
-    p.out = reinterpret_cast<__nv_bfloat16*>(out);
+    p.h_out = reinterpret_cast<__half*>(h_out);
+    p.out = reinterpret_cast<float*>(out);
     p.row_slot = row_slot;
     p.st = reinterpret_cast<DevStatus*>(status);
     p.timeout_ns = timeout_ns;

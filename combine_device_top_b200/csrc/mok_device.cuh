@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -177,11 +178,13 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
-// Instruction descriptor, kind::f16, bf16 x bf16 -> fp32:
-// [4,6) D fmt (1 = f32), [7,10) A fmt (1 = bf16), [10,13) B fmt (1 = bf16),
+// Instruction descriptor, kind::f16 with fp32 accumulation; A and B share
+// one type (bf16 when `bf16` is set, else fp16):
+// [4,6) D fmt (1 = f32), [7,10) A fmt (0 = f16, 1 = bf16), [10,13) B fmt,
 // [15] A major (1 = MN), [16] B major (1 = MN), [17,23) N>>3, [24,29) M>>4.
-__host__ __device__ __forceinline__ uint32_t umma_idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
+__host__ __device__ __forceinline__ uint32_t umma_idesc_f16(int M, int N, int a_mn_major, int b_mn_major, int bf16) {
+    const uint32_t t = bf16 ? 1u : 0u;
+    return (1u << 4) | (t << 7) | (t << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
@@ -232,6 +235,15 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two fp32 -> fp16x2, round to nearest even, magnitudes above 65504 clamped
+// to 65504.
+__device__ __forceinline__ uint32_t pack_half2_sat(float a, float b) {
+    a = fminf(fmaxf(a, -65504.f), 65504.f);
+    b = fminf(fmaxf(b, -65504.f), 65504.f);
+    __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 

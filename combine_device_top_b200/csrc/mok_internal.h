@@ -64,7 +64,12 @@ cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensor
                               cudaStream_t stream);
 
 // ---- tensor maps (driver entry point fetched at run time)
-bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                         uint32_t box_outer, const char** err);
+// 2D tiled map of a row-major [outer, inner] array of 16-bit elements
+// (bf16 or fp16), 128-byte swizzle, zero fill out of bounds.
+bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
+                        uint32_t box_inner, uint32_t box_outer, const char** err);
+
+// ---- weight preparation
+cudaError_t launch_bf16_to_fp16(const void* src, void* dst, size_t n, int num_sms, cudaStream_t stream);
 
 }  // namespace mok

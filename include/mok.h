@@ -143,9 +143,10 @@ size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int miniba
  * merge); MoK wiki summary, key points (SM split, TMA, local counters).
  *   x_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
  *   H, I      hidden and intermediate sizes; H % 128 == 0, I % 64 == 0
- *   w_gate    [E, H, I] bf16 (bf16 mode) or an MXFP8 weight pack
- *   w_up      [E, H, I] bf16 (bf16 mode) or an MXFP8 weight pack
- *   w_down    [E, I, H] bf16 (bf16 mode) or an MXFP8 weight pack
+ *   w_gate    [E, H, I] bf16
+ *   w_up      [E, H, I] bf16
+ *   w_down    [E, I, H] fp16: the copy mok_prepare_w_down() makes of the
+ *             bf16 W_down (once, at weight-load time)
  *   plan      from mok_plan() on the same stream (its workspace must live)
  *   minibatch rows of the expert-major layout per minibatch (persistent
  *             mode; >= 16); boundaries snap forward to expert boundaries
@@ -153,15 +154,30 @@ size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int miniba
  *   opts      may be NULL (persistent mode, defaults)
  *   ws        forward workspace (>= mok_forward_workspace_bytes)
  *   y_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
- * Arithmetic: bf16 inputs, fp32 accumulation, h stored bf16, each expert
- * output row stored bf16 at its slot, y[t] = bf16(sum_{j<k} g[t,j] *
- * o[t,j]) accumulated in fp32 with j ascending.  y does not depend on the
+ * Arithmetic: gate/up in bf16 x bf16 with fp32 accumulation; h =
+ * silu(gate) * up rounded to fp16 (saturating at +-65504); down projection
+ * fp16 x fp16 with fp32 accumulation; each expert output row stored fp32 at
+ * its slot; y[t] = bf16(sum_{j<k} g[t,j] * o[t,j]) accumulated in fp32
+ * with j ascending (one bf16 rounding of y).  y does not depend on the
  * mode, minibatch, ring size or R.
  */
 int mok_moe_forward(const void* const* x_shards, int H, int I,
                     const void* w_gate, const void* w_up, const void* w_down,
                     const mok_plan_t* plan, int minibatch, const mok_fwd_opts* opts,
                     void* ws, size_t ws_bytes, void* const* y_shards, mok_stream_t stream);
+
+/*
+ * mok_prepare_w_down -- one-time conversion of W_down from bf16 to the fp16
+ * copy the forward's down projection reads (elementwise, `count` elements,
+ * e.g. E*I*H).  Exact for every bf16 value of magnitude in [2^-14, 65504];
+ * smaller magnitudes round to fp16's subnormal grid (spacing 2^-24), larger
+ * ones saturate to +-65504.  Both buffers are device memory owned by the
+ * caller, 16-byte aligned, not overlapping.  Asynchronous on `stream`.
+ * (No counterpart in the pages: it serves the down projection's fp16
+ * arithmetic, which keeps the error of y near the floor of its own bf16
+ * rounding.)
+ */
+int mok_prepare_w_down(const void* w_down_bf16, void* w_down_fp16, size_t count, mok_stream_t stream);
 
 /*
  * mok_get_status -- synchronise `stream` and read the device status word of
@@ -188,9 +204,10 @@ int mok_gather(const void* const* x_shards, int H, const mok_plan_t* plan,
 size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E);
 
 /* Grouped SwiGLU FFN over the expert-major rows of `plan`:
- *   h[row]   = bf16(silu(rows[row] Wg[e]) * (rows[row] Wu[e]))   [N_s, I]
- *   out[row_slot[row]] = bf16(h[row] Wd[e])                         [N_s, H]
- * (e = expert of the row).  h is returned in the workspace only; `out` is
+ *   h[row]   = fp16(silu(rows[row] Wg[e]) * (rows[row] Wu[e]))   [N_s, I]
+ *   out[row_slot[row]] = h[row] Wd16[e]   (fp32)                 [N_s, H]
+ * (e = expert of the row; Wd16 = fp16 W_down from mok_prepare_w_down).
+ * h stays in the workspace; `out` is fp32 and
  * slot-indexed, i.e. [T, k, H].  Source: MoK article, routing paragraph
  * (grouped GEMM over contiguous per-expert tokens) and push-combine
  * paragraph. */
@@ -199,8 +216,8 @@ int mok_expert_ffn(const void* rows, int H, int I,
                    const mok_plan_t* plan, void* ws, size_t ws_bytes,
                    void* out, mok_stream_t stream);
 
-/* y[t] = bf16(sum_{j<k} gates[t,j] * float(out[t,j,:])), fp32, j ascending,
- * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] bf16.
+/* y[t] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]), fp32, j ascending,
+ * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] fp32.
  * Source: MoK article, benchmark paragraph (final weighted merge). */
 int mok_combine(const void* out, int H, const mok_plan_t* plan,
                 void* const* y_shards, mok_stream_t stream);
@@ -217,7 +234,7 @@ size_t mok_forward_host_workspace_bytes(int T, int H, int I, int E, int k, int m
  * mok_moe_forward_host -- copies HOST x [T, H] bf16 and HOST logits [T, E]
  * fp32 to the device, runs mok_plan and mok_moe_forward, copies y [T, H]
  * bf16 back to HOST memory and synchronises `stream`.  Weights are device
- * pointers as in mok_moe_forward.  Host buffers should be pinned for
+ * pointers as in mok_moe_forward (w_down: the fp16 copy).  Host buffers should be pinned for
  * full copy bandwidth (pageable memory works, slower).  ws: device
  * workspace of mok_forward_host_workspace_bytes().
  */

@@ -45,12 +45,17 @@ class Case:
         self.x = mokgen.tokens(cfg)
         self.logits = mokgen.router_logits(cfg, self.x)
         self.device = device
+        import combine_device_top_b200 as mok
+
         if weights_on_host:
             self.wg, self.wu, self.wd = mokgen.all_expert_weights(cfg)
-            self.dwg, self.dwu, self.dwd = (w.to(device) for w in (self.wg, self.wu, self.wd))
+            self.dwg, self.dwu, dwd = (w.to(device) for w in (self.wg, self.wu, self.wd))
         else:
             self.wg = self.wu = self.wd = None
-            self.dwg, self.dwu, self.dwd = mokgen.upload_expert_weights(cfg, device)
+            self.dwg, self.dwu, dwd = mokgen.upload_expert_weights(cfg, device)
+        # the forward reads the one-time fp16 copy of W_down
+        self.dwd = mok.prepare_w_down(dwd)
+        del dwd
         self.dx = self.x.to(device)
         self.dlogits = self.logits.to(device)
 
