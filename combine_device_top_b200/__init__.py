@@ -17,7 +17,8 @@ from functools import lru_cache
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmok.so")
+# MOK_LIB_PATH selects another build of the same ABI (e.g. a debug build)
+LIB_PATH = os.environ.get("MOK_LIB_PATH") or os.path.join(_PKG, "libmok.so")
 
 MOK_OK = 0
 MOK_ERR_INVALID_ARG = 1

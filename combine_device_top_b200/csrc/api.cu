@@ -87,6 +87,13 @@ bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t 
     return true;
 }
 
+bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint64_t rows, const char** err) {
+    for (int i = 0; i < B_MAPS; ++i)
+        if (!encode_tmap_2d_16b(&maps->m[i], bf16, base, inner, rows, 64, (uint32_t)(B_MAX_BOX >> i), err))
+            return false;
+    return true;
+}
+
 // ------------------------------------------------------------------ layouts
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -168,20 +175,22 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
     const int sms = device_sms(&dev);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     MOK_CUDA(gemm_configure(dev), "gemm configure");
-    CUtensorMap tm_wg, tm_wu, tm_wd, tm_rows, tm_h;
+    CUtensorMap tm_wg, tm_wu, tm_wd;
+    BMaps tm_rows, tm_h;
     const char* err = nullptr;
     if (!encode_tmap_2d_16b(&tm_wg, true, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
         !encode_tmap_2d_16b(&tm_wu, true, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
         !encode_tmap_2d_16b(&tm_wd, false, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, &err) ||
-        !encode_tmap_2d_16b(&tm_rows, true, rows, (uint64_t)H, (uint64_t)n_rows_buf, 64, 16, &err) ||
-        !encode_tmap_2d_16b(&tm_h, false, h, (uint64_t)I, (uint64_t)n_rows_buf, 64, 16, &err))
+        !encode_bmaps(&tm_rows, true, rows, (uint64_t)H, (uint64_t)n_rows_buf, &err) ||
+        !encode_bmaps(&tm_h, false, h, (uint64_t)I, (uint64_t)n_rows_buf, &err))
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
     GemmShape sh{H, I, E};
+    const GemmTuning tune = gemm_tuning();
     MOK_CUDA(launch_gemm_phase(0, tm_wg, tm_wu, tm_rows, sh, chunks, counts2, h, out, row_slot, status, timeout_ns,
-                               sms, stream),
+                               sms, tune, stream),
              "gate/up GEMM launch");
     MOK_CUDA(launch_gemm_phase(1, tm_wd, tm_wd, tm_h, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
-                               stream),
+                               tune, stream),
              "down GEMM launch");
     return MOK_OK;
 }

@@ -41,15 +41,13 @@ constexpr int NSTAGE = 4;
 constexpr int BK = 64;                       // K per stage: one 128-byte swizzle atom of bf16
 constexpr int A_BYTES = 128 * BK * 2;        // 16 KB: two {64 MN x 64 K} boxes
 constexpr int B_ROWS_MAX = CHUNK_MAX_ROWS;   // 256
-constexpr int B_BOX_ROWS = 16;
-constexpr int B_BOX_BYTES = B_BOX_ROWS * BK * 2;   // 2 KB
+constexpr int B_ROW_BYTES = BK * 2;               // 128 bytes of one token row per stage
 constexpr int B_BYTES = B_ROWS_MAX * BK * 2;       // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // 48 KB
 constexpr int EPI_LD = 33;                          // fp32 staging row pitch (bank-conflict free)
 constexpr int EPI_BYTES = 128 * EPI_LD * 4;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
-constexpr int GROUP_CHUNKS = 8;                     // raster: chunks per group
 
 constexpr int SMEM_STAGES_OFF = 0;
 constexpr int SMEM_EPI_OFF = NSTAGE * STAGE_BYTES;
@@ -69,13 +67,19 @@ struct GemmParams {
     const int32_t* row_slot;  // phase 1
     DevStatus* st;
     uint64_t timeout_ns;
+    int l2_prefetch;     // k-steps of weight tiles prefetched into L2 ahead of the loads
+    int group_chunks;    // raster: chunks per group (see unit_map)
 };
 
-__device__ __forceinline__ void unit_map(int u, int nch, int MT, int& c, int& m) {
-    const int grp = u / (GROUP_CHUNKS * MT);
-    const int rem = u - grp * GROUP_CHUNKS * MT;
-    const int c0 = grp * GROUP_CHUNKS;
-    const int gsz = min(GROUP_CHUNKS, nch - c0);
+// Unit u -> (chunk c, M tile m).  Units are rastered in groups of GC chunks:
+// inside a group the chunk index runs fastest, so the CTAs running at one
+// time share a few chunks' token tiles (L2) while streaming distinct weight
+// tiles.
+__device__ __forceinline__ void unit_map(int u, int nch, int MT, int GC, int& c, int& m) {
+    const int grp = u / (GC * MT);
+    const int rem = u - grp * GC * MT;
+    const int c0 = grp * GC;
+    const int gsz = min(GC, nch - c0);
     m = rem / gsz;
     c = c0 + (rem - m * gsz);
 }
@@ -83,7 +87,7 @@ __device__ __forceinline__ void unit_map(int u, int nch, int MT, int& c, int& m)
 template <int PHASE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                   const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+                   const __grid_constant__ BMaps tmB, const GemmParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA0);
         tma_prefetch_desc(&tmA1);
-        tma_prefetch_desc(&tmB);
+        for (int i = 0; i < B_MAPS; ++i) tma_prefetch_desc(&tmB.m[i]);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -134,12 +138,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t phase = 0;
             uint32_t issued = 0, issued_phase = 0;  // bit s: stage s holds a load of phase bit s
             bool ok = true;
+            const uint64_t evict_first = l2_policy_evict_first();
+            // Look-ahead cursor: the weight tiles of the k-step p.l2_prefetch
+            // steps ahead are prefetched into L2, so that more weight bytes are
+            // in flight per SM than the shared-memory stages alone hold.
+            int pu = blockIdx.x, pkb = 0, pm = 0, pe = 0, pu_mapped = -1;
+            auto prefetch_next = [&]() {
+                if (pu >= nunits) return;
+                if (pu != pu_mapped) {
+                    int c;
+                    unit_map(pu, nch, p.MT, p.group_chunks, c, pm);
+                    pe = p.chunks[c].expert;
+                    pu_mapped = pu;
+                }
+                const int ky = pe * p.w_rows + pkb * BK;
+                if (PHASE == 0) {
+                    tma_prefetch_l2_2d(&tmA0, pm * 64, ky);
+                    tma_prefetch_l2_2d(&tmA1, pm * 64, ky);
+                } else {
+                    tma_prefetch_l2_2d(&tmA0, pm * 128, ky);
+                    tma_prefetch_l2_2d(&tmA0, pm * 128 + 64, ky);
+                }
+                if (++pkb == KB) {
+                    pkb = 0;
+                    pu += gridDim.x;
+                }
+            };
+            for (int i = 0; i < p.l2_prefetch; ++i) prefetch_next();
             for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
                 int c, m;
-                unit_map(u, nch, p.MT, c, m);
+                unit_map(u, nch, p.MT, p.group_chunks, c, m);
                 const Chunk ck = p.chunks[c];
-                const int nbox = (ck.rows + B_BOX_ROWS - 1) / B_BOX_ROWS;
-                const uint32_t bytes = A_BYTES + nbox * B_BOX_BYTES;
+                // token rows rounded up to 16, loaded as one box per set bit
+                // (256, 128, 64, 32, 16 rows): at most 5 TMA ops per stage
+                const int r16 = (ck.rows + 15) & ~15;
+                const uint32_t bytes = A_BYTES + r16 * B_ROW_BYTES;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.st, p.timeout_ns, 10)) {
                         ok = false;
@@ -150,14 +183,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     const int ky = ck.expert * p.w_rows + kb * BK;
                     if (PHASE == 0) {
-                        tma_load_2d(sa, &tmA0, &full[stage], m * 64, ky);
-                        tma_load_2d(sa + A_BYTES / 2, &tmA1, &full[stage], m * 64, ky);
+                        tma_load_2d_hint(sa, &tmA0, &full[stage], m * 64, ky, evict_first);
+                        tma_load_2d_hint(sa + A_BYTES / 2, &tmA1, &full[stage], m * 64, ky, evict_first);
                     } else {
-                        tma_load_2d(sa, &tmA0, &full[stage], m * 128, ky);
-                        tma_load_2d(sa + A_BYTES / 2, &tmA0, &full[stage], m * 128 + 64, ky);
+                        tma_load_2d_hint(sa, &tmA0, &full[stage], m * 128, ky, evict_first);
+                        tma_load_2d_hint(sa + A_BYTES / 2, &tmA0, &full[stage], m * 128 + 64, ky, evict_first);
                     }
-                    for (int j = 0; j < nbox; ++j)
-                        tma_load_2d(sb + j * B_BOX_BYTES, &tmB, &full[stage], kb * BK, ck.row0 + j * B_BOX_ROWS);
+                    if (p.l2_prefetch > 0) prefetch_next();
+                    int roff = 0;
+#pragma unroll
+                    for (int i = 0; i < B_MAPS; ++i) {
+                        const int sz = B_MAX_BOX >> i;
+                        if (r16 & sz) {
+                            tma_load_2d(sb + roff * B_ROW_BYTES, &tmB.m[i], &full[stage], kb * BK, ck.row0 + roff);
+                            roff += sz;
+                        }
+                    }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == NSTAGE) {
@@ -180,7 +221,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
                 int c, m;
-                unit_map(u, nch, p.MT, c, m);
+                unit_map(u, nch, p.MT, p.group_chunks, c, m);
                 const Chunk ck = p.chunks[c];
                 const int N = (ck.rows + 15) & ~15;
                 // gate/up: bf16 x bf16; down: fp16 x fp16 (fp16 W_down copy, fp16 h)
@@ -237,7 +278,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (!ok) break;
             tc_fence_after();
             int c, m;
-            unit_map(u, nch, p.MT, c, m);
+            unit_map(u, nch, p.MT, p.group_chunks, c, m);
             const Chunk ck = p.chunks[c];
             const int ncc = (ck.rows + 31) >> 5;
             const int tok = et & 31, fq = et >> 5;
@@ -430,6 +471,17 @@ cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int 
 
 size_t gemm_smem_bytes() { return SMEM_ALLOC; }
 
+// Defaults measured on B200 (page shape and a 512-rows-per-expert case):
+// L2 prefetch of weight tiles did not pay (the token-side TMA op count was
+// the limit), small raster groups did.  MOK_GEMM_L2_PREFETCH and
+// MOK_GEMM_GROUP override them (tuning knobs only, results do not change).
+GemmTuning gemm_tuning() {
+    GemmTuning v{0, 2};
+    if (const char* s = getenv("MOK_GEMM_L2_PREFETCH")) v.l2_prefetch = atoi(s) < 0 ? 0 : atoi(s);
+    if (const char* s = getenv("MOK_GEMM_GROUP")) v.group_chunks = atoi(s) < 1 ? 1 : atoi(s);
+    return v;
+}
+
 cudaError_t gemm_configure(int dev) {
     static bool done[64] = {};
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -441,10 +493,10 @@ cudaError_t gemm_configure(int dev) {
     return e;
 }
 
-cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmB,
+cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensorMap& tmA1, const BMaps& tmB,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              cudaStream_t stream) {
+                              const GemmTuning& tune, cudaStream_t stream) {
     GemmParams p;
     p.chunks = chunks;
     p.counts2 = counts2;
@@ -458,6 +510,8 @@ cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensor
     p.row_slot = row_slot;
     p.st = reinterpret_cast<DevStatus*>(status);
     p.timeout_ns = timeout_ns;
+    p.l2_prefetch = tune.l2_prefetch;
+    p.group_chunks = tune.group_chunks > 0 ? tune.group_chunks : 1;
     if (phase == 0)
         k_grouped_gemm<0><<<grid, GEMM_THREADS, SMEM_ALLOC, stream>>>(tmA0, tmA1, tmB, p);
     else

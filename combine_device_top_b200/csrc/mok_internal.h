@@ -54,14 +54,29 @@ cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int 
 struct GemmShape {
     int H, I, E;
 };
+struct GemmTuning {
+    int l2_prefetch;   // k-steps of weight tiles prefetched into L2 ahead of the loads
+    int group_chunks;  // raster group size in chunks
+};
+GemmTuning gemm_tuning();  // defaults, overridable by MOK_GEMM_L2_PREFETCH / MOK_GEMM_GROUP
 size_t gemm_smem_bytes();
 cudaError_t gemm_configure(int dev);
+// Token-side (B operand) tensor maps of one buffer with box heights
+// 256, 128, 64, 32, 16 rows: a chunk of r rows (rounded up to 16) is loaded
+// as one box per set bit of r.
+constexpr int B_MAPS = 5;
+constexpr int B_MAX_BOX = 256;
+struct BMaps {
+    CUtensorMap m[B_MAPS];
+};
+bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint64_t rows, const char** err);
+
 // Staged grouped GEMM over every chunk: phase 0 = gate/up + SwiGLU -> h,
 // phase 1 = down -> out[row_slot].  Tensor maps are built by the caller.
-cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmB,
+cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensorMap& tmA1, const BMaps& tmB,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out,
                               void* out, const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              cudaStream_t stream);
+                              const GemmTuning& tune, cudaStream_t stream);
 
 // ---- tensor maps (driver entry point fetched at run time)
 // 2D tiled map of a row-major [outer, inner] array of 16-bit elements
