@@ -36,7 +36,7 @@ EXPORTS = (
     "mok_plan_workspace_bytes", "mok_plan", "mok_forward_workspace_bytes", "mok_moe_forward",
     "mok_get_status", "mok_last_error_string", "mok_gather", "mok_expert_ffn_workspace_bytes",
     "mok_expert_ffn", "mok_combine", "mok_forward_host_workspace_bytes", "mok_moe_forward_host",
-    "mok_prepare_w_down",
+    "mok_prepare_w_down", "mok_plan_noalloc",
 )
 
 
@@ -86,8 +86,9 @@ def lib() -> ctypes.CDLL:
     L.mok_moe_forward_host.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32,
                                        ctypes.POINTER(FwdOpts), vp, sz, vp, vp]
     L.mok_prepare_w_down.argtypes = [vp, vp, sz, vp]
+    L.mok_plan_noalloc.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
-              "mok_moe_forward_host", "mok_prepare_w_down"):
+              "mok_moe_forward_host", "mok_prepare_w_down", "mok_plan_noalloc"):
         getattr(L, n).restype = ctypes.c_int
     return L
 

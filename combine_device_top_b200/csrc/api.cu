@@ -28,6 +28,8 @@ static int fail(int code, const char* fmt, ...) {
     return code;
 }
 
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 static int cuda_fail(cudaError_t e, const char* what) {
     return fail(MOK_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }

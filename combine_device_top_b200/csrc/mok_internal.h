@@ -19,6 +19,13 @@ struct PlanLayout {
 size_t plan_layout(int T, int E, int k, PlanLayout* L);
 cudaError_t launch_plan(const float* logits, int T, int E, int k, int R, unsigned char* ws, const PlanLayout& L,
                         cudaStream_t stream);
+int plan_route_blocks(int T);
+cudaError_t launch_plan_parts(const float* logits, int T, int E, int k, int R, int32_t* counts, int32_t* offsets,
+                              int32_t* src_rank, int32_t* src_index, int32_t* row_slot, int32_t* pos,
+                              int32_t* topk_idx, float* gates, int32_t* blk_cnt, int32_t* rank,
+                              cudaStream_t stream);
+// Records a message for mok_last_error_string() and returns `code`.
+int report_error(int code, const char* msg);
 
 // ---- token shards as kernel parameters
 struct ShardsIn {

@@ -248,4 +248,32 @@ cudaError_t launch_plan(const float* logits, int T, int E, int k, int R, unsigne
     return cudaGetLastError();
 }
 
+// The same three launches with every array given explicitly (outputs and
+// the two scratch arrays: blk_cnt [ceil(T/256), E] and rank [T*k]).
+int plan_route_blocks(int T) { return (T + PLAN_TOK - 1) / PLAN_TOK; }
+
+cudaError_t launch_plan_parts(const float* logits, int T, int E, int k, int R, int32_t* counts, int32_t* offsets,
+                              int32_t* src_rank, int32_t* src_index, int32_t* row_slot, int32_t* pos,
+                              int32_t* topk_idx, float* gates, int32_t* blk_cnt, int32_t* rank,
+                              cudaStream_t stream) {
+    const size_t smem = sizeof(int32_t) * PLAN_TOK * k + sizeof(uint32_t) * PLAN_WARPS * E;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_route, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(sizeof(int32_t) * PLAN_TOK * MOK_MAX_TOPK +
+                                                   sizeof(uint32_t) * PLAN_WARPS * MOK_MAX_EXPERTS));
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
+    const int nb = plan_route_blocks(T);
+    if (T > 0) k_route<<<nb, PLAN_THREADS, smem, stream>>>(logits, T, E, k, topk_idx, gates, blk_cnt, rank);
+    k_scan<<<1, 1024, 0, stream>>>(blk_cnt, nb, E, T * k, counts, offsets);
+    if (T > 0)
+        k_scatter<<<nb, PLAN_THREADS, 0, stream>>>(topk_idx, rank, blk_cnt, offsets, T, E, k, T / R, src_rank,
+                                                   src_index, row_slot, pos);
+    return cudaGetLastError();
+}
+
 }  // namespace mok

@@ -104,6 +104,40 @@ size_t mok_plan_workspace_bytes(int T, int E, int k);
 int mok_plan(const float* logits, int T, int E, int top_k, int R,
              void* ws, size_t ws_bytes, mok_plan_t* plan, mok_stream_t stream);
 
+/* Size of the library-owned scratch array used by mok_plan_noalloc. */
+#define MOK_PLAN_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/*
+ * mok_plan_noalloc -- mok_plan for callers that cannot allocate device
+ * memory: code recording a stream capture (allocation is not allowed
+ * there), allocator-less runtimes that only hand out pre-registered
+ * buffers, or hooks that must not touch the device allocator.  The paper
+ * has no counterpart; this is a convenience of this library.
+ *   Same inputs and the same results as mok_plan, bit for bit, but the
+ *   caller passes the eight output arrays directly (device memory it owns:
+ *   counts [E], offsets [E+1], sched_src_rank / sched_src_index / row_slot /
+ *   pos / topk_idx [T*k] int32, gates [T*k] fp32) and no workspace.
+ *   The plan's internal scratch lives in one static device array of
+ *   MOK_PLAN_NOALLOC_SCRATCH_BYTES (2 MiB) inside the library, held by
+ *   every GPU that loads the library until the process exits.  A shape is
+ *   accepted when 4*T*k + 4*ceil(T/256)*E bytes (each part rounded up to
+ *   256) fit in it, e.g. T*k up to about 440k slots at E = 384, k = 8
+ *   (T = 16384, k = 8, E = 256 uses 576 KiB); larger
+ *   shapes return MOK_ERR_UNSUPPORTED with a message (use mok_plan).
+ *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library
+ *   routine is called.  The first call on a device looks up the array's
+ *   device address (cudaGetSymbolAddress, with that device current); make
+ *   that first call before any stream capture.
+ *   All calls on one device share the array: calls whose kernels may run at
+ *   the same time on the GPU (unordered streams) race on it.  Every call
+ *   writes each scratch entry before reading it, so no clearing is needed.
+ *   Asynchronous on `stream`; errors as for mok_plan.
+ */
+int mok_plan_noalloc(const float* logits, int T, int E, int top_k, int R,
+                     int32_t* counts, int32_t* offsets, int32_t* sched_src_rank,
+                     int32_t* sched_src_index, int32_t* row_slot, int32_t* pos,
+                     int32_t* topk_idx, float* gates, mok_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Steps 3-5: the forward layer.
  * ---------------------------------------------------------------------- */
