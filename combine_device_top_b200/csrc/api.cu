@@ -96,6 +96,15 @@ bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint
     return true;
 }
 
+bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
+                      int H, int I, int E, int buf_rows, const char** err) {
+    return encode_tmap_2d_16b(&m->wg, true, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
+           encode_tmap_2d_16b(&m->wu, true, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
+           encode_tmap_2d_16b(&m->wd, false, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, err) &&
+           encode_bmaps(&m->rows, true, rows, (uint64_t)H, (uint64_t)buf_rows, err) &&
+           encode_bmaps(&m->h, false, h, (uint64_t)I, (uint64_t)buf_rows, err);
+}
+
 // ------------------------------------------------------------------ layouts
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -135,7 +144,8 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
     l.counts2 = take(sizeof(int) * 4);
     l.chunks = take(sizeof(Chunk) * (size_t)l.max_chunks);
     l.mbs = take(sizeof(Minibatch) * (size_t)l.max_mb);
-    l.counters = take(sizeof(int) * 4 * (size_t)l.max_mb + 256);
+    // persistent-mode counters: gathered[max_mb], d_done[max_mb], g_done[max_chunks], d_total
+    l.counters = take(sizeof(int) * (2 * (size_t)l.max_mb + (size_t)l.max_chunks + 8));
     l.rows = take((size_t)l.buf_rows * H * 2);
     l.h = take((size_t)l.buf_rows * I * 2);
     l.out = take((size_t)ns * H * 4);
@@ -177,22 +187,15 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
     const int sms = device_sms(&dev);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     MOK_CUDA(gemm_configure(dev), "gemm configure");
-    CUtensorMap tm_wg, tm_wu, tm_wd;
-    BMaps tm_rows, tm_h;
+    GemmMaps maps;
     const char* err = nullptr;
-    if (!encode_tmap_2d_16b(&tm_wg, true, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
-        !encode_tmap_2d_16b(&tm_wu, true, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, &err) ||
-        !encode_tmap_2d_16b(&tm_wd, false, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, &err) ||
-        !encode_bmaps(&tm_rows, true, rows, (uint64_t)H, (uint64_t)n_rows_buf, &err) ||
-        !encode_bmaps(&tm_h, false, h, (uint64_t)I, (uint64_t)n_rows_buf, &err))
+    if (!encode_gemm_maps(&maps, wg, wu, wd, rows, h, H, I, E, n_rows_buf, &err))
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
     GemmShape sh{H, I, E};
     const GemmTuning tune = gemm_tuning();
-    MOK_CUDA(launch_gemm_phase(0, tm_wg, tm_wu, tm_rows, sh, chunks, counts2, h, out, row_slot, status, timeout_ns,
-                               sms, tune, stream),
+    MOK_CUDA(launch_gemm_phase(0, maps, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune, stream),
              "gate/up GEMM launch");
-    MOK_CUDA(launch_gemm_phase(1, tm_wd, tm_wd, tm_h, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
-                               tune, stream),
+    MOK_CUDA(launch_gemm_phase(1, maps, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune, stream),
              "down GEMM launch");
     return MOK_OK;
 }
@@ -274,10 +277,8 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     if (!w_gate || !w_up || !w_down) return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
     FwdLayout L;
     if (!fwd_layout(T, H, I, E, k, minibatch, opts, &L)) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
-    if (mode == MOK_MODE_PERSISTENT) {
-        if (L.cap < minibatch) return fail(MOK_ERR_INVALID_ARG, "ring_slots / 2 < minibatch");
-        return fail(MOK_ERR_UNSUPPORTED, "persistent mode not built yet");
-    }
+    if (mode == MOK_MODE_PERSISTENT && L.cap < minibatch)
+        return fail(MOK_ERR_INVALID_ARG, "ring_slots / 2 < minibatch");
     if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
     const int sms = device_sms(nullptr);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
@@ -298,6 +299,54 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     MOK_CUDA(launch_build_chunks(plan->offsets, E, ns, L.minibatch, L.cap, chunks, L.max_chunks, mbs, L.max_mb,
                                  counts2, status, stream),
              "work list launch");
+    if (mode == MOK_MODE_PERSISTENT) {
+        int dev = 0;
+        device_sms(&dev);
+        const int dispatch = (opts && opts->dispatch_ctas > 0) ? opts->dispatch_ctas : 16;
+        const int gemm = (opts && opts->gemm_ctas > 0) ? opts->gemm_ctas : sms - dispatch;
+        if (dispatch >= sms || gemm < 1 || dispatch + gemm > sms)
+            return fail(MOK_ERR_INVALID_ARG, "dispatch_ctas + gemm_ctas must be at most the %d SMs", sms);
+        int* counters = reinterpret_cast<int*>(base + L.counters);
+        MOK_CUDA(cudaMemsetAsync(counters, 0, sizeof(int) * (2 * (size_t)L.max_mb + (size_t)L.max_chunks + 8),
+                                 stream),
+                 "counter reset");
+        PersistLaunch P{};
+        P.grid = dispatch + gemm;
+        P.dispatch_ctas = dispatch;
+        P.cap = L.cap;
+        P.H = H;
+        P.I = I;
+        P.E = E;
+        P.T = T;
+        P.k = k;
+        P.S_r = T / R;
+        P.wg = w_gate;
+        P.wu = w_up;
+        P.wd = w_down;
+        P.ring = base + L.rows;
+        P.h = base + L.h;
+        P.out = reinterpret_cast<float*>(base + L.out);
+        P.chunks = chunks;
+        P.mbs = mbs;
+        P.counts2 = counts2;
+        P.gathered = counters;
+        P.d_done = counters + L.max_mb;
+        P.g_done = counters + 2 * L.max_mb;
+        P.d_total = counters + 2 * L.max_mb + L.max_chunks;
+        P.xs = xs;
+        P.ys = ys;
+        P.src_rank = plan->sched_src_rank;
+        P.src_index = plan->sched_src_index;
+        P.row_slot = plan->row_slot;
+        P.gates = plan->gates;
+        P.status = status;
+        P.timeout_ns = timeout;
+        MOK_CUDA(gemm_configure(dev), "gemm configure");
+        const char* err = "";
+        cudaError_t e = launch_forward_persistent(P, &err, stream);
+        if (e != cudaSuccess) return fail(MOK_ERR_CUDA, "%s: %s", err, cudaGetErrorString(e));
+        return MOK_OK;
+    }
     MOK_CUDA(launch_gather(xs, T / R, H, plan->sched_src_rank, plan->sched_src_index, ns, base + L.rows, sms, stream),
              "gather launch");
     rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, chunks, counts2,

@@ -1,0 +1,386 @@
+// gemm_core.cuh -- the warp-specialised tcgen05 grouped-GEMM core shared by
+// the staged kernels (gemm_sm100.cu) and the persistent SM-partitioned
+// kernel (persistent.cu).  Step 4 of the forward MoE layer.
+//
+// MoK article (tahou.com): routing paragraph (tokens of one expert laid out
+// contiguously so the grouped GEMM runs efficiently), MXFP8 paragraph
+// (SwiGLU inside the GEMM data path), push-combine paragraph (each result
+// goes back to its token's slot).
+//
+// Orientation.  Expert segments are short (about 171 rows per expert at 384
+// experts, top-8, 8192 tokens), so the weights take the M = 128 side of every
+// MMA and the tokens the N side (16..256 in steps of 16): an expert with 171
+// rows pads to N = 176 instead of two 128-row tiles, and each weight tile is
+// streamed from HBM once per chunk of <= 256 rows.
+//   gate/up unit (phase 0): A = 64 columns of Wg stacked on the same 64
+//     columns of Wu (M = 128, K = H, read MN-major straight from the
+//     [E, H, I] layout), B = the chunk's token rows (K-major).  Accumulator
+//     lanes 0-63 hold gate, 64-127 up; the epilogue forms
+//     h = silu(gate) * up and stores fp16 h rows.
+//   down unit (phase 1): A = 128 columns of the fp16 copy of Wd (MN-major
+//     from [E, I, H]), B = the chunk's fp16 h rows.  fp16 keeps 3 more
+//     mantissa bits of h than bf16 would, which keeps the largest element
+//     error of y near the floor set by rounding y itself to bf16.  The
+//     epilogue stores fp32 rows to out[row_slot[row]] (the push combine);
+//     fp32 rather than bf16 because a bf16 slot buffer adds a third bf16
+//     rounding that puts the largest element error of y above 2e-2 * rms(y)
+//     on heavy-tailed outputs.
+//
+// Roles in a CTA of 6 warps: warp 0 issues TMA loads into a 4-stage ring of
+// 48 KB stages, warp 1 allocates 512 TMEM columns and one thread of it issues
+// tcgen05.mma into one of two 256-column accumulators, warps 2-5 drain the
+// other accumulator (tcgen05.ld) through shared memory to global memory.
+// Token-side tiles are loaded as one TMA box per set bit of the 16-rounded
+// row count (256/128/64/32/16-row maps): the number of small token-side TMA
+// ops was what limited the first version on B200.  Every wait is bounded.
+//
+// A schedule policy (template parameter) tells each role which units this
+// CTA runs, what a unit's inputs wait for, and what its completion signals.
+#pragma once
+
+#include "mok_device.cuh"
+#include "mok_internal.h"
+
+namespace mok {
+
+constexpr int GEMM_THREADS = 192;
+constexpr int NSTAGE = 4;
+constexpr int BK = 64;                            // K per stage: one 128-byte swizzle atom
+constexpr int A_BYTES = 128 * BK * 2;             // 16 KB: two {64 MN x 64 K} boxes
+constexpr int B_ROW_BYTES = BK * 2;               // 128 bytes of one token row per stage
+constexpr int B_BYTES = CHUNK_MAX_ROWS * B_ROW_BYTES;  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
+constexpr int EPI_LD = 33;                        // fp32 staging row pitch (bank-conflict free)
+constexpr int EPI_BYTES = 128 * EPI_LD * 4;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COLS = 256;
+// Bound of the waits that drain this CTA's own TMA loads and MMAs before it
+// leaves: those complete by themselves, so the bound is generous and does
+// not follow the caller's (possibly tiny) timeout.
+constexpr uint64_t DRAIN_TIMEOUT_NS = 1000000000ull;
+constexpr int MT_G_FEATURES = 64;                 // gate/up unit: 64 gate + 64 up columns
+constexpr int MT_D_FEATURES = 128;                // down unit: 128 output columns
+
+constexpr int SMEM_STAGES_OFF = 0;
+constexpr int SMEM_EPI_OFF = NSTAGE * STAGE_BYTES;
+constexpr int SMEM_BAR_OFF = SMEM_EPI_OFF + EPI_BYTES;
+constexpr int SMEM_BYTES_USED = SMEM_BAR_OFF + 256;
+constexpr int SMEM_ALLOC = SMEM_BYTES_USED + 1024;  // slack for 1024-byte alignment
+
+// One unit of work: an M tile of one phase over one chunk.
+struct Unit {
+    int phase;   // 0 = gate/up, 1 = down
+    int expert;
+    int brow0;   // buffer row of the chunk's first row (token rows and h rows)
+    int rows;    // valid rows, 1..256
+    int m;       // M tile index
+    int grow0;   // global expert-major row of the chunk's first row (row_slot index)
+    int chunk;
+    int mb;
+};
+
+struct CoreArgs {
+    int H, I;
+    __half* h;                // [buffer rows, I] fp16
+    float* out;               // [N_s, H] fp32, slot-indexed
+    const int32_t* row_slot;  // [N_s]
+    DevStatus* st;
+    uint64_t timeout_ns;
+};
+
+// Unit u -> (chunk c, M tile m) in raster groups of GC chunks: inside a group
+// the chunk index runs fastest, so the CTAs running at one time share a few
+// chunks' token tiles (L2) while streaming distinct weight tiles.
+__device__ __forceinline__ void unit_map(int u, int nch, int MT, int GC, int& c, int& m) {
+    const int grp = u / (GC * MT);
+    const int rem = u - grp * GC * MT;
+    const int c0 = grp * GC;
+    const int gsz = min(GC, nch - c0);
+    m = rem / gsz;
+    c = c0 + (rem - m * gsz);
+}
+
+// Staged schedule: one phase over every chunk, units dealt round-robin to
+// the CTAs of the grid; no waits, no signals (kernel boundaries order the
+// phases).
+struct StagedSched {
+    static constexpr bool kSignals = false;
+    int phase, nch, MT, GC;
+    const Chunk* chunks;
+
+    __device__ bool get(int i, Unit& u) const {
+        const int idx = blockIdx.x + i * gridDim.x;
+        if (idx >= nch * MT) return false;
+        int c, m;
+        unit_map(idx, nch, MT, GC, c, m);
+        const Chunk ck = chunks[c];
+        u.phase = phase;
+        u.expert = ck.expert;
+        u.brow0 = ck.row0;
+        u.rows = ck.rows;
+        u.m = m;
+        u.grow0 = ck.row0;
+        u.chunk = c;
+        u.mb = ck.mb;
+        return true;
+    }
+    __device__ bool wait_inputs(const Unit&, DevStatus*, uint64_t) const { return true; }
+    __device__ void unit_done(const Unit&) const {}
+};
+
+// ------------------------------------------------------------------ producer
+template <class S>
+__device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const CoreArgs& a, const S& s,
+                                              unsigned char* smem, uint64_t* full, uint64_t* empty) {
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, issued_phase = 0;  // bit s: stage s holds a load of phase bit s
+    const uint64_t evict_first = l2_policy_evict_first();
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        if (!s.wait_inputs(u, a.st, a.timeout_ns)) break;
+        const int KB = (u.phase == 0 ? a.H : a.I) / BK;
+        const int wrows = u.phase == 0 ? a.H : a.I;
+        const BMaps& bm = u.phase == 0 ? maps.rows : maps.h;
+        // token rows rounded up to 16, one box per set bit: at most 5 TMA ops
+        const int r16 = (u.rows + 15) & ~15;
+        const uint32_t bytes = A_BYTES + r16 * B_ROW_BYTES;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 10)) {
+                ok = false;
+                break;
+            }
+            unsigned char* sa = smem + SMEM_STAGES_OFF + stage * STAGE_BYTES;
+            unsigned char* sb = sa + A_BYTES;
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            const int ky = u.expert * wrows + kb * BK;
+            if (u.phase == 0) {
+                tma_load_2d_hint(sa, &maps.wg, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
+                tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
+            } else {
+                tma_load_2d_hint(sa, &maps.wd, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
+                tma_load_2d_hint(sa + A_BYTES / 2, &maps.wd, &full[stage], u.m * MT_D_FEATURES + 64, ky,
+                                 evict_first);
+            }
+            int roff = 0;
+#pragma unroll
+            for (int b = 0; b < B_MAPS; ++b) {
+                const int sz = B_MAX_BOX >> b;
+                if (r16 & sz) {
+                    tma_load_2d(sb + roff * B_ROW_BYTES, &bm.m[b], &full[stage], kb * BK, u.brow0 + roff);
+                    roff += sz;
+                }
+            }
+            issued |= 1u << stage;
+            issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == NSTAGE) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (!ok) break;
+    }
+    // never leave with a load in flight into this CTA's shared memory
+    for (int st = 0; st < NSTAGE; ++st)
+        if ((issued >> st) & 1u) mbar_wait(&full[st], (issued_phase >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 11);
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <class S>
+__device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* full,
+                                         uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* fin,
+                                         uint32_t tmem_base) {
+    int stage = 0;
+    uint32_t phase = 0;
+    int tb = 0;
+    uint32_t tph = 0;
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        const int KB = (u.phase == 0 ? a.H : a.I) / BK;
+        const int N = (u.rows + 15) & ~15;
+        // gate/up: bf16 x bf16; down: fp16 x fp16 (fp16 W_down copy, fp16 h)
+        const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, u.phase == 0);
+        if (!mbar_wait(&tempty[tb], tph ^ 1u, a.st, a.timeout_ns, 20)) break;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + (uint32_t)(tb * ACC_COLS);
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 21)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + SMEM_STAGES_OFF + stage * STAGE_BYTES);
+            const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < BK / 16; ++ks) {
+                // A: MN-major SW128, 16 K rows per MMA = 2 atoms of 1 KB; the
+                //    two 64-wide MN halves are 8 KB apart (LBO).
+                const uint64_t ad = umma_desc_sw128(sa + ks * 2048, A_BYTES / 2, 1024);
+                // B: K-major SW128, 16 K = 32 bytes inside the atom; 8-row groups 1 KB apart.
+                const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
+                umma_bf16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == NSTAGE) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[tb]);
+        if (++tb == 2) {
+            tb = 0;
+            tph ^= 1u;
+        }
+    }
+    // wait for every MMA this thread issued before TMEM is released
+    umma_commit(fin);
+    mbar_wait(fin, 0, nullptr, DRAIN_TIMEOUT_NS, 22);
+}
+
+// ------------------------------------------------------------------ epilogue (warps 2..5)
+template <class S>
+__device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* tfull,
+                                              uint64_t* tempty, volatile int* ok_flag, uint32_t tmem_base) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;           // TMEM lane quadrant this warp may access
+    const int et = threadIdx.x - 64;  // 0..127
+    const int tok = et & 31, fq = et >> 5;
+    float* epi = reinterpret_cast<float*>(smem + SMEM_EPI_OFF);
+    int tb = 0;
+    uint32_t tph = 0;
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        // one thread waits, all 128 leave together on failure
+        if (et == 0) *ok_flag = mbar_wait(&tfull[tb], tph, a.st, a.timeout_ns, 30) ? 1 : 0;
+        named_bar_sync(1, 128);
+        const int ok = *ok_flag;
+        named_bar_sync(1, 128);
+        if (!ok) break;
+        tc_fence_after();
+        const int ncc = (u.rows + 31) >> 5;
+        for (int cc = 0; cc < ncc; ++cc) {
+            float v[32];
+            tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(tb * ACC_COLS + cc * 32), v);
+            float* myrow = epi + (q * 32 + lane) * EPI_LD;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) myrow[k] = v[k];
+            named_bar_sync(1, 128);
+            const int col = cc * 32 + tok;
+            if (col < u.rows) {
+                if (u.phase == 0) {
+                    // features m*64 + fq*16 .. +15: gate rows fq*16+k, up rows 64+fq*16+k
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int k = 0; k < 16; k += 2) {
+                        const float g0 = epi[(fq * 16 + k) * EPI_LD + tok];
+                        const float g1 = epi[(fq * 16 + k + 1) * EPI_LD + tok];
+                        const float u0 = epi[(64 + fq * 16 + k) * EPI_LD + tok];
+                        const float u1 = epi[(64 + fq * 16 + k + 1) * EPI_LD + tok];
+                        const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                        const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                        pk[k >> 1] = pack_half2_sat(h0, h1);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(a.h + (size_t)(u.brow0 + col) * a.I + u.m * MT_G_FEATURES +
+                                                          fq * 16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                } else {
+                    // fp32 push to the token's slot; the combine rounds y once
+                    const int slot = __ldg(a.row_slot + u.grow0 + col);
+                    float4* dst = reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + u.m * MT_D_FEATURES + fq * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const int f = fq * 32 + q4 * 4;
+                        dst[q4] = make_float4(epi[f * EPI_LD + tok], epi[(f + 1) * EPI_LD + tok],
+                                              epi[(f + 2) * EPI_LD + tok], epi[(f + 3) * EPI_LD + tok]);
+                    }
+                }
+            }
+            named_bar_sync(1, 128);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
+        if (++tb == 2) {
+            tb = 0;
+            tph ^= 1u;
+        }
+        if (S::kSignals) {
+            // h rows are read next by TMA (async proxy) in some CTA: make this
+            // thread's stores visible to that proxy, then publish once.
+            fence_proxy_async_global();
+            __threadfence();
+            named_bar_sync(1, 128);
+            if (et == 0) s.unit_done(u);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ one GEMM CTA
+// Runs every unit the schedule gives this CTA.  All GEMM_THREADS threads
+// must call it; it returns after TMEM is released.
+template <class S>
+__device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const CoreArgs& a, const S& s, unsigned char* smem) {
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
+    uint64_t* empty = full + NSTAGE;
+    uint64_t* tfull = empty + NSTAGE;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* fin = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    volatile int* ok_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < NSTAGE; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(fin, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&maps.wg);
+        tma_prefetch_desc(&maps.wu);
+        tma_prefetch_desc(&maps.wd);
+        for (int b = 0; b < B_MAPS; ++b) {
+            tma_prefetch_desc(&maps.rows.m[b]);
+            tma_prefetch_desc(&maps.h.m[b]);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) gemm_producer(maps, a, s, smem, full, empty);
+    } else if (warp == 1) {
+        if (lane == 0) gemm_mma(a, s, smem, full, empty, tfull, tempty, fin, tmem_base);
+    } else {
+        gemm_epilogue(a, s, smem, tfull, tempty, ok_flag, tmem_base);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+__device__ __forceinline__ unsigned char* align_smem_1024(unsigned char* p) {
+    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+}  // namespace mok

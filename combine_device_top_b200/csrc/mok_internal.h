@@ -62,10 +62,9 @@ struct GemmShape {
     int H, I, E;
 };
 struct GemmTuning {
-    int l2_prefetch;   // k-steps of weight tiles prefetched into L2 ahead of the loads
     int group_chunks;  // raster group size in chunks
 };
-GemmTuning gemm_tuning();  // defaults, overridable by MOK_GEMM_L2_PREFETCH / MOK_GEMM_GROUP
+GemmTuning gemm_tuning();  // defaults, overridable by MOK_GEMM_GROUP
 size_t gemm_smem_bytes();
 cudaError_t gemm_configure(int dev);
 // Token-side (B operand) tensor maps of one buffer with box heights
@@ -78,12 +77,41 @@ struct BMaps {
 };
 bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint64_t rows, const char** err);
 
+// Every tensor map the GEMM core reads.
+struct GemmMaps {
+    CUtensorMap wg, wu, wd;  // 64x64 boxes of Wg, Wu (bf16) and Wd (fp16)
+    BMaps rows;              // token rows (bf16) of the row buffer
+    BMaps h;                 // h rows (fp16) of the h buffer
+};
+bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
+                      int H, int I, int E, int buf_rows, const char** err);
+
 // Staged grouped GEMM over every chunk: phase 0 = gate/up + SwiGLU -> h,
-// phase 1 = down -> out[row_slot].  Tensor maps are built by the caller.
-cudaError_t launch_gemm_phase(int phase, const CUtensorMap& tmA0, const CUtensorMap& tmA1, const BMaps& tmB,
-                              const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out,
-                              void* out, const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              const GemmTuning& tune, cudaStream_t stream);
+// phase 1 = down -> out[row_slot].
+cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const GemmShape& sh, const Chunk* chunks,
+                              const int* counts2, void* h_out, void* out, const int32_t* row_slot, void* status,
+                              uint64_t timeout_ns, int grid, const GemmTuning& tune, cudaStream_t stream);
+
+// ---- the persistent SM-partitioned forward (persistent.cu)
+struct PersistLaunch {
+    int grid, dispatch_ctas, cap;  // CTAs, of which the first dispatch_ctas gather; ring half rows
+    int H, I, E, T, k, S_r;
+    const void *wg, *wu, *wd;      // weights (bf16, bf16, fp16)
+    void* ring;                    // [2*cap, H] bf16
+    void* h;                       // [2*cap, I] fp16
+    float* out;                    // [T*k, H] fp32
+    const Chunk* chunks;
+    const Minibatch* mbs;
+    const int* counts2;
+    int *gathered, *d_done, *g_done, *d_total;  // zeroed counters
+    ShardsIn xs;
+    ShardsOut ys;
+    const int32_t *src_rank, *src_index, *row_slot;
+    const float* gates;
+    void* status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, cudaStream_t stream);
 
 // ---- tensor maps (driver entry point fetched at run time)
 // 2D tiled map of a row-major [outer, inner] array of 16-bit elements
