@@ -200,6 +200,12 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
     return MOK_OK;
 }
 
+static bool all_aligned16(const void* const* p, int n) {
+    for (int i = 0; i < n; ++i)
+        if (reinterpret_cast<uintptr_t>(p[i]) & 15u) return false;
+    return true;
+}
+
 static bool all_nonnull(const void* const* p, int n) {
     if (!p) return false;
     for (int i = 0; i < n; ++i)
@@ -274,6 +280,8 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     const int T = plan->T, E = plan->E, k = plan->k, R = plan->R;
     if (T == 0) return MOK_OK;
     if (!all_nonnull(x_shards, R) || !all_nonnull(y_shards, R)) return fail(MOK_ERR_INVALID_ARG, "NULL shard pointer");
+    if (!all_aligned16(x_shards, R) || !all_aligned16(y_shards, R))
+        return fail(MOK_ERR_UNSUPPORTED, "shard pointers must be 16-byte aligned");
     if (!w_gate || !w_up || !w_down) return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
     FwdLayout L;
     if (!fwd_layout(T, H, I, E, k, minibatch, opts, &L)) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
@@ -347,8 +355,7 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         if (e != cudaSuccess) return fail(MOK_ERR_CUDA, "%s: %s", err, cudaGetErrorString(e));
         return MOK_OK;
     }
-    MOK_CUDA(launch_gather(xs, T / R, H, plan->sched_src_rank, plan->sched_src_index, ns, base + L.rows, sms, stream),
-             "gather launch");
+    MOK_CUDA(launch_gather(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
     rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, chunks, counts2,
                         base + L.h, base + L.out, status, timeout, stream);
     if (rc) return rc;
@@ -390,12 +397,14 @@ int mok_gather(const void* const* x_shards, int H, const mok_plan_t* plan, void*
     if (H <= 0 || H % 8) return fail(MOK_ERR_UNSUPPORTED, "H %% 8 != 0");
     if (plan->T == 0) return MOK_OK;
     if (!rows || !all_nonnull(x_shards, plan->R)) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if (!all_aligned16(x_shards, plan->R) || (reinterpret_cast<uintptr_t>(rows) & 15u))
+        return fail(MOK_ERR_UNSUPPORTED, "shard and row pointers must be 16-byte aligned");
     ShardsIn xs{};
     for (int r = 0; r < plan->R; ++r) xs.p[r] = x_shards[r];
     const int sms = device_sms(nullptr);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
-    MOK_CUDA(launch_gather(xs, plan->T / plan->R, H, plan->sched_src_rank, plan->sched_src_index,
-                           plan->T * plan->k, rows, sms, reinterpret_cast<cudaStream_t>(stream)),
+    MOK_CUDA(launch_gather(xs, plan->T / plan->R, H, plan->T, plan->k, plan->pos, rows, sms,
+                           reinterpret_cast<cudaStream_t>(stream)),
              "gather launch");
     return MOK_OK;
 }
@@ -444,6 +453,8 @@ int mok_combine(const void* out, int H, const mok_plan_t* plan, void* const* y_s
     if (H <= 0 || H % 8) return fail(MOK_ERR_UNSUPPORTED, "H %% 8 != 0");
     if (plan->T == 0) return MOK_OK;
     if (!out || !all_nonnull(y_shards, plan->R)) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if (!all_aligned16(y_shards, plan->R) || (reinterpret_cast<uintptr_t>(out) & 15u))
+        return fail(MOK_ERR_UNSUPPORTED, "shard and output pointers must be 16-byte aligned");
     ShardsOut ys{};
     for (int r = 0; r < plan->R; ++r) ys.p[r] = y_shards[r];
     const int sms = device_sms(nullptr);

@@ -2,11 +2,11 @@
 // (weighted combine) of the forward MoE layer as standalone kernels.  The
 // warp bodies are in dispatch_combine.cuh.
 //
-// Both kernels are HBM-bound streams of 16-byte vectors: one warp per row
-// (gather) or per token (combine), a grid of a few CTAs per SM looping over
-// the rows.  The gather reads each token k times (L2 absorbs part of the
-// reuse) and writes N_s*H*2 bytes; the combine reads N_s*H*4 bytes of fp32
-// per-slot outputs and writes T*H*2 bytes of bf16 y, rounding once.
+// Both kernels are HBM-bound streams of 16-byte vectors: one warp per token,
+// a grid of a few CTAs per SM looping over the tokens.  The gather reads each
+// token once and writes it to its k rows (T*H*2 bytes in, N_s*H*2 out); the
+// combine reads N_s*H*4 bytes of fp32 per-slot outputs and writes T*H*2
+// bytes of bf16 y, rounding once.
 #include "dispatch_combine.cuh"
 #include "mok_internal.h"
 
@@ -14,18 +14,37 @@ namespace mok {
 
 constexpr int DC_THREADS = 256;
 
-__global__ void __launch_bounds__(DC_THREADS) k_gather(ShardsIn xs, int S_r, int H,
-                                                       const int32_t* __restrict__ src_rank,
-                                                       const int32_t* __restrict__ src_index, int n_rows,
-                                                       uint4* __restrict__ rows) {
+// Token-major form of the same copy: one warp per token reads the token's
+// row once and writes it to each of its k rows (pos[t*k + j]).  Every source
+// row is read from HBM once instead of k times (with 940 MB of rows streaming
+// out, x does not stay in L2 between its k reads).
+__global__ void __launch_bounds__(DC_THREADS) k_gather_tokens(ShardsIn xs, int S_r, int H, int T, int k,
+                                                              const int32_t* __restrict__ pos,
+                                                              uint4* __restrict__ rows) {
     const int lane = threadIdx.x & 31;
-    const int nvec = H >> 3;  // 16-byte vectors per row
+    const int nvec = H >> 3;
     const int warps = gridDim.x * (DC_THREADS / 32);
-    for (int row = blockIdx.x * (DC_THREADS / 32) + (threadIdx.x >> 5); row < n_rows; row += warps) {
-        const int r = __ldg(src_rank + row);
-        const int i = __ldg(src_index + row);
-        warp_copy_row(reinterpret_cast<const uint4*>(xs.p[r]) + (size_t)i * nvec, rows + (size_t)row * nvec, nvec,
-                      lane);
+    for (int t = blockIdx.x * (DC_THREADS / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+        const int r = t / S_r;
+        const uint4* src = reinterpret_cast<const uint4*>(xs.p[r]) + (size_t)(t - r * S_r) * nvec;
+        const int my_row = lane < k ? __ldg(pos + (size_t)t * k + lane) : 0;
+        int v0 = 0;
+        for (; v0 + 128 <= nvec; v0 += 128) {  // warp-uniform trip count
+            const int v = v0 + lane;
+            const uint4 a = __ldg(src + v), b = __ldg(src + v + 32), c = __ldg(src + v + 64), d = __ldg(src + v + 96);
+            for (int j = 0; j < k; ++j) {
+                uint4* dst = rows + (size_t)__shfl_sync(0xffffffffu, my_row, j) * nvec;
+                dst[v] = a;
+                dst[v + 32] = b;
+                dst[v + 64] = c;
+                dst[v + 96] = d;
+            }
+        }
+        // tail: lanes may differ in trip count, so no warp collectives here
+        for (int v = v0 + lane; v < nvec; v += 32) {
+            const uint4 a = __ldg(src + v);
+            for (int j = 0; j < k; ++j) rows[(size_t)__ldg(pos + (size_t)t * k + j) * nvec + v] = a;
+        }
     }
 }
 
@@ -42,13 +61,12 @@ __global__ void __launch_bounds__(DC_THREADS) k_combine(const float4* __restrict
     }
 }
 
-cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, const int32_t* src_rank, const int32_t* src_index,
-                          int n_rows, void* rows, int num_sms, cudaStream_t stream) {
-    if (n_rows <= 0) return cudaSuccess;
-    const int want = (n_rows + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
+cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
+                          int num_sms, cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    const int want = (T + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     const int grid = want < num_sms * 8 ? want : num_sms * 8;
-    k_gather<<<grid, DC_THREADS, 0, stream>>>(xs, S_r, H, src_rank, src_index, n_rows,
-                                              reinterpret_cast<uint4*>(rows));
+    k_gather_tokens<<<grid, DC_THREADS, 0, stream>>>(xs, S_r, H, T, k, pos, reinterpret_cast<uint4*>(rows));
     return cudaGetLastError();
 }
 

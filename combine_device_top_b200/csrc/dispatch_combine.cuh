@@ -27,6 +27,62 @@ __device__ __forceinline__ void warp_copy_row(const uint4* __restrict__ src, uin
     for (; v < nvec; v += 32) dst[v] = __ldg(src + v);
 }
 
+// Bulk stores allowed to be still reading shared memory while the next rows load.
+constexpr int BULK_STORES_IN_FLIGHT = 4;
+
+// One thread streams n rows of row_bytes through S shared-memory slots with
+// bulk async copies: row i is loaded from src_row(i) into a slot and stored
+// from there to dst_row(i).  About S - BULK_STORES_IN_FLIGHT rows load while
+// the previous stores drain, so one thread keeps ~200 KB in flight.
+// `loads` counts the loads ever issued through these slots (it fixes the
+// mbarrier phases across calls) and is advanced.  Returns false if a wait
+// gave up; the thread's own copies are drained either way before it returns,
+// and every store has completed when it returns true.  Needs
+// S > BULK_STORES_IN_FLIGHT.
+template <class SrcF, class DstF>
+__device__ __forceinline__ bool bulk_stream_rows(int n, SrcF src_row, DstF dst_row, uint32_t row_bytes,
+                                                 unsigned char* slots, uint64_t* full, int S, uint32_t& loads,
+                                                 DevStatus* st, uint64_t timeout_ns, uint64_t drain_ns) {
+    constexpr int D = BULK_STORES_IN_FLIGHT;
+    const uint32_t base = loads;
+    int loaded = 0;
+    for (; loaded < n && loaded < S; ++loaded) {
+        const int slot = (int)((base + loaded) % (uint32_t)S);
+        mbar_arrive_expect_tx(&full[slot], row_bytes);
+        bulk_load(slots + (size_t)slot * row_bytes, src_row(loaded), row_bytes, &full[slot]);
+    }
+    bool ok = true;
+    int s = 0;
+    for (; s < n; ++s) {
+        const uint32_t g = base + s;
+        const int slot = (int)(g % (uint32_t)S);
+        if (!mbar_wait(&full[slot], (g / (uint32_t)S) & 1u, st, timeout_ns, 70)) {
+            ok = false;
+            break;
+        }
+        bulk_store(dst_row(s), slots + (size_t)slot * row_bytes, row_bytes);
+        bulk_commit();
+        if (s >= D) {
+            bulk_wait_read<D>();  // the store of row s - D has read its slot
+            const int i = s - D + S;
+            if (i < n) {
+                const int slot2 = (int)((base + i) % (uint32_t)S);
+                mbar_arrive_expect_tx(&full[slot2], row_bytes);
+                bulk_load(slots + (size_t)slot2 * row_bytes, src_row(i), row_bytes, &full[slot2]);
+                loaded = i + 1;
+            }
+        }
+    }
+    // a wait gave up: let every load already issued land before leaving
+    for (int i = s; i < loaded; ++i) {
+        const uint32_t g = base + i;
+        mbar_wait(&full[g % (uint32_t)S], (g / (uint32_t)S) & 1u, nullptr, drain_ns, 71);
+    }
+    bulk_wait_all();
+    loads = base + loaded;
+    return ok;
+}
+
 // One warp: y[t] = bf16(sum_{j<k} g[t,j] * out[t,j,:]) in fp32, j ascending.
 // out is fp32 [T, k, H]; each lane owns 8 consecutive features (two 16-byte
 // loads per slot, one 16-byte store).  nvec = H / 8.  Slots are loaded KB at

@@ -35,8 +35,9 @@ struct ShardsOut {
     void* p[MOK_MAX_SHARDS];
 };
 
-cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, const int32_t* src_rank, const int32_t* src_index,
-                          int n_rows, void* rows, int num_sms, cudaStream_t stream);
+// rows[pos[t*k + j]] = x[t] for every slot (token-major walk of the pull schedule)
+cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
+                          int num_sms, cudaStream_t stream);
 cudaError_t launch_combine(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
                            int num_sms, cudaStream_t stream);
 

@@ -85,9 +85,12 @@ struct PersistSched {
             u.phase = 1;
             local -= n * p->MTG;
         }
-        const int c = mb.chunk0 + local % n;  // chunk index runs fastest
+        // M tile runs fastest: a chunk's gate/up units finish together early
+        // in the minibatch, so its down units (ordered the same way) rarely wait
+        const int MT = u.phase == 0 ? p->MTG : p->MTD;
+        const int c = mb.chunk0 + local / MT;
         const Chunk ck = p->chunks[c];
-        u.m = local / n;
+        u.m = local % MT;
         u.chunk = c;
         u.mb = lo;
         u.expert = ck.expert;
@@ -128,6 +131,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     if ((int)blockIdx.x < D) {
         // ---------------------------------------- dispatch side: fill the ring
+        // One thread streams rows through the CTA's otherwise idle shared
+        // memory with bulk async copies (about 200 KB in flight per CTA);
+        // rows too wide for enough slots fall back to warp copies.
+        const uint32_t row_bytes = (uint32_t)a.H * 2u;
+        const int S = min(16, SMEM_BAR_OFF / (int)row_bytes);
+        const bool bulk = S > BULK_STORES_IN_FLIGHT;
+        uint64_t* slot_full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
+        if (threadIdx.x == 0 && bulk) {
+            for (int i = 0; i < S; ++i) mbar_init(&slot_full[i], 1);
+            fence_mbar_init();
+        }
+        __syncthreads();
+        uint32_t loads = 0;
         for (int b = 0; b < nmb; ++b) {
             if (threadIdx.x == 0) {
                 bool ok = !failed(a.st);
@@ -146,16 +162,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int r0 = mb.row0 + (int)((long long)n * blockIdx.x / D);
             const int r1 = mb.row0 + (int)((long long)n * (blockIdx.x + 1) / D);
             uint4* half = reinterpret_cast<uint4*>(p.ring) + (size_t)((b & 1) * p.cap) * nvec;
-            for (int r = r0 + warp; r < r1; r += GEMM_THREADS / 32) {
-                const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
-                warp_copy_row(reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec,
-                              half + (size_t)(r - mb.row0) * nvec, nvec, lane);
+            if (bulk) {
+                if (threadIdx.x == 0) {
+                    auto src = [&](int i) -> const void* {
+                        const int r = r0 + i;
+                        return reinterpret_cast<const uint4*>(p.xs.p[__ldg(p.src_rank + r)]) +
+                               (size_t)__ldg(p.src_index + r) * nvec;
+                    };
+                    auto dst = [&](int i) -> void* { return half + (size_t)(r0 + i - mb.row0) * nvec; };
+                    bulk_stream_rows(r1 - r0, src, dst, row_bytes, smem, slot_full, S, loads, a.st, a.timeout_ns,
+                                     DRAIN_TIMEOUT_NS);
+                }
+            } else {
+                for (int r = r0 + warp; r < r1; r += GEMM_THREADS / 32) {
+                    const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
+                    warp_copy_row(reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec,
+                                  half + (size_t)(r - mb.row0) * nvec, nvec, lane);
+                }
             }
             // the rows are read next by TMA in the GEMM CTAs
             fence_proxy_async_global();
             __threadfence();
             __syncthreads();
-            if (threadIdx.x == 0) red_release_gpu_add(&p.gathered[b], 1);
+            if (threadIdx.x == 0 && !failed(a.st)) red_release_gpu_add(&p.gathered[b], 1);
         }
     } else {
         // ---------------------------------------- GEMM side
