@@ -96,8 +96,24 @@ bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint
     return true;
 }
 
+// Wd viewed as {64 (columns inside a 64-wide block), E*I (rows), H/64 (column
+// blocks)} with strides {H*2, 128} bytes: a {64, 64, 2} box is the MMA's
+// two-atom MN-major tile of a 128-column down unit, in one TMA op.
+static bool encode_wd3(CUtensorMap* map, const void* wd, int H, int I, int E) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)E * I, (cuuint64_t)H / 64};
+    cuuint64_t strides[2] = {(cuuint64_t)H * 2, 128};
+    cuuint32_t box[3] = {64, 64, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(wd), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
                       int H, int I, int E, int buf_rows, const char** err) {
+    m->has_wd3 = encode_wd3(&m->wd3, wd, H, I, E) ? 1 : 0;
     return encode_tmap_2d_16b(&m->wg, true, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
            encode_tmap_2d_16b(&m->wu, true, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
            encode_tmap_2d_16b(&m->wd, false, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, err) &&

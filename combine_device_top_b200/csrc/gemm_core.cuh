@@ -142,9 +142,13 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const CoreAr
         const int KB = (u.phase == 0 ? a.H : a.I) / BK;
         const int wrows = u.phase == 0 ? a.H : a.I;
         const BMaps& bm = u.phase == 0 ? maps.rows : maps.h;
-        // token rows rounded up to 16, one box per set bit: at most 5 TMA ops
+        // token rows rounded up to 16 and loaded as ONE box of the next power
+        // of two (16..256 rows): the count of TMA ops per SM, not bytes, was
+        // measured to be the limit, so a few extra L2 bytes buy fewer ops
         const int r16 = (u.rows + 15) & ~15;
-        const uint32_t bytes = A_BYTES + r16 * B_ROW_BYTES;
+        int bx = 0;
+        while (bx + 1 < B_MAPS && (B_MAX_BOX >> (bx + 1)) >= r16) ++bx;
+        const uint32_t bytes = A_BYTES + (uint32_t)(B_MAX_BOX >> bx) * B_ROW_BYTES;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 10)) {
@@ -158,20 +162,15 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const CoreAr
             if (u.phase == 0) {
                 tma_load_2d_hint(sa, &maps.wg, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
                 tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
+            } else if (maps.has_wd3) {
+                // both 64-column halves of the 128-column down tile in one op
+                tma_load_3d_hint(sa, &maps.wd3, &full[stage], 0, ky, u.m * 2, evict_first);
             } else {
                 tma_load_2d_hint(sa, &maps.wd, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
                 tma_load_2d_hint(sa + A_BYTES / 2, &maps.wd, &full[stage], u.m * MT_D_FEATURES + 64, ky,
                                  evict_first);
             }
-            int roff = 0;
-#pragma unroll
-            for (int b = 0; b < B_MAPS; ++b) {
-                const int sz = B_MAX_BOX >> b;
-                if (r16 & sz) {
-                    tma_load_2d(sb + roff * B_ROW_BYTES, &bm.m[b], &full[stage], kb * BK, u.brow0 + roff);
-                    roff += sz;
-                }
-            }
+            tma_load_2d(sb, &bm.m[bx], &full[stage], kb * BK, u.brow0);
             issued |= 1u << stage;
             issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == NSTAGE) {
@@ -349,6 +348,7 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const CoreArgs& a
         tma_prefetch_desc(&maps.wg);
         tma_prefetch_desc(&maps.wu);
         tma_prefetch_desc(&maps.wd);
+        if (maps.has_wd3) tma_prefetch_desc(&maps.wd3);
         for (int b = 0; b < B_MAPS; ++b) {
             tma_prefetch_desc(&maps.rows.m[b]);
             tma_prefetch_desc(&maps.h.m[b]);

@@ -81,8 +81,10 @@ bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint
 // Every tensor map the GEMM core reads.
 struct GemmMaps {
     CUtensorMap wg, wu, wd;  // 64x64 boxes of Wg, Wu (bf16) and Wd (fp16)
+    CUtensorMap wd3;         // Wd as {64, E*I, H/64}: one op loads both 64-column halves of a down tile
     BMaps rows;              // token rows (bf16) of the row buffer
     BMaps h;                 // h rows (fp16) of the h buffer
+    int has_wd3;             // wd3 could be encoded (else two 2D ops per down stage)
 };
 bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
                       int H, int I, int E, int buf_rows, const char** err);
