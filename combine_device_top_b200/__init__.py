@@ -36,7 +36,7 @@ EXPORTS = (
     "mok_plan_workspace_bytes", "mok_plan", "mok_forward_workspace_bytes", "mok_moe_forward",
     "mok_get_status", "mok_last_error_string", "mok_gather", "mok_expert_ffn_workspace_bytes",
     "mok_expert_ffn", "mok_combine", "mok_forward_host_workspace_bytes", "mok_moe_forward_host",
-    "mok_prepare_w_down", "mok_plan_noalloc",
+    "mok_prepare_w_down", "mok_plan_noalloc", "mok_mxfp8_quantize_rows", "mok_quantize_weights_mxfp8",
 )
 
 
@@ -87,8 +87,11 @@ def lib() -> ctypes.CDLL:
                                        ctypes.POINTER(FwdOpts), vp, sz, vp, vp]
     L.mok_prepare_w_down.argtypes = [vp, vp, sz, vp]
     L.mok_plan_noalloc.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.mok_mxfp8_quantize_rows.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    L.mok_quantize_weights_mxfp8.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
-              "mok_moe_forward_host", "mok_prepare_w_down", "mok_plan_noalloc"):
+              "mok_moe_forward_host", "mok_prepare_w_down", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
+              "mok_quantize_weights_mxfp8"):
         getattr(L, n).restype = ctypes.c_int
     return L
 
@@ -179,6 +182,29 @@ def prepare_w_down(w_down: torch.Tensor, out: torch.Tensor | None = None, stream
     return out
 
 
+def mxfp8_quantize_rows(src: torch.Tensor, stream=None):
+    """Blocks of 32 along each row of a [rows, K] bf16/fp32 tensor -> (q uint8, scales uint8)."""
+    assert src.is_cuda and src.is_contiguous() and src.dtype in (torch.bfloat16, torch.float32)
+    rows, K = src.shape
+    q = torch.empty((rows, K), dtype=torch.uint8, device=src.device)
+    s = torch.empty((rows, K // 32), dtype=torch.uint8, device=src.device)
+    _check(lib().mok_mxfp8_quantize_rows(ctypes.c_void_p(src.data_ptr()), int(src.dtype == torch.float32), rows, K,
+                                         ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(s.data_ptr()),
+                                         _stream(stream)))
+    return q, s
+
+
+def quantize_weights_mxfp8(w: torch.Tensor, stream=None):
+    """Weights [E, K, N] bf16 -> (q [E, K, N] uint8, scales [E, K/32, N] uint8), blocks along K."""
+    assert w.is_cuda and w.is_contiguous() and w.dtype == torch.bfloat16
+    E, K, N = w.shape
+    q = torch.empty((E, K, N), dtype=torch.uint8, device=w.device)
+    s = torch.empty((E, K // 32, N), dtype=torch.uint8, device=w.device)
+    _check(lib().mok_quantize_weights_mxfp8(ctypes.c_void_p(w.data_ptr()), E, K, N, ctypes.c_void_p(q.data_ptr()),
+                                            ctypes.c_void_p(s.data_ptr()), _stream(stream)))
+    return q, s
+
+
 def fwd_opts(mode: int = MOK_MODE_PERSISTENT, ring_slots: int = 0, dispatch_ctas: int = 0, gemm_ctas: int = 0,
              mxfp8: bool = False, timeout_ns: int = 0) -> FwdOpts:
     return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), 0, timeout_ns)
@@ -213,6 +239,32 @@ def moe_forward(x_shards, w_gate, w_up, w_down, p: Plan, minibatch: int = 2560, 
                                  ctypes.c_void_p(w_down.data_ptr()), ctypes.byref(p.c), minibatch,
                                  ctypes.byref(opts) if opts else None, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
                                  ya, _stream(stream)))
+    return y_shards, ws
+
+
+class MxWeights(ctypes.Structure):
+    _fields_ = [("gate", ctypes.c_void_p), ("gate_scales", ctypes.c_void_p), ("up", ctypes.c_void_p),
+                ("up_scales", ctypes.c_void_p), ("down", ctypes.c_void_p), ("down_scales", ctypes.c_void_p)]
+
+
+def moe_forward_mxfp8(x_shards, pack, p: Plan, y_shards=None, ws: torch.Tensor | None = None, stream=None):
+    """The forward layer on the MXFP8 path (staged mode).  ``pack`` = (qg, sg,
+    qu, su, qd, sd) from :func:`quantize_weights_mxfp8`.  Returns (y_shards, ws)."""
+    qg, sg, qu, su, qd, sd = pack
+    R = p.c.R
+    H = x_shards[0].shape[1]
+    I = qg.shape[-1]
+    dev = x_shards[0].device
+    opts = fwd_opts(mode=MOK_MODE_STAGED, mxfp8=True)
+    if y_shards is None:
+        y_shards = [torch.empty_like(s) for s in x_shards]
+    if ws is None:
+        ws = _workspace(forward_workspace_bytes(p.c.T, H, I, p.c.E, p.c.k, 0, opts), dev)
+    w = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
+    _check(lib().mok_moe_forward(_ptr_array(x_shards), H, I, ctypes.cast(ctypes.byref(w), ctypes.c_void_p), None,
+                                 None, ctypes.byref(p.c), 0, ctypes.byref(opts), ctypes.c_void_p(ws.data_ptr()),
+                                 ws.numel(), _ptr_array(y_shards), _stream(stream)))
+    assert len(x_shards) == R
     return y_shards, ws
 
 

@@ -121,6 +121,31 @@ bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* w
            encode_bmaps(&m->h, false, h, (uint64_t)I, (uint64_t)buf_rows, err);
 }
 
+// 2D map of a row-major [outer, inner] byte array, no swizzle.
+static bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_mx_maps(MxMaps* m, const mok_mxfp8_weights& w, int H, int I, int E, const char** err) {
+    const bool ok = encode_2d_u8(&m->gq, w.gate, (uint64_t)I, (uint64_t)E * H, 64, 64) &&
+                    encode_2d_u8(&m->uq, w.up, (uint64_t)I, (uint64_t)E * H, 64, 64) &&
+                    encode_2d_u8(&m->dq, w.down, (uint64_t)H, (uint64_t)E * I, 128, 64) &&
+                    encode_2d_u8(&m->gs, w.gate_scales, (uint64_t)I, (uint64_t)E * H / 32, 64, 2) &&
+                    encode_2d_u8(&m->us, w.up_scales, (uint64_t)I, (uint64_t)E * H / 32, 64, 2) &&
+                    encode_2d_u8(&m->ds, w.down_scales, (uint64_t)H, (uint64_t)E * I / 32, 128, 2);
+    if (!ok) *err = "cuTensorMapEncodeTiled failed (MXFP8 weights)";
+    return ok;
+}
+
 // ------------------------------------------------------------------ layouts
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -196,22 +221,33 @@ static int check_hi(int H, int I) {
 }
 
 // ------------------------------------------------------------------ pieces
+// mxw != nullptr: MXFP8 weights (wg/wu/wd are then ignored) and bf16 h.
 static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const void* wg, const void* wu,
                           const void* wd, int E, const int32_t* row_slot, const Chunk* chunks, const int* counts2,
-                          void* h, void* out, DevStatus* status, uint64_t timeout_ns, cudaStream_t stream) {
+                          void* h, void* out, DevStatus* status, uint64_t timeout_ns, cudaStream_t stream,
+                          const mok_mxfp8_weights* mxw = nullptr) {
     int dev = 0;
     const int sms = device_sms(&dev);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     MOK_CUDA(gemm_configure(dev), "gemm configure");
     GemmMaps maps;
+    MxMaps mx;
     const char* err = nullptr;
+    if (mxw) {
+        // the bf16 weight maps are not read on the MXFP8 path: any valid base will do
+        wg = wu = wd = mxw->gate;
+        if (!encode_mx_maps(&mx, *mxw, H, I, E, &err)) return fail(MOK_ERR_CUDA, "tensor map: %s", err);
+    }
     if (!encode_gemm_maps(&maps, wg, wu, wd, rows, h, H, I, E, n_rows_buf, &err))
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
     GemmShape sh{H, I, E};
     const GemmTuning tune = gemm_tuning();
-    MOK_CUDA(launch_gemm_phase(0, maps, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune, stream),
+    const MxMaps* mxp = mxw ? &mx : nullptr;
+    MOK_CUDA(launch_gemm_phase(0, maps, mxp, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune,
+                               stream),
              "gate/up GEMM launch");
-    MOK_CUDA(launch_gemm_phase(1, maps, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune, stream),
+    MOK_CUDA(launch_gemm_phase(1, maps, mxp, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune,
+                               stream),
              "down GEMM launch");
     return MOK_OK;
 }
@@ -291,7 +327,15 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     const int mode = opts ? opts->mode : MOK_MODE_PERSISTENT;
     if (mode != MOK_MODE_STAGED && mode != MOK_MODE_PERSISTENT) return fail(MOK_ERR_INVALID_ARG, "unknown mode %d", mode);
     if (opts && opts->reserved != 0) return fail(MOK_ERR_INVALID_ARG, "opts.reserved must be 0");
-    if (opts && opts->mxfp8) return fail(MOK_ERR_UNSUPPORTED, "MXFP8 path not built");
+    const mok_mxfp8_weights* mxw = nullptr;
+    if (opts && opts->mxfp8) {
+        if (mode != MOK_MODE_STAGED) return fail(MOK_ERR_UNSUPPORTED, "MXFP8 path: staged mode only");
+        mxw = static_cast<const mok_mxfp8_weights*>(w_gate);
+        if (!mxw || !mxw->gate || !mxw->gate_scales || !mxw->up || !mxw->up_scales || !mxw->down ||
+            !mxw->down_scales)
+            return fail(MOK_ERR_INVALID_ARG, "MXFP8 weight pack with NULL members");
+        w_up = w_down = mxw->gate;  // not read on this path
+    }
     if (mode == MOK_MODE_PERSISTENT && minibatch < 16) return fail(MOK_ERR_INVALID_ARG, "minibatch < 16");
     const int T = plan->T, E = plan->E, k = plan->k, R = plan->R;
     if (T == 0) return MOK_OK;
@@ -371,9 +415,12 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         if (e != cudaSuccess) return fail(MOK_ERR_CUDA, "%s: %s", err, cudaGetErrorString(e));
         return MOK_OK;
     }
-    MOK_CUDA(launch_gather(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
+    if (mxw)
+        MOK_CUDA(launch_gather_mx(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
+    else
+        MOK_CUDA(launch_gather(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
     rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, chunks, counts2,
-                        base + L.h, base + L.out, status, timeout, stream);
+                        base + L.h, base + L.out, status, timeout, stream, mxw);
     if (rc) return rc;
     MOK_CUDA(launch_combine(base + L.out, plan->gates, T, k, H, T / R, ys, sms, stream), "combine launch");
     return MOK_OK;
@@ -391,6 +438,32 @@ int mok_prepare_w_down(const void* w_down_bf16, void* w_down_fp16, size_t count,
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     MOK_CUDA(launch_bf16_to_fp16(w_down_bf16, w_down_fp16, count, sms, reinterpret_cast<cudaStream_t>(stream)),
              "weight conversion launch");
+    return MOK_OK;
+}
+
+int mok_mxfp8_quantize_rows(const void* src, int src_f32, int rows, int K, void* q, void* scales,
+                            mok_stream_t stream) {
+    if (rows < 0 || K <= 0) return fail(MOK_ERR_INVALID_ARG, "rows, K out of range");
+    if (K % 32) return fail(MOK_ERR_UNSUPPORTED, "K %% 32 != 0");
+    if (rows == 0) return MOK_OK;
+    if (!src || !q || !scales) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if (reinterpret_cast<uintptr_t>(q) & 7u) return fail(MOK_ERR_UNSUPPORTED, "q must be 8-byte aligned");
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_mx_quant_rows(src, src_f32 != 0, rows, K, q, scales, sms, reinterpret_cast<cudaStream_t>(stream)),
+             "quantiser launch");
+    return MOK_OK;
+}
+
+int mok_quantize_weights_mxfp8(const void* w_bf16, int E, int K, int N, void* q, void* scales,
+                               mok_stream_t stream) {
+    if (E <= 0 || K <= 0 || N <= 0) return fail(MOK_ERR_INVALID_ARG, "E, K, N out of range");
+    if (K % 32) return fail(MOK_ERR_UNSUPPORTED, "K %% 32 != 0");
+    if (!w_bf16 || !q || !scales) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_mx_quant_cols(w_bf16, E * (K / 32), N, q, scales, sms, reinterpret_cast<cudaStream_t>(stream)),
+             "quantiser launch");
     return MOK_OK;
 }
 

@@ -9,6 +9,7 @@
 // bytes of bf16 y, rounding once.
 #include "dispatch_combine.cuh"
 #include "mok_internal.h"
+#include "mxfp8.cuh"
 
 namespace mok {
 
@@ -46,6 +47,64 @@ __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens(ShardsIn xs, int S
             for (int j = 0; j < k; ++j) rows[(size_t)__ldg(pos + (size_t)t * k + j) * nvec + v] = a;
         }
     }
+}
+
+// The same copy with MXFP8 quantisation fused in (MoK article: activation
+// quantisation inside the dispatch): each 32-element block of the token row
+// is quantised to E4M3 with its E8M0 scale and written to the k rows as the
+// exact bf16 value of the quantised block (what the tensor cores multiply).
+// Each lane owns 8 consecutive elements, 4 lanes a block; the step loop is
+// warp-uniform (lanes past the end join the shuffles with zeros).
+__global__ void __launch_bounds__(DC_THREADS) k_gather_tokens_mx(ShardsIn xs, int S_r, int H, int T, int k,
+                                                                 const int32_t* __restrict__ pos,
+                                                                 uint4* __restrict__ rows) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = H >> 3;
+    const int warps = gridDim.x * (DC_THREADS / 32);
+    for (int t = blockIdx.x * (DC_THREADS / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+        const int r = t / S_r;
+        const uint4* src = reinterpret_cast<const uint4*>(xs.p[r]) + (size_t)(t - r * S_r) * nvec;
+        const int my_row = lane < k ? __ldg(pos + (size_t)t * k + lane) : 0;
+        for (int c0 = 0; c0 < H; c0 += 256) {
+            const int c = c0 + lane * 8;
+            const bool live = c < H;
+            const uint4 raw = live ? __ldg(src + (c >> 3)) : make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            float v[8];
+            float amax = 0.f;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float2 f = __bfloat1622float2(b2[p]);
+                v[2 * p] = f.x;
+                v[2 * p + 1] = f.y;
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            const int s = mx_block_exponent(amax);
+            const float inv = mx_pow2(-s), scl = mx_pow2(s);
+            uint32_t o[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float2 d = mx_e4m3x2_to_float2(mx_e4m3x2(v[2 * p] * inv, v[2 * p + 1] * inv));
+                o[p] = pack_bf16x2(d.x * scl, d.y * scl);
+            }
+            const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int j = 0; j < k; ++j) {
+                const int row = __shfl_sync(0xffffffffu, my_row, j);
+                if (live) rows[(size_t)row * nvec + (c >> 3)] = ov;
+            }
+        }
+    }
+}
+
+cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
+                             int num_sms, cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    const int want = (T + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
+    const int grid = want < num_sms * 8 ? want : num_sms * 8;
+    k_gather_tokens_mx<<<grid, DC_THREADS, 0, stream>>>(xs, S_r, H, T, k, pos, reinterpret_cast<uint4*>(rows));
+    return cudaGetLastError();
 }
 
 template <int KMAX>

@@ -4,8 +4,8 @@
 //
 // MoK article (tahou.com): routing paragraph (tokens of one expert laid out
 // contiguously so the grouped GEMM runs efficiently), MXFP8 paragraph
-// (SwiGLU inside the GEMM data path), push-combine paragraph (each result
-// goes back to its token's slot).
+// (quantisation inside the GEMM / SwiGLU data path), push-combine paragraph
+// (each result goes back to its token's slot).
 //
 // Orientation.  Expert segments are short (about 171 rows per expert at 384
 // experts, top-8, 8192 tokens), so the weights take the M = 128 side of every
@@ -16,23 +16,29 @@
 //     columns of Wu (M = 128, K = H, read MN-major straight from the
 //     [E, H, I] layout), B = the chunk's token rows (K-major).  Accumulator
 //     lanes 0-63 hold gate, 64-127 up; the epilogue forms
-//     h = silu(gate) * up and stores fp16 h rows.
-//   down unit (phase 1): A = 128 columns of the fp16 copy of Wd (MN-major
-//     from [E, I, H]), B = the chunk's fp16 h rows.  fp16 keeps 3 more
-//     mantissa bits of h than bf16 would, which keeps the largest element
-//     error of y near the floor set by rounding y itself to bf16.  The
-//     epilogue stores fp32 rows to out[row_slot[row]] (the push combine);
-//     fp32 rather than bf16 because a bf16 slot buffer adds a third bf16
-//     rounding that puts the largest element error of y above 2e-2 * rms(y)
-//     on heavy-tailed outputs.
+//     h = silu(gate) * up and stores h rows.
+//   down unit (phase 1): A = 128 columns of Wd (MN-major from [E, I, H]),
+//     B = the chunk's h rows.  The epilogue stores fp32 rows to
+//     out[row_slot[row]] (the push combine); fp32 rather than bf16 because a
+//     bf16 slot buffer adds a rounding that puts the largest element error of
+//     y above 2e-2 * rms(y) on heavy-tailed outputs.
+// Precision: the bf16 path computes gate/up in bf16 and the down projection
+// in fp16 (fp16 h and the fp16 copy of Wd: 3 more mantissa bits on h keep
+// the error of y at the floor of its own bf16 rounding).  The MXFP8 path
+// reads E4M3 weight bytes with E8M0 block scales and a converter warpgroup
+// turns each tile into exact bf16 values in shared memory (an E4M3 value
+// times 2^s has at most 4 significant bits); x and h are MXFP8-quantised
+// (quantised and dequantised exactly) before they reach the MMA.
 //
-// Roles in a CTA of 6 warps: warp 0 issues TMA loads into a 4-stage ring of
-// 48 KB stages, warp 1 allocates 512 TMEM columns and one thread of it issues
-// tcgen05.mma into one of two 256-column accumulators, warps 2-5 drain the
-// other accumulator (tcgen05.ld) through shared memory to global memory.
-// Token-side tiles are loaded as one TMA box per set bit of the 16-rounded
-// row count (256/128/64/32/16-row maps): the number of small token-side TMA
-// ops was what limited the first version on B200.  Every wait is bounded.
+// Roles in a CTA: warp 0 issues TMA loads into a ring of stages, warp 1
+// allocates 512 TMEM columns and one thread of it issues tcgen05.mma into
+// one of two 256-column accumulators, warps 2-5 drain the other accumulator
+// (tcgen05.ld) through shared memory to global memory, and (MXFP8 only)
+// warps 6-9 convert weight tiles.  The token tile of a stage is ONE TMA box
+// of the next power of two of the 16-rounded row count, and a down unit's
+// two 64-column weight halves come from one 3D map: measured on B200, the
+// number of TMA ops per SM (not bytes) limits this kernel.  Every wait is
+// bounded.
 //
 // A schedule policy (template parameter) tells each role which units this
 // CTA runs, what a unit's inputs wait for, and what its completion signals.
@@ -40,16 +46,14 @@
 
 #include "mok_device.cuh"
 #include "mok_internal.h"
+#include "mxfp8.cuh"
 
 namespace mok {
 
-constexpr int GEMM_THREADS = 192;
-constexpr int NSTAGE = 4;
 constexpr int BK = 64;                            // K per stage: one 128-byte swizzle atom
-constexpr int A_BYTES = 128 * BK * 2;             // 16 KB: two {64 MN x 64 K} boxes
+constexpr int A_BYTES = 128 * BK * 2;             // 16 KB: two {64 MN x 64 K} bf16/fp16 halves
 constexpr int B_ROW_BYTES = BK * 2;               // 128 bytes of one token row per stage
 constexpr int B_BYTES = CHUNK_MAX_ROWS * B_ROW_BYTES;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
 constexpr int EPI_LD = 33;                        // fp32 staging row pitch (bank-conflict free)
 constexpr int EPI_BYTES = 128 * EPI_LD * 4;
 constexpr int TMEM_COLS = 512;
@@ -61,11 +65,37 @@ constexpr uint64_t DRAIN_TIMEOUT_NS = 1000000000ull;
 constexpr int MT_G_FEATURES = 64;                 // gate/up unit: 64 gate + 64 up columns
 constexpr int MT_D_FEATURES = 128;                // down unit: 128 output columns
 
-constexpr int SMEM_STAGES_OFF = 0;
-constexpr int SMEM_EPI_OFF = NSTAGE * STAGE_BYTES;
-constexpr int SMEM_BAR_OFF = SMEM_EPI_OFF + EPI_BYTES;
-constexpr int SMEM_BYTES_USED = SMEM_BAR_OFF + 256;
-constexpr int SMEM_ALLOC = SMEM_BYTES_USED + 1024;  // slack for 1024-byte alignment
+// Stage layouts.  bf16 path: [A 16 KB][B 32 KB] x 4.  MXFP8 path:
+// [A bf16, converted 16 KB][B 32 KB][A E4M3 bytes 8 KB][scales 1 KB] x 3.
+struct Bf16Cfg {
+    static constexpr bool MX = false;
+    static constexpr int THREADS = 192;
+    static constexpr int NST = 4;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int A_OFF = 0, B_OFF = A_BYTES;
+    static constexpr int EPI_OFF = NST * STAGE;
+    static constexpr int XCH_OFF = EPI_OFF + EPI_BYTES;  // unused
+    static constexpr int BAR_OFF = XCH_OFF;
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + slack for 1024-byte alignment
+};
+struct MxCfg {
+    static constexpr bool MX = true;
+    static constexpr int THREADS = 320;
+    static constexpr int NST = 3;
+    static constexpr int A_OFF = 0, B_OFF = A_BYTES;
+    static constexpr int RAW_OFF = A_BYTES + B_BYTES;  // 64 x 128 E4M3 bytes
+    static constexpr int SC_OFF = RAW_OFF + 8192;      // 2 x 128 scale bytes
+    static constexpr int STAGE = SC_OFF + 1024;
+    static constexpr int EPI_OFF = NST * STAGE;
+    static constexpr int XCH_OFF = EPI_OFF + EPI_BYTES;  // amax exchange of the h quantiser
+    static constexpr int BAR_OFF = XCH_OFF + 512;
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+};
+// Shared-memory layout used by code outside the GEMM roles (dispatch CTAs of
+// the persistent kernel place their row slots below SMEM_BAR_OFF).
+constexpr int GEMM_THREADS = Bf16Cfg::THREADS;
+constexpr int SMEM_BAR_OFF = Bf16Cfg::BAR_OFF;
+constexpr int SMEM_ALLOC = Bf16Cfg::SMEM;
 
 // One unit of work: an M tile of one phase over one chunk.
 struct Unit {
@@ -81,7 +111,7 @@ struct Unit {
 
 struct CoreArgs {
     int H, I;
-    __half* h;                // [buffer rows, I] fp16
+    void* h;                  // [buffer rows, I]: fp16 (bf16 path) or bf16 (MXFP8 path)
     float* out;               // [N_s, H] fp32, slot-indexed
     const int32_t* row_slot;  // [N_s]
     DevStatus* st;
@@ -128,9 +158,20 @@ struct StagedSched {
     __device__ void unit_done(const Unit&) const {}
 };
 
+// Token tile of a unit: one box of the next power of two >= the 16-rounded
+// row count.  Returns the map index (box rows = B_MAX_BOX >> index).
+__device__ __forceinline__ int token_box(int rows) {
+    const int r16 = (rows + 15) & ~15;
+    int bx = 0;
+    while (bx + 1 < B_MAPS && (B_MAX_BOX >> (bx + 1)) >= r16) ++bx;
+    return bx;
+}
+
 // ------------------------------------------------------------------ producer
-template <class S>
-__device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const CoreArgs& a, const S& s,
+// Loads the weight tile (bf16/fp16 halves, or MXFP8 bytes + scales) and the
+// token tile of every k-step of every unit into the stage ring.
+template <class S, class C>
+__device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps* mx, const CoreArgs& a, const S& s,
                                               unsigned char* smem, uint64_t* full, uint64_t* empty) {
     int stage = 0;
     uint32_t phase = 0;
@@ -139,41 +180,56 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const CoreAr
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
         if (!s.wait_inputs(u, a.st, a.timeout_ns)) break;
-        const int KB = (u.phase == 0 ? a.H : a.I) / BK;
-        const int wrows = u.phase == 0 ? a.H : a.I;
+        const int K = u.phase == 0 ? a.H : a.I;
+        const int KB = K / BK;
         const BMaps& bm = u.phase == 0 ? maps.rows : maps.h;
-        // token rows rounded up to 16 and loaded as ONE box of the next power
-        // of two (16..256 rows): the count of TMA ops per SM, not bytes, was
-        // measured to be the limit, so a few extra L2 bytes buy fewer ops
-        const int r16 = (u.rows + 15) & ~15;
-        int bx = 0;
-        while (bx + 1 < B_MAPS && (B_MAX_BOX >> (bx + 1)) >= r16) ++bx;
-        const uint32_t bytes = A_BYTES + (uint32_t)(B_MAX_BOX >> bx) * B_ROW_BYTES;
+        const int bx = token_box(u.rows);
+        uint32_t bytes = (uint32_t)(B_MAX_BOX >> bx) * B_ROW_BYTES;
+        if (C::MX)
+            bytes += u.phase == 0 ? 2 * (4096 + 128) : (8192 + 256);  // E4M3 bytes + scale bytes
+        else
+            bytes += A_BYTES;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 10)) {
                 ok = false;
                 break;
             }
-            unsigned char* sa = smem + SMEM_STAGES_OFF + stage * STAGE_BYTES;
-            unsigned char* sb = sa + A_BYTES;
+            unsigned char* st = smem + stage * C::STAGE;
             mbar_arrive_expect_tx(&full[stage], bytes);
-            const int ky = u.expert * wrows + kb * BK;
-            if (u.phase == 0) {
-                tma_load_2d_hint(sa, &maps.wg, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
-                tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
-            } else if (maps.has_wd3) {
-                // both 64-column halves of the 128-column down tile in one op
-                tma_load_3d_hint(sa, &maps.wd3, &full[stage], 0, ky, u.m * 2, evict_first);
+            const int ky = u.expert * K + kb * BK;
+            if constexpr (C::MX) {
+                unsigned char* raw = st + MxCfg::RAW_OFF;
+                unsigned char* sc = st + MxCfg::SC_OFF;
+                const int kys = (u.expert * K + kb * BK) / 32;  // scale row of the first K block
+                if (u.phase == 0) {
+                    tma_load_2d_hint(raw, &mx->gq, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
+                    tma_load_2d_hint(raw + 4096, &mx->uq, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
+                    tma_load_2d(sc, &mx->gs, &full[stage], u.m * MT_G_FEATURES, kys);
+                    tma_load_2d(sc + 128, &mx->us, &full[stage], u.m * MT_G_FEATURES, kys);
+                } else {
+                    tma_load_2d_hint(raw, &mx->dq, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
+                    tma_load_2d(sc, &mx->ds, &full[stage], u.m * MT_D_FEATURES, kys);
+                }
             } else {
-                tma_load_2d_hint(sa, &maps.wd, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
-                tma_load_2d_hint(sa + A_BYTES / 2, &maps.wd, &full[stage], u.m * MT_D_FEATURES + 64, ky,
-                                 evict_first);
+                unsigned char* sa = st + C::A_OFF;
+                if (u.phase == 0) {
+                    tma_load_2d_hint(sa, &maps.wg, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
+                    tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], u.m * MT_G_FEATURES, ky,
+                                     evict_first);
+                } else if (maps.has_wd3) {
+                    // both 64-column halves of the 128-column down tile in one op
+                    tma_load_3d_hint(sa, &maps.wd3, &full[stage], 0, ky, u.m * 2, evict_first);
+                } else {
+                    tma_load_2d_hint(sa, &maps.wd, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
+                    tma_load_2d_hint(sa + A_BYTES / 2, &maps.wd, &full[stage], u.m * MT_D_FEATURES + 64, ky,
+                                     evict_first);
+                }
             }
-            tma_load_2d(sb, &bm.m[bx], &full[stage], kb * BK, u.brow0);
+            tma_load_2d(st + C::B_OFF, &bm.m[bx], &full[stage], kb * BK, u.brow0);
             issued |= 1u << stage;
             issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-            if (++stage == NSTAGE) {
+            if (++stage == C::NST) {
                 stage = 0;
                 phase ^= 1u;
             }
@@ -181,13 +237,79 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const CoreAr
         if (!ok) break;
     }
     // never leave with a load in flight into this CTA's shared memory
-    for (int st = 0; st < NSTAGE; ++st)
+    for (int st = 0; st < C::NST; ++st)
         if ((issued >> st) & 1u) mbar_wait(&full[st], (issued_phase >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 11);
 }
 
-// ------------------------------------------------------------------ MMA issuer
+// ------------------------------------------------------------------ MXFP8 converter (warps 6..9)
+// Per stage: E4M3 bytes (gate/up: two [64 K][64] tiles; down: one [64 K][128]
+// tile) and E8M0 scales ([2 blocks][64] per gate/up tile, [2][128] down) ->
+// the MN-major 128-byte-swizzled bf16 A tile the MMA reads: half h (MN
+// 0-63 / 64-127) at h * 8 KB, K row k at k * 128 bytes, 16-byte chunk j at
+// position j ^ (k & 7).  Each thread converts 8 tasks of 8 elements.
 template <class S>
-__device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* full,
+__device__ __forceinline__ void gemm_converter(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* full,
+                                               uint64_t* conv) {
+    const int ct = threadIdx.x - 192;  // 0..127
+    int stage = 0;
+    uint32_t phase = 0;
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        const int KB = (u.phase == 0 ? a.H : a.I) / BK;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 80)) {
+                ok = false;
+                break;
+            }
+            unsigned char* st = smem + stage * MxCfg::STAGE;
+            const unsigned char* raw = st + MxCfg::RAW_OFF;
+            const unsigned char* sc = st + MxCfg::SC_OFF;
+            unsigned char* dst = st + MxCfg::A_OFF;
+#pragma unroll 2
+            for (int t = 0; t < 8; ++t) {
+                const int task = t * 128 + ct;
+                const int h = task >> 9, k = (task >> 3) & 63, g = task & 7;
+                const unsigned char* src;
+                const unsigned char* scl;
+                if (u.phase == 0) {
+                    src = raw + h * 4096 + k * 64 + g * 8;
+                    scl = sc + h * 128 + (k >> 5) * 64 + g * 8;
+                } else {
+                    src = raw + k * 128 + h * 64 + g * 8;
+                    scl = sc + (k >> 5) * 128 + h * 64 + g * 8;
+                }
+                const uint2 qv = *reinterpret_cast<const uint2*>(src);
+                const uint2 sv = *reinterpret_cast<const uint2*>(scl);
+                uint32_t o[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const uint32_t qw = p < 2 ? qv.x : qv.y;
+                    const uint32_t sw = p < 2 ? sv.x : sv.y;
+                    const int sh = (p & 1) * 16;
+                    const float2 f = mx_e4m3x2_to_float2((uint16_t)(qw >> sh));
+                    const float s0 = mx_pow2((int)((sw >> sh) & 0xff) - 127);
+                    const float s1 = mx_pow2((int)((sw >> (sh + 8)) & 0xff) - 127);
+                    o[p] = pack_bf16x2(f.x * s0, f.y * s1);
+                }
+                *reinterpret_cast<uint4*>(dst + h * 8192 + k * 128 + ((g ^ (k & 7)) << 4)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            fence_proxy_async_shared();  // generic writes -> the MMA's (async proxy) reads
+            mbar_arrive(&conv[stage]);
+            if (++stage == MxCfg::NST) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (!ok) break;
+    }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+// ready[stage]: the TMA barrier (bf16) or the converter barrier (MXFP8).
+template <class S, class C>
+__device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* ready,
                                          uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* fin,
                                          uint32_t tmem_base) {
     int stage = 0;
@@ -198,20 +320,21 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
     for (int i = 0; s.get(i, u); ++i) {
         const int KB = (u.phase == 0 ? a.H : a.I) / BK;
         const int N = (u.rows + 15) & ~15;
-        // gate/up: bf16 x bf16; down: fp16 x fp16 (fp16 W_down copy, fp16 h)
-        const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, u.phase == 0);
+        // bf16 path: gate/up bf16 x bf16, down fp16 x fp16; MXFP8 path: bf16 x bf16
+        const uint32_t idesc =
+            umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, (C::MX || u.phase == 0) ? 1 : 0);
         if (!mbar_wait(&tempty[tb], tph ^ 1u, a.st, a.timeout_ns, 20)) break;
         tc_fence_after();
         const uint32_t dt = tmem_base + (uint32_t)(tb * ACC_COLS);
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
-            if (!mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 21)) {
+            if (!mbar_wait(&ready[stage], phase, a.st, a.timeout_ns, 21)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t sa = smem_u32(smem + SMEM_STAGES_OFF + stage * STAGE_BYTES);
-            const uint32_t sb = sa + A_BYTES;
+            const uint32_t sa = smem_u32(smem + stage * C::STAGE + C::A_OFF);
+            const uint32_t sb = smem_u32(smem + stage * C::STAGE + C::B_OFF);
 #pragma unroll
             for (int ks = 0; ks < BK / 16; ++ks) {
                 // A: MN-major SW128, 16 K rows per MMA = 2 atoms of 1 KB; the
@@ -222,7 +345,7 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
                 umma_bf16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
             }
             umma_commit(&empty[stage]);
-            if (++stage == NSTAGE) {
+            if (++stage == C::NST) {
                 stage = 0;
                 phase ^= 1u;
             }
@@ -240,14 +363,15 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
 }
 
 // ------------------------------------------------------------------ epilogue (warps 2..5)
-template <class S>
+template <class S, class C>
 __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* tfull,
                                               uint64_t* tempty, volatile int* ok_flag, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
     const int et = threadIdx.x - 64;  // 0..127
     const int tok = et & 31, fq = et >> 5;
-    float* epi = reinterpret_cast<float*>(smem + SMEM_EPI_OFF);
+    float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF);
+    float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);  // [4][32] block maxima (MXFP8)
     int tb = 0;
     uint32_t tph = 0;
     Unit u;
@@ -268,34 +392,52 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
             for (int k = 0; k < 32; ++k) myrow[k] = v[k];
             named_bar_sync(1, 128);
             const int col = cc * 32 + tok;
-            if (col < u.rows) {
-                if (u.phase == 0) {
-                    // features m*64 + fq*16 .. +15: gate rows fq*16+k, up rows 64+fq*16+k
-                    uint32_t pk[8];
+            const bool live = col < u.rows;
+            if (u.phase == 0) {
+                // features m*64 + fq*16 .. +15: gate rows fq*16+k, up rows 64+fq*16+k
+                float hv[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float g = epi[(fq * 16 + k) * EPI_LD + tok];
+                    const float up = epi[(64 + fq * 16 + k) * EPI_LD + tok];
+                    hv[k] = g / (1.0f + __expf(-g)) * up;
+                }
+                uint32_t pk[8];
+                if constexpr (C::MX) {
+                    // MXFP8 h: blocks of 32 features = thread pairs fq ^ 1 (same token)
+                    float amax = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(hv[k]));
+                    xch[fq * 32 + tok] = amax;
+                    named_bar_sync(1, 128);
+                    amax = fmaxf(amax, xch[(fq ^ 1) * 32 + tok]);
+                    const int sx = mx_block_exponent(amax);
+                    const float inv = mx_pow2(-sx), scl = mx_pow2(sx);
 #pragma unroll
                     for (int k = 0; k < 16; k += 2) {
-                        const float g0 = epi[(fq * 16 + k) * EPI_LD + tok];
-                        const float g1 = epi[(fq * 16 + k + 1) * EPI_LD + tok];
-                        const float u0 = epi[(64 + fq * 16 + k) * EPI_LD + tok];
-                        const float u1 = epi[(64 + fq * 16 + k + 1) * EPI_LD + tok];
-                        const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                        const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                        pk[k >> 1] = pack_half2_sat(h0, h1);
+                        const float2 d = mx_e4m3x2_to_float2(mx_e4m3x2(hv[k] * inv, hv[k + 1] * inv));
+                        pk[k >> 1] = pack_bf16x2(d.x * scl, d.y * scl);
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(a.h + (size_t)(u.brow0 + col) * a.I + u.m * MT_G_FEATURES +
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 16; k += 2) pk[k >> 1] = pack_half2_sat(hv[k], hv[k + 1]);
+                }
+                if (live) {
+                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) +
+                                                          (size_t)(u.brow0 + col) * a.I + u.m * MT_G_FEATURES +
                                                           fq * 16);
                     dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                } else {
-                    // fp32 push to the token's slot; the combine rounds y once
-                    const int slot = __ldg(a.row_slot + u.grow0 + col);
-                    float4* dst = reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + u.m * MT_D_FEATURES + fq * 32);
+                }
+            } else if (live) {
+                // fp32 push to the token's slot; the combine rounds y once
+                const int slot = __ldg(a.row_slot + u.grow0 + col);
+                float4* dst = reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + u.m * MT_D_FEATURES + fq * 32);
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        const int f = fq * 32 + q4 * 4;
-                        dst[q4] = make_float4(epi[f * EPI_LD + tok], epi[(f + 1) * EPI_LD + tok],
-                                              epi[(f + 2) * EPI_LD + tok], epi[(f + 3) * EPI_LD + tok]);
-                    }
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const int f = fq * 32 + q4 * 4;
+                    dst[q4] = make_float4(epi[f * EPI_LD + tok], epi[(f + 1) * EPI_LD + tok],
+                                          epi[(f + 2) * EPI_LD + tok], epi[(f + 3) * EPI_LD + tok]);
                 }
             }
             named_bar_sync(1, 128);
@@ -319,13 +461,15 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
 }
 
 // ------------------------------------------------------------------ one GEMM CTA
-// Runs every unit the schedule gives this CTA.  All GEMM_THREADS threads
-// must call it; it returns after TMEM is released.
-template <class S>
-__device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const CoreArgs& a, const S& s, unsigned char* smem) {
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
-    uint64_t* empty = full + NSTAGE;
-    uint64_t* tfull = empty + NSTAGE;
+// Runs every unit the schedule gives this CTA.  All C::THREADS threads must
+// call it; it returns after TMEM is released.  mx: MXFP8 maps (C::MX only).
+template <class S, class C>
+__device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx, const CoreArgs& a, const S& s,
+                                         unsigned char* smem) {
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint64_t* empty = full + C::NST;
+    uint64_t* conv = empty + C::NST;  // MXFP8 only
+    uint64_t* tfull = conv + C::NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* fin = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
@@ -333,9 +477,10 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const CoreArgs& a
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int st = 0; st < NSTAGE; ++st) {
+        for (int st = 0; st < C::NST; ++st) {
             mbar_init(&full[st], 1);
             mbar_init(&empty[st], 1);
+            mbar_init(&conv[st], 128);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
@@ -345,10 +490,19 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const CoreArgs& a
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&maps.wg);
-        tma_prefetch_desc(&maps.wu);
-        tma_prefetch_desc(&maps.wd);
-        if (maps.has_wd3) tma_prefetch_desc(&maps.wd3);
+        if constexpr (C::MX) {
+            tma_prefetch_desc(&mx->gq);
+            tma_prefetch_desc(&mx->uq);
+            tma_prefetch_desc(&mx->dq);
+            tma_prefetch_desc(&mx->gs);
+            tma_prefetch_desc(&mx->us);
+            tma_prefetch_desc(&mx->ds);
+        } else {
+            tma_prefetch_desc(&maps.wg);
+            tma_prefetch_desc(&maps.wu);
+            tma_prefetch_desc(&maps.wd);
+            if (maps.has_wd3) tma_prefetch_desc(&maps.wd3);
+        }
         for (int b = 0; b < B_MAPS; ++b) {
             tma_prefetch_desc(&maps.rows.m[b]);
             tma_prefetch_desc(&maps.h.m[b]);
@@ -364,11 +518,13 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const CoreArgs& a
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) gemm_producer(maps, a, s, smem, full, empty);
+        if (lane == 0) gemm_producer<S, C>(maps, mx, a, s, smem, full, empty);
     } else if (warp == 1) {
-        if (lane == 0) gemm_mma(a, s, smem, full, empty, tfull, tempty, fin, tmem_base);
-    } else {
-        gemm_epilogue(a, s, smem, tfull, tempty, ok_flag, tmem_base);
+        if (lane == 0) gemm_mma<S, C>(a, s, smem, C::MX ? conv : full, empty, tfull, tempty, fin, tmem_base);
+    } else if (warp < 6) {
+        gemm_epilogue<S, C>(a, s, smem, tfull, tempty, ok_flag, tmem_base);
+    } else if constexpr (C::MX) {
+        gemm_converter(a, s, smem, full, conv);
     }
 
     tc_fence_before();

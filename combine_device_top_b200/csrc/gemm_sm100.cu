@@ -2,13 +2,16 @@
 // MoE layer as its own launches): one persistent launch per phase, gate/up
 // + SwiGLU then down + push, over every chunk of the device-built work list.
 // The tcgen05/TMEM/TMA core and its design notes are in gemm_core.cuh.
+#include <cstring>
+
 #include "gemm_core.cuh"
 
 namespace mok {
 
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_grouped_gemm(const __grid_constant__ GemmMaps maps, const CoreArgs a, const Chunk* __restrict__ chunks,
-                   const int* __restrict__ counts2, int phase, int MT, int GC) {
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    k_grouped_gemm(const __grid_constant__ GemmMaps maps, const __grid_constant__ MxMaps mx, const CoreArgs a,
+                   const Chunk* __restrict__ chunks, const int* __restrict__ counts2, int phase, int MT, int GC) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align_smem_1024(smem_raw);
     StagedSched s;
@@ -17,7 +20,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     s.MT = MT;
     s.GC = GC;
     s.chunks = chunks;
-    gemm_cta(maps, a, s, smem);
+    gemm_cta<StagedSched, C>(maps, &mx, a, s, smem);
 }
 
 size_t gemm_smem_bytes() { return SMEM_ALLOC; }
@@ -35,25 +38,37 @@ cudaError_t gemm_configure(int dev) {
     static bool done[64] = {};
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (done[dev]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<Bf16Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Bf16Cfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm<MxCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, MxCfg::SMEM);
     if (e == cudaSuccess) done[dev] = true;
     return e;
 }
 
-cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const GemmShape& sh, const Chunk* chunks,
-                              const int* counts2, void* h_out, void* out, const int32_t* row_slot, void* status,
-                              uint64_t timeout_ns, int grid, const GemmTuning& tune, cudaStream_t stream) {
+cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const GemmShape& sh,
+                              const Chunk* chunks, const int* counts2, void* h_out, void* out,
+                              const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
+                              const GemmTuning& tune, cudaStream_t stream) {
     CoreArgs a;
     a.H = sh.H;
     a.I = sh.I;
-    a.h = reinterpret_cast<__half*>(h_out);
+    a.h = h_out;
     a.out = reinterpret_cast<float*>(out);
     a.row_slot = row_slot;
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
     const int MT = phase == 0 ? sh.I / MT_G_FEATURES : sh.H / MT_D_FEATURES;
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
-    k_grouped_gemm<<<grid, GEMM_THREADS, SMEM_ALLOC, stream>>>(maps, a, chunks, counts2, phase, MT, GC);
+    if (mx) {
+        k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,
+                                                                            MT, GC);
+    } else {
+        MxMaps none;
+        memset(&none, 0, sizeof none);
+        k_grouped_gemm<Bf16Cfg><<<grid, Bf16Cfg::THREADS, Bf16Cfg::SMEM, stream>>>(maps, none, a, chunks, counts2,
+                                                                                  phase, MT, GC);
+    }
     return cudaGetLastError();
 }
 

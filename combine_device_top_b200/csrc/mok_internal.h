@@ -38,6 +38,10 @@ struct ShardsOut {
 // rows[pos[t*k + j]] = x[t] for every slot (token-major walk of the pull schedule)
 cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
                           int num_sms, cudaStream_t stream);
+// the same with MXFP8 quantisation of every 32-element block (rows hold the
+// exact bf16 values of the quantised blocks)
+cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
+                             int num_sms, cudaStream_t stream);
 cudaError_t launch_combine(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
                            int num_sms, cudaStream_t stream);
 
@@ -89,11 +93,21 @@ struct GemmMaps {
 bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
                       int H, int I, int E, int buf_rows, const char** err);
 
+// Extra maps of the MXFP8 GEMM: E4M3 weight bytes and E8M0 scale bytes.
+struct MxMaps {
+    CUtensorMap gq, uq, dq;  // bytes: {64, 64} boxes of Wg/Wu [E*H, I]; {128, 64} boxes of Wd [E*I, H]
+    CUtensorMap gs, us, ds;  // scales: {64, 2} boxes of [E*H/32, I]; {128, 2} boxes of [E*I/32, H]
+};
+bool encode_mx_maps(MxMaps* m, const mok_mxfp8_weights& w, int H, int I, int E, const char** err);
+
 // Staged grouped GEMM over every chunk: phase 0 = gate/up + SwiGLU -> h,
 // phase 1 = down -> out[row_slot].
-cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const GemmShape& sh, const Chunk* chunks,
-                              const int* counts2, void* h_out, void* out, const int32_t* row_slot, void* status,
-                              uint64_t timeout_ns, int grid, const GemmTuning& tune, cudaStream_t stream);
+struct MxMaps;
+// mx: MXFP8 weight maps (MXFP8 path; h is bf16 then), or nullptr (bf16 path).
+cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const GemmShape& sh,
+                              const Chunk* chunks, const int* counts2, void* h_out, void* out,
+                              const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
+                              const GemmTuning& tune, cudaStream_t stream);
 
 // ---- the persistent SM-partitioned forward (persistent.cu)
 struct PersistLaunch {
@@ -121,6 +135,12 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
 // (bf16 or fp16), 128-byte swizzle, zero fill out of bounds.
 bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
                         uint32_t box_inner, uint32_t box_outer, const char** err);
+
+// ---- MXFP8 quantisers (mxfp8.cu)
+cudaError_t launch_mx_quant_rows(const void* src, bool f32, int rows, int K, void* q, void* scales, int num_sms,
+                                 cudaStream_t stream);
+cudaError_t launch_mx_quant_cols(const void* src, int nblocks, int N, void* q, void* scales, int num_sms,
+                                 cudaStream_t stream);
 
 // ---- weight preparation
 cudaError_t launch_bf16_to_fp16(const void* src, void* dst, size_t n, int num_sms, cudaStream_t stream);

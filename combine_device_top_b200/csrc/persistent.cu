@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         s.gidx = blockIdx.x - D;
         s.gctas = gridDim.x - D;
         s.total = nch * (p.MTG + p.MTD);
-        gemm_cta(maps, a, s, smem);
+        gemm_cta<PersistSched, Bf16Cfg>(maps, nullptr, a, s, smem);
     }
 
     // -------------------------------------------- combine, once every down unit is done
@@ -243,7 +243,7 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     CoreArgs a;
     a.H = L.H;
     a.I = L.I;
-    a.h = reinterpret_cast<__half*>(L.h);
+    a.h = L.h;
     a.out = L.out;
     a.row_slot = L.row_slot;
     a.st = reinterpret_cast<DevStatus*>(L.status);

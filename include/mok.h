@@ -161,6 +161,18 @@ typedef struct mok_fwd_opts {
     uint64_t timeout_ns;   /* bound on every device-side wait; 0 = 2 s          */
 } mok_fwd_opts;
 
+/* MXFP8 weight pack (opts->mxfp8 = 1): pass a pointer to this HOST struct
+ * as mok_moe_forward's w_gate (w_up and w_down are then ignored).  Every
+ * member is a device pointer made by mok_quantize_weights_mxfp8. */
+typedef struct mok_mxfp8_weights {
+    const void* gate;         /* [E, H, I] E4M3      */
+    const void* gate_scales;  /* [E, H/32, I] E8M0   */
+    const void* up;           /* [E, H, I] E4M3      */
+    const void* up_scales;    /* [E, H/32, I] E8M0   */
+    const void* down;         /* [E, I, H] E4M3      */
+    const void* down_scales;  /* [E, I/32, H] E8M0   */
+} mok_mxfp8_weights;
+
 /* Bytes of forward workspace; 0 if the shape is invalid.  opts may be NULL
  * (defaults).  minibatch = rows per minibatch (see mok_moe_forward). */
 size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int minibatch,
@@ -212,6 +224,29 @@ int mok_moe_forward(const void* const* x_shards, int H, int I,
  * rounding.)
  */
 int mok_prepare_w_down(const void* w_down_bf16, void* w_down_fp16, size_t count, mok_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * MXFP8 (OCP MX v1.0: 32-element blocks, E8M0 scale byte = s + 127 with
+ * s = floor(log2(max|v|)) - 8 clamped to [-127, 127], an all-zero block
+ * gets 0x00; E4M3 elements = v / 2^s rounded to nearest even, saturating at
+ * +-448).  Source: MoK article, paragraph after the ring buffer (MXFP8
+ * activation quantisation fused into dispatch, grouped GEMM and SwiGLU).
+ * ---------------------------------------------------------------------- */
+
+/* Activation layout: blocks of 32 consecutive elements along each row.
+ *   src     [rows, K] bf16 (src_f32 = 0) or fp32 (src_f32 = 1); K % 32 == 0
+ *   q       [rows, K] E4M3 bytes;  scales [rows, K/32] E8M0 bytes
+ * This is the quantiser the MXFP8 forward fuses into the gather (x) and the
+ * SwiGLU epilogue (h). */
+int mok_mxfp8_quantize_rows(const void* src, int src_f32, int rows, int K, void* q, void* scales,
+                            mok_stream_t stream);
+
+/* Weight layout: w [E, K, N] bf16 (K = contraction index, N = output
+ * columns, i.e. Wg/Wu with K = H, N = I and Wd with K = I, N = H); blocks of
+ * 32 along K of each column.  q [E, K, N] E4M3 bytes (same layout as w),
+ * scales [E, K/32, N] E8M0 bytes.  K % 32 == 0.  One-time, at weight load. */
+int mok_quantize_weights_mxfp8(const void* w_bf16, int E, int K, int N, void* q, void* scales,
+                               mok_stream_t stream);
 
 /*
  * mok_get_status -- synchronise `stream` and read the device status word of

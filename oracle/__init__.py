@@ -140,6 +140,34 @@ def expert_ffn(x_rows: torch.Tensor, wg: torch.Tensor, wu: torch.Tensor, wd: tor
     return o
 
 
+def mxfp8_expert_ffn(x_rows: torch.Tensor, wg: torch.Tensor, wu: torch.Tensor, wd: torch.Tensor) -> torch.Tensor:
+    """One expert's SwiGLU FFN on the MXFP8 path (x, weights and h quantised
+    in 32-blocks, exact accumulation); bf16 inputs, float64 result [n, H]."""
+    x_rows = _c(x_rows, torch.bfloat16)
+    n, H = x_rows.shape
+    I = wg.shape[1]
+    o = torch.empty((n, H), dtype=torch.float64)
+    _check(lib().oracle_mxfp8_expert_ffn(_ptr(x_rows), n, H, I, _ptr(_c(wg, torch.bfloat16)),
+                                         _ptr(_c(wu, torch.bfloat16)), _ptr(_c(wd, torch.bfloat16)), _ptr(o),
+                                         None, None, None), "mxfp8_expert_ffn")
+    return o
+
+
+def moe_forward_mxfp8(x, logits, wg, wu, wd, k: int, R: int):
+    """Whole layer on the MXFP8 path (small inputs) -> y [T,H] float64."""
+    T, H = x.shape
+    E = wg.shape[0]
+    p = plan(logits, k, R)
+    rows = gather(x, R, p["src_rank"], p["src_index"])
+    o_slot = torch.zeros((T * k, H), dtype=torch.float64)
+    off = p["offsets"]
+    for e in range(E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b > a:
+            o_slot[p["row_slot"][a:b].long()] = mxfp8_expert_ffn(rows[a:b], wg[e], wu[e], wd[e])
+    return combine(o_slot.view(T, k, H), p["gates"])
+
+
 def combine(o_slot: torch.Tensor, gates: torch.Tensor) -> torch.Tensor:
     """o_slot [T,k,H] float64, gates [T,k] -> y [T,H] float64."""
     o_slot = _c(o_slot, torch.float64)

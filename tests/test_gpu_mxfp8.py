@@ -1,0 +1,146 @@
+"""MXFP8 on the GPU: quantiser bytes and scales bit-exact against the
+oracle's emulation of the OCP MX definition, and the MXFP8 forward layer
+against the emulated oracle (relative Frobenius <= 2e-2)."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import combine_device_top_b200 as mok
+import mokgen
+import oracle
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _oracle_quant(v: np.ndarray):
+    """Blocks of 32 consecutive values -> (bytes, scales) from the oracle."""
+    L = oracle.lib()
+    v = np.ascontiguousarray(v, dtype=np.float32).reshape(-1)
+    nb = v.size // 32
+    q = np.zeros(v.size, np.uint8)
+    s = np.zeros(nb, np.uint8)
+    assert L.oracle_mxfp8_quantize(v.ctypes.data, nb, q.ctypes.data, s.ctypes.data) == 0
+    return q, s
+
+
+def _spread(rows, K, seed):
+    """bf16 rows with block magnitudes spread over many binades, zeros and ties."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(rows, K, generator=g)
+    mag = torch.pow(2.0, torch.randint(-40, 40, (rows, K // 32), generator=g).float())
+    x = x * mag.repeat_interleave(32, dim=1)
+    x[0, :32] = 0.0
+    x[1, :32] = -0.0
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("rows,K", [(64, 256), (37, 7168), (5, 32)])
+def test_row_quantiser_bit_exact_bf16(rows, K):
+    x = _spread(rows, K, seed=rows + K)
+    q, s = mok.mxfp8_quantize_rows(x.cuda())
+    wq, ws = _oracle_quant(x.float().numpy())
+    assert np.array_equal(q.cpu().numpy().reshape(-1), wq)
+    assert np.array_equal(s.cpu().numpy().reshape(-1), ws)
+
+
+def test_row_quantiser_bit_exact_fp32_golden_blocks():
+    """fp32 input (the form the SwiGLU epilogue quantises): the hand-computed
+    edge-case blocks plus random fp32 data."""
+    with open(os.path.join(GOLDEN, "mxfp8_blocks.json")) as f:
+        spec = json.load(f)
+    blocks = []
+    for case in spec["cases"]:
+        v = np.zeros(32, np.float32)
+        for i, val in case["values"].items():
+            v[int(i)] = val
+        blocks.append(v)
+    g = np.random.default_rng(3)
+    rnd = (g.standard_normal((10, 32)) * np.exp2(g.integers(-60, 60, (10, 1)))).astype(np.float32)
+    data = np.concatenate([np.stack(blocks), rnd]).reshape(-1, 64)  # two blocks per row
+    q, s = mok.mxfp8_quantize_rows(torch.from_numpy(data).cuda())
+    wq, ws = _oracle_quant(data)
+    assert np.array_equal(q.cpu().numpy().reshape(-1), wq)
+    assert np.array_equal(s.cpu().numpy().reshape(-1), ws)
+    # and the golden bytes themselves
+    gq = q.cpu().numpy().reshape(-1, 32)
+    gs = s.cpu().numpy().reshape(-1)
+    for i, case in enumerate(spec["cases"]):
+        assert gs[i] == int(case["scale"], 16), case["name"]
+        for j, b in case["bytes"].items():
+            assert gq[i, int(j)] == int(b, 16), (case["name"], j)
+
+
+REL_FRO_MX = 2e-2
+
+MX_CASES = {
+    "tiny": mokgen.scaled(mokgen.CONFIGS["tiny"], seed=201),
+    "page_like": mokgen.scaled(mokgen.CONFIGS["page"], T=256, E=12, seed=202),
+    "ragged": mokgen.scaled(mokgen.CONFIGS["tiny"], T=600, H=384, I=192, E=5, k=3, R=3, seed=203),
+}
+
+
+def _mx_pack(dwg, dwu, dwd):
+    qg, sg = mok.quantize_weights_mxfp8(dwg)
+    qu, su = mok.quantize_weights_mxfp8(dwu)
+    qd, sd = mok.quantize_weights_mxfp8(dwd)
+    return (qg, sg, qu, su, qd, sd)
+
+
+@pytest.mark.parametrize("name", list(MX_CASES))
+def test_mxfp8_forward_matches_emulated_oracle(name):
+    cfg = MX_CASES[name]
+    x = mokgen.tokens(cfg)
+    logits = mokgen.router_logits(cfg, x)
+    wg, wu, wd = mokgen.all_expert_weights(cfg)
+    pack = _mx_pack(wg.cuda(), wu.cuda(), wd.cuda())
+    p = mok.plan(logits.cuda(), cfg.k, cfg.R)
+    ys, ws = mok.moe_forward_mxfp8(mok.shards(x.cuda(), cfg.R), pack, p)
+    assert mok.get_status(ws) == mok.MOK_OK
+    y = torch.cat([s.cpu() for s in ys]).double()
+    want = oracle.moe_forward_mxfp8(x, logits, wg, wu, wd, cfg.k, cfg.R)
+    rel = (torch.linalg.norm(y - want) / torch.linalg.norm(want)).item()
+    assert rel <= REL_FRO_MX, rel
+
+
+@pytest.mark.slow
+def test_mxfp8_forward_full_size_sampled():
+    """The page shape on the MXFP8 path: every row computed on the GPU,
+    sampled tokens against the emulated oracle."""
+    cfg = mokgen.CONFIGS["page_mxfp8"]
+    x = mokgen.tokens(cfg)
+    logits = mokgen.router_logits(cfg, x)
+    wg, wu, wd = mokgen.upload_expert_weights(cfg, "cuda")
+    pack = _mx_pack(wg, wu, wd)
+    del wg, wu, wd
+    torch.cuda.empty_cache()
+    p = mok.plan(logits.cuda(), cfg.k, cfg.R)
+    ys, ws = mok.moe_forward_mxfp8(mok.shards(x.cuda(), cfg.R), pack, p)
+    assert mok.get_status(ws) == mok.MOK_OK
+    y = torch.cat([s.cpu() for s in ys]).double()
+    ids = sorted(set(torch.randperm(cfg.T, generator=torch.Generator().manual_seed(4))[:6].tolist()))
+    idx, g = oracle.topk_gates(logits[ids], cfg.k)
+    want = torch.zeros((len(ids), cfg.H), dtype=torch.float64)
+    for a in range(len(ids)):
+        for j in range(cfg.k):
+            e = int(idx[a, j])
+            o = oracle.mxfp8_expert_ffn(x[ids[a]:ids[a] + 1], *mokgen.expert_weights(cfg, e))
+            want[a] += float(g[a, j]) * o[0]
+    rel = (torch.linalg.norm(y[ids] - want) / torch.linalg.norm(want)).item()
+    assert rel <= REL_FRO_MX, rel
+
+
+def test_weight_quantiser_bit_exact():
+    E, K, N = 3, 256, 192
+    w = _spread(E * K, N, seed=9).reshape(E, K, N)
+    q, s = mok.quantize_weights_mxfp8(w.cuda())
+    q, s = q.cpu().numpy(), s.cpu().numpy()
+    for e in range(E):
+        cols = w[e].float().t().contiguous().numpy()  # [N, K]: blocks along K are contiguous
+        wq, ws = _oracle_quant(cols)
+        assert np.array_equal(q[e].T.reshape(-1), wq)
+        assert np.array_equal(s[e].T.reshape(-1), ws)
