@@ -114,12 +114,21 @@ def algorithmic_work(cfg):
     ns = cfg.slots
     w_bytes = cfg.E * 3 * cfg.H * cfg.I * 2
     gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 4  # weights, rows in, h out+in, fp32 out
+    gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * 2
+    if cfg.mxfp8:
+        # weights: E4M3 bytes plus one E8M0 scale per 32 values; the quantised
+        # token rows and h are kept in their exact bf16 form (2 bytes a value)
+        w_bytes = cfg.E * 3 * cfg.H * cfg.I * (1.0 + 1.0 / 32)
+        gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 4
+    combine_bytes = ns * cfg.H * 4 + ns * 4 + cfg.T * cfg.H * 2
     return {
         "gemm_flops": 6.0 * cfg.H * cfg.I * ns,
         "gemm_bytes": float(gemm_bytes),
         "weight_bytes": float(w_bytes),
-        "gather_bytes": float(cfg.T * cfg.H * 2 + ns * cfg.H * 2),
-        "combine_bytes": float(ns * cfg.H * 4 + ns * 4 + cfg.T * cfg.H * 2),
+        "gather_bytes": float(gather_bytes),
+        "combine_bytes": float(combine_bytes),
+        # gather + grouped GEMM + combine: what one mok_moe_forward call must move
+        "forward_bytes": float(gather_bytes + gemm_bytes + combine_bytes),
         "plan_bytes": float(cfg.T * cfg.E * 4 + ns * 4 * 8),
     }
 
@@ -132,18 +141,27 @@ def run_mok(args, cfg, rank, world, device):
     logits = mokgen.router_logits(cfg, x)
     dx, dlogits = x.to(device), logits.to(device)
     wg, wu, wd_bf16 = mokgen.upload_expert_weights(cfg, device)
-    wd = mok.prepare_w_down(wd_bf16)      # one-time weight preparation, untimed
-    del wd_bf16
+    pack = None
+    if cfg.mxfp8:
+        # one-time MXFP8 weight quantisation, untimed
+        pack = (*mok.quantize_weights_mxfp8(wg), *mok.quantize_weights_mxfp8(wu), *mok.quantize_weights_mxfp8(wd_bf16))
+        del wg, wu, wd_bf16
+        wg = wu = wd = None
+        torch.cuda.empty_cache()
+    else:
+        wd = mok.prepare_w_down(wd_bf16)      # one-time weight preparation, untimed
+        del wd_bf16
     x_shards = mok.shards(dx, cfg.R)
     y = torch.empty_like(dx)
     y_shards = mok.shards(y, cfg.R)
-    mode = mok.MOK_MODE_STAGED if args.mode == "staged" else mok.MOK_MODE_PERSISTENT
-    opts = mok.fwd_opts(mode=mode, ring_slots=cfg.ring_slots)
+    mode = mok.MOK_MODE_STAGED if (args.mode == "staged" or cfg.mxfp8) else mok.MOK_MODE_PERSISTENT
+    opts = mok.fwd_opts(mode=mode, ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8)
     minibatch = args.minibatch or cfg.minibatch
     p = mok.plan(dlogits, cfg.k, cfg.R)
     fws = torch.empty(mok.forward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
                       dtype=torch.uint8, device=device)
-    staged = mode == mok.MOK_MODE_STAGED
+    # the bf16 staged mode is timed one ABI step at a time (per-phase events)
+    staged = mode == mok.MOK_MODE_STAGED and not cfg.mxfp8
     if staged:
         rows = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
         out = torch.empty((cfg.slots, cfg.H), dtype=torch.float32, device=device)
@@ -170,6 +188,8 @@ def run_mok(args, cfg, rank, world, device):
             if evs:
                 evs[3].record(stream)
             mok.combine(out, p, y_shards)
+        elif pack is not None:
+            mok.moe_forward_mxfp8(x_shards, pack, p, y_shards=y_shards, ws=fws)
         else:
             mok.moe_forward(x_shards, wg, wu, wd, p, minibatch, opts, y_shards=y_shards, ws=fws)
         if evs:
@@ -209,16 +229,17 @@ def run_mok(args, cfg, rank, world, device):
     if rank == 0 or world > 1:
         hx, hl = x.pin_memory(), logits.pin_memory()
         hy = torch.empty_like(x).pin_memory()
+        wts = (pack, None, None) if pack is not None else (wg, wu, wd)
         hws = torch.empty(mok.forward_host_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
                           dtype=torch.uint8, device=device)
         for _ in range(2):
-            mok.moe_forward_host(hx, hl, cfg.k, cfg.R, wg, wu, wd, minibatch, opts, hws, hy)
+            mok.moe_forward_host(hx, hl, cfg.k, cfg.R, *wts, minibatch, opts, hws, hy)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(1, min(args.steps, 5))
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(n_e2e):
-            mok.moe_forward_host(hx, hl, cfg.k, cfg.R, wg, wu, wd, minibatch, opts, hws, hy)
+            mok.moe_forward_host(hx, hl, cfg.k, cfg.R, *wts, minibatch, opts, hws, hy)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / n_e2e
@@ -230,7 +251,9 @@ def run_mok(args, cfg, rank, world, device):
         res["h2d"] = cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4
         res["d2h"] = cfg.T * cfg.H * 2
         del hws
-    res["launches_per_step"] = (3 + 1 + 1 + 2 + 1) if staged else (3 + 2)
+    # plan: route, scan, scatter; staged forward: chunk list, gather, gate/up, down, combine;
+    # persistent forward: chunk list, one persistent kernel
+    res["launches_per_step"] = (3 + 1 + 1 + 2 + 1) if mode == mok.MOK_MODE_STAGED else (3 + 2)
     res["max_over_mean_load"] = (lambda c: c.max().item() / c.mean().item())(p.counts().float())
     return res
 
@@ -294,9 +317,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     metric = "MoE fwd tokens/s (H7168/I2048)"
-    config = {"workload": f"{cfg.name}: {cfg.describe()}, bf16 weights [E,H,I]/[E,I,H]",
+    wdesc = ("MXFP8 E4M3 weights + E8M0 scales per 32 along K (quantised once, untimed)" if cfg.mxfp8
+             else "bf16 weights [E,H,I]/[E,I,H]")
+    config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
               "tokens_per_step_per_gpu": cfg.T, "minibatch": args.minibatch or cfg.minibatch,
-              "mode": args.mode, "l2": "inputs larger than L2 (33.8 GB of expert weights streamed per step)"}
+              "mode": "staged" if cfg.mxfp8 else args.mode,
+              "l2": f"inputs larger than L2 ({algorithmic_work(cfg)['weight_bytes'] / 1e9:.1f} GB of expert "
+                    f"weights streamed per step)"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -328,7 +355,8 @@ def main():
     ph = res["phases_ms"]
     line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config}
+            "vs_baseline": None, "dtype": "mxfp8-e4m3 (bf16 MMA)" if cfg.mxfp8 else "bf16",
+            "data": "synthetic", "config": config}
     if args.mode == "staged":
         t_plan, t_gather, t_gemm, t_comb = ph
         gemm_s = t_gemm / 1e3
@@ -354,7 +382,20 @@ def main():
             "plan_share": t_plan / ms,
         }
     else:
-        line["phases_ms"] = {"plan": ph[0], "forward": ph[1]}
+        # one mok_moe_forward call (gather, grouped GEMM and combine together) is the timed kernel work
+        t_plan, t_fwd = ph
+        fwd_s = t_fwd / 1e3
+        gbs = work["forward_bytes"] / fwd_s / 1e9
+        tflops = work["gemm_flops"] / fwd_s / 1e12
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                "kernel": ("MXFP8 forward (gather, gate/up+SwiGLU, down, combine launches)" if cfg.mxfp8 else
+                           "persistent forward kernel (dispatch, grouped GEMM, combine in one launch)"),
+                "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
+                "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"]}
+        line["roofline"] = roof
+        line["phases_ms"] = {"plan": t_plan, "forward": t_fwd}
+        line["phase_rates"] = {"forward_GBps": gbs, "forward_TFLOPs": tflops, "plan_share": t_plan / ms}
     if "e2e_ms" in res:
         line["e2e"] = {"value": cfg.T * world / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
                        "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]}

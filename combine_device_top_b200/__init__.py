@@ -318,13 +318,21 @@ def forward_host_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None 
 
 def moe_forward_host(x_host: torch.Tensor, logits_host: torch.Tensor, top_k: int, R: int, w_gate, w_up, w_down,
                      minibatch: int, opts: FwdOpts | None, ws: torch.Tensor, y_host: torch.Tensor, stream=None):
-    """End to end from host memory: ``mok_moe_forward_host``."""
+    """End to end from host memory: ``mok_moe_forward_host``.  On the MXFP8
+    path (``opts.mxfp8``) ``w_gate`` is the pack from :func:`quantize_weights_mxfp8`
+    (qg, sg, qu, su, qd, sd) and ``w_up``/``w_down`` are None."""
     T, H = x_host.shape
     E = logits_host.shape[1]
-    I = w_gate.shape[-1]
+    if isinstance(w_gate, tuple):
+        qg, sg, qu, su, qd, sd = w_gate
+        I = qg.shape[-1]
+        mx = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
+        wptrs = (ctypes.cast(ctypes.byref(mx), ctypes.c_void_p), None, None)
+    else:
+        I = w_gate.shape[-1]
+        wptrs = tuple(ctypes.c_void_p(w.data_ptr()) for w in (w_gate, w_up, w_down))
     _check(lib().mok_moe_forward_host(ctypes.c_void_p(x_host.data_ptr()), ctypes.c_void_p(logits_host.data_ptr()),
-                                      T, H, I, E, top_k, R, ctypes.c_void_p(w_gate.data_ptr()),
-                                      ctypes.c_void_p(w_up.data_ptr()), ctypes.c_void_p(w_down.data_ptr()),
+                                      T, H, I, E, top_k, R, *wptrs,
                                       minibatch, ctypes.byref(opts) if opts else None,
                                       ctypes.c_void_p(ws.data_ptr()), ws.numel(),
                                       ctypes.c_void_p(y_host.data_ptr()), _stream(stream)))

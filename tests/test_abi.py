@@ -97,6 +97,29 @@ def test_forward_rejects_unsupported_shapes():
     assert rc == mok.MOK_ERR_INVALID_ARG
 
 
+def test_forward_mxfp8_argument_rules():
+    """The MXFP8 path is staged only and needs every member of its weight pack."""
+    p = mok.PlanT(16, 8, 2, 2)
+    for name in ("counts", "offsets", "sched_src_rank", "sched_src_index", "row_slot", "pos", "topk_idx", "gates"):
+        setattr(p, name, 4096)
+    L = mok.lib()
+    arr = (ctypes.c_void_p * 2)(4096, 8192)
+    full = mok.MxWeights(4096, 4096, 4096, 4096, 4096, 4096)
+    pack = ctypes.cast(ctypes.byref(full), ctypes.c_void_p)
+    o = mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT, mxfp8=True)
+    rc = L.mok_moe_forward(arr, 128, 128, pack, None, None, ctypes.byref(p), 256, ctypes.byref(o), 256, 1 << 30,
+                           arr, None)
+    assert rc == mok.MOK_ERR_UNSUPPORTED and "MXFP8" in mok.last_error()
+    o = mok.fwd_opts(mode=mok.MOK_MODE_STAGED, mxfp8=True)
+    holed = mok.MxWeights(4096, 4096, 4096, 0, 4096, 4096)
+    rc = L.mok_moe_forward(arr, 128, 128, ctypes.cast(ctypes.byref(holed), ctypes.c_void_p), None, None,
+                           ctypes.byref(p), 0, ctypes.byref(o), 256, 1 << 30, arr, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG and "NULL" in mok.last_error()
+    rc = L.mok_moe_forward(arr, 128, 128, None, None, None, ctypes.byref(p), 0, ctypes.byref(o), 256, 1 << 30,
+                           arr, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG
+
+
 def test_get_status_argument_checks():
     L = mok.lib()
     rc = L.mok_get_status(None, 0, None, None)
