@@ -29,7 +29,6 @@ import signal
 import statistics
 import subprocess
 import sys
-import tempfile
 import time
 
 import torch
@@ -53,27 +52,53 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling during the timed region.
+
+    The sampler is started first and the timed region begins only after its
+    first line has appeared; each line carries the host time it was read at,
+    and only lines read between ``mark_start()`` and ``mark_stop()`` count."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 100
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = None
+        self.lines = []          # (host time, csv line)
+        self.t0 = self.t1 = None
+        self.reader = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line))
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(prefix="mok_clocks_", suffix=".csv")
-            os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", str(self.PERIOD_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True,
+                bufsize=1)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        deadline = time.time() + 10.0
+        while not self.lines and time.time() < deadline and self.proc.poll() is None:
+            time.sleep(0.01)
         return self
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_stop(self):
+        self.t1 = time.time()
+        if self.proc is not None:
+            # one more period so the last part of the region is sampled
+            time.sleep(self.PERIOD_MS / 1e3 * 1.5)
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -82,30 +107,33 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            self.reader.join(timeout=5)
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
+        if self.proc is None or self.t0 is None:
             return None
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [s.strip() for s in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        os.unlink(self.path)
+        # a line read at time t describes the GPU within one period before t
+        lo, hi = self.t0, self.t1 + self.PERIOD_MS / 1e3
+        for t, line in self.lines:
+            if not (lo <= t <= hi):
+                continue
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "period_ms": self.PERIOD_MS}
 
 
 # ------------------------------------------------------------------ workload
@@ -209,11 +237,13 @@ def run_mok(args, cfg, rank, world, device):
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                       else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])) as clk:
+        clk.mark_start()
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         stop.record(stream)
         torch.cuda.synchronize()
+        clk.mark_stop()
     if world > 1:
         torch.distributed.barrier()
     total_ms = start.elapsed_time(stop)
@@ -296,7 +326,7 @@ def cpu_oracle_sample(cfg, budget_s: float = 12.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mok", choices=["mok", "reference"])
     ap.add_argument("--config", default="page", choices=list(mokgen.CONFIGS))
@@ -316,7 +346,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    metric = "MoE fwd tokens/s (H7168/I2048)"
+    # value is tokens/s; the tensor-core fraction and the gather/combine GB/s
+    # of the same metric are in "roofline" and "phase_rates"
+    metric = "MoE fwd tokens/s (H7168/I2048); % BF16 TC peak; gather/combine HBM GB/s"
     wdesc = ("MXFP8 E4M3 weights + E8M0 scales per 32 along K (quantised once, untimed)" if cfg.mxfp8
              else "bf16 weights [E,H,I]/[E,I,H]")
     config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
@@ -357,7 +389,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "mxfp8-e4m3 (bf16 MMA)" if cfg.mxfp8 else "bf16",
             "data": "synthetic", "config": config}
-    if args.mode == "staged":
+    if len(ph) == 4:
         t_plan, t_gather, t_gemm, t_comb = ph
         gemm_s = t_gemm / 1e3
         tflops = work["gemm_flops"] / gemm_s / 1e12

@@ -91,7 +91,7 @@ bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t 
 
 bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint64_t rows, const char** err) {
     for (int i = 0; i < B_MAPS; ++i)
-        if (!encode_tmap_2d_16b(&maps->m[i], bf16, base, inner, rows, 64, (uint32_t)(B_MAX_BOX >> i), err))
+        if (!encode_tmap_2d_16b(&maps->m[i], bf16, base, inner, rows, 64, (uint32_t)(16 * (i + 1)), err))
             return false;
     return true;
 }

@@ -35,10 +35,10 @@
 // one of two 256-column accumulators, warps 2-5 drain the other accumulator
 // (tcgen05.ld) through shared memory to global memory, and (MXFP8 only)
 // warps 6-9 convert weight tiles.  The token tile of a stage is ONE TMA box
-// of the next power of two of the 16-rounded row count, and a down unit's
-// two 64-column weight halves come from one 3D map: measured on B200, the
-// number of TMA ops per SM (not bytes) limits this kernel.  Every wait is
-// bounded.
+// of exactly the 16-rounded row count, and a down unit's two 64-column
+// weight halves come from one 3D map.  Measured on B200: the number of TMA
+// ops per SM, and then the bytes each SM takes in from L2 (about 64 B per
+// clock), limit this kernel.  Every wait is bounded.
 //
 // A schedule policy (template parameter) tells each role which units this
 // CTA runs, what a unit's inputs wait for, and what its completion signals.
@@ -65,14 +65,16 @@ constexpr uint64_t DRAIN_TIMEOUT_NS = 1000000000ull;
 constexpr int MT_G_FEATURES = 64;                 // gate/up unit: 64 gate + 64 up columns
 constexpr int MT_D_FEATURES = 128;                // down unit: 128 output columns
 
-// Stage layouts.  bf16 path: [A 16 KB][B 32 KB] x 4.  MXFP8 path:
-// [A bf16, converted 16 KB][B 32 KB][A E4M3 bytes 8 KB][scales 1 KB] x 3.
+// Stage layouts.  bf16 path: [A0 16 KB][A1 16 KB][B 32 KB] x 3 (a unit is
+// a pair of M tiles that share the token tile).  MXFP8 path: [A bf16,
+// converted 16 KB][B 32 KB][A E4M3 bytes 8 KB][scales 1 KB] x 3.
 struct Bf16Cfg {
     static constexpr bool MX = false;
+    static constexpr int SUB = 2;  // M tiles per unit
     static constexpr int THREADS = 192;
-    static constexpr int NST = 4;
-    static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int A_OFF = 0, B_OFF = A_BYTES;
+    static constexpr int NST = 3;
+    static constexpr int STAGE = SUB * A_BYTES + B_BYTES;
+    static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
     static constexpr int EPI_OFF = NST * STAGE;
     static constexpr int XCH_OFF = EPI_OFF + EPI_BYTES;  // unused
     static constexpr int BAR_OFF = XCH_OFF;
@@ -80,6 +82,7 @@ struct Bf16Cfg {
 };
 struct MxCfg {
     static constexpr bool MX = true;
+    static constexpr int SUB = 1;
     static constexpr int THREADS = 320;
     static constexpr int NST = 3;
     static constexpr int A_OFF = 0, B_OFF = A_BYTES;
@@ -97,13 +100,14 @@ constexpr int GEMM_THREADS = Bf16Cfg::THREADS;
 constexpr int SMEM_BAR_OFF = Bf16Cfg::BAR_OFF;
 constexpr int SMEM_ALLOC = Bf16Cfg::SMEM;
 
-// One unit of work: an M tile of one phase over one chunk.
+// One unit of work: C::SUB consecutive M tiles (fewer at the end of the M
+// range) of one phase over one chunk; the tiles share every token tile.
 struct Unit {
     int phase;   // 0 = gate/up, 1 = down
     int expert;
     int brow0;   // buffer row of the chunk's first row (token rows and h rows)
     int rows;    // valid rows, 1..256
-    int m;       // M tile index
+    int m;       // unit index along M: first M tile = m * C::SUB
     int grow0;   // global expert-major row of the chunk's first row (row_slot index)
     int chunk;
     int mb;
@@ -158,14 +162,19 @@ struct StagedSched {
     __device__ void unit_done(const Unit&) const {}
 };
 
-// Token tile of a unit: one box of the next power of two >= the 16-rounded
-// row count.  Returns the map index (box rows = B_MAX_BOX >> index).
-__device__ __forceinline__ int token_box(int rows) {
-    const int r16 = (rows + 15) & ~15;
-    int bx = 0;
-    while (bx + 1 < B_MAPS && (B_MAX_BOX >> (bx + 1)) >= r16) ++bx;
-    return bx;
+// M tiles of a phase (64 gate + 64 up features, or 128 down features, each),
+// and how many of them unit u covers.
+__device__ __forceinline__ int phase_tiles(const CoreArgs& a, int phase) {
+    return phase == 0 ? a.I / MT_G_FEATURES : a.H / MT_D_FEATURES;
 }
+template <class C>
+__device__ __forceinline__ int unit_subs(const CoreArgs& a, const Unit& u) {
+    return min(C::SUB, phase_tiles(a, u.phase) - u.m * C::SUB);
+}
+
+// Token tile of a unit: one box of the 16-rounded row count.  Returns the
+// map index (box rows = 16 * (index + 1)); rows is 1..256.
+__device__ __forceinline__ int token_box(int rows) { return ((rows + 15) >> 4) - 1; }
 
 // ------------------------------------------------------------------ producer
 // Loads the weight tile (bf16/fp16 halves, or MXFP8 bytes + scales) and the
@@ -184,11 +193,12 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
         const int KB = K / BK;
         const BMaps& bm = u.phase == 0 ? maps.rows : maps.h;
         const int bx = token_box(u.rows);
-        uint32_t bytes = (uint32_t)(B_MAX_BOX >> bx) * B_ROW_BYTES;
+        const int nsub = unit_subs<C>(a, u);
+        uint32_t bytes = (uint32_t)(16 * (bx + 1)) * B_ROW_BYTES;
         if (C::MX)
             bytes += u.phase == 0 ? 2 * (4096 + 128) : (8192 + 256);  // E4M3 bytes + scale bytes
         else
-            bytes += A_BYTES;
+            bytes += (uint32_t)nsub * A_BYTES;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 10)) {
@@ -212,18 +222,21 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
                     tma_load_2d(sc, &mx->ds, &full[stage], u.m * MT_D_FEATURES, kys);
                 }
             } else {
-                unsigned char* sa = st + C::A_OFF;
-                if (u.phase == 0) {
-                    tma_load_2d_hint(sa, &maps.wg, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
-                    tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], u.m * MT_G_FEATURES, ky,
-                                     evict_first);
-                } else if (maps.has_wd3) {
-                    // both 64-column halves of the 128-column down tile in one op
-                    tma_load_3d_hint(sa, &maps.wd3, &full[stage], 0, ky, u.m * 2, evict_first);
-                } else {
-                    tma_load_2d_hint(sa, &maps.wd, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
-                    tma_load_2d_hint(sa + A_BYTES / 2, &maps.wd, &full[stage], u.m * MT_D_FEATURES + 64, ky,
-                                     evict_first);
+                for (int sub = 0; sub < nsub; ++sub) {
+                    unsigned char* sa = st + C::A_OFF + sub * A_BYTES;
+                    const int mt = u.m * C::SUB + sub;
+                    if (u.phase == 0) {
+                        tma_load_2d_hint(sa, &maps.wg, &full[stage], mt * MT_G_FEATURES, ky, evict_first);
+                        tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], mt * MT_G_FEATURES, ky,
+                                         evict_first);
+                    } else if (maps.has_wd3) {
+                        // both 64-column halves of the 128-column down tile in one op
+                        tma_load_3d_hint(sa, &maps.wd3, &full[stage], 0, ky, mt * 2, evict_first);
+                    } else {
+                        tma_load_2d_hint(sa, &maps.wd, &full[stage], mt * MT_D_FEATURES, ky, evict_first);
+                        tma_load_2d_hint(sa + A_BYTES / 2, &maps.wd, &full[stage], mt * MT_D_FEATURES + 64, ky,
+                                         evict_first);
+                    }
                 }
             }
             tma_load_2d(st + C::B_OFF, &bm.m[bx], &full[stage], kb * BK, u.brow0);
@@ -306,6 +319,17 @@ __device__ __forceinline__ void gemm_converter(const CoreArgs& a, const S& s, un
     }
 }
 
+// ------------------------------------------------------------------ TMEM placement
+// TMEM holds two 256-column accumulator buffers used in ring order; each use
+// is a "ticket" (buffer = ticket & 1, barrier parity = (ticket >> 1) & 1).
+// A unit whose M tiles fit in one buffer (one tile, or two tiles of N <= 128
+// columns: tile s at column 128 s) takes one ticket; two tiles of N > 128
+// take two consecutive tickets, one buffer each.
+__device__ __forceinline__ int unit_tickets(int nsub, int N) { return (nsub == 2 && N > 128) ? 2 : 1; }
+__device__ __forceinline__ uint32_t acc_col(uint32_t tk, int sub, bool wide) {
+    return wide ? ((tk + (uint32_t)sub) & 1u) * ACC_COLS : (tk & 1u) * ACC_COLS + (uint32_t)sub * 128u;
+}
+
 // ------------------------------------------------------------------ MMA issuer
 // ready[stage]: the TMA barrier (bf16) or the converter barrier (MXFP8).
 template <class S, class C>
@@ -314,19 +338,24 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
                                          uint32_t tmem_base) {
     int stage = 0;
     uint32_t phase = 0;
-    int tb = 0;
-    uint32_t tph = 0;
+    uint32_t tk = 0;  // next accumulator ticket
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
         const int KB = (u.phase == 0 ? a.H : a.I) / BK;
         const int N = (u.rows + 15) & ~15;
+        const int nsub = unit_subs<C>(a, u);
+        const int nt = unit_tickets(nsub, N);
+        const bool wide = nt == 2;
         // bf16 path: gate/up bf16 x bf16, down fp16 x fp16; MXFP8 path: bf16 x bf16
         const uint32_t idesc =
             umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, (C::MX || u.phase == 0) ? 1 : 0);
-        if (!mbar_wait(&tempty[tb], tph ^ 1u, a.st, a.timeout_ns, 20)) break;
-        tc_fence_after();
-        const uint32_t dt = tmem_base + (uint32_t)(tb * ACC_COLS);
         bool ok = true;
+        for (int t = 0; t < nt && ok; ++t) {
+            const uint32_t tkt = tk + (uint32_t)t;
+            ok = mbar_wait(&tempty[tkt & 1u], ((tkt >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 20);
+        }
+        if (!ok) break;
+        tc_fence_after();
         for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&ready[stage], phase, a.st, a.timeout_ns, 21)) {
                 ok = false;
@@ -337,12 +366,17 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
             const uint32_t sb = smem_u32(smem + stage * C::STAGE + C::B_OFF);
 #pragma unroll
             for (int ks = 0; ks < BK / 16; ++ks) {
-                // A: MN-major SW128, 16 K rows per MMA = 2 atoms of 1 KB; the
-                //    two 64-wide MN halves are 8 KB apart (LBO).
-                const uint64_t ad = umma_desc_sw128(sa + ks * 2048, A_BYTES / 2, 1024);
                 // B: K-major SW128, 16 K = 32 bytes inside the atom; 8-row groups 1 KB apart.
                 const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
-                umma_bf16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+#pragma unroll
+                for (int sub = 0; sub < C::SUB; ++sub) {
+                    if (sub < nsub) {
+                        // A: MN-major SW128, 16 K rows per MMA = 2 atoms of 1 KB;
+                        //    the two 64-wide MN halves are 8 KB apart (LBO).
+                        const uint64_t ad = umma_desc_sw128(sa + sub * A_BYTES + ks * 2048, A_BYTES / 2, 1024);
+                        umma_bf16(tmem_base + acc_col(tk, sub, wide), ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                    }
+                }
             }
             umma_commit(&empty[stage]);
             if (++stage == C::NST) {
@@ -351,11 +385,8 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
             }
         }
         if (!ok) break;
-        umma_commit(&tfull[tb]);
-        if (++tb == 2) {
-            tb = 0;
-            tph ^= 1u;
-        }
+        for (int t = 0; t < nt; ++t) umma_commit(&tfull[(tk + (uint32_t)t) & 1u]);
+        tk += (uint32_t)nt;
     }
     // wait for every MMA this thread issued before TMEM is released
     umma_commit(fin);
@@ -363,92 +394,112 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
 }
 
 // ------------------------------------------------------------------ epilogue (warps 2..5)
-template <class S, class C>
-__device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* tfull,
-                                              uint64_t* tempty, volatile int* ok_flag, uint32_t tmem_base) {
+// Drains one M tile's accumulator (TMEM columns col0 .. col0 + rows) through
+// shared memory: SwiGLU -> h rows (gate/up) or fp32 rows pushed to the
+// tokens' slots (down).
+template <class C>
+__device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u, int mt, uint32_t col0, float* epi,
+                                               float* xch, uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
     const int et = threadIdx.x - 64;  // 0..127
     const int tok = et & 31, fq = et >> 5;
+    const int ncc = (u.rows + 31) >> 5;
+    for (int cc = 0; cc < ncc; ++cc) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + col0 + (uint32_t)(cc * 32), v);
+        float* myrow = epi + (q * 32 + lane) * EPI_LD;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) myrow[k] = v[k];
+        named_bar_sync(1, 128);
+        const int col = cc * 32 + tok;
+        const bool live = col < u.rows;
+        if (u.phase == 0) {
+            // features mt*64 + fq*16 .. +15: gate rows fq*16+k, up rows 64+fq*16+k
+            float hv[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float g = epi[(fq * 16 + k) * EPI_LD + tok];
+                const float up = epi[(64 + fq * 16 + k) * EPI_LD + tok];
+                hv[k] = g / (1.0f + __expf(-g)) * up;
+            }
+            uint32_t pk[8];
+            if constexpr (C::MX) {
+                // MXFP8 h: blocks of 32 features = thread pairs fq ^ 1 (same token)
+                float amax = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(hv[k]));
+                xch[fq * 32 + tok] = amax;
+                named_bar_sync(1, 128);
+                amax = fmaxf(amax, xch[(fq ^ 1) * 32 + tok]);
+                const int sx = mx_block_exponent(amax);
+                const float inv = mx_pow2(-sx), scl = mx_pow2(sx);
+#pragma unroll
+                for (int k = 0; k < 16; k += 2) {
+                    const float2 d = mx_e4m3x2_to_float2(mx_e4m3x2(hv[k] * inv, hv[k + 1] * inv));
+                    pk[k >> 1] = pack_bf16x2(d.x * scl, d.y * scl);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; k += 2) pk[k >> 1] = pack_half2_sat(hv[k], hv[k + 1]);
+            }
+            if (live) {
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) +
+                                                      (size_t)(u.brow0 + col) * a.I + mt * MT_G_FEATURES + fq * 16);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+        } else if (live) {
+            // fp32 push to the token's slot; the combine rounds y once
+            const int slot = __ldg(a.row_slot + u.grow0 + col);
+            float4* dst = reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + mt * MT_D_FEATURES + fq * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+                const int f = fq * 32 + q4 * 4;
+                dst[q4] = make_float4(epi[f * EPI_LD + tok], epi[(f + 1) * EPI_LD + tok],
+                                      epi[(f + 2) * EPI_LD + tok], epi[(f + 3) * EPI_LD + tok]);
+            }
+        }
+        named_bar_sync(1, 128);
+    }
+}
+
+template <class S, class C>
+__device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* tfull,
+                                              uint64_t* tempty, volatile int* ok_flag, uint32_t tmem_base) {
+    const int lane = threadIdx.x & 31;
+    const int et = threadIdx.x - 64;  // 0..127
     float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF);
     float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);  // [4][32] block maxima (MXFP8)
-    int tb = 0;
-    uint32_t tph = 0;
+    uint32_t tk = 0;  // next accumulator ticket (the MMA issuer's sequence)
+    bool ok = true;
     Unit u;
-    for (int i = 0; s.get(i, u); ++i) {
-        // one thread waits, all 128 leave together on failure
-        if (et == 0) *ok_flag = mbar_wait(&tfull[tb], tph, a.st, a.timeout_ns, 30) ? 1 : 0;
-        named_bar_sync(1, 128);
-        const int ok = *ok_flag;
-        named_bar_sync(1, 128);
-        if (!ok) break;
-        tc_fence_after();
-        const int ncc = (u.rows + 31) >> 5;
-        for (int cc = 0; cc < ncc; ++cc) {
-            float v[32];
-            tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(tb * ACC_COLS + cc * 32), v);
-            float* myrow = epi + (q * 32 + lane) * EPI_LD;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) myrow[k] = v[k];
-            named_bar_sync(1, 128);
-            const int col = cc * 32 + tok;
-            const bool live = col < u.rows;
-            if (u.phase == 0) {
-                // features m*64 + fq*16 .. +15: gate rows fq*16+k, up rows 64+fq*16+k
-                float hv[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float g = epi[(fq * 16 + k) * EPI_LD + tok];
-                    const float up = epi[(64 + fq * 16 + k) * EPI_LD + tok];
-                    hv[k] = g / (1.0f + __expf(-g)) * up;
-                }
-                uint32_t pk[8];
-                if constexpr (C::MX) {
-                    // MXFP8 h: blocks of 32 features = thread pairs fq ^ 1 (same token)
-                    float amax = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(hv[k]));
-                    xch[fq * 32 + tok] = amax;
-                    named_bar_sync(1, 128);
-                    amax = fmaxf(amax, xch[(fq ^ 1) * 32 + tok]);
-                    const int sx = mx_block_exponent(amax);
-                    const float inv = mx_pow2(-sx), scl = mx_pow2(sx);
-#pragma unroll
-                    for (int k = 0; k < 16; k += 2) {
-                        const float2 d = mx_e4m3x2_to_float2(mx_e4m3x2(hv[k] * inv, hv[k + 1] * inv));
-                        pk[k >> 1] = pack_bf16x2(d.x * scl, d.y * scl);
-                    }
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 16; k += 2) pk[k >> 1] = pack_half2_sat(hv[k], hv[k + 1]);
-                }
-                if (live) {
-                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) +
-                                                          (size_t)(u.brow0 + col) * a.I + u.m * MT_G_FEATURES +
-                                                          fq * 16);
-                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                }
-            } else if (live) {
-                // fp32 push to the token's slot; the combine rounds y once
-                const int slot = __ldg(a.row_slot + u.grow0 + col);
-                float4* dst = reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + u.m * MT_D_FEATURES + fq * 32);
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    const int f = fq * 32 + q4 * 4;
-                    dst[q4] = make_float4(epi[f * EPI_LD + tok], epi[(f + 1) * EPI_LD + tok],
-                                          epi[(f + 2) * EPI_LD + tok], epi[(f + 3) * EPI_LD + tok]);
-                }
+    for (int i = 0; ok && s.get(i, u); ++i) {
+        const int nsub = unit_subs<C>(a, u);
+        const int nt = unit_tickets(nsub, (u.rows + 15) & ~15);
+        const bool wide = nt == 2;
+        for (int sub = 0; sub < nsub && ok; ++sub) {
+            const uint32_t tkt = wide ? tk + (uint32_t)sub : tk;
+            if (sub == 0 || wide) {
+                // one thread waits, all 128 leave together on failure
+                if (et == 0)
+                    *ok_flag = mbar_wait(&tfull[tkt & 1u], (tkt >> 1) & 1u, a.st, a.timeout_ns, 30) ? 1 : 0;
+                named_bar_sync(1, 128);
+                ok = *ok_flag != 0;
+                named_bar_sync(1, 128);
+                if (!ok) break;
+                tc_fence_after();
             }
-            named_bar_sync(1, 128);
+            epi_drain_tile<C>(a, u, u.m * C::SUB + sub, acc_col(tk, sub, wide), epi, xch, tmem_base);
+            if (wide || sub == nsub - 1) {
+                // this buffer is drained: the MMA issuer may reuse it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[tkt & 1u]);
+            }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[tb]);
-        if (++tb == 2) {
-            tb = 0;
-            tph ^= 1u;
-        }
+        if (!ok) break;
+        tk += (uint32_t)nt;
         if (S::kSignals) {
             // h rows are read next by TMA (async proxy) in some CTA: make this
             // thread's stores visible to that proxy, then publish once.

@@ -58,7 +58,9 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.row_slot = row_slot;
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
-    const int MT = phase == 0 ? sh.I / MT_G_FEATURES : sh.H / MT_D_FEATURES;
+    const int tiles = phase == 0 ? sh.I / MT_G_FEATURES : sh.H / MT_D_FEATURES;
+    const int sub = mx ? MxCfg::SUB : Bf16Cfg::SUB;
+    const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
     if (mx) {
         k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,

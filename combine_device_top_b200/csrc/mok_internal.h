@@ -72,10 +72,10 @@ struct GemmTuning {
 GemmTuning gemm_tuning();  // defaults, overridable by MOK_GEMM_GROUP
 size_t gemm_smem_bytes();
 cudaError_t gemm_configure(int dev);
-// Token-side (B operand) tensor maps of one buffer with box heights
-// 256, 128, 64, 32, 16 rows: a chunk of r rows (rounded up to 16) is loaded
-// as one box per set bit of r.
-constexpr int B_MAPS = 5;
+// Token-side (B operand) tensor maps of one buffer with box heights 16, 32,
+// ..., 256 rows (map i has 16 * (i + 1) rows): a chunk of r rows is loaded
+// as ONE box of r rounded up to 16.
+constexpr int B_MAPS = 16;
 constexpr int B_MAX_BOX = 256;
 struct BMaps {
     CUtensorMap m[B_MAPS];

@@ -19,7 +19,7 @@
 //                of every minibatch in order -- gate/up units of b, then its
 //                down units -- dealt round-robin.  A gate/up unit waits for
 //                gathered[b] == D; a down unit waits for its chunk's gate/up
-//                units (g_done[c] == I/64); completions are published with
+//                units (g_done[c] == their count); completions are published with
 //                release atomics.
 //   all CTAs     after every down unit is done: the fixed-order combine.
 // Dependencies only point to lower unit indices (or to the dispatch side,
@@ -43,7 +43,7 @@ struct PersistParams {
     const Minibatch* mbs;
     const int* counts2;  // [0] chunks, [1] minibatches
     int cap;             // rows per ring half
-    int MTG, MTD;        // M tiles per chunk of the gate/up and down phases
+    int MTG, MTD;        // units (groups of Bf16Cfg::SUB M tiles) per chunk of the gate/up and down phases
     int dispatch_ctas;
     // counters (zeroed before the launch)
     int* gathered;  // [max_mb]  dispatch CTAs done with minibatch b
@@ -253,8 +253,9 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.mbs = L.mbs;
     p.counts2 = L.counts2;
     p.cap = L.cap;
-    p.MTG = L.I / MT_G_FEATURES;
-    p.MTD = L.H / MT_D_FEATURES;
+    // units per chunk: pairs of M tiles (the last one may be single)
+    p.MTG = (L.I / MT_G_FEATURES + Bf16Cfg::SUB - 1) / Bf16Cfg::SUB;
+    p.MTD = (L.H / MT_D_FEATURES + Bf16Cfg::SUB - 1) / Bf16Cfg::SUB;
     p.dispatch_ctas = L.dispatch_ctas;
     p.gathered = L.gathered;
     p.d_done = L.d_done;
