@@ -241,7 +241,7 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
     if (!encode_gemm_maps(&maps, wg, wu, wd, rows, h, H, I, E, n_rows_buf, &err))
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
     GemmShape sh{H, I, E};
-    const GemmTuning tune = gemm_tuning();
+    const GemmTuning tune = gemm_tuning(n_rows_buf, E);
     const MxMaps* mxp = mxw ? &mx : nullptr;
     MOK_CUDA(launch_gemm_phase(0, maps, mxp, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune,
                                stream),

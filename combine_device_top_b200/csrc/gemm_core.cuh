@@ -65,14 +65,16 @@ constexpr uint64_t DRAIN_TIMEOUT_NS = 1000000000ull;
 constexpr int MT_G_FEATURES = 64;                 // gate/up unit: 64 gate + 64 up columns
 constexpr int MT_D_FEATURES = 128;                // down unit: 128 output columns
 
-// Stage layouts.  bf16 path: [A0 16 KB][A1 16 KB][B 32 KB] x 3 (a unit is
-// a pair of M tiles that share the token tile).  MXFP8 path: [A bf16,
-// converted 16 KB][B 32 KB][A E4M3 bytes 8 KB][scales 1 KB] x 3.
-struct Bf16Cfg {
+// Stage layouts.  bf16 path, one M tile per unit: [A 16 KB][B 32 KB] x 4.
+// bf16 path, pairs of M tiles sharing the token tile: [A0 16 KB][A1 16 KB]
+// [B 32 KB] x 3.  MXFP8 path: [A bf16, converted 16 KB][B 32 KB][A E4M3
+// bytes 8 KB][scales 1 KB] x 3.
+template <int SUB_, int NST_>
+struct Bf16CfgT {
     static constexpr bool MX = false;
-    static constexpr int SUB = 2;  // M tiles per unit
+    static constexpr int SUB = SUB_;  // M tiles per unit
     static constexpr int THREADS = 192;
-    static constexpr int NST = 3;
+    static constexpr int NST = NST_;
     static constexpr int STAGE = SUB * A_BYTES + B_BYTES;
     static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
     static constexpr int EPI_OFF = NST * STAGE;
@@ -80,6 +82,9 @@ struct Bf16Cfg {
     static constexpr int BAR_OFF = XCH_OFF;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + slack for 1024-byte alignment
 };
+using Bf16Cfg = Bf16CfgT<1, 4>;
+using Bf16PairCfg = Bf16CfgT<2, 3>;
+static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share the barrier offset");
 struct MxCfg {
     static constexpr bool MX = true;
     static constexpr int SUB = 1;

@@ -26,11 +26,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 size_t gemm_smem_bytes() { return SMEM_ALLOC; }
 
 // Defaults measured on B200 (page shape and a 512-rows-per-expert case):
-// small raster groups paid.  MOK_GEMM_GROUP overrides the group size (a
-// tuning knob only: results do not change).
-GemmTuning gemm_tuning() {
-    GemmTuning v{2};
+// small raster groups paid.  Pairs of M tiles halve the token-tile bytes
+// each SM takes in per weight byte, but a pair of chunks taller than 128 rows
+// fills TMEM, so its epilogue no longer overlaps the next unit's MMAs: pairs
+// paid at about 171 rows per expert and cost at 512 (measured), so they are
+// used when the mean rows per expert is at most 192.  MOK_GEMM_GROUP and
+// MOK_GEMM_PAIR (0/1) override (tuning knobs only: results do not change).
+GemmTuning gemm_tuning(int rows, int E) {
+    GemmTuning v{2, rows <= 192 * E ? 1 : 0};
     if (const char* s = getenv("MOK_GEMM_GROUP")) v.group_chunks = atoi(s) < 1 ? 1 : atoi(s);
+    if (const char* s = getenv("MOK_GEMM_PAIR")) v.pair = atoi(s) != 0;
     return v;
 }
 
@@ -40,6 +45,9 @@ cudaError_t gemm_configure(int dev) {
     if (done[dev]) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<Bf16Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Bf16Cfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm<Bf16PairCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Bf16PairCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm<MxCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, MxCfg::SMEM);
     if (e == cudaSuccess) done[dev] = true;
@@ -59,7 +67,7 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
     const int tiles = phase == 0 ? sh.I / MT_G_FEATURES : sh.H / MT_D_FEATURES;
-    const int sub = mx ? MxCfg::SUB : Bf16Cfg::SUB;
+    const int sub = mx ? MxCfg::SUB : tune.pair ? Bf16PairCfg::SUB : Bf16Cfg::SUB;
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
     if (mx) {
@@ -68,8 +76,12 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     } else {
         MxMaps none;
         memset(&none, 0, sizeof none);
-        k_grouped_gemm<Bf16Cfg><<<grid, Bf16Cfg::THREADS, Bf16Cfg::SMEM, stream>>>(maps, none, a, chunks, counts2,
-                                                                                  phase, MT, GC);
+        if (tune.pair)
+            k_grouped_gemm<Bf16PairCfg><<<grid, Bf16PairCfg::THREADS, Bf16PairCfg::SMEM, stream>>>(
+                maps, none, a, chunks, counts2, phase, MT, GC);
+        else
+            k_grouped_gemm<Bf16Cfg><<<grid, Bf16Cfg::THREADS, Bf16Cfg::SMEM, stream>>>(maps, none, a, chunks,
+                                                                                      counts2, phase, MT, GC);
     }
     return cudaGetLastError();
 }

@@ -55,11 +55,15 @@ struct Minibatch {
     int row0, row1, chunk0, chunk1;
 };
 constexpr int CHUNK_MAX_ROWS = 256;
+// MXFP8 path: two accumulators of <= 224 columns leave TMEM room for the
+// block scale factors.
+constexpr int CHUNK_MAX_ROWS_MX = 224;
 
 int max_chunks(int n_slots, int E, int n_mb);
 int max_minibatches(int n_slots, int minibatch);
-cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int minibatch, int cap, Chunk* chunks,
-                                int max_chunks, Minibatch* mbs, int max_mb, int* counts2, void* status,
+// max_rows: chunk height cap, CHUNK_MAX_ROWS or CHUNK_MAX_ROWS_MX
+cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int minibatch, int cap, int max_rows,
+                                Chunk* chunks, int max_chunks, Minibatch* mbs, int max_mb, int* counts2, void* status,
                                 cudaStream_t stream);
 
 // ---- the grouped GEMM (tcgen05)
@@ -68,8 +72,11 @@ struct GemmShape {
 };
 struct GemmTuning {
     int group_chunks;  // raster group size in chunks
+    int pair;          // 1: units of two M tiles sharing each token tile (bf16 path)
 };
-GemmTuning gemm_tuning();  // defaults, overridable by MOK_GEMM_GROUP
+// defaults for `rows` expert-major rows over E experts, overridable by
+// MOK_GEMM_GROUP / MOK_GEMM_PAIR
+GemmTuning gemm_tuning(int rows, int E);
 size_t gemm_smem_bytes();
 cudaError_t gemm_configure(int dev);
 // Token-side (B operand) tensor maps of one buffer with box heights 16, 32,

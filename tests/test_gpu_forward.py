@@ -83,6 +83,27 @@ def test_grouped_gemm_swiglu_matches_oracle(name):
     assert_bf16_close(out.cpu(), want, name)
 
 
+@pytest.mark.parametrize("name", ["multi_chunk", "many_experts", "tiny"])
+def test_grouped_gemm_m_tile_pairing_is_exact(name, monkeypatch):
+    """Units of one M tile and units of two M tiles sharing each token tile
+    (with 1 or 2 TMEM buffers per unit, and a single tile at an odd end of
+    the M range) compute every output with the same MMA sequence: results
+    are bit-identical, and both match the oracle."""
+    case = Case(FFN_CASES[name])
+    cfg = case.cfg
+    p = mok.plan(case.dlogits, cfg.k, cfg.R)
+    rows = mok.gather(case.x_shards(), p)
+    got = {}
+    for pair in ("0", "1"):
+        monkeypatch.setenv("MOK_GEMM_PAIR", pair)
+        out, ws = mok.expert_ffn(rows, case.dwg, case.dwu, case.dwd, p)
+        assert mok.get_status(ws) == mok.MOK_OK
+        got[pair] = out.cpu()
+    assert torch.equal(got["0"], got["1"])
+    want, _, _ = _oracle_slots(case, p)
+    assert_bf16_close(got["1"], want, name)
+
+
 def test_grouped_gemm_single_expert_vs_torch_fp32():
     """E = 1, k = 1: the grouped GEMM is a dense SwiGLU FFN; compare with a
     plain PyTorch fp32 reference of the same op on the GPU."""
