@@ -364,8 +364,8 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     }
     const int ns = T * k;
     MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
-    MOK_CUDA(launch_build_chunks(plan->offsets, E, ns, L.minibatch, L.cap, chunks, L.max_chunks, mbs, L.max_mb,
-                                 counts2, status, stream),
+    MOK_CUDA(launch_build_chunks(plan->offsets, E, ns, L.minibatch, L.cap, mxw ? CHUNK_MAX_ROWS_MX : CHUNK_MAX_ROWS,
+                                 chunks, L.max_chunks, mbs, L.max_mb, counts2, status, stream),
              "work list launch");
     if (mode == MOK_MODE_PERSISTENT) {
         int dev = 0;
@@ -530,7 +530,8 @@ int mok_expert_ffn(const void* rows, int H, int I, const void* w_gate, const voi
     off += align256(sizeof(Minibatch) * (size_t)mb);
     void* h = base + off;
     MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
-    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, chunks, mc, mbs, mb, counts2, status, stream),
+    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, CHUNK_MAX_ROWS, chunks, mc, mbs, mb, counts2,
+                                 status, stream),
              "work list launch");
     return run_expert_ffn(rows, ns, H, I, w_gate, w_up, w_down, plan->E, plan->row_slot, chunks, counts2, h, out,
                           status, kDefaultTimeoutNs, stream);

@@ -1,6 +1,6 @@
 // worklist.cu -- the device-built work list of the grouped GEMM: minibatch
-// boundaries over the expert-major rows and chunks of <= 256 rows of one
-// expert inside one minibatch.  Built from `offsets` on the device, so the
+// boundaries over the expert-major rows and chunks of at most max_rows (256,
+// or 224 on the MXFP8 path) rows of one expert inside one minibatch.  Built from `offsets` on the device, so the
 // forward needs no host round trip (MoK wiki summary, key points: schedule
 // built on the device without CPU-GPU traffic; MoK article, minibatch
 // paragraph: a minibatch is the unit handed to the expert computation).
@@ -12,18 +12,19 @@ namespace mok {
 // ------------------------------------------------------------------ work list
 // One block.  Minibatch boundaries: from row b0, the first expert boundary at
 // or after b0 + minibatch, but never more than `cap` rows; then every
-// (expert, minibatch) piece is cut into ceil(len / 256) chunks of nearly
-// equal size (multiples of 16 rows except the last).
-__device__ __forceinline__ int piece_chunks(int L) { return (L + CHUNK_MAX_ROWS - 1) / CHUNK_MAX_ROWS; }
-__device__ __forceinline__ int piece_base(int L) {
-    const int n = piece_chunks(L);
+// (expert, minibatch) piece is cut into ceil(len / maxr) chunks of nearly
+// equal size (multiples of 16 rows except the last; maxr is a multiple of 16).
+__device__ __forceinline__ int piece_chunks(int L, int maxr) { return (L + maxr - 1) / maxr; }
+__device__ __forceinline__ int piece_base(int L, int maxr) {
+    const int n = piece_chunks(L, maxr);
     int base = (((L + n - 1) / n) + 15) & ~15;
-    if ((n - 1) * base >= L) base = CHUNK_MAX_ROWS;
+    if ((n - 1) * base >= L) base = maxr;
     return base;
 }
 
 __global__ void __launch_bounds__(1024) k_build_chunks(const int32_t* __restrict__ offsets, int E, int n_slots,
-                                                       int M, int cap, Chunk* __restrict__ chunks, int max_chunks,
+                                                       int M, int cap, int maxr, Chunk* __restrict__ chunks,
+                                                       int max_chunks,
                                                        Minibatch* __restrict__ mbs, int max_mb,
                                                        int* __restrict__ counts2, DevStatus* st) {
     __shared__ int s_nmb;
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(1024) k_build_chunks(const int32_t* __restrict
             first_mb = lo;
             for (int mb = first_mb; mb < nmb && mbs[mb].row0 < b; ++mb) {
                 const int L = min(b, mbs[mb].row1) - max(a, mbs[mb].row0);
-                if (L > 0) cnt += piece_chunks(L);
+                if (L > 0) cnt += piece_chunks(L, maxr);
             }
         }
     }
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(1024) k_build_chunks(const int32_t* __restrict
             const int r0 = max(a, mbs[mb].row0);
             const int L = min(b, mbs[mb].row1) - r0;
             if (L <= 0) continue;
-            const int n = piece_chunks(L), base = piece_base(L);
+            const int n = piece_chunks(L, maxr), base = piece_base(L, maxr);
             for (int i = 0; i < n; ++i, ++idx) {
                 const int rr = (i < n - 1) ? base : L - (n - 1) * base;
                 if (idx < max_chunks) chunks[idx] = Chunk{e, r0 + i * base, rr, mb};
@@ -129,13 +130,15 @@ int max_minibatches(int n_slots, int minibatch) {
     if (minibatch <= 0) minibatch = 1;
     return n_slots / minibatch + 2;
 }
-int max_chunks(int n_slots, int E, int n_mb) { return n_slots / CHUNK_MAX_ROWS + E + n_mb + 2; }
+// bound for every chunk height cap >= CHUNK_MAX_ROWS_MX
+int max_chunks(int n_slots, int E, int n_mb) { return n_slots / CHUNK_MAX_ROWS_MX + E + n_mb + 2; }
 
-cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int minibatch, int cap, Chunk* chunks,
-                                int max_ch, Minibatch* mbs, int max_mb, int* counts2, void* status,
+cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int minibatch, int cap, int max_rows,
+                                Chunk* chunks, int max_ch, Minibatch* mbs, int max_mb, int* counts2, void* status,
                                 cudaStream_t stream) {
-    k_build_chunks<<<1, 1024, 0, stream>>>(offsets, E, n_slots, minibatch, cap, chunks, max_ch, mbs, max_mb, counts2,
-                                           reinterpret_cast<DevStatus*>(status));
+    if (max_rows < CHUNK_MAX_ROWS_MX || max_rows > CHUNK_MAX_ROWS || max_rows % 16) return cudaErrorInvalidValue;
+    k_build_chunks<<<1, 1024, 0, stream>>>(offsets, E, n_slots, minibatch, cap, max_rows, chunks, max_ch, mbs, max_mb,
+                                           counts2, reinterpret_cast<DevStatus*>(status));
     return cudaGetLastError();
 }
 
