@@ -144,10 +144,11 @@ def algorithmic_work(cfg):
     gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 4  # weights, rows in, h out+in, fp32 out
     gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * 2
     if cfg.mxfp8:
-        # weights: E4M3 bytes plus one E8M0 scale per 32 values; the quantised
-        # token rows and h are kept in their exact bf16 form (2 bytes a value)
-        w_bytes = cfg.E * 3 * cfg.H * cfg.I * (1.0 + 1.0 / 32)
-        gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 4
+        # weights, token rows and h: E4M3 bytes plus one E8M0 scale per 32 values
+        mx = 1.0 + 1.0 / 32
+        w_bytes = cfg.E * 3 * cfg.H * cfg.I * mx
+        gemm_bytes = w_bytes + ns * cfg.H * mx + 2 * ns * cfg.I * mx + ns * cfg.H * 4
+        gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * mx
     combine_bytes = ns * cfg.H * 4 + ns * 4 + cfg.T * cfg.H * 2
     return {
         "gemm_flops": 6.0 * cfg.H * cfg.I * ns,

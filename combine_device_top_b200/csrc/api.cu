@@ -121,9 +121,9 @@ bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* w
            encode_bmaps(&m->h, false, h, (uint64_t)I, (uint64_t)buf_rows, err);
 }
 
-// 2D map of a row-major [outer, inner] byte array, no swizzle.
+// 2D map of a row-major [outer, inner] byte array.
 static bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                         uint32_t box_outer) {
+                         uint32_t box_outer, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[2] = {inner, outer};
@@ -131,19 +131,30 @@ static bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uin
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool encode_mx_maps(MxMaps* m, const mok_mxfp8_weights& w, int H, int I, int E, const char** err) {
-    const bool ok = encode_2d_u8(&m->gq, w.gate, (uint64_t)I, (uint64_t)E * H, 64, 64) &&
-                    encode_2d_u8(&m->uq, w.up, (uint64_t)I, (uint64_t)E * H, 64, 64) &&
-                    encode_2d_u8(&m->dq, w.down, (uint64_t)H, (uint64_t)E * I, 128, 64) &&
-                    encode_2d_u8(&m->gs, w.gate_scales, (uint64_t)I, (uint64_t)E * H / 32, 64, 2) &&
-                    encode_2d_u8(&m->us, w.up_scales, (uint64_t)I, (uint64_t)E * H / 32, 64, 2) &&
-                    encode_2d_u8(&m->ds, w.down_scales, (uint64_t)H, (uint64_t)E * I / 32, 128, 2);
+    const bool ok =
+        encode_2d_u8(&m->gq, w.gate, (uint64_t)I, (uint64_t)E * H, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
+        encode_2d_u8(&m->uq, w.up, (uint64_t)I, (uint64_t)E * H, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
+        encode_2d_u8(&m->dq, w.down, (uint64_t)H, (uint64_t)E * I, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        encode_2d_u8(&m->gs, w.gate_scales, (uint64_t)I, (uint64_t)E * H / 32, 64, 4) &&
+        encode_2d_u8(&m->us, w.up_scales, (uint64_t)I, (uint64_t)E * H / 32, 64, 4) &&
+        encode_2d_u8(&m->ds, w.down_scales, (uint64_t)H, (uint64_t)E * I / 32, 128, 4);
     if (!ok) *err = "cuTensorMapEncodeTiled failed (MXFP8 weights)";
     return ok;
+}
+
+bool encode_bmaps_u8(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err) {
+    for (int i = 0; i < B_MAPS; ++i)
+        if (!encode_2d_u8(&maps->m[i], base, inner, rows, 128, (uint32_t)(16 * (i + 1)),
+                          CU_TENSOR_MAP_SWIZZLE_128B)) {
+            *err = "cuTensorMapEncodeTiled failed (MXFP8 token rows)";
+            return false;
+        }
+    return true;
 }
 
 // ------------------------------------------------------------------ layouts
@@ -151,7 +162,8 @@ static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct FwdLayout {
     size_t status, counts2, chunks, mbs, counters, rows, h, out, total;
-    int max_chunks, max_mb, buf_rows, cap, minibatch, mode;
+    size_t xsc, hsc;  // MXFP8 path: token-side scale planes
+    int max_chunks, max_mb, buf_rows, cap, minibatch, mode, mx;
 };
 
 static const uint64_t kDefaultTimeoutNs = 2000000000ull;
@@ -187,8 +199,17 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
     l.mbs = take(sizeof(Minibatch) * (size_t)l.max_mb);
     // persistent-mode counters: gathered[max_mb], d_done[max_mb], g_done[max_chunks], d_total
     l.counters = take(sizeof(int) * (2 * (size_t)l.max_mb + (size_t)l.max_chunks + 8));
-    l.rows = take((size_t)l.buf_rows * H * 2);
-    l.h = take((size_t)l.buf_rows * I * 2);
+    l.mx = (o && o->mxfp8) ? 1 : 0;
+    if (l.mx) {
+        // E4M3 rows and h, with their scale planes
+        l.rows = take((size_t)l.buf_rows * H);
+        l.h = take((size_t)l.buf_rows * I);
+        l.xsc = take(mx_sc_bytes(l.buf_rows, H));
+        l.hsc = take(mx_sc_bytes(l.buf_rows, I));
+    } else {
+        l.rows = take((size_t)l.buf_rows * H * 2);
+        l.h = take((size_t)l.buf_rows * I * 2);
+    }
     l.out = take((size_t)ns * H * 4);
     l.total = off;
     *L = l;
@@ -221,33 +242,36 @@ static int check_hi(int H, int I) {
 }
 
 // ------------------------------------------------------------------ pieces
-// mxw != nullptr: MXFP8 weights (wg/wu/wd are then ignored) and bf16 h.
+// mxw != nullptr: MXFP8 weights (wg/wu/wd are then ignored); rows and h are
+// E4M3 with the token-side scale planes of mxs.
 static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const void* wg, const void* wu,
                           const void* wd, int E, const int32_t* row_slot, const Chunk* chunks, const int* counts2,
                           void* h, void* out, DevStatus* status, uint64_t timeout_ns, cudaStream_t stream,
-                          const mok_mxfp8_weights* mxw = nullptr) {
+                          const mok_mxfp8_weights* mxw = nullptr, const MxTokenScales* mxs = nullptr) {
     int dev = 0;
     const int sms = device_sms(&dev);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     MOK_CUDA(gemm_configure(dev), "gemm configure");
     GemmMaps maps;
+    memset(&maps, 0, sizeof maps);
     MxMaps mx;
     const char* err = nullptr;
     if (mxw) {
-        // the bf16 weight maps are not read on the MXFP8 path: any valid base will do
-        wg = wu = wd = mxw->gate;
-        if (!encode_mx_maps(&mx, *mxw, H, I, E, &err)) return fail(MOK_ERR_CUDA, "tensor map: %s", err);
-    }
-    if (!encode_gemm_maps(&maps, wg, wu, wd, rows, h, H, I, E, n_rows_buf, &err))
+        if (!encode_mx_maps(&mx, *mxw, H, I, E, &err) ||
+            !encode_bmaps_u8(&maps.rows, rows, (uint64_t)H, (uint64_t)n_rows_buf, &err) ||
+            !encode_bmaps_u8(&maps.h, h, (uint64_t)I, (uint64_t)n_rows_buf, &err))
+            return fail(MOK_ERR_CUDA, "tensor map: %s", err);
+    } else if (!encode_gemm_maps(&maps, wg, wu, wd, rows, h, H, I, E, n_rows_buf, &err)) {
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
+    }
     GemmShape sh{H, I, E};
     const GemmTuning tune = gemm_tuning(n_rows_buf, E);
     const MxMaps* mxp = mxw ? &mx : nullptr;
-    MOK_CUDA(launch_gemm_phase(0, maps, mxp, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune,
-                               stream),
+    MOK_CUDA(launch_gemm_phase(0, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
+                               tune, stream),
              "gate/up GEMM launch");
-    MOK_CUDA(launch_gemm_phase(1, maps, mxp, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms, tune,
-                               stream),
+    MOK_CUDA(launch_gemm_phase(1, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
+                               tune, stream),
              "down GEMM launch");
     return MOK_OK;
 }
@@ -415,12 +439,19 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         if (e != cudaSuccess) return fail(MOK_ERR_CUDA, "%s: %s", err, cudaGetErrorString(e));
         return MOK_OK;
     }
-    if (mxw)
-        MOK_CUDA(launch_gather_mx(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
-    else
+    MxTokenScales mxs{};
+    if (mxw) {
+        mxs.xsc = base + L.xsc;
+        mxs.hsc = base + L.hsc;
+        mxs.sc_rows = mx_sc_rows(L.buf_rows);
+        MOK_CUDA(launch_gather_mx(xs, T / R, H, T, k, plan->pos, base + L.rows, base + L.xsc, mxs.sc_rows, sms,
+                                  stream),
+                 "gather launch");
+    } else {
         MOK_CUDA(launch_gather(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
+    }
     rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, chunks, counts2,
-                        base + L.h, base + L.out, status, timeout, stream, mxw);
+                        base + L.h, base + L.out, status, timeout, stream, mxw, mxw ? &mxs : nullptr);
     if (rc) return rc;
     MOK_CUDA(launch_combine(base + L.out, plan->gates, T, k, H, T / R, ys, sms, stream), "combine launch");
     return MOK_OK;

@@ -51,13 +51,16 @@ __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens(ShardsIn xs, int S
 
 // The same copy with MXFP8 quantisation fused in (MoK article: activation
 // quantisation inside the dispatch): each 32-element block of the token row
-// is quantised to E4M3 with its E8M0 scale and written to the k rows as the
-// exact bf16 value of the quantised block (what the tensor cores multiply).
-// Each lane owns 8 consecutive elements, 4 lanes a block; the step loop is
-// warp-uniform (lanes past the end join the shuffles with zeros).
+// is quantised to E4M3 with its E8M0 scale; the k rows receive the E4M3
+// bytes and the scale planes [H/128][sc_rows][4] the block scales (plane g,
+// byte b: block 4g + b), the operand form of the block-scaled MMA.
+// Each lane owns 8 consecutive elements, 4 lanes a block, a half-warp one
+// 4-block scale word; the step loop is warp-uniform (lanes past the end
+// join the shuffles with zeros).
 __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens_mx(ShardsIn xs, int S_r, int H, int T, int k,
                                                                  const int32_t* __restrict__ pos,
-                                                                 uint4* __restrict__ rows) {
+                                                                 uint8_t* __restrict__ rows, uint8_t* __restrict__ xsc,
+                                                                 int sc_rows) {
     const int lane = threadIdx.x & 31;
     const int nvec = H >> 3;
     const int warps = gridDim.x * (DC_THREADS / 32);
@@ -82,28 +85,36 @@ __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens_mx(ShardsIn xs, in
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
             const int s = mx_block_exponent(amax);
-            const float inv = mx_pow2(-s), scl = mx_pow2(s);
-            uint32_t o[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 d = mx_e4m3x2_to_float2(mx_e4m3x2(v[2 * p] * inv, v[2 * p + 1] * inv));
-                o[p] = pack_bf16x2(d.x * scl, d.y * scl);
-            }
-            const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+            const float inv = mx_pow2(-s);
+            const uint2 q = make_uint2((uint32_t)mx_e4m3x2(v[0] * inv, v[1] * inv) |
+                                           ((uint32_t)mx_e4m3x2(v[2] * inv, v[3] * inv) << 16),
+                                       (uint32_t)mx_e4m3x2(v[4] * inv, v[5] * inv) |
+                                           ((uint32_t)mx_e4m3x2(v[6] * inv, v[7] * inv) << 16));
+            // the half-warp's 4 block scales as one word (block 4g + b in byte b)
+            const uint32_t sb = (uint32_t)(s + 127);
+            const int h0 = lane & 16;
+            const uint32_t word = __shfl_sync(0xffffffffu, sb, h0) | (__shfl_sync(0xffffffffu, sb, h0 + 4) << 8) |
+                                  (__shfl_sync(0xffffffffu, sb, h0 + 8) << 16) |
+                                  (__shfl_sync(0xffffffffu, sb, h0 + 12) << 24);
+            uint32_t* plane = reinterpret_cast<uint32_t*>(xsc) + (size_t)((c0 >> 7) + (lane >> 4)) * sc_rows;
             for (int j = 0; j < k; ++j) {
                 const int row = __shfl_sync(0xffffffffu, my_row, j);
-                if (live) rows[(size_t)row * nvec + (c >> 3)] = ov;
+                if (live) {
+                    *reinterpret_cast<uint2*>(rows + (size_t)row * H + c) = q;
+                    if ((lane & 15) == 0) plane[row] = word;
+                }
             }
         }
     }
 }
 
 cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
-                             int num_sms, cudaStream_t stream) {
+                             void* xsc, int sc_rows, int num_sms, cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
     const int want = (T + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     const int grid = want < num_sms * 8 ? want : num_sms * 8;
-    k_gather_tokens_mx<<<grid, DC_THREADS, 0, stream>>>(xs, S_r, H, T, k, pos, reinterpret_cast<uint4*>(rows));
+    k_gather_tokens_mx<<<grid, DC_THREADS, 0, stream>>>(xs, S_r, H, T, k, pos, reinterpret_cast<uint8_t*>(rows),
+                                                         reinterpret_cast<uint8_t*>(xsc), sc_rows);
     return cudaGetLastError();
 }
 

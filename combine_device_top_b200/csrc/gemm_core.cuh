@@ -25,16 +25,16 @@
 // Precision: the bf16 path computes gate/up in bf16 and the down projection
 // in fp16 (fp16 h and the fp16 copy of Wd: 3 more mantissa bits on h keep
 // the error of y at the floor of its own bf16 rounding).  The MXFP8 path
-// reads E4M3 weight bytes with E8M0 block scales and a converter warpgroup
-// turns each tile into exact bf16 values in shared memory (an E4M3 value
-// times 2^s has at most 4 significant bits); x and h are MXFP8-quantised
-// (quantised and dequantised exactly) before they reach the MMA.
+// runs the block-scaled tensor-core MMA (kind::mxf8f6f4): E4M3 weights and
+// E4M3 token rows / h rows, each with one E8M0 scale per 32 K values, which
+// the MMA reads from TMEM; the products are exact and accumulate in fp32.
+// The gather quantises x and the gate/up epilogue quantises h.
 //
 // Roles in a CTA: warp 0 issues TMA loads into a ring of stages, warp 1
 // allocates 512 TMEM columns and one thread of it issues tcgen05.mma into
 // one of two 256-column accumulators, warps 2-5 drain the other accumulator
 // (tcgen05.ld) through shared memory to global memory, and (MXFP8 only)
-// warps 6-9 convert weight tiles.  The token tile of a stage is ONE TMA box
+// warp 6 lays each stage's scales out for the copy into TMEM.  The token tile of a stage is ONE TMA box
 // of exactly the 16-rounded row count, and a down unit's two 64-column
 // weight halves come from one 3D map.  Measured on B200: the number of TMA
 // ops per SM, and then the bytes each SM takes in from L2 (about 64 B per
@@ -75,6 +75,7 @@ struct Bf16CfgT {
     static constexpr int SUB = SUB_;  // M tiles per unit
     static constexpr int THREADS = 192;
     static constexpr int NST = NST_;
+    static constexpr int BKX = BK;  // K per stage
     static constexpr int STAGE = SUB * A_BYTES + B_BYTES;
     static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
     static constexpr int EPI_OFF = NST * STAGE;
@@ -85,20 +86,31 @@ struct Bf16CfgT {
 using Bf16Cfg = Bf16CfgT<1, 4>;
 using Bf16PairCfg = Bf16CfgT<2, 3>;
 static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share the barrier offset");
+// MXFP8 path (block-scaled tcgen05 MMA, K = 128 per stage):
+// [A E4M3 16 KB][B E4M3 <= 224 rows x 128 B][A scales as loaded 512 B]
+// [B scales as loaded <= 1 KB][A scales, MMA layout 512 B][B scales, MMA
+// layout 1 KB] x 4.
 struct MxCfg {
     static constexpr bool MX = true;
     static constexpr int SUB = 1;
-    static constexpr int THREADS = 320;
-    static constexpr int NST = 3;
-    static constexpr int A_OFF = 0, B_OFF = A_BYTES;
-    static constexpr int RAW_OFF = A_BYTES + B_BYTES;  // 64 x 128 E4M3 bytes
-    static constexpr int SC_OFF = RAW_OFF + 8192;      // 2 x 128 scale bytes
-    static constexpr int STAGE = SC_OFF + 1024;
+    static constexpr int THREADS = 224;  // + warp 6: scale-factor layout
+    static constexpr int NST = 4;
+    static constexpr int BKX = 128;      // K per stage
+    static constexpr int A_OFF = 0, B_OFF = 16384;
+    static constexpr int SFA_RAW_OFF = B_OFF + CHUNK_MAX_ROWS_MX * 128;  // [4 K blocks][128 rows]
+    static constexpr int SFB_RAW_OFF = SFA_RAW_OFF + 512;                // [rows][4 K blocks], 16-byte aligned copy
+    static constexpr int SFA_OFF = SFB_RAW_OFF + 1024;                   // one 512-byte scale atom
+    static constexpr int SFB_OFF = SFA_OFF + 512;                        // two atoms (rows 0-127, 128-255)
+    static constexpr int STAGE = SFB_OFF + 1024;
     static constexpr int EPI_OFF = NST * STAGE;
     static constexpr int XCH_OFF = EPI_OFF + EPI_BYTES;  // amax exchange of the h quantiser
     static constexpr int BAR_OFF = XCH_OFF + 512;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    // TMEM: accumulators at columns 0 and 256 (N <= 224), scale factors above
+    static constexpr uint32_t TM_SFA = 480, TM_SFB = 484;
 };
+static_assert(MxCfg::STAGE % 1024 == 0, "MXFP8 stages must keep 1024-byte alignment");
+static_assert(MxCfg::SMEM <= 232448, "MXFP8 layout exceeds shared memory");
 // Shared-memory layout used by code outside the GEMM roles (dispatch CTAs of
 // the persistent kernel place their row slots below SMEM_BAR_OFF).
 constexpr int GEMM_THREADS = Bf16Cfg::THREADS;
@@ -120,11 +132,16 @@ struct Unit {
 
 struct CoreArgs {
     int H, I;
-    void* h;                  // [buffer rows, I]: fp16 (bf16 path) or bf16 (MXFP8 path)
+    void* h;                  // [buffer rows, I]: fp16 (bf16 path) or E4M3 (MXFP8 path)
     float* out;               // [N_s, H] fp32, slot-indexed
     const int32_t* row_slot;  // [N_s]
     DevStatus* st;
     uint64_t timeout_ns;
+    // MXFP8 path: E8M0 scales of the token side as planes [K/128][sc_rows][4]
+    // (plane g, row r, byte b: the scale of K block 4g + b of row r)
+    const uint8_t* xsc;       // token rows (gate/up B operand), K = H
+    uint8_t* hsc;             // h rows (written by gate/up, read by down), K = I
+    int sc_rows;              // rows per plane, a multiple of 4
 };
 
 // Unit u -> (chunk c, M tile m) in raster groups of GC chunks: inside a group
@@ -195,13 +212,17 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
     for (int i = 0; s.get(i, u); ++i) {
         if (!s.wait_inputs(u, a.st, a.timeout_ns)) break;
         const int K = u.phase == 0 ? a.H : a.I;
-        const int KB = K / BK;
+        const int KB = (K + C::BKX - 1) / C::BKX;
         const BMaps& bm = u.phase == 0 ? maps.rows : maps.h;
         const int bx = token_box(u.rows);
         const int nsub = unit_subs<C>(a, u);
         uint32_t bytes = (uint32_t)(16 * (bx + 1)) * B_ROW_BYTES;
+        // MXFP8: the token side's scales for this stage are one 16-byte
+        // aligned run of the plane, starting up to 3 rows before the chunk
+        const int sc_lead = u.brow0 & 3;
+        const uint32_t sc_bytes = (uint32_t)(4 * (sc_lead + u.rows) + 15) & ~15u;
         if (C::MX)
-            bytes += u.phase == 0 ? 2 * (4096 + 128) : (8192 + 256);  // E4M3 bytes + scale bytes
+            bytes += 16384 + 512 + sc_bytes;  // E4M3 weight tile + its scales + the token scales
         else
             bytes += (uint32_t)nsub * A_BYTES;
         bool ok = true;
@@ -212,20 +233,23 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
             }
             unsigned char* st = smem + stage * C::STAGE;
             mbar_arrive_expect_tx(&full[stage], bytes);
-            const int ky = u.expert * K + kb * BK;
+            const int ky = u.expert * K + kb * C::BKX;
             if constexpr (C::MX) {
-                unsigned char* raw = st + MxCfg::RAW_OFF;
-                unsigned char* sc = st + MxCfg::SC_OFF;
-                const int kys = (u.expert * K + kb * BK) / 32;  // scale row of the first K block
+                unsigned char* sfa = st + MxCfg::SFA_RAW_OFF;
+                const int kys = ky / 32;  // scale row of the stage's first K block
                 if (u.phase == 0) {
-                    tma_load_2d_hint(raw, &mx->gq, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
-                    tma_load_2d_hint(raw + 4096, &mx->uq, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
-                    tma_load_2d(sc, &mx->gs, &full[stage], u.m * MT_G_FEATURES, kys);
-                    tma_load_2d(sc + 128, &mx->us, &full[stage], u.m * MT_G_FEATURES, kys);
+                    // gate and up columns of the M tile: two 64-byte-swizzled 64-column boxes
+                    tma_load_2d_hint(st + MxCfg::A_OFF, &mx->gq, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
+                    tma_load_2d_hint(st + MxCfg::A_OFF + 8192, &mx->uq, &full[stage], u.m * MT_G_FEATURES, ky,
+                                     evict_first);
+                    tma_load_2d(sfa, &mx->gs, &full[stage], u.m * MT_G_FEATURES, kys);
+                    tma_load_2d(sfa + 256, &mx->us, &full[stage], u.m * MT_G_FEATURES, kys);
                 } else {
-                    tma_load_2d_hint(raw, &mx->dq, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
-                    tma_load_2d(sc, &mx->ds, &full[stage], u.m * MT_D_FEATURES, kys);
+                    tma_load_2d_hint(st + MxCfg::A_OFF, &mx->dq, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
+                    tma_load_2d(sfa, &mx->ds, &full[stage], u.m * MT_D_FEATURES, kys);
                 }
+                const uint8_t* plane = (u.phase == 0 ? a.xsc : a.hsc) + (size_t)kb * a.sc_rows * 4;
+                bulk_load(st + MxCfg::SFB_RAW_OFF, plane + (size_t)(u.brow0 - sc_lead) * 4, sc_bytes, &full[stage]);
             } else {
                 for (int sub = 0; sub < nsub; ++sub) {
                     unsigned char* sa = st + C::A_OFF + sub * A_BYTES;
@@ -244,7 +268,7 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
                     }
                 }
             }
-            tma_load_2d(st + C::B_OFF, &bm.m[bx], &full[stage], kb * BK, u.brow0);
+            tma_load_2d(st + C::B_OFF, &bm.m[bx], &full[stage], kb * C::BKX, u.brow0);
             issued |= 1u << stage;
             issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == C::NST) {
@@ -259,21 +283,29 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
         if ((issued >> st) & 1u) mbar_wait(&full[st], (issued_phase >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 11);
 }
 
-// ------------------------------------------------------------------ MXFP8 converter (warps 6..9)
-// Per stage: E4M3 bytes (gate/up: two [64 K][64] tiles; down: one [64 K][128]
-// tile) and E8M0 scales ([2 blocks][64] per gate/up tile, [2][128] down) ->
-// the MN-major 128-byte-swizzled bf16 A tile the MMA reads: half h (MN
-// 0-63 / 64-127) at h * 8 KB, K row k at k * 128 bytes, 16-byte chunk j at
-// position j ^ (k & 7).  Each thread converts 8 tasks of 8 elements.
+// ------------------------------------------------------------------ MXFP8 scale-factor layout (warp 6)
+// The block-scaled MMA reads the scales of a 128-row operand tile from TMEM
+// as 32 lanes x 4 columns of 32-bit words: row r = r0 + 32 r1 at lane r0,
+// column r1, byte b = K block b of the stage (the copy to TMEM takes them
+// from shared memory as 32 rows of 16 bytes: row r0 = the 4 words r1 =
+// 0..3).  Per stage this warp rearranges the scales as loaded into that
+// atom layout:
+//   weights (A): loaded [4 K blocks][128 features] (gate/up: [4][64] gate
+//     then [4][64] up, features 0-63 gate and 64-127 up of the M tile);
+//   tokens (B): loaded [rows][4 K blocks] starting sc_lead rows early; rows
+//     past the chunk get scale 0 (their MMA columns are never stored);
+//     rows 128-255 form a second atom.
 template <class S>
-__device__ __forceinline__ void gemm_converter(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* full,
-                                               uint64_t* conv) {
-    const int ct = threadIdx.x - 192;  // 0..127
+__device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* full,
+                                               uint64_t* sfready) {
+    const int lane = threadIdx.x & 31;
     int stage = 0;
     uint32_t phase = 0;
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
-        const int KB = (u.phase == 0 ? a.H : a.I) / BK;
+        const int K = u.phase == 0 ? a.H : a.I;
+        const int KB = (K + MxCfg::BKX - 1) / MxCfg::BKX;
+        const int lead = u.brow0 & 3;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 80)) {
@@ -281,40 +313,32 @@ __device__ __forceinline__ void gemm_converter(const CoreArgs& a, const S& s, un
                 break;
             }
             unsigned char* st = smem + stage * MxCfg::STAGE;
-            const unsigned char* raw = st + MxCfg::RAW_OFF;
-            const unsigned char* sc = st + MxCfg::SC_OFF;
-            unsigned char* dst = st + MxCfg::A_OFF;
-#pragma unroll 2
-            for (int t = 0; t < 8; ++t) {
-                const int task = t * 128 + ct;
-                const int h = task >> 9, k = (task >> 3) & 63, g = task & 7;
-                const unsigned char* src;
-                const unsigned char* scl;
-                if (u.phase == 0) {
-                    src = raw + h * 4096 + k * 64 + g * 8;
-                    scl = sc + h * 128 + (k >> 5) * 64 + g * 8;
-                } else {
-                    src = raw + k * 128 + h * 64 + g * 8;
-                    scl = sc + (k >> 5) * 128 + h * 64 + g * 8;
-                }
-                const uint2 qv = *reinterpret_cast<const uint2*>(src);
-                const uint2 sv = *reinterpret_cast<const uint2*>(scl);
-                uint32_t o[4];
+            const uint8_t* ra = st + MxCfg::SFA_RAW_OFF;
+            const uint32_t* rb = reinterpret_cast<const uint32_t*>(st + MxCfg::SFB_RAW_OFF) + lead;
+            uint32_t wa[4];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const uint32_t qw = p < 2 ? qv.x : qv.y;
-                    const uint32_t sw = p < 2 ? sv.x : sv.y;
-                    const int sh = (p & 1) * 16;
-                    const float2 f = mx_e4m3x2_to_float2((uint16_t)(qw >> sh));
-                    const float s0 = mx_pow2((int)((sw >> sh) & 0xff) - 127);
-                    const float s1 = mx_pow2((int)((sw >> (sh + 8)) & 0xff) - 127);
-                    o[p] = pack_bf16x2(f.x * s0, f.y * s1);
-                }
-                *reinterpret_cast<uint4*>(dst + h * 8192 + k * 128 + ((g ^ (k & 7)) << 4)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
+            for (int r1 = 0; r1 < 4; ++r1) {
+                const int r = lane + 32 * r1;
+                // feature r of the tile: gate/up keeps 64 gate then 64 up rows of 64 bytes
+                const uint8_t* col = u.phase == 0 ? ra + (r >> 6) * 256 + (r & 63) : ra + r;
+                const int pitch = u.phase == 0 ? 64 : 128;
+                wa[r1] = (uint32_t)col[0] | ((uint32_t)col[pitch] << 8) | ((uint32_t)col[2 * pitch] << 16) |
+                         ((uint32_t)col[3 * pitch] << 24);
             }
-            fence_proxy_async_shared();  // generic writes -> the MMA's (async proxy) reads
-            mbar_arrive(&conv[stage]);
+            *reinterpret_cast<uint4*>(st + MxCfg::SFA_OFF + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+#pragma unroll
+            for (int r2 = 0; r2 < 2; ++r2) {
+                uint32_t wb[4];
+#pragma unroll
+                for (int r1 = 0; r1 < 4; ++r1) {
+                    const int r = lane + 32 * r1 + 128 * r2;
+                    wb[r1] = r < u.rows ? rb[r] : 0u;
+                }
+                *reinterpret_cast<uint4*>(st + MxCfg::SFB_OFF + 512 * r2 + 16 * lane) =
+                    make_uint4(wb[0], wb[1], wb[2], wb[3]);
+            }
+            fence_proxy_async_shared();  // generic writes -> the TMEM copy (async proxy) reads
+            mbar_arrive(&sfready[stage]);
             if (++stage == MxCfg::NST) {
                 stage = 0;
                 phase ^= 1u;
@@ -336,7 +360,7 @@ __device__ __forceinline__ uint32_t acc_col(uint32_t tk, int sub, bool wide) {
 }
 
 // ------------------------------------------------------------------ MMA issuer
-// ready[stage]: the TMA barrier (bf16) or the converter barrier (MXFP8).
+// ready[stage]: the TMA barrier (bf16) or the scale-layout barrier (MXFP8).
 template <class S, class C>
 __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* ready,
                                          uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* fin,
@@ -346,14 +370,14 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
     uint32_t tk = 0;  // next accumulator ticket
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
-        const int KB = (u.phase == 0 ? a.H : a.I) / BK;
+        const int K = u.phase == 0 ? a.H : a.I;
+        const int KB = (K + C::BKX - 1) / C::BKX;
         const int N = (u.rows + 15) & ~15;
         const int nsub = unit_subs<C>(a, u);
         const int nt = unit_tickets(nsub, N);
         const bool wide = nt == 2;
-        // bf16 path: gate/up bf16 x bf16, down fp16 x fp16; MXFP8 path: bf16 x bf16
-        const uint32_t idesc =
-            umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, (C::MX || u.phase == 0) ? 1 : 0);
+        // bf16 path: gate/up bf16 x bf16, down fp16 x fp16
+        const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, u.phase == 0 ? 1 : 0);
         bool ok = true;
         for (int t = 0; t < nt && ok; ++t) {
             const uint32_t tkt = tk + (uint32_t)t;
@@ -369,17 +393,39 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
             tc_fence_after();
             const uint32_t sa = smem_u32(smem + stage * C::STAGE + C::A_OFF);
             const uint32_t sb = smem_u32(smem + stage * C::STAGE + C::B_OFF);
+            if constexpr (C::MX) {
+                // scale factors of this stage into TMEM (executed in order with the MMAs)
+                unsigned char* st = smem + stage * C::STAGE;
+                tmem_cp_32x128b_warpx4(tmem_base + MxCfg::TM_SFA, st + MxCfg::SFA_OFF);
+                tmem_cp_32x128b_warpx4(tmem_base + MxCfg::TM_SFB, st + MxCfg::SFB_OFF);
+                if (N > 128) tmem_cp_32x128b_warpx4(tmem_base + MxCfg::TM_SFB + 4, st + MxCfg::SFB_OFF + 512);
+                const int nks = min(4, (K - kb * C::BKX) / 32);  // 32 K values per MMA
+                for (int ks = 0; ks < nks; ++ks) {
+                    // A: MN-major E4M3; gate/up = two 64-byte-swizzled 64-column halves 8 KB
+                    //    apart (8-row K groups 512 bytes apart), down = one 128-byte-swizzled
+                    //    128-column tile (K groups 1 KB apart); 32 K rows per MMA.
+                    const uint64_t ad = u.phase == 0 ? umma_desc(sa + ks * 2048, 8192, 512, UMMA_LAYOUT_SW64)
+                                                     : umma_desc(sa + ks * 4096, 0, 1024, UMMA_LAYOUT_SW128);
+                    // B: K-major E4M3 SW128, 32 K = 32 bytes inside the atom
+                    const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
+                    const uint32_t sel = (uint32_t)ks << 30;  // scale byte of these 32 K values
+                    umma_mxf8(tmem_base + acc_col(tk, 0, false), ad, bd, umma_idesc_mxf8(128, N, 1, 0, (uint32_t)ks),
+                              tmem_base + MxCfg::TM_SFA + sel, tmem_base + MxCfg::TM_SFB + sel,
+                              (kb | ks) != 0 ? 1u : 0u);
+                }
+            } else {
 #pragma unroll
-            for (int ks = 0; ks < BK / 16; ++ks) {
-                // B: K-major SW128, 16 K = 32 bytes inside the atom; 8-row groups 1 KB apart.
-                const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
+                for (int ks = 0; ks < BK / 16; ++ks) {
+                    // B: K-major SW128, 16 K = 32 bytes inside the atom; 8-row groups 1 KB apart.
+                    const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
 #pragma unroll
-                for (int sub = 0; sub < C::SUB; ++sub) {
-                    if (sub < nsub) {
-                        // A: MN-major SW128, 16 K rows per MMA = 2 atoms of 1 KB;
-                        //    the two 64-wide MN halves are 8 KB apart (LBO).
-                        const uint64_t ad = umma_desc_sw128(sa + sub * A_BYTES + ks * 2048, A_BYTES / 2, 1024);
-                        umma_bf16(tmem_base + acc_col(tk, sub, wide), ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                    for (int sub = 0; sub < C::SUB; ++sub) {
+                        if (sub < nsub) {
+                            // A: MN-major SW128, 16 K rows per MMA = 2 atoms of 1 KB;
+                            //    the two 64-wide MN halves are 8 KB apart (LBO).
+                            const uint64_t ad = umma_desc_sw128(sa + sub * A_BYTES + ks * 2048, A_BYTES / 2, 1024);
+                            umma_bf16(tmem_base + acc_col(tk, sub, wide), ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                        }
                     }
                 }
             }
@@ -428,9 +474,9 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 const float up = epi[(64 + fq * 16 + k) * EPI_LD + tok];
                 hv[k] = g / (1.0f + __expf(-g)) * up;
             }
-            uint32_t pk[8];
             if constexpr (C::MX) {
-                // MXFP8 h: blocks of 32 features = thread pairs fq ^ 1 (same token)
+                // MXFP8 h: blocks of 32 features = thread pairs fq ^ 1 (same token);
+                // E4M3 bytes to h, the block's E8M0 byte to its scale plane
                 float amax = 0.f;
 #pragma unroll
                 for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(hv[k]));
@@ -438,21 +484,31 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 named_bar_sync(1, 128);
                 amax = fmaxf(amax, xch[(fq ^ 1) * 32 + tok]);
                 const int sx = mx_block_exponent(amax);
-                const float inv = mx_pow2(-sx), scl = mx_pow2(sx);
+                const float inv = mx_pow2(-sx);
+                uint32_t pq[4];
 #pragma unroll
-                for (int k = 0; k < 16; k += 2) {
-                    const float2 d = mx_e4m3x2_to_float2(mx_e4m3x2(hv[k] * inv, hv[k + 1] * inv));
-                    pk[k >> 1] = pack_bf16x2(d.x * scl, d.y * scl);
+                for (int k = 0; k < 16; k += 4)
+                    pq[k >> 2] = (uint32_t)mx_e4m3x2(hv[k] * inv, hv[k + 1] * inv) |
+                                 ((uint32_t)mx_e4m3x2(hv[k + 2] * inv, hv[k + 3] * inv) << 16);
+                if (live) {
+                    const size_t row = (size_t)(u.brow0 + col);
+                    *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.h) + row * a.I + mt * MT_G_FEATURES +
+                                              fq * 16) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
+                    if ((fq & 1) == 0) {
+                        const int b = 2 * mt + (fq >> 1);  // 32-feature block along I
+                        a.hsc[((size_t)(b >> 2) * a.sc_rows + row) * 4 + (b & 3)] = (uint8_t)(sx + 127);
+                    }
                 }
             } else {
+                uint32_t pk[8];
 #pragma unroll
                 for (int k = 0; k < 16; k += 2) pk[k >> 1] = pack_half2_sat(hv[k], hv[k + 1]);
-            }
-            if (live) {
-                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) +
-                                                      (size_t)(u.brow0 + col) * a.I + mt * MT_G_FEATURES + fq * 16);
-                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                if (live) {
+                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) +
+                                                          (size_t)(u.brow0 + col) * a.I + mt * MT_G_FEATURES + fq * 16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
             }
         } else if (live) {
             // fp32 push to the token's slot; the combine rounds y once
@@ -524,8 +580,8 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
                                          unsigned char* smem) {
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     uint64_t* empty = full + C::NST;
-    uint64_t* conv = empty + C::NST;  // MXFP8 only
-    uint64_t* tfull = conv + C::NST;
+    uint64_t* sfready = empty + C::NST;  // MXFP8 only: stage scales in the MMA layout
+    uint64_t* tfull = sfready + C::NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* fin = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
@@ -536,7 +592,7 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
         for (int st = 0; st < C::NST; ++st) {
             mbar_init(&full[st], 1);
             mbar_init(&empty[st], 1);
-            mbar_init(&conv[st], 128);
+            mbar_init(&sfready[st], 32);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
@@ -576,11 +632,11 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
     if (warp == 0) {
         if (lane == 0) gemm_producer<S, C>(maps, mx, a, s, smem, full, empty);
     } else if (warp == 1) {
-        if (lane == 0) gemm_mma<S, C>(a, s, smem, C::MX ? conv : full, empty, tfull, tempty, fin, tmem_base);
+        if (lane == 0) gemm_mma<S, C>(a, s, smem, C::MX ? sfready : full, empty, tfull, tempty, fin, tmem_base);
     } else if (warp < 6) {
         gemm_epilogue<S, C>(a, s, smem, tfull, tempty, ok_flag, tmem_base);
     } else if constexpr (C::MX) {
-        gemm_converter(a, s, smem, full, conv);
+        gemm_sf_layout(a, s, smem, full, sfready);
     }
 
     tc_fence_before();

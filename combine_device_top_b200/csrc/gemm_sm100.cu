@@ -54,11 +54,17 @@ cudaError_t gemm_configure(int dev) {
     return e;
 }
 
-cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const GemmShape& sh,
-                              const Chunk* chunks, const int* counts2, void* h_out, void* out,
+cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const MxTokenScales* mxs,
+                              const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
                               const GemmTuning& tune, cudaStream_t stream) {
-    CoreArgs a;
+    if (mx && !mxs) return cudaErrorInvalidValue;
+    CoreArgs a{};
+    if (mxs) {
+        a.xsc = mxs->xsc;
+        a.hsc = mxs->hsc;
+        a.sc_rows = mxs->sc_rows;
+    }
     a.H = sh.H;
     a.I = sh.I;
     a.h = h_out;

@@ -223,14 +223,19 @@ __device__ __forceinline__ void tc_fence_after() {
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 format):
 // [0,14) start>>4, [16,30) LBO>>4, [32,46) SBO>>4, [46,48) version = 1,
 // [49,52) base offset, [52] LBO mode, [61,64) layout (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Layout codes: 0 = no swizzle, 2 = 128-byte swizzle, 4 = 64-byte swizzle.
+constexpr uint32_t UMMA_LAYOUT_NONE = 0, UMMA_LAYOUT_SW128 = 2, UMMA_LAYOUT_SW64 = 4;
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1u << 46;
-    d |= (uint64_t)2u << 61;
+    d |= (uint64_t)(layout & 7u) << 61;
     return d;
+}
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return umma_desc(saddr, lbo, sbo, UMMA_LAYOUT_SW128);
 }
 
 // Instruction descriptor, kind::f16 with fp32 accumulation; A and B share
@@ -252,6 +257,40 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: A and B E4M3
+// (format 0), one E8M0 scale per 32 K values (scale format bit 23 = 1),
+// fp32 accumulation; sf_id (0..3) picks the byte of each 32-bit scale-factor
+// TMEM word that this MMA's 32 K values use, for A [29,31) and B [4,6):
+// [7,10) A fmt, [10,13) B fmt, [15] A major (1 = MN), [16] B major,
+// [17,23) N>>3, [24,29) M>>4.
+__device__ __forceinline__ uint32_t umma_idesc_mxf8(int M, int N, int a_mn_major, int b_mn_major, uint32_t sf_id) {
+    return (sf_id << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+           (1u << 23) | ((uint32_t)(M >> 4) << 24) | (sf_id << 29);
+}
+
+// D[tmem] (+)= (A * 2^SFA)[smem] * (B * 2^SFB)[smem]^T, E4M3 operands with
+// E8M0 block scales read from TMEM (sfa/sfb: TMEM addresses whose top two
+// bits repeat the byte index of the idesc's sf_id fields).
+__device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Copy 32 rows x 16 bytes from shared memory (no swizzle, rows 16 bytes
+// apart in 8-row groups of 128 bytes) to TMEM lanes 0-31, columns c..c+3,
+// repeated in each of the four 32-lane quarters: the scale-factor layout
+// the block-scaled MMA reads (row r of a 128-row operand: lane r % 32,
+// column c + r / 32, one byte per 32-value K block).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, const void* smem_src) {
+    const uint64_t d = umma_desc(smem_u32(smem_src), 16, 128, UMMA_LAYOUT_NONE);
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread complete.

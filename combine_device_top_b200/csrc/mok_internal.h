@@ -38,10 +38,10 @@ struct ShardsOut {
 // rows[pos[t*k + j]] = x[t] for every slot (token-major walk of the pull schedule)
 cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
                           int num_sms, cudaStream_t stream);
-// the same with MXFP8 quantisation of every 32-element block (rows hold the
-// exact bf16 values of the quantised blocks)
+// the same with MXFP8 quantisation of every 32-element block: rows [*, H]
+// E4M3, block scales in planes [H/128][sc_rows][4] (see mx_sc_rows)
 cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
-                             int num_sms, cudaStream_t stream);
+                             void* xsc, int sc_rows, int num_sms, cudaStream_t stream);
 cudaError_t launch_combine(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
                            int num_sms, cudaStream_t stream);
 
@@ -102,17 +102,33 @@ bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* w
 
 // Extra maps of the MXFP8 GEMM: E4M3 weight bytes and E8M0 scale bytes.
 struct MxMaps {
-    CUtensorMap gq, uq, dq;  // bytes: {64, 64} boxes of Wg/Wu [E*H, I]; {128, 64} boxes of Wd [E*I, H]
-    CUtensorMap gs, us, ds;  // scales: {64, 2} boxes of [E*H/32, I]; {128, 2} boxes of [E*I/32, H]
+    CUtensorMap gq, uq;  // {64 columns, 128 K rows} boxes of Wg/Wu [E*H, I], 64-byte swizzle
+    CUtensorMap dq;      // {128, 128} boxes of Wd [E*I, H], 128-byte swizzle
+    CUtensorMap gs, us;  // scales: {64, 4} boxes of [E*H/32, I]
+    CUtensorMap ds;      // scales: {128, 4} boxes of [E*I/32, H]
 };
 bool encode_mx_maps(MxMaps* m, const mok_mxfp8_weights& w, int H, int I, int E, const char** err);
+// Token-side maps of the MXFP8 GEMM: E4M3 rows [rows, inner] in boxes of
+// {128 bytes, 16 (i + 1) rows}, 128-byte swizzle.
+bool encode_bmaps_u8(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err);
+// Token-side scale planes of the MXFP8 path: [ceil(K / 128)][sc_rows][4]
+// bytes; sc_rows = rows rounded up to 4, plus 4 (a stage's copy may start up
+// to 3 rows early and is rounded up to 16 bytes).
+inline int mx_sc_rows(int rows) { return ((rows + 3) & ~3) + 4; }
+inline size_t mx_sc_bytes(int rows, int K) { return (size_t)((K + 127) / 128) * mx_sc_rows(rows) * 4; }
+struct MxTokenScales {
+    const uint8_t* xsc;  // x rows, K = H (written by the gather)
+    uint8_t* hsc;        // h rows, K = I (written by the gate/up epilogue)
+    int sc_rows;
+};
 
 // Staged grouped GEMM over every chunk: phase 0 = gate/up + SwiGLU -> h,
 // phase 1 = down -> out[row_slot].
 struct MxMaps;
-// mx: MXFP8 weight maps (MXFP8 path; h is bf16 then), or nullptr (bf16 path).
-cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const GemmShape& sh,
-                              const Chunk* chunks, const int* counts2, void* h_out, void* out,
+// mx: MXFP8 weight maps (MXFP8 path: rows and h are E4M3 with the scale
+// planes of mxs), or nullptr (bf16 path).
+cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const MxTokenScales* mxs,
+                              const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
                               const GemmTuning& tune, cudaStream_t stream);
 

@@ -240,7 +240,7 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     GemmMaps maps;
     if (!encode_gemm_maps(&maps, L.wg, L.wu, L.wd, L.ring, L.h, L.H, L.I, L.E, 2 * L.cap, err))
         return cudaErrorInvalidValue;
-    CoreArgs a;
+    CoreArgs a{};
     a.H = L.H;
     a.I = L.I;
     a.h = L.h;
