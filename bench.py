@@ -136,6 +136,23 @@ class ClockSampler:
                 "samples": len(sm), "period_ms": self.PERIOD_MS}
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (the job is as slow as its slowest
+    rank); the value itself on one process."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def job_rate(units_per_rank: float, ms: float, world: int) -> float:
+    """Whole-job throughput: the units every rank processed over the (max over
+    ranks) time, per second."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ workload
 def algorithmic_work(cfg):
     """Algorithmic bytes / flops of one forward (one step)."""
@@ -249,10 +266,7 @@ def run_mok(args, cfg, rank, world, device):
         torch.distributed.barrier()
     total_ms = start.elapsed_time(stop)
     phases = [[evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j in range(n_ev - 1)]
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = t.item()
+    total_ms = max_over_ranks(total_ms, device)
 
     res = {"total_ms": total_ms, "phases_ms": [sum(ph) / len(ph) for ph in phases], "clocks": clk.summary()}
 
@@ -273,18 +287,13 @@ def run_mok(args, cfg, rank, world, device):
             mok.moe_forward_host(hx, hl, cfg.k, cfg.R, *wts, minibatch, opts, hws, hy)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = t.item()
-        res["e2e_ms"] = e2e_ms
+        res["e2e_ms"] = max_over_ranks(e0.elapsed_time(e1) / n_e2e, device)
         res["h2d"] = cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4
         res["d2h"] = cfg.T * cfg.H * 2
         del hws
-    # plan: route, scan, scatter; staged forward: chunk list, gather, gate/up, down, combine;
+    # plan: top-k, rank, scan, scatter; staged forward: chunk list, gather, gate/up, down, combine;
     # persistent forward: chunk list, one persistent kernel
-    res["launches_per_step"] = (3 + 1 + 1 + 2 + 1) if mode == mok.MOK_MODE_STAGED else (3 + 2)
+    res["launches_per_step"] = (4 + 1 + 1 + 2 + 1) if mode == mok.MOK_MODE_STAGED else (4 + 2)
     res["max_over_mean_load"] = (lambda c: c.max().item() / c.mean().item())(p.counts().float())
     return res
 
@@ -384,7 +393,7 @@ def main():
     peaks, peak_src = load_peaks()
     work = algorithmic_work(cfg)
     ms = res["total_ms"] / args.steps
-    value = cfg.T * world / (ms / 1e3)
+    value = job_rate(cfg.T, ms, world)
     ph = res["phases_ms"]
     line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -430,7 +439,7 @@ def main():
         line["phases_ms"] = {"plan": t_plan, "forward": t_fwd}
         line["phase_rates"] = {"forward_GBps": gbs, "forward_TFLOPs": tflops, "plan_share": t_plan / ms}
     if "e2e_ms" in res:
-        line["e2e"] = {"value": cfg.T * world / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
+        line["e2e"] = {"value": job_rate(cfg.T, res["e2e_ms"], world), "unit": "tokens/s",
                        "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]}
     line["gpu_launches"] = res["launches_per_step"] * args.steps
     if res["clocks"]:

@@ -529,6 +529,28 @@ int mok_gather(const void* const* x_shards, int H, const mok_plan_t* plan, void*
     return MOK_OK;
 }
 
+int mok_mxfp8_scale_rows(int n_rows) { return n_rows < 0 ? 0 : mx_sc_rows(n_rows); }
+
+int mok_gather_mxfp8(const void* const* x_shards, int H, const mok_plan_t* plan, void* rows_q, void* scales,
+                     mok_stream_t stream) {
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if (H <= 0 || H % 128) return fail(MOK_ERR_UNSUPPORTED, "H %% 128 != 0");
+    if (plan->T == 0) return MOK_OK;
+    if (!rows_q || !scales || !all_nonnull(x_shards, plan->R)) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if (!all_aligned16(x_shards, plan->R) || ((reinterpret_cast<uintptr_t>(rows_q) |
+                                               reinterpret_cast<uintptr_t>(scales)) & 15u))
+        return fail(MOK_ERR_UNSUPPORTED, "shard, row and scale pointers must be 16-byte aligned");
+    ShardsIn xs{};
+    for (int r = 0; r < plan->R; ++r) xs.p[r] = x_shards[r];
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_gather_mx(xs, plan->T / plan->R, H, plan->T, plan->k, plan->pos, rows_q, scales,
+                              mx_sc_rows(plan->T * plan->k), sms, reinterpret_cast<cudaStream_t>(stream)),
+             "gather launch");
+    return MOK_OK;
+}
+
 size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E) {
     if (n_rows < 0 || I <= 0 || E <= 0) return 0;
     const int mb = max_minibatches(n_rows, n_rows > 0 ? n_rows : 1);

@@ -8,18 +8,18 @@
 // {src_rank, src_index} table built on the device with no sort and no
 // CPU-GPU traffic.
 //
-// Three launches, all on the caller's stream, nothing read back:
-//   k_route   (T/256 blocks) warp-per-token top-k over the E logits held
-//             in registers (k rounds of a warp arg-max, ties to the lower
-//             index), softmax gates, then stable ranks of each token inside
-//             its block per expert through shared-memory bit masks
-//             (one bit per token of a 32-token warp tile) and per-block
-//             expert histograms.
+// Four launches, all on the caller's stream, nothing read back:
+//   k_topk    (one warp per token, every token in flight at once) top-k
+//             over the E logits held in registers (k rounds of a warp
+//             arg-max, ties to the lower index) and the softmax gates.
+//   k_rank    (T/256 blocks) stable ranks of each token inside its block
+//             per expert through shared-memory bit masks (one bit per token
+//             of a 32-token warp tile) and per-block expert histograms.
 //   k_scan    (1 block) per expert: exclusive prefix of the block
 //             histograms, totals, the exclusive scan over experts ->
 //             counts, offsets.
-//   k_scatter (T/256 blocks) row = offsets[e] + block prefix + rank; writes
-//             the schedule, row_slot and pos.
+//   k_scatter (one thread per slot) row = offsets[e] + block prefix +
+//             rank; writes the schedule, row_slot and pos.
 // The row order inside an expert segment is ascending token index, which
 // makes the schedule deterministic and independent of the launch shape.
 #include "mok_device.cuh"
@@ -36,30 +36,21 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
     return v > bv || (v == bv && e < be);
 }
 
-// dynamic smem: sel[PLAN_TOK][k] int32 | mask[PLAN_WARPS][E] uint32
-__global__ void __launch_bounds__(PLAN_THREADS) k_route(const float* __restrict__ logits, int T, int E, int k,
-                                                        int32_t* __restrict__ topk_idx, float* __restrict__ gates,
-                                                        int32_t* __restrict__ blk_cnt, int32_t* __restrict__ rank_blk) {
-    extern __shared__ __align__(16) unsigned char plan_smem[];
-    int32_t* sel = reinterpret_cast<int32_t*>(plan_smem);
-    uint32_t* mask = reinterpret_cast<uint32_t*>(sel + PLAN_TOK * k);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t_blk = blockIdx.x * PLAN_TOK;
-    const int nc = (E + 31) >> 5;
-
-    // ---- top-k + gates, one token per warp at a time
-    for (int i = 0; i < 32; ++i) {
-        const int lt = warp * 32 + i;
-        const int t = t_blk + lt;
-        if (t >= T) break;
+// One warp per token (grid-stride over tokens).  NC: 32-expert chunks held
+// per lane (ceil(E / 32) <= NC).
+template <int NC>
+__global__ void __launch_bounds__(PLAN_THREADS) k_topk(const float* __restrict__ logits, int T, int E, int k,
+                                                       int32_t* __restrict__ topk_idx, float* __restrict__ gates) {
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * PLAN_WARPS;
+    for (int t = blockIdx.x * PLAN_WARPS + (threadIdx.x >> 5); t < T; t += warps) {
         const float* row = logits + (size_t)t * E;
-        float v[MAX_CHUNKS_PER_LANE];
+        float v[NC];
 #pragma unroll
-        for (int c = 0; c < MAX_CHUNKS_PER_LANE; ++c) {
+        for (int c = 0; c < NC; ++c) {
             const int e = c * 32 + lane;
             float x = -INFINITY;
-            if (c < nc && e < E) {
+            if (e < E) {
                 x = __ldg(row + e);
                 if (x != x) x = -INFINITY;  // NaN compares as -inf
             }
@@ -72,9 +63,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) k_route(const float* __restrict_
             float bv = -INFINITY;
             int be = 0x7fffffff;
 #pragma unroll
-            for (int c = 0; c < MAX_CHUNKS_PER_LANE; ++c) {
+            for (int c = 0; c < NC; ++c) {
                 const int e = c * 32 + lane;
-                if (c < nc && e < E && !((taken >> c) & 1u) && better(v[c], e, bv, be)) {
+                if (e < E && !((taken >> c) & 1u) && better(v[c], e, bv, be)) {
                     bv = v[c];
                     be = e;
                 }
@@ -103,14 +94,26 @@ __global__ void __launch_bounds__(PLAN_THREADS) k_route(const float* __restrict_
         if (lane < k) {
             topk_idx[(size_t)t * k + lane] = my_idx;
             gates[(size_t)t * k + lane] = ex / s;
-            sel[lt * k + lane] = my_idx;
         }
     }
+}
+
+// dynamic smem: sel[PLAN_TOK][k] int32 | mask[PLAN_WARPS][E] uint32
+__global__ void __launch_bounds__(PLAN_THREADS) k_rank(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                                                       int32_t* __restrict__ blk_cnt, int32_t* __restrict__ rank_blk) {
+    extern __shared__ __align__(16) unsigned char plan_smem[];
+    int32_t* sel = reinterpret_cast<int32_t*>(plan_smem);
+    uint32_t* mask = reinterpret_cast<uint32_t*>(sel + PLAN_TOK * k);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t_blk = blockIdx.x * PLAN_TOK;
+    const int n_sel = min(PLAN_TOK, T - t_blk) * k;
+    for (int i = threadIdx.x; i < n_sel; i += PLAN_THREADS) sel[i] = topk_idx[(size_t)t_blk * k + i];
 
     // ---- stable ranks inside the block, per expert
     uint32_t* my_mask = mask + warp * E;
     for (int e = lane; e < E; e += 32) my_mask[e] = 0u;
-    __syncwarp();
+    __syncthreads();
     const int lt = warp * 32 + lane;
     const bool live = (t_blk + lt) < T;
     if (live)
@@ -178,14 +181,11 @@ __global__ void __launch_bounds__(PLAN_THREADS) k_scatter(const int32_t* __restr
                                                           int S_r, int32_t* __restrict__ src_rank,
                                                           int32_t* __restrict__ src_index,
                                                           int32_t* __restrict__ row_slot, int32_t* __restrict__ pos) {
-    const int t0 = blockIdx.x * PLAN_TOK;
-    const int n = min(PLAN_TOK, T - t0) * k;
-    const int32_t* pre = blk_pre + (size_t)blockIdx.x * E;
-    for (int i = threadIdx.x; i < n; i += PLAN_THREADS) {
-        const int s = t0 * k + i;
+    const int ns = T * k;
+    for (int s = blockIdx.x * PLAN_THREADS + threadIdx.x; s < ns; s += gridDim.x * PLAN_THREADS) {
         const int t = s / k;
         const int e = topk_idx[s];
-        const int row = offsets[e] + pre[e] + rank_blk[s];
+        const int row = offsets[e] + blk_pre[(size_t)(t / PLAN_TOK) * E + e] + rank_blk[s];
         src_rank[row] = t / S_r;
         src_index[row] = t - (t / S_r) * S_r;
         row_slot[row] = s;
@@ -220,59 +220,69 @@ size_t plan_layout(int T, int E, int k, PlanLayout* L) {
     return off;
 }
 
-cudaError_t launch_plan(const float* logits, int T, int E, int k, int R, unsigned char* ws, const PlanLayout& L,
-                        cudaStream_t stream) {
-    const size_t smem = sizeof(int32_t) * PLAN_TOK * k + sizeof(uint32_t) * PLAN_WARPS * E;
+// Top-k launch: every token's warp resident at once where the GPU holds them.
+static cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* topk_idx, float* gates,
+                               cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int want = (T + PLAN_WARPS - 1) / PLAN_WARPS;
+    const int grid = want < sms * 8 ? want : sms * 8;
+    const int nc = (E + 31) >> 5;
+    if (nc <= 1) k_topk<1><<<grid, PLAN_THREADS, 0, stream>>>(logits, T, E, k, topk_idx, gates);
+    else if (nc <= 2) k_topk<2><<<grid, PLAN_THREADS, 0, stream>>>(logits, T, E, k, topk_idx, gates);
+    else if (nc <= 4) k_topk<4><<<grid, PLAN_THREADS, 0, stream>>>(logits, T, E, k, topk_idx, gates);
+    else if (nc <= 8) k_topk<8><<<grid, PLAN_THREADS, 0, stream>>>(logits, T, E, k, topk_idx, gates);
+    else if (nc <= 12) k_topk<12><<<grid, PLAN_THREADS, 0, stream>>>(logits, T, E, k, topk_idx, gates);
+    else if (nc <= 16) k_topk<16><<<grid, PLAN_THREADS, 0, stream>>>(logits, T, E, k, topk_idx, gates);
+    else k_topk<MAX_CHUNKS_PER_LANE><<<grid, PLAN_THREADS, 0, stream>>>(logits, T, E, k, topk_idx, gates);
+    return cudaGetLastError();
+}
+
+static cudaError_t rank_configure() {
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_route, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)(sizeof(int32_t) * PLAN_TOK * MOK_MAX_TOPK +
                                                    sizeof(uint32_t) * PLAN_WARPS * MOK_MAX_EXPERTS));
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    auto I32 = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
-    if (T > 0) {
-        k_route<<<L.nb, PLAN_THREADS, smem, stream>>>(logits, T, E, k, I32(L.topk),
-                                                      reinterpret_cast<float*>(ws + L.gates), I32(L.blk_cnt),
-                                                      I32(L.rank));
-    }
-    k_scan<<<1, 1024, 0, stream>>>(I32(L.blk_cnt), L.nb, E, T * k, I32(L.counts), I32(L.offsets));
-    if (T > 0) {
-        k_scatter<<<L.nb, PLAN_THREADS, 0, stream>>>(I32(L.topk), I32(L.rank), I32(L.blk_cnt), I32(L.offsets), T, E,
-                                                     k, T / R, I32(L.src_rank), I32(L.src_index), I32(L.row_slot),
-                                                     I32(L.pos));
-    }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
-// The same three launches with every array given explicitly (outputs and
-// the two scratch arrays: blk_cnt [ceil(T/256), E] and rank [T*k]).
+cudaError_t launch_plan(const float* logits, int T, int E, int k, int R, unsigned char* ws, const PlanLayout& L,
+                        cudaStream_t stream) {
+    auto I32 = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
+    return launch_plan_parts(logits, T, E, k, R, I32(L.counts), I32(L.offsets), I32(L.src_rank), I32(L.src_index),
+                             I32(L.row_slot), I32(L.pos), I32(L.topk), reinterpret_cast<float*>(ws + L.gates),
+                             I32(L.blk_cnt), I32(L.rank), stream);
+}
+
+// The same launches with every array given explicitly (outputs and the two
+// scratch arrays: blk_cnt [ceil(T/256), E] and rank [T*k]).
 int plan_route_blocks(int T) { return (T + PLAN_TOK - 1) / PLAN_TOK; }
 
 cudaError_t launch_plan_parts(const float* logits, int T, int E, int k, int R, int32_t* counts, int32_t* offsets,
                               int32_t* src_rank, int32_t* src_index, int32_t* row_slot, int32_t* pos,
                               int32_t* topk_idx, float* gates, int32_t* blk_cnt, int32_t* rank,
                               cudaStream_t stream) {
+    cudaError_t e = rank_configure();
+    if (e != cudaSuccess) return e;
     const size_t smem = sizeof(int32_t) * PLAN_TOK * k + sizeof(uint32_t) * PLAN_WARPS * E;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_route, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(sizeof(int32_t) * PLAN_TOK * MOK_MAX_TOPK +
-                                                   sizeof(uint32_t) * PLAN_WARPS * MOK_MAX_EXPERTS));
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
     const int nb = plan_route_blocks(T);
-    if (T > 0) k_route<<<nb, PLAN_THREADS, smem, stream>>>(logits, T, E, k, topk_idx, gates, blk_cnt, rank);
+    if ((e = launch_topk(logits, T, E, k, topk_idx, gates, stream)) != cudaSuccess) return e;
+    if (T > 0) k_rank<<<nb, PLAN_THREADS, smem, stream>>>(topk_idx, T, E, k, blk_cnt, rank);
     k_scan<<<1, 1024, 0, stream>>>(blk_cnt, nb, E, T * k, counts, offsets);
-    if (T > 0)
-        k_scatter<<<nb, PLAN_THREADS, 0, stream>>>(topk_idx, rank, blk_cnt, offsets, T, E, k, T / R, src_rank,
-                                                   src_index, row_slot, pos);
+    if (T > 0) {
+        // one thread per slot
+        const int blocks = (T * k + PLAN_THREADS - 1) / PLAN_THREADS;
+        k_scatter<<<blocks < 4096 ? blocks : 4096, PLAN_THREADS, 0, stream>>>(
+            topk_idx, rank, blk_cnt, offsets, T, E, k, T / R, src_rank, src_index, row_slot, pos);
+    }
     return cudaGetLastError();
 }
 

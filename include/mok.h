@@ -269,6 +269,18 @@ const char* mok_last_error_string(void);
 int mok_gather(const void* const* x_shards, int H, const mok_plan_t* plan,
                void* rows, mok_stream_t stream);
 
+/* The MXFP8 gather (what mok_moe_forward's MXFP8 path runs): every row is
+ * quantised in 32-element blocks as mok_mxfp8_quantize_rows does, in the
+ * operand form of the block-scaled MMA:
+ *   rows_q [N_s, H] E4M3 bytes, rows_q[row] = the blocks of the row's token;
+ *   scales [H/128][sc_rows][4] E8M0 bytes: plane g, row r, byte b = the
+ *     scale of block 4g + b of row r; sc_rows = mok_mxfp8_scale_rows(N_s).
+ * H % 128 == 0; rows_q and scales 16-byte aligned.  Source: MoK article,
+ * paragraph on MXFP8 activation quantisation inside the dispatch. */
+int mok_mxfp8_scale_rows(int n_rows);
+int mok_gather_mxfp8(const void* const* x_shards, int H, const mok_plan_t* plan,
+                     void* rows_q, void* scales, mok_stream_t stream);
+
 /* Bytes of scratch for mok_expert_ffn. */
 size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E);
 

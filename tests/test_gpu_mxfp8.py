@@ -134,6 +134,28 @@ def test_mxfp8_forward_full_size_sampled():
     assert rel <= REL_FRO_MX, rel
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_mxfp8_gather_bit_exact(name):
+    """The fused quantising gather: row bytes and scale planes equal the
+    oracle's quantisation of each row's token, bit for bit."""
+    cfg = MX_CASES[name]
+    if cfg.H % 128:
+        cfg = mokgen.scaled(cfg, H=256)
+    x = mokgen.tokens(cfg)
+    logits = mokgen.router_logits(cfg, x)
+    p = mok.plan(logits.cuda(), cfg.k, cfg.R)
+    rows_q, planes = mok.gather_mxfp8(mok.shards(x.cuda(), cfg.R), p)
+    rows_q, planes = rows_q.cpu().numpy(), planes.cpu().numpy()
+    pl = oracle.plan(logits, cfg.k, cfg.R)
+    tok = (pl["src_rank"] * (cfg.T // cfg.R) + pl["src_index"]).numpy()
+    wq, ws = _oracle_quant(x.float().numpy()[tok])
+    ns = cfg.T * cfg.k
+    assert np.array_equal(rows_q.reshape(-1), wq)
+    # planes [H/128][sc_rows][4] -> per row, blocks in order
+    got_s = planes[:, :ns, :].transpose(1, 0, 2).reshape(ns, cfg.H // 32)
+    assert np.array_equal(got_s.reshape(-1), ws)
+
+
 def test_weight_quantiser_bit_exact():
     E, K, N = 3, 256, 192
     w = _spread(E * K, N, seed=9).reshape(E, K, N)
