@@ -136,6 +136,19 @@ class ClockSampler:
                 "samples": len(sm), "period_ms": self.PERIOD_MS}
 
 
+# ------------------------------------------------------------------ measured DRAM traffic
+# dram__bytes_read.sum + dram__bytes_write.sum of the two grouped-GEMM
+# launches of one step, from one ncu capture of a small case of the same
+# kernel, scaled to the full workload by the experts (and rows) processed;
+# the capture, its command and the scaling are in the profiles/ summary
+# named beside each entry.  None where no capture of the current kernel
+# exists for that workload.
+GEMM_TRAFFIC_GB_PER_STEP = {
+    "page": (36.5, "profiles/grouped_gemm_bf16_page_e37.md"),
+    "page_mxfp8": (19.9, "profiles/grouped_gemm_mxfp8_page_e32.md"),
+}
+
+
 # ------------------------------------------------------------------ ranks
 def max_over_ranks(value: float, device) -> float:
     """The largest of every rank's value (the job is as slow as its slowest
@@ -200,19 +213,26 @@ def run_mok(args, cfg, rank, world, device):
     x_shards = mok.shards(dx, cfg.R)
     y = torch.empty_like(dx)
     y_shards = mok.shards(y, cfg.R)
-    mode = mok.MOK_MODE_STAGED if (args.mode == "staged" or cfg.mxfp8) else mok.MOK_MODE_PERSISTENT
+    mode = mok.MOK_MODE_STAGED if args.mode == "staged" else mok.MOK_MODE_PERSISTENT
     opts = mok.fwd_opts(mode=mode, ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8)
     minibatch = args.minibatch or cfg.minibatch
     p = mok.plan(dlogits, cfg.k, cfg.R)
     fws = torch.empty(mok.forward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
                       dtype=torch.uint8, device=device)
-    # the bf16 staged mode is timed one ABI step at a time (per-phase events)
-    staged = mode == mok.MOK_MODE_STAGED and not cfg.mxfp8
+    # staged mode is timed one ABI step at a time (per-phase events)
+    staged = mode == mok.MOK_MODE_STAGED
     if staged:
-        rows = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
         out = torch.empty((cfg.slots, cfg.H), dtype=torch.float32, device=device)
-        ffn_ws = torch.empty(mok.lib().mok_expert_ffn_workspace_bytes(cfg.slots, cfg.I, cfg.E), dtype=torch.uint8,
-                             device=device)
+        if cfg.mxfp8:
+            rows_q = torch.empty((cfg.slots, cfg.H), dtype=torch.uint8, device=device)
+            planes = torch.zeros((cfg.H // 128, mok.lib().mok_mxfp8_scale_rows(cfg.slots), 4), dtype=torch.uint8,
+                                 device=device)
+            ffn_ws = torch.empty(mok.lib().mok_expert_ffn_mxfp8_workspace_bytes(cfg.slots, cfg.I, cfg.E),
+                                 dtype=torch.uint8, device=device)
+        else:
+            rows = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
+            ffn_ws = torch.empty(mok.lib().mok_expert_ffn_workspace_bytes(cfg.slots, cfg.I, cfg.E),
+                                 dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
     # A step in staged mode goes through the ABI one step at a time so that
@@ -227,15 +247,19 @@ def run_mok(args, cfg, rank, world, device):
         if evs:
             evs[1].record(stream)
         if staged:
-            mok.gather(x_shards, p, rows)
+            if pack is not None:
+                mok.gather_mxfp8(x_shards, p, rows_q, planes)
+            else:
+                mok.gather(x_shards, p, rows)
             if evs:
                 evs[2].record(stream)
-            mok.expert_ffn(rows, wg, wu, wd, p, out=out, ws=ffn_ws)
+            if pack is not None:
+                mok.expert_ffn_mxfp8(rows_q, planes, pack, p, out=out, ws=ffn_ws)
+            else:
+                mok.expert_ffn(rows, wg, wu, wd, p, out=out, ws=ffn_ws)
             if evs:
                 evs[3].record(stream)
             mok.combine(out, p, y_shards)
-        elif pack is not None:
-            mok.moe_forward_mxfp8(x_shards, pack, p, y_shards=y_shards, ws=fws)
         else:
             mok.moe_forward(x_shards, wg, wu, wd, p, minibatch, opts, y_shards=y_shards, ws=fws)
         if evs:
@@ -348,6 +372,9 @@ def main():
                     help="profiling case: E experts and T scaled by the same factor (same rows per expert)")
     args = ap.parse_args()
     cfg = mokgen.CONFIGS[args.config]
+    if cfg.mxfp8 and args.mode != "staged":
+        print("the MXFP8 path runs in staged mode only; timing staged mode", file=sys.stderr)
+        args.mode = "staged"
     if args.scale_experts:
         n = args.scale_experts
         T = max(cfg.R, round(cfg.T * n / cfg.E / cfg.R) * cfg.R)
@@ -363,7 +390,7 @@ def main():
              else "bf16 weights [E,H,I]/[E,I,H]")
     config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
               "tokens_per_step_per_gpu": cfg.T, "minibatch": args.minibatch or cfg.minibatch,
-              "mode": "staged" if cfg.mxfp8 else args.mode,
+              "mode": args.mode,
               "l2": f"inputs larger than L2 ({algorithmic_work(cfg)['weight_bytes'] / 1e9:.1f} GB of expert "
                     f"weights streamed per step)"}
 
@@ -404,17 +431,26 @@ def main():
         gemm_s = t_gemm / 1e3
         tflops = work["gemm_flops"] / gemm_s / 1e12
         gbs = work["gemm_bytes"] / gemm_s / 1e9
-        t_tc = work["gemm_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+        # the MMA's own dtype peak: fp8 runs at twice the measured bf16 rate (nominal 4.5 / 2.25 PFLOP/s)
+        tc_peak = peaks["bf16_tflops_sustained"] * (2.0 if cfg.mxfp8 else 1.0)
+        t_tc = work["gemm_flops"] / (tc_peak * 1e12)
         t_hbm = work["gemm_bytes"] / (peaks["hbm_gbs"] * 1e9)
         if t_hbm >= t_tc:
             roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gbs / peaks["hbm_gbs"]}
         else:
-            roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops_sustained"],
-                    "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops_sustained"]}
-        roof.update({"traffic": None, "kernel": "grouped GEMM (gate/up+SwiGLU and down launches)",
+            roof = {"bound": "tensor", "achieved": tflops, "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": tflops / tc_peak}
+        traffic = GEMM_TRAFFIC_GB_PER_STEP.get(cfg.name) if not args.scale_experts else None
+        if traffic and args.mode != "staged" and not cfg.mxfp8:
+            traffic = None
+        roof.update({"traffic": traffic[0] * 1e9 if traffic else None,
+                     "traffic_note": (f"bytes per step, both GEMM launches, scaled from {traffic[1]}" if traffic
+                                      else "no capture of this workload"),
+                     "kernel": "grouped GEMM (gate/up+SwiGLU and down launches)",
                      "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
-                     "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"]})
+                     "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"],
+                     "tensor_frac_of_dtype_peak": tflops / tc_peak})
         line["roofline"] = roof
         line["phases_ms"] = {"plan": t_plan, "gather": t_gather, "grouped_gemm": t_gemm, "combine": t_comb}
         line["phase_rates"] = {
@@ -431,8 +467,7 @@ def main():
         tflops = work["gemm_flops"] / fwd_s / 1e12
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"], "traffic": None,
-                "kernel": ("MXFP8 forward (gather, gate/up+SwiGLU, down, combine launches)" if cfg.mxfp8 else
-                           "persistent forward kernel (dispatch, grouped GEMM, combine in one launch)"),
+                "kernel": "persistent forward kernel (dispatch, grouped GEMM, combine in one launch)",
                 "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
                 "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"]}
         line["roofline"] = roof

@@ -37,7 +37,7 @@ EXPORTS = (
     "mok_get_status", "mok_last_error_string", "mok_gather", "mok_expert_ffn_workspace_bytes",
     "mok_expert_ffn", "mok_combine", "mok_forward_host_workspace_bytes", "mok_moe_forward_host",
     "mok_prepare_w_down", "mok_plan_noalloc", "mok_mxfp8_quantize_rows", "mok_quantize_weights_mxfp8",
-    "mok_mxfp8_scale_rows", "mok_gather_mxfp8",
+    "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8_workspace_bytes", "mok_expert_ffn_mxfp8",
 )
 
 
@@ -92,9 +92,12 @@ def lib() -> ctypes.CDLL:
     L.mok_quantize_weights_mxfp8.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     L.mok_mxfp8_scale_rows.argtypes = [i32]
     L.mok_gather_mxfp8.argtypes = [vp, i32, ctypes.POINTER(PlanT), vp, vp, vp]
+    L.mok_expert_ffn_mxfp8_workspace_bytes.argtypes = [i32, i32, i32]
+    L.mok_expert_ffn_mxfp8_workspace_bytes.restype = sz
+    L.mok_expert_ffn_mxfp8.argtypes = [vp, vp, i32, i32, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
               "mok_moe_forward_host", "mok_prepare_w_down", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
-              "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8"):
+              "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8"):
         getattr(L, n).restype = ctypes.c_int
     return L
 
@@ -290,15 +293,35 @@ def gather(x_shards, p: Plan, rows: torch.Tensor | None = None, stream=None) -> 
     return rows
 
 
-def gather_mxfp8(x_shards, p: Plan, stream=None):
+def gather_mxfp8(x_shards, p: Plan, rows_q=None, scales=None, stream=None):
     """The MXFP8 gather: (rows_q [N_s, H] uint8 E4M3, scales [H/128, sc_rows, 4] uint8 E8M0)."""
     H = x_shards[0].shape[1]
     dev = x_shards[0].device
-    rows_q = torch.empty((p.ns, H), dtype=torch.uint8, device=dev)
-    scales = torch.zeros((H // 128, lib().mok_mxfp8_scale_rows(p.ns), 4), dtype=torch.uint8, device=dev)
+    if rows_q is None:
+        rows_q = torch.empty((p.ns, H), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.zeros((H // 128, lib().mok_mxfp8_scale_rows(p.ns), 4), dtype=torch.uint8, device=dev)
     _check(lib().mok_gather_mxfp8(_ptr_array(x_shards), H, ctypes.byref(p.c), ctypes.c_void_p(rows_q.data_ptr()),
                                   ctypes.c_void_p(scales.data_ptr()), _stream(stream)))
     return rows_q, scales
+
+
+def expert_ffn_mxfp8(rows_q, scales, pack, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
+    """The MXFP8 grouped SwiGLU FFN over mok_gather_mxfp8's output; pack =
+    (qg, sg, qu, su, qd, sd).  Returns (out [T*k, H] fp32 slot-indexed, ws)."""
+    qg, sg, qu, su, qd, sd = pack
+    H = rows_q.shape[1]
+    I = qg.shape[-1]
+    if out is None:
+        out = torch.empty((p.ns, H), dtype=torch.float32, device=rows_q.device)
+    if ws is None:
+        ws = _workspace(lib().mok_expert_ffn_mxfp8_workspace_bytes(p.ns, I, p.c.E), rows_q.device)
+    w = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
+    _check(lib().mok_expert_ffn_mxfp8(ctypes.c_void_p(rows_q.data_ptr()), ctypes.c_void_p(scales.data_ptr()), H, I,
+                                      ctypes.cast(ctypes.byref(w), ctypes.c_void_p), ctypes.byref(p.c),
+                                      ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.c_void_p(out.data_ptr()),
+                                      _stream(stream)))
+    return out, ws
 
 
 def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):

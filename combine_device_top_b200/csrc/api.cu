@@ -590,6 +590,54 @@ int mok_expert_ffn(const void* rows, int H, int I, const void* w_gate, const voi
                           status, kDefaultTimeoutNs, stream);
 }
 
+size_t mok_expert_ffn_mxfp8_workspace_bytes(int n_rows, int I, int E) {
+    if (n_rows < 0 || I <= 0 || E <= 0) return 0;
+    const int mb = max_minibatches(n_rows, n_rows > 0 ? n_rows : 1);
+    const int mc = max_chunks(n_rows, E, mb);
+    return align256(sizeof(DevStatus)) + align256(sizeof(int) * 4) + align256(sizeof(Chunk) * (size_t)mc) +
+           align256(sizeof(Minibatch) * (size_t)mb) + align256((size_t)n_rows * I) + align256(mx_sc_bytes(n_rows, I));
+}
+
+int mok_expert_ffn_mxfp8(const void* rows_q, const void* scales, int H, int I, const mok_mxfp8_weights* w,
+                         const mok_plan_t* plan, void* ws, size_t ws_bytes, void* out, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if ((rc = check_hi(H, I))) return rc;
+    const int ns = plan->T * plan->k;
+    if ((rc = check_ws(ws, ws_bytes, mok_expert_ffn_mxfp8_workspace_bytes(ns, I, plan->E)))) return rc;
+    if (ns == 0) return MOK_OK;
+    if (!rows_q || !scales || !out || !w || !w->gate || !w->gate_scales || !w->up || !w->up_scales || !w->down ||
+        !w->down_scales)
+        return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(rows_q) | reinterpret_cast<uintptr_t>(scales)) & 15u)
+        return fail(MOK_ERR_UNSUPPORTED, "row and scale pointers must be 16-byte aligned");
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    const int mb = max_minibatches(ns, ns);
+    const int mc = max_chunks(ns, plan->E, mb);
+    size_t off = 0;
+    DevStatus* status = reinterpret_cast<DevStatus*>(base + off);
+    off += align256(sizeof(DevStatus));
+    int* counts2 = reinterpret_cast<int*>(base + off);
+    off += align256(sizeof(int) * 4);
+    Chunk* chunks = reinterpret_cast<Chunk*>(base + off);
+    off += align256(sizeof(Chunk) * (size_t)mc);
+    Minibatch* mbs = reinterpret_cast<Minibatch*>(base + off);
+    off += align256(sizeof(Minibatch) * (size_t)mb);
+    void* h = base + off;
+    off += align256((size_t)ns * I);
+    MxTokenScales mxs{};
+    mxs.xsc = static_cast<const uint8_t*>(scales);
+    mxs.hsc = base + off;
+    mxs.sc_rows = mx_sc_rows(ns);
+    MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
+    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, CHUNK_MAX_ROWS_MX, chunks, mc, mbs, mb, counts2,
+                                 status, stream),
+             "work list launch");
+    return run_expert_ffn(rows_q, ns, H, I, nullptr, nullptr, nullptr, plan->E, plan->row_slot, chunks, counts2, h,
+                          out, status, kDefaultTimeoutNs, stream, w, &mxs);
+}
+
 int mok_combine(const void* out, int H, const mok_plan_t* plan, void* const* y_shards, mok_stream_t stream) {
     int rc = check_plan(plan);
     if (rc) return rc;

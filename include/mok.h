@@ -297,6 +297,19 @@ int mok_expert_ffn(const void* rows, int H, int I,
                    const mok_plan_t* plan, void* ws, size_t ws_bytes,
                    void* out, mok_stream_t stream);
 
+/* Bytes of scratch for mok_expert_ffn_mxfp8. */
+size_t mok_expert_ffn_mxfp8_workspace_bytes(int n_rows, int I, int E);
+
+/* The grouped SwiGLU FFN of the MXFP8 path (block-scaled tensor-core MMA)
+ * over the output of mok_gather_mxfp8 (rows_q, scales; same layouts), with
+ * the weight pack `w` (host struct) of mok_quantize_weights_mxfp8.  h is
+ * quantised to MXFP8 in the SwiGLU epilogue and stays in the workspace;
+ * out: [T, k, H] fp32, slot-indexed, as mok_expert_ffn.  Source: MoK
+ * article, paragraph on MXFP8 inside the GEMM and SwiGLU. */
+int mok_expert_ffn_mxfp8(const void* rows_q, const void* scales, int H, int I,
+                         const mok_mxfp8_weights* w, const mok_plan_t* plan,
+                         void* ws, size_t ws_bytes, void* out, mok_stream_t stream);
+
 /* y[t] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]), fp32, j ascending,
  * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] fp32.
  * Source: MoK article, benchmark paragraph (final weighted merge). */

@@ -107,6 +107,26 @@ def test_mxfp8_forward_matches_emulated_oracle(name):
     assert rel <= REL_FRO_MX, rel
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_mxfp8_steps_one_at_a_time_equal_forward(name):
+    """mok_gather_mxfp8 + mok_expert_ffn_mxfp8 + mok_combine compute exactly
+    what mok_moe_forward's MXFP8 path computes."""
+    cfg = MX_CASES[name]
+    x = mokgen.tokens(cfg)
+    logits = mokgen.router_logits(cfg, x)
+    wg, wu, wd = mokgen.all_expert_weights(cfg)
+    pack = _mx_pack(wg.cuda(), wu.cuda(), wd.cuda())
+    p = mok.plan(logits.cuda(), cfg.k, cfg.R)
+    xs = mok.shards(x.cuda(), cfg.R)
+    ys, _ = mok.moe_forward_mxfp8(xs, pack, p)
+    rows_q, planes = mok.gather_mxfp8(xs, p)
+    out, ws = mok.expert_ffn_mxfp8(rows_q, planes, pack, p)
+    assert mok.get_status(ws) == mok.MOK_OK
+    y2 = [torch.empty_like(s) for s in xs]
+    mok.combine(out, p, y2)
+    assert torch.equal(torch.cat([s.cpu() for s in ys]), torch.cat([s.cpu() for s in y2]))
+
+
 @pytest.mark.slow
 def test_mxfp8_forward_full_size_sampled():
     """The page shape on the MXFP8 path: every row computed on the GPU,
