@@ -86,31 +86,37 @@ struct Bf16CfgT {
 using Bf16Cfg = Bf16CfgT<1, 4>;
 using Bf16PairCfg = Bf16CfgT<2, 3>;
 static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share the barrier offset");
-// MXFP8 path (block-scaled tcgen05 MMA, K = 128 per stage):
-// [A E4M3 16 KB][B E4M3 <= 224 rows x 128 B][A scales as loaded 512 B]
-// [B scales as loaded <= 1 KB][A scales, MMA layout 512 B][B scales, MMA
-// layout 1 KB] x 4.
-struct MxCfg {
+// MXFP8 path (block-scaled tcgen05 MMA, K = 128 per stage), SUB weight
+// tiles per unit: [A E4M3 SUB x 16 KB][B E4M3 <= 224 rows x 128 B][A scales
+// as loaded SUB x 512 B][B scales as loaded <= 1 KB][A scales, MMA layout
+// SUB x 512 B][B scales, MMA layout 1 KB] x NST.
+template <int SUB_, int NST_>
+struct MxCfgT {
     static constexpr bool MX = true;
-    static constexpr int SUB = 1;
+    static constexpr int SUB = SUB_;
     static constexpr int THREADS = 224;  // + warp 6: scale-factor layout
-    static constexpr int NST = 4;
+    static constexpr int NST = NST_;
     static constexpr int BKX = 128;      // K per stage
-    static constexpr int A_OFF = 0, B_OFF = 16384;
-    static constexpr int SFA_RAW_OFF = B_OFF + CHUNK_MAX_ROWS_MX * 128;  // [4 K blocks][128 rows]
-    static constexpr int SFB_RAW_OFF = SFA_RAW_OFF + 512;                // [rows][4 K blocks], 16-byte aligned copy
-    static constexpr int SFA_OFF = SFB_RAW_OFF + 1024;                   // one 512-byte scale atom
-    static constexpr int SFB_OFF = SFA_OFF + 512;                        // two atoms (rows 0-127, 128-255)
+    static constexpr int A_OFF = 0, B_OFF = SUB * 16384;
+    static constexpr int SFA_RAW_OFF = B_OFF + CHUNK_MAX_ROWS_MX * 128;  // per tile [4 K blocks][128 rows]
+    static constexpr int SFB_RAW_OFF = SFA_RAW_OFF + SUB * 512;          // [rows][4 K blocks], 16-byte aligned copy
+    static constexpr int SFA_OFF = SFB_RAW_OFF + 1024;                   // one 512-byte scale atom per tile
+    static constexpr int SFB_OFF = SFA_OFF + SUB * 512;                  // two atoms (rows 0-127, 128-255)
     static constexpr int STAGE = SFB_OFF + 1024;
     static constexpr int EPI_OFF = NST * STAGE;
     static constexpr int XCH_OFF = EPI_OFF + EPI_BYTES;  // amax exchange of the h quantiser
     static constexpr int BAR_OFF = XCH_OFF + 512;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
-    // TMEM: accumulators at columns 0 and 256 (N <= 224), scale factors above
-    static constexpr uint32_t TM_SFA = 480, TM_SFB = 484;
+    // TMEM: accumulators in columns [0, 480) (N <= 224), then the scale
+    // factors of the SUB weight tiles (4 columns each) and of the tokens (8)
+    static constexpr uint32_t TM_SFA = 480, TM_SFB = 480 + 4 * SUB;
+    static_assert(STAGE % 1024 == 0, "MXFP8 stages must keep 1024-byte alignment");
+    static_assert(SMEM <= 232448, "MXFP8 layout exceeds shared memory");
+    static_assert(TM_SFB + 8 <= 512, "scale factors must fit in TMEM");
 };
-static_assert(MxCfg::STAGE % 1024 == 0, "MXFP8 stages must keep 1024-byte alignment");
-static_assert(MxCfg::SMEM <= 232448, "MXFP8 layout exceeds shared memory");
+using MxCfg = MxCfgT<1, 4>;
+using MxPairCfg = MxCfgT<2, 3>;
+
 // Shared-memory layout used by code outside the GEMM roles (dispatch CTAs of
 // the persistent kernel place their row slots below SMEM_BAR_OFF).
 constexpr int GEMM_THREADS = Bf16Cfg::THREADS;
@@ -222,7 +228,7 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
         const int sc_lead = u.brow0 & 3;
         const uint32_t sc_bytes = (uint32_t)(4 * (sc_lead + u.rows) + 15) & ~15u;
         if (C::MX)
-            bytes += 16384 + 512 + sc_bytes;  // E4M3 weight tile + its scales + the token scales
+            bytes += (uint32_t)nsub * (16384 + 512) + sc_bytes;  // E4M3 weight tiles + their scales + token scales
         else
             bytes += (uint32_t)nsub * A_BYTES;
         bool ok = true;
@@ -235,21 +241,24 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
             mbar_arrive_expect_tx(&full[stage], bytes);
             const int ky = u.expert * K + kb * C::BKX;
             if constexpr (C::MX) {
-                unsigned char* sfa = st + MxCfg::SFA_RAW_OFF;
                 const int kys = ky / 32;  // scale row of the stage's first K block
-                if (u.phase == 0) {
-                    // gate and up columns of the M tile: two 64-byte-swizzled 64-column boxes
-                    tma_load_2d_hint(st + MxCfg::A_OFF, &mx->gq, &full[stage], u.m * MT_G_FEATURES, ky, evict_first);
-                    tma_load_2d_hint(st + MxCfg::A_OFF + 8192, &mx->uq, &full[stage], u.m * MT_G_FEATURES, ky,
-                                     evict_first);
-                    tma_load_2d(sfa, &mx->gs, &full[stage], u.m * MT_G_FEATURES, kys);
-                    tma_load_2d(sfa + 256, &mx->us, &full[stage], u.m * MT_G_FEATURES, kys);
-                } else {
-                    tma_load_2d_hint(st + MxCfg::A_OFF, &mx->dq, &full[stage], u.m * MT_D_FEATURES, ky, evict_first);
-                    tma_load_2d(sfa, &mx->ds, &full[stage], u.m * MT_D_FEATURES, kys);
+                for (int sub = 0; sub < nsub; ++sub) {
+                    unsigned char* sa = st + C::A_OFF + sub * 16384;
+                    unsigned char* sfa = st + C::SFA_RAW_OFF + sub * 512;
+                    const int mt = u.m * C::SUB + sub;
+                    if (u.phase == 0) {
+                        // gate and up columns of the M tile: two 64-byte-swizzled 64-column boxes
+                        tma_load_2d_hint(sa, &mx->gq, &full[stage], mt * MT_G_FEATURES, ky, evict_first);
+                        tma_load_2d_hint(sa + 8192, &mx->uq, &full[stage], mt * MT_G_FEATURES, ky, evict_first);
+                        tma_load_2d(sfa, &mx->gs, &full[stage], mt * MT_G_FEATURES, kys);
+                        tma_load_2d(sfa + 256, &mx->us, &full[stage], mt * MT_G_FEATURES, kys);
+                    } else {
+                        tma_load_2d_hint(sa, &mx->dq, &full[stage], mt * MT_D_FEATURES, ky, evict_first);
+                        tma_load_2d(sfa, &mx->ds, &full[stage], mt * MT_D_FEATURES, kys);
+                    }
                 }
                 const uint8_t* plane = (u.phase == 0 ? a.xsc : a.hsc) + (size_t)kb * a.sc_rows * 4;
-                bulk_load(st + MxCfg::SFB_RAW_OFF, plane + (size_t)(u.brow0 - sc_lead) * 4, sc_bytes, &full[stage]);
+                bulk_load(st + C::SFB_RAW_OFF, plane + (size_t)(u.brow0 - sc_lead) * 4, sc_bytes, &full[stage]);
             } else {
                 for (int sub = 0; sub < nsub; ++sub) {
                     unsigned char* sa = st + C::A_OFF + sub * A_BYTES;
@@ -295,7 +304,7 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
 //   tokens (B): loaded [rows][4 K blocks] starting sc_lead rows early; rows
 //     past the chunk get scale 0 (their MMA columns are never stored);
 //     rows 128-255 form a second atom.
-template <class S>
+template <class S, class C>
 __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* full,
                                                uint64_t* sfready) {
     const int lane = threadIdx.x & 31;
@@ -304,7 +313,8 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
         const int K = u.phase == 0 ? a.H : a.I;
-        const int KB = (K + MxCfg::BKX - 1) / MxCfg::BKX;
+        const int KB = (K + C::BKX - 1) / C::BKX;
+        const int nsub = unit_subs<C>(a, u);
         const int lead = u.brow0 & 3;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
@@ -312,20 +322,23 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
                 ok = false;
                 break;
             }
-            unsigned char* st = smem + stage * MxCfg::STAGE;
-            const uint8_t* ra = st + MxCfg::SFA_RAW_OFF;
-            const uint32_t* rb = reinterpret_cast<const uint32_t*>(st + MxCfg::SFB_RAW_OFF) + lead;
-            uint32_t wa[4];
+            unsigned char* st = smem + stage * C::STAGE;
+            const uint32_t* rb = reinterpret_cast<const uint32_t*>(st + C::SFB_RAW_OFF) + lead;
+            for (int sub = 0; sub < nsub; ++sub) {
+                const uint8_t* ra = st + C::SFA_RAW_OFF + sub * 512;
+                uint32_t wa[4];
 #pragma unroll
-            for (int r1 = 0; r1 < 4; ++r1) {
-                const int r = lane + 32 * r1;
-                // feature r of the tile: gate/up keeps 64 gate then 64 up rows of 64 bytes
-                const uint8_t* col = u.phase == 0 ? ra + (r >> 6) * 256 + (r & 63) : ra + r;
-                const int pitch = u.phase == 0 ? 64 : 128;
-                wa[r1] = (uint32_t)col[0] | ((uint32_t)col[pitch] << 8) | ((uint32_t)col[2 * pitch] << 16) |
-                         ((uint32_t)col[3 * pitch] << 24);
+                for (int r1 = 0; r1 < 4; ++r1) {
+                    const int r = lane + 32 * r1;
+                    // feature r of the tile: gate/up keeps 64 gate then 64 up rows of 64 bytes
+                    const uint8_t* col = u.phase == 0 ? ra + (r >> 6) * 256 + (r & 63) : ra + r;
+                    const int pitch = u.phase == 0 ? 64 : 128;
+                    wa[r1] = (uint32_t)col[0] | ((uint32_t)col[pitch] << 8) | ((uint32_t)col[2 * pitch] << 16) |
+                             ((uint32_t)col[3 * pitch] << 24);
+                }
+                *reinterpret_cast<uint4*>(st + C::SFA_OFF + sub * 512 + 16 * lane) =
+                    make_uint4(wa[0], wa[1], wa[2], wa[3]);
             }
-            *reinterpret_cast<uint4*>(st + MxCfg::SFA_OFF + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
 #pragma unroll
             for (int r2 = 0; r2 < 2; ++r2) {
                 uint32_t wb[4];
@@ -334,12 +347,12 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
                     const int r = lane + 32 * r1 + 128 * r2;
                     wb[r1] = r < u.rows ? rb[r] : 0u;
                 }
-                *reinterpret_cast<uint4*>(st + MxCfg::SFB_OFF + 512 * r2 + 16 * lane) =
+                *reinterpret_cast<uint4*>(st + C::SFB_OFF + 512 * r2 + 16 * lane) =
                     make_uint4(wb[0], wb[1], wb[2], wb[3]);
             }
             fence_proxy_async_shared();  // generic writes -> the TMEM copy (async proxy) reads
             mbar_arrive(&sfready[stage]);
-            if (++stage == MxCfg::NST) {
+            if (++stage == C::NST) {
                 stage = 0;
                 phase ^= 1u;
             }
@@ -354,7 +367,13 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
 // A unit whose M tiles fit in one buffer (one tile, or two tiles of N <= 128
 // columns: tile s at column 128 s) takes one ticket; two tiles of N > 128
 // take two consecutive tickets, one buffer each.
-__device__ __forceinline__ int unit_tickets(int nsub, int N) { return (nsub == 2 && N > 128) ? 2 : 1; }
+// A pair of tiles fits one buffer up to N = 128 columns each; the MXFP8
+// path stops at 96 so that buffer 1's second tile ends below its scale
+// factors (column 480).
+template <class C>
+__device__ __forceinline__ int unit_tickets(int nsub, int N) {
+    return (nsub == 2 && N > (C::MX ? 96 : 128)) ? 2 : 1;
+}
 __device__ __forceinline__ uint32_t acc_col(uint32_t tk, int sub, bool wide) {
     return wide ? ((tk + (uint32_t)sub) & 1u) * ACC_COLS : (tk & 1u) * ACC_COLS + (uint32_t)sub * 128u;
 }
@@ -374,7 +393,7 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
         const int KB = (K + C::BKX - 1) / C::BKX;
         const int N = (u.rows + 15) & ~15;
         const int nsub = unit_subs<C>(a, u);
-        const int nt = unit_tickets(nsub, N);
+        const int nt = unit_tickets<C>(nsub, N);
         const bool wide = nt == 2;
         // bf16 path: gate/up bf16 x bf16, down fp16 x fp16
         const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, u.phase == 0 ? 1 : 0);
@@ -396,22 +415,27 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
             if constexpr (C::MX) {
                 // scale factors of this stage into TMEM (executed in order with the MMAs)
                 unsigned char* st = smem + stage * C::STAGE;
-                tmem_cp_32x128b_warpx4(tmem_base + MxCfg::TM_SFA, st + MxCfg::SFA_OFF);
-                tmem_cp_32x128b_warpx4(tmem_base + MxCfg::TM_SFB, st + MxCfg::SFB_OFF);
-                if (N > 128) tmem_cp_32x128b_warpx4(tmem_base + MxCfg::TM_SFB + 4, st + MxCfg::SFB_OFF + 512);
+                for (int sub = 0; sub < nsub; ++sub)
+                    tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFA + 4 * sub, st + C::SFA_OFF + sub * 512);
+                tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFB, st + C::SFB_OFF);
+                if (N > 128) tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFB + 4, st + C::SFB_OFF + 512);
                 const int nks = min(4, (K - kb * C::BKX) / 32);  // 32 K values per MMA
                 for (int ks = 0; ks < nks; ++ks) {
-                    // A: MN-major E4M3; gate/up = two 64-byte-swizzled 64-column halves 8 KB
-                    //    apart (8-row K groups 512 bytes apart), down = one 128-byte-swizzled
-                    //    128-column tile (K groups 1 KB apart); 32 K rows per MMA.
-                    const uint64_t ad = u.phase == 0 ? umma_desc(sa + ks * 2048, 8192, 512, UMMA_LAYOUT_SW64)
-                                                     : umma_desc(sa + ks * 4096, 0, 1024, UMMA_LAYOUT_SW128);
                     // B: K-major E4M3 SW128, 32 K = 32 bytes inside the atom
                     const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
                     const uint32_t sel = (uint32_t)ks << 30;  // scale byte of these 32 K values
-                    umma_mxf8(tmem_base + acc_col(tk, 0, false), ad, bd, umma_idesc_mxf8(128, N, 1, 0, (uint32_t)ks),
-                              tmem_base + MxCfg::TM_SFA + sel, tmem_base + MxCfg::TM_SFB + sel,
-                              (kb | ks) != 0 ? 1u : 0u);
+                    const uint32_t idx = umma_idesc_mxf8(128, N, 1, 0, (uint32_t)ks);
+                    for (int sub = 0; sub < nsub; ++sub) {
+                        // A: MN-major E4M3; gate/up = two 64-byte-swizzled 64-column halves 8 KB
+                        //    apart (8-row K groups 512 bytes apart), down = one 128-byte-swizzled
+                        //    128-column tile (K groups 1 KB apart); 32 K rows per MMA.
+                        const uint32_t a0 = sa + sub * 16384;
+                        const uint64_t ad = u.phase == 0 ? umma_desc(a0 + ks * 2048, 8192, 512, UMMA_LAYOUT_SW64)
+                                                         : umma_desc(a0 + ks * 4096, 0, 1024, UMMA_LAYOUT_SW128);
+                        umma_mxf8(tmem_base + acc_col(tk, sub, wide), ad, bd, idx,
+                                  tmem_base + C::TM_SFA + 4 * sub + sel, tmem_base + C::TM_SFB + sel,
+                                  (kb | ks) != 0 ? 1u : 0u);
+                    }
                 }
             } else {
 #pragma unroll
@@ -537,7 +561,7 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
     Unit u;
     for (int i = 0; ok && s.get(i, u); ++i) {
         const int nsub = unit_subs<C>(a, u);
-        const int nt = unit_tickets(nsub, (u.rows + 15) & ~15);
+        const int nt = unit_tickets<C>(nsub, (u.rows + 15) & ~15);
         const bool wide = nt == 2;
         for (int sub = 0; sub < nsub && ok; ++sub) {
             const uint32_t tkt = wide ? tk + (uint32_t)sub : tk;
@@ -636,7 +660,7 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
     } else if (warp < 6) {
         gemm_epilogue<S, C>(a, s, smem, tfull, tempty, ok_flag, tmem_base);
     } else if constexpr (C::MX) {
-        gemm_sf_layout(a, s, smem, full, sfready);
+        gemm_sf_layout<S, C>(a, s, smem, full, sfready);
     }
 
     tc_fence_before();

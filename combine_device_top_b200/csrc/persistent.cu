@@ -117,7 +117,9 @@ struct PersistSched {
     }
 };
 
-template <int KMAX>
+// C: the GEMM CTAs' configuration (one M tile per unit, or pairs); both
+// share the thread count and shared-memory layout the dispatch side uses.
+template <int KMAX, class C>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_moe_persistent(const __grid_constant__ GemmMaps maps, const CoreArgs a, const __grid_constant__ PersistParams p) {
     extern __shared__ unsigned char smem_raw[];
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         s.gidx = blockIdx.x - D;
         s.gctas = gridDim.x - D;
         s.total = nch * (p.MTG + p.MTD);
-        gemm_cta<PersistSched, Bf16Cfg>(maps, nullptr, a, s, smem);
+        gemm_cta<PersistSched, C>(maps, nullptr, a, s, smem);
     }
 
     // -------------------------------------------- combine, once every down unit is done
@@ -211,28 +213,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
 }
 
-template <int KMAX>
+template <int KMAX, class C>
 static cudaError_t launch_persistent_k(int grid, const GemmMaps& maps, const CoreArgs& a, const PersistParams& p,
                                        cudaStream_t stream) {
+    static_assert(C::THREADS == GEMM_THREADS && C::SMEM == SMEM_ALLOC && C::BAR_OFF == SMEM_BAR_OFF,
+                  "the dispatch side assumes the GEMM side's block shape");
     static bool attr[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr[dev]) {
-        e = cudaFuncSetAttribute(k_moe_persistent<KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+        e = cudaFuncSetAttribute(k_moe_persistent<KMAX, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
         if (e != cudaSuccess) return e;
         attr[dev] = true;
     }
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_moe_persistent<KMAX>, GEMM_THREADS, SMEM_ALLOC);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_moe_persistent<KMAX, C>, GEMM_THREADS, SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     if (per_sm < 1 || grid > per_sm * sms) return cudaErrorCooperativeLaunchTooLarge;
     void* args[] = {const_cast<GemmMaps*>(&maps), const_cast<CoreArgs*>(&a), const_cast<PersistParams*>(&p)};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_moe_persistent<KMAX>), dim3(grid),
+    return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_moe_persistent<KMAX, C>), dim3(grid),
                                        dim3(GEMM_THREADS), args, SMEM_ALLOC, stream);
 }
 
@@ -253,9 +257,12 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.mbs = L.mbs;
     p.counts2 = L.counts2;
     p.cap = L.cap;
-    // units per chunk: pairs of M tiles (the last one may be single)
-    p.MTG = (L.I / MT_G_FEATURES + Bf16Cfg::SUB - 1) / Bf16Cfg::SUB;
-    p.MTD = (L.H / MT_D_FEATURES + Bf16Cfg::SUB - 1) / Bf16Cfg::SUB;
+    // the staged GEMM's rule for M-tile pairs: mean rows per expert <= 192
+    const bool pair = gemm_tuning(L.T * L.k, L.E).pair != 0;
+    const int sub = pair ? Bf16PairCfg::SUB : Bf16Cfg::SUB;
+    // units per chunk (with pairs the last one may be single)
+    p.MTG = (L.I / MT_G_FEATURES + sub - 1) / sub;
+    p.MTD = (L.H / MT_D_FEATURES + sub - 1) / sub;
     p.dispatch_ctas = L.dispatch_ctas;
     p.gathered = L.gathered;
     p.d_done = L.d_done;
@@ -271,8 +278,12 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.gates = L.gates;
     p.ring = reinterpret_cast<__nv_bfloat16*>(L.ring);
     *err = "persistent launch";
-    if (L.k <= 2) return launch_persistent_k<2>(L.grid, maps, a, p, stream);
-    return launch_persistent_k<8>(L.grid, maps, a, p, stream);
+    if (pair) {
+        if (L.k <= 2) return launch_persistent_k<2, Bf16PairCfg>(L.grid, maps, a, p, stream);
+        return launch_persistent_k<8, Bf16PairCfg>(L.grid, maps, a, p, stream);
+    }
+    if (L.k <= 2) return launch_persistent_k<2, Bf16Cfg>(L.grid, maps, a, p, stream);
+    return launch_persistent_k<8, Bf16Cfg>(L.grid, maps, a, p, stream);
 }
 
 }  // namespace mok
