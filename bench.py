@@ -323,12 +323,13 @@ def run_mok(args, cfg, rank, world, device):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def cpu_oracle_sample(cfg, budget_s: float = 12.0):
+def cpu_oracle_sample(cfg, budget_s: float = 12.0, threads: int = 0):
     """Oracle expert FFN on whole experts of the workload, experts 0, 1, ...
-    until about budget_s seconds of CPU work; returns tokens/s (= rows/s / k)."""
+    until about budget_s seconds of CPU work, on `threads` host threads (0:
+    every core this process may use); returns tokens/s (= rows/s / k)."""
     import oracle
 
-    cores = len(os.sched_getaffinity(0))
+    cores = threads if threads > 0 else len(os.sched_getaffinity(0))
     oracle.set_num_threads(cores)
     x = mokgen.tokens(cfg)
     logits = mokgen.router_logits(cfg, x)
@@ -482,6 +483,7 @@ def main():
     line["expert_load_max_over_mean"] = res["max_over_mean_load"]
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_oracle_sample(cfg, args.cpu_budget)
+        line["cpu_baseline_1thread"] = cpu_oracle_sample(cfg, args.cpu_budget / 2, threads=1)
     print(json.dumps(line), flush=True)
     return 0
 

@@ -115,7 +115,6 @@ struct MxCfgT {
     static_assert(TM_SFB + 8 <= 512, "scale factors must fit in TMEM");
 };
 using MxCfg = MxCfgT<1, 4>;
-using MxPairCfg = MxCfgT<2, 3>;
 
 // Shared-memory layout used by code outside the GEMM roles (dispatch CTAs of
 // the persistent kernel place their row slots below SMEM_BAR_OFF).

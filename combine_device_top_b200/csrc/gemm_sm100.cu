@@ -50,9 +50,7 @@ cudaError_t gemm_configure(int dev) {
                                  Bf16PairCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm<MxCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, MxCfg::SMEM);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_grouped_gemm<MxPairCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 MxPairCfg::SMEM);
+
     if (e == cudaSuccess) done[dev] = true;
     return e;
 }
@@ -76,16 +74,16 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
     const int tiles = phase == 0 ? sh.I / MT_G_FEATURES : sh.H / MT_D_FEATURES;
-    const int sub = tune.pair ? 2 : 1;
+    // MXFP8 keeps one tile per unit: measured, pairs were 9-10 % slower there
+    // (a tall pair fills TMEM, and its heavier quantising epilogue then
+    // stalls the next unit's MMAs)
+    const bool pair = tune.pair && !mx;
+    const int sub = pair ? 2 : 1;
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
     if (mx) {
-        if (tune.pair)
-            k_grouped_gemm<MxPairCfg><<<grid, MxPairCfg::THREADS, MxPairCfg::SMEM, stream>>>(
-                maps, *mx, a, chunks, counts2, phase, MT, GC);
-        else
-            k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2,
-                                                                                phase, MT, GC);
+        k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,
+                                                                            MT, GC);
     } else {
         MxMaps none;
         memset(&none, 0, sizeof none);

@@ -127,27 +127,6 @@ def test_mxfp8_steps_one_at_a_time_equal_forward(name):
     assert torch.equal(torch.cat([s.cpu() for s in ys]), torch.cat([s.cpu() for s in y2]))
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "page_like"])
-def test_mxfp8_m_tile_pairing_is_exact(name, monkeypatch):
-    """Units of one weight tile and pairs of tiles sharing each token tile
-    (one TMEM buffer for pairs up to 96 rows, two above, a single tile at an
-    odd end of the M range) issue the same MMAs per tile: bit-identical."""
-    cfg = MX_CASES[name]
-    x = mokgen.tokens(cfg)
-    logits = mokgen.router_logits(cfg, x)
-    wg, wu, wd = mokgen.all_expert_weights(cfg)
-    pack = _mx_pack(wg.cuda(), wu.cuda(), wd.cuda())
-    p = mok.plan(logits.cuda(), cfg.k, cfg.R)
-    rows_q, planes = mok.gather_mxfp8(mok.shards(x.cuda(), cfg.R), p)
-    got = {}
-    for pair in ("0", "1"):
-        monkeypatch.setenv("MOK_GEMM_PAIR", pair)
-        out, ws = mok.expert_ffn_mxfp8(rows_q, planes, pack, p)
-        assert mok.get_status(ws) == mok.MOK_OK
-        got[pair] = out.cpu()
-    assert torch.equal(got["0"], got["1"])
-
-
 @pytest.mark.slow
 def test_mxfp8_forward_full_size_sampled():
     """The page shape on the MXFP8 path: every row computed on the GPU,
