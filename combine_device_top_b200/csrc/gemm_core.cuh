@@ -54,8 +54,8 @@ constexpr int BK = 64;                            // K per stage: one 128-byte s
 constexpr int A_BYTES = 128 * BK * 2;             // 16 KB: two {64 MN x 64 K} bf16/fp16 halves
 constexpr int B_ROW_BYTES = BK * 2;               // 128 bytes of one token row per stage
 constexpr int B_BYTES = CHUNK_MAX_ROWS * B_ROW_BYTES;  // 32 KB
-constexpr int EPI_LD = 33;                        // fp32 staging row pitch (bank-conflict free)
-constexpr int EPI_BYTES = 128 * EPI_LD * 4;
+constexpr int EPI_TLD = 132;                      // fp32 staging pitch: 32 tokens x 128 features (+4)
+constexpr int EPI_BYTES = 32 * EPI_TLD * 4;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 // Bound of the waits that drain this CTA's own TMA loads and MMAs before it
@@ -79,8 +79,7 @@ struct Bf16CfgT {
     static constexpr int STAGE = SUB * A_BYTES + B_BYTES;
     static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
     static constexpr int EPI_OFF = NST * STAGE;
-    static constexpr int XCH_OFF = EPI_OFF + EPI_BYTES;  // unused
-    static constexpr int BAR_OFF = XCH_OFF;
+    static constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + slack for 1024-byte alignment
 };
 using Bf16Cfg = Bf16CfgT<1, 4>;
@@ -104,8 +103,7 @@ struct MxCfgT {
     static constexpr int SFB_OFF = SFA_OFF + SUB * 512;                  // two atoms (rows 0-127, 128-255)
     static constexpr int STAGE = SFB_OFF + 1024;
     static constexpr int EPI_OFF = NST * STAGE;
-    static constexpr int XCH_OFF = EPI_OFF + EPI_BYTES;  // amax exchange of the h quantiser
-    static constexpr int BAR_OFF = XCH_OFF + 512;
+    static constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
     // TMEM: accumulators in columns [0, 480) (N <= 224), then the scale
     // factors of the SUB weight tiles (4 columns each) and of the tokens (8)
@@ -468,80 +466,84 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
 }
 
 // ------------------------------------------------------------------ epilogue (warps 2..5)
-// Drains one M tile's accumulator (TMEM columns col0 .. col0 + rows) through
-// shared memory: SwiGLU -> h rows (gate/up) or fp32 rows pushed to the
-// tokens' slots (down).
+// Drains one M tile's accumulator (TMEM columns col0 .. col0 + rows), 32
+// tokens at a time, through a token-major staging tile in shared memory
+// (epi[token][feature], pitch EPI_TLD), so that every global store is a
+// row-contiguous run: gate/up writes h rows (8 lanes per 64-feature row),
+// down pushes 512-byte fp32 rows (a warp per row) to the tokens' slots.
 template <class C>
 __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u, int mt, uint32_t col0, float* epi,
-                                               float* xch, uint32_t tmem_base) {
+                                               uint32_t tmem_base) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp & 3;           // TMEM lane quadrant this warp may access
-    const int et = threadIdx.x - 64;  // 0..127
-    const int tok = et & 31, fq = et >> 5;
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access: features q*32 .. q*32+31
     const int ncc = (u.rows + 31) >> 5;
     for (int cc = 0; cc < ncc; ++cc) {
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + col0 + (uint32_t)(cc * 32), v);
-        float* myrow = epi + (q * 32 + lane) * EPI_LD;
+        // token-major: lanes hold consecutive features, so each store row is contiguous
 #pragma unroll
-        for (int k = 0; k < 32; ++k) myrow[k] = v[k];
+        for (int t = 0; t < 32; ++t) epi[t * EPI_TLD + q * 32 + lane] = v[t];
         named_bar_sync(1, 128);
-        const int col = cc * 32 + tok;
-        const bool live = col < u.rows;
         if (u.phase == 0) {
-            // features mt*64 + fq*16 .. +15: gate rows fq*16+k, up rows 64+fq*16+k
-            float hv[16];
+            // h features mt*64 + j: gate in staging columns j, up in 64 + j.  Lane
+            // group g = lane / 8 takes token rows; lane % 8 owns 8 features.
+            const int j0 = (lane & 7) * 8;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float g = epi[(fq * 16 + k) * EPI_LD + tok];
-                const float up = epi[(64 + fq * 16 + k) * EPI_LD + tok];
-                hv[k] = g / (1.0f + __expf(-g)) * up;
-            }
-            if constexpr (C::MX) {
-                // MXFP8 h: blocks of 32 features = thread pairs fq ^ 1 (same token);
-                // E4M3 bytes to h, the block's E8M0 byte to its scale plane
-                float amax = 0.f;
+            for (int it = 0; it < 2; ++it) {
+                const int t = it * 16 + q * 4 + (lane >> 3);  // token of this chunk
+                const float* er = epi + t * EPI_TLD;
+                const float4 g0 = *reinterpret_cast<const float4*>(er + j0);
+                const float4 g1 = *reinterpret_cast<const float4*>(er + j0 + 4);
+                const float4 u0 = *reinterpret_cast<const float4*>(er + 64 + j0);
+                const float4 u1 = *reinterpret_cast<const float4*>(er + 64 + j0 + 4);
+                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                float hv[8];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(hv[k]));
-                xch[fq * 32 + tok] = amax;
-                named_bar_sync(1, 128);
-                amax = fmaxf(amax, xch[(fq ^ 1) * 32 + tok]);
-                const int sx = mx_block_exponent(amax);
-                const float inv = mx_pow2(-sx);
-                uint32_t pq[4];
+                for (int k = 0; k < 8; ++k) hv[k] = gv[k] / (1.0f + __expf(-gv[k])) * uv[k];
+                const int col = cc * 32 + t;
+                const bool live = col < u.rows;
+                const size_t row = (size_t)(u.brow0 + col);
+                if constexpr (C::MX) {
+                    // MXFP8 h: a 32-feature block = 4 lanes of one row (lane % 8 in 0-3 or 4-7)
+                    float amax = 0.f;
 #pragma unroll
-                for (int k = 0; k < 16; k += 4)
-                    pq[k >> 2] = (uint32_t)mx_e4m3x2(hv[k] * inv, hv[k + 1] * inv) |
-                                 ((uint32_t)mx_e4m3x2(hv[k + 2] * inv, hv[k + 3] * inv) << 16);
-                if (live) {
-                    const size_t row = (size_t)(u.brow0 + col);
-                    *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.h) + row * a.I + mt * MT_G_FEATURES +
-                                              fq * 16) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
-                    if ((fq & 1) == 0) {
-                        const int b = 2 * mt + (fq >> 1);  // 32-feature block along I
-                        a.hsc[((size_t)(b >> 2) * a.sc_rows + row) * 4 + (b & 3)] = (uint8_t)(sx + 127);
+                    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(hv[k]));
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                    const int sx = mx_block_exponent(amax);
+                    const float inv = mx_pow2(-sx);
+                    const uint2 pq = make_uint2((uint32_t)mx_e4m3x2(hv[0] * inv, hv[1] * inv) |
+                                                    ((uint32_t)mx_e4m3x2(hv[2] * inv, hv[3] * inv) << 16),
+                                                (uint32_t)mx_e4m3x2(hv[4] * inv, hv[5] * inv) |
+                                                    ((uint32_t)mx_e4m3x2(hv[6] * inv, hv[7] * inv) << 16));
+                    if (live) {
+                        *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.h) + row * a.I + mt * MT_G_FEATURES +
+                                                  j0) = pq;
+                        if ((lane & 3) == 0) {
+                            const int b = 2 * mt + ((lane & 7) >> 2);  // 32-feature block along I
+                            a.hsc[((size_t)(b >> 2) * a.sc_rows + row) * 4 + (b & 3)] = (uint8_t)(sx + 127);
+                        }
                     }
-                }
-            } else {
-                uint32_t pk[8];
-#pragma unroll
-                for (int k = 0; k < 16; k += 2) pk[k >> 1] = pack_half2_sat(hv[k], hv[k + 1]);
-                if (live) {
-                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) +
-                                                          (size_t)(u.brow0 + col) * a.I + mt * MT_G_FEATURES + fq * 16);
-                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                } else {
+                    const uint4 pk = make_uint4(pack_half2_sat(hv[0], hv[1]), pack_half2_sat(hv[2], hv[3]),
+                                                pack_half2_sat(hv[4], hv[5]), pack_half2_sat(hv[6], hv[7]));
+                    if (live)
+                        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) + row * a.I + mt * MT_G_FEATURES +
+                                                  j0) = pk;
                 }
             }
-        } else if (live) {
-            // fp32 push to the token's slot; the combine rounds y once
-            const int slot = __ldg(a.row_slot + u.grow0 + col);
-            float4* dst = reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + mt * MT_D_FEATURES + fq * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-                const int f = fq * 32 + q4 * 4;
-                dst[q4] = make_float4(epi[f * EPI_LD + tok], epi[(f + 1) * EPI_LD + tok],
-                                      epi[(f + 2) * EPI_LD + tok], epi[(f + 3) * EPI_LD + tok]);
+        } else {
+            // fp32 push to the token's slot, one 512-byte row per warp store; the combine rounds y once
+#pragma unroll 4
+            for (int it = 0; it < 8; ++it) {
+                const int t = it * 4 + q;
+                const int col = cc * 32 + t;
+                if (col < u.rows) {
+                    const int slot = __ldg(a.row_slot + u.grow0 + col);
+                    reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + mt * MT_D_FEATURES)[lane] =
+                        *reinterpret_cast<const float4*>(epi + t * EPI_TLD + 4 * lane);
+                }
             }
         }
         named_bar_sync(1, 128);
@@ -554,7 +556,6 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
     const int lane = threadIdx.x & 31;
     const int et = threadIdx.x - 64;  // 0..127
     float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF);
-    float* xch = reinterpret_cast<float*>(smem + C::XCH_OFF);  // [4][32] block maxima (MXFP8)
     uint32_t tk = 0;  // next accumulator ticket (the MMA issuer's sequence)
     bool ok = true;
     Unit u;
@@ -574,7 +575,7 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
                 if (!ok) break;
                 tc_fence_after();
             }
-            epi_drain_tile<C>(a, u, u.m * C::SUB + sub, acc_col(tk, sub, wide), epi, xch, tmem_base);
+            epi_drain_tile<C>(a, u, u.m * C::SUB + sub, acc_col(tk, sub, wide), epi, tmem_base);
             if (wide || sub == nsub - 1) {
                 // this buffer is drained: the MMA issuer may reuse it
                 tc_fence_before();
