@@ -74,10 +74,12 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
     const int tiles = phase == 0 ? sh.I / MT_G_FEATURES : sh.H / MT_D_FEATURES;
-    // MXFP8 keeps one tile per unit: measured, pairs were 9-10 % slower there
-    // (a tall pair fills TMEM, and its heavier quantising epilogue then
-    // stalls the next unit's MMAs)
-    const bool pair = tune.pair && !mx;
+    // Pairs only for the bf16 gate/up launch.  MXFP8 keeps one tile per unit:
+    // measured, pairs were 6-10 % slower there (a tall pair fills TMEM, and
+    // its quantising epilogue then stalls the next unit's MMAs).  The down
+    // launch's units are short (K = I), so that stall weighs more there:
+    // pairs for gate/up only measured 3 % faster than pairs for both.
+    const bool pair = tune.pair && !mx && phase == 0;
     const int sub = pair ? 2 : 1;
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
@@ -87,7 +89,7 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     } else {
         MxMaps none;
         memset(&none, 0, sizeof none);
-        if (tune.pair)
+        if (pair)
             k_grouped_gemm<Bf16PairCfg><<<grid, Bf16PairCfg::THREADS, Bf16PairCfg::SMEM, stream>>>(
                 maps, none, a, chunks, counts2, phase, MT, GC);
         else
