@@ -124,3 +124,26 @@ def test_get_status_argument_checks():
     L = mok.lib()
     rc = L.mok_get_status(None, 0, None, None)
     assert rc == mok.MOK_ERR_INVALID_ARG
+
+
+def test_mxfp8_step_entry_points_reject_bad_arguments():
+    """The MXFP8 gather and FFN check shapes, pointers and alignment on the
+    host, before any device work."""
+    p = mok.PlanT(16, 8, 2, 2)
+    for name in ("counts", "offsets", "sched_src_rank", "sched_src_index", "row_slot", "pos", "topk_idx", "gates"):
+        setattr(p, name, 4096)
+    L = mok.lib()
+    arr = (ctypes.c_void_p * 2)(4096, 8192)
+    # H must be a multiple of 128 for the quantising gather
+    assert L.mok_gather_mxfp8(arr, 192, ctypes.byref(p), 4096, 8192, None) == mok.MOK_ERR_UNSUPPORTED
+    assert L.mok_gather_mxfp8(arr, 256, ctypes.byref(p), None, 8192, None) == mok.MOK_ERR_INVALID_ARG
+    assert L.mok_gather_mxfp8(arr, 256, ctypes.byref(p), 4100, 8192, None) == mok.MOK_ERR_UNSUPPORTED
+    assert L.mok_mxfp8_scale_rows(10) == 16 and L.mok_mxfp8_scale_rows(12) == 16 and L.mok_mxfp8_scale_rows(13) == 20
+    need = L.mok_expert_ffn_mxfp8_workspace_bytes(32, 256, 8)
+    assert need > 0
+    w = mok.MxWeights(4096, 4096, 4096, 4096, 4096, 0)
+    rc = L.mok_expert_ffn_mxfp8(4096, 8192, 256, 256, ctypes.cast(ctypes.byref(w), ctypes.c_void_p), ctypes.byref(p),
+                                256, need, 4096, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG and "NULL" in mok.last_error()
+    rc = L.mok_expert_ffn_mxfp8(4096, 8192, 256, 256, None, ctypes.byref(p), 256, need - 1, 4096, None)
+    assert rc == mok.MOK_ERR_WORKSPACE
