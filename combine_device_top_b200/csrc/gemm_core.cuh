@@ -32,9 +32,9 @@
 //
 // Roles in a CTA: warp 0 issues TMA loads into a ring of stages, warp 1
 // allocates 512 TMEM columns and one thread of it issues tcgen05.mma into
-// one of two 256-column accumulators, warps 2-5 drain the other accumulator
+// one of two 256-column accumulators, warps 2-9 (two groups) drain the other accumulator
 // (tcgen05.ld) through shared memory to global memory, and (MXFP8 only)
-// warp 6 lays each stage's scales out for the copy into TMEM.  The token tile of a stage is ONE TMA box
+// warp 10 lays each stage's scales out for the copy into TMEM.  The token tile of a stage is ONE TMA box
 // of exactly the 16-rounded row count, and a down unit's two 64-column
 // weight halves come from one 3D map.  Measured on B200: the number of TMA
 // ops per SM, and then the bytes each SM takes in from L2 (about 64 B per
@@ -73,13 +73,13 @@ template <int SUB_, int NST_>
 struct Bf16CfgT {
     static constexpr bool MX = false;
     static constexpr int SUB = SUB_;  // M tiles per unit
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 320;  // warps: 0 TMA, 1 MMA, 2-9 two epilogue groups
     static constexpr int NST = NST_;
     static constexpr int BKX = BK;  // K per stage
     static constexpr int STAGE = SUB * A_BYTES + B_BYTES;
     static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
-    static constexpr int EPI_OFF = NST * STAGE;
-    static constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
+    static constexpr int EPI_OFF = NST * STAGE;           // one staging tile per epilogue group
+    static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + slack for 1024-byte alignment
 };
 using Bf16Cfg = Bf16CfgT<1, 4>;
@@ -93,7 +93,7 @@ template <int SUB_, int NST_>
 struct MxCfgT {
     static constexpr bool MX = true;
     static constexpr int SUB = SUB_;
-    static constexpr int THREADS = 224;  // + warp 6: scale-factor layout
+    static constexpr int THREADS = 352;  // warps: 0 TMA, 1 MMA, 2-9 epilogue, 10 scale-factor layout
     static constexpr int NST = NST_;
     static constexpr int BKX = 128;      // K per stage
     static constexpr int A_OFF = 0, B_OFF = SUB * 16384;
@@ -102,8 +102,8 @@ struct MxCfgT {
     static constexpr int SFA_OFF = SFB_RAW_OFF + 1024;                   // one 512-byte scale atom per tile
     static constexpr int SFB_OFF = SFA_OFF + SUB * 512;                  // two atoms (rows 0-127, 128-255)
     static constexpr int STAGE = SFB_OFF + 1024;
-    static constexpr int EPI_OFF = NST * STAGE;
-    static constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
+    static constexpr int EPI_OFF = NST * STAGE;           // one staging tile per epilogue group
+    static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
     // TMEM: accumulators in columns [0, 480) (N <= 224), then the scale
     // factors of the SUB weight tiles (4 columns each) and of the tokens (8)
@@ -289,7 +289,7 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
         if ((issued >> st) & 1u) mbar_wait(&full[st], (issued_phase >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 11);
 }
 
-// ------------------------------------------------------------------ MXFP8 scale-factor layout (warp 6)
+// ------------------------------------------------------------------ MXFP8 scale-factor layout (warp 10)
 // The block-scaled MMA reads the scales of a 128-row operand tile from TMEM
 // as 32 lanes x 4 columns of 32-bit words: row r = r0 + 32 r1 at lane r0,
 // column r1, byte b = K block b of the stage (the copy to TMEM takes them
@@ -465,25 +465,27 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
     mbar_wait(fin, 0, nullptr, DRAIN_TIMEOUT_NS, 22);
 }
 
-// ------------------------------------------------------------------ epilogue (warps 2..5)
+// ------------------------------------------------------------------ epilogue (warps 2..9)
 // Drains one M tile's accumulator (TMEM columns col0 .. col0 + rows), 32
 // tokens at a time, through a token-major staging tile in shared memory
 // (epi[token][feature], pitch EPI_TLD), so that every global store is a
 // row-contiguous run: gate/up writes h rows (8 lanes per 64-feature row),
 // down pushes 512-byte fp32 rows (a warp per row) to the tokens' slots.
+// Chunks cc0, cc0 + ccstep, ... of the tile are drained by this warpgroup
+// (named barrier `bar`, staging tile `epi`).
 template <class C>
 __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u, int mt, uint32_t col0, float* epi,
-                                               uint32_t tmem_base) {
+                                               uint32_t tmem_base, int cc0, int ccstep, int bar) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access: features q*32 .. q*32+31
     const int ncc = (u.rows + 31) >> 5;
-    for (int cc = 0; cc < ncc; ++cc) {
+    for (int cc = cc0; cc < ncc; cc += ccstep) {
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + col0 + (uint32_t)(cc * 32), v);
         // token-major: lanes hold consecutive features, so each store row is contiguous
 #pragma unroll
         for (int t = 0; t < 32; ++t) epi[t * EPI_TLD + q * 32 + lane] = v[t];
-        named_bar_sync(1, 128);
+        named_bar_sync(bar, 128);
         if (u.phase == 0) {
             // h features mt*64 + j: gate in staging columns j, up in 64 + j.  Lane
             // group g = lane / 8 takes token rows; lane % 8 owns 8 features.
@@ -546,16 +548,24 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 }
             }
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(bar, 128);
     }
 }
 
+// Two warpgroups drain each unit side by side (warps 2-5 and 6-9, each
+// covering the four TMEM lane quadrants): a pair's tiles one each, a single
+// tile's 32-token chunks alternately.  Each group arrives once on every
+// ticket of the unit when it has finished its share (tempty counts 8).
 template <class S, class C>
 __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* tfull,
-                                              uint64_t* tempty, volatile int* ok_flag, uint32_t tmem_base) {
+                                              uint64_t* tempty, volatile int* ok_flags, int* done_cnt,
+                                              uint32_t tmem_base) {
     const int lane = threadIdx.x & 31;
-    const int et = threadIdx.x - 64;  // 0..127
-    float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF);
+    const int g = (threadIdx.x - 64) >> 7;     // warpgroup 0 or 1
+    const int et = (threadIdx.x - 64) & 127;   // 0..127 inside the group
+    const int bar = 1 + g;                     // the group's named barrier
+    volatile int* ok_flag = ok_flags + g;
+    float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF + g * EPI_BYTES);
     uint32_t tk = 0;  // next accumulator ticket (the MMA issuer's sequence)
     bool ok = true;
     Unit u;
@@ -563,35 +573,42 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
         const int nsub = unit_subs<C>(a, u);
         const int nt = unit_tickets<C>(nsub, (u.rows + 15) & ~15);
         const bool wide = nt == 2;
-        for (int sub = 0; sub < nsub && ok; ++sub) {
+        // this group's share: tile `g` of a pair, or every other chunk of a single tile
+        const int sub = nsub == 2 ? g : 0;
+        {
             const uint32_t tkt = wide ? tk + (uint32_t)sub : tk;
-            if (sub == 0 || wide) {
-                // one thread waits, all 128 leave together on failure
-                if (et == 0)
-                    *ok_flag = mbar_wait(&tfull[tkt & 1u], (tkt >> 1) & 1u, a.st, a.timeout_ns, 30) ? 1 : 0;
-                named_bar_sync(1, 128);
-                ok = *ok_flag != 0;
-                named_bar_sync(1, 128);
-                if (!ok) break;
-                tc_fence_after();
-            }
-            epi_drain_tile<C>(a, u, u.m * C::SUB + sub, acc_col(tk, sub, wide), epi, tmem_base);
-            if (wide || sub == nsub - 1) {
-                // this buffer is drained: the MMA issuer may reuse it
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[tkt & 1u]);
-            }
+            // one thread waits, all 128 of the group leave together on failure
+            if (et == 0) *ok_flag = mbar_wait(&tfull[tkt & 1u], (tkt >> 1) & 1u, a.st, a.timeout_ns, 30) ? 1 : 0;
+            named_bar_sync(bar, 128);
+            ok = *ok_flag != 0;
+            named_bar_sync(bar, 128);
+            if (!ok) break;
+            tc_fence_after();
+            epi_drain_tile<C>(a, u, u.m * C::SUB + sub, acc_col(tk, sub, wide), epi, tmem_base,
+                              nsub == 2 ? 0 : g, nsub == 2 ? 1 : 2, bar);
         }
-        if (!ok) break;
+        // this group is done with every buffer of the unit
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            for (int t = 0; t < nt; ++t) mbar_arrive(&tempty[(tk + (uint32_t)t) & 1u]);
         tk += (uint32_t)nt;
         if (S::kSignals) {
             // h rows are read next by TMA (async proxy) in some CTA: make this
-            // thread's stores visible to that proxy, then publish once.
+            // group's stores visible to that proxy; the group that finishes
+            // the unit second publishes it once.  The groups are at most one
+            // unit apart (a buffer is reused only after both released it), so
+            // two counters, by unit parity, pair their arrivals.
             fence_proxy_async_global();
             __threadfence();
-            named_bar_sync(1, 128);
-            if (et == 0) s.unit_done(u);
+            named_bar_sync(bar, 128);
+            if (et == 0) {
+                __threadfence();
+                if (atomicAdd(done_cnt + (i & 1), 1) & 1) {
+                    __threadfence();
+                    s.unit_done(u);
+                }
+            }
         }
     }
 }
@@ -609,10 +626,14 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
     uint64_t* tempty = tfull + 2;
     uint64_t* fin = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
-    volatile int* ok_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* ok_flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // one per epilogue group
+    int* done_cnt = const_cast<int*>(ok_flags) + 2;                            // two, by unit parity
+    static_assert((3 * C::NST + 5) * 8 + 4 * 5 <= 256, "barrier region");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        done_cnt[0] = 0;
+        done_cnt[1] = 0;
         for (int st = 0; st < C::NST; ++st) {
             mbar_init(&full[st], 1);
             mbar_init(&empty[st], 1);
@@ -620,7 +641,7 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], 8);  // 4 warps of each epilogue group
         }
         mbar_init(fin, 1);
         fence_mbar_init();
@@ -657,8 +678,8 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
         if (lane == 0) gemm_producer<S, C>(maps, mx, a, s, smem, full, empty);
     } else if (warp == 1) {
         if (lane == 0) gemm_mma<S, C>(a, s, smem, C::MX ? sfready : full, empty, tfull, tempty, fin, tmem_base);
-    } else if (warp < 6) {
-        gemm_epilogue<S, C>(a, s, smem, tfull, tempty, ok_flag, tmem_base);
+    } else if (warp < 10) {
+        gemm_epilogue<S, C>(a, s, smem, tfull, tempty, ok_flags, done_cnt, tmem_base);
     } else if constexpr (C::MX) {
         gemm_sf_layout<S, C>(a, s, smem, full, sfready);
     }
