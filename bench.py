@@ -145,7 +145,7 @@ class ClockSampler:
 # exists for that workload.
 GEMM_TRAFFIC_GB_PER_STEP = {
     "page": (36.5, "profiles/grouped_gemm_bf16_page_e37.md"),
-    "page_mxfp8": (19.8, "profiles/grouped_gemm_mxfp8_page_e32.md"),
+    "page_mxfp8": (19.7, "profiles/grouped_gemm_mxfp8_page_e32.md"),
 }
 
 
