@@ -32,13 +32,15 @@
 //
 // Roles in a CTA: warp 0 issues TMA loads into a ring of stages, warp 1
 // allocates 512 TMEM columns and one thread of it issues tcgen05.mma into
-// one of two 256-column accumulators, warps 2-9 (two groups) drain the other accumulator
-// (tcgen05.ld) through shared memory to global memory, and (MXFP8 only)
-// warp 10 lays each stage's scales out for the copy into TMEM.  The token tile of a stage is ONE TMA box
-// of exactly the 16-rounded row count, and a down unit's two 64-column
-// weight halves come from one 3D map.  Measured on B200: the number of TMA
-// ops per SM, and then the bytes each SM takes in from L2 (about 64 B per
-// clock), limit this kernel.  Every wait is bounded.
+// one of two 256-column accumulators, warps 2-9 (two groups of four) drain
+// the other accumulator (tcgen05.ld) through shared memory to global
+// memory, and (MXFP8 only) warp 10 lays each stage's scales out for the
+// copy into TMEM.  The token tile of a stage is ONE TMA box of exactly the
+// 16-rounded row count, and a down unit's two 64-column weight halves come
+// from one 3D map: measured on B200, the number of TMA ops per SM and then
+// the bytes each SM takes in from L2 limited earlier versions.  With a unit
+// of two M tiles (bf16 gate/up at <= 192 rows per expert) the tiles share
+// every token tile.  Every wait is bounded.
 //
 // A schedule policy (template parameter) tells each role which units this
 // CTA runs, what a unit's inputs wait for, and what its completion signals.
