@@ -143,10 +143,7 @@ class ClockSampler:
 # the capture, its command and the scaling are in the profiles/ summary
 # named beside each entry.  None where no capture of the current kernel
 # exists for that workload.
-GEMM_TRAFFIC_GB_PER_STEP = {
-    "page": (36.5, "profiles/grouped_gemm_bf16_page_e37.md"),
-    "page_mxfp8": (19.7, "profiles/grouped_gemm_mxfp8_page_e32.md"),
-}
+GEMM_TRAFFIC_GB_PER_STEP = {}
 
 
 # ------------------------------------------------------------------ ranks
@@ -171,15 +168,15 @@ def algorithmic_work(cfg):
     """Algorithmic bytes / flops of one forward (one step)."""
     ns = cfg.slots
     w_bytes = cfg.E * 3 * cfg.H * cfg.I * 2
-    gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 4  # weights, rows in, h out+in, fp32 out
+    gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 2  # weights, rows in, h out+in, fp16 out
     gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * 2
     if cfg.mxfp8:
         # weights, token rows and h: E4M3 bytes plus one E8M0 scale per 32 values
         mx = 1.0 + 1.0 / 32
         w_bytes = cfg.E * 3 * cfg.H * cfg.I * mx
-        gemm_bytes = w_bytes + ns * cfg.H * mx + 2 * ns * cfg.I * mx + ns * cfg.H * 4
+        gemm_bytes = w_bytes + ns * cfg.H * mx + 2 * ns * cfg.I * mx + ns * cfg.H * 2
         gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * mx
-    combine_bytes = ns * cfg.H * 4 + ns * 4 + cfg.T * cfg.H * 2
+    combine_bytes = ns * cfg.H * 2 + ns * 4 + cfg.T * cfg.H * 2
     return {
         "gemm_flops": 6.0 * cfg.H * cfg.I * ns,
         "gemm_bytes": float(gemm_bytes),
@@ -222,7 +219,7 @@ def run_mok(args, cfg, rank, world, device):
     # staged mode is timed one ABI step at a time (per-phase events)
     staged = mode == mok.MOK_MODE_STAGED
     if staged:
-        out = torch.empty((cfg.slots, cfg.H), dtype=torch.float32, device=device)
+        out = torch.empty((cfg.slots, cfg.H), dtype=torch.float16, device=device)
         if cfg.mxfp8:
             rows_q = torch.empty((cfg.slots, cfg.H), dtype=torch.uint8, device=device)
             planes = torch.zeros((cfg.H // 128, mok.lib().mok_mxfp8_scale_rows(cfg.slots), 4), dtype=torch.uint8,

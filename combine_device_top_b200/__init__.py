@@ -308,12 +308,13 @@ def gather_mxfp8(x_shards, p: Plan, rows_q=None, scales=None, stream=None):
 
 def expert_ffn_mxfp8(rows_q, scales, pack, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
     """The MXFP8 grouped SwiGLU FFN over mok_gather_mxfp8's output; pack =
-    (qg, sg, qu, su, qd, sd).  Returns (out [T*k, H] fp32 slot-indexed, ws)."""
+    (qg, sg, qu, su, qd, sd).  Returns (out [T*k, H] fp16 slot-indexed, ws)."""
     qg, sg, qu, su, qd, sd = pack
     H = rows_q.shape[1]
     I = qg.shape[-1]
     if out is None:
-        out = torch.empty((p.ns, H), dtype=torch.float32, device=rows_q.device)
+        out = torch.empty((p.ns, H), dtype=torch.float16, device=rows_q.device)
+    assert out.dtype == torch.float16
     if ws is None:
         ws = _workspace(lib().mok_expert_ffn_mxfp8_workspace_bytes(p.ns, I, p.c.E), rows_q.device)
     w = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
@@ -325,12 +326,12 @@ def expert_ffn_mxfp8(rows_q, scales, pack, p: Plan, out: torch.Tensor | None = N
 
 
 def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
-    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] fp32 slot-indexed, ws)."""
+    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] fp16 slot-indexed, ws)."""
     H = rows.shape[1]
     I = w_gate.shape[-1]
     if out is None:
-        out = torch.empty((p.ns, H), dtype=torch.float32, device=rows.device)
-    assert out.dtype == torch.float32
+        out = torch.empty((p.ns, H), dtype=torch.float16, device=rows.device)
+    assert out.dtype == torch.float16
     if ws is None:
         ws = _workspace(lib().mok_expert_ffn_workspace_bytes(p.ns, I, p.c.E), rows.device)
     _check(lib().mok_expert_ffn(ctypes.c_void_p(rows.data_ptr()), H, I, ctypes.c_void_p(w_gate.data_ptr()),
@@ -341,8 +342,8 @@ def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = N
 
 
 def combine(out: torch.Tensor, p: Plan, y_shards, stream=None):
-    """y = fixed-order gate-weighted sum of the fp32 per-slot outputs."""
-    assert out.dtype == torch.float32
+    """y = fixed-order gate-weighted sum of the fp16 per-slot outputs (fp32 accumulation)."""
+    assert out.dtype == torch.float16
     H = out.shape[-1]
     _check(lib().mok_combine(ctypes.c_void_p(out.data_ptr()), H, ctypes.byref(p.c), _ptr_array(y_shards),
                              _stream(stream)))

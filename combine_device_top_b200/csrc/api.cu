@@ -210,7 +210,7 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
         l.rows = take((size_t)l.buf_rows * H * 2);
         l.h = take((size_t)l.buf_rows * I * 2);
     }
-    l.out = take((size_t)ns * H * 4);
+    l.out = take((size_t)ns * H * 2);  // fp16 slot outputs
     l.total = off;
     *L = l;
     return true;
@@ -417,7 +417,7 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         P.wd = w_down;
         P.ring = base + L.rows;
         P.h = base + L.h;
-        P.out = reinterpret_cast<float*>(base + L.out);
+        P.out = reinterpret_cast<__half*>(base + L.out);
         P.chunks = chunks;
         P.mbs = mbs;
         P.counts2 = counts2;

@@ -119,7 +119,7 @@ cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, c
 }
 
 template <int KMAX>
-__global__ void __launch_bounds__(DC_THREADS) k_combine(const float4* __restrict__ out, const float* __restrict__ gates,
+__global__ void __launch_bounds__(DC_THREADS) k_combine(const uint4* __restrict__ out, const float* __restrict__ gates,
                                                         int T, int k, int H, int S_r, ShardsOut ys) {
     const int lane = threadIdx.x & 31;
     const int nvec = H >> 3;
@@ -145,7 +145,7 @@ cudaError_t launch_combine(const void* out, const float* gates, int T, int k, in
     if (T <= 0) return cudaSuccess;
     const int want = (T + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     const int grid = want < num_sms * 8 ? want : num_sms * 8;
-    const float4* o = reinterpret_cast<const float4*>(out);
+    const uint4* o = reinterpret_cast<const uint4*>(out);
     if (k <= 2)
         k_combine<2><<<grid, DC_THREADS, 0, stream>>>(o, gates, T, k, H, S_r, ys);
     else

@@ -84,41 +84,39 @@ __device__ __forceinline__ bool bulk_stream_rows(int n, SrcF src_row, DstF dst_r
 }
 
 // One warp: y[t] = bf16(sum_{j<k} g[t,j] * out[t,j,:]) in fp32, j ascending.
-// out is fp32 [T, k, H]; each lane owns 8 consecutive features (two 16-byte
-// loads per slot, one 16-byte store).  nvec = H / 8.  Slots are loaded KB at
+// out is fp16 [T, k, H]; each lane owns 8 consecutive features (one 16-byte
+// load per slot, one 16-byte store).  nvec = H / 8.  Slots are loaded KB at
 // a time (KB loads in flight), then accumulated in order.
 template <int KB>
-__device__ __forceinline__ void warp_combine_token(const float4* __restrict__ out, const float* __restrict__ gates,
+__device__ __forceinline__ void warp_combine_token(const uint4* __restrict__ out, const float* __restrict__ gates,
                                                    int t, int k, int nvec, uint4* __restrict__ dst, int lane) {
-    const float4* src = out + (size_t)t * k * (2 * nvec);
+    const uint4* src = out + (size_t)t * k * nvec;
     const float* gt = gates + (size_t)t * k;
     // lanes may run different numbers of iterations (nvec % 32 != 0): no
     // warp collectives inside; the gates are broadcast loads (L1 hits)
     for (int v = lane; v < nvec; v += 32) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j0 = 0; j0 < k; j0 += KB) {
-            float4 a[KB], b[KB];
+            uint4 a[KB];
             float g[KB];
 #pragma unroll
             for (int jj = 0; jj < KB; ++jj) {
                 const int j = j0 + jj;
                 if (j < k) {
                     g[jj] = __ldg(gt + j);
-                    a[jj] = __ldcs(src + (size_t)j * 2 * nvec + 2 * v);
-                    b[jj] = __ldcs(src + (size_t)j * 2 * nvec + 2 * v + 1);
+                    a[jj] = __ldcs(src + (size_t)j * nvec + v);
                 }
             }
 #pragma unroll
             for (int jj = 0; jj < KB; ++jj)
                 if (j0 + jj < k) {
-                    acc[0] = fmaf(g[jj], a[jj].x, acc[0]);
-                    acc[1] = fmaf(g[jj], a[jj].y, acc[1]);
-                    acc[2] = fmaf(g[jj], a[jj].z, acc[2]);
-                    acc[3] = fmaf(g[jj], a[jj].w, acc[3]);
-                    acc[4] = fmaf(g[jj], b[jj].x, acc[4]);
-                    acc[5] = fmaf(g[jj], b[jj].y, acc[5]);
-                    acc[6] = fmaf(g[jj], b[jj].z, acc[6]);
-                    acc[7] = fmaf(g[jj], b[jj].w, acc[7]);
+                    const __half2* h2 = reinterpret_cast<const __half2*>(&a[jj]);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 f = __half22float2(h2[p]);
+                        acc[2 * p] = fmaf(g[jj], f.x, acc[2 * p]);
+                        acc[2 * p + 1] = fmaf(g[jj], f.y, acc[2 * p + 1]);
+                    }
                 }
         }
         uint4 o;

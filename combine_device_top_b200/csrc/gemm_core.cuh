@@ -18,10 +18,11 @@
 //     lanes 0-63 hold gate, 64-127 up; the epilogue forms
 //     h = silu(gate) * up and stores h rows.
 //   down unit (phase 1): A = 128 columns of Wd (MN-major from [E, I, H]),
-//     B = the chunk's h rows.  The epilogue stores fp32 rows to
-//     out[row_slot[row]] (the push combine); fp32 rather than bf16 because a
+//     B = the chunk's h rows.  The epilogue stores fp16 rows to
+//     out[row_slot[row]] (the push combine); fp16 rather than bf16 because a
 //     bf16 slot buffer adds a rounding that puts the largest element error of
-//     y above 2e-2 * rms(y) on heavy-tailed outputs.
+//     y above 2e-2 * rms(y) on heavy-tailed outputs (fp16's 3 more mantissa
+//     bits keep it at the floor of y's own bf16 rounding).
 // Precision: the bf16 path computes gate/up in bf16 and the down projection
 // in fp16 (fp16 h and the fp16 copy of Wd: 3 more mantissa bits on h keep
 // the error of y at the floor of its own bf16 rounding).  The MXFP8 path
@@ -138,7 +139,7 @@ struct Unit {
 struct CoreArgs {
     int H, I;
     void* h;                  // [buffer rows, I]: fp16 (bf16 path) or E4M3 (MXFP8 path)
-    float* out;               // [N_s, H] fp32, slot-indexed
+    __half* out;              // [N_s, H] fp16, slot-indexed
     const int32_t* row_slot;  // [N_s]
     DevStatus* st;
     uint64_t timeout_ns;
@@ -472,7 +473,7 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
 // tokens at a time, through a token-major staging tile in shared memory
 // (epi[token][feature], pitch EPI_TLD), so that every global store is a
 // row-contiguous run: gate/up writes h rows (8 lanes per 64-feature row),
-// down pushes 512-byte fp32 rows (a warp per row) to the tokens' slots.
+// down pushes 256-byte fp16 rows (a warp per row) to the tokens' slots.
 // Chunks cc0, cc0 + ccstep, ... of the tile are drained by this warpgroup
 // (named barrier `bar`, staging tile `epi`).
 template <class C>
@@ -538,15 +539,16 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 }
             }
         } else {
-            // fp32 push to the token's slot, one 512-byte row per warp store; the combine rounds y once
+            // fp16 push to the token's slot, one 256-byte row per warp store; the combine rounds y once
 #pragma unroll 4
             for (int it = 0; it < 8; ++it) {
                 const int t = it * 4 + q;
                 const int col = cc * 32 + t;
                 if (col < u.rows) {
                     const int slot = __ldg(a.row_slot + u.grow0 + col);
-                    reinterpret_cast<float4*>(a.out + (size_t)slot * a.H + mt * MT_D_FEATURES)[lane] =
-                        *reinterpret_cast<const float4*>(epi + t * EPI_TLD + 4 * lane);
+                    const float4 o4 = *reinterpret_cast<const float4*>(epi + t * EPI_TLD + 4 * lane);
+                    reinterpret_cast<uint2*>(a.out + (size_t)slot * a.H + mt * MT_D_FEATURES)[lane] =
+                        make_uint2(pack_half2_sat(o4.x, o4.y), pack_half2_sat(o4.z, o4.w));
                 }
             }
         }

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -139,7 +140,7 @@ struct PersistLaunch {
     const void *wg, *wu, *wd;      // weights (bf16, bf16, fp16)
     void* ring;                    // [2*cap, H] bf16
     void* h;                       // [2*cap, I] fp16
-    float* out;                    // [T*k, H] fp32
+    __half* out;                   // [T*k, H] fp16
     const Chunk* chunks;
     const Minibatch* mbs;
     const int* counts2;

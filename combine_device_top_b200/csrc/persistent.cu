@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     for (int t = blockIdx.x * (GEMM_THREADS / 32) + warp; t < p.T; t += warps) {
         const int r = t / p.S_r;
         uint4* dst = reinterpret_cast<uint4*>(p.ys.p[r]) + (size_t)(t - r * p.S_r) * nvec;
-        warp_combine_token<KMAX>(reinterpret_cast<const float4*>(a.out), p.gates, t, p.k, nvec, dst, lane);
+        warp_combine_token<KMAX>(reinterpret_cast<const uint4*>(a.out), p.gates, t, p.k, nvec, dst, lane);
     }
 }
 

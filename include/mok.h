@@ -203,15 +203,15 @@ size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int miniba
  *   y_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
  * Arithmetic: gate/up in bf16 x bf16 with fp32 accumulation; h =
  * silu(gate) * up rounded to fp16 (saturating at +-65504); down projection
- * fp16 x fp16 with fp32 accumulation; each expert output row stored fp32 at
- * its slot; y[t] = bf16(sum_{j<k} g[t,j] * o[t,j]) accumulated in fp32
+ * fp16 x fp16 with fp32 accumulation; each expert output row stored fp16 at
+ * its slot (saturating); y[t] = bf16(sum_{j<k} g[t,j] * o[t,j]) accumulated in fp32
  * with j ascending (one bf16 rounding of y).  y does not depend on the
  * mode, minibatch, ring size or R.
  * MXFP8 path (opts->mxfp8 = 1, staged mode, w_gate = a mok_mxfp8_weights
  * HOST struct): x is quantised in the gather and h in the SwiGLU epilogue
  * (32-element blocks, E8M0 scale + E4M3 values, as mok_mxfp8_quantize_rows
  * does); both GEMMs run on the block-scaled E4M3 x E4M3 tensor-core MMA
- * with fp32 accumulation; slot outputs fp32 and the combine as above.
+ * with fp32 accumulation; slot outputs fp16 and the combine as above.
  */
 int mok_moe_forward(const void* const* x_shards, int H, int I,
                     const void* w_gate, const void* w_up, const void* w_down,
@@ -292,9 +292,9 @@ size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E);
 
 /* Grouped SwiGLU FFN over the expert-major rows of `plan`:
  *   h[row]   = fp16(silu(rows[row] Wg[e]) * (rows[row] Wu[e]))   [N_s, I]
- *   out[row_slot[row]] = h[row] Wd16[e]   (fp32)                 [N_s, H]
+ *   out[row_slot[row]] = fp16(h[row] Wd16[e])  (fp32 accumulation) [N_s, H]
  * (e = expert of the row; Wd16 = fp16 W_down from mok_prepare_w_down).
- * h stays in the workspace; `out` is fp32 and
+ * h stays in the workspace; `out` is fp16 and
  * slot-indexed, i.e. [T, k, H].  Source: MoK article, routing paragraph
  * (grouped GEMM over contiguous per-expert tokens) and push-combine
  * paragraph. */
@@ -310,14 +310,14 @@ size_t mok_expert_ffn_mxfp8_workspace_bytes(int n_rows, int I, int E);
  * over the output of mok_gather_mxfp8 (rows_q, scales; same layouts), with
  * the weight pack `w` (host struct) of mok_quantize_weights_mxfp8.  h is
  * quantised to MXFP8 in the SwiGLU epilogue and stays in the workspace;
- * out: [T, k, H] fp32, slot-indexed, as mok_expert_ffn.  Source: MoK
+ * out: [T, k, H] fp16, slot-indexed, as mok_expert_ffn.  Source: MoK
  * article, paragraph on MXFP8 inside the GEMM and SwiGLU. */
 int mok_expert_ffn_mxfp8(const void* rows_q, const void* scales, int H, int I,
                          const mok_mxfp8_weights* w, const mok_plan_t* plan,
                          void* ws, size_t ws_bytes, void* out, mok_stream_t stream);
 
 /* y[t] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]), fp32, j ascending,
- * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] fp32.
+ * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] fp16.
  * Source: MoK article, benchmark paragraph (final weighted merge). */
 int mok_combine(const void* out, int H, const mok_plan_t* plan,
                 void* const* y_shards, mok_stream_t stream);

@@ -58,7 +58,8 @@ def test_combine_matches_oracle():
     case = Case(FFN_CASES["many_experts"])
     cfg = case.cfg
     p = mok.plan(case.dlogits, cfg.k, cfg.R)
-    out = mokgen.normal(5, 77, (cfg.T * cfg.k, cfg.H), 1.0, dtype=torch.float32)
+    # fp16 per-slot outputs, as the grouped GEMM stores them
+    out = mokgen.normal(5, 77, (cfg.T * cfg.k, cfg.H), 1.0, dtype=torch.float32).to(torch.float16)
     ys = [torch.empty((cfg.S_r, cfg.H), dtype=torch.bfloat16, device="cuda") for _ in range(cfg.R)]
     mok.combine(out.cuda(), p, ys)
     torch.cuda.synchronize()
