@@ -143,7 +143,10 @@ class ClockSampler:
 # the capture, its command and the scaling are in the profiles/ summary
 # named beside each entry.  None where no capture of the current kernel
 # exists for that workload.
-GEMM_TRAFFIC_GB_PER_STEP = {}
+GEMM_TRAFFIC_GB_PER_STEP = {
+    "page": (35.6, "profiles/grouped_gemm_bf16_page_e37.md"),
+    "page_mxfp8": (18.9, "profiles/grouped_gemm_mxfp8_page_e32.md"),
+}
 
 
 # ------------------------------------------------------------------ ranks
