@@ -214,7 +214,7 @@ def run_mok(args, cfg, rank, world, device):
     y = torch.empty_like(dx)
     y_shards = mok.shards(y, cfg.R)
     mode = mok.MOK_MODE_STAGED if args.mode == "staged" else mok.MOK_MODE_PERSISTENT
-    opts = mok.fwd_opts(mode=mode, ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8)
+    opts = mok.fwd_opts(mode=mode, ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8, dispatch_ctas=args.dispatch_ctas)
     minibatch = args.minibatch or cfg.minibatch
     p = mok.plan(dlogits, cfg.k, cfg.R)
     fws = torch.empty(mok.forward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
@@ -260,6 +260,8 @@ def run_mok(args, cfg, rank, world, device):
             if evs:
                 evs[3].record(stream)
             mok.combine(out, p, y_shards)
+        elif pack is not None:
+            mok.moe_forward_mxfp8(x_shards, pack, p, y_shards=y_shards, ws=fws, minibatch=minibatch, opts=opts)
         else:
             mok.moe_forward(x_shards, wg, wu, wd, p, minibatch, opts, y_shards=y_shards, ws=fws)
         if evs:
@@ -367,15 +369,14 @@ def main():
     ap.add_argument("--config", default="page", choices=list(mokgen.CONFIGS))
     ap.add_argument("--mode", default="staged", choices=["staged", "persistent"])
     ap.add_argument("--minibatch", type=int, default=0)
+    ap.add_argument("--dispatch-ctas", type=int, default=0,
+                    help="persistent mode: CTAs on the dispatch side (0: the library default, 16)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--scale-experts", type=int, default=0,
                     help="profiling case: E experts and T scaled by the same factor (same rows per expert)")
     args = ap.parse_args()
     cfg = mokgen.CONFIGS[args.config]
-    if cfg.mxfp8 and args.mode != "staged":
-        print("the MXFP8 path runs in staged mode only; timing staged mode", file=sys.stderr)
-        args.mode = "staged"
     if args.scale_experts:
         n = args.scale_experts
         T = max(cfg.R, round(cfg.T * n / cfg.E / cfg.R) * cfg.R)
@@ -392,6 +393,7 @@ def main():
     config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
               "tokens_per_step_per_gpu": cfg.T, "minibatch": args.minibatch or cfg.minibatch,
               "mode": args.mode,
+              **({"dispatch_ctas": args.dispatch_ctas or 16} if args.mode == "persistent" else {}),
               "l2": f"inputs larger than L2 ({algorithmic_work(cfg)['weight_bytes'] / 1e9:.1f} GB of expert "
                     f"weights streamed per step)"}
 

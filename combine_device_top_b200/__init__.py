@@ -253,23 +253,28 @@ class MxWeights(ctypes.Structure):
                 ("up_scales", ctypes.c_void_p), ("down", ctypes.c_void_p), ("down_scales", ctypes.c_void_p)]
 
 
-def moe_forward_mxfp8(x_shards, pack, p: Plan, y_shards=None, ws: torch.Tensor | None = None, stream=None):
-    """The forward layer on the MXFP8 path (staged mode).  ``pack`` = (qg, sg,
-    qu, su, qd, sd) from :func:`quantize_weights_mxfp8`.  Returns (y_shards, ws)."""
+def moe_forward_mxfp8(x_shards, pack, p: Plan, y_shards=None, ws: torch.Tensor | None = None, stream=None,
+                      minibatch: int = 0, opts: FwdOpts | None = None):
+    """The forward layer on the MXFP8 path.  ``pack`` = (qg, sg, qu, su, qd,
+    sd) from :func:`quantize_weights_mxfp8`.  Staged mode by default; pass
+    ``opts=fwd_opts(mode=MOK_MODE_PERSISTENT, mxfp8=True)`` and a minibatch
+    for the persistent kernel.  Returns (y_shards, ws)."""
     qg, sg, qu, su, qd, sd = pack
     R = p.c.R
     H = x_shards[0].shape[1]
     I = qg.shape[-1]
     dev = x_shards[0].device
-    opts = fwd_opts(mode=MOK_MODE_STAGED, mxfp8=True)
+    if opts is None:
+        opts = fwd_opts(mode=MOK_MODE_STAGED, mxfp8=True)
+    assert opts.mxfp8 == 1, "moe_forward_mxfp8 needs opts with mxfp8=True"
     if y_shards is None:
         y_shards = [torch.empty_like(s) for s in x_shards]
     if ws is None:
-        ws = _workspace(forward_workspace_bytes(p.c.T, H, I, p.c.E, p.c.k, 0, opts), dev)
+        ws = _workspace(forward_workspace_bytes(p.c.T, H, I, p.c.E, p.c.k, minibatch, opts), dev)
     w = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
     _check(lib().mok_moe_forward(_ptr_array(x_shards), H, I, ctypes.cast(ctypes.byref(w), ctypes.c_void_p), None,
-                                 None, ctypes.byref(p.c), 0, ctypes.byref(opts), ctypes.c_void_p(ws.data_ptr()),
-                                 ws.numel(), _ptr_array(y_shards), _stream(stream)))
+                                 None, ctypes.byref(p.c), minibatch, ctypes.byref(opts),
+                                 ctypes.c_void_p(ws.data_ptr()), ws.numel(), _ptr_array(y_shards), _stream(stream)))
     assert len(x_shards) == R
     return y_shards, ws
 

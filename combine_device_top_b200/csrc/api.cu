@@ -353,7 +353,6 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     if (opts && opts->reserved != 0) return fail(MOK_ERR_INVALID_ARG, "opts.reserved must be 0");
     const mok_mxfp8_weights* mxw = nullptr;
     if (opts && opts->mxfp8) {
-        if (mode != MOK_MODE_STAGED) return fail(MOK_ERR_UNSUPPORTED, "MXFP8 path: staged mode only");
         mxw = static_cast<const mok_mxfp8_weights*>(w_gate);
         if (!mxw || !mxw->gate || !mxw->gate_scales || !mxw->up || !mxw->up_scales || !mxw->down ||
             !mxw->down_scales)
@@ -415,6 +414,12 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         P.wg = w_gate;
         P.wu = w_up;
         P.wd = w_down;
+        P.mxw = mxw;
+        if (mxw) {
+            P.ring_sc = base + L.xsc;
+            P.h_sc = base + L.hsc;
+            P.sc_rows = mx_sc_rows(L.buf_rows);
+        }
         P.ring = base + L.rows;
         P.h = base + L.h;
         P.out = reinterpret_cast<__half*>(base + L.out);

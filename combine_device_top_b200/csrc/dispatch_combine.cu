@@ -5,7 +5,7 @@
 // Both kernels are HBM-bound streams of 16-byte vectors: one warp per token,
 // a grid of a few CTAs per SM looping over the tokens.  The gather reads each
 // token once and writes it to its k rows (T*H*2 bytes in, N_s*H*2 out); the
-// combine reads N_s*H*4 bytes of fp32 per-slot outputs and writes T*H*2
+// combine reads N_s*H*2 bytes of fp16 per-slot outputs and writes T*H*2
 // bytes of bf16 y, rounding once.
 #include "dispatch_combine.cuh"
 #include "mok_internal.h"
@@ -55,8 +55,8 @@ __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens(ShardsIn xs, int S
 // bytes and the scale planes [H/128][sc_rows][4] the block scales (plane g,
 // byte b: block 4g + b), the operand form of the block-scaled MMA.
 // Each lane owns 8 consecutive elements, 4 lanes a block, a half-warp one
-// 4-block scale word; the step loop is warp-uniform (lanes past the end
-// join the shuffles with zeros).
+// 4-block scale word (warp_mx_quant8); the step loop is warp-uniform (lanes
+// past the end join the shuffles with zeros).
 __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens_mx(ShardsIn xs, int S_r, int H, int T, int k,
                                                                  const int32_t* __restrict__ pos,
                                                                  uint8_t* __restrict__ rows, uint8_t* __restrict__ xsc,
@@ -72,30 +72,9 @@ __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens_mx(ShardsIn xs, in
             const int c = c0 + lane * 8;
             const bool live = c < H;
             const uint4 raw = live ? __ldg(src + (c >> 3)) : make_uint4(0, 0, 0, 0);
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-            float v[8];
-            float amax = 0.f;
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 f = __bfloat1622float2(b2[p]);
-                v[2 * p] = f.x;
-                v[2 * p + 1] = f.y;
-                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            const int s = mx_block_exponent(amax);
-            const float inv = mx_pow2(-s);
-            const uint2 q = make_uint2((uint32_t)mx_e4m3x2(v[0] * inv, v[1] * inv) |
-                                           ((uint32_t)mx_e4m3x2(v[2] * inv, v[3] * inv) << 16),
-                                       (uint32_t)mx_e4m3x2(v[4] * inv, v[5] * inv) |
-                                           ((uint32_t)mx_e4m3x2(v[6] * inv, v[7] * inv) << 16));
-            // the half-warp's 4 block scales as one word (block 4g + b in byte b)
-            const uint32_t sb = (uint32_t)(s + 127);
-            const int h0 = lane & 16;
-            const uint32_t word = __shfl_sync(0xffffffffu, sb, h0) | (__shfl_sync(0xffffffffu, sb, h0 + 4) << 8) |
-                                  (__shfl_sync(0xffffffffu, sb, h0 + 8) << 16) |
-                                  (__shfl_sync(0xffffffffu, sb, h0 + 12) << 24);
+            uint2 q;
+            uint32_t word;
+            warp_mx_quant8(raw, q, word, lane);
             uint32_t* plane = reinterpret_cast<uint32_t*>(xsc) + (size_t)((c0 >> 7) + (lane >> 4)) * sc_rows;
             for (int j = 0; j < k; ++j) {
                 const int row = __shfl_sync(0xffffffffu, my_row, j);

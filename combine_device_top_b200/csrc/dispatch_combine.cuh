@@ -10,6 +10,7 @@
 #pragma once
 
 #include "mok_device.cuh"
+#include "mxfp8.cuh"
 
 namespace mok {
 
@@ -81,6 +82,35 @@ __device__ __forceinline__ bool bulk_stream_rows(int n, SrcF src_row, DstF dst_r
     bulk_wait_all();
     loads = base + loaded;
     return ok;
+}
+
+// MXFP8 quantisation of 256 consecutive elements of a bf16 row by one warp
+// (OCP MX: 32-element blocks, E8M0 scale, E4M3 values; mxfp8.cuh).  Lane l
+// holds elements 8l .. 8l + 7 in raw (zeros past the row's end), so 4 lanes
+// form a block.  Returns the lane's 8 E4M3 bytes in q and, in word, the 4
+// block scales of the lane's half-warp (block 4g + b of the half-warp in
+// byte b), valid on every lane.  All 32 lanes must call it.
+__device__ __forceinline__ void warp_mx_quant8(const uint4& raw, uint2& q, uint32_t& word, int lane) {
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    float v[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 f = __bfloat1622float2(b2[p]);
+        v[2 * p] = f.x;
+        v[2 * p + 1] = f.y;
+        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const int s = mx_block_exponent(amax);
+    const float inv = mx_pow2(-s);
+    q = make_uint2((uint32_t)mx_e4m3x2(v[0] * inv, v[1] * inv) | ((uint32_t)mx_e4m3x2(v[2] * inv, v[3] * inv) << 16),
+                   (uint32_t)mx_e4m3x2(v[4] * inv, v[5] * inv) | ((uint32_t)mx_e4m3x2(v[6] * inv, v[7] * inv) << 16));
+    const uint32_t sb = (uint32_t)(s + 127);
+    const int h0 = lane & 16;
+    word = __shfl_sync(0xffffffffu, sb, h0) | (__shfl_sync(0xffffffffu, sb, h0 + 4) << 8) |
+           (__shfl_sync(0xffffffffu, sb, h0 + 8) << 16) | (__shfl_sync(0xffffffffu, sb, h0 + 12) << 24);
 }
 
 // One warp: y[t] = bf16(sum_{j<k} g[t,j] * out[t,j,:]) in fp32, j ascending.

@@ -117,12 +117,6 @@ struct MxCfgT {
 };
 using MxCfg = MxCfgT<1, 4>;
 
-// Shared-memory layout used by code outside the GEMM roles (dispatch CTAs of
-// the persistent kernel place their row slots below SMEM_BAR_OFF).
-constexpr int GEMM_THREADS = Bf16Cfg::THREADS;
-constexpr int SMEM_BAR_OFF = Bf16Cfg::BAR_OFF;
-constexpr int SMEM_ALLOC = Bf16Cfg::SMEM;
-
 // One unit of work: C::SUB consecutive M tiles (fewer at the end of the M
 // range) of one phase over one chunk; the tiles share every token tile.
 struct Unit {

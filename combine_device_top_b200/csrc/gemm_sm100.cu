@@ -23,8 +23,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     gemm_cta<StagedSched, C>(maps, &mx, a, s, smem);
 }
 
-size_t gemm_smem_bytes() { return SMEM_ALLOC; }
-
 // Defaults measured on B200 (page shape and a 512-rows-per-expert case):
 // small raster groups paid.  Pairs of M tiles halve the token-tile bytes
 // each SM takes in per weight byte, but a pair of chunks taller than 128 rows

@@ -78,7 +78,6 @@ struct GemmTuning {
 // defaults for `rows` expert-major rows over E experts, overridable by
 // MOK_GEMM_GROUP / MOK_GEMM_PAIR
 GemmTuning gemm_tuning(int rows, int E);
-size_t gemm_smem_bytes();
 cudaError_t gemm_configure(int dev);
 // Token-side (B operand) tensor maps of one buffer with box heights 16, 32,
 // ..., 256 rows (map i has 16 * (i + 1) rows): a chunk of r rows is loaded
@@ -137,9 +136,12 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
 struct PersistLaunch {
     int grid, dispatch_ctas, cap;  // CTAs, of which the first dispatch_ctas gather; ring half rows
     int H, I, E, T, k, S_r;
-    const void *wg, *wu, *wd;      // weights (bf16, bf16, fp16)
-    void* ring;                    // [2*cap, H] bf16
-    void* h;                       // [2*cap, I] fp16
+    const void *wg, *wu, *wd;      // weights (bf16, bf16, fp16); unused on the MXFP8 path
+    const mok_mxfp8_weights* mxw;  // MXFP8 weights, or nullptr (bf16 path)
+    void* ring;                    // [2*cap, H] bf16, or E4M3 (MXFP8)
+    void* h;                       // [2*cap, I] fp16, or E4M3 (MXFP8)
+    uint8_t *ring_sc, *h_sc;       // MXFP8: scale planes of ring and h rows (sc_rows = mx_sc_rows(2*cap))
+    int sc_rows;
     __half* out;                   // [T*k, H] fp16
     const Chunk* chunks;
     const Minibatch* mbs;

@@ -14,7 +14,8 @@
 // One launch (cooperative, so every CTA is resident), one CTA per SM:
 //   CTAs [0, D)  dispatch/combine side: for each minibatch b, wait until ring
 //                half b % 2 is free (all down units of minibatch b - 2 done),
-//                gather b's rows into it, publish gathered[b].
+//                gather b's rows into it (MXFP8 path: quantised to E4M3 rows
+//                plus the ring's scale planes), publish gathered[b].
 //   CTAs [D, G)  GEMM side: the tcgen05 core of gemm_core.cuh over the units
 //                of every minibatch in order -- gate/up units of b, then its
 //                down units -- dealt round-robin.  A gate/up unit waits for
@@ -28,10 +29,13 @@
 // bounded; a wait that gives up records MOK_ERR_TIMEOUT and the kernel
 // leaves its loops.
 //
-// Memory ordering: rows and h are written with generic stores and read by
-// TMA (async proxy) in other CTAs.  Writers fence.proxy.async + threadfence,
+// Memory ordering: rows and h (and, MXFP8, their scale planes) are written
+// with generic stores and read by TMA or bulk copies (async proxy) in other
+// CTAs.  Writers fence.proxy.async + threadfence,
 // then one thread does a release add; readers do an acquire load, then
 // fence.proxy.async, then issue TMA.
+#include <cstring>
+
 #include "dispatch_combine.cuh"
 #include "gemm_core.cuh"
 
@@ -57,7 +61,8 @@ struct PersistParams {
     const int32_t* src_rank;
     const int32_t* src_index;
     const float* gates;
-    __nv_bfloat16* ring;  // [2 * cap, H]
+    void* ring;        // [2 * cap, H] bf16, or E4M3 bytes (MXFP8 path)
+    uint8_t* ring_sc;  // MXFP8 path: the ring rows' scale planes [H/128][sc_rows][4]
 };
 
 struct PersistSched {
@@ -117,11 +122,12 @@ struct PersistSched {
     }
 };
 
-// C: the GEMM CTAs' configuration (one M tile per unit, or pairs); both
-// share the thread count and shared-memory layout the dispatch side uses.
+// C: the GEMM CTAs' configuration (bf16 with one M tile per unit or pairs,
+// or MXFP8); the dispatch CTAs run with the same block shape.
 template <int KMAX, class C>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_moe_persistent(const __grid_constant__ GemmMaps maps, const CoreArgs a, const __grid_constant__ PersistParams p) {
+__global__ void __launch_bounds__(C::THREADS, 1)
+    k_moe_persistent(const __grid_constant__ GemmMaps maps, const __grid_constant__ MxMaps mx, const CoreArgs a,
+                     const __grid_constant__ PersistParams p) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ int s_ok;
     unsigned char* smem = align_smem_1024(smem_raw);
@@ -133,13 +139,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
     if ((int)blockIdx.x < D) {
         // ---------------------------------------- dispatch side: fill the ring
-        // One thread streams rows through the CTA's otherwise idle shared
-        // memory with bulk async copies (about 200 KB in flight per CTA);
-        // rows too wide for enough slots fall back to warp copies.
+        // bf16: one thread streams rows through the CTA's otherwise idle
+        // shared memory with bulk async copies (about 200 KB in flight per
+        // CTA); rows too wide for enough slots fall back to warp copies.
+        // MXFP8: a warp per row quantises it on the way (registers only).
         const uint32_t row_bytes = (uint32_t)a.H * 2u;
-        const int S = min(16, SMEM_BAR_OFF / (int)row_bytes);
-        const bool bulk = S > BULK_STORES_IN_FLIGHT;
-        uint64_t* slot_full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
+        const int S = min(16, C::BAR_OFF / (int)row_bytes);
+        const bool bulk = !C::MX && S > BULK_STORES_IN_FLIGHT;
+        uint64_t* slot_full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
         if (threadIdx.x == 0 && bulk) {
             for (int i = 0; i < S; ++i) mbar_init(&slot_full[i], 1);
             fence_mbar_init();
@@ -164,7 +171,40 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int r0 = mb.row0 + (int)((long long)n * blockIdx.x / D);
             const int r1 = mb.row0 + (int)((long long)n * (blockIdx.x + 1) / D);
             uint4* half = reinterpret_cast<uint4*>(p.ring) + (size_t)((b & 1) * p.cap) * nvec;
-            if (bulk) {
+            if constexpr (C::MX) {
+                // E4M3 row at ring row brow, its H/32 block scales in the planes;
+                // four 256-element steps' loads in flight per lane
+                uint32_t* planes = reinterpret_cast<uint32_t*>(p.ring_sc);
+                for (int r = r0 + warp; r < r1; r += C::THREADS / 32) {
+                    const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
+                    const uint4* src = reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec;
+                    const int brow = (b & 1) * p.cap + (r - mb.row0);
+                    uint8_t* dst = reinterpret_cast<uint8_t*>(p.ring) + (size_t)brow * a.H;
+                    for (int c0 = 0; c0 < a.H; c0 += 1024) {
+                        uint4 raw[4];
+#pragma unroll
+                        for (int s4 = 0; s4 < 4; ++s4) {
+                            const int c = c0 + 256 * s4 + lane * 8;
+                            raw[s4] = c < a.H ? __ldg(src + (c >> 3)) : make_uint4(0, 0, 0, 0);
+                        }
+#pragma unroll
+                        for (int s4 = 0; s4 < 4; ++s4) {
+                            const int cs = c0 + 256 * s4;
+                            if (cs < a.H) {  // warp-uniform
+                                uint2 q;
+                                uint32_t word;
+                                warp_mx_quant8(raw[s4], q, word, lane);
+                                const int c = cs + lane * 8;
+                                if (c < a.H) {
+                                    *reinterpret_cast<uint2*>(dst + c) = q;
+                                    if ((lane & 15) == 0)
+                                        planes[(size_t)((cs >> 7) + (lane >> 4)) * a.sc_rows + brow] = word;
+                                }
+                            }
+                        }
+                    }
+                }
+            } else if (bulk) {
                 if (threadIdx.x == 0) {
                     auto src = [&](int i) -> const void* {
                         const int r = r0 + i;
@@ -176,7 +216,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                                      DRAIN_TIMEOUT_NS);
                 }
             } else {
-                for (int r = r0 + warp; r < r1; r += GEMM_THREADS / 32) {
+                for (int r = r0 + warp; r < r1; r += C::THREADS / 32) {
                     const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
                     warp_copy_row(reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec,
                                   half + (size_t)(r - mb.row0) * nvec, nvec, lane);
@@ -197,7 +237,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         s.gidx = blockIdx.x - D;
         s.gctas = gridDim.x - D;
         s.total = nch * (p.MTG + p.MTD);
-        gemm_cta<PersistSched, C>(maps, nullptr, a, s, smem);
+        gemm_cta<PersistSched, C>(maps, &mx, a, s, smem);
     }
 
     // -------------------------------------------- combine, once every down unit is done
@@ -205,8 +245,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         s_ok = (!failed(a.st) && flag_wait_geq(p.d_total, nch * p.MTD, a.st, a.timeout_ns, 60)) ? 1 : 0;
     __syncthreads();
     if (!s_ok) return;
-    const int warps = gridDim.x * (GEMM_THREADS / 32);
-    for (int t = blockIdx.x * (GEMM_THREADS / 32) + warp; t < p.T; t += warps) {
+    const int warps = gridDim.x * (C::THREADS / 32);
+    for (int t = blockIdx.x * (C::THREADS / 32) + warp; t < p.T; t += warps) {
         const int r = t / p.S_r;
         uint4* dst = reinterpret_cast<uint4*>(p.ys.p[r]) + (size_t)(t - r * p.S_r) * nvec;
         warp_combine_token<KMAX>(reinterpret_cast<const uint4*>(a.out), p.gates, t, p.k, nvec, dst, lane);
@@ -214,36 +254,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 template <int KMAX, class C>
-static cudaError_t launch_persistent_k(int grid, const GemmMaps& maps, const CoreArgs& a, const PersistParams& p,
-                                       cudaStream_t stream) {
-    static_assert(C::THREADS == GEMM_THREADS && C::SMEM == SMEM_ALLOC && C::BAR_OFF == SMEM_BAR_OFF,
-                  "the dispatch side assumes the GEMM side's block shape");
+static cudaError_t launch_persistent_k(int grid, const GemmMaps& maps, const MxMaps& mx, const CoreArgs& a,
+                                       const PersistParams& p, cudaStream_t stream) {
     static bool attr[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr[dev]) {
-        e = cudaFuncSetAttribute(k_moe_persistent<KMAX, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+        e = cudaFuncSetAttribute(k_moe_persistent<KMAX, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr[dev] = true;
     }
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_moe_persistent<KMAX, C>, GEMM_THREADS, SMEM_ALLOC);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_moe_persistent<KMAX, C>, C::THREADS, C::SMEM);
     if (e != cudaSuccess) return e;
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     if (per_sm < 1 || grid > per_sm * sms) return cudaErrorCooperativeLaunchTooLarge;
-    void* args[] = {const_cast<GemmMaps*>(&maps), const_cast<CoreArgs*>(&a), const_cast<PersistParams*>(&p)};
+    void* args[] = {const_cast<GemmMaps*>(&maps), const_cast<MxMaps*>(&mx), const_cast<CoreArgs*>(&a),
+                    const_cast<PersistParams*>(&p)};
     return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_moe_persistent<KMAX, C>), dim3(grid),
-                                       dim3(GEMM_THREADS), args, SMEM_ALLOC, stream);
+                                       dim3(C::THREADS), args, C::SMEM, stream);
 }
 
 cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, cudaStream_t stream) {
     GemmMaps maps;
-    if (!encode_gemm_maps(&maps, L.wg, L.wu, L.wd, L.ring, L.h, L.H, L.I, L.E, 2 * L.cap, err))
+    MxMaps mx;
+    memset(&maps, 0, sizeof maps);
+    memset(&mx, 0, sizeof mx);
+    if (L.mxw) {
+        if (!encode_mx_maps(&mx, *L.mxw, L.H, L.I, L.E, err) ||
+            !encode_bmaps_u8(&maps.rows, L.ring, (uint64_t)L.H, (uint64_t)2 * L.cap, err) ||
+            !encode_bmaps_u8(&maps.h, L.h, (uint64_t)L.I, (uint64_t)2 * L.cap, err))
+            return cudaErrorInvalidValue;
+    } else if (!encode_gemm_maps(&maps, L.wg, L.wu, L.wd, L.ring, L.h, L.H, L.I, L.E, 2 * L.cap, err)) {
         return cudaErrorInvalidValue;
+    }
     CoreArgs a{};
     a.H = L.H;
     a.I = L.I;
@@ -252,13 +300,19 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     a.row_slot = L.row_slot;
     a.st = reinterpret_cast<DevStatus*>(L.status);
     a.timeout_ns = L.timeout_ns;
+    if (L.mxw) {
+        a.xsc = L.ring_sc;
+        a.hsc = L.h_sc;
+        a.sc_rows = L.sc_rows;
+    }
     PersistParams p;
     p.chunks = L.chunks;
     p.mbs = L.mbs;
     p.counts2 = L.counts2;
     p.cap = L.cap;
     // the staged GEMM's rule for M-tile pairs: mean rows per expert <= 192
-    const bool pair = gemm_tuning(L.T * L.k, L.E).pair != 0;
+    // (bf16 only; the MXFP8 path runs one M tile per unit)
+    const bool pair = !L.mxw && gemm_tuning(L.T * L.k, L.E).pair != 0;
     const int sub = pair ? Bf16PairCfg::SUB : Bf16Cfg::SUB;
     // units per chunk (with pairs the last one may be single)
     p.MTG = (L.I / MT_G_FEATURES + sub - 1) / sub;
@@ -276,14 +330,19 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.src_rank = L.src_rank;
     p.src_index = L.src_index;
     p.gates = L.gates;
-    p.ring = reinterpret_cast<__nv_bfloat16*>(L.ring);
+    p.ring = L.ring;
+    p.ring_sc = L.ring_sc;
     *err = "persistent launch";
-    if (pair) {
-        if (L.k <= 2) return launch_persistent_k<2, Bf16PairCfg>(L.grid, maps, a, p, stream);
-        return launch_persistent_k<8, Bf16PairCfg>(L.grid, maps, a, p, stream);
+    if (L.mxw) {
+        if (L.k <= 2) return launch_persistent_k<2, MxCfg>(L.grid, maps, mx, a, p, stream);
+        return launch_persistent_k<8, MxCfg>(L.grid, maps, mx, a, p, stream);
     }
-    if (L.k <= 2) return launch_persistent_k<2, Bf16Cfg>(L.grid, maps, a, p, stream);
-    return launch_persistent_k<8, Bf16Cfg>(L.grid, maps, a, p, stream);
+    if (pair) {
+        if (L.k <= 2) return launch_persistent_k<2, Bf16PairCfg>(L.grid, maps, mx, a, p, stream);
+        return launch_persistent_k<8, Bf16PairCfg>(L.grid, maps, mx, a, p, stream);
+    }
+    if (L.k <= 2) return launch_persistent_k<2, Bf16Cfg>(L.grid, maps, mx, a, p, stream);
+    return launch_persistent_k<8, Bf16Cfg>(L.grid, maps, mx, a, p, stream);
 }
 
 }  // namespace mok

@@ -156,8 +156,8 @@ typedef struct mok_fwd_opts {
                            /* 0 = default (16)                                  */
     int32_t gemm_ctas;     /* GEMM CTAs; 0 = all remaining SMs                  */
     int32_t mxfp8;         /* 1 = MXFP8 path (weights from                      */
-                           /* mok_quantize_weights_mxfp8; staged mode only,     */
-                           /* else MOK_ERR_UNSUPPORTED); 0 = bf16               */
+                           /* mok_quantize_weights_mxfp8; either mode);         */
+                           /* 0 = bf16                                          */
     int32_t reserved;      /* must be 0                                         */
     uint64_t timeout_ns;   /* bound on every device-side wait; 0 = 2 s          */
 } mok_fwd_opts;
@@ -207,8 +207,9 @@ size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int miniba
  * its slot (saturating); y[t] = bf16(sum_{j<k} g[t,j] * o[t,j]) accumulated in fp32
  * with j ascending (one bf16 rounding of y).  y does not depend on the
  * mode, minibatch, ring size or R.
- * MXFP8 path (opts->mxfp8 = 1, staged mode, w_gate = a mok_mxfp8_weights
- * HOST struct): x is quantised in the gather and h in the SwiGLU epilogue
+ * MXFP8 path (opts->mxfp8 = 1, either mode, w_gate = a mok_mxfp8_weights
+ * HOST struct): x is quantised in the gather (persistent mode: by the
+ * dispatch CTAs, into the ring) and h in the SwiGLU epilogue
  * (32-element blocks, E8M0 scale + E4M3 values, as mok_mxfp8_quantize_rows
  * does); both GEMMs run on the block-scaled E4M3 x E4M3 tensor-core MMA
  * with fp32 accumulation; slot outputs fp16 and the combine as above.

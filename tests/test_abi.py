@@ -98,7 +98,9 @@ def test_forward_rejects_unsupported_shapes():
 
 
 def test_forward_mxfp8_argument_rules():
-    """The MXFP8 path is staged only and needs every member of its weight pack."""
+    """The MXFP8 path runs in either mode, under the persistent mode's own
+    rules, and needs every member of its weight pack.  Every call here fails
+    validation before any launch (the pointers are not device memory)."""
     p = mok.PlanT(16, 8, 2, 2)
     for name in ("counts", "offsets", "sched_src_rank", "sched_src_index", "row_slot", "pos", "topk_idx", "gates"):
         setattr(p, name, 4096)
@@ -107,9 +109,16 @@ def test_forward_mxfp8_argument_rules():
     full = mok.MxWeights(4096, 4096, 4096, 4096, 4096, 4096)
     pack = ctypes.cast(ctypes.byref(full), ctypes.c_void_p)
     o = mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT, mxfp8=True)
-    rc = L.mok_moe_forward(arr, 128, 128, pack, None, None, ctypes.byref(p), 256, ctypes.byref(o), 256, 1 << 30,
+    rc = L.mok_moe_forward(arr, 128, 128, pack, None, None, ctypes.byref(p), 8, ctypes.byref(o), 256, 1 << 30,
                            arr, None)
-    assert rc == mok.MOK_ERR_UNSUPPORTED and "MXFP8" in mok.last_error()
+    assert rc == mok.MOK_ERR_INVALID_ARG and "minibatch" in mok.last_error()
+    rc = L.mok_moe_forward(arr, 128, 128, pack, None, None, ctypes.byref(p), 256, ctypes.byref(o), 256, 1, arr, None)
+    assert rc == mok.MOK_ERR_WORKSPACE
+    # the persistent MXFP8 workspace holds E4M3 rows and h plus their scale planes
+    need_mx = L.mok_forward_workspace_bytes(16, 128, 128, 8, 2, 256, ctypes.byref(o))
+    need_bf = L.mok_forward_workspace_bytes(16, 128, 128, 8, 2, 256,
+                                            ctypes.byref(mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT)))
+    assert 0 < need_mx < need_bf
     o = mok.fwd_opts(mode=mok.MOK_MODE_STAGED, mxfp8=True)
     holed = mok.MxWeights(4096, 4096, 4096, 0, 4096, 4096)
     rc = L.mok_moe_forward(arr, 128, 128, ctypes.cast(ctypes.byref(holed), ctypes.c_void_p), None, None,

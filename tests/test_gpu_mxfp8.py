@@ -127,10 +127,38 @@ def test_mxfp8_steps_one_at_a_time_equal_forward(name):
     assert torch.equal(torch.cat([s.cpu() for s in ys]), torch.cat([s.cpu() for s in y2]))
 
 
+@pytest.mark.parametrize("name,minibatch,ring,dispatch", [("tiny", 64, 0, 16), ("page_like", 256, 0, 4),
+                                                          ("page_like", 16, 0, 2), ("ragged", 600, 1300, 8)])
+def test_mxfp8_persistent_equals_staged(name, minibatch, ring, dispatch):
+    """The persistent SM-partitioned kernel on the MXFP8 path (its dispatch
+    CTAs quantise the rows into the ring) computes the staged path's bits at
+    every minibatch size, ring size and dispatch/GEMM split: quantisation is
+    per row and per 32-block, and each token's MMA column does not depend on
+    how the rows are cut into chunks."""
+    cfg = MX_CASES[name]
+    x = mokgen.tokens(cfg)
+    logits = mokgen.router_logits(cfg, x)
+    wg, wu, wd = mokgen.all_expert_weights(cfg)
+    pack = _mx_pack(wg.cuda(), wu.cuda(), wd.cuda())
+    p = mok.plan(logits.cuda(), cfg.k, cfg.R)
+    xs = mok.shards(x.cuda(), cfg.R)
+    ys_s, ws_s = mok.moe_forward_mxfp8(xs, pack, p)
+    opts = mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT, mxfp8=True, ring_slots=ring, dispatch_ctas=dispatch)
+    ys_p, ws_p = mok.moe_forward_mxfp8(xs, pack, p, minibatch=minibatch, opts=opts)
+    assert mok.get_status(ws_s) == mok.MOK_OK and mok.get_status(ws_p) == mok.MOK_OK
+    y_s = torch.cat([s.cpu() for s in ys_s])
+    y_p = torch.cat([s.cpu() for s in ys_p])
+    want = oracle.moe_forward_mxfp8(x, logits, wg, wu, wd, cfg.k, cfg.R)
+    rel = (torch.linalg.norm(y_p.double() - want) / torch.linalg.norm(want)).item()
+    assert rel <= REL_FRO_MX, rel
+    assert torch.equal(y_p, y_s), (y_p.double() - y_s.double()).abs().max().item()
+
+
 @pytest.mark.slow
 def test_mxfp8_forward_full_size_sampled():
-    """The page shape on the MXFP8 path: every row computed on the GPU,
-    sampled tokens against the emulated oracle."""
+    """The page shape on the MXFP8 path: every row computed on the GPU (staged,
+    and the persistent kernel bit-identical to it), sampled tokens against
+    the emulated oracle."""
     cfg = mokgen.CONFIGS["page_mxfp8"]
     x = mokgen.tokens(cfg)
     logits = mokgen.router_logits(cfg, x)
@@ -139,9 +167,17 @@ def test_mxfp8_forward_full_size_sampled():
     del wg, wu, wd
     torch.cuda.empty_cache()
     p = mok.plan(logits.cuda(), cfg.k, cfg.R)
-    ys, ws = mok.moe_forward_mxfp8(mok.shards(x.cuda(), cfg.R), pack, p)
+    xs = mok.shards(x.cuda(), cfg.R)
+    ys, ws = mok.moe_forward_mxfp8(xs, pack, p)
     assert mok.get_status(ws) == mok.MOK_OK
     y = torch.cat([s.cpu() for s in ys]).double()
+    del ws
+    # the persistent kernel at the minibatch bench.py times computes the same bits
+    opts = mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT, mxfp8=True)
+    ys_p, ws_p = mok.moe_forward_mxfp8(xs, pack, p, minibatch=2560, opts=opts)
+    assert mok.get_status(ws_p) == mok.MOK_OK
+    assert torch.equal(torch.cat([s.cpu() for s in ys_p]).double(), y)
+    del ws_p
     ids = sorted(set(torch.randperm(cfg.T, generator=torch.Generator().manual_seed(4))[:6].tolist()))
     idx, g = oracle.topk_gates(logits[ids], cfg.k)
     want = torch.zeros((len(ids), cfg.H), dtype=torch.float64)
