@@ -17,6 +17,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+from contextlib import contextmanager
 from functools import lru_cache
 
 import numpy as np
@@ -39,9 +40,41 @@ def build(force: bool = False) -> str:
     return _SO
 
 
-@lru_cache(maxsize=1)
+def build_from(srcs, out: str) -> str:
+    """Compile the given copies of the oracle's C sources into ``out`` with
+    the oracle's own flags (the planted-mistake tests build mutated copies)."""
+    subprocess.check_call(["gcc", *CFLAGS, *srcs, "-o", out, "-lm"])
+    return out
+
+
+_override = None
+
+
 def lib():
-    L = ctypes.CDLL(build())
+    """The oracle's C library: this package's build, or the one a
+    :func:`library` block selected."""
+    return _override if _override is not None else _own_lib()
+
+
+@contextmanager
+def library(path: str):
+    """Run every oracle function inside the block on another build of the
+    oracle's sources (test use: mutated copies)."""
+    global _override
+    prev = _override
+    _override = _bind(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _override = prev
+
+
+@lru_cache(maxsize=1)
+def _own_lib():
+    return _bind(ctypes.CDLL(build()))
+
+
+def _bind(L):
     i32, vp = ctypes.c_int, ctypes.c_void_p
     L.oracle_topk_gates.argtypes = [vp, i32, i32, i32, vp, vp]
     L.oracle_schedule.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]

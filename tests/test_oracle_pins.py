@@ -235,6 +235,25 @@ def test_e4m3_decode_table_values():
     assert len(set(vals)) == 127 and vals[-1] == 448.0
 
 
+def test_e4m3_midpoints_round_to_even():
+    """Round half to even, from the grid alone: the midpoint of two adjacent
+    positive E4M3 values (scale 2^0) encodes to the neighbour whose code is
+    even, and a point just off the midpoint to the nearer neighbour."""
+    L = oracle.lib()
+    codes = sorted(range(0x7F), key=L.oracle_e4m3_decode)   # 0x00 .. 0x7E ascending
+    for lo, hi in zip(codes[:-1], codes[1:]):
+        a, b = L.oracle_e4m3_decode(lo), L.oracle_e4m3_decode(hi)
+        mid = (a + b) / 2
+        eps = (b - a) / 8
+        v = np.zeros(32 * 3, np.float32)
+        v[0::32] = 448.0                  # every block's exponent is 0
+        v[1], v[33], v[65] = mid, mid - eps, mid + eps
+        q, s = _quant(v)
+        assert (s == 127).all()
+        assert q[1] == (lo if lo % 2 == 0 else hi), (hex(lo), hex(hi))
+        assert q[33] == lo and q[65] == hi, (hex(lo), hex(hi))
+
+
 def test_mxfp8_relative_error_bound():
     """Non-saturated elements above the subnormal range are within 2^-4
     relative of the input (3 mantissa bits, round to nearest)."""
