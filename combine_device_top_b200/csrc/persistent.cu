@@ -47,7 +47,7 @@ struct PersistParams {
     const Minibatch* mbs;
     const int* counts2;  // [0] chunks, [1] minibatches
     int cap;             // rows per ring half
-    int MTG, MTD;        // units (groups of Bf16Cfg::SUB M tiles) per chunk of the gate/up and down phases
+    int MTG, MTD;        // units (groups of C::SUB M tiles) per chunk of the gate/up and down phases
     int dispatch_ctas;
     // counters (zeroed before the launch)
     int* gathered;  // [max_mb]  dispatch CTAs done with minibatch b
