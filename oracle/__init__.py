@@ -4,8 +4,10 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product (``combine_device_top_b200``)
 never imports it and shares no code with it.
 
-The arithmetic lives in ``mok_oracle.c`` (plain C, double precision, compiled
-with gcc); this file is ctypes marshalling plus small conveniences.  Each C
+The arithmetic lives in ``mok_oracle.c`` (forward), ``mxfp8_oracle.c``
+(MXFP8 emulation) and ``mok_oracle_bwd.c`` (backward): plain C, double
+precision, compiled with gcc; this file is ctypes marshalling plus small
+conveniences.  Each C
 function cites the passage of the pages it follows.
 
 Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
@@ -24,7 +26,7 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = [os.path.join(_HERE, "mok_oracle.c"), os.path.join(_HERE, "mxfp8_oracle.c")]
+_SRCS = [os.path.join(_HERE, f) for f in ("mok_oracle.c", "mxfp8_oracle.c", "mok_oracle_bwd.c")]
 _SO = os.path.join(_HERE, "liboracle.so")
 CFLAGS = ["-O3", "-march=x86-64-v3", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
 
@@ -90,6 +92,9 @@ def _bind(L):
         L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_decode.restype = ctypes.c_double
         L.oracle_mxfp8_expert_ffn.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    if hasattr(L, "oracle_moe_backward"):
+        L.oracle_moe_backward.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.oracle_moe_backward.restype = ctypes.c_int
     for name in ("oracle_topk_gates", "oracle_schedule", "oracle_gather", "oracle_expert_ffn",
                  "oracle_combine", "oracle_moe_forward", "oracle_num_threads"):
         getattr(L, name).restype = ctypes.c_int
@@ -224,6 +229,24 @@ def moe_forward(x, logits, wg, wu, wd, k: int, R: int):
                                     _ptr(_c(wd, torch.bfloat16)), _ptr(y), _ptr(idx), _ptr(g)),
            "moe_forward")
     return y, idx, g
+
+
+def moe_backward(x, logits, wg, wu, wd, dy, k: int, R: int):
+    """Backward of the whole layer on small inputs (``mok_oracle_bwd.c``):
+    given dy [T,H], returns dict(dx [T,H], dwg, dwu [E,H,I], dwd [E,I,H],
+    dlogits [T,E]), all float64."""
+    x = _c(x, torch.bfloat16)
+    logits = _c(logits, torch.float32)
+    T, H = x.shape
+    E, _, I = wg.shape
+    out = dict(dx=torch.empty((T, H), dtype=torch.float64), dwg=torch.empty((E, H, I), dtype=torch.float64),
+               dwu=torch.empty((E, H, I), dtype=torch.float64), dwd=torch.empty((E, I, H), dtype=torch.float64),
+               dlogits=torch.empty((T, E), dtype=torch.float64))
+    _check(lib().oracle_moe_backward(_ptr(x), _ptr(logits), T, H, I, E, k, R, _ptr(_c(wg, torch.bfloat16)),
+                                     _ptr(_c(wu, torch.bfloat16)), _ptr(_c(wd, torch.bfloat16)),
+                                     _ptr(_c(dy, torch.float64)), *(_ptr(out[n]) for n in
+                                     ("dx", "dwg", "dwu", "dwd", "dlogits"))), "moe_backward")
+    return out
 
 
 def forward_tokens(cfg, x, logits, token_ids, weight_fn, k=None):

@@ -4,10 +4,11 @@ Each mutant is a copy of the oracle's C sources with ONE plausible error of
 the kinds the pins are there to catch: a tie rule turned round, a wrong
 sign, a dropped term, a wrong or transposed index, a forgotten shard base,
 a result left at the wrong slot, an off-by-one exponent, another rounding
-rule.  The copy is compiled with the oracle's own flags and every pin of
-test_oracle_pins.py runs on it; at least one pin must fail.  An unmodified
-copy, built the same way, must pass them all (the control), so a failure
-comes from the planted mistake and not from the harness.
+rule, a term of the backward's chain rule.  The copy is compiled with the
+oracle's own flags and every pin of test_oracle_pins.py runs on it; at
+least one pin must fail.  An unmodified copy, built the same way, must pass
+them all (the control), so a failure comes from the planted mistake and not
+from the harness.
 """
 import os
 import shutil
@@ -18,7 +19,7 @@ import oracle
 import test_oracle_pins as pins
 
 ORACLE_DIR = os.path.dirname(os.path.abspath(oracle.__file__))
-SOURCES = ("mok_oracle.c", "mxfp8_oracle.c")
+SOURCES = ("mok_oracle.c", "mxfp8_oracle.c", "mok_oracle_bwd.c")
 
 # name -> (source file, text as written, text with the mistake)
 MUTANTS = {
@@ -72,6 +73,21 @@ MUTANTS = {
     "mx_zero_block_scale": ("mxfp8_oracle.c", "if (amax == 0.0) return -127;", "if (amax == 0.0) return 0;"),
     "mx_h_not_quantised": (
         "mxfp8_oracle.c", "mx_roundtrip(hv, I, hq);", "memcpy(hq, hv, sizeof(double) * (size_t)I);"),
+    # backward
+    "bwd_silu_derivative_term_dropped": (
+        "mok_oracle_bwd.c", "da[i] = dh[i] * b[i] * (s + a[i] * s * (1.0 - s));", "da[i] = dh[i] * b[i] * s;"),
+    "bwd_softmax_dot_dropped": (
+        "mok_oracle_bwd.c", "g[(size_t)t * k + j] * (dg[(size_t)t * k + j] - dot);",
+        "g[(size_t)t * k + j] * dg[(size_t)t * k + j];"),
+    "bwd_reverse_combine_without_gate": (
+        "mok_oracle_bwd.c", "dout[c] = g[slot] * dyt[c];", "dout[c] = dyt[c];"),
+    "bwd_dwd_from_preactivation": (
+        "mok_oracle_bwd.c", "dWd[(size_t)i * H + c] += h[i] * dout[c];", "dWd[(size_t)i * H + c] += a[i] * dout[c];"),
+    "bwd_dwu_takes_gate_branch": (
+        "mok_oracle_bwd.c", "dWu[(size_t)c * I + i] += xr[c] * db[i];", "dWu[(size_t)c * I + i] += xr[c] * da[i];"),
+    "bwd_up_gradient_sign": ("mok_oracle_bwd.c", "db[i] = dh[i] * a[i] * s;", "db[i] = -dh[i] * a[i] * s;"),
+    "bwd_dx_pushed_to_wrong_token": (
+        "mok_oracle_bwd.c", "dx[(size_t)t * H + c] += acc;", "dx[(size_t)((t + 1) % T) * H + c] += acc;"),
 }
 
 

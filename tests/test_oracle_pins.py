@@ -316,3 +316,63 @@ def test_two_wave_minibatch_golden():
     tiles_per_row = (2 * g["I"] / g["tile_cols"]) / g["tile_rows"]
     m = g["waves"] * g["sms"] / tiles_per_row
     assert m == g["minibatch_min"]
+
+
+# ---------------------------------------------------------------- backward (next row: the oracle first)
+def _dense_layer_autograd(x, logits, wg, wu, wd, dy, k):
+    """The forward layer's definition in float64 torch ops, differentiated by
+    torch.autograd: every expert evaluated densely, the top-k chosen by the
+    (logit desc, index asc) order, gates = torch.softmax of the chosen
+    logits.  Returns the gradients of sum(y * dy)."""
+    T, E = logits.shape
+    xd = x.double().requires_grad_()
+    ld = logits.double().requires_grad_()
+    ws = [w.double().requires_grad_() for w in (wg, wu, wd)]
+    sel = torch.tensor([sorted(range(E), key=lambda e: (-logits[t, e].item(), e))[:k] for t in range(T)])
+    g = torch.softmax(torch.gather(ld, 1, sel), dim=1)
+    y = torch.zeros(T, x.shape[1], dtype=torch.float64)
+    for t in range(T):
+        for j in range(k):
+            e = int(sel[t, j])
+            o = (torch.nn.functional.silu(xd[t] @ ws[0][e]) * (xd[t] @ ws[1][e])) @ ws[2][e]
+            y[t] = y[t] + g[t, j] * o
+    (y * dy).sum().backward()
+    return dict(dx=xd.grad, dwg=ws[0].grad, dwu=ws[1].grad, dwd=ws[2].grad, dlogits=ld.grad), sel
+
+
+@pytest.mark.parametrize("T,H,I,E,k,R", [(6, 32, 24, 5, 2, 2), (4, 16, 40, 3, 3, 4), (5, 24, 16, 6, 1, 1)])
+def test_backward_matches_autograd_of_dense_layer(T, H, I, E, k, R):
+    cfg, x, logits, wg, wu, wd = _rand_case(T, H, I, E, k, R, seed=60 + T + E)
+    dy = torch.randn(T, H, dtype=torch.float64, generator=torch.Generator().manual_seed(T * E))
+    got = oracle.moe_backward(x, logits, wg, wu, wd, dy, k, R)
+    want, _ = _dense_layer_autograd(x, logits, wg, wu, wd, dy, k)
+    for name in ("dx", "dwg", "dwu", "dwd", "dlogits"):
+        assert torch.allclose(got[name], want[name], rtol=1e-9, atol=1e-12), name
+
+
+def test_backward_gate_gradient_invariants():
+    """Adding one constant to a token's selected logits leaves y unchanged,
+    so their gradients sum to zero; unselected logits get no gradient; with
+    k = 1 the gate is constant and every logit gradient is zero."""
+    cfg, x, logits, wg, wu, wd = _rand_case(32, 32, 16, 7, 3, 2, seed=71)
+    dy = torch.randn(32, 32, dtype=torch.float64, generator=torch.Generator().manual_seed(2))
+    got = oracle.moe_backward(x, logits, wg, wu, wd, dy, 3, 2)
+    idx, _ = oracle.topk_gates(logits, 3)
+    mask = torch.zeros(32, 7, dtype=torch.bool)
+    mask.scatter_(1, idx.long(), True)
+    dl = got["dlogits"]
+    assert (dl[~mask] == 0).all()
+    assert torch.allclose(dl.sum(1), torch.zeros(32, dtype=torch.float64), atol=1e-12)
+    assert (dl[mask] != 0).any()
+    got1 = oracle.moe_backward(x, logits, wg, wu, wd, dy, 1, 2)
+    assert (got1["dlogits"] == 0).all()
+
+
+def test_backward_unselected_expert_gets_no_weight_gradient():
+    cfg, x, logits, wg, wu, wd = _rand_case(16, 32, 16, 4, 2, 2, seed=72)
+    logits = logits.clone()
+    logits[:, 2] = -1e4                      # expert 2 is never chosen
+    dy = torch.randn(16, 32, dtype=torch.float64, generator=torch.Generator().manual_seed(3))
+    got = oracle.moe_backward(x, logits, wg, wu, wd, dy, 2, 2)
+    for name in ("dwg", "dwu", "dwd"):
+        assert (got[name][2] == 0).all() and (got[name][0] != 0).any(), name
