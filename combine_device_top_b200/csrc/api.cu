@@ -349,7 +349,8 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     if (rc) return rc;
     if ((rc = check_hi(H, I))) return rc;
     const int mode = opts ? opts->mode : MOK_MODE_PERSISTENT;
-    if (mode != MOK_MODE_STAGED && mode != MOK_MODE_PERSISTENT) return fail(MOK_ERR_INVALID_ARG, "unknown mode %d", mode);
+    if (mode != MOK_MODE_STAGED && mode != MOK_MODE_PERSISTENT)
+        return fail(MOK_ERR_INVALID_ARG, "unknown mode %d", mode);
     if (opts && opts->reserved != 0) return fail(MOK_ERR_INVALID_ARG, "opts.reserved must be 0");
     const mok_mxfp8_weights* mxw = nullptr;
     if (opts && opts->mxfp8) {

@@ -1,9 +1,10 @@
 // worklist.cu -- the device-built work list of the grouped GEMM: minibatch
 // boundaries over the expert-major rows and chunks of at most max_rows (256,
-// or 224 on the MXFP8 path) rows of one expert inside one minibatch.  Built from `offsets` on the device, so the
-// forward needs no host round trip (MoK wiki summary, key points: schedule
-// built on the device without CPU-GPU traffic; MoK article, minibatch
-// paragraph: a minibatch is the unit handed to the expert computation).
+// or 224 on the MXFP8 path) rows of one expert inside one minibatch.  Built
+// from `offsets` on the device, so the forward needs no host round trip (MoK
+// wiki summary, key points: schedule built on the device without CPU-GPU
+// traffic; MoK article, minibatch paragraph: a minibatch is the unit handed
+// to the expert computation).
 #include "mok_device.cuh"
 #include "mok_internal.h"
 
