@@ -73,6 +73,14 @@ MUTANTS = {
     "mx_zero_block_scale": ("mxfp8_oracle.c", "if (amax == 0.0) return -127;", "if (amax == 0.0) return 0;"),
     "mx_h_not_quantised": (
         "mxfp8_oracle.c", "mx_roundtrip(hv, I, hq);", "memcpy(hq, hv, sizeof(double) * (size_t)I);"),
+    "mx_x_not_quantised": (
+        "mxfp8_oracle.c", "mx_roundtrip(xr, H, xq);", "memcpy(xq, xr, sizeof(double) * (size_t)H);"),
+    "mx_up_weights_not_quantised": (
+        "mxfp8_oracle.c", "mx_roundtrip(col, H, qu + (size_t)i * H);",
+        "memcpy(qu + (size_t)i * H, col, sizeof(double) * (size_t)H);"),
+    "mx_down_weight_read_transposed": (
+        "mxfp8_oracle.c", "for (int k = 0; k < I; ++k) col[k] = o_bf16(wd[(size_t)k * H + c]);",
+        "for (int k = 0; k < I; ++k) col[k] = o_bf16(wd[((size_t)c * I + k) % ((size_t)I * H)]);"),
     # backward
     "bwd_silu_derivative_term_dropped": (
         "mok_oracle_bwd.c", "da[i] = dh[i] * b[i] * (s + a[i] * s * (1.0 - s));", "da[i] = dh[i] * b[i] * s;"),

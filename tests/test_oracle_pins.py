@@ -306,6 +306,39 @@ def test_mxfp8_ffn_exact_on_representable_inputs():
     assert np.allclose(o, want, rtol=1e-12, atol=1e-300)
 
 
+def _dequant_rows(a: np.ndarray) -> np.ndarray:
+    """Rows of a 2D array through the pinned quantiser (blocks of 32 along
+    each row) and back to exact values."""
+    L = oracle.lib()
+    q, s = _quant(np.ascontiguousarray(a, dtype=np.float32).reshape(-1))
+    dec = np.array([L.oracle_e4m3_decode(int(v)) for v in q])
+    return (dec * np.repeat(np.ldexp(1.0, s.astype(int) - 127), 32)).reshape(a.shape)
+
+
+def test_mxfp8_ffn_is_quantise_then_exact_gemms():
+    """On arbitrary (off-grid) inputs the MXFP8 FFN equals its definition
+    assembled from the separately pinned quantiser: x quantised along H, Wg
+    and Wu along their contraction index H (per output column), Wd along I
+    (per output column), exact products, h rounded to fp32 and quantised
+    along I, exact down projection."""
+    n, H, I = 3, 96, 64
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(n, H, generator=g).to(torch.bfloat16)
+    wg, wu = ((torch.randn(H, I, generator=g) / H ** 0.5).to(torch.bfloat16) for _ in range(2))
+    wd = (torch.randn(I, H, generator=g) / I ** 0.5).to(torch.bfloat16)
+    got = oracle.mxfp8_expert_ffn(x, wg, wu, wd).numpy()
+    xq = _dequant_rows(x.float().numpy())
+    gq = _dequant_rows(wg.float().numpy().T).T            # blocks along H for each column of Wg
+    uq = _dequant_rows(wu.float().numpy().T).T
+    dq = _dequant_rows(wd.float().numpy().T).T            # blocks along I for each column of Wd
+    a, b = xq @ gq, xq @ uq
+    h = (a / (1.0 + np.exp(-a)) * b).astype(np.float32)
+    want = _dequant_rows(h) @ dq
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-15)
+    # and the quantisation is not the identity on these inputs
+    assert not np.allclose(xq, x.double().numpy(), rtol=1e-6)
+
+
 # ---------------------------------------------------------------- pages' worked number
 def test_two_wave_minibatch_golden():
     """The pages' one reproducible number: about 2368 tokens for two full waves
