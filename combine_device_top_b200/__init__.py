@@ -229,7 +229,8 @@ def moe_forward(x_shards, w_gate, w_up, w_down, p: Plan, minibatch: int = 2560, 
                 y_shards=None, ws: torch.Tensor | None = None, stream=None):
     """Steps 3-5: ``mok_moe_forward``.  Returns (y_shards, ws)."""
     R = p.c.R
-    assert len(x_shards) == R
+    # the library reads R pointers from each shard array
+    assert len(x_shards) == R and (y_shards is None or len(y_shards) == R)
     H = x_shards[0].shape[1]
     I = w_gate.shape[-1]
     dev = x_shards[0].device
@@ -261,6 +262,8 @@ def moe_forward_mxfp8(x_shards, pack, p: Plan, y_shards=None, ws: torch.Tensor |
     for the persistent kernel.  Returns (y_shards, ws)."""
     qg, sg, qu, su, qd, sd = pack
     R = p.c.R
+    # the library reads R pointers from each shard array
+    assert len(x_shards) == R and (y_shards is None or len(y_shards) == R)
     H = x_shards[0].shape[1]
     I = qg.shape[-1]
     dev = x_shards[0].device
@@ -270,12 +273,14 @@ def moe_forward_mxfp8(x_shards, pack, p: Plan, y_shards=None, ws: torch.Tensor |
     if y_shards is None:
         y_shards = [torch.empty_like(s) for s in x_shards]
     if ws is None:
-        ws = _workspace(forward_workspace_bytes(p.c.T, H, I, p.c.E, p.c.k, minibatch, opts), dev)
+        need = forward_workspace_bytes(p.c.T, H, I, p.c.E, p.c.k, minibatch, opts)
+        if need == 0:
+            raise MokError(MOK_ERR_INVALID_ARG, "invalid forward shape")
+        ws = _workspace(need, dev)
     w = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
     _check(lib().mok_moe_forward(_ptr_array(x_shards), H, I, ctypes.cast(ctypes.byref(w), ctypes.c_void_p), None,
                                  None, ctypes.byref(p.c), minibatch, ctypes.byref(opts),
                                  ctypes.c_void_p(ws.data_ptr()), ws.numel(), _ptr_array(y_shards), _stream(stream)))
-    assert len(x_shards) == R
     return y_shards, ws
 
 
@@ -290,6 +295,7 @@ def last_error() -> str:
 
 
 def gather(x_shards, p: Plan, rows: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    assert len(x_shards) == p.c.R
     H = x_shards[0].shape[1]
     if rows is None:
         rows = torch.empty((p.ns, H), dtype=torch.bfloat16, device=x_shards[0].device)
@@ -300,6 +306,7 @@ def gather(x_shards, p: Plan, rows: torch.Tensor | None = None, stream=None) -> 
 
 def gather_mxfp8(x_shards, p: Plan, rows_q=None, scales=None, stream=None):
     """The MXFP8 gather: (rows_q [N_s, H] uint8 E4M3, scales [H/128, sc_rows, 4] uint8 E8M0)."""
+    assert len(x_shards) == p.c.R
     H = x_shards[0].shape[1]
     dev = x_shards[0].device
     if rows_q is None:
@@ -348,7 +355,7 @@ def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = N
 
 def combine(out: torch.Tensor, p: Plan, y_shards, stream=None):
     """y = fixed-order gate-weighted sum of the fp16 per-slot outputs (fp32 accumulation)."""
-    assert out.dtype == torch.float16
+    assert out.dtype == torch.float16 and len(y_shards) == p.c.R
     H = out.shape[-1]
     _check(lib().mok_combine(ctypes.c_void_p(out.data_ptr()), H, ctypes.byref(p.c), _ptr_array(y_shards),
                              _stream(stream)))
