@@ -156,3 +156,25 @@ def test_mxfp8_step_entry_points_reject_bad_arguments():
     assert rc == mok.MOK_ERR_INVALID_ARG and "NULL" in mok.last_error()
     rc = L.mok_expert_ffn_mxfp8(4096, 8192, 256, 256, None, ctypes.byref(p), 256, need - 1, 4096, None)
     assert rc == mok.MOK_ERR_WORKSPACE
+
+
+def test_binding_checks_shard_count_before_calling_the_library():
+    """The library reads R pointers from each shard array, so the binding
+    rejects a list of another length before any call (no device needed)."""
+    import torch
+
+    p = mok.Plan(mok.PlanT(16, 8, 2, 2), torch.empty(256, dtype=torch.uint8))
+    one = [torch.empty(8, 128, dtype=torch.bfloat16)]          # R = 2 expected
+    w = torch.empty(8, 128, 128, dtype=torch.bfloat16)
+    pack = tuple(torch.empty(8, 128, 128, dtype=torch.uint8) for _ in range(6))
+    out = torch.empty(32, 128, dtype=torch.float16)
+    with pytest.raises(AssertionError):
+        mok.moe_forward(one, w, w, w, p)
+    with pytest.raises(AssertionError):
+        mok.moe_forward_mxfp8(one, pack, p)
+    with pytest.raises(AssertionError):
+        mok.gather(one, p)
+    with pytest.raises(AssertionError):
+        mok.gather_mxfp8(one, p)
+    with pytest.raises(AssertionError):
+        mok.combine(out, p, one)
