@@ -5,7 +5,8 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 never imports it and shares no code with it.
 
 The arithmetic lives in ``mok_oracle.c`` (forward), ``mxfp8_oracle.c``
-(MXFP8 emulation) and ``mok_oracle_bwd.c`` (backward): plain C, double
+(MXFP8 emulation), ``mok_oracle_bwd.c`` (backward) and
+``mok_oracle_router.c`` (router projection): plain C, double
 precision, compiled with gcc; this file is ctypes marshalling plus small
 conveniences.  Each C
 function cites the passage of the pages it follows.
@@ -26,7 +27,8 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = [os.path.join(_HERE, f) for f in ("mok_oracle.c", "mxfp8_oracle.c", "mok_oracle_bwd.c")]
+_SRCS = [os.path.join(_HERE, f) for f in ("mok_oracle.c", "mxfp8_oracle.c", "mok_oracle_bwd.c",
+                                           "mok_oracle_router.c")]
 _SO = os.path.join(_HERE, "liboracle.so")
 CFLAGS = ["-O3", "-march=x86-64-v3", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
 
@@ -92,6 +94,9 @@ def _bind(L):
         L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_decode.restype = ctypes.c_double
         L.oracle_mxfp8_expert_ffn.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    if hasattr(L, "oracle_router_logits"):
+        L.oracle_router_logits.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+        L.oracle_router_logits.restype = ctypes.c_int
     if hasattr(L, "oracle_moe_backward"):
         L.oracle_moe_backward.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.oracle_moe_backward.restype = ctypes.c_int
@@ -229,6 +234,20 @@ def moe_forward(x, logits, wg, wu, wd, k: int, R: int):
                                     _ptr(_c(wd, torch.bfloat16)), _ptr(y), _ptr(idx), _ptr(g)),
            "moe_forward")
     return y, idx, g
+
+
+def router_logits(x, w_r, prior=None):
+    """Router projection (``mok_oracle_router.c``): x bf16 [T,H], W_r fp32
+    [H,E], optional fp32 prior [E] -> logits [T,E] float64."""
+    x = _c(x, torch.bfloat16)
+    w_r = _c(w_r, torch.float32)
+    T, H = x.shape
+    E = w_r.shape[1]
+    out = torch.empty((T, E), dtype=torch.float64)
+    pr = _c(prior, torch.float32) if prior is not None else None
+    _check(lib().oracle_router_logits(_ptr(x), _ptr(w_r), _ptr(pr) if pr is not None else None, T, H, E,
+                                      _ptr(out)), "router_logits")
+    return out
 
 
 def moe_backward(x, logits, wg, wu, wd, dy, k: int, R: int):

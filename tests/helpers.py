@@ -81,3 +81,31 @@ def sample_tokens(T: int, n: int, seed: int = 0) -> list[int]:
     g = torch.Generator().manual_seed(seed)
     ids = torch.randperm(T, generator=g)[:n].tolist()
     return sorted(set(ids + [0, T - 1]))
+
+
+def topk_within_tolerance(idx: torch.Tensor, exact: torch.Tensor, tol: torch.Tensor):
+    """Check a top-k selection made from rounded logits against exact ones.
+
+    idx [T, k] (rank order), exact [T, E] float64, tol [T] float64: the
+    largest difference rounding may cause between two logits of a token.
+    Where exact logits lie within tol of each other either order is
+    correct; everywhere else the selection and its order are fixed.
+    Returns (ok [T], strict [T]): ok = the selection is one of the correct
+    ones (k distinct experts, none left out that beats a chosen one by more
+    than tol, rank order non-increasing up to tol); strict = the token has a
+    single correct selection (every gap that decides it exceeds tol), so it
+    must equal the exact top-k with the lower-index tie rule.
+    """
+    T, k = idx.shape
+    E = exact.shape[1]
+    idx = idx.long()
+    sel = torch.gather(exact, 1, idx)                                  # [T, k]
+    chosen = torch.zeros(T, E, dtype=torch.bool).scatter_(1, idx, True)
+    distinct = chosen.sum(1) == k
+    rest_max = torch.where(chosen, torch.full_like(exact, -math.inf), exact).max(1).values
+    kth = sel.min(1).values
+    order_ok = (sel[:, :-1] >= sel[:, 1:] - tol[:, None]).all(1) if k > 1 else torch.ones(T, dtype=torch.bool)
+    ok = distinct & (kth >= rest_max - tol) & order_ok
+    gaps_ok = ((sel[:, :-1] - sel[:, 1:]).abs() > tol[:, None]).all(1) if k > 1 else torch.ones(T, dtype=torch.bool)
+    strict = ok & (kth > rest_max + tol) & gaps_ok
+    return ok, strict

@@ -19,7 +19,7 @@ import oracle
 import test_oracle_pins as pins
 
 ORACLE_DIR = os.path.dirname(os.path.abspath(oracle.__file__))
-SOURCES = ("mok_oracle.c", "mxfp8_oracle.c", "mok_oracle_bwd.c")
+SOURCES = ("mok_oracle.c", "mxfp8_oracle.c", "mok_oracle_bwd.c", "mok_oracle_router.c")
 
 # name -> (source file, text as written, text with the mistake)
 MUTANTS = {
@@ -81,6 +81,13 @@ MUTANTS = {
     "mx_down_weight_read_transposed": (
         "mxfp8_oracle.c", "for (int k = 0; k < I; ++k) col[k] = o_bf16(wd[(size_t)k * H + c]);",
         "for (int k = 0; k < I; ++k) col[k] = o_bf16(wd[((size_t)c * I + k) % ((size_t)I * H)]);"),
+    # router projection
+    "router_prior_dropped": (
+        "mok_oracle_router.c", "for (int e = 0; e < E; ++e) out[e] = prior ? (double)prior[e] : 0.0;",
+        "for (int e = 0; e < E; ++e) out[e] = 0.0;"),
+    "router_weight_read_transposed": (
+        "mok_oracle_router.c", "out[e] += xv * (double)w[e];",
+        "out[e] += xv * (double)wr[((size_t)e * H + h) % ((size_t)H * E)];"),
     # backward
     "bwd_silu_derivative_term_dropped": (
         "mok_oracle_bwd.c", "da[i] = dh[i] * b[i] * (s + a[i] * s * (1.0 - s));", "da[i] = dh[i] * b[i] * s;"),

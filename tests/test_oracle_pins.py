@@ -409,3 +409,34 @@ def test_backward_unselected_expert_gets_no_weight_gradient():
     got = oracle.moe_backward(x, logits, wg, wu, wd, dy, 2, 2)
     for name in ("dwg", "dwu", "dwd"):
         assert (got[name][2] == 0).all() and (got[name][0] != 0).any(), name
+
+
+# ---------------------------------------------------------------- router projection (next row)
+def test_router_identity_closed_form():
+    """W_r = [I_E; 0] picks the first E features: logits = x[:, :E] (+ prior), exactly."""
+    T, H, E = 16, 48, 12
+    x = mokgen.normal(1, 5, (T, H), 1.0)
+    w = torch.zeros(H, E)
+    w[:E, :E] = torch.eye(E)
+    prior = torch.linspace(-1.0, 1.0, E)
+    assert torch.equal(oracle.router_logits(x, w), x[:, :E].double())
+    assert torch.equal(oracle.router_logits(x, w, prior), x[:, :E].double() + prior.double())
+
+
+@pytest.mark.parametrize("name", ["tiny", "page", "zipf"])
+def test_router_matches_fp32_host_logits_within_rounding_bound(name):
+    """The harness's fp32 logits (its own fp32 product) lie within the
+    textbook bound of an fp32 dot product of H terms plus the prior add,
+    gamma_{H+1} * (sum_h |x_h w_he| + |prior_e|), of the oracle's values."""
+    cfg = mokgen.scaled(mokgen.CONFIGS[name], T=64)
+    x = mokgen.tokens(cfg)
+    w = mokgen.router_weight(cfg)
+    prior = mokgen.zipf_log_prior(cfg.E, cfg.zipf_s) if cfg.zipf_s else None
+    exact = oracle.router_logits(x, w, prior)
+    host = mokgen.router_logits(cfg, x).double()
+    mag = x.double().abs() @ w.double().abs()
+    if prior is not None:
+        mag = mag + prior.double().abs()
+    n, u = cfg.H + 1, 2.0 ** -24
+    bound = n * u / (1 - n * u) * mag
+    assert ((host - exact).abs() <= bound).all()
