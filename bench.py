@@ -1,7 +1,7 @@
 """Benchmark of the forward MoE layer (Mixture-of-Kittens hot path) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mok|reference]
-                    [--config page] [--mode staged|persistent] [--minibatch 2560]
+                    [--config page] [--mode staged|persistent] [--minibatch 0]
 
 One step = one pass of the whole hot path over one batch of synthetic
 tokens already resident in HBM: mok_plan (router top-k, gates, histogram,
@@ -14,16 +14,21 @@ is the page shape: T = 8192 tokens, hidden 7168, expert intermediate 2048,
 Metric: tokens/s of the forward layer (whole job: sum over ranks).  With N
 GPUs each rank runs an independent replica of the workload (the layer on
 one GPU does not shard; no collective is on the data path) and the time is
-the max over ranks.  Rank 0 prints one JSON line.
+the max over ranks.  Rank 0 prints one JSON line.  The default run also
+times, on the device, the persistent SM-partitioned kernel on the same
+workload and the zipf-routed shape (T 16384, E 256: the tensor-bound
+H7168/I2048 GEMM), as sub-records of the same line.
 
 --impl reference times the CPU oracle (test infrastructure, plain C with
-fp64 accumulation) on a bounded sample of the same workload.
+fp64 accumulation) on bounded samples of the same workload: each step is
+the oracle's FFN on one whole expert's rows plus that expert's share of the
+oracle plan.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
-import math
 import os
 import signal
 import statistics
@@ -39,6 +44,14 @@ sys.path.insert(0, ROOT)
 import mokgen  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal dense tensor-core peaks of one B200 (TFLOP/s), for context beside the measured ones
+NOMINAL_DENSE_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0}
+# a timed region shorter than this is a burst: the tensor peak it is compared
+# with is the measured burst figure; longer regions use the sustained one
+SUSTAINED_REGION_S = 1.0
+# kernel sources whose hash identifies the grouped GEMM a DRAM capture was taken of
+GEMM_SOURCES = ("gemm_core.cuh", "gemm_sm100.cu", "mok_device.cuh", "mxfp8.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
 def load_peaks():
@@ -48,6 +61,31 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(PEAKS_FALLBACK), "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "combine_device_top_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, mode: str):
+    """DRAM bytes (read + write) of the grouped GEMM's launches of one step
+    from a committed ncu capture of THIS kernel source (matched by hash) on
+    this workload and mode, or (None, reason)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture"
+    with open(TRAFFIC_FILE) as f:
+        entries = json.load(f).get("entries", [])
+    sha = gemm_source_hash()
+    for e in entries:
+        if e.get("workload") == workload and e.get("mode") == mode:
+            if e.get("gemm_source_sha") != sha:
+                return None, "the kernel changed since its capture"
+            return float(e["bytes_per_step"]), e.get("how", "")
+    return None, "no capture of this workload"
 
 
 # ------------------------------------------------------------------ clocks
@@ -136,19 +174,6 @@ class ClockSampler:
                 "samples": len(sm), "period_ms": self.PERIOD_MS}
 
 
-# ------------------------------------------------------------------ measured DRAM traffic
-# dram__bytes_read.sum + dram__bytes_write.sum of the two grouped-GEMM
-# launches of one step, from one ncu capture of a small case of the same
-# kernel, scaled to the full workload by the experts (and rows) processed;
-# the capture, its command and the scaling are in the profiles/ summary
-# named beside each entry.  None where no capture of the current kernel
-# exists for that workload.
-GEMM_TRAFFIC_GB_PER_STEP = {
-    "page": (35.6, "profiles/grouped_gemm_bf16_page_e37.md"),
-    "page_mxfp8": (18.9, "profiles/grouped_gemm_mxfp8_page_e32.md"),
-}
-
-
 # ------------------------------------------------------------------ ranks
 def max_over_ranks(value: float, device) -> float:
     """The largest of every rank's value (the job is as slow as its slowest
@@ -170,16 +195,17 @@ def job_rate(units_per_rank: float, ms: float, world: int) -> float:
 def algorithmic_work(cfg):
     """Algorithmic bytes / flops of one forward (one step)."""
     ns = cfg.slots
-    w_bytes = cfg.E * 3 * cfg.H * cfg.I * 2
-    gemm_bytes = w_bytes + ns * cfg.H * 2 + 2 * ns * cfg.I * 2 + ns * cfg.H * 2  # weights, rows in, h out+in, fp16 out
-    gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * 2
     if cfg.mxfp8:
-        # weights, token rows and h: E4M3 bytes plus one E8M0 scale per 32 values
-        mx = 1.0 + 1.0 / 32
-        w_bytes = cfg.E * 3 * cfg.H * cfg.I * mx
-        gemm_bytes = w_bytes + ns * cfg.H * mx + 2 * ns * cfg.I * mx + ns * cfg.H * 2
-        gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * mx
-    combine_bytes = ns * cfg.H * 2 + ns * 4 + cfg.T * cfg.H * 2
+        # weights, token rows and h: E4M3 bytes plus one E8M0 scale per 32
+        # values; slot outputs bf16
+        el, slot = 1.0 + 1.0 / 32, 2.0
+    else:
+        # bf16 weights, rows and h; slot outputs fp32
+        el, slot = 2.0, 4.0
+    w_bytes = cfg.E * 3 * cfg.H * cfg.I * el
+    gemm_bytes = w_bytes + ns * cfg.H * el + 2 * ns * cfg.I * el + ns * cfg.H * slot  # weights, rows, h out+in, slots
+    gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * el
+    combine_bytes = ns * cfg.H * slot + ns * 4 + cfg.T * cfg.H * 2
     return {
         "gemm_flops": 6.0 * cfg.H * cfg.I * ns,
         "gemm_bytes": float(gemm_bytes),
@@ -192,143 +218,264 @@ def algorithmic_work(cfg):
     }
 
 
-def run_mok(args, cfg, rank, world, device):
+class Workload:
+    """One configuration's inputs on the device (weights generated per expert
+    and uploaded; MXFP8 weights quantised once, untimed)."""
+
+    def __init__(self, cfg, device):
+        import combine_device_top_b200 as mok
+
+        self.cfg, self.device = cfg, device
+        self.x = mokgen.tokens(cfg)
+        self.logits = mokgen.router_logits(cfg, self.x)
+        self.dx, self.dlogits = self.x.to(device), self.logits.to(device)
+        wg, wu, wd = mokgen.upload_expert_weights(cfg, device)
+        self.pack = None
+        if cfg.mxfp8:
+            self.pack = (*mok.quantize_weights_mxfp8(wg), *mok.quantize_weights_mxfp8(wu),
+                         *mok.quantize_weights_mxfp8(wd))
+            del wg, wu, wd
+            self.w = None
+            torch.cuda.empty_cache()
+        else:
+            self.w = (wg, wu, wd)
+        self.x_shards = mok.shards(self.dx, cfg.R)
+        self.y = torch.empty_like(self.dx)
+        self.y_shards = mok.shards(self.y, cfg.R)
+        self.plan = mok.plan(self.dlogits, cfg.k, cfg.R)
+
+    def free(self):
+        self.w = self.pack = None
+        self.dx = self.dlogits = self.y = self.x_shards = self.y_shards = self.plan = None
+        torch.cuda.empty_cache()
+
+
+def _gpu_index():
+    if "CUDA_VISIBLE_DEVICES" in os.environ:
+        return int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])
+    return torch.cuda.current_device()
+
+
+def time_steps(wl: Workload, mode: str, steps: int, warmup: int, minibatch: int, dispatch_ctas: int = 0,
+               world: int = 1):
+    """Time `steps` steps after `warmup` untimed ones; staged mode goes through
+    the per-step ABI calls (the same kernels as mok_moe_forward's staged
+    mode) so that events on the launching stream time each phase."""
     import combine_device_top_b200 as mok
 
-    torch.cuda.set_device(device)
-    x = mokgen.tokens(cfg)
-    logits = mokgen.router_logits(cfg, x)
-    dx, dlogits = x.to(device), logits.to(device)
-    wg, wu, wd_bf16 = mokgen.upload_expert_weights(cfg, device)
-    pack = None
-    if cfg.mxfp8:
-        # one-time MXFP8 weight quantisation, untimed
-        pack = (*mok.quantize_weights_mxfp8(wg), *mok.quantize_weights_mxfp8(wu), *mok.quantize_weights_mxfp8(wd_bf16))
-        del wg, wu, wd_bf16
-        wg = wu = wd = None
-        torch.cuda.empty_cache()
-    else:
-        wd = mok.prepare_w_down(wd_bf16)      # one-time weight preparation, untimed
-        del wd_bf16
-    x_shards = mok.shards(dx, cfg.R)
-    y = torch.empty_like(dx)
-    y_shards = mok.shards(y, cfg.R)
-    mode = mok.MOK_MODE_STAGED if args.mode == "staged" else mok.MOK_MODE_PERSISTENT
-    opts = mok.fwd_opts(mode=mode, ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8, dispatch_ctas=args.dispatch_ctas)
-    minibatch = args.minibatch or cfg.minibatch
-    p = mok.plan(dlogits, cfg.k, cfg.R)
-    fws = torch.empty(mok.forward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
-                      dtype=torch.uint8, device=device)
-    # staged mode is timed one ABI step at a time (per-phase events)
-    staged = mode == mok.MOK_MODE_STAGED
+    cfg, device = wl.cfg, wl.device
+    staged = mode == "staged"
+    opts = mok.fwd_opts(mode=mok.MOK_MODE_STAGED if staged else mok.MOK_MODE_PERSISTENT,
+                        ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8, dispatch_ctas=dispatch_ctas)
+    p = wl.plan
+    bufs = {}
     if staged:
-        out = torch.empty((cfg.slots, cfg.H), dtype=torch.float16, device=device)
         if cfg.mxfp8:
-            rows_q = torch.empty((cfg.slots, cfg.H), dtype=torch.uint8, device=device)
-            planes = torch.zeros((cfg.H // 128, mok.lib().mok_mxfp8_scale_rows(cfg.slots), 4), dtype=torch.uint8,
-                                 device=device)
-            ffn_ws = torch.empty(mok.lib().mok_expert_ffn_mxfp8_workspace_bytes(cfg.slots, cfg.I, cfg.E),
-                                 dtype=torch.uint8, device=device)
+            bufs["out"] = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
+            bufs["rows_q"] = torch.empty((cfg.slots, cfg.H), dtype=torch.uint8, device=device)
+            bufs["planes"] = torch.zeros((cfg.H // 128, mok.lib().mok_mxfp8_scale_rows(cfg.slots), 4),
+                                         dtype=torch.uint8, device=device)
+            bufs["ffn_ws"] = torch.empty(mok.lib().mok_expert_ffn_mxfp8_workspace_bytes(cfg.slots, cfg.I, cfg.E),
+                                         dtype=torch.uint8, device=device)
         else:
-            rows = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
-            ffn_ws = torch.empty(mok.lib().mok_expert_ffn_workspace_bytes(cfg.slots, cfg.I, cfg.E),
-                                 dtype=torch.uint8, device=device)
+            bufs["out"] = torch.empty((cfg.slots, cfg.H), dtype=torch.float32, device=device)
+            bufs["rows"] = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
+            bufs["ffn_ws"] = torch.empty(mok.lib().mok_expert_ffn_workspace_bytes(cfg.slots, cfg.I, cfg.E),
+                                         dtype=torch.uint8, device=device)
+    else:
+        bufs["fws"] = torch.empty(mok.forward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
+                                  dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
-
-    # A step in staged mode goes through the ABI one step at a time so that
-    # each phase is bracketed by events; it runs the same kernels as
-    # mok_moe_forward's staged mode.
     n_ev = 5 if staged else 3
 
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        mok.plan(dlogits, cfg.k, cfg.R, ws=p.ws)
+        mok.plan(wl.dlogits, cfg.k, cfg.R, ws=p.ws)
         if evs:
             evs[1].record(stream)
         if staged:
-            if pack is not None:
-                mok.gather_mxfp8(x_shards, p, rows_q, planes)
+            if wl.pack is not None:
+                mok.gather_mxfp8(wl.x_shards, p, bufs["rows_q"], bufs["planes"])
             else:
-                mok.gather(x_shards, p, rows)
+                mok.gather(wl.x_shards, p, bufs["rows"])
             if evs:
                 evs[2].record(stream)
-            if pack is not None:
-                mok.expert_ffn_mxfp8(rows_q, planes, pack, p, out=out, ws=ffn_ws)
+            if wl.pack is not None:
+                mok.expert_ffn_mxfp8(bufs["rows_q"], bufs["planes"], wl.pack, p, out=bufs["out"], ws=bufs["ffn_ws"])
             else:
-                mok.expert_ffn(rows, wg, wu, wd, p, out=out, ws=ffn_ws)
+                mok.expert_ffn(bufs["rows"], *wl.w, p, out=bufs["out"], ws=bufs["ffn_ws"])
             if evs:
                 evs[3].record(stream)
-            mok.combine(out, p, y_shards)
-        elif pack is not None:
-            mok.moe_forward_mxfp8(x_shards, pack, p, y_shards=y_shards, ws=fws, minibatch=minibatch, opts=opts)
+            mok.combine(bufs["out"], p, wl.y_shards)
+        elif wl.pack is not None:
+            mok.moe_forward_mxfp8(wl.x_shards, wl.pack, p, y_shards=wl.y_shards, ws=bufs["fws"],
+                                  minibatch=minibatch, opts=opts)
         else:
-            mok.moe_forward(x_shards, wg, wu, wd, p, minibatch, opts, y_shards=y_shards, ws=fws)
+            mok.moe_forward(wl.x_shards, *wl.w, p, minibatch, opts, y_shards=wl.y_shards, ws=bufs["fws"])
         if evs:
             evs[n_ev - 1].record(stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     # correctness of the timed configuration is covered by tests; here only a sanity check
-    if not torch.isfinite(y.float()).all():
+    if not torch.isfinite(wl.y.float()).all():
         raise RuntimeError("non-finite output")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                      else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])) as clk:
+    with ClockSampler(_gpu_index()) as clk:
         clk.mark_start()
         start.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             step(evs[i])
         stop.record(stream)
         torch.cuda.synchronize()
         clk.mark_stop()
     if world > 1:
         torch.distributed.barrier()
-    total_ms = start.elapsed_time(stop)
-    phases = [[evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j in range(n_ev - 1)]
-    total_ms = max_over_ranks(total_ms, device)
-
-    res = {"total_ms": total_ms, "phases_ms": [sum(ph) / len(ph) for ph in phases], "clocks": clk.summary()}
-
-    # end to end from pinned host memory through mok_moe_forward_host
-    if rank == 0 or world > 1:
-        hx, hl = x.pin_memory(), logits.pin_memory()
-        hy = torch.empty_like(x).pin_memory()
-        wts = (pack, None, None) if pack is not None else (wg, wu, wd)
-        hws = torch.empty(mok.forward_host_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
-                          dtype=torch.uint8, device=device)
-        for _ in range(2):
-            mok.moe_forward_host(hx, hl, cfg.k, cfg.R, *wts, minibatch, opts, hws, hy)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_e2e = max(1, min(args.steps, 5))
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(n_e2e):
-            mok.moe_forward_host(hx, hl, cfg.k, cfg.R, *wts, minibatch, opts, hws, hy)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        res["e2e_ms"] = max_over_ranks(e0.elapsed_time(e1) / n_e2e, device)
-        res["h2d"] = cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4
-        res["d2h"] = cfg.T * cfg.H * 2
-        del hws
-    # plan: top-k, rank, scan, scatter; staged forward: chunk list, gather, gate/up, down, combine;
-    # persistent forward: chunk list, one persistent kernel
-    res["launches_per_step"] = (4 + 1 + 1 + 2 + 1) if mode == mok.MOK_MODE_STAGED else (4 + 2)
-    res["max_over_mean_load"] = (lambda c: c.max().item() / c.mean().item())(p.counts().float())
+    total_ms = max_over_ranks(start.elapsed_time(stop), device)
+    phases = [[evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)] for j in range(n_ev - 1)]
+    res = {"total_ms": total_ms, "phases_ms": [sum(ph) / len(ph) for ph in phases], "clocks": clk.summary(),
+           # plan: top-k, rank, scan, scatter; staged: gather, chunk list, gate/up, down, combine;
+           # persistent: chunk list, one persistent kernel
+           "launches_per_step": (4 + 1 + 1 + 2 + 1) if staged else (4 + 2),
+           "max_over_mean_load": (lambda c: c.max().item() / c.mean().item())(p.counts().float())}
+    if not staged:
+        row0, units = mok.minibatch_bounds(p, cfg.H, cfg.I, minibatch, opts,
+                                           w_gate=None if wl.pack is None else _mx_ptr(wl.pack))
+        res["minibatches"] = len(row0)
+        res["min_units_per_minibatch"] = min(units[:-1]) if len(units) > 1 else units[0]
+    del bufs
+    torch.cuda.empty_cache()
     return res
 
 
+def _mx_ptr(pack):
+    import ctypes
+
+    import combine_device_top_b200 as mok
+
+    qg, sg, qu, su, qd, sd = pack
+    _mx_ptr.keep = mok.MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(),
+                                 sd.data_ptr())
+    return ctypes.cast(ctypes.byref(_mx_ptr.keep), ctypes.c_void_p)
+
+
+def time_e2e(wl: Workload, mode: str, steps: int, minibatch: int, world: int):
+    """End to end from pinned host memory through mok_moe_forward_host: each
+    step uploads x and the logits and reads y back."""
+    import combine_device_top_b200 as mok
+
+    cfg, device = wl.cfg, wl.device
+    opts = mok.fwd_opts(mode=mok.MOK_MODE_STAGED if mode == "staged" else mok.MOK_MODE_PERSISTENT,
+                        ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8)
+    hx, hl = wl.x.pin_memory(), wl.logits.pin_memory()
+    hy = torch.empty_like(wl.x).pin_memory()
+    wts = (wl.pack, None, None) if wl.pack is not None else wl.w
+    hws = torch.empty(mok.forward_host_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, minibatch, opts),
+                      dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        mok.moe_forward_host(hx, hl, cfg.k, cfg.R, *wts, minibatch, opts, hws, hy)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(1, min(steps, 5))
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        mok.moe_forward_host(hx, hl, cfg.k, cfg.R, *wts, minibatch, opts, hws, hy)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del hws
+    torch.cuda.empty_cache()
+    return {"e2e_ms": max_over_ranks(e0.elapsed_time(e1) / n, device), "h2d": cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4,
+            "d2h": cfg.T * cfg.H * 2, "e2e_steps": n}
+
+
+# ------------------------------------------------------------------ roofline
+def tensor_peaks(peaks, mxfp8: bool, region_s: float):
+    """(peak TFLOP/s of the MMA's dtype for a region this long, its kind)."""
+    burst = region_s < SUSTAINED_REGION_S
+    bf16 = peaks["bf16_tflops"] if burst else peaks["bf16_tflops_sustained"]
+    # fp8 runs at twice the bf16 rate (nominal 4.5 / 2.25 PFLOP/s)
+    kind = ("burst" if burst else "sustained") + f" (timed region {region_s:.2f} s)"
+    return bf16 * (2.0 if mxfp8 else 1.0), bf16, kind
+
+
+def staged_roofline(cfg, res, peaks, peak_src, mode, steps):
+    work = algorithmic_work(cfg)
+    t_plan, t_gather, t_gemm, t_comb = res["phases_ms"]
+    gemm_s = t_gemm / 1e3
+    tflops = work["gemm_flops"] / gemm_s / 1e12
+    gbs = work["gemm_bytes"] / gemm_s / 1e9
+    region_s = res["total_ms"] / 1e3
+    tc_peak, bf16_peak, kind = tensor_peaks(peaks, cfg.mxfp8, region_s)
+    t_tc = work["gemm_flops"] / (tc_peak * 1e12)
+    t_hbm = work["gemm_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": tc_peak, "unit": "TFLOP/s", "frac": tflops / tc_peak}
+    traffic, how = measured_traffic(cfg.name, mode)
+    nominal = NOMINAL_DENSE_TFLOPS["fp8" if cfg.mxfp8 else "bf16"]
+    roof.update({
+        "traffic": traffic, "traffic_note": how if traffic else how,
+        "kernel": "k_grouped_gemm: the gate/up+SwiGLU and down launches of one step (figures per step)",
+        "launches_per_step": 2,
+        "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
+        "tensor_peak_kind": kind,
+        "tensor_frac_of_measured_bf16": tflops / bf16_peak,
+        "tensor_frac_of_dtype_peak": tflops / tc_peak,
+        "tensor_frac_of_nominal_dense": tflops / nominal,
+    })
+    rates = {"gather_GBps": work["gather_bytes"] / (t_gather / 1e3) / 1e9,
+             "combine_GBps": work["combine_bytes"] / (t_comb / 1e3) / 1e9,
+             "gather_frac_of_hbm": work["gather_bytes"] / (t_gather / 1e3) / 1e9 / peaks["hbm_gbs"],
+             "combine_frac_of_hbm": work["combine_bytes"] / (t_comb / 1e3) / 1e9 / peaks["hbm_gbs"],
+             "gemm_TFLOPs": tflops, "gemm_GBps": gbs, "plan_share": t_plan / (res["total_ms"] / steps)}
+    return roof, {"plan": t_plan, "gather": t_gather, "grouped_gemm": t_gemm, "combine": t_comb}, rates
+
+
+def persistent_roofline(cfg, res, peaks, peak_src, steps):
+    work = algorithmic_work(cfg)
+    t_plan, t_fwd = res["phases_ms"]
+    fwd_s = t_fwd / 1e3
+    gbs = work["forward_bytes"] / fwd_s / 1e9
+    tflops = work["gemm_flops"] / fwd_s / 1e12
+    tc_peak, bf16_peak, kind = tensor_peaks(peaks, cfg.mxfp8, res["total_ms"] / 1e3)
+    roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "traffic": measured_traffic(cfg.name, "persistent")[0],
+            "kernel": "k_moe_persistent (dispatch, grouped GEMM, combine in one launch; figures per step)",
+            "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
+            "tensor_peak_kind": kind, "tensor_frac_of_dtype_peak": tflops / tc_peak}
+    return roof, {"plan": t_plan, "forward": t_fwd}, {"forward_GBps": gbs, "forward_TFLOPs": tflops,
+                                                       "plan_share": t_plan / (res["total_ms"] / steps)}
+
+
+def sub_record(cfg, mode, res, peaks, peak_src, steps):
+    ms = res["total_ms"] / steps
+    rec = {"workload": f"{cfg.name}: {cfg.describe()}", "mode": mode, "tokens_per_s": cfg.T / (ms / 1e3),
+           "ms_per_step": ms, "steps": steps}
+    if mode == "staged":
+        roof, ph, rates = staged_roofline(cfg, res, peaks, peak_src, mode, steps)
+    else:
+        roof, ph, rates = persistent_roofline(cfg, res, peaks, peak_src, steps)
+        rec["minibatches"] = res["minibatches"]
+        rec["min_gate_up_units_per_minibatch"] = res["min_units_per_minibatch"]
+    rec.update({"roofline": roof, "phases_ms": ph, "phase_rates": rates, "clocks": res["clocks"],
+                "expert_load_max_over_mean": res["max_over_mean_load"]})
+    return rec
+
+
 # ------------------------------------------------------------------ CPU oracle
-def cpu_oracle_sample(cfg, budget_s: float = 12.0, threads: int = 0):
-    """Oracle expert FFN on whole experts of the workload, experts 0, 1, ...
-    until about budget_s seconds of CPU work, on `threads` host threads (0:
-    every core this process may use); returns tokens/s (= rows/s / k)."""
+def oracle_steps(cfg, steps: int, warmup: int, threads: int = 0):
+    """The oracle on bounded samples of the workload: step i runs the
+    oracle's SwiGLU FFN over every row of one whole expert (experts taken in
+    order, warm-up ones first) plus that expert's share of the full oracle
+    plan.  Returns the measured rate (tokens/s = rows/s / k) and what ran."""
     import oracle
 
     cores = threads if threads > 0 else len(os.sched_getaffinity(0))
@@ -340,24 +487,25 @@ def cpu_oracle_sample(cfg, budget_s: float = 12.0, threads: int = 0):
     t_plan = time.perf_counter() - t0
     rows_all = oracle.gather(x, cfg.R, pl["src_rank"], pl["src_index"])
     off = pl["offsets"]
-    spent, rows_done, experts = 0.0, 0, 0
-    for e in range(cfg.E):
+    experts = [e for e in range(cfg.E) if off[e + 1] > off[e]]
+    spent, rows_done, ran = 0.0, 0, []
+    for i in range(warmup + steps):
+        e = experts[i % len(experts)]
         a, b = int(off[e]), int(off[e + 1])
-        if b <= a:
-            continue
         wg, wu, wd = mokgen.expert_weights(cfg, e)
         t0 = time.perf_counter()
         oracle.expert_ffn(rows_all[a:b], wg, wu, wd)
-        spent += time.perf_counter() - t0
-        rows_done += b - a
-        experts += 1
-        if spent >= budget_s:
-            break
-    # plan time is charged in proportion to the sampled rows
-    t = spent + t_plan * rows_done / cfg.slots
-    return {"value": (rows_done / cfg.k) / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"oracle SwiGLU FFN of experts 0..{experts - 1} ({rows_done} of {cfg.slots} rows) of the "
-                      f"{cfg.name} workload plus its share of the full oracle plan; tokens/s = rows/s / k"}
+        dt = time.perf_counter() - t0 + t_plan * (b - a) / cfg.slots
+        if i >= warmup:
+            spent += dt
+            rows_done += b - a
+            ran.append(e)
+    return {"value": (rows_done / cfg.k) / spent, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "steps_run": steps, "warmup_run": warmup, "sampled_seconds": spent,
+            "sample_tokens_per_step": rows_done / cfg.k / steps, "extrapolated": True,
+            "sample": f"oracle SwiGLU FFN of whole experts {ran[0]}..{ran[-1]} ({rows_done} of {cfg.slots} rows "
+                      f"of the {cfg.name} workload, one expert per step) plus their share of the full oracle plan; "
+                      f"tokens/s = rows/s / k, extrapolated from the sample to the layer"}
 
 
 def main():
@@ -368,11 +516,14 @@ def main():
     ap.add_argument("--impl", default="mok", choices=["mok", "reference"])
     ap.add_argument("--config", default="page", choices=list(mokgen.CONFIGS))
     ap.add_argument("--mode", default="staged", choices=["staged", "persistent"])
-    ap.add_argument("--minibatch", type=int, default=0)
+    ap.add_argument("--minibatch", type=int, default=-1,
+                    help="persistent mode: least rows per minibatch (0: the two-wave rule alone; "
+                         "default: the configuration's)")
     ap.add_argument("--dispatch-ctas", type=int, default=0,
                     help="persistent mode: CTAs on the dispatch side (0: the library default, 16)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-sub-records", action="store_true", help="time only the main workload")
+    ap.add_argument("--cpu-steps", type=int, default=64, help="experts the CPU baseline samples")
     ap.add_argument("--scale-experts", type=int, default=0,
                     help="profiling case: E experts and T scaled by the same factor (same rows per expert)")
     args = ap.parse_args()
@@ -381,6 +532,7 @@ def main():
         n = args.scale_experts
         T = max(cfg.R, round(cfg.T * n / cfg.E / cfg.R) * cfg.R)
         cfg = mokgen.scaled(cfg, E=n, T=T)
+    minibatch = cfg.minibatch if args.minibatch < 0 else args.minibatch
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -391,21 +543,22 @@ def main():
     wdesc = ("MXFP8 E4M3 weights + E8M0 scales per 32 along K (quantised once, untimed)" if cfg.mxfp8
              else "bf16 weights [E,H,I]/[E,I,H]")
     config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
-              "tokens_per_step_per_gpu": cfg.T, "minibatch": args.minibatch or cfg.minibatch,
-              "mode": args.mode,
-              **({"dispatch_ctas": args.dispatch_ctas or 16} if args.mode == "persistent" else {}),
+              "tokens_per_step_per_gpu": cfg.T, "mode": args.mode,
+              **({"minibatch": minibatch, "dispatch_ctas": args.dispatch_ctas or 16}
+                 if args.mode == "persistent" else {}),
               "l2": f"inputs larger than L2 ({algorithmic_work(cfg)['weight_bytes'] / 1e9:.1f} GB of expert "
                     f"weights streamed per step)"}
 
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = cpu_oracle_sample(cfg, args.cpu_budget)
-        t_step_ms = cfg.T / cb["value"] * 1e3
+        cb = oracle_steps(cfg, args.steps, args.warmup)
         line = {"metric": metric, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step_ms, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
-                "impl": "reference", "cpu_baseline": dict(cb),
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["sampled_seconds"] / args.steps * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config, "impl": "reference", "extrapolated": True,
+                "sample_tokens_per_step": cb["sample_tokens_per_step"], "sampled_seconds": cb["sampled_seconds"],
+                "cpu_baseline": dict(cb),
                 "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
@@ -413,7 +566,23 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
     device = torch.device("cuda", local_rank)
-    res = run_mok(args, cfg, rank, world, device)
+    torch.cuda.set_device(device)
+    wl = Workload(cfg, device)
+    res = time_steps(wl, args.mode, args.steps, args.warmup, minibatch, args.dispatch_ctas, world)
+    e2e = time_e2e(wl, args.mode, args.steps, minibatch, world)
+    subs = {}
+    if not args.no_sub_records and not args.scale_experts and world == 1 and args.config == "page":
+        peaks, peak_src = load_peaks()
+        other = "persistent" if args.mode == "staged" else "staged"
+        r2 = time_steps(wl, other, args.steps, args.warmup, minibatch, args.dispatch_ctas)
+        subs[f"{cfg.name}_{other}"] = sub_record(cfg, other, r2, peaks, peak_src, args.steps)
+        wl.free()
+        del wl
+        zcfg = mokgen.CONFIGS["zipf"]
+        zl = Workload(zcfg, device)
+        rz = time_steps(zl, "staged", args.steps, args.warmup, zcfg.minibatch)
+        subs["zipf_staged"] = sub_record(zcfg, "staged", rz, peaks, peak_src, args.steps)
+        zl.free()
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -421,71 +590,32 @@ def main():
         return 0
 
     peaks, peak_src = load_peaks()
-    work = algorithmic_work(cfg)
     ms = res["total_ms"] / args.steps
     value = job_rate(cfg.T, ms, world)
-    ph = res["phases_ms"]
     line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "mxfp8-e4m3 (bf16 MMA)" if cfg.mxfp8 else "bf16",
+            "vs_baseline": None, "dtype": "mxfp8-e4m3" if cfg.mxfp8 else "bf16",
             "data": "synthetic", "config": config}
-    if len(ph) == 4:
-        t_plan, t_gather, t_gemm, t_comb = ph
-        gemm_s = t_gemm / 1e3
-        tflops = work["gemm_flops"] / gemm_s / 1e12
-        gbs = work["gemm_bytes"] / gemm_s / 1e9
-        # the MMA's own dtype peak: fp8 runs at twice the measured bf16 rate (nominal 4.5 / 2.25 PFLOP/s)
-        tc_peak = peaks["bf16_tflops_sustained"] * (2.0 if cfg.mxfp8 else 1.0)
-        t_tc = work["gemm_flops"] / (tc_peak * 1e12)
-        t_hbm = work["gemm_bytes"] / (peaks["hbm_gbs"] * 1e9)
-        if t_hbm >= t_tc:
-            roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": gbs / peaks["hbm_gbs"]}
-        else:
-            roof = {"bound": "tensor", "achieved": tflops, "peak": tc_peak,
-                    "unit": "TFLOP/s", "frac": tflops / tc_peak}
-        traffic = GEMM_TRAFFIC_GB_PER_STEP.get(cfg.name) if not args.scale_experts else None
-        if traffic and args.mode != "staged" and not cfg.mxfp8:
-            traffic = None
-        roof.update({"traffic": traffic[0] * 1e9 if traffic else None,
-                     "traffic_note": (f"bytes per step, both GEMM launches, scaled from {traffic[1]}" if traffic
-                                      else "no capture of this workload"),
-                     "kernel": "grouped GEMM (gate/up+SwiGLU and down launches)",
-                     "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
-                     "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"],
-                     "tensor_frac_of_dtype_peak": tflops / tc_peak})
-        line["roofline"] = roof
-        line["phases_ms"] = {"plan": t_plan, "gather": t_gather, "grouped_gemm": t_gemm, "combine": t_comb}
-        line["phase_rates"] = {
-            "gather_GBps": work["gather_bytes"] / (t_gather / 1e3) / 1e9,
-            "combine_GBps": work["combine_bytes"] / (t_comb / 1e3) / 1e9,
-            "gemm_TFLOPs": tflops, "gemm_GBps": gbs,
-            "plan_share": t_plan / ms,
-        }
+    if args.mode == "staged":
+        roof, ph, rates = staged_roofline(cfg, res, peaks, peak_src, "staged", args.steps)
     else:
-        # one mok_moe_forward call (gather, grouped GEMM and combine together) is the timed kernel work
-        t_plan, t_fwd = ph
-        fwd_s = t_fwd / 1e3
-        gbs = work["forward_bytes"] / fwd_s / 1e9
-        tflops = work["gemm_flops"] / fwd_s / 1e12
-        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / peaks["hbm_gbs"], "traffic": None,
-                "kernel": "persistent forward kernel (dispatch, grouped GEMM, combine in one launch)",
-                "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
-                "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"]}
-        line["roofline"] = roof
-        line["phases_ms"] = {"plan": t_plan, "forward": t_fwd}
-        line["phase_rates"] = {"forward_GBps": gbs, "forward_TFLOPs": tflops, "plan_share": t_plan / ms}
-    if "e2e_ms" in res:
-        line["e2e"] = {"value": job_rate(cfg.T, res["e2e_ms"], world), "unit": "tokens/s",
-                       "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]}
+        roof, ph, rates = persistent_roofline(cfg, res, peaks, peak_src, args.steps)
+        line["minibatches"] = res["minibatches"]
+        line["min_gate_up_units_per_minibatch"] = res["min_units_per_minibatch"]
+    line["roofline"] = roof
+    line["phases_ms"] = ph
+    line["phase_rates"] = rates
+    line["e2e"] = {"value": job_rate(cfg.T, e2e["e2e_ms"], world), "unit": "tokens/s",
+                   "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["e2e_steps"]}
     line["gpu_launches"] = res["launches_per_step"] * args.steps
     if res["clocks"]:
         line["clocks"] = res["clocks"]
     line["expert_load_max_over_mean"] = res["max_over_mean_load"]
+    if subs:
+        line["sub_records"] = subs
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_oracle_sample(cfg, args.cpu_budget)
-        line["cpu_baseline_1thread"] = cpu_oracle_sample(cfg, args.cpu_budget / 2, threads=1)
+        cb = oracle_steps(cfg, args.cpu_steps, 1)
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "extrapolated")}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -30,14 +30,17 @@ MOK_ERR_CAPACITY = 6
 MOK_MODE_PERSISTENT = 0
 MOK_MODE_STAGED = 1
 MOK_MAX_SHARDS = 64
+MOK_SLOTS_F32 = 0
+MOK_SLOTS_BF16 = 1
 
 # every entry point of include/mok.h
 EXPORTS = (
     "mok_plan_workspace_bytes", "mok_plan", "mok_forward_workspace_bytes", "mok_moe_forward",
     "mok_get_status", "mok_last_error_string", "mok_gather", "mok_expert_ffn_workspace_bytes",
     "mok_expert_ffn", "mok_combine", "mok_forward_host_workspace_bytes", "mok_moe_forward_host",
-    "mok_prepare_w_down", "mok_plan_noalloc", "mok_mxfp8_quantize_rows", "mok_quantize_weights_mxfp8",
+    "mok_plan_noalloc", "mok_mxfp8_quantize_rows", "mok_quantize_weights_mxfp8",
     "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8_workspace_bytes", "mok_expert_ffn_mxfp8",
+    "mok_two_wave_rows", "mok_minibatch_bounds",
 )
 
 
@@ -57,7 +60,7 @@ class PlanT(ctypes.Structure):
 
 class FwdOpts(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("dispatch_ctas", ctypes.c_int32),
-                ("gemm_ctas", ctypes.c_int32), ("mxfp8", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("gemm_ctas", ctypes.c_int32), ("mxfp8", ctypes.c_int32), ("min_waves", ctypes.c_int32),
                 ("timeout_ns", ctypes.c_uint64)]
 
 
@@ -81,12 +84,11 @@ def lib() -> ctypes.CDLL:
     L.mok_expert_ffn_workspace_bytes.argtypes = [i32, i32, i32]
     L.mok_expert_ffn_workspace_bytes.restype = sz
     L.mok_expert_ffn.argtypes = [vp, i32, i32, vp, vp, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
-    L.mok_combine.argtypes = [vp, i32, ctypes.POINTER(PlanT), vp, vp]
+    L.mok_combine.argtypes = [vp, i32, i32, ctypes.POINTER(PlanT), vp, vp]
     L.mok_forward_host_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(FwdOpts)]
     L.mok_forward_host_workspace_bytes.restype = sz
     L.mok_moe_forward_host.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32,
                                        ctypes.POINTER(FwdOpts), vp, sz, vp, vp]
-    L.mok_prepare_w_down.argtypes = [vp, vp, sz, vp]
     L.mok_plan_noalloc.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.mok_mxfp8_quantize_rows.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     L.mok_quantize_weights_mxfp8.argtypes = [vp, i32, i32, i32, vp, vp, vp]
@@ -95,9 +97,13 @@ def lib() -> ctypes.CDLL:
     L.mok_expert_ffn_mxfp8_workspace_bytes.argtypes = [i32, i32, i32]
     L.mok_expert_ffn_mxfp8_workspace_bytes.restype = sz
     L.mok_expert_ffn_mxfp8.argtypes = [vp, vp, i32, i32, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
+    L.mok_two_wave_rows.argtypes = [i32, i32, i32, i32]
+    L.mok_minibatch_bounds.argtypes = [ctypes.POINTER(PlanT), i32, i32, vp, i32, ctypes.POINTER(FwdOpts), vp, sz,
+                                       vp, vp, i32, ctypes.POINTER(ctypes.c_int), vp]
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
-              "mok_moe_forward_host", "mok_prepare_w_down", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
-              "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8"):
+              "mok_moe_forward_host", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
+              "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8",
+              "mok_two_wave_rows", "mok_minibatch_bounds"):
         getattr(L, n).restype = ctypes.c_int
     return L
 
@@ -178,16 +184,6 @@ def plan(logits: torch.Tensor, top_k: int, R: int, ws: torch.Tensor | None = Non
     return Plan(p, ws)
 
 
-def prepare_w_down(w_down: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """One-time fp16 copy of a bf16 W_down [E, I, H] (``mok_prepare_w_down``)."""
-    assert w_down.is_cuda and w_down.dtype == torch.bfloat16 and w_down.is_contiguous()
-    if out is None:
-        out = torch.empty(w_down.shape, dtype=torch.float16, device=w_down.device)
-    _check(lib().mok_prepare_w_down(ctypes.c_void_p(w_down.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-                                    w_down.numel(), _stream(stream)))
-    return out
-
-
 def mxfp8_quantize_rows(src: torch.Tensor, stream=None):
     """Blocks of 32 along each row of a [rows, K] bf16/fp32 tensor -> (q uint8, scales uint8)."""
     assert src.is_cuda and src.is_contiguous() and src.dtype in (torch.bfloat16, torch.float32)
@@ -212,8 +208,8 @@ def quantize_weights_mxfp8(w: torch.Tensor, stream=None):
 
 
 def fwd_opts(mode: int = MOK_MODE_PERSISTENT, ring_slots: int = 0, dispatch_ctas: int = 0, gemm_ctas: int = 0,
-             mxfp8: bool = False, timeout_ns: int = 0) -> FwdOpts:
-    return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), 0, timeout_ns)
+             mxfp8: bool = False, timeout_ns: int = 0, min_waves: int = 0) -> FwdOpts:
+    return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), min_waves, timeout_ns)
 
 
 def forward_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None = None) -> int:
@@ -231,6 +227,8 @@ def moe_forward(x_shards, w_gate, w_up, w_down, p: Plan, minibatch: int = 2560, 
     R = p.c.R
     # the library reads R pointers from each shard array
     assert len(x_shards) == R and (y_shards is None or len(y_shards) == R)
+    for w in (w_gate, w_up, w_down):
+        assert w.dtype == torch.bfloat16, "the weights are bf16"
     H = x_shards[0].shape[1]
     I = w_gate.shape[-1]
     dev = x_shards[0].device
@@ -284,6 +282,27 @@ def moe_forward_mxfp8(x_shards, pack, p: Plan, y_shards=None, ws: torch.Tensor |
     return y_shards, ws
 
 
+def two_wave_rows(I: int, gemm_ctas: int, tile_rows: int, tile_features: int) -> int:
+    """``mok_two_wave_rows``: rows of two full waves of gate/up output tiles."""
+    return lib().mok_two_wave_rows(I, gemm_ctas, tile_rows, tile_features)
+
+
+def minibatch_bounds(p: Plan, H: int, I: int, minibatch: int, opts: FwdOpts, w_gate=None, ws=None, stream=None):
+    """``mok_minibatch_bounds``: (first row of each minibatch, gate/up units of
+    each) that mok_moe_forward uses for these arguments."""
+    dev = p.ws.device
+    if ws is None:
+        ws = _workspace(forward_workspace_bytes(p.c.T, H, I, p.c.E, p.c.k, minibatch, opts), dev)
+    cap = p.ns + 2
+    row0 = (ctypes.c_int32 * cap)()
+    units = (ctypes.c_int32 * cap)()
+    n = ctypes.c_int(0)
+    _check(lib().mok_minibatch_bounds(ctypes.byref(p.c), H, I, w_gate, minibatch, ctypes.byref(opts),
+                                      ctypes.c_void_p(ws.data_ptr()), ws.numel(), row0, units, cap, ctypes.byref(n),
+                                      _stream(stream)))
+    return list(row0[:n.value]), list(units[:n.value])
+
+
 def get_status(ws: torch.Tensor, stream=None) -> int:
     code = ctypes.c_int(-1)
     _check(lib().mok_get_status(ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream), ctypes.byref(code)))
@@ -320,13 +339,13 @@ def gather_mxfp8(x_shards, p: Plan, rows_q=None, scales=None, stream=None):
 
 def expert_ffn_mxfp8(rows_q, scales, pack, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
     """The MXFP8 grouped SwiGLU FFN over mok_gather_mxfp8's output; pack =
-    (qg, sg, qu, su, qd, sd).  Returns (out [T*k, H] fp16 slot-indexed, ws)."""
+    (qg, sg, qu, su, qd, sd).  Returns (out [T*k, H] bf16 slot-indexed, ws)."""
     qg, sg, qu, su, qd, sd = pack
     H = rows_q.shape[1]
     I = qg.shape[-1]
     if out is None:
-        out = torch.empty((p.ns, H), dtype=torch.float16, device=rows_q.device)
-    assert out.dtype == torch.float16
+        out = torch.empty((p.ns, H), dtype=torch.bfloat16, device=rows_q.device)
+    assert out.dtype == torch.bfloat16
     if ws is None:
         ws = _workspace(lib().mok_expert_ffn_mxfp8_workspace_bytes(p.ns, I, p.c.E), rows_q.device)
     w = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
@@ -338,12 +357,14 @@ def expert_ffn_mxfp8(rows_q, scales, pack, p: Plan, out: torch.Tensor | None = N
 
 
 def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
-    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] fp16 slot-indexed, ws)."""
+    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] fp32 slot-indexed, ws)."""
     H = rows.shape[1]
     I = w_gate.shape[-1]
+    for w in (w_gate, w_up, w_down):
+        assert w.dtype == torch.bfloat16, "the weights are bf16"
     if out is None:
-        out = torch.empty((p.ns, H), dtype=torch.float16, device=rows.device)
-    assert out.dtype == torch.float16
+        out = torch.empty((p.ns, H), dtype=torch.float32, device=rows.device)
+    assert out.dtype == torch.float32
     if ws is None:
         ws = _workspace(lib().mok_expert_ffn_workspace_bytes(p.ns, I, p.c.E), rows.device)
     _check(lib().mok_expert_ffn(ctypes.c_void_p(rows.data_ptr()), H, I, ctypes.c_void_p(w_gate.data_ptr()),
@@ -354,10 +375,12 @@ def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = N
 
 
 def combine(out: torch.Tensor, p: Plan, y_shards, stream=None):
-    """y = fixed-order gate-weighted sum of the fp16 per-slot outputs (fp32 accumulation)."""
-    assert out.dtype == torch.float16 and len(y_shards) == p.c.R
+    """y = fixed-order gate-weighted sum of the per-slot outputs (fp32, or bf16 on the MXFP8 path;
+    fp32 accumulation)."""
+    assert out.dtype in (torch.float32, torch.bfloat16) and len(y_shards) == p.c.R
     H = out.shape[-1]
-    _check(lib().mok_combine(ctypes.c_void_p(out.data_ptr()), H, ctypes.byref(p.c), _ptr_array(y_shards),
+    dt = MOK_SLOTS_F32 if out.dtype == torch.float32 else MOK_SLOTS_BF16
+    _check(lib().mok_combine(ctypes.c_void_p(out.data_ptr()), dt, H, ctypes.byref(p.c), _ptr_array(y_shards),
                              _stream(stream)))
     return y_shards
 

@@ -67,8 +67,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
-                        uint32_t box_inner, uint32_t box_outer, const char** err) {
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer, const char** err) {
     auto enc = get_encode();
     if (!enc) {
         *err = "cuTensorMapEncodeTiled unavailable";
@@ -78,8 +78,7 @@ bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t 
     cuuint64_t strides[1] = {inner * 2};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                     const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -89,9 +88,9 @@ bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t 
     return true;
 }
 
-bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint64_t rows, const char** err) {
+bool encode_bmaps(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err) {
     for (int i = 0; i < B_MAPS; ++i)
-        if (!encode_tmap_2d_16b(&maps->m[i], bf16, base, inner, rows, 64, (uint32_t)(16 * (i + 1)), err))
+        if (!encode_tmap_2d_bf16(&maps->m[i], base, inner, rows, 64, (uint32_t)(16 * (i + 1)), err))
             return false;
     return true;
 }
@@ -106,7 +105,7 @@ static bool encode_wd3(CUtensorMap* map, const void* wd, int H, int I, int E) {
     cuuint64_t strides[2] = {(cuuint64_t)H * 2, 128};
     cuuint32_t box[3] = {64, 64, 2};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(wd), dims, strides, box, estr,
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(wd), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -114,11 +113,11 @@ static bool encode_wd3(CUtensorMap* map, const void* wd, int H, int I, int E) {
 bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
                       int H, int I, int E, int buf_rows, const char** err) {
     m->has_wd3 = encode_wd3(&m->wd3, wd, H, I, E) ? 1 : 0;
-    return encode_tmap_2d_16b(&m->wg, true, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
-           encode_tmap_2d_16b(&m->wu, true, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
-           encode_tmap_2d_16b(&m->wd, false, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, err) &&
-           encode_bmaps(&m->rows, true, rows, (uint64_t)H, (uint64_t)buf_rows, err) &&
-           encode_bmaps(&m->h, false, h, (uint64_t)I, (uint64_t)buf_rows, err);
+    return encode_tmap_2d_bf16(&m->wg, wg, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
+           encode_tmap_2d_bf16(&m->wu, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
+           encode_tmap_2d_bf16(&m->wd, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, err) &&
+           encode_bmaps(&m->rows, rows, (uint64_t)H, (uint64_t)buf_rows, err) &&
+           encode_bmaps(&m->h, h, (uint64_t)I, (uint64_t)buf_rows, err);
 }
 
 // 2D map of a row-major [outer, inner] byte array.
@@ -179,7 +178,8 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
         l.cap = l.minibatch;
         l.buf_rows = (int)ns;
     } else {
-        l.minibatch = minibatch;
+        // 0: the two-wave rule alone; at least 16 rows either way
+        l.minibatch = minibatch > 16 ? minibatch : 16;
         const int ring = (o && o->ring_slots > 0) ? o->ring_slots : 2 * (minibatch > 4096 ? minibatch : 4096);
         l.cap = ring / 2;
         l.buf_rows = ring;
@@ -210,7 +210,7 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
         l.rows = take((size_t)l.buf_rows * H * 2);
         l.h = take((size_t)l.buf_rows * I * 2);
     }
-    l.out = take((size_t)ns * H * 2);  // fp16 slot outputs
+    l.out = take((size_t)ns * H * (l.mx ? 2 : 4));  // slot outputs: fp32, or bf16 on the MXFP8 path
     l.total = off;
     *L = l;
     return true;
@@ -228,6 +228,11 @@ static int check_plan(const mok_plan_t* p) {
     if (p->T < 0 || p->E <= 0 || p->k <= 0 || p->k > p->E || p->R <= 0 || p->R > MOK_MAX_SHARDS ||
         (p->T > 0 && p->T % p->R))
         return fail(MOK_ERR_INVALID_ARG, "plan holds an invalid shape");
+    // a hand-filled plan (e.g. from mok_plan_noalloc's outputs) gets the same
+    // limits as mok_plan: the work list and the combine are built for them
+    if (p->E > MOK_MAX_EXPERTS) return fail(MOK_ERR_UNSUPPORTED, "plan E > %d", MOK_MAX_EXPERTS);
+    if (p->k > MOK_MAX_TOPK) return fail(MOK_ERR_UNSUPPORTED, "plan k > %d", MOK_MAX_TOPK);
+    if ((int64_t)p->T * p->k > 0x3fffffff) return fail(MOK_ERR_UNSUPPORTED, "plan T * k too large");
     if (!p->counts || !p->offsets || !p->sched_src_rank || !p->sched_src_index || !p->row_slot || !p->pos ||
         !p->topk_idx || !p->gates)
         return fail(MOK_ERR_INVALID_ARG, "plan has NULL views (was mok_plan called?)");
@@ -341,6 +346,118 @@ size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int miniba
     return L.total;
 }
 
+}  // extern "C"
+
+namespace mok {
+
+// Everything mok_moe_forward decides before its kernels: validated shape,
+// workspace layout, SM split and the device-built work list (minibatches
+// and chunks) in the workspace.
+struct FwdSetup {
+    FwdLayout L;
+    int sms, dispatch, gemm, upc, min_units;
+    bool pair;
+    uint64_t timeout;
+    const mok_mxfp8_weights* mxw;
+    DevStatus* status;
+    int* counts2;
+    Chunk* chunks;
+    Minibatch* mbs;
+};
+
+static int setup_forward(int H, int I, const void* w_gate, const mok_plan_t* plan, int minibatch,
+                         const mok_fwd_opts* opts, void* ws, size_t ws_bytes, cudaStream_t stream, FwdSetup* F) {
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if ((rc = check_hi(H, I))) return rc;
+    const int mode = opts ? opts->mode : MOK_MODE_PERSISTENT;
+    if (mode != MOK_MODE_STAGED && mode != MOK_MODE_PERSISTENT)
+        return fail(MOK_ERR_INVALID_ARG, "unknown mode %d", mode);
+    F->mxw = nullptr;
+    if (opts && opts->mxfp8) {
+        F->mxw = static_cast<const mok_mxfp8_weights*>(w_gate);
+        const mok_mxfp8_weights* m = F->mxw;
+        if (!m || !m->gate || !m->gate_scales || !m->up || !m->up_scales || !m->down || !m->down_scales)
+            return fail(MOK_ERR_INVALID_ARG, "MXFP8 weight pack with NULL members");
+    }
+    if (mode == MOK_MODE_PERSISTENT && minibatch != 0 && minibatch < 16)
+        return fail(MOK_ERR_INVALID_ARG, "minibatch must be 0 (two-wave rule) or >= 16");
+    if (minibatch < 0) return fail(MOK_ERR_INVALID_ARG, "minibatch < 0");
+    const int T = plan->T, E = plan->E, k = plan->k;
+    if (!fwd_layout(T, H, I, E, k, minibatch, opts, &F->L)) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
+    if (mode == MOK_MODE_PERSISTENT && F->L.cap < F->L.minibatch)
+        return fail(MOK_ERR_INVALID_ARG, "ring_slots / 2 < minibatch");
+    if ((rc = check_ws(ws, ws_bytes, F->L.total))) return rc;
+    F->sms = device_sms(nullptr);
+    if (F->sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    F->dispatch = 0;
+    F->gemm = F->sms;
+    if (mode == MOK_MODE_PERSISTENT) {
+        F->dispatch = (opts && opts->dispatch_ctas > 0) ? opts->dispatch_ctas : 16;
+        F->gemm = (opts && opts->gemm_ctas > 0) ? opts->gemm_ctas : F->sms - F->dispatch;
+        if (F->dispatch >= F->sms || F->gemm < 1 || F->dispatch + F->gemm > F->sms)
+            return fail(MOK_ERR_INVALID_ARG, "dispatch_ctas + gemm_ctas must be at most the %d SMs", F->sms);
+    }
+    // gate/up units per chunk: M tiles of 64 gate + 64 up features, in
+    // pairs where the pairing rule holds (bf16 path)
+    const int ns = T * k;
+    F->pair = !F->mxw && gemm_tuning(ns, E).pair != 0;
+    const int sub = F->pair ? 2 : 1;
+    F->upc = (I / 64 + sub - 1) / sub;
+    // minibatches of at least `waves` full waves of gate/up units (the
+    // pages' rule: two), persistent mode only
+    const int waves = (opts && opts->min_waves != 0) ? opts->min_waves : 2;
+    F->min_units = (mode == MOK_MODE_PERSISTENT && waves > 0) ? waves * F->gemm : 0;
+    F->timeout = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    F->status = reinterpret_cast<DevStatus*>(base + F->L.status);
+    F->counts2 = reinterpret_cast<int*>(base + F->L.counts2);
+    F->chunks = reinterpret_cast<Chunk*>(base + F->L.chunks);
+    F->mbs = reinterpret_cast<Minibatch*>(base + F->L.mbs);
+    if (T == 0) return MOK_OK;
+    MOK_CUDA(cudaMemsetAsync(F->status, 0, sizeof(DevStatus), stream), "status reset");
+    MOK_CUDA(launch_build_chunks(plan->offsets, E, ns, F->L.minibatch, F->L.cap,
+                                 F->mxw ? CHUNK_MAX_ROWS_MX : CHUNK_MAX_ROWS, F->min_units, F->upc, F->chunks,
+                                 F->L.max_chunks, F->mbs, F->L.max_mb, F->counts2, F->status, stream),
+             "work list launch");
+    return MOK_OK;
+}
+
+}  // namespace mok
+
+extern "C" {
+
+int mok_two_wave_rows(int I, int gemm_ctas, int tile_rows, int tile_features) {
+    return two_wave_rows(I, gemm_ctas, 2, tile_rows, tile_features);
+}
+
+int mok_minibatch_bounds(const mok_plan_t* plan, int H, int I, const void* w_gate, int minibatch,
+                         const mok_fwd_opts* opts, void* ws, size_t ws_bytes, int32_t* row0, int32_t* units,
+                         int max_mb, int* n_mb, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!row0 || !n_mb || max_mb < 1) return fail(MOK_ERR_INVALID_ARG, "row0, n_mb, max_mb");
+    FwdSetup F;
+    int rc = setup_forward(H, I, w_gate, plan, minibatch, opts, ws, ws_bytes, stream, &F);
+    if (rc) return rc;
+    *n_mb = 0;
+    if (plan->T == 0) return MOK_OK;
+    MOK_CUDA(cudaStreamSynchronize(stream), "stream synchronize");
+    int c2[2];
+    MOK_CUDA(cudaMemcpy(c2, F.counts2, sizeof c2, cudaMemcpyDeviceToHost), "work list read");
+    DevStatus st;
+    MOK_CUDA(cudaMemcpy(&st, F.status, sizeof st, cudaMemcpyDeviceToHost), "status read");
+    if (st.code != MOK_OK) return fail(st.code, "work list: device status %d", st.code);
+    const int n = c2[1] < max_mb ? c2[1] : max_mb;
+    for (int b = 0; b < n; ++b) {
+        Minibatch m;
+        MOK_CUDA(cudaMemcpy(&m, F.mbs + b, sizeof m, cudaMemcpyDeviceToHost), "work list read");
+        row0[b] = m.row0;
+        if (units) units[b] = (m.chunk1 - m.chunk0) * F.upc;
+    }
+    *n_mb = c2[1];
+    return MOK_OK;
+}
+
 int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gate, const void* w_up,
                     const void* w_down, const mok_plan_t* plan, int minibatch, const mok_fwd_opts* opts, void* ws,
                     size_t ws_bytes, void* const* y_shards, mok_stream_t stream_) {
@@ -348,38 +465,25 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     int rc = check_plan(plan);
     if (rc) return rc;
     if ((rc = check_hi(H, I))) return rc;
-    const int mode = opts ? opts->mode : MOK_MODE_PERSISTENT;
-    if (mode != MOK_MODE_STAGED && mode != MOK_MODE_PERSISTENT)
-        return fail(MOK_ERR_INVALID_ARG, "unknown mode %d", mode);
-    if (opts && opts->reserved != 0) return fail(MOK_ERR_INVALID_ARG, "opts.reserved must be 0");
-    const mok_mxfp8_weights* mxw = nullptr;
-    if (opts && opts->mxfp8) {
-        mxw = static_cast<const mok_mxfp8_weights*>(w_gate);
-        if (!mxw || !mxw->gate || !mxw->gate_scales || !mxw->up || !mxw->up_scales || !mxw->down ||
-            !mxw->down_scales)
-            return fail(MOK_ERR_INVALID_ARG, "MXFP8 weight pack with NULL members");
-        w_up = w_down = mxw->gate;  // not read on this path
+    if (opts && opts->mode != MOK_MODE_STAGED && opts->mode != MOK_MODE_PERSISTENT)
+        return fail(MOK_ERR_INVALID_ARG, "unknown mode %d", opts->mode);
+    if (plan->T > 0) {
+        if (!all_nonnull(x_shards, plan->R) || !all_nonnull(y_shards, plan->R))
+            return fail(MOK_ERR_INVALID_ARG, "NULL shard pointer");
+        if (!all_aligned16(x_shards, plan->R) || !all_aligned16(y_shards, plan->R))
+            return fail(MOK_ERR_UNSUPPORTED, "shard pointers must be 16-byte aligned");
     }
-    if (mode == MOK_MODE_PERSISTENT && minibatch < 16) return fail(MOK_ERR_INVALID_ARG, "minibatch < 16");
+    const bool mx = opts && opts->mxfp8;
+    if (!mx && (!w_gate || !w_up || !w_down)) return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
+    FwdSetup F;
+    rc = setup_forward(H, I, w_gate, plan, minibatch, opts, ws, ws_bytes, stream, &F);
+    if (rc) return rc;
     const int T = plan->T, E = plan->E, k = plan->k, R = plan->R;
     if (T == 0) return MOK_OK;
-    if (!all_nonnull(x_shards, R) || !all_nonnull(y_shards, R)) return fail(MOK_ERR_INVALID_ARG, "NULL shard pointer");
-    if (!all_aligned16(x_shards, R) || !all_aligned16(y_shards, R))
-        return fail(MOK_ERR_UNSUPPORTED, "shard pointers must be 16-byte aligned");
-    if (!w_gate || !w_up || !w_down) return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
-    FwdLayout L;
-    if (!fwd_layout(T, H, I, E, k, minibatch, opts, &L)) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
-    if (mode == MOK_MODE_PERSISTENT && L.cap < minibatch)
-        return fail(MOK_ERR_INVALID_ARG, "ring_slots / 2 < minibatch");
-    if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
-    const int sms = device_sms(nullptr);
-    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
-    const uint64_t timeout = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
+    const mok_mxfp8_weights* mxw = F.mxw;
+    const FwdLayout& L = F.L;
+    const int sms = F.sms;
     unsigned char* base = static_cast<unsigned char*>(ws);
-    DevStatus* status = reinterpret_cast<DevStatus*>(base + L.status);
-    int* counts2 = reinterpret_cast<int*>(base + L.counts2);
-    Chunk* chunks = reinterpret_cast<Chunk*>(base + L.chunks);
-    Minibatch* mbs = reinterpret_cast<Minibatch*>(base + L.mbs);
     ShardsIn xs{};
     ShardsOut ys{};
     for (int r = 0; r < R; ++r) {
@@ -387,24 +491,17 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         ys.p[r] = y_shards[r];
     }
     const int ns = T * k;
-    MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
-    MOK_CUDA(launch_build_chunks(plan->offsets, E, ns, L.minibatch, L.cap, mxw ? CHUNK_MAX_ROWS_MX : CHUNK_MAX_ROWS,
-                                 chunks, L.max_chunks, mbs, L.max_mb, counts2, status, stream),
-             "work list launch");
-    if (mode == MOK_MODE_PERSISTENT) {
+    if (L.mode == MOK_MODE_PERSISTENT) {
         int dev = 0;
         device_sms(&dev);
-        const int dispatch = (opts && opts->dispatch_ctas > 0) ? opts->dispatch_ctas : 16;
-        const int gemm = (opts && opts->gemm_ctas > 0) ? opts->gemm_ctas : sms - dispatch;
-        if (dispatch >= sms || gemm < 1 || dispatch + gemm > sms)
-            return fail(MOK_ERR_INVALID_ARG, "dispatch_ctas + gemm_ctas must be at most the %d SMs", sms);
         int* counters = reinterpret_cast<int*>(base + L.counters);
         MOK_CUDA(cudaMemsetAsync(counters, 0, sizeof(int) * (2 * (size_t)L.max_mb + (size_t)L.max_chunks + 8),
                                  stream),
                  "counter reset");
         PersistLaunch P{};
-        P.grid = dispatch + gemm;
-        P.dispatch_ctas = dispatch;
+        P.grid = F.dispatch + F.gemm;
+        P.dispatch_ctas = F.dispatch;
+        P.pair = F.pair;
         P.cap = L.cap;
         P.H = H;
         P.I = I;
@@ -423,10 +520,10 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         }
         P.ring = base + L.rows;
         P.h = base + L.h;
-        P.out = reinterpret_cast<__half*>(base + L.out);
-        P.chunks = chunks;
-        P.mbs = mbs;
-        P.counts2 = counts2;
+        P.out = base + L.out;
+        P.chunks = F.chunks;
+        P.mbs = F.mbs;
+        P.counts2 = F.counts2;
         P.gathered = counters;
         P.d_done = counters + L.max_mb;
         P.g_done = counters + 2 * L.max_mb;
@@ -437,8 +534,8 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         P.src_index = plan->sched_src_index;
         P.row_slot = plan->row_slot;
         P.gates = plan->gates;
-        P.status = status;
-        P.timeout_ns = timeout;
+        P.status = F.status;
+        P.timeout_ns = F.timeout;
         MOK_CUDA(gemm_configure(dev), "gemm configure");
         const char* err = "";
         cudaError_t e = launch_forward_persistent(P, &err, stream);
@@ -456,25 +553,11 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     } else {
         MOK_CUDA(launch_gather(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
     }
-    rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, chunks, counts2,
-                        base + L.h, base + L.out, status, timeout, stream, mxw, mxw ? &mxs : nullptr);
+    rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, F.chunks, F.counts2,
+                        base + L.h, base + L.out, F.status, F.timeout, stream, mxw, mxw ? &mxs : nullptr);
     if (rc) return rc;
-    MOK_CUDA(launch_combine(base + L.out, plan->gates, T, k, H, T / R, ys, sms, stream), "combine launch");
-    return MOK_OK;
-}
-
-int mok_prepare_w_down(const void* w_down_bf16, void* w_down_fp16, size_t count, mok_stream_t stream) {
-    if (count == 0) return MOK_OK;
-    if (!w_down_bf16 || !w_down_fp16) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
-    if ((reinterpret_cast<uintptr_t>(w_down_bf16) | reinterpret_cast<uintptr_t>(w_down_fp16)) & 15u)
-        return fail(MOK_ERR_UNSUPPORTED, "weight buffers must be 16-byte aligned");
-    const char* a = static_cast<const char*>(w_down_bf16);
-    const char* b = static_cast<const char*>(w_down_fp16);
-    if (a < b + count * 2 && b < a + count * 2) return fail(MOK_ERR_INVALID_ARG, "source and destination overlap");
-    const int sms = device_sms(nullptr);
-    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
-    MOK_CUDA(launch_bf16_to_fp16(w_down_bf16, w_down_fp16, count, sms, reinterpret_cast<cudaStream_t>(stream)),
-             "weight conversion launch");
+    MOK_CUDA(launch_combine(base + L.out, mxw != nullptr, plan->gates, T, k, H, T / R, ys, sms, stream),
+             "combine launch");
     return MOK_OK;
 }
 
@@ -589,8 +672,8 @@ int mok_expert_ffn(const void* rows, int H, int I, const void* w_gate, const voi
     off += align256(sizeof(Minibatch) * (size_t)mb);
     void* h = base + off;
     MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
-    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, CHUNK_MAX_ROWS, chunks, mc, mbs, mb, counts2,
-                                 status, stream),
+    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, CHUNK_MAX_ROWS, 0, 1, chunks, mc, mbs, mb,
+                                 counts2, status, stream),
              "work list launch");
     return run_expert_ffn(rows, ns, H, I, w_gate, w_up, w_down, plan->E, plan->row_slot, chunks, counts2, h, out,
                           status, kDefaultTimeoutNs, stream);
@@ -637,16 +720,19 @@ int mok_expert_ffn_mxfp8(const void* rows_q, const void* scales, int H, int I, c
     mxs.hsc = base + off;
     mxs.sc_rows = mx_sc_rows(ns);
     MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
-    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, CHUNK_MAX_ROWS_MX, chunks, mc, mbs, mb, counts2,
-                                 status, stream),
+    MOK_CUDA(launch_build_chunks(plan->offsets, plan->E, ns, ns, ns, CHUNK_MAX_ROWS_MX, 0, 1, chunks, mc, mbs, mb,
+                                 counts2, status, stream),
              "work list launch");
     return run_expert_ffn(rows_q, ns, H, I, nullptr, nullptr, nullptr, plan->E, plan->row_slot, chunks, counts2, h,
                           out, status, kDefaultTimeoutNs, stream, w, &mxs);
 }
 
-int mok_combine(const void* out, int H, const mok_plan_t* plan, void* const* y_shards, mok_stream_t stream) {
+int mok_combine(const void* out, int out_dtype, int H, const mok_plan_t* plan, void* const* y_shards,
+                mok_stream_t stream) {
     int rc = check_plan(plan);
     if (rc) return rc;
+    if (out_dtype != MOK_SLOTS_F32 && out_dtype != MOK_SLOTS_BF16)
+        return fail(MOK_ERR_INVALID_ARG, "unknown slot dtype %d", out_dtype);
     if (H <= 0 || H % 8) return fail(MOK_ERR_UNSUPPORTED, "H %% 8 != 0");
     if (plan->T == 0) return MOK_OK;
     if (!out || !all_nonnull(y_shards, plan->R)) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
@@ -656,8 +742,8 @@ int mok_combine(const void* out, int H, const mok_plan_t* plan, void* const* y_s
     for (int r = 0; r < plan->R; ++r) ys.p[r] = y_shards[r];
     const int sms = device_sms(nullptr);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
-    MOK_CUDA(launch_combine(out, plan->gates, plan->T, plan->k, H, plan->T / plan->R, ys, sms,
-                            reinterpret_cast<cudaStream_t>(stream)),
+    MOK_CUDA(launch_combine(out, out_dtype == MOK_SLOTS_BF16, plan->gates, plan->T, plan->k, H, plan->T / plan->R,
+                            ys, sms, reinterpret_cast<cudaStream_t>(stream)),
              "combine launch");
     return MOK_OK;
 }

@@ -5,8 +5,9 @@
 // Both kernels are HBM-bound streams of 16-byte vectors: one warp per token,
 // a grid of a few CTAs per SM looping over the tokens.  The gather reads each
 // token once and writes it to its k rows (T*H*2 bytes in, N_s*H*2 out); the
-// combine reads N_s*H*2 bytes of fp16 per-slot outputs and writes T*H*2
-// bytes of bf16 y, rounding once.
+// combine reads the per-slot outputs (N_s*H*4 bytes of fp32 on the bf16
+// path, N_s*H*2 of bf16 on the MXFP8 path) and writes T*H*2 bytes of bf16 y,
+// rounding once.
 #include "dispatch_combine.cuh"
 #include "mok_internal.h"
 #include "mxfp8.cuh"
@@ -97,8 +98,8 @@ cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, c
     return cudaGetLastError();
 }
 
-template <int KMAX>
-__global__ void __launch_bounds__(DC_THREADS) k_combine(const uint4* __restrict__ out, const float* __restrict__ gates,
+template <int KMAX, class S>
+__global__ void __launch_bounds__(DC_THREADS) k_combine(const void* __restrict__ out, const float* __restrict__ gates,
                                                         int T, int k, int H, int S_r, ShardsOut ys) {
     const int lane = threadIdx.x & 31;
     const int nvec = H >> 3;
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(DC_THREADS) k_combine(const uint4* __restrict_
     for (int t = blockIdx.x * (DC_THREADS / 32) + (threadIdx.x >> 5); t < T; t += warps) {
         const int r = t / S_r;
         uint4* dst = reinterpret_cast<uint4*>(ys.p[r]) + (size_t)(t - r * S_r) * nvec;
-        warp_combine_token<KMAX>(out, gates, t, k, nvec, dst, lane);
+        warp_combine_token<KMAX, S>(out, gates, t, k, nvec, dst, lane);
     }
 }
 
@@ -119,16 +120,28 @@ cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, cons
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
-                           int num_sms, cudaStream_t stream) {
+template <class S>
+static void launch_combine_t(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
+                             int grid, cudaStream_t stream) {
+    // KB slots' loads in flight per lane: all of them up to 8 (fp32 slots:
+    // 2 x 16 bytes each); k > 8 takes several rounds
+    if (k <= 2)
+        k_combine<2, S><<<grid, DC_THREADS, 0, stream>>>(out, gates, T, k, H, S_r, ys);
+    else if (k <= 4)
+        k_combine<4, S><<<grid, DC_THREADS, 0, stream>>>(out, gates, T, k, H, S_r, ys);
+    else
+        k_combine<8, S><<<grid, DC_THREADS, 0, stream>>>(out, gates, T, k, H, S_r, ys);
+}
+
+cudaError_t launch_combine(const void* out, bool slots_bf16, const float* gates, int T, int k, int H, int S_r,
+                           const ShardsOut& ys, int num_sms, cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
     const int want = (T + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     const int grid = want < num_sms * 8 ? want : num_sms * 8;
-    const uint4* o = reinterpret_cast<const uint4*>(out);
-    if (k <= 2)
-        k_combine<2><<<grid, DC_THREADS, 0, stream>>>(o, gates, T, k, H, S_r, ys);
+    if (slots_bf16)
+        launch_combine_t<SlotBf16>(out, gates, T, k, H, S_r, ys, grid, stream);
     else
-        k_combine<8><<<grid, DC_THREADS, 0, stream>>>(o, gates, T, k, H, S_r, ys);
+        launch_combine_t<SlotF32>(out, gates, T, k, H, S_r, ys, grid, stream);
     return cudaGetLastError();
 }
 

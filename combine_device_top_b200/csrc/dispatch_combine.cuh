@@ -113,40 +113,62 @@ __device__ __forceinline__ void warp_mx_quant8(const uint4& raw, uint2& q, uint3
            (__shfl_sync(0xffffffffu, sb, h0 + 8) << 16) | (__shfl_sync(0xffffffffu, sb, h0 + 12) << 24);
 }
 
+// Slot outputs as the grouped GEMM stores them: fp32 (bf16 path) or bf16
+// (MXFP8 path).  SlotF32 / SlotBf16 load the 8 consecutive features of
+// slot row `row` that a lane owns (v = index of the 8-feature group).
+struct SlotF32 {
+    static constexpr int BYTES = 4;
+    __device__ static __forceinline__ void load(const void* out, size_t row, int nvec, int v, float (&f)[8]) {
+        const float4* p = reinterpret_cast<const float4*>(out) + (row * nvec + v) * 2;
+        const float4 a = __ldcs(p), b = __ldcs(p + 1);
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    }
+};
+struct SlotBf16 {
+    static constexpr int BYTES = 2;
+    __device__ static __forceinline__ void load(const void* out, size_t row, int nvec, int v, float (&f)[8]) {
+        const uint4 a = __ldcs(reinterpret_cast<const uint4*>(out) + row * nvec + v);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 x = __bfloat1622float2(b2[p]);
+            f[2 * p] = x.x;
+            f[2 * p + 1] = x.y;
+        }
+    }
+};
+
 // One warp: y[t] = bf16(sum_{j<k} g[t,j] * out[t,j,:]) in fp32, j ascending.
-// out is fp16 [T, k, H]; each lane owns 8 consecutive features (one 16-byte
-// load per slot, one 16-byte store).  nvec = H / 8.  Slots are loaded KB at
-// a time (KB loads in flight), then accumulated in order.
-template <int KB>
-__device__ __forceinline__ void warp_combine_token(const uint4* __restrict__ out, const float* __restrict__ gates,
+// out is [T, k, H] of slot type S; each lane owns 8 consecutive features
+// (one 16-byte store of y).  nvec = H / 8.  Slots are loaded KB at a time
+// (KB loads in flight), then accumulated in order; k > KB takes several
+// rounds of KB.
+template <int KB, class S>
+__device__ __forceinline__ void warp_combine_token(const void* __restrict__ out, const float* __restrict__ gates,
                                                    int t, int k, int nvec, uint4* __restrict__ dst, int lane) {
-    const uint4* src = out + (size_t)t * k * nvec;
-    const float* gt = gates + (size_t)t * k;
+    const size_t row0 = (size_t)t * k;
+    const float* gt = gates + row0;
     // lanes may run different numbers of iterations (nvec % 32 != 0): no
     // warp collectives inside; the gates are broadcast loads (L1 hits)
     for (int v = lane; v < nvec; v += 32) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j0 = 0; j0 < k; j0 += KB) {
-            uint4 a[KB];
+            float a[KB][8];
             float g[KB];
 #pragma unroll
             for (int jj = 0; jj < KB; ++jj) {
                 const int j = j0 + jj;
                 if (j < k) {
                     g[jj] = __ldg(gt + j);
-                    a[jj] = __ldcs(src + (size_t)j * nvec + v);
+                    S::load(out, row0 + j, nvec, v, a[jj]);
                 }
             }
 #pragma unroll
             for (int jj = 0; jj < KB; ++jj)
                 if (j0 + jj < k) {
-                    const __half2* h2 = reinterpret_cast<const __half2*>(&a[jj]);
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const float2 f = __half22float2(h2[p]);
-                        acc[2 * p] = fmaf(g[jj], f.x, acc[2 * p]);
-                        acc[2 * p + 1] = fmaf(g[jj], f.y, acc[2 * p + 1]);
-                    }
+                    for (int p = 0; p < 8; ++p) acc[p] = fmaf(g[jj], a[jj][p], acc[p]);
                 }
         }
         uint4 o;

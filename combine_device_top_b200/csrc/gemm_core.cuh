@@ -18,18 +18,18 @@
 //     lanes 0-63 hold gate, 64-127 up; the epilogue forms
 //     h = silu(gate) * up and stores h rows.
 //   down unit (phase 1): A = 128 columns of Wd (MN-major from [E, I, H]),
-//     B = the chunk's h rows.  The epilogue stores fp16 rows to
-//     out[row_slot[row]] (the push combine); fp16 rather than bf16 because a
-//     bf16 slot buffer adds a rounding that puts the largest element error of
-//     y above 2e-2 * rms(y) on heavy-tailed outputs (fp16's 3 more mantissa
-//     bits keep it at the floor of y's own bf16 rounding).
-// Precision: the bf16 path computes gate/up in bf16 and the down projection
-// in fp16 (fp16 h and the fp16 copy of Wd: 3 more mantissa bits on h keep
-// the error of y at the floor of its own bf16 rounding).  The MXFP8 path
-// runs the block-scaled tensor-core MMA (kind::mxf8f6f4): E4M3 weights and
-// E4M3 token rows / h rows, each with one E8M0 scale per 32 K values, which
-// the MMA reads from TMEM; the products are exact and accumulate in fp32.
-// The gather quantises x and the gate/up epilogue quantises h.
+//     B = the chunk's h rows.  The epilogue pushes each row's 128 outputs
+//     to out[row_slot[row]] (the push combine): fp32 on the bf16 path, bf16
+//     on the MXFP8 path.
+// Precision: the bf16 path runs both GEMMs as bf16 x bf16 with fp32
+// accumulation on the caller's bf16 weights; h = silu(gate) * up is rounded
+// once to bf16 (the range of fp32, no saturation) and the slot outputs stay
+// fp32, so the only roundings before y's own are h's.  The MXFP8 path runs
+// the block-scaled tensor-core MMA (kind::mxf8f6f4): E4M3 weights and E4M3
+// token rows / h rows, each with one E8M0 scale per 32 K values, which the
+// MMA reads from TMEM; the products are exact and accumulate in fp32.  The
+// gather quantises x, the gate/up epilogue quantises h, and the slot
+// outputs are bf16.
 //
 // Roles in a CTA: warp 0 issues TMA loads into a ring of stages, warp 1
 // allocates 512 TMEM columns and one thread of it issues tcgen05.mma into
@@ -54,7 +54,7 @@
 namespace mok {
 
 constexpr int BK = 64;                            // K per stage: one 128-byte swizzle atom
-constexpr int A_BYTES = 128 * BK * 2;             // 16 KB: two {64 MN x 64 K} bf16/fp16 halves
+constexpr int A_BYTES = 128 * BK * 2;             // 16 KB: two {64 MN x 64 K} bf16 halves
 constexpr int B_ROW_BYTES = BK * 2;               // 128 bytes of one token row per stage
 constexpr int B_BYTES = CHUNK_MAX_ROWS * B_ROW_BYTES;  // 32 KB
 constexpr int EPI_TLD = 132;                      // fp32 staging pitch: 32 tokens x 128 features (+4)
@@ -132,8 +132,8 @@ struct Unit {
 
 struct CoreArgs {
     int H, I;
-    void* h;                  // [buffer rows, I]: fp16 (bf16 path) or E4M3 (MXFP8 path)
-    __half* out;              // [N_s, H] fp16, slot-indexed
+    void* h;                  // [buffer rows, I]: bf16 (bf16 path) or E4M3 (MXFP8 path)
+    void* out;                // [N_s, H] slot-indexed: fp32 (bf16 path) or bf16 (MXFP8 path)
     const int32_t* row_slot;  // [N_s]
     DevStatus* st;
     uint64_t timeout_ns;
@@ -199,7 +199,7 @@ __device__ __forceinline__ int unit_subs(const CoreArgs& a, const Unit& u) {
 __device__ __forceinline__ int token_box(int rows) { return ((rows + 15) >> 4) - 1; }
 
 // ------------------------------------------------------------------ producer
-// Loads the weight tile (bf16/fp16 halves, or MXFP8 bytes + scales) and the
+// Loads the weight tile (bf16 halves, or MXFP8 bytes + scales) and the
 // token tile of every k-step of every unit into the stage ring.
 template <class S, class C>
 __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps* mx, const CoreArgs& a, const S& s,
@@ -389,8 +389,8 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
         const int nsub = unit_subs<C>(a, u);
         const int nt = unit_tickets<C>(nsub, N);
         const bool wide = nt == 2;
-        // bf16 path: gate/up bf16 x bf16, down fp16 x fp16
-        const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, u.phase == 0 ? 1 : 0);
+        // bf16 path: both phases bf16 x bf16
+        const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, /*bf16*/ 1);
         bool ok = true;
         for (int t = 0; t < nt && ok; ++t) {
             const uint32_t tkt = tk + (uint32_t)t;
@@ -467,7 +467,8 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
 // tokens at a time, through a token-major staging tile in shared memory
 // (epi[token][feature], pitch EPI_TLD), so that every global store is a
 // row-contiguous run: gate/up writes h rows (8 lanes per 64-feature row),
-// down pushes 256-byte fp16 rows (a warp per row) to the tokens' slots.
+// down pushes a row's 128 outputs (a warp per row: 512 bytes of fp32, or
+// 256 bytes of bf16 on the MXFP8 path) to the tokens' slots.
 // Chunks cc0, cc0 + ccstep, ... of the tile are drained by this warpgroup
 // (named barrier `bar`, staging tile `epi`).
 template <class C>
@@ -525,15 +526,16 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                         }
                     }
                 } else {
-                    const uint4 pk = make_uint4(pack_half2_sat(hv[0], hv[1]), pack_half2_sat(hv[2], hv[3]),
-                                                pack_half2_sat(hv[4], hv[5]), pack_half2_sat(hv[6], hv[7]));
+                    const uint4 pk = make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
+                                                pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7]));
                     if (live)
                         *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) + row * a.I + mt * MT_G_FEATURES +
                                                   j0) = pk;
                 }
             }
         } else {
-            // fp16 push to the token's slot, one 256-byte row per warp store; the combine rounds y once
+            // push to the token's slot, one row per warp store (fp32: 512 bytes, MXFP8 path bf16: 256
+            // bytes); the combine rounds y once
 #pragma unroll 4
             for (int it = 0; it < 8; ++it) {
                 const int t = it * 4 + q;
@@ -541,8 +543,12 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 if (col < u.rows) {
                     const int slot = __ldg(a.row_slot + u.grow0 + col);
                     const float4 o4 = *reinterpret_cast<const float4*>(epi + t * EPI_TLD + 4 * lane);
-                    reinterpret_cast<uint2*>(a.out + (size_t)slot * a.H + mt * MT_D_FEATURES)[lane] =
-                        make_uint2(pack_half2_sat(o4.x, o4.y), pack_half2_sat(o4.z, o4.w));
+                    const size_t at = (size_t)slot * a.H + mt * MT_D_FEATURES;
+                    if constexpr (C::MX)
+                        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + at)[lane] =
+                            make_uint2(pack_bf16x2(o4.x, o4.y), pack_bf16x2(o4.z, o4.w));
+                    else
+                        reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + at)[lane] = o4;
                 }
             }
         }

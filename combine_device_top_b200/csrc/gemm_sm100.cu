@@ -67,7 +67,7 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.H = sh.H;
     a.I = sh.I;
     a.h = h_out;
-    a.out = reinterpret_cast<__half*>(out);
+    a.out = out;
     a.row_slot = row_slot;
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;

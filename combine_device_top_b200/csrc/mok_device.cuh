@@ -239,7 +239,7 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
 }
 
 // Instruction descriptor, kind::f16 with fp32 accumulation; A and B share
-// one type (bf16 when `bf16` is set, else fp16):
+// one type (bf16 when `bf16` is set, else fp16; this library uses bf16):
 // [4,6) D fmt (1 = f32), [7,10) A fmt (0 = f16, 1 = bf16), [10,13) B fmt,
 // [15] A major (1 = MN), [16] B major (1 = MN), [17,23) N>>3, [24,29) M>>4.
 __host__ __device__ __forceinline__ uint32_t umma_idesc_f16(int M, int N, int a_mn_major, int b_mn_major, int bf16) {
@@ -329,15 +329,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Two fp32 -> fp16x2, round to nearest even, magnitudes above 65504 clamped
-// to 65504.
-__device__ __forceinline__ uint32_t pack_half2_sat(float a, float b) {
-    a = fminf(fmaxf(a, -65504.f), 65504.f);
-    b = fminf(fmaxf(b, -65504.f), 65504.f);
-    __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 

@@ -43,8 +43,10 @@ cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, cons
 // E4M3, block scales in planes [H/128][sc_rows][4] (see mx_sc_rows)
 cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
                              void* xsc, int sc_rows, int num_sms, cudaStream_t stream);
-cudaError_t launch_combine(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
-                           int num_sms, cudaStream_t stream);
+// y = fixed-order weighted sum of the slot outputs out [T*k, H]: fp32, or
+// bf16 when slots_bf16 (the MXFP8 path)
+cudaError_t launch_combine(const void* out, bool slots_bf16, const float* gates, int T, int k, int H, int S_r,
+                           const ShardsOut& ys, int num_sms, cudaStream_t stream);
 
 // ---- work decomposition of the grouped GEMM
 // A chunk is <= 256 consecutive rows of one expert inside one minibatch.
@@ -62,10 +64,17 @@ constexpr int CHUNK_MAX_ROWS_MX = 224;
 
 int max_chunks(int n_slots, int E, int n_mb);
 int max_minibatches(int n_slots, int minibatch);
-// max_rows: chunk height cap, CHUNK_MAX_ROWS or CHUNK_MAX_ROWS_MX
+// Rows of the expert-major layout that give `waves` full waves of
+// gemm_ctas CTAs when a unit is a tile of tile_rows rows x tile_features of
+// the 2I gate+up output columns: ceil(waves * ctas * rows * features / 2I).
+int two_wave_rows(int I, int gemm_ctas, int waves, int tile_rows, int tile_features);
+// max_rows: chunk height cap, CHUNK_MAX_ROWS or CHUNK_MAX_ROWS_MX.  A
+// minibatch ends at the first expert boundary where it holds at least
+// `minibatch` rows and min_units gate/up units (units_per_chunk per chunk),
+// or at `cap` rows.
 cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int minibatch, int cap, int max_rows,
-                                Chunk* chunks, int max_chunks, Minibatch* mbs, int max_mb, int* counts2, void* status,
-                                cudaStream_t stream);
+                                int min_units, int units_per_chunk, Chunk* chunks, int max_chunks, Minibatch* mbs,
+                                int max_mb, int* counts2, void* status, cudaStream_t stream);
 
 // ---- the grouped GEMM (tcgen05)
 struct GemmShape {
@@ -87,14 +96,14 @@ constexpr int B_MAX_BOX = 256;
 struct BMaps {
     CUtensorMap m[B_MAPS];
 };
-bool encode_bmaps(BMaps* maps, bool bf16, const void* base, uint64_t inner, uint64_t rows, const char** err);
+bool encode_bmaps(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err);
 
 // Every tensor map the GEMM core reads.
 struct GemmMaps {
-    CUtensorMap wg, wu, wd;  // 64x64 boxes of Wg, Wu (bf16) and Wd (fp16)
+    CUtensorMap wg, wu, wd;  // 64x64 boxes of Wg, Wu and Wd (bf16)
     CUtensorMap wd3;         // Wd as {64, E*I, H/64}: one op loads both 64-column halves of a down tile
     BMaps rows;              // token rows (bf16) of the row buffer
-    BMaps h;                 // h rows (fp16) of the h buffer
+    BMaps h;                 // h rows (bf16) of the h buffer
     int has_wd3;             // wd3 could be encoded (else two 2D ops per down stage)
 };
 bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
@@ -123,7 +132,7 @@ struct MxTokenScales {
 };
 
 // Staged grouped GEMM over every chunk: phase 0 = gate/up + SwiGLU -> h,
-// phase 1 = down -> out[row_slot].
+// phase 1 = down -> out[row_slot] (fp32 slots; bf16 on the MXFP8 path).
 struct MxMaps;
 // mx: MXFP8 weight maps (MXFP8 path: rows and h are E4M3 with the scale
 // planes of mxs), or nullptr (bf16 path).
@@ -135,14 +144,15 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
 // ---- the persistent SM-partitioned forward (persistent.cu)
 struct PersistLaunch {
     int grid, dispatch_ctas, cap;  // CTAs, of which the first dispatch_ctas gather; ring half rows
+    bool pair;                     // bf16 GEMM units of two M tiles (the work list counted units this way)
     int H, I, E, T, k, S_r;
-    const void *wg, *wu, *wd;      // weights (bf16, bf16, fp16); unused on the MXFP8 path
+    const void *wg, *wu, *wd;      // bf16 weights; unused on the MXFP8 path
     const mok_mxfp8_weights* mxw;  // MXFP8 weights, or nullptr (bf16 path)
     void* ring;                    // [2*cap, H] bf16, or E4M3 (MXFP8)
-    void* h;                       // [2*cap, I] fp16, or E4M3 (MXFP8)
+    void* h;                       // [2*cap, I] bf16, or E4M3 (MXFP8)
     uint8_t *ring_sc, *h_sc;       // MXFP8: scale planes of ring and h rows (sc_rows = mx_sc_rows(2*cap))
     int sc_rows;
-    __half* out;                   // [T*k, H] fp16
+    void* out;                     // [T*k, H] fp32, or bf16 (MXFP8)
     const Chunk* chunks;
     const Minibatch* mbs;
     const int* counts2;
@@ -157,18 +167,15 @@ struct PersistLaunch {
 cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, cudaStream_t stream);
 
 // ---- tensor maps (driver entry point fetched at run time)
-// 2D tiled map of a row-major [outer, inner] array of 16-bit elements
-// (bf16 or fp16), 128-byte swizzle, zero fill out of bounds.
-bool encode_tmap_2d_16b(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t outer,
-                        uint32_t box_inner, uint32_t box_outer, const char** err);
+// 2D tiled map of a row-major [outer, inner] array of bf16 elements,
+// 128-byte swizzle, zero fill out of bounds.
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer, const char** err);
 
 // ---- MXFP8 quantisers (mxfp8.cu)
 cudaError_t launch_mx_quant_rows(const void* src, bool f32, int rows, int K, void* q, void* scales, int num_sms,
                                  cudaStream_t stream);
 cudaError_t launch_mx_quant_cols(const void* src, int nblocks, int N, void* q, void* scales, int num_sms,
                                  cudaStream_t stream);
-
-// ---- weight preparation
-cudaError_t launch_bf16_to_fp16(const void* src, void* dst, size_t n, int num_sms, cudaStream_t stream);
 
 }  // namespace mok

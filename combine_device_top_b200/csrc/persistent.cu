@@ -249,7 +249,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int t = blockIdx.x * (C::THREADS / 32) + warp; t < p.T; t += warps) {
         const int r = t / p.S_r;
         uint4* dst = reinterpret_cast<uint4*>(p.ys.p[r]) + (size_t)(t - r * p.S_r) * nvec;
-        warp_combine_token<KMAX>(reinterpret_cast<const uint4*>(a.out), p.gates, t, p.k, nvec, dst, lane);
+        if constexpr (C::MX)
+            warp_combine_token<KMAX, SlotBf16>(a.out, p.gates, t, p.k, nvec, dst, lane);
+        else
+            warp_combine_token<KMAX, SlotF32>(a.out, p.gates, t, p.k, nvec, dst, lane);
     }
 }
 
@@ -310,9 +313,10 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.mbs = L.mbs;
     p.counts2 = L.counts2;
     p.cap = L.cap;
-    // the staged GEMM's rule for M-tile pairs: mean rows per expert <= 192
-    // (bf16 only; the MXFP8 path runs one M tile per unit)
-    const bool pair = !L.mxw && gemm_tuning(L.T * L.k, L.E).pair != 0;
+    // the staged GEMM's rule for M-tile pairs (mean rows per expert <= 192),
+    // decided by the caller with the work list; bf16 only, the MXFP8 path
+    // runs one M tile per unit
+    const bool pair = !L.mxw && L.pair;
     const int sub = pair ? Bf16PairCfg::SUB : Bf16Cfg::SUB;
     // units per chunk (with pairs the last one may be single)
     p.MTG = (L.I / MT_G_FEATURES + sub - 1) / sub;
@@ -333,6 +337,7 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.ring = L.ring;
     p.ring_sc = L.ring_sc;
     *err = "persistent launch";
+    // KMAX slots' loads in flight per lane in the combine (k > KMAX: several rounds)
     if (L.mxw) {
         if (L.k <= 2) return launch_persistent_k<2, MxCfg>(L.grid, maps, mx, a, p, stream);
         return launch_persistent_k<8, MxCfg>(L.grid, maps, mx, a, p, stream);

@@ -11,8 +11,10 @@
 namespace mok {
 
 // ------------------------------------------------------------------ work list
-// One block.  Minibatch boundaries: from row b0, the first expert boundary at
-// or after b0 + minibatch, but never more than `cap` rows; then every
+// One block.  Minibatch boundaries: from row b0, walk the expert boundaries
+// until the minibatch holds at least M rows AND at least min_units gate/up
+// units (chunks x units per chunk: two full waves of the GEMM CTAs is the
+// pages' rule), but never more than `cap` rows (one ring half); then every
 // (expert, minibatch) piece is cut into ceil(len / maxr) chunks of nearly
 // equal size (multiples of 16 rows except the last; maxr is a multiple of 16).
 __device__ __forceinline__ int piece_chunks(int L, int maxr) { return (L + maxr - 1) / maxr; }
@@ -24,35 +26,32 @@ __device__ __forceinline__ int piece_base(int L, int maxr) {
 }
 
 __global__ void __launch_bounds__(1024) k_build_chunks(const int32_t* __restrict__ offsets, int E, int n_slots,
-                                                       int M, int cap, int maxr, Chunk* __restrict__ chunks,
-                                                       int max_chunks,
+                                                       int M, int cap, int maxr, int min_units, int upc,
+                                                       Chunk* __restrict__ chunks, int max_chunks,
                                                        Minibatch* __restrict__ mbs, int max_mb,
                                                        int* __restrict__ counts2, DevStatus* st) {
     __shared__ int s_nmb;
     __shared__ int warp_sums[32];
     if (threadIdx.x == 0) {
-        int b0 = 0, n = 0;
+        int b0 = 0, n = 0, e = 0;
         while (b0 < n_slots) {
-            int b1;
-            const int target = b0 + M;
-            if (target >= n_slots) {
-                b1 = n_slots;
-            } else {
-                int lo = 0, hi = E;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (offsets[mid] >= target) hi = mid; else lo = mid + 1;
-                }
-                b1 = offsets[lo];
-                if (b1 > b0 + cap) b1 = b0 + cap;
+            while (e < E - 1 && offsets[e + 1] <= b0) ++e;  // expert holding row b0
+            const int limit = min(n_slots, b0 + cap);
+            int b = b0, units = 0, ee = e;
+            while (true) {
+                const int end = min(offsets[ee + 1], limit);
+                units += piece_chunks(end - b, maxr) * upc;
+                b = end;
+                if (b >= limit || (b >= b0 + M && units >= min_units) || ee == E - 1) break;
+                ++ee;
             }
             if (n >= max_mb) {
                 set_status(st, MOK_ERR_CAPACITY, 1, n, max_mb);
                 break;
             }
-            mbs[n] = Minibatch{b0, b1, 0, 0};
+            mbs[n] = Minibatch{b0, b, 0, 0};
             ++n;
-            b0 = b1;
+            b0 = b;
         }
         s_nmb = n;
     }
@@ -131,15 +130,23 @@ int max_minibatches(int n_slots, int minibatch) {
     if (minibatch <= 0) minibatch = 1;
     return n_slots / minibatch + 2;
 }
+
+int two_wave_rows(int I, int gemm_ctas, int waves, int tile_rows, int tile_features) {
+    if (I <= 0 || gemm_ctas <= 0 || waves <= 0 || tile_rows <= 0 || tile_features <= 0) return 0;
+    const long long num = (long long)waves * gemm_ctas * tile_rows * tile_features;
+    const long long den = 2LL * I;
+    return (int)((num + den - 1) / den);
+}
 // bound for every chunk height cap >= CHUNK_MAX_ROWS_MX
 int max_chunks(int n_slots, int E, int n_mb) { return n_slots / CHUNK_MAX_ROWS_MX + E + n_mb + 2; }
 
 cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int minibatch, int cap, int max_rows,
-                                Chunk* chunks, int max_ch, Minibatch* mbs, int max_mb, int* counts2, void* status,
-                                cudaStream_t stream) {
+                                int min_units, int units_per_chunk, Chunk* chunks, int max_ch, Minibatch* mbs,
+                                int max_mb, int* counts2, void* status, cudaStream_t stream) {
     if (max_rows < CHUNK_MAX_ROWS_MX || max_rows > CHUNK_MAX_ROWS || max_rows % 16) return cudaErrorInvalidValue;
-    k_build_chunks<<<1, 1024, 0, stream>>>(offsets, E, n_slots, minibatch, cap, max_rows, chunks, max_ch, mbs, max_mb,
-                                           counts2, reinterpret_cast<DevStatus*>(status));
+    if (units_per_chunk < 1) return cudaErrorInvalidValue;
+    k_build_chunks<<<1, 1024, 0, stream>>>(offsets, E, n_slots, minibatch, cap, max_rows, min_units, units_per_chunk,
+                                           chunks, max_ch, mbs, max_mb, counts2, reinterpret_cast<DevStatus*>(status));
     return cudaGetLastError();
 }
 

@@ -64,11 +64,18 @@ enum {
 
 enum { MOK_MAX_SHARDS = 64, MOK_MAX_EXPERTS = 1024, MOK_MAX_TOPK = 32 };
 
+/* Element type of the per-slot expert outputs out [T, k, H] that the
+ * grouped GEMM pushes and the combine reads: fp32 on the bf16 path, bf16 on
+ * the MXFP8 path. */
+enum { MOK_SLOTS_F32 = 0, MOK_SLOTS_BF16 = 1 };
+
 /* ------------------------------------------------------------------------
  * Step 1 + 2: the plan.
  * ---------------------------------------------------------------------- */
 
-/* Views into the plan workspace, filled by mok_plan().  All device arrays. */
+/* Views into the plan workspace, filled by mok_plan().  All device arrays.
+ * A caller of mok_plan_noalloc fills one by hand from the arrays it passed
+ * there (and T, E, k, R); the forward accepts it like mok_plan's. */
 typedef struct mok_plan_t {
     int32_t T, E, k, R;
     int32_t* counts;          /* [E]   tokens routed to expert e              */
@@ -127,7 +134,11 @@ int mok_plan(const float* logits, int T, int E, int top_k, int R,
  *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library
  *   routine is called.  The first call on a device looks up the array's
  *   device address (cudaGetSymbolAddress, with that device current); make
- *   that first call before any stream capture.
+ *   that first call before any stream capture.  The looked-up address is
+ *   kept for the life of the process and belongs to the device's primary
+ *   context (the one the CUDA runtime uses): after cudaDeviceReset, or when
+ *   the calling thread has another context of that device current, it is
+ *   stale, so do not call this entry point then.
  *   All calls on one device share the array: calls whose kernels may run at
  *   the same time on the GPU (unordered streams) race on it.  Every call
  *   writes each scratch entry before reading it, so no clearing is needed.
@@ -158,7 +169,9 @@ typedef struct mok_fwd_opts {
     int32_t mxfp8;         /* 1 = MXFP8 path (weights from                      */
                            /* mok_quantize_weights_mxfp8; either mode);         */
                            /* 0 = bf16                                          */
-    int32_t reserved;      /* must be 0                                         */
+    int32_t min_waves;     /* persistent mode: a minibatch holds at least this  */
+                           /* many full waves of gate/up units of the GEMM     */
+                           /* CTAs; 0 = 2 (the pages' rule); < 0 = no floor    */
     uint64_t timeout_ns;   /* bound on every device-side wait; 0 = 2 s          */
 } mok_fwd_opts;
 
@@ -192,27 +205,31 @@ size_t mok_forward_workspace_bytes(int T, int H, int I, int E, int k, int miniba
  *   H, I      hidden and intermediate sizes; H % 128 == 0, I % 64 == 0
  *   w_gate    [E, H, I] bf16
  *   w_up      [E, H, I] bf16
- *   w_down    [E, I, H] fp16: the copy mok_prepare_w_down() makes of the
- *             bf16 W_down (once, at weight-load time)
+ *   w_down    [E, I, H] bf16
  *   plan      from mok_plan() on the same stream (its workspace must live)
- *   minibatch rows of the expert-major layout per minibatch (persistent
- *             mode; >= 16); boundaries snap forward to expert boundaries
- *             where the ring allows.  Ignored in staged mode.
+ *   minibatch persistent mode: the least rows of the expert-major layout
+ *             per minibatch (>= 16), or 0 for the two-wave rule alone.  A
+ *             minibatch ends at the first expert boundary where it holds
+ *             at least `minibatch` rows and opts->min_waves (default 2)
+ *             full waves of gate/up units for the GEMM CTAs, or at half
+ *             the ring (an expert taller than that is split).  Ignored in
+ *             staged mode (one minibatch).
  *   opts      may be NULL (persistent mode, defaults)
  *   ws        forward workspace (>= mok_forward_workspace_bytes)
  *   y_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
  * Arithmetic: gate/up in bf16 x bf16 with fp32 accumulation; h =
- * silu(gate) * up rounded to fp16 (saturating at +-65504); down projection
- * fp16 x fp16 with fp32 accumulation; each expert output row stored fp16 at
- * its slot (saturating); y[t] = bf16(sum_{j<k} g[t,j] * o[t,j]) accumulated in fp32
- * with j ascending (one bf16 rounding of y).  y does not depend on the
+ * silu(gate) * up rounded once to bf16; down projection bf16 x bf16 with
+ * fp32 accumulation; each expert output row stored fp32 at its slot;
+ * y[t] = bf16(sum_{j<k} g[t,j] * o[t,j]) accumulated in fp32 with j
+ * ascending (one bf16 rounding of y).  No step saturates: every stored
+ * intermediate has the exponent range of fp32.  y does not depend on the
  * mode, minibatch, ring size or R.
  * MXFP8 path (opts->mxfp8 = 1, either mode, w_gate = a mok_mxfp8_weights
  * HOST struct): x is quantised in the gather (persistent mode: by the
  * dispatch CTAs, into the ring) and h in the SwiGLU epilogue
  * (32-element blocks, E8M0 scale + E4M3 values, as mok_mxfp8_quantize_rows
  * does); both GEMMs run on the block-scaled E4M3 x E4M3 tensor-core MMA
- * with fp32 accumulation; slot outputs fp16 and the combine as above.
+ * with fp32 accumulation; slot outputs bf16 and the combine as above.
  */
 int mok_moe_forward(const void* const* x_shards, int H, int I,
                     const void* w_gate, const void* w_up, const void* w_down,
@@ -220,17 +237,33 @@ int mok_moe_forward(const void* const* x_shards, int H, int I,
                     void* ws, size_t ws_bytes, void* const* y_shards, mok_stream_t stream);
 
 /*
- * mok_prepare_w_down -- one-time conversion of W_down from bf16 to the fp16
- * copy the forward's down projection reads (elementwise, `count` elements,
- * e.g. E*I*H).  Exact for every bf16 value of magnitude in [2^-14, 65504];
- * smaller magnitudes round to fp16's subnormal grid (spacing 2^-24), larger
- * ones saturate to +-65504.  Both buffers are device memory owned by the
- * caller, 16-byte aligned, not overlapping.  Asynchronous on `stream`.
- * (No counterpart in the pages: it serves the down projection's fp16
- * arithmetic, which keeps the error of y near the floor of its own bf16
- * rounding.)
+ * mok_two_wave_rows -- the two-wave minibatch size: the rows of the
+ * expert-major layout whose gate/up output tiles (tile_rows rows x
+ * tile_features of the 2I gate and up columns each) make two full waves of
+ * `gemm_ctas` CTAs, ceil(2 * gemm_ctas * tile_rows * tile_features / (2 I)).
+ * Source: MoK article, minibatch paragraph (a minibatch must fill at least
+ * two waves of the GEMM SMs, about 2368 tokens at hidden 7168 /
+ * intermediate 2048; that is 128 x 256 tiles over 148 SMs); MoK wiki
+ * summary, minibatch bullet.  The forward's own units are chunks of up to
+ * 256 rows x 128 features (256 with M-tile pairs), and it counts them on
+ * the device (see mok_moe_forward's minibatch); this host formula gives the
+ * rows that suffice when every chunk is full height.  Returns 0 for
+ * non-positive arguments.
  */
-int mok_prepare_w_down(const void* w_down_bf16, void* w_down_fp16, size_t count, mok_stream_t stream);
+int mok_two_wave_rows(int I, int gemm_ctas, int tile_rows, int tile_features);
+
+/*
+ * mok_minibatch_bounds -- the minibatches mok_moe_forward would use for
+ * these arguments (persistent mode): builds the work list in `ws` exactly
+ * as the forward does, synchronises `stream`, and writes to HOST arrays the
+ * first row of each minibatch (row0) and, if `units` is not NULL, its
+ * gate/up unit count; at most max_mb entries; *n_mb receives the number of
+ * minibatches.  Arguments and errors as for mok_moe_forward (x and y are
+ * not needed).  An inspection call: it synchronises the host.
+ */
+int mok_minibatch_bounds(const mok_plan_t* plan, int H, int I, const void* w_gate, int minibatch,
+                         const mok_fwd_opts* opts, void* ws, size_t ws_bytes, int32_t* row0,
+                         int32_t* units, int max_mb, int* n_mb, mok_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * MXFP8 (OCP MX v1.0: 32-element blocks, E8M0 scale byte = s + 127 with
@@ -292,13 +325,12 @@ int mok_gather_mxfp8(const void* const* x_shards, int H, const mok_plan_t* plan,
 size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E);
 
 /* Grouped SwiGLU FFN over the expert-major rows of `plan`:
- *   h[row]   = fp16(silu(rows[row] Wg[e]) * (rows[row] Wu[e]))   [N_s, I]
- *   out[row_slot[row]] = fp16(h[row] Wd16[e])  (fp32 accumulation) [N_s, H]
- * (e = expert of the row; Wd16 = fp16 W_down from mok_prepare_w_down).
- * h stays in the workspace; `out` is fp16 and
- * slot-indexed, i.e. [T, k, H].  Source: MoK article, routing paragraph
- * (grouped GEMM over contiguous per-expert tokens) and push-combine
- * paragraph. */
+ *   h[row]   = bf16(silu(rows[row] Wg[e]) * (rows[row] Wu[e]))   [N_s, I]
+ *   out[row_slot[row]] = h[row] Wd[e]  (fp32 accumulation and result) [N_s, H]
+ * (e = expert of the row; all weights bf16).  h stays in the workspace;
+ * `out` is fp32 (MOK_SLOTS_F32) and slot-indexed, i.e. [T, k, H].  Source:
+ * MoK article, routing paragraph (grouped GEMM over contiguous per-expert
+ * tokens) and push-combine paragraph. */
 int mok_expert_ffn(const void* rows, int H, int I,
                    const void* w_gate, const void* w_up, const void* w_down,
                    const mok_plan_t* plan, void* ws, size_t ws_bytes,
@@ -311,16 +343,17 @@ size_t mok_expert_ffn_mxfp8_workspace_bytes(int n_rows, int I, int E);
  * over the output of mok_gather_mxfp8 (rows_q, scales; same layouts), with
  * the weight pack `w` (host struct) of mok_quantize_weights_mxfp8.  h is
  * quantised to MXFP8 in the SwiGLU epilogue and stays in the workspace;
- * out: [T, k, H] fp16, slot-indexed, as mok_expert_ffn.  Source: MoK
+ * out: [T, k, H] bf16 (MOK_SLOTS_BF16), slot-indexed.  Source: MoK
  * article, paragraph on MXFP8 inside the GEMM and SwiGLU. */
 int mok_expert_ffn_mxfp8(const void* rows_q, const void* scales, int H, int I,
                          const mok_mxfp8_weights* w, const mok_plan_t* plan,
                          void* ws, size_t ws_bytes, void* out, mok_stream_t stream);
 
 /* y[t] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]), fp32, j ascending,
- * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] fp16.
+ * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] of out_dtype
+ * (MOK_SLOTS_F32 or MOK_SLOTS_BF16), 16-byte aligned.
  * Source: MoK article, benchmark paragraph (final weighted merge). */
-int mok_combine(const void* out, int H, const mok_plan_t* plan,
+int mok_combine(const void* out, int out_dtype, int H, const mok_plan_t* plan,
                 void* const* y_shards, mok_stream_t stream);
 
 /* ------------------------------------------------------------------------
@@ -335,7 +368,7 @@ size_t mok_forward_host_workspace_bytes(int T, int H, int I, int E, int k, int m
  * mok_moe_forward_host -- copies HOST x [T, H] bf16 and HOST logits [T, E]
  * fp32 to the device, runs mok_plan and mok_moe_forward, copies y [T, H]
  * bf16 back to HOST memory and synchronises `stream`.  Weights are device
- * pointers as in mok_moe_forward (w_down: the fp16 copy).  Host buffers should be pinned for
+ * pointers as in mok_moe_forward.  Host buffers should be pinned for
  * full copy bandwidth (pageable memory works, slower).  ws: device
  * workspace of mok_forward_host_workspace_bytes().
  */

@@ -129,47 +129,65 @@ int oracle_mxfp8_expert_ffn(const uint16_t* x_rows, int n, int H, int I,
     double* qg = (double*)malloc(sizeof(double) * (size_t)H * I);   /* [I][H]: column i over K=H */
     double* qu = (double*)malloc(sizeof(double) * (size_t)H * I);
     double* qd = (double*)malloc(sizeof(double) * (size_t)I * H);   /* [H][I]: column c over K=I */
-    double* col = (double*)malloc(sizeof(double) * (size_t)(H > I ? H : I));
-    double* xr = (double*)malloc(sizeof(double) * (size_t)H);
-    double* xq = (double*)malloc(sizeof(double) * (size_t)H);
-    double* hv = (double*)malloc(sizeof(double) * (size_t)I);
-    double* hq = (double*)malloc(sizeof(double) * (size_t)I);
-    float* hf = (float*)malloc(sizeof(float) * (size_t)I);
-    int rc = ORACLE_ENOMEM;
-    if (!qg || !qu || !qd || !col || !xr || !xq || !hv || !hq || !hf) goto done;
-    /* weights: blocks along the contraction index of each output column */
-    for (int i = 0; i < I; ++i) {
-        for (int k = 0; k < H; ++k) col[k] = o_bf16(wg[(size_t)k * I + i]);
-        mx_roundtrip(col, H, qg + (size_t)i * H);
-        for (int k = 0; k < H; ++k) col[k] = o_bf16(wu[(size_t)k * I + i]);
-        mx_roundtrip(col, H, qu + (size_t)i * H);
+    int rc = ORACLE_OK;
+    if (!qg || !qu || !qd) {
+        free(qg); free(qu); free(qd);
+        return ORACLE_ENOMEM;
     }
-    for (int c = 0; c < H; ++c) {
-        for (int k = 0; k < I; ++k) col[k] = o_bf16(wd[(size_t)k * H + c]);
-        mx_roundtrip(col, I, qd + (size_t)c * I);
-    }
-    for (int r = 0; r < n; ++r) {
-        for (int k = 0; k < H; ++k) xr[k] = o_bf16(x_rows[(size_t)r * H + k]);
-        mx_roundtrip(xr, H, xq);
+    /* Columns and rows are independent; threads split them and each element
+     * is computed exactly as in a serial run. */
+#pragma omp parallel
+    {
+        double* col = (double*)malloc(sizeof(double) * (size_t)(H > I ? H : I));
+        double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+        double* xq = (double*)malloc(sizeof(double) * (size_t)H);
+        double* hv = (double*)malloc(sizeof(double) * (size_t)I);
+        double* hq = (double*)malloc(sizeof(double) * (size_t)I);
+        float* hf = (float*)malloc(sizeof(float) * (size_t)I);
+        const int ok = col && xr && xq && hv && hq && hf;
+        if (!ok) {
+#pragma omp atomic write
+            rc = ORACLE_ENOMEM;
+        }
+        /* weights: blocks along the contraction index of each output column */
+#pragma omp for schedule(static)
         for (int i = 0; i < I; ++i) {
-            double a = 0.0, b = 0.0;
-            const double* g = qg + (size_t)i * H;
-            const double* u = qu + (size_t)i * H;
-            for (int k = 0; k < H; ++k) { a += xq[k] * g[k]; b += xq[k] * u[k]; }
-            hf[i] = (float)(a / (1.0 + exp(-a)) * b);
+            if (!ok) continue;
+            for (int k = 0; k < H; ++k) col[k] = o_bf16(wg[(size_t)k * I + i]);
+            mx_roundtrip(col, H, qg + (size_t)i * H);
+            for (int k = 0; k < H; ++k) col[k] = o_bf16(wu[(size_t)k * I + i]);
+            mx_roundtrip(col, H, qu + (size_t)i * H);
         }
-        if (h_q && h_s) oracle_mxfp8_quantize(hf, I / 32, h_q + (size_t)r * I, h_s + (size_t)r * (I / 32));
-        for (int i = 0; i < I; ++i) hv[i] = (double)hf[i];
-        mx_roundtrip(hv, I, hq);
+#pragma omp for schedule(static)
         for (int c = 0; c < H; ++c) {
-            double acc = 0.0;
-            const double* d = qd + (size_t)c * I;
-            for (int i = 0; i < I; ++i) acc += hq[i] * d[i];
-            o[(size_t)r * H + c] = acc;
+            if (!ok) continue;
+            for (int k = 0; k < I; ++k) col[k] = o_bf16(wd[(size_t)k * H + c]);
+            mx_roundtrip(col, I, qd + (size_t)c * I);
         }
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < n; ++r) {
+            if (!ok) continue;
+            for (int k = 0; k < H; ++k) xr[k] = o_bf16(x_rows[(size_t)r * H + k]);
+            mx_roundtrip(xr, H, xq);
+            for (int i = 0; i < I; ++i) {
+                double a = 0.0, b = 0.0;
+                const double* g = qg + (size_t)i * H;
+                const double* u = qu + (size_t)i * H;
+                for (int k = 0; k < H; ++k) { a += xq[k] * g[k]; b += xq[k] * u[k]; }
+                hf[i] = (float)(a / (1.0 + exp(-a)) * b);
+            }
+            if (h_q && h_s) oracle_mxfp8_quantize(hf, I / 32, h_q + (size_t)r * I, h_s + (size_t)r * (I / 32));
+            for (int i = 0; i < I; ++i) hv[i] = (double)hf[i];
+            mx_roundtrip(hv, I, hq);
+            for (int c = 0; c < H; ++c) {
+                double acc = 0.0;
+                const double* d = qd + (size_t)c * I;
+                for (int i = 0; i < I; ++i) acc += hq[i] * d[i];
+                o[(size_t)r * H + c] = acc;
+            }
+        }
+        free(col); free(xr); free(xq); free(hv); free(hq); free(hf);
     }
-    rc = ORACLE_OK;
-done:
-    free(qg); free(qu); free(qd); free(col); free(xr); free(xq); free(hv); free(hq); free(hf);
+    free(qg); free(qu); free(qd);
     return rc;
 }

@@ -97,6 +97,33 @@ def test_forward_rejects_unsupported_shapes():
     assert rc == mok.MOK_ERR_INVALID_ARG
 
 
+def _filled_plan(T, E, k, R):
+    p = mok.PlanT(T, E, k, R)
+    for name in ("counts", "offsets", "sched_src_rank", "sched_src_index", "row_slot", "pos", "topk_idx", "gates"):
+        setattr(p, name, 4096)
+    return p
+
+
+@pytest.mark.parametrize("T,E,k,what", [(16, 2048, 2, "E"), (64, 64, 33, "k"), (1 << 26, 64, 32, "T * k")])
+def test_hand_filled_plan_gets_the_plan_limits(T, E, k, what):
+    """A plan filled by hand (e.g. from mok_plan_noalloc's outputs) is held to
+    mok_plan's limits before anything is launched."""
+    p = _filled_plan(T, E, k, 1)
+    L = mok.lib()
+    arr = (ctypes.c_void_p * 1)(4096)
+    rc = L.mok_moe_forward(arr, 128, 128, 1, 1, 1, ctypes.byref(p), 256, None, 256, 1 << 30, arr, None)
+    assert rc == mok.MOK_ERR_UNSUPPORTED and what in mok.last_error(), mok.last_error()
+    rc = L.mok_combine(4096, mok.MOK_SLOTS_F32, 128, ctypes.byref(p), arr, None)
+    assert rc == mok.MOK_ERR_UNSUPPORTED
+
+
+def test_combine_rejects_an_unknown_slot_type():
+    p = _filled_plan(16, 8, 2, 2)
+    arr = (ctypes.c_void_p * 2)(4096, 8192)
+    rc = mok.lib().mok_combine(4096, 7, 128, ctypes.byref(p), arr, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG and "slot" in mok.last_error()
+
+
 def test_forward_mxfp8_argument_rules():
     """The MXFP8 path runs in either mode, under the persistent mode's own
     rules, and needs every member of its weight pack.  Every call here fails
@@ -167,7 +194,7 @@ def test_binding_checks_shard_count_before_calling_the_library():
     one = [torch.empty(8, 128, dtype=torch.bfloat16)]          # R = 2 expected
     w = torch.empty(8, 128, 128, dtype=torch.bfloat16)
     pack = tuple(torch.empty(8, 128, 128, dtype=torch.uint8) for _ in range(6))
-    out = torch.empty(32, 128, dtype=torch.float16)
+    out = torch.empty(32, 128, dtype=torch.float32)
     with pytest.raises(AssertionError):
         mok.moe_forward(one, w, w, w, p)
     with pytest.raises(AssertionError):
@@ -178,3 +205,22 @@ def test_binding_checks_shard_count_before_calling_the_library():
         mok.gather_mxfp8(one, p)
     with pytest.raises(AssertionError):
         mok.combine(out, p, one)
+
+
+def test_two_wave_rows_reproduces_the_pages_minibatch():
+    """The library's two-wave formula gives the pages' 2368 rows at hidden
+    7168 / intermediate 2048 on 148 SMs with the fixture's tiling, and the
+    kernel's own chunk units (256 rows x 128 features, or 256 with M-tile
+    pairs) on the 132 GEMM CTAs of the default persistent split."""
+    import json
+
+    with open(os.path.join(ROOT, "tests", "golden", "two_wave_minibatch.json")) as f:
+        g = json.load(f)
+    L = mok.lib()
+    assert L.mok_two_wave_rows(g["I"], g["sms"], g["tile_rows"], g["tile_cols"]) == g["minibatch_min"]
+    assert L.mok_two_wave_rows(2048, 148, 128, 256) == 2368
+    assert L.mok_two_wave_rows(2048, 132, 256, 128) == 2112
+    assert L.mok_two_wave_rows(2048, 132, 256, 256) == 4224
+    assert L.mok_two_wave_rows(14336, 148, 256, 128) == 339         # rounded up
+    assert L.mok_two_wave_rows(0, 148, 128, 256) == 0
+    assert L.mok_two_wave_rows(2048, -1, 128, 256) == 0

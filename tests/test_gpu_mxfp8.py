@@ -154,42 +154,6 @@ def test_mxfp8_persistent_equals_staged(name, minibatch, ring, dispatch):
     assert torch.equal(y_p, y_s), (y_p.double() - y_s.double()).abs().max().item()
 
 
-@pytest.mark.slow
-def test_mxfp8_forward_full_size_sampled():
-    """The page shape on the MXFP8 path: every row computed on the GPU (staged,
-    and the persistent kernel bit-identical to it), sampled tokens against
-    the emulated oracle."""
-    cfg = mokgen.CONFIGS["page_mxfp8"]
-    x = mokgen.tokens(cfg)
-    logits = mokgen.router_logits(cfg, x)
-    wg, wu, wd = mokgen.upload_expert_weights(cfg, "cuda")
-    pack = _mx_pack(wg, wu, wd)
-    del wg, wu, wd
-    torch.cuda.empty_cache()
-    p = mok.plan(logits.cuda(), cfg.k, cfg.R)
-    xs = mok.shards(x.cuda(), cfg.R)
-    ys, ws = mok.moe_forward_mxfp8(xs, pack, p)
-    assert mok.get_status(ws) == mok.MOK_OK
-    y = torch.cat([s.cpu() for s in ys]).double()
-    del ws
-    # the persistent kernel at the minibatch bench.py times computes the same bits
-    opts = mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT, mxfp8=True)
-    ys_p, ws_p = mok.moe_forward_mxfp8(xs, pack, p, minibatch=2560, opts=opts)
-    assert mok.get_status(ws_p) == mok.MOK_OK
-    assert torch.equal(torch.cat([s.cpu() for s in ys_p]).double(), y)
-    del ws_p
-    ids = sorted(set(torch.randperm(cfg.T, generator=torch.Generator().manual_seed(4))[:6].tolist()))
-    idx, g = oracle.topk_gates(logits[ids], cfg.k)
-    want = torch.zeros((len(ids), cfg.H), dtype=torch.float64)
-    for a in range(len(ids)):
-        for j in range(cfg.k):
-            e = int(idx[a, j])
-            o = oracle.mxfp8_expert_ffn(x[ids[a]:ids[a] + 1], *mokgen.expert_weights(cfg, e))
-            want[a] += float(g[a, j]) * o[0]
-    rel = (torch.linalg.norm(y[ids] - want) / torch.linalg.norm(want)).item()
-    assert rel <= REL_FRO_MX, rel
-
-
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
 def test_mxfp8_gather_bit_exact(name):
     """The fused quantising gather: row bytes and scale planes equal the
