@@ -40,7 +40,8 @@ EXPORTS = (
     "mok_expert_ffn", "mok_combine", "mok_forward_host_workspace_bytes", "mok_moe_forward_host",
     "mok_plan_noalloc", "mok_mxfp8_quantize_rows", "mok_quantize_weights_mxfp8",
     "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8_workspace_bytes", "mok_expert_ffn_mxfp8",
-    "mok_two_wave_rows", "mok_minibatch_bounds",
+    "mok_two_wave_rows", "mok_minibatch_bounds", "mok_forward_host_batches_workspace_bytes",
+    "mok_moe_forward_host_batches",
 )
 
 
@@ -98,12 +99,16 @@ def lib() -> ctypes.CDLL:
     L.mok_expert_ffn_mxfp8_workspace_bytes.restype = sz
     L.mok_expert_ffn_mxfp8.argtypes = [vp, vp, i32, i32, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
     L.mok_two_wave_rows.argtypes = [i32, i32, i32, i32]
+    L.mok_forward_host_batches_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(FwdOpts)]
+    L.mok_forward_host_batches_workspace_bytes.restype = sz
+    L.mok_moe_forward_host_batches.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32,
+                                               ctypes.POINTER(FwdOpts), vp, sz, vp]
     L.mok_minibatch_bounds.argtypes = [ctypes.POINTER(PlanT), i32, i32, vp, i32, ctypes.POINTER(FwdOpts), vp, sz,
                                        vp, vp, i32, ctypes.POINTER(ctypes.c_int), vp]
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
               "mok_moe_forward_host", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
               "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8",
-              "mok_two_wave_rows", "mok_minibatch_bounds"):
+              "mok_two_wave_rows", "mok_minibatch_bounds", "mok_moe_forward_host_batches"):
         getattr(L, n).restype = ctypes.c_int
     return L
 
@@ -389,6 +394,14 @@ def forward_host_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None 
     return lib().mok_forward_host_workspace_bytes(T, H, I, E, k, minibatch, ctypes.byref(opts) if opts else None)
 
 
+def _host_weights(w_gate, w_up, w_down):
+    if isinstance(w_gate, tuple):
+        qg, sg, qu, su, qd, sd = w_gate
+        mx = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
+        return qg.shape[-1], (ctypes.cast(ctypes.byref(mx), ctypes.c_void_p), None, None), mx
+    return w_gate.shape[-1], tuple(ctypes.c_void_p(w.data_ptr()) for w in (w_gate, w_up, w_down)), None
+
+
 def moe_forward_host(x_host: torch.Tensor, logits_host: torch.Tensor, top_k: int, R: int, w_gate, w_up, w_down,
                      minibatch: int, opts: FwdOpts | None, ws: torch.Tensor, y_host: torch.Tensor, stream=None):
     """End to end from host memory: ``mok_moe_forward_host``.  On the MXFP8
@@ -396,17 +409,35 @@ def moe_forward_host(x_host: torch.Tensor, logits_host: torch.Tensor, top_k: int
     (qg, sg, qu, su, qd, sd) and ``w_up``/``w_down`` are None."""
     T, H = x_host.shape
     E = logits_host.shape[1]
-    if isinstance(w_gate, tuple):
-        qg, sg, qu, su, qd, sd = w_gate
-        I = qg.shape[-1]
-        mx = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
-        wptrs = (ctypes.cast(ctypes.byref(mx), ctypes.c_void_p), None, None)
-    else:
-        I = w_gate.shape[-1]
-        wptrs = tuple(ctypes.c_void_p(w.data_ptr()) for w in (w_gate, w_up, w_down))
+    I, wptrs, keep = _host_weights(w_gate, w_up, w_down)
     _check(lib().mok_moe_forward_host(ctypes.c_void_p(x_host.data_ptr()), ctypes.c_void_p(logits_host.data_ptr()),
                                       T, H, I, E, top_k, R, *wptrs,
                                       minibatch, ctypes.byref(opts) if opts else None,
                                       ctypes.c_void_p(ws.data_ptr()), ws.numel(),
                                       ctypes.c_void_p(y_host.data_ptr()), _stream(stream)))
+    del keep
     return y_host
+
+
+def forward_host_batches_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None = None) -> int:
+    return lib().mok_forward_host_batches_workspace_bytes(T, H, I, E, k, minibatch,
+                                                          ctypes.byref(opts) if opts else None)
+
+
+def moe_forward_host_batches(xs_host, logits_host, top_k: int, R: int, w_gate, w_up, w_down, minibatch: int,
+                             opts: FwdOpts | None, ws: torch.Tensor, ys_host, stream=None):
+    """``mok_moe_forward_host_batches``: lists of n host tensors (x [T, H] bf16,
+    logits [T, E] fp32, y [T, H] bf16), copies overlapped with the compute."""
+    n = len(xs_host)
+    assert len(logits_host) == n and len(ys_host) == n
+    if n == 0:
+        return ys_host
+    T, H = xs_host[0].shape
+    E = logits_host[0].shape[1]
+    I, wptrs, keep = _host_weights(w_gate, w_up, w_down)
+    xa, la, ya = _ptr_array(xs_host), _ptr_array(logits_host), _ptr_array(ys_host)
+    _check(lib().mok_moe_forward_host_batches(n, xa, la, ya, T, H, I, E, top_k, R, *wptrs, minibatch,
+                                              ctypes.byref(opts) if opts else None, ctypes.c_void_p(ws.data_ptr()),
+                                              ws.numel(), _stream(stream)))
+    del keep
+    return ys_host

@@ -160,12 +160,17 @@ bool encode_bmaps_u8(BMaps* maps, const void* base, uint64_t inner, uint64_t row
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct FwdLayout {
-    size_t status, counts2, chunks, mbs, counters, rows, h, out, total;
+    size_t status, counts2, chunks, mbs, counters, counter_ints, rows, h, out, total;
     size_t xsc, hsc;  // MXFP8 path: token-side scale planes
     int max_chunks, max_mb, buf_rows, cap, minibatch, mode, mx;
 };
 
 static const uint64_t kDefaultTimeoutNs = 2000000000ull;
+// Dispatch CTAs of the persistent kernel by default: on the bf16 path one
+// thread per CTA streams rows with bulk copies (about 200 KB in flight), so
+// a few CTAs keep ahead of the GEMM; the MXFP8 path quantises with every
+// warp of its CTAs and needs more of them.
+static const int kDefaultDispatchBf16 = 4;
 
 static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* o, FwdLayout* L) {
     if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return false;
@@ -197,8 +202,10 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
     l.counts2 = take(sizeof(int) * 4);
     l.chunks = take(sizeof(Chunk) * (size_t)l.max_chunks);
     l.mbs = take(sizeof(Minibatch) * (size_t)l.max_mb);
-    // persistent-mode counters: gathered[max_mb], d_done[max_mb], g_done[max_chunks], d_total
-    l.counters = take(sizeof(int) * (2 * (size_t)l.max_mb + (size_t)l.max_chunks + 8));
+    // persistent-mode counters: chunk_ready, g_done, d_chunk [max_chunks],
+    // d_done [max_mb], tok_cnt, ready_q [T], q_tail, q_claim
+    l.counter_ints = 3 * (size_t)l.max_chunks + (size_t)l.max_mb + 2 * (size_t)T + 8;
+    l.counters = take(sizeof(int) * l.counter_ints);
     l.mx = (o && o->mxfp8) ? 1 : 0;
     if (l.mx) {
         // E4M3 rows and h, with their scale planes
@@ -393,7 +400,7 @@ static int setup_forward(int H, int I, const void* w_gate, const mok_plan_t* pla
     F->dispatch = 0;
     F->gemm = F->sms;
     if (mode == MOK_MODE_PERSISTENT) {
-        F->dispatch = (opts && opts->dispatch_ctas > 0) ? opts->dispatch_ctas : 16;
+        F->dispatch = (opts && opts->dispatch_ctas > 0) ? opts->dispatch_ctas : (F->mxw ? 16 : kDefaultDispatchBf16);
         F->gemm = (opts && opts->gemm_ctas > 0) ? opts->gemm_ctas : F->sms - F->dispatch;
         if (F->dispatch >= F->sms || F->gemm < 1 || F->dispatch + F->gemm > F->sms)
             return fail(MOK_ERR_INVALID_ARG, "dispatch_ctas + gemm_ctas must be at most the %d SMs", F->sms);
@@ -495,9 +502,7 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         int dev = 0;
         device_sms(&dev);
         int* counters = reinterpret_cast<int*>(base + L.counters);
-        MOK_CUDA(cudaMemsetAsync(counters, 0, sizeof(int) * (2 * (size_t)L.max_mb + (size_t)L.max_chunks + 8),
-                                 stream),
-                 "counter reset");
+        MOK_CUDA(cudaMemsetAsync(counters, 0, sizeof(int) * L.counter_ints, stream), "counter reset");
         PersistLaunch P{};
         P.grid = F.dispatch + F.gemm;
         P.dispatch_ctas = F.dispatch;
@@ -524,10 +529,14 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         P.chunks = F.chunks;
         P.mbs = F.mbs;
         P.counts2 = F.counts2;
-        P.gathered = counters;
-        P.d_done = counters + L.max_mb;
-        P.g_done = counters + 2 * L.max_mb;
-        P.d_total = counters + 2 * L.max_mb + L.max_chunks;
+        P.chunk_ready = counters;
+        P.g_done = counters + L.max_chunks;
+        P.d_chunk = counters + 2 * (size_t)L.max_chunks;
+        P.d_done = counters + 3 * (size_t)L.max_chunks;
+        P.tok_cnt = P.d_done + L.max_mb;
+        P.ready_q = P.tok_cnt + T;
+        P.q_tail = P.ready_q + T;
+        P.q_claim = P.q_tail + 1;
         P.xs = xs;
         P.ys = ys;
         P.src_rank = plan->sched_src_rank;
@@ -748,50 +757,200 @@ int mok_combine(const void* out, int out_dtype, int H, const mok_plan_t* plan, v
     return MOK_OK;
 }
 
-size_t mok_forward_host_workspace_bytes(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* opts) {
+}  // extern "C"
+
+namespace mok {
+
+// Host-buffer forward: nbuf sets of device staging buffers {x, y, logits}
+// (256-byte aligned), one plan workspace and one forward workspace.
+struct HostLayout {
+    size_t xb, lb, set_bytes, plan_bytes, plan_off, fwd_off, total;
+};
+
+static bool host_layout(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* opts, int nbuf,
+                        HostLayout* L) {
     const size_t p = mok_plan_workspace_bytes(T, E, k);
     const size_t f = mok_forward_workspace_bytes(T, H, I, E, k, minibatch, opts);
-    if (!p || !f) return 0;
-    return align256((size_t)T * H * 2) * 2 + align256((size_t)T * E * 4) + align256(p) + f;
+    if (!p || !f || T <= 0 || H <= 0) return false;
+    L->xb = (size_t)T * H * 2;
+    L->lb = (size_t)T * E * 4;
+    L->set_bytes = align256(L->xb) * 2 + align256(L->lb);
+    L->plan_bytes = align256(p);
+    L->plan_off = L->set_bytes * nbuf;
+    L->fwd_off = L->plan_off + L->plan_bytes;
+    L->total = L->fwd_off + f;
+    return true;
+}
+
+// Streams and events of the pipelined host forward, one set per device,
+// made on first use and kept for the process; `mu` serialises the calls
+// that use them.
+struct HostPipe {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t uploaded[2], computed[2], downloaded[2];
+};
+
+static int host_pipe(int dev, HostPipe** out) {
+    static HostPipe pipes[64];
+    static std::mutex init_mu;
+    if (dev < 0 || dev >= 64) return fail(MOK_ERR_CUDA, "device ordinal %d out of range", dev);
+    HostPipe& hp = pipes[dev];
+    std::lock_guard<std::mutex> g(init_mu);
+    if (!hp.ready) {
+        MOK_CUDA(cudaStreamCreateWithFlags(&hp.up, cudaStreamNonBlocking), "stream create");
+        MOK_CUDA(cudaStreamCreateWithFlags(&hp.down, cudaStreamNonBlocking), "stream create");
+        for (int b = 0; b < 2; ++b) {
+            MOK_CUDA(cudaEventCreateWithFlags(&hp.uploaded[b], cudaEventDisableTiming), "event create");
+            MOK_CUDA(cudaEventCreateWithFlags(&hp.computed[b], cudaEventDisableTiming), "event create");
+            MOK_CUDA(cudaEventCreateWithFlags(&hp.downloaded[b], cudaEventDisableTiming), "event create");
+        }
+        hp.ready = true;
+    }
+    *out = &hp;
+    return MOK_OK;
+}
+
+static int enqueue_host_batches(int n, const void* const* x_host, const float* const* logits_host,
+                                void* const* y_host, int T, int H, int I, int E, int top_k, int R,
+                                const void* w_gate, const void* w_up, const void* w_down, int minibatch,
+                                const mok_fwd_opts* opts, unsigned char* base, const HostLayout& L, int nbuf,
+                                HostPipe* hp, cudaStream_t stream, cudaStream_t up, cudaStream_t down) {
+    unsigned char* plan_ws = base + L.plan_off;
+    unsigned char* fwd_ws = base + L.fwd_off;
+    const size_t fwd_bytes = L.total - L.fwd_off;
+    const int S_r = T / R;
+    int rc = MOK_OK;
+    for (int i = 0; i < n; ++i) {
+        const int b = i % nbuf;
+        unsigned char* x_dev = base + (size_t)b * L.set_bytes;
+        unsigned char* y_dev = x_dev + align256(L.xb);
+        unsigned char* l_dev = y_dev + align256(L.xb);
+        if (hp) MOK_CUDA(cudaStreamWaitEvent(up, hp->computed[b], 0), "stream wait");
+        MOK_CUDA(cudaMemcpyAsync(l_dev, logits_host[i], L.lb, cudaMemcpyHostToDevice, up), "logits upload");
+        MOK_CUDA(cudaMemcpyAsync(x_dev, x_host[i], L.xb, cudaMemcpyHostToDevice, up), "x upload");
+        if (hp) {
+            MOK_CUDA(cudaEventRecord(hp->uploaded[b], up), "event record");
+            MOK_CUDA(cudaStreamWaitEvent(stream, hp->uploaded[b], 0), "stream wait");
+            MOK_CUDA(cudaStreamWaitEvent(stream, hp->downloaded[b], 0), "stream wait");
+        }
+        mok_plan_t plan;
+        if ((rc = mok_plan(reinterpret_cast<const float*>(l_dev), T, E, top_k, R, plan_ws, L.plan_bytes, &plan,
+                           reinterpret_cast<mok_stream_t>(stream))))
+            return rc;
+        const void* xs[MOK_MAX_SHARDS];
+        void* ys[MOK_MAX_SHARDS];
+        for (int r = 0; r < R; ++r) {
+            xs[r] = x_dev + (size_t)r * S_r * H * 2;
+            ys[r] = y_dev + (size_t)r * S_r * H * 2;
+        }
+        if ((rc = mok_moe_forward(xs, H, I, w_gate, w_up, w_down, &plan, minibatch, opts, fwd_ws, fwd_bytes, ys,
+                                  reinterpret_cast<mok_stream_t>(stream))))
+            return rc;
+        if (hp) {
+            MOK_CUDA(cudaEventRecord(hp->computed[b], stream), "event record");
+            MOK_CUDA(cudaStreamWaitEvent(down, hp->computed[b], 0), "stream wait");
+        }
+        MOK_CUDA(cudaMemcpyAsync(y_host[i], y_dev, L.xb, cudaMemcpyDeviceToHost, down), "y download");
+        if (hp) MOK_CUDA(cudaEventRecord(hp->downloaded[b], down), "event record");
+    }
+    if (hp) {
+        // `stream` ends after the last download
+        MOK_CUDA(cudaStreamWaitEvent(stream, hp->downloaded[(n - 1) % 2], 0), "stream wait");
+        MOK_CUDA(cudaStreamWaitEvent(stream, hp->downloaded[n % 2], 0), "stream wait");
+    }
+    return MOK_OK;
+}
+
+// n batches through plan + forward from host buffers.  Batch i uses staging
+// set i % nbuf.  With nbuf = 2, batch i+1's upload (stream `up`) and batch
+// i-1's download (stream `down`) run while batch i computes on `stream`:
+//   up:     wait computed[b] (batch i-2 is done with x[b], logits[b]);
+//           copy logits, x; record uploaded[b]
+//   stream: wait uploaded[b], downloaded[b] (batch i-2's y[b] has left);
+//           plan; forward; record computed[b]
+//   down:   wait computed[b]; copy y; record downloaded[b]
+// With nbuf = 1 everything runs on `stream` in order.
+static int forward_host_batches(int n, const void* const* x_host, const float* const* logits_host,
+                                void* const* y_host, int T, int H, int I, int E, int top_k, int R,
+                                const void* w_gate, const void* w_up, const void* w_down, int minibatch,
+                                const mok_fwd_opts* opts, void* ws, size_t ws_bytes, int nbuf,
+                                cudaStream_t stream) {
+    if (n < 0) return fail(MOK_ERR_INVALID_ARG, "n < 0");
+    if (n == 0) return MOK_OK;
+    if (!x_host || !logits_host || !y_host) return fail(MOK_ERR_INVALID_ARG, "NULL host pointer array");
+    for (int i = 0; i < n; ++i)
+        if (!x_host[i] || !logits_host[i] || !y_host[i]) return fail(MOK_ERR_INVALID_ARG, "NULL host pointer");
+    if (T <= 0 || R <= 0 || R > MOK_MAX_SHARDS || T % R) return fail(MOK_ERR_INVALID_ARG, "T, R invalid");
+    HostLayout L;
+    if (!host_layout(T, H, I, E, top_k, minibatch, opts, nbuf, &L)) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
+    int rc = check_ws(ws, ws_bytes, L.total);
+    if (rc) return rc;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    HostPipe* hp = nullptr;
+    std::unique_lock<std::mutex> lock;
+    if (nbuf == 2) {
+        int dev = 0;
+        MOK_CUDA(cudaGetDevice(&dev), "get device");
+        if ((rc = host_pipe(dev, &hp))) return rc;
+        lock = std::unique_lock<std::mutex>(hp->mu);
+        // the copy streams start after the work already queued on `stream`
+        MOK_CUDA(cudaEventRecord(hp->computed[0], stream), "event record");
+        MOK_CUDA(cudaStreamWaitEvent(hp->up, hp->computed[0], 0), "stream wait");
+        MOK_CUDA(cudaStreamWaitEvent(hp->down, hp->computed[0], 0), "stream wait");
+        MOK_CUDA(cudaEventRecord(hp->computed[1], stream), "event record");
+        MOK_CUDA(cudaEventRecord(hp->downloaded[0], stream), "event record");
+        MOK_CUDA(cudaEventRecord(hp->downloaded[1], stream), "event record");
+    }
+    cudaStream_t up = hp ? hp->up : stream, down = hp ? hp->down : stream;
+    rc = enqueue_host_batches(n, x_host, logits_host, y_host, T, H, I, E, top_k, R, w_gate, w_up, w_down, minibatch,
+                              opts, base, L, nbuf, hp, stream, up, down);
+    if (rc != MOK_OK) {
+        // leave no copy in flight on the caller's host buffers
+        if (hp) {
+            cudaStreamSynchronize(up);
+            cudaStreamSynchronize(down);
+        }
+        cudaStreamSynchronize(stream);
+        return rc;
+    }
+    MOK_CUDA(cudaStreamSynchronize(stream), "stream synchronize");
+    return MOK_OK;
+}
+
+}  // namespace mok
+
+extern "C" {
+
+size_t mok_forward_host_workspace_bytes(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* opts) {
+    HostLayout L;
+    return host_layout(T, H, I, E, k, minibatch, opts, 1, &L) ? L.total : 0;
 }
 
 int mok_moe_forward_host(const void* x_host, const float* logits_host, int T, int H, int I, int E, int top_k, int R,
                          const void* w_gate, const void* w_up, const void* w_down, int minibatch,
-                         const mok_fwd_opts* opts, void* ws, size_t ws_bytes, void* y_host, mok_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+                         const mok_fwd_opts* opts, void* ws, size_t ws_bytes, void* y_host, mok_stream_t stream) {
     if (!x_host || !logits_host || !y_host) return fail(MOK_ERR_INVALID_ARG, "NULL host pointer");
-    if (T <= 0 || R <= 0 || R > MOK_MAX_SHARDS || T % R) return fail(MOK_ERR_INVALID_ARG, "T, R invalid");
-    const size_t need = mok_forward_host_workspace_bytes(T, H, I, E, top_k, minibatch, opts);
-    if (!need) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
-    int rc = check_ws(ws, ws_bytes, need);
-    if (rc) return rc;
-    unsigned char* base = static_cast<unsigned char*>(ws);
-    const size_t xb = (size_t)T * H * 2, lb = (size_t)T * E * 4;
-    unsigned char* x_dev = base;
-    unsigned char* y_dev = x_dev + align256(xb);
-    unsigned char* l_dev = y_dev + align256(xb);
-    unsigned char* plan_ws = l_dev + align256(lb);
-    const size_t plan_bytes = align256(mok_plan_workspace_bytes(T, E, top_k));
-    unsigned char* fwd_ws = plan_ws + plan_bytes;
-    const size_t fwd_bytes = ws_bytes - (size_t)(fwd_ws - base);
-    MOK_CUDA(cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream), "x upload");
-    MOK_CUDA(cudaMemcpyAsync(l_dev, logits_host, lb, cudaMemcpyHostToDevice, stream), "logits upload");
-    mok_plan_t plan;
-    if ((rc = mok_plan(reinterpret_cast<const float*>(l_dev), T, E, top_k, R, plan_ws, plan_bytes, &plan, stream_)))
-        return rc;
-    const void* xs[MOK_MAX_SHARDS];
-    void* ys[MOK_MAX_SHARDS];
-    const int S_r = T / R;
-    for (int r = 0; r < R; ++r) {
-        xs[r] = x_dev + (size_t)r * S_r * H * 2;
-        ys[r] = y_dev + (size_t)r * S_r * H * 2;
-    }
-    if ((rc = mok_moe_forward(xs, H, I, w_gate, w_up, w_down, &plan, minibatch, opts, fwd_ws, fwd_bytes, ys,
-                              stream_)))
-        return rc;
-    MOK_CUDA(cudaMemcpyAsync(y_host, y_dev, xb, cudaMemcpyDeviceToHost, stream), "y download");
-    MOK_CUDA(cudaStreamSynchronize(stream), "stream synchronize");
-    return MOK_OK;
+    const void* xh[1] = {x_host};
+    const float* lh[1] = {logits_host};
+    void* yh[1] = {y_host};
+    return forward_host_batches(1, xh, lh, yh, T, H, I, E, top_k, R, w_gate, w_up, w_down, minibatch, opts, ws,
+                                ws_bytes, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t mok_forward_host_batches_workspace_bytes(int T, int H, int I, int E, int k, int minibatch,
+                                                const mok_fwd_opts* opts) {
+    HostLayout L;
+    return host_layout(T, H, I, E, k, minibatch, opts, 2, &L) ? L.total : 0;
+}
+
+int mok_moe_forward_host_batches(int n, const void* const* x_host, const float* const* logits_host,
+                                 void* const* y_host, int T, int H, int I, int E, int top_k, int R,
+                                 const void* w_gate, const void* w_up, const void* w_down, int minibatch,
+                                 const mok_fwd_opts* opts, void* ws, size_t ws_bytes, mok_stream_t stream) {
+    return forward_host_batches(n, x_host, logits_host, y_host, T, H, I, E, top_k, R, w_gate, w_up, w_down, minibatch,
+                                opts, ws, ws_bytes, 2, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -181,7 +181,8 @@ struct StagedSched {
         return true;
     }
     __device__ bool wait_inputs(const Unit&, DevStatus*, uint64_t) const { return true; }
-    __device__ void unit_done(const Unit&) const {}
+    __device__ bool unit_done(const Unit&) const { return false; }
+    __device__ void chunk_done(const Unit&, int, int) const {}
 };
 
 // M tiles of a phase (64 gate + 64 up features, or 128 down features, each),
@@ -602,17 +603,25 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
             // group's stores visible to that proxy; the group that finishes
             // the unit second publishes it once.  The groups are at most one
             // unit apart (a buffer is reused only after both released it), so
-            // two counters, by unit parity, pair their arrivals.
+            // two counters, by unit parity, pair their arrivals.  When that
+            // publication completes a chunk's down units, the whole group
+            // passes the chunk's rows on (s.chunk_done).
             fence_proxy_async_global();
             __threadfence();
             named_bar_sync(bar, 128);
             if (et == 0) {
                 __threadfence();
+                int fin = 0;
                 if (atomicAdd(done_cnt + (i & 1), 1) & 1) {
                     __threadfence();
-                    s.unit_done(u);
+                    fin = s.unit_done(u) ? 1 : 0;
                 }
+                *ok_flag = fin;
             }
+            named_bar_sync(bar, 128);
+            const bool fin = *ok_flag != 0;
+            named_bar_sync(bar, 128);  // ok_flag is written again at the next unit
+            if (fin) s.chunk_done(u, et, 128);
         }
     }
 }

@@ -156,7 +156,9 @@ struct PersistLaunch {
     const Chunk* chunks;
     const Minibatch* mbs;
     const int* counts2;
-    int *gathered, *d_done, *g_done, *d_total;  // zeroed counters
+    // zeroed counters: chunk_ready, g_done, d_chunk [max_chunks]; d_done
+    // [max_mb]; tok_cnt, ready_q [T]; q_tail, q_claim [1]
+    int *chunk_ready, *g_done, *d_chunk, *d_done, *tok_cnt, *ready_q, *q_tail, *q_claim;
     ShardsIn xs;
     ShardsOut ys;
     const int32_t *src_rank, *src_index, *row_slot;

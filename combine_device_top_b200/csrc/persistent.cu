@@ -12,28 +12,38 @@
 // points (SM split, local counters).
 //
 // One launch (cooperative, so every CTA is resident), one CTA per SM:
-//   CTAs [0, D)  dispatch/combine side: for each minibatch b, wait until ring
-//                half b % 2 is free (all down units of minibatch b - 2 done),
-//                gather b's rows into it (MXFP8 path: quantised to E4M3 rows
-//                plus the ring's scale planes), publish gathered[b].
+//   CTAs [0, D)  dispatch side: for each minibatch b, wait until ring half
+//                b % 2 is free (all down units of minibatch b - 2 done), then
+//                copy b's chunks into it, chunks dealt round-robin to the D
+//                CTAs (MXFP8 path: quantised to E4M3 rows plus the ring's
+//                scale planes), publishing chunk_ready[c] after each chunk.
 //   CTAs [D, G)  GEMM side: the tcgen05 core of gemm_core.cuh over the units
 //                of every minibatch in order -- gate/up units of b, then its
 //                down units -- dealt round-robin.  A gate/up unit waits for
-//                gathered[b] == D; a down unit waits for its chunk's gate/up
-//                units (g_done[c] == their count); completions are published with
-//                release atomics.
-//   all CTAs     after every down unit is done: the fixed-order combine.
+//                its chunk's rows (chunk_ready[c]); a down unit waits for its
+//                chunk's gate/up units (g_done[c] == their count).  When the
+//                last down unit of a chunk is published, its epilogue group
+//                counts each of the chunk's rows into its token (tok_cnt);
+//                a token whose k slots are complete is appended to ready_q.
+//   all CTAs     once their own role is done, combine tokens from ready_q in
+//                queue order (a warp per token): the combine of early
+//                tokens overlaps the GEMM of later experts (macrobatch
+//                overlap), and the rest runs on every SM at the end.
 // Dependencies only point to lower unit indices (or to the dispatch side,
-// which waits only on lower indices), so the lowest unfinished unit can
-// always proceed: no deadlock without any host involvement.  Every wait is
-// bounded; a wait that gives up records MOK_ERR_TIMEOUT and the kernel
-// leaves its loops.
+// which waits only on lower indices), and the combine waits only on the GEMM
+// side, so the lowest unfinished unit can always proceed: no deadlock
+// without any host involvement.  Every wait is bounded; a wait that gives up
+// records MOK_ERR_TIMEOUT and the kernel leaves its loops.
 //
 // Memory ordering: rows and h (and, MXFP8, their scale planes) are written
-// with generic stores and read by TMA or bulk copies (async proxy) in other
-// CTAs.  Writers fence.proxy.async + threadfence,
-// then one thread does a release add; readers do an acquire load, then
-// fence.proxy.async, then issue TMA.
+// with generic stores or bulk copies and read by TMA or bulk copies (async
+// proxy) in other CTAs.  Writers fence.proxy.async + threadfence, then one
+// thread does a release add; readers do an acquire load, then
+// fence.proxy.async, then issue TMA.  Slot outputs reach the combine through
+// a chain of release/acquire atomics: each down unit's publication (release),
+// the chunk's completing acquire-release add, the token counter's
+// acquire-release add, the queue entry's release store and the combining
+// warp's acquire load.
 #include <cstring>
 
 #include "dispatch_combine.cuh"
@@ -50,16 +60,21 @@ struct PersistParams {
     int MTG, MTD;        // units (groups of C::SUB M tiles) per chunk of the gate/up and down phases
     int dispatch_ctas;
     // counters (zeroed before the launch)
-    int* gathered;  // [max_mb]  dispatch CTAs done with minibatch b
-    int* d_done;    // [max_mb]  down units done in minibatch b
-    int* g_done;    // [max_chunks] gate/up units done for chunk c
-    int* d_total;   // [1]       down units done overall
+    int* chunk_ready;  // [max_chunks] 1 once the chunk's rows are in the ring
+    int* g_done;       // [max_chunks] gate/up units done for chunk c
+    int* d_chunk;      // [max_chunks] down units done for chunk c
+    int* d_done;       // [max_mb]     down units done in minibatch b (ring half reuse)
+    int* tok_cnt;      // [T] slots of token t whose outputs are complete
+    int* ready_q;      // [T] 1 + token, in the order tokens became complete (0: not yet)
+    int* q_tail;       // tokens appended to ready_q
+    int* q_claim;      // queue positions claimed by combining warps
     // token data
     ShardsIn xs;
     ShardsOut ys;
     int S_r, T, k;
     const int32_t* src_rank;
     const int32_t* src_index;
+    const int32_t* row_slot;
     const float* gates;
     void* ring;        // [2 * cap, H] bf16, or E4M3 bytes (MXFP8 path)
     uint8_t* ring_sc;  // MXFP8 path: the ring rows' scale planes [H/128][sc_rows][4]
@@ -106,18 +121,33 @@ struct PersistSched {
     }
 
     __device__ bool wait_inputs(const Unit& u, DevStatus* st, uint64_t timeout_ns) const {
-        const bool ok = u.phase == 0 ? flag_wait_geq(&p->gathered[u.mb], p->dispatch_ctas, st, timeout_ns, 40)
+        const bool ok = u.phase == 0 ? flag_wait_geq(&p->chunk_ready[u.chunk], 1, st, timeout_ns, 40)
                                      : flag_wait_geq(&p->g_done[u.chunk], p->MTG, st, timeout_ns, 41);
         fence_proxy_async_global();
         return ok;
     }
 
-    __device__ void unit_done(const Unit& u) const {
+    // Publishes a finished unit; true when it was the last down unit of its chunk.
+    __device__ bool unit_done(const Unit& u) const {
         if (u.phase == 0) {
             red_release_gpu_add(&p->g_done[u.chunk], 1);
-        } else {
-            red_release_gpu_add(&p->d_done[u.mb], 1);
-            red_release_gpu_add(p->d_total, 1);
+            return false;
+        }
+        red_release_gpu_add(&p->d_done[u.mb], 1);
+        return atom_acq_rel_gpu_add(&p->d_chunk[u.chunk], 1) == p->MTD - 1;
+    }
+
+    // Every output of the chunk's rows is stored: count each row into its
+    // token; a token whose k slots are all counted joins the combine queue.
+    // Called by the n threads of one epilogue group (thread `tid`).
+    __device__ void chunk_done(const Unit& u, int tid, int n) const {
+        __threadfence();
+        for (int r = tid; r < u.rows; r += n) {
+            const int t = __ldg(p->row_slot + u.grow0 + r) / p->k;
+            if (atom_acq_rel_gpu_add(&p->tok_cnt[t], 1) == p->k - 1) {
+                const int at = atomicAdd(p->q_tail, 1);
+                st_release_gpu(&p->ready_q[at], t + 1);
+            }
         }
     }
 };
@@ -153,80 +183,82 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         __syncthreads();
         uint32_t loads = 0;
-        for (int b = 0; b < nmb; ++b) {
+        bool ok = true;
+        for (int b = 0; b < nmb && ok; ++b) {
             if (threadIdx.x == 0) {
-                bool ok = !failed(a.st);
-                if (ok && b >= 2) {  // ring half b % 2 is free once minibatch b - 2 is fully consumed
+                bool w = !failed(a.st);
+                if (w && b >= 2) {  // ring half b % 2 is free once minibatch b - 2 is fully consumed
                     const Minibatch old = p.mbs[b - 2];
-                    ok = flag_wait_geq(&p.d_done[b - 2], (old.chunk1 - old.chunk0) * p.MTD, a.st, a.timeout_ns, 50);
+                    w = flag_wait_geq(&p.d_done[b - 2], (old.chunk1 - old.chunk0) * p.MTD, a.st, a.timeout_ns, 50);
                 }
-                s_ok = ok ? 1 : 0;
+                s_ok = w ? 1 : 0;
             }
             __syncthreads();
-            const int ok = s_ok;
+            ok = s_ok != 0;
             __syncthreads();
             if (!ok) break;
             const Minibatch mb = p.mbs[b];
-            const int n = mb.row1 - mb.row0;
-            const int r0 = mb.row0 + (int)((long long)n * blockIdx.x / D);
-            const int r1 = mb.row0 + (int)((long long)n * (blockIdx.x + 1) / D);
             uint4* half = reinterpret_cast<uint4*>(p.ring) + (size_t)((b & 1) * p.cap) * nvec;
-            if constexpr (C::MX) {
-                // E4M3 row at ring row brow, its H/32 block scales in the planes;
-                // four 256-element steps' loads in flight per lane
-                uint32_t* planes = reinterpret_cast<uint32_t*>(p.ring_sc);
-                for (int r = r0 + warp; r < r1; r += C::THREADS / 32) {
-                    const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
-                    const uint4* src = reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec;
-                    const int brow = (b & 1) * p.cap + (r - mb.row0);
-                    uint8_t* dst = reinterpret_cast<uint8_t*>(p.ring) + (size_t)brow * a.H;
-                    for (int c0 = 0; c0 < a.H; c0 += 1024) {
-                        uint4 raw[4];
+            for (int c = mb.chunk0 + (int)blockIdx.x; c < mb.chunk1; c += D) {
+                const Chunk ck = p.chunks[c];
+                const int r0 = ck.row0, r1 = ck.row0 + ck.rows;
+                if constexpr (C::MX) {
+                    // E4M3 row at ring row brow, its H/32 block scales in the planes;
+                    // four 256-element steps' loads in flight per lane
+                    uint32_t* planes = reinterpret_cast<uint32_t*>(p.ring_sc);
+                    for (int r = r0 + warp; r < r1; r += C::THREADS / 32) {
+                        const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
+                        const uint4* src = reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec;
+                        const int brow = (b & 1) * p.cap + (r - mb.row0);
+                        uint8_t* dst = reinterpret_cast<uint8_t*>(p.ring) + (size_t)brow * a.H;
+                        for (int c0 = 0; c0 < a.H; c0 += 1024) {
+                            uint4 raw[4];
 #pragma unroll
-                        for (int s4 = 0; s4 < 4; ++s4) {
-                            const int c = c0 + 256 * s4 + lane * 8;
-                            raw[s4] = c < a.H ? __ldg(src + (c >> 3)) : make_uint4(0, 0, 0, 0);
-                        }
+                            for (int s4 = 0; s4 < 4; ++s4) {
+                                const int cc = c0 + 256 * s4 + lane * 8;
+                                raw[s4] = cc < a.H ? __ldg(src + (cc >> 3)) : make_uint4(0, 0, 0, 0);
+                            }
 #pragma unroll
-                        for (int s4 = 0; s4 < 4; ++s4) {
-                            const int cs = c0 + 256 * s4;
-                            if (cs < a.H) {  // warp-uniform
-                                uint2 q;
-                                uint32_t word;
-                                warp_mx_quant8(raw[s4], q, word, lane);
-                                const int c = cs + lane * 8;
-                                if (c < a.H) {
-                                    *reinterpret_cast<uint2*>(dst + c) = q;
-                                    if ((lane & 15) == 0)
-                                        planes[(size_t)((cs >> 7) + (lane >> 4)) * a.sc_rows + brow] = word;
+                            for (int s4 = 0; s4 < 4; ++s4) {
+                                const int cs = c0 + 256 * s4;
+                                if (cs < a.H) {  // warp-uniform
+                                    uint2 q;
+                                    uint32_t word;
+                                    warp_mx_quant8(raw[s4], q, word, lane);
+                                    const int cc = cs + lane * 8;
+                                    if (cc < a.H) {
+                                        *reinterpret_cast<uint2*>(dst + cc) = q;
+                                        if ((lane & 15) == 0)
+                                            planes[(size_t)((cs >> 7) + (lane >> 4)) * a.sc_rows + brow] = word;
+                                    }
                                 }
                             }
                         }
                     }
+                } else if (bulk) {
+                    if (threadIdx.x == 0) {
+                        auto src = [&](int i) -> const void* {
+                            const int r = r0 + i;
+                            return reinterpret_cast<const uint4*>(p.xs.p[__ldg(p.src_rank + r)]) +
+                                   (size_t)__ldg(p.src_index + r) * nvec;
+                        };
+                        auto dst = [&](int i) -> void* { return half + (size_t)(r0 + i - mb.row0) * nvec; };
+                        bulk_stream_rows(r1 - r0, src, dst, row_bytes, smem, slot_full, S, loads, a.st, a.timeout_ns,
+                                         DRAIN_TIMEOUT_NS);
+                    }
+                } else {
+                    for (int r = r0 + warp; r < r1; r += C::THREADS / 32) {
+                        const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
+                        warp_copy_row(reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec,
+                                      half + (size_t)(r - mb.row0) * nvec, nvec, lane);
+                    }
                 }
-            } else if (bulk) {
-                if (threadIdx.x == 0) {
-                    auto src = [&](int i) -> const void* {
-                        const int r = r0 + i;
-                        return reinterpret_cast<const uint4*>(p.xs.p[__ldg(p.src_rank + r)]) +
-                               (size_t)__ldg(p.src_index + r) * nvec;
-                    };
-                    auto dst = [&](int i) -> void* { return half + (size_t)(r0 + i - mb.row0) * nvec; };
-                    bulk_stream_rows(r1 - r0, src, dst, row_bytes, smem, slot_full, S, loads, a.st, a.timeout_ns,
-                                     DRAIN_TIMEOUT_NS);
-                }
-            } else {
-                for (int r = r0 + warp; r < r1; r += C::THREADS / 32) {
-                    const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
-                    warp_copy_row(reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec,
-                                  half + (size_t)(r - mb.row0) * nvec, nvec, lane);
-                }
+                // the rows are read next by TMA in the GEMM CTAs
+                fence_proxy_async_global();
+                __threadfence();
+                __syncthreads();
+                if (threadIdx.x == 0 && !failed(a.st)) red_release_gpu_add(&p.chunk_ready[c], 1);
             }
-            // the rows are read next by TMA in the GEMM CTAs
-            fence_proxy_async_global();
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0 && !failed(a.st)) red_release_gpu_add(&p.gathered[b], 1);
         }
     } else {
         // ---------------------------------------- GEMM side
@@ -240,13 +272,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         gemm_cta<PersistSched, C>(maps, &mx, a, s, smem);
     }
 
-    // -------------------------------------------- combine, once every down unit is done
-    if (threadIdx.x == 0)
-        s_ok = (!failed(a.st) && flag_wait_geq(p.d_total, nch * p.MTD, a.st, a.timeout_ns, 60)) ? 1 : 0;
-    __syncthreads();
-    if (!s_ok) return;
-    const int warps = gridDim.x * (C::THREADS / 32);
-    for (int t = blockIdx.x * (C::THREADS / 32) + warp; t < p.T; t += warps) {
+    // -------------------------------------------- combine tokens as they complete
+    // A warp claims the next queue position and waits (bounded) for the
+    // token that completes there; the fixed-order sum itself is the staged
+    // combine's, so y does not depend on which warp combines a token or when.
+    while (true) {
+        int at = 0;
+        if (lane == 0) at = atomicAdd(p.q_claim, 1);
+        at = __shfl_sync(0xffffffffu, at, 0);
+        if (at >= p.T) break;
+        // lane 0 waits; the warp leaves or goes on as one
+        int ready = 0;
+        if (lane == 0) ready = flag_wait_geq(&p.ready_q[at], 1, a.st, a.timeout_ns, 60) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, ready, 0) == 0) break;
+        // every lane acquires the entry, so its loads of the slot rows come after it
+        const int t = ld_acquire_gpu(&p.ready_q[at]) - 1;
         const int r = t / p.S_r;
         uint4* dst = reinterpret_cast<uint4*>(p.ys.p[r]) + (size_t)(t - r * p.S_r) * nvec;
         if constexpr (C::MX)
@@ -322,10 +362,14 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.MTG = (L.I / MT_G_FEATURES + sub - 1) / sub;
     p.MTD = (L.H / MT_D_FEATURES + sub - 1) / sub;
     p.dispatch_ctas = L.dispatch_ctas;
-    p.gathered = L.gathered;
-    p.d_done = L.d_done;
+    p.chunk_ready = L.chunk_ready;
     p.g_done = L.g_done;
-    p.d_total = L.d_total;
+    p.d_chunk = L.d_chunk;
+    p.d_done = L.d_done;
+    p.tok_cnt = L.tok_cnt;
+    p.ready_q = L.ready_q;
+    p.q_tail = L.q_tail;
+    p.q_claim = L.q_claim;
     p.xs = L.xs;
     p.ys = L.ys;
     p.S_r = L.S_r;
@@ -333,6 +377,7 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.k = L.k;
     p.src_rank = L.src_rank;
     p.src_index = L.src_index;
+    p.row_slot = L.row_slot;
     p.gates = L.gates;
     p.ring = L.ring;
     p.ring_sc = L.ring_sc;

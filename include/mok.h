@@ -24,7 +24,7 @@
  *    256-byte aligned.
  *  - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
  *    is the legacy default stream).  No call synchronises the host except
- *    mok_get_status() and mok_moe_forward_host().
+ *    mok_get_status(), mok_minibatch_bounds() and the *_host() calls.
  *  - Inputs are never modified.
  *  - Return value: MOK_OK or a MOK_ERR_* code; mok_last_error_string()
  *    gives a message for the calling thread's last failure.  Argument and
@@ -163,8 +163,10 @@ typedef struct mok_fwd_opts {
     int32_t mode;          /* MOK_MODE_*                                        */
     int32_t ring_slots;    /* rows of the ring token buffer (persistent mode);  */
                            /* 0 = 2 * max(minibatch, 4096) rows                 */
-    int32_t dispatch_ctas; /* CTAs doing gather/combine in persistent mode;     */
-                           /* 0 = default (16)                                  */
+    int32_t dispatch_ctas; /* CTAs doing the dispatch in persistent mode;       */
+                           /* 0 = default (4 bf16: bulk copies; 16 MXFP8:      */
+                           /* quantising warps).  Every CTA combines once its  */
+                           /* own role is done                                 */
     int32_t gemm_ctas;     /* GEMM CTAs; 0 = all remaining SMs                  */
     int32_t mxfp8;         /* 1 = MXFP8 path (weights from                      */
                            /* mok_quantize_weights_mxfp8; either mode);         */
@@ -377,6 +379,33 @@ int mok_moe_forward_host(const void* x_host, const float* logits_host,
                          const void* w_gate, const void* w_up, const void* w_down,
                          int minibatch, const mok_fwd_opts* opts,
                          void* ws, size_t ws_bytes, void* y_host, mok_stream_t stream);
+
+/* Bytes of workspace for mok_moe_forward_host_batches: two sets of device
+ * staging buffers (x, y, logits), one plan and one forward workspace. */
+size_t mok_forward_host_batches_workspace_bytes(int T, int H, int I, int E, int k, int minibatch,
+                                                const mok_fwd_opts* opts);
+
+/*
+ * mok_moe_forward_host_batches -- n batches of T tokens through the layer
+ * from HOST buffers, with the copies overlapped with the compute: batch i
+ * uses device staging set i % 2, and while batch i computes on `stream`,
+ * batch i+1's x and logits are uploaded and batch i-1's y is downloaded on
+ * two other streams (one per copy direction).  x_host[i] [T, H] bf16,
+ * logits_host[i] [T, E] fp32 and y_host[i] [T, H] bf16 are HOST arrays of
+ * n pointers; pinned memory gives the overlap (pageable copies serialise).
+ * Batch i's y_host[i] may be the same buffer as another batch's.  The
+ * results equal n calls of mok_moe_forward_host, bit for bit.  Returns
+ * after every copy has finished (synchronises `stream`); on an error, no
+ * copy is left in flight.  The two copy streams and their events are made
+ * on a device's first call and kept until the process exits; calls on one
+ * device run one at a time (a mutex).  (This serves the pages' data path
+ * from host memory; the pages have no counterpart of the call itself.)
+ */
+int mok_moe_forward_host_batches(int n, const void* const* x_host, const float* const* logits_host,
+                                 void* const* y_host, int T, int H, int I, int E, int top_k, int R,
+                                 const void* w_gate, const void* w_up, const void* w_down,
+                                 int minibatch, const mok_fwd_opts* opts,
+                                 void* ws, size_t ws_bytes, mok_stream_t stream);
 
 #ifdef __cplusplus
 }

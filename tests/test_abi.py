@@ -224,3 +224,20 @@ def test_two_wave_rows_reproduces_the_pages_minibatch():
     assert L.mok_two_wave_rows(14336, 148, 256, 128) == 339         # rounded up
     assert L.mok_two_wave_rows(0, 148, 128, 256) == 0
     assert L.mok_two_wave_rows(2048, -1, 128, 256) == 0
+
+
+def test_host_batches_reject_null_host_pointers_before_any_copy():
+    L = mok.lib()
+    opts = mok.fwd_opts(mode=mok.MOK_MODE_STAGED)
+    need = L.mok_forward_host_batches_workspace_bytes(64, 128, 128, 8, 2, 64, ctypes.byref(opts))
+    assert need > L.mok_forward_host_workspace_bytes(64, 128, 128, 8, 2, 64, ctypes.byref(opts)) > 0
+    arr = (ctypes.c_void_p * 2)(4096, None)
+    good = (ctypes.c_void_p * 2)(4096, 8192)
+    rc = L.mok_moe_forward_host_batches(2, good, arr, good, 64, 128, 128, 8, 2, 2, 1, 1, 1, 64, ctypes.byref(opts),
+                                        4096, need, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG and "NULL" in mok.last_error()
+    assert L.mok_moe_forward_host_batches(0, None, None, None, 64, 128, 128, 8, 2, 2, 1, 1, 1, 64, None, None, 0,
+                                          None) == mok.MOK_OK
+    rc = L.mok_moe_forward_host_batches(2, good, good, good, 63, 128, 128, 8, 2, 2, 1, 1, 1, 64, ctypes.byref(opts),
+                                        4096, need, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG

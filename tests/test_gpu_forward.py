@@ -156,6 +156,36 @@ def test_forward_host_entry_matches_device_entry():
     assert torch.equal(y_host, torch.cat([s.cpu() for s in ys]))
 
 
+@pytest.mark.parametrize("mode", [STAGED, mok.MOK_MODE_PERSISTENT])
+def test_forward_host_batches_equal_single_host_calls(mode):
+    """Four different batches through the overlapped host pipeline (two
+    staging sets, copies on their own streams) give the bits of four
+    separate mok_moe_forward_host calls."""
+    case = Case(FFN_CASES["multi_chunk"])
+    cfg = case.cfg
+    opts = mok.fwd_opts(mode=mode)
+    xs = [(case.x.float() * (1.0 + 0.25 * i)).to(torch.bfloat16).pin_memory() for i in range(4)]
+    ls = [(case.logits + 0.5 * i * torch.roll(case.logits, i, 1)).contiguous().pin_memory() for i in range(4)]
+    ws1 = torch.empty(mok.forward_host_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, 64, opts),
+                      dtype=torch.uint8, device="cuda")
+    want = []
+    for i in range(4):
+        y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+        mok.moe_forward_host(xs[i], ls[i], cfg.k, cfg.R, case.dwg, case.dwu, case.dwd, 64, opts, ws1, y)
+        want.append(y.clone())
+    wsb = torch.empty(mok.forward_host_batches_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, 64, opts),
+                      dtype=torch.uint8, device="cuda")
+    ys = [torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    mok.moe_forward_host_batches(xs, ls, cfg.k, cfg.R, case.dwg, case.dwu, case.dwd, 64, opts, wsb, ys)
+    for i in range(4):
+        assert torch.equal(ys[i], want[i]), i
+    # again on the same workspace, every batch written to one shared buffer: the last batch wins
+    shared = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    mok.moe_forward_host_batches(xs[::-1], ls[::-1], cfg.k, cfg.R, case.dwg, case.dwu, case.dwd, 64, opts, wsb,
+                                 [shared] * 4)
+    assert torch.equal(shared, want[0])
+
+
 def _forward_staged(case: Case, logits=None):
     cfg = case.cfg
     dlogits = case.dlogits if logits is None else logits.cuda()

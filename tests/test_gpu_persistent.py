@@ -103,9 +103,9 @@ def test_minibatches_hold_two_waves_of_gemm_units(name, minibatch):
     x = mokgen.tokens(cfg)
     logits = mokgen.router_logits(cfg, x)
     p = mok.plan(logits.cuda(), cfg.k, cfg.R)
-    opts = mok.fwd_opts(mode=PERSIST, ring_slots=cfg.ring_slots)
+    opts = mok.fwd_opts(mode=PERSIST, ring_slots=cfg.ring_slots, dispatch_ctas=8)
     row0, units = mok.minibatch_bounds(p, cfg.H, cfg.I, minibatch, opts)
-    gemm_ctas = torch.cuda.get_device_properties(0).multi_processor_count - 16
+    gemm_ctas = torch.cuda.get_device_properties(0).multi_processor_count - 8
     ns, cap = cfg.slots, cfg.ring_slots // 2
     bounds = row0 + [ns]
     offsets = set(p.offsets().cpu().tolist())
