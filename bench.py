@@ -396,6 +396,39 @@ def time_e2e(wl: Workload, mode: str, steps: int, minibatch: int, world: int):
             "d2h": cfg.T * cfg.H * 2, "e2e_steps": n}
 
 
+def time_router(wl: Workload, steps: int, warmup: int):
+    """mok_plan_router on the workload's tokens: the router projection on the
+    tensor cores fused with the top-k, plus the schedule kernels.  Inputs
+    (x, the split router weights) resident in HBM; CUDA events on the
+    launching stream."""
+    import combine_device_top_b200 as mok
+
+    cfg, device = wl.cfg, wl.device
+    w = mokgen.router_weight(cfg).to(device)
+    prior = mokgen.zipf_log_prior(cfg.E, cfg.zipf_s).to(device) if cfg.zipf_s else None
+    hi, lo = mok.router_prepare(w)
+    ws = torch.empty(mok.lib().mok_plan_workspace_bytes(cfg.T, cfg.E, cfg.k), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        mok.plan_router(wl.x_shards, hi, lo, cfg.E, cfg.k, prior, ws=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        mok.plan_router(wl.x_shards, hi, lo, cfg.E, cfg.k, prior, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if mok.get_status(ws) != mok.MOK_OK:
+        raise RuntimeError("router status " + mok.last_error())
+    ms = e0.elapsed_time(e1) / steps
+    flops = 2.0 * cfg.T * cfg.H * cfg.E            # useful: one projection
+    return {"workload": f"{cfg.name}: {cfg.describe()}", "ms_per_call": ms, "tokens_per_s": cfg.T / (ms / 1e3),
+            "useful_TFLOPs": flops / (ms / 1e3) / 1e12, "mma_TFLOPs": 2 * flops / (ms / 1e3) / 1e12,
+            "x_GBps": cfg.T * cfg.H * 2 / (ms / 1e3) / 1e9, "ctas": (cfg.T + 127) // 128, "steps": steps,
+            "note": "mok_plan_router: x (w_hi + w_lo) on tcgen05 (two bf16 MMAs per product), top-k and gates "
+                    "in the same kernel, then the schedule kernels"}
+
+
 # ------------------------------------------------------------------ roofline
 def tensor_peaks(peaks, mxfp8: bool, region_s: float):
     """(peak TFLOP/s of the MMA's dtype for a region this long, its kind)."""
@@ -521,7 +554,7 @@ def main():
                     help="persistent mode: least rows per minibatch (0: the two-wave rule alone; "
                          "default: the configuration's)")
     ap.add_argument("--dispatch-ctas", type=int, default=0,
-                    help="persistent mode: CTAs on the dispatch side (0: the library default, 4 bf16 / 16 MXFP8)")
+                    help="persistent mode: CTAs on the dispatch side (0: the library default, 8 bf16 / 16 MXFP8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub-records", action="store_true", help="time only the main workload")
     ap.add_argument("--cpu-steps", type=int, default=64, help="experts the CPU baseline samples")
@@ -545,7 +578,7 @@ def main():
              else "bf16 weights [E,H,I]/[E,I,H]")
     config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
               "tokens_per_step_per_gpu": cfg.T, "mode": args.mode,
-              **({"minibatch": minibatch, "dispatch_ctas": args.dispatch_ctas or (16 if cfg.mxfp8 else 4)}
+              **({"minibatch": minibatch, "dispatch_ctas": args.dispatch_ctas or (16 if cfg.mxfp8 else 8)}
                  if args.mode == "persistent" else {}),
               "l2": f"inputs larger than L2 ({algorithmic_work(cfg)['weight_bytes'] / 1e9:.1f} GB of expert "
                     f"weights streamed per step)"}
@@ -577,6 +610,7 @@ def main():
         other = "persistent" if args.mode == "staged" else "staged"
         r2 = time_steps(wl, other, args.steps, args.warmup, minibatch, args.dispatch_ctas)
         subs[f"{cfg.name}_{other}"] = sub_record(cfg, other, r2, peaks, peak_src, args.steps)
+        subs[f"{cfg.name}_router_plan"] = time_router(wl, args.steps, args.warmup)
         wl.free()
         del wl
         zcfg = mokgen.CONFIGS["zipf"]

@@ -41,7 +41,7 @@ EXPORTS = (
     "mok_plan_noalloc", "mok_mxfp8_quantize_rows", "mok_quantize_weights_mxfp8",
     "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8_workspace_bytes", "mok_expert_ffn_mxfp8",
     "mok_two_wave_rows", "mok_minibatch_bounds", "mok_forward_host_batches_workspace_bytes",
-    "mok_moe_forward_host_batches",
+    "mok_moe_forward_host_batches", "mok_router_weights_bytes", "mok_router_prepare", "mok_plan_router",
 )
 
 
@@ -99,6 +99,10 @@ def lib() -> ctypes.CDLL:
     L.mok_expert_ffn_mxfp8_workspace_bytes.restype = sz
     L.mok_expert_ffn_mxfp8.argtypes = [vp, vp, i32, i32, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
     L.mok_two_wave_rows.argtypes = [i32, i32, i32, i32]
+    L.mok_router_weights_bytes.argtypes = [i32, i32]
+    L.mok_router_weights_bytes.restype = sz
+    L.mok_router_prepare.argtypes = [vp, i32, i32, vp, vp, vp]
+    L.mok_plan_router.argtypes = [vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, ctypes.POINTER(PlanT), vp]
     L.mok_forward_host_batches_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(FwdOpts)]
     L.mok_forward_host_batches_workspace_bytes.restype = sz
     L.mok_moe_forward_host_batches.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, i32,
@@ -108,7 +112,8 @@ def lib() -> ctypes.CDLL:
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
               "mok_moe_forward_host", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
               "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8",
-              "mok_two_wave_rows", "mok_minibatch_bounds", "mok_moe_forward_host_batches"):
+              "mok_two_wave_rows", "mok_minibatch_bounds", "mok_moe_forward_host_batches", "mok_router_prepare",
+              "mok_plan_router"):
         getattr(L, n).restype = ctypes.c_int
     return L
 
@@ -186,6 +191,42 @@ def plan(logits: torch.Tensor, top_k: int, R: int, ws: torch.Tensor | None = Non
     p = PlanT()
     _check(lib().mok_plan(ctypes.c_void_p(logits.data_ptr()), T, E, top_k, R, ctypes.c_void_p(ws.data_ptr()),
                           ws.numel(), ctypes.byref(p), _stream(stream)))
+    return Plan(p, ws)
+
+
+def router_prepare(w_r: torch.Tensor, stream=None):
+    """``mok_router_prepare``: W_r [H, E] fp32 (device) -> (w_hi, w_lo), each
+    [E rounded up to 128, H] bf16."""
+    assert w_r.is_cuda and w_r.dtype == torch.float32 and w_r.is_contiguous()
+    H, E = w_r.shape
+    nbytes = lib().mok_router_weights_bytes(H, E)
+    if nbytes == 0:
+        raise MokError(MOK_ERR_UNSUPPORTED, "router shape")
+    rows = nbytes // (2 * H)
+    hi = torch.empty((rows, H), dtype=torch.bfloat16, device=w_r.device)
+    lo = torch.empty_like(hi)
+    _check(lib().mok_router_prepare(ctypes.c_void_p(w_r.data_ptr()), H, E, ctypes.c_void_p(hi.data_ptr()),
+                                    ctypes.c_void_p(lo.data_ptr()), _stream(stream)))
+    return hi, lo
+
+
+def plan_router(x_shards, w_hi: torch.Tensor, w_lo: torch.Tensor, E: int, top_k: int, prior=None,
+                logits_out: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None) -> Plan:
+    """``mok_plan_router``: the plan with the router projection on the device."""
+    R = len(x_shards)
+    S_r, H = x_shards[0].shape
+    T = S_r * R
+    need = lib().mok_plan_workspace_bytes(T, E, top_k)
+    if need == 0:
+        raise MokError(MOK_ERR_INVALID_ARG, "invalid plan shape")
+    if ws is None:
+        ws = _workspace(need, x_shards[0].device)
+    p = PlanT()
+    _check(lib().mok_plan_router(_ptr_array(x_shards), H, ctypes.c_void_p(w_hi.data_ptr()),
+                                 ctypes.c_void_p(w_lo.data_ptr()),
+                                 ctypes.c_void_p(prior.data_ptr()) if prior is not None else None, T, E, top_k, R,
+                                 ctypes.c_void_p(logits_out.data_ptr()) if logits_out is not None else None,
+                                 ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.byref(p), _stream(stream)))
     return Plan(p, ws)
 
 

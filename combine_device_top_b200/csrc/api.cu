@@ -166,11 +166,12 @@ struct FwdLayout {
 };
 
 static const uint64_t kDefaultTimeoutNs = 2000000000ull;
-// Dispatch CTAs of the persistent kernel by default: on the bf16 path one
-// thread per CTA streams rows with bulk copies (about 200 KB in flight), so
-// a few CTAs keep ahead of the GEMM; the MXFP8 path quantises with every
-// warp of its CTAs and needs more of them.
-static const int kDefaultDispatchBf16 = 4;
+// Dispatch CTAs of the persistent kernel by default.  On the bf16 path one
+// thread per CTA streams rows with bulk copies (about 200 KB in flight, some
+// 30 GB/s per CTA measured); at the page shape 2, 4, 8 and 16 CTAs gave
+// 15.7, 9.7, 8.0 and 8.4 ms per forward on B200 (one session).  The MXFP8
+// path quantises with every warp of its CTAs (16 measured best).
+static const int kDefaultDispatchBf16 = 8;
 
 static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* o, FwdLayout* L) {
     if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return false;
@@ -344,6 +345,80 @@ int mok_plan(const float* logits, int T, int E, int top_k, int R, void* ws, size
     plan->gates = reinterpret_cast<float*>(base + L.gates);
     if (device_sms(nullptr) <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     MOK_CUDA(launch_plan(logits, T, E, top_k, R, base, L, reinterpret_cast<cudaStream_t>(stream)), "plan launch");
+    return MOK_OK;
+}
+
+size_t mok_router_weights_bytes(int H, int E) {
+    if (H <= 0 || E <= 0 || E > MOK_ROUTER_MAX_EXPERTS) return 0;
+    return (size_t)router_e_pad(E) * H * 2;
+}
+
+int mok_router_prepare(const float* w_r, int H, int E, void* w_hi, void* w_lo, mok_stream_t stream) {
+    if (H <= 0 || E <= 0) return fail(MOK_ERR_INVALID_ARG, "H, E out of range");
+    if (E > MOK_ROUTER_MAX_EXPERTS) return fail(MOK_ERR_UNSUPPORTED, "E > %d", MOK_ROUTER_MAX_EXPERTS);
+    if (H % 64) return fail(MOK_ERR_UNSUPPORTED, "H %% 64 != 0 (H = %d)", H);
+    if (!w_r || !w_hi || !w_lo) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(w_hi) | reinterpret_cast<uintptr_t>(w_lo)) & 15u)
+        return fail(MOK_ERR_UNSUPPORTED, "w_hi and w_lo must be 16-byte aligned");
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(launch_router_split(w_r, H, E, w_hi, w_lo, sms, reinterpret_cast<cudaStream_t>(stream)),
+             "router weight split launch");
+    return MOK_OK;
+}
+
+int mok_plan_router(const void* const* x_shards, int H, const void* w_hi, const void* w_lo, const float* prior,
+                    int T, int E, int top_k, int R, float* logits_out, void* ws, size_t ws_bytes, mok_plan_t* plan,
+                    mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!plan) return fail(MOK_ERR_INVALID_ARG, "plan is NULL");
+    if (T < 0 || E <= 0 || top_k <= 0 || R <= 0 || H <= 0) return fail(MOK_ERR_INVALID_ARG, "T, E, top_k, R, H");
+    if (E > MOK_ROUTER_MAX_EXPERTS) return fail(MOK_ERR_UNSUPPORTED, "E > %d", MOK_ROUTER_MAX_EXPERTS);
+    if (top_k > E) return fail(MOK_ERR_INVALID_ARG, "top_k > E");
+    if (top_k > MOK_MAX_TOPK) return fail(MOK_ERR_UNSUPPORTED, "top_k > %d", MOK_MAX_TOPK);
+    if (R > MOK_MAX_SHARDS) return fail(MOK_ERR_UNSUPPORTED, "R > %d", MOK_MAX_SHARDS);
+    if (T % R) return fail(MOK_ERR_UNSUPPORTED, "T %% R != 0 (T = %d, R = %d)", T, R);
+    if (H % 64) return fail(MOK_ERR_UNSUPPORTED, "H %% 64 != 0 (H = %d)", H);
+    if ((int64_t)T * top_k > 0x3fffffff) return fail(MOK_ERR_UNSUPPORTED, "T * top_k too large");
+    if (!w_hi || !w_lo) return fail(MOK_ERR_INVALID_ARG, "NULL router weights");
+    if ((reinterpret_cast<uintptr_t>(w_hi) | reinterpret_cast<uintptr_t>(w_lo)) & 15u)
+        return fail(MOK_ERR_UNSUPPORTED, "w_hi and w_lo must be 16-byte aligned");
+    if (T > 0) {
+        if (!all_nonnull(x_shards, R)) return fail(MOK_ERR_INVALID_ARG, "NULL shard pointer");
+        if (!all_aligned16(x_shards, R)) return fail(MOK_ERR_UNSUPPORTED, "shard pointers must be 16-byte aligned");
+    }
+    PlanLayout L;
+    const size_t need = plan_layout(T, E, top_k, &L);
+    int rc = check_ws(ws, ws_bytes, need);
+    if (rc) return rc;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    auto I32 = [&](size_t o) { return reinterpret_cast<int32_t*>(base + o); };
+    plan->T = T;
+    plan->E = E;
+    plan->k = top_k;
+    plan->R = R;
+    plan->counts = I32(L.counts);
+    plan->offsets = I32(L.offsets);
+    plan->sched_src_rank = I32(L.src_rank);
+    plan->sched_src_index = I32(L.src_index);
+    plan->row_slot = I32(L.row_slot);
+    plan->pos = I32(L.pos);
+    plan->topk_idx = I32(L.topk);
+    plan->gates = reinterpret_cast<float*>(base + L.gates);
+    if (device_sms(nullptr) <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    MOK_CUDA(cudaMemsetAsync(base + L.status, 0, sizeof(DevStatus), stream), "status reset");
+    if (T > 0) {
+        ShardsIn xs{};
+        for (int r = 0; r < R; ++r) xs.p[r] = x_shards[r];
+        const char* err = "";
+        cudaError_t e = launch_router(xs, T / R, T, H, E, top_k, w_hi, w_lo, prior, logits_out, plan->topk_idx,
+                                      plan->gates, base + L.status, kDefaultTimeoutNs, &err, stream);
+        if (e != cudaSuccess) return fail(MOK_ERR_CUDA, "%s: %s", err, cudaGetErrorString(e));
+    }
+    MOK_CUDA(launch_plan_schedule(T, E, top_k, R, plan->counts, plan->offsets, plan->sched_src_rank,
+                                  plan->sched_src_index, plan->row_slot, plan->pos, plan->topk_idx, I32(L.blk_cnt),
+                                  I32(L.rank), stream),
+             "plan launch");
     return MOK_OK;
 }
 

@@ -114,22 +114,30 @@ __device__ __forceinline__ void warp_mx_quant8(const uint4& raw, uint2& q, uint3
 }
 
 // Slot outputs as the grouped GEMM stores them: fp32 (bf16 path) or bf16
-// (MXFP8 path).  SlotF32 / SlotBf16 load the 8 consecutive features of
-// slot row `row` that a lane owns (v = index of the 8-feature group).
+// (MXFP8 path).  A lane owns 8 consecutive features of a slot row (v = index
+// of the 8-feature group): load() issues the raw 16-byte loads, widen()
+// turns them into 8 floats.  The combine issues every load of a round
+// before it widens any, so all of them are in flight together.
 struct SlotF32 {
-    static constexpr int BYTES = 4;
-    __device__ static __forceinline__ void load(const void* out, size_t row, int nvec, int v, float (&f)[8]) {
+    struct Raw {
+        float4 a, b;
+    };
+    __device__ static __forceinline__ Raw load(const void* out, size_t row, int nvec, int v) {
         const float4* p = reinterpret_cast<const float4*>(out) + (row * nvec + v) * 2;
-        const float4 a = __ldcs(p), b = __ldcs(p + 1);
-        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+        return Raw{__ldcs(p), __ldcs(p + 1)};
+    }
+    __device__ static __forceinline__ void widen(const Raw& r, float (&f)[8]) {
+        f[0] = r.a.x; f[1] = r.a.y; f[2] = r.a.z; f[3] = r.a.w;
+        f[4] = r.b.x; f[5] = r.b.y; f[6] = r.b.z; f[7] = r.b.w;
     }
 };
 struct SlotBf16 {
-    static constexpr int BYTES = 2;
-    __device__ static __forceinline__ void load(const void* out, size_t row, int nvec, int v, float (&f)[8]) {
-        const uint4 a = __ldcs(reinterpret_cast<const uint4*>(out) + row * nvec + v);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    using Raw = uint4;
+    __device__ static __forceinline__ Raw load(const void* out, size_t row, int nvec, int v) {
+        return __ldcs(reinterpret_cast<const uint4*>(out) + row * nvec + v);
+    }
+    __device__ static __forceinline__ void widen(const Raw& r, float (&f)[8]) {
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&r);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             const float2 x = __bfloat1622float2(b2[p]);
@@ -154,21 +162,23 @@ __device__ __forceinline__ void warp_combine_token(const void* __restrict__ out,
     for (int v = lane; v < nvec; v += 32) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j0 = 0; j0 < k; j0 += KB) {
-            float a[KB][8];
+            typename S::Raw raw[KB];
             float g[KB];
 #pragma unroll
             for (int jj = 0; jj < KB; ++jj) {
                 const int j = j0 + jj;
                 if (j < k) {
                     g[jj] = __ldg(gt + j);
-                    S::load(out, row0 + j, nvec, v, a[jj]);
+                    raw[jj] = S::load(out, row0 + j, nvec, v);
                 }
             }
 #pragma unroll
             for (int jj = 0; jj < KB; ++jj)
                 if (j0 + jj < k) {
+                    float f[8];
+                    S::widen(raw[jj], f);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) acc[p] = fmaf(g[jj], a[jj][p], acc[p]);
+                    for (int p = 0; p < 8; ++p) acc[p] = fmaf(g[jj], f[p], acc[p]);
                 }
         }
         uint4 o;

@@ -15,7 +15,7 @@ namespace mok {
 // ---- plan workspace (byte offsets from the workspace base)
 struct PlanLayout {
     int nb;  // route blocks
-    size_t counts, offsets, src_rank, src_index, row_slot, pos, topk, gates, blk_cnt, rank, total;
+    size_t status, counts, offsets, src_rank, src_index, row_slot, pos, topk, gates, blk_cnt, rank, total;
 };
 size_t plan_layout(int T, int E, int k, PlanLayout* L);
 cudaError_t launch_plan(const float* logits, int T, int E, int k, int R, unsigned char* ws, const PlanLayout& L,
@@ -25,6 +25,10 @@ cudaError_t launch_plan_parts(const float* logits, int T, int E, int k, int R, i
                               int32_t* src_rank, int32_t* src_index, int32_t* row_slot, int32_t* pos,
                               int32_t* topk_idx, float* gates, int32_t* blk_cnt, int32_t* rank,
                               cudaStream_t stream);
+// Steps after the top-k (histogram, scan, schedule) from a given topk_idx.
+cudaError_t launch_plan_schedule(int T, int E, int k, int R, int32_t* counts, int32_t* offsets, int32_t* src_rank,
+                                 int32_t* src_index, int32_t* row_slot, int32_t* pos, const int32_t* topk_idx,
+                                 int32_t* blk_cnt, int32_t* rank, cudaStream_t stream);
 // Records a message for mok_last_error_string() and returns `code`.
 int report_error(int code, const char* msg);
 
@@ -173,6 +177,16 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
 // 128-byte swizzle, zero fill out of bounds.
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                          uint32_t box_outer, const char** err);
+
+// ---- the router projection fused with the top-k (router.cu)
+// Experts rounded up to the 128-row tiles of the router weights.
+int router_e_pad(int E);
+// w [H, E] fp32 -> hi, lo [E_pad, H] bf16 (hi + lo = w to about 16 bits)
+cudaError_t launch_router_split(const float* w, int H, int E, void* hi, void* lo, int num_sms, cudaStream_t stream);
+// logits = x W_r (+ prior), then top-k and gates per token; logits may be nullptr
+cudaError_t launch_router(const ShardsIn& xs, int S_r, int T, int H, int E, int k, const void* w_hi,
+                          const void* w_lo, const float* prior, float* logits, int32_t* topk_idx, float* gates,
+                          void* status, uint64_t timeout_ns, const char** err, cudaStream_t stream);
 
 // ---- MXFP8 quantisers (mxfp8.cu)
 cudaError_t launch_mx_quant_rows(const void* src, bool f32, int rows, int K, void* q, void* scales, int num_sms,

@@ -24,6 +24,7 @@
 // makes the schedule deterministic and independent of the launch shape.
 #include "mok_device.cuh"
 #include "mok_internal.h"
+#include "topk.cuh"
 
 namespace mok {
 
@@ -32,10 +33,6 @@ constexpr int PLAN_WARPS = PLAN_THREADS / 32;
 constexpr int PLAN_TOK = PLAN_WARPS * 32;  // tokens per block
 constexpr int MAX_CHUNKS_PER_LANE = MOK_MAX_EXPERTS / 32;
 
-__device__ __forceinline__ bool better(float v, int e, float bv, int be) {
-    return v > bv || (v == bv && e < be);
-}
-
 // One warp per token (grid-stride over tokens).  NC: 32-expert chunks held
 // per lane (ceil(E / 32) <= NC).
 template <int NC>
@@ -43,59 +40,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) k_topk(const float* __restrict__
                                                        int32_t* __restrict__ topk_idx, float* __restrict__ gates) {
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * PLAN_WARPS;
-    for (int t = blockIdx.x * PLAN_WARPS + (threadIdx.x >> 5); t < T; t += warps) {
-        const float* row = logits + (size_t)t * E;
-        float v[NC];
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            const int e = c * 32 + lane;
-            float x = -INFINITY;
-            if (e < E) {
-                x = __ldg(row + e);
-                if (x != x) x = -INFINITY;  // NaN compares as -inf
-            }
-            v[c] = x;
-        }
-        uint32_t taken = 0;
-        int my_idx = 0;
-        float my_val = 0.f, m = 0.f;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                const int e = c * 32 + lane;
-                if (e < E && !((taken >> c) & 1u) && better(v[c], e, bv, be)) {
-                    bv = v[c];
-                    be = e;
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (better(ov, oe, bv, be)) {
-                    bv = ov;
-                    be = oe;
-                }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            if (j == 0) m = bv;
-            if (lane == j) {
-                my_idx = be;
-                my_val = bv;
-            }
-        }
-        // softmax over the k selected logits (the first is the maximum)
-        float ex = (lane < k) ? expf(my_val - m) : 0.f;
-        float s = ex;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane < k) {
-            topk_idx[(size_t)t * k + lane] = my_idx;
-            gates[(size_t)t * k + lane] = ex / s;
-        }
-    }
+    for (int t = blockIdx.x * PLAN_WARPS + (threadIdx.x >> 5); t < T; t += warps)
+        warp_topk_token<NC>(logits + (size_t)t * E, E, k, lane, topk_idx + (size_t)t * k, gates + (size_t)t * k);
 }
 
 // dynamic smem: sel[PLAN_TOK][k] int32 | mask[PLAN_WARPS][E] uint32
@@ -205,6 +151,7 @@ size_t plan_layout(int T, int E, int k, PlanLayout* L) {
     };
     PlanLayout l;
     l.nb = nb;
+    l.status = take(64);  // device status word of the router kernel (mok_plan_router)
     l.counts = take(sizeof(int32_t) * E);
     l.offsets = take(sizeof(int32_t) * (E + 1));
     l.src_rank = take(sizeof(int32_t) * ns);
@@ -266,15 +213,13 @@ cudaError_t launch_plan(const float* logits, int T, int E, int k, int R, unsigne
 // scratch arrays: blk_cnt [ceil(T/256), E] and rank [T*k]).
 int plan_route_blocks(int T) { return (T + PLAN_TOK - 1) / PLAN_TOK; }
 
-cudaError_t launch_plan_parts(const float* logits, int T, int E, int k, int R, int32_t* counts, int32_t* offsets,
-                              int32_t* src_rank, int32_t* src_index, int32_t* row_slot, int32_t* pos,
-                              int32_t* topk_idx, float* gates, int32_t* blk_cnt, int32_t* rank,
-                              cudaStream_t stream) {
+cudaError_t launch_plan_schedule(int T, int E, int k, int R, int32_t* counts, int32_t* offsets, int32_t* src_rank,
+                                 int32_t* src_index, int32_t* row_slot, int32_t* pos, const int32_t* topk_idx,
+                                 int32_t* blk_cnt, int32_t* rank, cudaStream_t stream) {
     cudaError_t e = rank_configure();
     if (e != cudaSuccess) return e;
     const size_t smem = sizeof(int32_t) * PLAN_TOK * k + sizeof(uint32_t) * PLAN_WARPS * E;
     const int nb = plan_route_blocks(T);
-    if ((e = launch_topk(logits, T, E, k, topk_idx, gates, stream)) != cudaSuccess) return e;
     if (T > 0) k_rank<<<nb, PLAN_THREADS, smem, stream>>>(topk_idx, T, E, k, blk_cnt, rank);
     k_scan<<<1, 1024, 0, stream>>>(blk_cnt, nb, E, T * k, counts, offsets);
     if (T > 0) {
@@ -284,6 +229,17 @@ cudaError_t launch_plan_parts(const float* logits, int T, int E, int k, int R, i
             topk_idx, rank, blk_cnt, offsets, T, E, k, T / R, src_rank, src_index, row_slot, pos);
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_plan_parts(const float* logits, int T, int E, int k, int R, int32_t* counts, int32_t* offsets,
+                              int32_t* src_rank, int32_t* src_index, int32_t* row_slot, int32_t* pos,
+                              int32_t* topk_idx, float* gates, int32_t* blk_cnt, int32_t* rank,
+                              cudaStream_t stream) {
+    cudaError_t e = rank_configure();
+    if (e != cudaSuccess) return e;
+    if ((e = launch_topk(logits, T, E, k, topk_idx, gates, stream)) != cudaSuccess) return e;
+    return launch_plan_schedule(T, E, k, R, counts, offsets, src_rank, src_index, row_slot, pos, topk_idx, blk_cnt,
+                                rank, stream);
 }
 
 }  // namespace mok

@@ -111,6 +111,54 @@ size_t mok_plan_workspace_bytes(int T, int E, int k);
 int mok_plan(const float* logits, int T, int E, int top_k, int R,
              void* ws, size_t ws_bytes, mok_plan_t* plan, mok_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Step 1 with the router projection on the device.
+ * ---------------------------------------------------------------------- */
+
+enum { MOK_ROUTER_MAX_EXPERTS = 384 };
+
+/* Bytes of EACH of the two router weight parts made by mok_router_prepare:
+ * [E rounded up to 128, H] bf16.  0 for an unsupported shape. */
+size_t mok_router_weights_bytes(int H, int E);
+
+/*
+ * mok_router_prepare -- one-time split of the router weights W_r [H, E]
+ * fp32 (device) into two bf16 parts [E_pad, H] (expert-major, H
+ * contiguous; E_pad = E rounded up to 128, padding rows zero):
+ * w_hi = bf16(W_r), w_lo = bf16(W_r - w_hi), so w_hi + w_lo carries about
+ * 16 significant bits of W_r with fp32's exponent range.  H % 64 == 0,
+ * E <= MOK_ROUTER_MAX_EXPERTS; w_hi and w_lo (device, caller-owned,
+ * mok_router_weights_bytes each) 16-byte aligned.  Asynchronous.
+ */
+int mok_router_prepare(const float* w_r, int H, int E, void* w_hi, void* w_lo, mok_stream_t stream);
+
+/*
+ * mok_plan_router -- mok_plan with the router projection computed on the
+ * device: logits[t, e] = sum_h x[t, h] W_r[h, e] + prior[e], on the tensor
+ * cores as x w_hi + x w_lo with fp32 accumulation, then the same top-k,
+ * gates, histogram and pull schedule as mok_plan, in one router kernel
+ * (projection, top-k and gates fused) plus the schedule kernels.
+ * Source: MoK article, routing paragraph (a router assigns every token to
+ * its experts; the projection is the plain reading the oracle's router
+ * follows); MoK wiki summary, schedule bullet (the schedule is built on the
+ * device without CPU traffic).
+ *   x_shards    HOST array of R device pointers, shard r = [S_r, H] bf16
+ *   w_hi, w_lo  from mok_router_prepare
+ *   prior       [E] fp32 added to every token's logits, or NULL
+ *   logits_out  [T, E] fp32 device array that receives the logits, or NULL
+ *   ws, plan    as for mok_plan (same workspace size)
+ * The logits differ from the exact projection by about 2^-17 + (H/16) 2^-23
+ * of sum_h |x[t,h] W_r[h,e]| at most (the split, then one fp32 accumulator
+ * addition per 16-wide MMA); logits closer than that may
+ * be ordered either way (ties in the computed values still go to the lower
+ * index).  A device-side failure (a bounded wait that gave up) is recorded
+ * in the plan workspace's status word: mok_get_status(ws, ...) reads it
+ * (mok_plan does not write that word).  Asynchronous on `stream`.
+ */
+int mok_plan_router(const void* const* x_shards, int H, const void* w_hi, const void* w_lo,
+                    const float* prior, int T, int E, int top_k, int R, float* logits_out,
+                    void* ws, size_t ws_bytes, mok_plan_t* plan, mok_stream_t stream);
+
 /* Size of the library-owned scratch array used by mok_plan_noalloc. */
 #define MOK_PLAN_NOALLOC_SCRATCH_BYTES (2u << 20)
 
@@ -164,7 +212,7 @@ typedef struct mok_fwd_opts {
     int32_t ring_slots;    /* rows of the ring token buffer (persistent mode);  */
                            /* 0 = 2 * max(minibatch, 4096) rows                 */
     int32_t dispatch_ctas; /* CTAs doing the dispatch in persistent mode;       */
-                           /* 0 = default (4 bf16: bulk copies; 16 MXFP8:      */
+                           /* 0 = default (8 bf16: bulk copies; 16 MXFP8:      */
                            /* quantising warps).  Every CTA combines once its  */
                            /* own role is done                                 */
     int32_t gemm_ctas;     /* GEMM CTAs; 0 = all remaining SMs                  */
@@ -292,7 +340,7 @@ int mok_quantize_weights_mxfp8(const void* w_bf16, int E, int K, int N, void* q,
 
 /*
  * mok_get_status -- synchronise `stream` and read the device status word of
- * a forward workspace.  *device_code receives MOK_OK, MOK_ERR_TIMEOUT or
+ * a forward workspace (or of a plan workspace after mok_plan_router).  *device_code receives MOK_OK, MOK_ERR_TIMEOUT or
  * MOK_ERR_CAPACITY; the return value is MOK_OK unless the read itself
  * failed.  The status word is cleared at the start of every forward.
  */

@@ -241,3 +241,28 @@ def test_host_batches_reject_null_host_pointers_before_any_copy():
     rc = L.mok_moe_forward_host_batches(2, good, good, good, 63, 128, 128, 8, 2, 2, 1, 1, 1, 64, ctypes.byref(opts),
                                         4096, need, None)
     assert rc == mok.MOK_ERR_INVALID_ARG
+
+
+def test_router_entry_points_check_arguments():
+    L = mok.lib()
+    assert L.mok_router_weights_bytes(7168, 384) == 384 * 7168 * 2
+    assert L.mok_router_weights_bytes(512, 8) == 128 * 512 * 2          # experts padded to 128 rows
+    assert L.mok_router_weights_bytes(512, 385) == 0                      # above MOK_ROUTER_MAX_EXPERTS
+    assert L.mok_router_prepare(4096, 512, 385, 4096, 8192, None) == mok.MOK_ERR_UNSUPPORTED
+    assert L.mok_router_prepare(4096, 500, 8, 4096, 8192, None) == mok.MOK_ERR_UNSUPPORTED   # H % 64
+    assert L.mok_router_prepare(None, 512, 8, 4096, 8192, None) == mok.MOK_ERR_INVALID_ARG
+    assert L.mok_router_prepare(4096, 512, 8, 4097, 8192, None) == mok.MOK_ERR_UNSUPPORTED  # alignment
+    p = mok.PlanT()
+    arr = (ctypes.c_void_p * 2)(4096, 8192)
+    need = L.mok_plan_workspace_bytes(64, 8, 2)
+
+    def call(T=64, E=8, k=2, R=2, H=128, hi=4096, lo=8192, xs=arr, ws=4096, nbytes=need):
+        return L.mok_plan_router(xs, H, hi, lo, None, T, E, k, R, None, ws, nbytes, ctypes.byref(p), None)
+
+    assert call(E=400) == mok.MOK_ERR_UNSUPPORTED
+    assert call(H=96) == mok.MOK_ERR_UNSUPPORTED
+    assert call(k=9) == mok.MOK_ERR_INVALID_ARG
+    assert call(T=63) == mok.MOK_ERR_UNSUPPORTED
+    assert call(lo=8200) == mok.MOK_ERR_UNSUPPORTED
+    assert call(xs=(ctypes.c_void_p * 2)(4096, 8200)) == mok.MOK_ERR_UNSUPPORTED
+    assert call(ws=4096, nbytes=need - 1) == mok.MOK_ERR_WORKSPACE
