@@ -42,6 +42,7 @@ EXPORTS = (
     "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8_workspace_bytes", "mok_expert_ffn_mxfp8",
     "mok_two_wave_rows", "mok_minibatch_bounds", "mok_forward_host_batches_workspace_bytes",
     "mok_moe_forward_host_batches", "mok_router_weights_bytes", "mok_router_prepare", "mok_plan_router",
+    "mok_backward_workspace_bytes", "mok_moe_backward",
 )
 
 
@@ -62,7 +63,7 @@ class PlanT(ctypes.Structure):
 class FwdOpts(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("dispatch_ctas", ctypes.c_int32),
                 ("gemm_ctas", ctypes.c_int32), ("mxfp8", ctypes.c_int32), ("min_waves", ctypes.c_int32),
-                ("timeout_ns", ctypes.c_uint64)]
+                ("save_for_backward", ctypes.c_int32), ("reserved", ctypes.c_int32), ("timeout_ns", ctypes.c_uint64)]
 
 
 @lru_cache(maxsize=1)
@@ -99,6 +100,10 @@ def lib() -> ctypes.CDLL:
     L.mok_expert_ffn_mxfp8_workspace_bytes.restype = sz
     L.mok_expert_ffn_mxfp8.argtypes = [vp, vp, i32, i32, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
     L.mok_two_wave_rows.argtypes = [i32, i32, i32, i32]
+    L.mok_backward_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    L.mok_backward_workspace_bytes.restype = sz
+    L.mok_moe_backward.argtypes = [vp, i32, i32, vp, vp, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp, vp, vp, vp, vp, sz,
+                                   vp]
     L.mok_router_weights_bytes.argtypes = [i32, i32]
     L.mok_router_weights_bytes.restype = sz
     L.mok_router_prepare.argtypes = [vp, i32, i32, vp, vp, vp]
@@ -113,7 +118,7 @@ def lib() -> ctypes.CDLL:
               "mok_moe_forward_host", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
               "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8",
               "mok_two_wave_rows", "mok_minibatch_bounds", "mok_moe_forward_host_batches", "mok_router_prepare",
-              "mok_plan_router"):
+              "mok_plan_router", "mok_moe_backward"):
         getattr(L, n).restype = ctypes.c_int
     return L
 
@@ -254,8 +259,9 @@ def quantize_weights_mxfp8(w: torch.Tensor, stream=None):
 
 
 def fwd_opts(mode: int = MOK_MODE_PERSISTENT, ring_slots: int = 0, dispatch_ctas: int = 0, gemm_ctas: int = 0,
-             mxfp8: bool = False, timeout_ns: int = 0, min_waves: int = 0) -> FwdOpts:
-    return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), min_waves, timeout_ns)
+             mxfp8: bool = False, timeout_ns: int = 0, min_waves: int = 0, save_for_backward: bool = False) -> FwdOpts:
+    return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), min_waves, int(save_for_backward), 0,
+                   timeout_ns)
 
 
 def forward_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None = None) -> int:
@@ -347,6 +353,38 @@ def minibatch_bounds(p: Plan, H: int, I: int, minibatch: int, opts: FwdOpts, w_g
                                       ctypes.c_void_p(ws.data_ptr()), ws.numel(), row0, units, cap, ctypes.byref(n),
                                       _stream(stream)))
     return list(row0[:n.value]), list(units[:n.value])
+
+
+def moe_backward(dy_shards, w_gate, w_up, w_down, p: Plan, fwd_ws: torch.Tensor, dx_shards=None, dw=None,
+                 dlogits=None, ws: torch.Tensor | None = None, stream=None):
+    """``mok_moe_backward``: the layer's gradients given dy (shards of [S_r, H]
+    bf16).  ``fwd_ws`` is the workspace of a staged :func:`moe_forward` with
+    ``save_for_backward``.  Returns (dx_shards, (dWg, dWu, dWd), dlogits, ws)."""
+    R = p.c.R
+    assert len(dy_shards) == R and (dx_shards is None or len(dx_shards) == R)
+    H = dy_shards[0].shape[1]
+    I = w_gate.shape[-1]
+    E, T, k = p.c.E, p.c.T, p.c.k
+    dev = dy_shards[0].device
+    for w in (w_gate, w_up, w_down):
+        assert w.dtype == torch.bfloat16, "the weights are bf16"
+    if dx_shards is None:
+        dx_shards = [torch.empty_like(s) for s in dy_shards]
+    if dw is None:
+        dw = (torch.empty((E, H, I), dtype=torch.bfloat16, device=dev),
+              torch.empty((E, H, I), dtype=torch.bfloat16, device=dev),
+              torch.empty((E, I, H), dtype=torch.bfloat16, device=dev))
+    if dlogits is None:
+        dlogits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(lib().mok_backward_workspace_bytes(T, H, I, E, k), dev)
+    _check(lib().mok_moe_backward(_ptr_array(dy_shards), H, I, ctypes.c_void_p(w_gate.data_ptr()),
+                                  ctypes.c_void_p(w_up.data_ptr()), ctypes.c_void_p(w_down.data_ptr()),
+                                  ctypes.byref(p.c), ctypes.c_void_p(fwd_ws.data_ptr()), fwd_ws.numel(),
+                                  _ptr_array(dx_shards), *(ctypes.c_void_p(t.data_ptr()) for t in dw),
+                                  ctypes.c_void_p(dlogits.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                  _stream(stream)))
+    return dx_shards, dw, dlogits, ws
 
 
 def get_status(ws: torch.Tensor, stream=None) -> int:

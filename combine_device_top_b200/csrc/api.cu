@@ -160,7 +160,8 @@ bool encode_bmaps_u8(BMaps* maps, const void* base, uint64_t inner, uint64_t row
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct FwdLayout {
-    size_t status, counts2, chunks, mbs, counters, counter_ints, rows, h, out, total;
+    size_t status, counts2, chunks, mbs, counters, counter_ints, rows, h, out, save_a, save_b, total;
+    int save;
     size_t xsc, hsc;  // MXFP8 path: token-side scale planes
     int max_chunks, max_mb, buf_rows, cap, minibatch, mode, mx;
 };
@@ -219,6 +220,13 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
         l.h = take((size_t)l.buf_rows * I * 2);
     }
     l.out = take((size_t)ns * H * (l.mx ? 2 : 4));  // slot outputs: fp32, or bf16 on the MXFP8 path
+    // kept for the backward (staged bf16 path): gate and up pre-activations
+    l.save = (o && o->save_for_backward) ? 1 : 0;
+    if (l.save) {
+        if (l.mx || l.mode != MOK_MODE_STAGED) return false;
+        l.save_a = take((size_t)ns * I * 2);
+        l.save_b = take((size_t)ns * I * 2);
+    }
     l.total = off;
     *L = l;
     return true;
@@ -260,7 +268,8 @@ static int check_hi(int H, int I) {
 static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const void* wg, const void* wu,
                           const void* wd, int E, const int32_t* row_slot, const Chunk* chunks, const int* counts2,
                           void* h, void* out, DevStatus* status, uint64_t timeout_ns, cudaStream_t stream,
-                          const mok_mxfp8_weights* mxw = nullptr, const MxTokenScales* mxs = nullptr) {
+                          const mok_mxfp8_weights* mxw = nullptr, const MxTokenScales* mxs = nullptr,
+                          const BwdBuffers* save = nullptr) {
     int dev = 0;
     const int sms = device_sms(&dev);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
@@ -281,7 +290,7 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
     const GemmTuning tune = gemm_tuning(n_rows_buf, E);
     const MxMaps* mxp = mxw ? &mx : nullptr;
     MOK_CUDA(launch_gemm_phase(0, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
-                               tune, stream),
+                               tune, stream, save),
              "gate/up GEMM launch");
     MOK_CUDA(launch_gemm_phase(1, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
                                tune, stream),
@@ -462,6 +471,9 @@ static int setup_forward(int H, int I, const void* w_gate, const mok_plan_t* pla
         if (!m || !m->gate || !m->gate_scales || !m->up || !m->up_scales || !m->down || !m->down_scales)
             return fail(MOK_ERR_INVALID_ARG, "MXFP8 weight pack with NULL members");
     }
+    if (opts && opts->reserved != 0) return fail(MOK_ERR_INVALID_ARG, "opts.reserved must be 0");
+    if (opts && opts->save_for_backward && (mode != MOK_MODE_STAGED || (opts->mxfp8 != 0)))
+        return fail(MOK_ERR_UNSUPPORTED, "save_for_backward needs the staged bf16 path");
     if (mode == MOK_MODE_PERSISTENT && minibatch != 0 && minibatch < 16)
         return fail(MOK_ERR_INVALID_ARG, "minibatch must be 0 (two-wave rule) or >= 16");
     if (minibatch < 0) return fail(MOK_ERR_INVALID_ARG, "minibatch < 0");
@@ -637,11 +649,111 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
     } else {
         MOK_CUDA(launch_gather(xs, T / R, H, T, k, plan->pos, base + L.rows, sms, stream), "gather launch");
     }
+    BwdBuffers save{};
+    if (L.save) {
+        save.save_a = reinterpret_cast<uint16_t*>(base + L.save_a);
+        save.save_b = reinterpret_cast<uint16_t*>(base + L.save_b);
+    }
     rc = run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, E, plan->row_slot, F.chunks, F.counts2,
-                        base + L.h, base + L.out, F.status, F.timeout, stream, mxw, mxw ? &mxs : nullptr);
+                        base + L.h, base + L.out, F.status, F.timeout, stream, mxw, mxw ? &mxs : nullptr,
+                        L.save ? &save : nullptr);
     if (rc) return rc;
     MOK_CUDA(launch_combine(base + L.out, mxw != nullptr, plan->gates, T, k, H, T / R, ys, sms, stream),
              "combine launch");
+    return MOK_OK;
+}
+
+size_t mok_backward_workspace_bytes(int T, int H, int I, int E, int k) {
+    if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return 0;
+    const size_t ns = (size_t)T * k;
+    return align256(sizeof(DevStatus)) + align256(ns * H * 2) + align256(ns * (size_t)I * 4) +
+           align256(ns * H * 4);
+}
+
+int mok_moe_backward(const void* const* dy_shards, int H, int I, const void* w_gate, const void* w_up,
+                     const void* w_down, const mok_plan_t* plan, const void* fwd_ws, size_t fwd_ws_bytes,
+                     void* const* dx_shards, void* dw_gate, void* dw_up, void* dw_down, float* dlogits, void* ws,
+                     size_t ws_bytes, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if ((rc = check_hi(H, I))) return rc;
+    if (I % 128) return fail(MOK_ERR_UNSUPPORTED, "the backward needs I %% 128 == 0 (I = %d)", I);
+    const int T = plan->T, E = plan->E, k = plan->k, R = plan->R;
+    if (T == 0) return MOK_OK;
+    if (!all_nonnull(dy_shards, R) || !all_nonnull(dx_shards, R)) return fail(MOK_ERR_INVALID_ARG, "NULL shard pointer");
+    if (!all_aligned16(dy_shards, R) || !all_aligned16(dx_shards, R))
+        return fail(MOK_ERR_UNSUPPORTED, "shard pointers must be 16-byte aligned");
+    if (!w_gate || !w_up || !w_down || !dw_gate || !dw_up || !dw_down || !dlogits || !fwd_ws)
+        return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    if ((reinterpret_cast<uintptr_t>(dw_gate) | reinterpret_cast<uintptr_t>(dw_up) |
+         reinterpret_cast<uintptr_t>(dw_down)) & 15u)
+        return fail(MOK_ERR_UNSUPPORTED, "weight gradients must be 16-byte aligned");
+    // the forward workspace as a staged forward with save_for_backward laid it out
+    mok_fwd_opts fo{};
+    fo.mode = MOK_MODE_STAGED;
+    fo.save_for_backward = 1;
+    FwdLayout FL;
+    if (!fwd_layout(T, H, I, E, k, 0, &fo, &FL)) return fail(MOK_ERR_INVALID_ARG, "invalid shape");
+    if ((rc = check_ws(fwd_ws, fwd_ws_bytes, FL.total))) return rc;
+    if ((rc = check_ws(ws, ws_bytes, mok_backward_workspace_bytes(T, H, I, E, k)))) return rc;
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    int dev = 0;
+    device_sms(&dev);
+    const unsigned char* fb = static_cast<const unsigned char*>(fwd_ws);
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    const size_t ns = (size_t)T * k;
+    size_t off = 0;
+    DevStatus* status = reinterpret_cast<DevStatus*>(base);
+    off += align256(sizeof(DevStatus));
+    void* do_rows = base + off;
+    off += align256(ns * H * 2);
+    uint16_t* dab = reinterpret_cast<uint16_t*>(base + off);
+    off += align256(ns * (size_t)I * 4);
+    float* dx_slots = reinterpret_cast<float*>(base + off);
+    ShardsIn dys{};
+    ShardsOut dxs{};
+    for (int r = 0; r < R; ++r) {
+        dys.p[r] = dy_shards[r];
+        dxs.p[r] = dx_shards[r];
+    }
+    MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
+    // 1. pull reverse-combine: do rows, gate gradients, dlogits
+    MOK_CUDA(launch_reverse_combine(dys, T / R, H, T, k, E, plan->pos, plan->gates, plan->topk_idx,
+                                    reinterpret_cast<const float*>(fb + FL.out), do_rows, dlogits, sms, stream),
+             "reverse combine launch");
+    // 2. dh = do Wd^T with the SwiGLU backward -> [da | db]; 3. dx rows = da Wg^T + db Wu^T -> slots
+    MOK_CUDA(gemm_configure(dev), "gemm configure");
+    GemmMaps maps;
+    memset(&maps, 0, sizeof maps);
+    const char* err = nullptr;
+    if (!encode_tmap_2d_bf16(&maps.wd, w_down, (uint64_t)H, (uint64_t)E * I, 64, 128, &err) ||
+        !encode_tmap_2d_bf16(&maps.wg, w_gate, (uint64_t)I, (uint64_t)E * H, 64, 128, &err) ||
+        !encode_tmap_2d_bf16(&maps.wu, w_up, (uint64_t)I, (uint64_t)E * H, 64, 128, &err) ||
+        !encode_bmaps(&maps.rows, do_rows, (uint64_t)H, (uint64_t)ns, &err) ||
+        !encode_bmaps(&maps.h, dab, (uint64_t)2 * I, (uint64_t)ns, &err))
+        return fail(MOK_ERR_CUDA, "tensor map: %s", err);
+    BwdBuffers bb{};
+    bb.save_a = reinterpret_cast<uint16_t*>(const_cast<unsigned char*>(fb) + FL.save_a);
+    bb.save_b = reinterpret_cast<uint16_t*>(const_cast<unsigned char*>(fb) + FL.save_b);
+    bb.dab = dab;
+    const Chunk* chunks = reinterpret_cast<const Chunk*>(fb + FL.chunks);
+    const int* counts2 = reinterpret_cast<const int*>(fb + FL.counts2);
+    GemmShape sh{H, I, E};
+    GemmTuning tune = gemm_tuning((int)ns, E);
+    MOK_CUDA(launch_gemm_phase(2, maps, nullptr, nullptr, sh, chunks, counts2, nullptr, nullptr, plan->row_slot, status,
+                               kDefaultTimeoutNs, sms, tune, stream, &bb),
+             "dh GEMM launch");
+    MOK_CUDA(launch_gemm_phase(3, maps, nullptr, nullptr, sh, chunks, counts2, nullptr, dx_slots, plan->row_slot,
+                               status, kDefaultTimeoutNs, sms, tune, stream, &bb),
+             "dx GEMM launch");
+    // 4. push reverse-dispatch: dx_t = sum of its k rows (the combine with unit weights)
+    MOK_CUDA(launch_combine(dx_slots, false, nullptr, T, k, H, T / R, dxs, sms, stream), "reverse dispatch launch");
+    // 5. weight gradients per expert over its rows
+    cudaError_t e = launch_wgrad(fb + FL.rows, fb + FL.h, do_rows, dab, (int)ns, plan->offsets, H, I, E, dw_gate,
+                                 dw_up, dw_down, status, kDefaultTimeoutNs, sms, &err, stream);
+    if (e != cudaSuccess) return fail(MOK_ERR_CUDA, "%s: %s", err ? err : "", cudaGetErrorString(e));
     return MOK_OK;
 }
 

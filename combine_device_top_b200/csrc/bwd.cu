@@ -1,0 +1,393 @@
+// bwd.cu -- the backward of the forward MoE layer (bf16 path): the pull
+// reverse-combine and the weight-gradient grouped GEMM.  The data-gradient
+// GEMMs (dh with the SwiGLU backward, dx pushed to the token slots) are
+// phases 2 and 3 of the grouped-GEMM core (gemm_core.cuh); the push
+// reverse-dispatch sum is the combine with unit weights.
+//
+// MoK article (tahou.com), the Pull/Push paragraph: the backward pairs a
+// pull reverse-combine (the expert side reads the output gradient of every
+// token it served) with a push reverse-dispatch (each row's input gradient
+// goes straight back to its token).  The arithmetic is the chain rule of
+// the forward layer, in that order of steps:
+//   do_tj = g_tj dy_t,  dg_tj = <dy_t, o_tj>          (reverse combine)
+//   dh = do Wd^T;  da = dh b silu'(a),  db = dh silu(a)
+//   dx_row = da Wg^T + db Wu^T,  dx_t = sum_j dx_row(t, j) (reverse dispatch)
+//   dWd = h^T do,  dWg = x^T da,  dWu = x^T db          (per expert, over its rows)
+//   dl_tj = g_tj (dg_tj - sum_i g_ti dg_ti)              (softmax backward)
+#include "mok_device.cuh"
+#include "mok_internal.h"
+
+namespace mok {
+
+// ------------------------------------------------------------------ reverse combine
+// One warp per token: dy_t is read once (16-byte vectors, 8 features per
+// lane); for each of its k slots the warp writes the bf16 row do = g dy_t to
+// the slot's expert-major row and accumulates <dy_t, o_slot> from the
+// forward's fp32 slot outputs; then the softmax backward over the k gates
+// gives the token's dlogits row (zeros outside its selection).
+template <int KB>
+__global__ void __launch_bounds__(256) k_reverse_combine(ShardsIn dys, int S_r, int H, int T, int k, int E,
+                                                         const int32_t* __restrict__ pos,
+                                                         const float* __restrict__ gates,
+                                                         const int32_t* __restrict__ topk_idx,
+                                                         const float* __restrict__ o_slots,
+                                                         uint4* __restrict__ do_rows, float* __restrict__ dlogits) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = H >> 3;
+    const int warps = gridDim.x * 8;
+    for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += warps) {
+        const int r = t / S_r;
+        const uint4* dy = reinterpret_cast<const uint4*>(dys.p[r]) + (size_t)(t - r * S_r) * nvec;
+        const int my_row = lane < k ? __ldg(pos + (size_t)t * k + lane) : 0;
+        const float my_g = lane < k ? __ldg(gates + (size_t)t * k + lane) : 0.f;
+        int rows[KB];
+        float gs[KB], dgp[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            rows[j] = __shfl_sync(0xffffffffu, my_row, j & 31);
+            gs[j] = __shfl_sync(0xffffffffu, my_g, j & 31);
+            dgp[j] = 0.f;
+        }
+        // lanes may run different numbers of iterations: no warp collectives inside
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 raw = __ldg(dy + v);
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+            float d[8];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                d[2 * p] = __uint_as_float(w[p] << 16);
+                d[2 * p + 1] = __uint_as_float(w[p] & 0xffff0000u);
+            }
+#pragma unroll
+            for (int j = 0; j < KB; ++j) {
+                if (j < k) {
+                    const float4* o = reinterpret_cast<const float4*>(o_slots + ((size_t)t * k + j) * H) + 2 * v;
+                    const float4 o0 = __ldcs(o), o1 = __ldcs(o + 1);
+                    dgp[j] += d[0] * o0.x + d[1] * o0.y + d[2] * o0.z + d[3] * o0.w + d[4] * o1.x + d[5] * o1.y +
+                              d[6] * o1.z + d[7] * o1.w;
+                    const float g = gs[j];
+                    do_rows[(size_t)rows[j] * nvec + v] =
+                        make_uint4(pack_bf16x2(g * d[0], g * d[1]), pack_bf16x2(g * d[2], g * d[3]),
+                                   pack_bf16x2(g * d[4], g * d[5]), pack_bf16x2(g * d[6], g * d[7]));
+                }
+            }
+        }
+        // dg_j over the warp; every lane ends with every sum
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dgp[j] += __shfl_xor_sync(0xffffffffu, dgp[j], off);
+        }
+        float dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < KB; ++j)
+            if (j < k) dot += gs[j] * dgp[j];
+        float* dl = dlogits + (size_t)t * E;
+        for (int e = lane; e < E; e += 32) dl[e] = 0.f;
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < KB; ++j)
+            if (j < k && lane == (j & 31)) dl[__ldg(topk_idx + (size_t)t * k + j)] = gs[j] * (dgp[j] - dot);
+    }
+}
+
+cudaError_t launch_reverse_combine(const ShardsIn& dys, int S_r, int H, int T, int k, int E, const int32_t* pos,
+                                   const float* gates, const int32_t* topk_idx, const float* o_slots, void* do_rows,
+                                   float* dlogits, int num_sms, cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    const int want = (T + 7) / 8;
+    const int grid = want < num_sms * 8 ? want : num_sms * 8;
+    uint4* d = reinterpret_cast<uint4*>(do_rows);
+    if (k <= 2)
+        k_reverse_combine<2><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, d, dlogits);
+    else if (k <= 8)
+        k_reverse_combine<8><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, d, dlogits);
+    else
+        k_reverse_combine<32><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, d,
+                                                        dlogits);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ weight gradients
+// Units (expert e, gradient, M tile of 128 output rows, N tile of NB output
+// columns), expert-major so that the CTAs working at one time share an
+// expert's rows in L2:
+//   dWd[e] [I, H] = h^T do:   M = i, N = h, A = h rows, B = do rows
+//   dWg[e] [H, I] = x^T da:   M = h, N = i, A = x rows, B = da (dab cols 0..I)
+//   dWu[e] [H, I] = x^T db:   M = h, N = i, A = x rows, B = db (dab cols I..2I)
+// K = the expert's rows, 64 per stage; both operands are MN-major tiles of
+// {64 columns, 64 rows} boxes (128-byte swizzle).  Rows of the last stage
+// past the expert belong to the next expert (or are TMA zero fill): the MMA
+// warp zeroes them in shared memory before the MMAs.  Accumulators: two of
+// NB columns in TMEM, so one unit's epilogue overlaps the next's MMAs.
+// Output bf16 rows, 2 NB bytes per TMEM lane.
+constexpr int WG_THREADS = 192;  // warp 0 TMA, warp 1 zeroing + MMA, warps 2-5 epilogue
+constexpr int WG_NST = 4;
+constexpr int WG_A_BYTES = 128 * 64 * 2;  // 16 KB
+// bound of the waits that drain this CTA's own loads and MMAs before it leaves
+constexpr uint64_t DRAIN_NS_WG = 1000000000ull;
+
+struct WgradMaps {
+    CUtensorMap x, h, dor, dab;  // {64, 64} boxes of rows [N_s, H], [N_s, I], [N_s, H], [N_s, 2I]
+};
+
+struct WgradArgs {
+    int H, I, E, nb;           // nb: N tile (256 or 128)
+    int dm_t, dn_t, gm_t, gn_t;  // M / N tiles of dWd and of dWg (= dWu)
+    int upe;                   // units per expert
+    const int32_t* offsets;    // [E+1]
+    uint16_t *dwg, *dwu, *dwd;
+    DevStatus* st;
+    uint64_t timeout_ns;
+};
+
+struct WgUnit {
+    int e, g, m0, n0, r0, rows;  // g: 0 dWd, 1 dWg, 2 dWu
+};
+
+__device__ __forceinline__ bool wg_unit(const WgradArgs& a, int u, WgUnit& w) {
+    if (u >= a.E * a.upe) return false;
+    w.e = u / a.upe;
+    int r = u - w.e * a.upe;
+    const int nd = a.dm_t * a.dn_t, ng = a.gm_t * a.gn_t;
+    if (r < nd) {
+        w.g = 0;
+        w.m0 = (r / a.dn_t) * 128;
+        w.n0 = (r % a.dn_t) * a.nb;
+    } else {
+        r -= nd;
+        w.g = r < ng ? 1 : 2;
+        if (r >= ng) r -= ng;
+        w.m0 = (r / a.gn_t) * 128;
+        w.n0 = (r % a.gn_t) * a.nb;
+    }
+    w.r0 = __ldg(a.offsets + w.e);
+    w.rows = __ldg(a.offsets + w.e + 1) - w.r0;
+    return true;
+}
+
+__global__ void __launch_bounds__(WG_THREADS, 1)
+    k_wgrad(const __grid_constant__ WgradMaps maps, const WgradArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                           ~uintptr_t(1023));
+    const int b_bytes = a.nb * 64 * 2;
+    const int stage_bytes = WG_A_BYTES + b_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + WG_NST * stage_bytes);
+    uint64_t* empty = full + WG_NST;
+    uint64_t* tfull = empty + WG_NST;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* fin = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < WG_NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+        }
+        mbar_init(fin, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&maps.x);
+        tma_prefetch_desc(&maps.h);
+        tma_prefetch_desc(&maps.dor);
+        tma_prefetch_desc(&maps.dab);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    WgUnit w;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, issued_phase = 0;
+            bool ok = true;
+            for (int i = 0; ok && wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
+                const int KB = (w.rows + 63) / 64;
+                const CUtensorMap* am = w.g == 0 ? &maps.h : &maps.x;
+                const CUtensorMap* bm = w.g == 0 ? &maps.dor : &maps.dab;
+                const int bx0 = w.n0 + (w.g == 2 ? a.I : 0);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 100)) {
+                        ok = false;
+                        break;
+                    }
+                    unsigned char* st = smem + stage * stage_bytes;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(WG_A_BYTES + b_bytes));
+                    const int y = w.r0 + kb * 64;
+                    tma_load_2d(st, am, &full[stage], w.m0, y);
+                    tma_load_2d(st + 8192, am, &full[stage], w.m0 + 64, y);
+                    for (int c = 0; c < a.nb / 64; ++c)
+                        tma_load_2d(st + WG_A_BYTES + c * 8192, bm, &full[stage], bx0 + c * 64, y);
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == WG_NST) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            for (int s = 0; s < WG_NST; ++s)
+                if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, nullptr, DRAIN_NS_WG, 101);
+        }
+    } else if (warp == 1) {
+        int stage = 0;
+        uint32_t phase = 0, tk = 0;
+        const uint32_t idesc = umma_idesc_f16(128, a.nb, /*A MN-major*/ 1, /*B MN-major*/ 1, /*bf16*/ 1);
+        bool ok = true;
+        for (int i = 0; ok && wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
+            if (w.rows == 0) continue;  // the epilogue writes zeros; no accumulator is used
+            const int KB = (w.rows + 63) / 64;
+            if (lane == 0) ok = mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 102);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            tc_fence_after();
+            for (int kb = 0; kb < KB; ++kb) {
+                int got = 0;
+                if (lane == 0) got = mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 103) ? 1 : 0;
+                if (__shfl_sync(0xffffffffu, got, 0) == 0) {
+                    ok = false;
+                    break;
+                }
+                unsigned char* st = smem + stage * stage_bytes;
+                const int valid = min(64, w.rows - kb * 64);
+                if (valid < 64) {
+                    // rows past the expert: zero their 128-byte K lines in every 64-wide block of A and B
+                    const int nblk = 2 + a.nb / 64;
+                    const int lines = 64 - valid;
+                    for (int i2 = lane; i2 < nblk * lines * 8; i2 += 32) {
+                        const int blk = i2 / (lines * 8), rem = i2 - blk * lines * 8;
+                        const int line = valid + rem / 8, chunk = rem % 8;
+                        *reinterpret_cast<uint4*>(st + blk * 8192 + line * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(st), sb = sa + WG_A_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        // both MN-major SW128: 16 K rows = 2 atoms of 1 KB; 64-wide blocks 8 KB apart
+                        const uint64_t ad = umma_desc_sw128(sa + ks * 2048, 8192, 1024);
+                        const uint64_t bd = umma_desc_sw128(sb + ks * 2048, 8192, 1024);
+                        umma_bf16(tmem + (tk & 1u) * 256u, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == WG_NST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(&tfull[tk & 1u]);
+            ++tk;
+        }
+        if (lane == 0) {
+            umma_commit(fin);
+            mbar_wait(fin, 0, nullptr, DRAIN_NS_WG, 104);
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: TMEM lane = output row m0 + 32 q + lane, NB bf16 columns
+        const int q = warp & 3;
+        uint32_t tk = 0;
+        for (int i = 0; wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
+            uint16_t* out = w.g == 0 ? a.dwd + (size_t)w.e * a.I * a.H : (w.g == 1 ? a.dwg : a.dwu) + (size_t)w.e * a.H * a.I;
+            const int ldo = w.g == 0 ? a.H : a.I;
+            uint16_t* orow = out + (size_t)(w.m0 + q * 32 + lane) * ldo + w.n0;
+            if (w.rows == 0) {
+                for (int c = 0; c < a.nb; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+                continue;
+            }
+            int got = 0;
+            if (lane == 0) got = mbar_wait(&tfull[tk & 1u], (tk >> 1) & 1u, a.st, a.timeout_ns, 105) ? 1 : 0;
+            if (__shfl_sync(0xffffffffu, got, 0) == 0) break;
+            tc_fence_after();
+            for (int c = 0; c < a.nb; c += 32) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (tk & 1u) * 256u + (uint32_t)c, v);
+#pragma unroll
+                for (int p = 0; p < 32; p += 8)
+                    *reinterpret_cast<uint4*>(orow + c + p) =
+                        make_uint4(pack_bf16x2(v[p], v[p + 1]), pack_bf16x2(v[p + 2], v[p + 3]),
+                                   pack_bf16x2(v[p + 4], v[p + 5]), pack_bf16x2(v[p + 6], v[p + 7]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[tk & 1u]);
+            ++tk;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+static bool encode_rows64(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, const char** err) {
+    return encode_tmap_2d_bf16(m, base, inner, rows, 64, 64, err);
+}
+
+cudaError_t launch_wgrad(const void* x_rows, const void* h_rows, const void* do_rows, const void* dab, int n_rows,
+                         const int32_t* offsets, int H, int I, int E, void* dwg, void* dwu, void* dwd, void* status,
+                         uint64_t timeout_ns, int num_sms, const char** err, cudaStream_t stream) {
+    WgradMaps maps;
+    if (!encode_rows64(&maps.x, x_rows, (uint64_t)H, (uint64_t)n_rows, err) ||
+        !encode_rows64(&maps.h, h_rows, (uint64_t)I, (uint64_t)n_rows, err) ||
+        !encode_rows64(&maps.dor, do_rows, (uint64_t)H, (uint64_t)n_rows, err) ||
+        !encode_rows64(&maps.dab, dab, (uint64_t)2 * I, (uint64_t)n_rows, err))
+        return cudaErrorInvalidValue;
+    WgradArgs a{};
+    a.H = H;
+    a.I = I;
+    a.E = E;
+    a.nb = (H % 256 == 0 && I % 256 == 0) ? 256 : 128;
+    a.dm_t = I / 128;
+    a.dn_t = H / a.nb;
+    a.gm_t = H / 128;
+    a.gn_t = I / a.nb;
+    a.upe = a.dm_t * a.dn_t + 2 * a.gm_t * a.gn_t;
+    a.offsets = offsets;
+    a.dwg = reinterpret_cast<uint16_t*>(dwg);
+    a.dwu = reinterpret_cast<uint16_t*>(dwu);
+    a.dwd = reinterpret_cast<uint16_t*>(dwd);
+    a.st = reinterpret_cast<DevStatus*>(status);
+    a.timeout_ns = timeout_ns;
+    const int smem = WG_NST * (WG_A_BYTES + a.nb * 128) + 256 + 1024;
+    static bool attr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr[dev]) {
+        e = cudaFuncSetAttribute(k_wgrad, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 WG_NST * (WG_A_BYTES + 256 * 128) + 256 + 1024);
+        if (e != cudaSuccess) return e;
+        attr[dev] = true;
+    }
+    const long long units = (long long)E * a.upe;
+    const int grid = (int)(units < num_sms ? units : num_sms);
+    *err = "weight-gradient launch";
+    if (grid <= 0) return cudaSuccess;
+    k_wgrad<<<grid, WG_THREADS, smem, stream>>>(maps, a);
+    return cudaGetLastError();
+}
+
+}  // namespace mok

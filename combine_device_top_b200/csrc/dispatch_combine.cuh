@@ -147,7 +147,8 @@ struct SlotBf16 {
     }
 };
 
-// One warp: y[t] = bf16(sum_{j<k} g[t,j] * out[t,j,:]) in fp32, j ascending.
+// One warp: y[t] = bf16(sum_{j<k} g[t,j] * out[t,j,:]) in fp32, j ascending
+// (gates == nullptr: every g = 1, the backward's reverse-dispatch sum).
 // out is [T, k, H] of slot type S; each lane owns 8 consecutive features
 // (one 16-byte store of y).  nvec = H / 8.  Slots are loaded KB at a time
 // (KB loads in flight), then accumulated in order; k > KB takes several
@@ -156,7 +157,7 @@ template <int KB, class S>
 __device__ __forceinline__ void warp_combine_token(const void* __restrict__ out, const float* __restrict__ gates,
                                                    int t, int k, int nvec, uint4* __restrict__ dst, int lane) {
     const size_t row0 = (size_t)t * k;
-    const float* gt = gates + row0;
+    const float* gt = gates ? gates + row0 : nullptr;
     // lanes may run different numbers of iterations (nvec % 32 != 0): no
     // warp collectives inside; the gates are broadcast loads (L1 hits)
     for (int v = lane; v < nvec; v += 32) {
@@ -168,7 +169,7 @@ __device__ __forceinline__ void warp_combine_token(const void* __restrict__ out,
             for (int jj = 0; jj < KB; ++jj) {
                 const int j = j0 + jj;
                 if (j < k) {
-                    g[jj] = __ldg(gt + j);
+                    g[jj] = gates ? __ldg(gt + j) : 1.f;
                     raw[jj] = S::load(out, row0 + j, nvec, v);
                 }
             }

@@ -142,6 +142,12 @@ struct CoreArgs {
     const uint8_t* xsc;       // token rows (gate/up B operand), K = H
     uint8_t* hsc;             // h rows (written by gate/up, read by down), K = I
     int sc_rows;              // rows per plane, a multiple of 4
+    // bf16 path, kept for the backward: gate and up pre-activations a, b
+    // [buffer rows, I] bf16 (written by gate/up when not null; read by the
+    // dh phase), and the dh phase's output [da | db] rows [buffer rows, 2I]
+    uint16_t* save_a;
+    uint16_t* save_b;
+    uint16_t* dab;
 };
 
 // Unit u -> (chunk c, M tile m) in raster groups of GC chunks: inside a group
@@ -187,8 +193,15 @@ struct StagedSched {
 
 // M tiles of a phase (64 gate + 64 up features, or 128 down features, each),
 // and how many of them unit u covers.
+// Backward phases (bf16 path): 2 = dh = do Wd^T with the SwiGLU backward
+// in the epilogue (M = I features), 3 = dx rows = da Wg^T + db Wu^T pushed
+// to the token slots (M = H features); both read A K-major.
 __device__ __forceinline__ int phase_tiles(const CoreArgs& a, int phase) {
-    return phase == 0 ? a.I / MT_G_FEATURES : a.H / MT_D_FEATURES;
+    return phase == 0 ? a.I / MT_G_FEATURES : phase == 2 ? a.I / MT_D_FEATURES : a.H / MT_D_FEATURES;
+}
+// Contraction length of a phase.
+__device__ __forceinline__ int phase_k(const CoreArgs& a, int phase) {
+    return phase == 0 || phase == 2 ? a.H : phase == 1 ? a.I : 2 * a.I;
 }
 template <class C>
 __device__ __forceinline__ int unit_subs(const CoreArgs& a, const Unit& u) {
@@ -212,9 +225,9 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
         if (!s.wait_inputs(u, a.st, a.timeout_ns)) break;
-        const int K = u.phase == 0 ? a.H : a.I;
+        const int K = phase_k(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
-        const BMaps& bm = u.phase == 0 ? maps.rows : maps.h;
+        const BMaps& bm = (u.phase == 0 || u.phase == 2) ? maps.rows : maps.h;
         const int bx = token_box(u.rows);
         const int nsub = unit_subs<C>(a, u);
         uint32_t bytes = (uint32_t)(16 * (bx + 1)) * B_ROW_BYTES;
@@ -262,6 +275,16 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
                         tma_load_2d_hint(sa, &maps.wg, &full[stage], mt * MT_G_FEATURES, ky, evict_first);
                         tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], mt * MT_G_FEATURES, ky,
                                          evict_first);
+                    } else if (u.phase == 2) {
+                        // Wd [E*I, H] K-major: 128 feature rows x 64 K in one box
+                        tma_load_2d_hint(sa, &maps.wd, &full[stage], kb * BK, u.expert * a.I + mt * MT_D_FEATURES,
+                                         evict_first);
+                    } else if (u.phase == 3) {
+                        // Wg then Wu [E*H, I] K-major: K runs over I twice
+                        const int KI = a.I / BK;
+                        const bool up = kb >= KI;
+                        tma_load_2d_hint(sa, up ? &maps.wu : &maps.wg, &full[stage], (kb - (up ? KI : 0)) * BK,
+                                         u.expert * a.H + mt * MT_D_FEATURES, evict_first);
                     } else if (maps.has_wd3) {
                         // both 64-column halves of the 128-column down tile in one op
                         tma_load_3d_hint(sa, &maps.wd3, &full[stage], 0, ky, mt * 2, evict_first);
@@ -307,7 +330,7 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
     uint32_t phase = 0;
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
-        const int K = u.phase == 0 ? a.H : a.I;
+        const int K = phase_k(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
         const int nsub = unit_subs<C>(a, u);
         const int lead = u.brow0 & 3;
@@ -384,14 +407,15 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
     uint32_t tk = 0;  // next accumulator ticket
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
-        const int K = u.phase == 0 ? a.H : a.I;
+        const int K = phase_k(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
         const int N = (u.rows + 15) & ~15;
         const int nsub = unit_subs<C>(a, u);
         const int nt = unit_tickets<C>(nsub, N);
         const bool wide = nt == 2;
-        // bf16 path: both phases bf16 x bf16
-        const uint32_t idesc = umma_idesc_f16(128, N, /*A MN-major*/ 1, /*B K-major*/ 0, /*bf16*/ 1);
+        // bf16 path: every phase bf16 x bf16; A MN-major (forward) or K-major (backward)
+        const bool a_kmaj = u.phase >= 2;
+        const uint32_t idesc = umma_idesc_f16(128, N, a_kmaj ? 0 : 1, /*B K-major*/ 0, /*bf16*/ 1);
         bool ok = true;
         for (int t = 0; t < nt && ok; ++t) {
             const uint32_t tkt = tk + (uint32_t)t;
@@ -440,9 +464,12 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
 #pragma unroll
                     for (int sub = 0; sub < C::SUB; ++sub) {
                         if (sub < nsub) {
-                            // A: MN-major SW128, 16 K rows per MMA = 2 atoms of 1 KB;
-                            //    the two 64-wide MN halves are 8 KB apart (LBO).
-                            const uint64_t ad = umma_desc_sw128(sa + sub * A_BYTES + ks * 2048, A_BYTES / 2, 1024);
+                            // A MN-major SW128: 16 K rows per MMA = 2 atoms of 1 KB, the two
+                            //   64-wide MN halves 8 KB apart (LBO);
+                            // A K-major SW128: 16 K = 32 bytes inside the atom, 8-row groups 1 KB apart.
+                            const uint64_t ad =
+                                a_kmaj ? umma_desc_sw128(sa + sub * A_BYTES + ks * 32, 16, 1024)
+                                       : umma_desc_sw128(sa + sub * A_BYTES + ks * 2048, A_BYTES / 2, 1024);
                             umma_bf16(tmem_base + acc_col(tk, sub, wide), ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
                         }
                     }
@@ -529,14 +556,55 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 } else {
                     const uint4 pk = make_uint4(pack_bf16x2(hv[0], hv[1]), pack_bf16x2(hv[2], hv[3]),
                                                 pack_bf16x2(hv[4], hv[5]), pack_bf16x2(hv[6], hv[7]));
-                    if (live)
-                        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) + row * a.I + mt * MT_G_FEATURES +
-                                                  j0) = pk;
+                    const size_t at = row * a.I + mt * MT_G_FEATURES + j0;
+                    if (live) {
+                        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) + at) = pk;
+                        if (a.save_a) {
+                            *reinterpret_cast<uint4*>(a.save_a + at) =
+                                make_uint4(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]),
+                                           pack_bf16x2(gv[4], gv[5]), pack_bf16x2(gv[6], gv[7]));
+                            *reinterpret_cast<uint4*>(a.save_b + at) =
+                                make_uint4(pack_bf16x2(uv[0], uv[1]), pack_bf16x2(uv[2], uv[3]),
+                                           pack_bf16x2(uv[4], uv[5]), pack_bf16x2(uv[6], uv[7]));
+                        }
+                    }
+                }
+            }
+        } else if (u.phase == 2) {
+            // dh of features mt*128 + 4*lane .. +3, a warp per token: the SwiGLU backward with the
+            // row's saved a, b (bf16); da and db rows pushed as bf16 into dab [rows, 2I]
+#pragma unroll 2
+            for (int it = 0; it < 8; ++it) {
+                const int t = it * 4 + q;
+                const int col = cc * 32 + t;
+                if (col < u.rows) {
+                    const size_t row = (size_t)(u.brow0 + col);
+                    const int i0 = mt * MT_D_FEATURES + 4 * lane;
+                    const float4 d4 = *reinterpret_cast<const float4*>(epi + t * EPI_TLD + 4 * lane);
+                    const uint2 av = *reinterpret_cast<const uint2*>(a.save_a + row * a.I + i0);
+                    const uint2 bv = *reinterpret_cast<const uint2*>(a.save_b + row * a.I + i0);
+                    const float dh[4] = {d4.x, d4.y, d4.z, d4.w};
+                    const float af[4] = {__uint_as_float(av.x << 16), __uint_as_float(av.x & 0xffff0000u),
+                                         __uint_as_float(av.y << 16), __uint_as_float(av.y & 0xffff0000u)};
+                    const float bf[4] = {__uint_as_float(bv.x << 16), __uint_as_float(bv.x & 0xffff0000u),
+                                         __uint_as_float(bv.y << 16), __uint_as_float(bv.y & 0xffff0000u)};
+                    float da[4], db[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        // silu(a) = a s, silu'(a) = s + a s (1 - s), s = 1 / (1 + e^-a)
+                        const float sg = 1.0f / (1.0f + __expf(-af[p]));
+                        db[p] = dh[p] * af[p] * sg;
+                        da[p] = dh[p] * bf[p] * (sg + af[p] * sg * (1.0f - sg));
+                    }
+                    uint16_t* out = a.dab + row * (size_t)(2 * a.I) + i0;
+                    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]));
+                    *reinterpret_cast<uint2*>(out + a.I) =
+                        make_uint2(pack_bf16x2(db[0], db[1]), pack_bf16x2(db[2], db[3]));
                 }
             }
         } else {
             // push to the token's slot, one row per warp store (fp32: 512 bytes, MXFP8 path bf16: 256
-            // bytes); the combine rounds y once
+            // bytes); the combine rounds y once.  Phase 3 (dx rows) pushes the same way.
 #pragma unroll 4
             for (int it = 0; it < 8; ++it) {
                 const int t = it * 4 + q;

@@ -56,9 +56,15 @@ cudaError_t gemm_configure(int dev) {
 cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const MxTokenScales* mxs,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              const GemmTuning& tune, cudaStream_t stream) {
+                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd) {
     if (mx && !mxs) return cudaErrorInvalidValue;
+    if (phase >= 2 && (mx || !bwd || !bwd->save_a || !bwd->save_b || !bwd->dab)) return cudaErrorInvalidValue;
     CoreArgs a{};
+    if (bwd) {
+        a.save_a = bwd->save_a;
+        a.save_b = bwd->save_b;
+        a.dab = bwd->dab;
+    }
     if (mxs) {
         a.xsc = mxs->xsc;
         a.hsc = mxs->hsc;
@@ -71,7 +77,7 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.row_slot = row_slot;
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
-    const int tiles = phase == 0 ? sh.I / MT_G_FEATURES : sh.H / MT_D_FEATURES;
+    const int tiles = phase == 0 ? sh.I / MT_G_FEATURES : phase == 2 ? sh.I / MT_D_FEATURES : sh.H / MT_D_FEATURES;
     // Pairs only for the bf16 gate/up launch.  MXFP8 keeps one tile per unit:
     // measured, pairs were 6-10 % slower there (a tall pair fills TMEM, and
     // its quantising epilogue then stalls the next unit's MMAs).  The down

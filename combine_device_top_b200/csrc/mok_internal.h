@@ -140,10 +140,19 @@ struct MxTokenScales {
 struct MxMaps;
 // mx: MXFP8 weight maps (MXFP8 path: rows and h are E4M3 with the scale
 // planes of mxs), or nullptr (bf16 path).
+// Buffers of the bf16 path kept for / used by the backward: a, b [rows, I]
+// bf16 (phase 0 writes them when not null; phase 2 reads them) and
+// dab = [da | db] rows [rows, 2I] bf16 (phase 2 writes, phase 3 reads).
+struct BwdBuffers {
+    uint16_t *save_a, *save_b, *dab;
+};
+// phase 2 (dh + SwiGLU backward -> dab) and 3 (dx rows -> out[row_slot])
+// read maps.wd / maps.wg, maps.wu as K-major maps ({64 K, 128 rows} boxes
+// of [E*I, H] / [E*H, I]) and B from maps.rows (do rows) / maps.h (dab).
 cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const MxTokenScales* mxs,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              const GemmTuning& tune, cudaStream_t stream);
+                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd = nullptr);
 
 // ---- the persistent SM-partitioned forward (persistent.cu)
 struct PersistLaunch {
@@ -177,6 +186,16 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
 // 128-byte swizzle, zero fill out of bounds.
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                          uint32_t box_outer, const char** err);
+
+// ---- the backward (bwd.cu)
+// do rows (bf16, expert-major) = g dy_t; dlogits [T, E] by the softmax backward
+cudaError_t launch_reverse_combine(const ShardsIn& dys, int S_r, int H, int T, int k, int E, const int32_t* pos,
+                                   const float* gates, const int32_t* topk_idx, const float* o_slots, void* do_rows,
+                                   float* dlogits, int num_sms, cudaStream_t stream);
+// dWd = h^T do, dWg = x^T da, dWu = x^T db per expert (bf16 outputs)
+cudaError_t launch_wgrad(const void* x_rows, const void* h_rows, const void* do_rows, const void* dab, int n_rows,
+                         const int32_t* offsets, int H, int I, int E, void* dwg, void* dwu, void* dwd, void* status,
+                         uint64_t timeout_ns, int num_sms, const char** err, cudaStream_t stream);
 
 // ---- the router projection fused with the top-k (router.cu)
 // Experts rounded up to the 128-row tiles of the router weights.

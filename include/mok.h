@@ -222,6 +222,10 @@ typedef struct mok_fwd_opts {
     int32_t min_waves;     /* persistent mode: a minibatch holds at least this  */
                            /* many full waves of gate/up units of the GEMM     */
                            /* CTAs; 0 = 2 (the pages' rule); < 0 = no floor    */
+    int32_t save_for_backward; /* staged bf16 path: 1 = keep the gate and up    */
+                           /* pre-activations (bf16) in the workspace for      */
+                           /* mok_moe_backward                                 */
+    int32_t reserved;      /* must be 0                                         */
     uint64_t timeout_ns;   /* bound on every device-side wait; 0 = 2 s          */
 } mok_fwd_opts;
 
@@ -314,6 +318,49 @@ int mok_two_wave_rows(int I, int gemm_ctas, int tile_rows, int tile_features);
 int mok_minibatch_bounds(const mok_plan_t* plan, int H, int I, const void* w_gate, int minibatch,
                          const mok_fwd_opts* opts, void* ws, size_t ws_bytes, int32_t* row0,
                          int32_t* units, int max_mb, int* n_mb, mok_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The backward of the layer (bf16 path).
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of backward workspace: do rows [N_s, H] bf16, [da | db] rows
+ * [N_s, 2I] bf16, dx rows [N_s, H] fp32 and a status word. */
+size_t mok_backward_workspace_bytes(int T, int H, int I, int E, int k);
+
+/*
+ * mok_moe_backward -- gradients of the layer given dy.
+ * Source: MoK article, the Pull/Push paragraph (the backward pairs a pull
+ * reverse-combine with a push reverse-dispatch); the arithmetic is the
+ * chain rule of the forward, step by step:
+ *   1. pull reverse-combine: for each slot (t, j), do = g[t,j] dy_t as a
+ *      bf16 row in the expert-major layout, dg[t,j] = <dy_t, o[t,j]>;
+ *   2. dh = do Wd^T (fp32 accumulation); da = dh b silu'(a),
+ *      db = dh silu(a), rounded to bf16;
+ *   3. dx rows = da Wg^T + db Wu^T (fp32), pushed to their token's slot;
+ *   4. push reverse-dispatch: dx_t = bf16(sum_j dx rows of t), j ascending;
+ *   5. dWd[e] = h^T do, dWg[e] = x^T da, dWu[e] = x^T db over the expert's
+ *      rows (fp32 accumulation, bf16 results; an expert with no rows gets
+ *      zeros);
+ *   6. dlogits[t, sel[t,j]] = g[t,j] (dg[t,j] - sum_i g[t,i] dg[t,i]), 0 for
+ *      unselected experts (the selection has no gradient).
+ *   dy_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
+ *   w_*        the forward's bf16 weights
+ *   plan       the forward's plan
+ *   fwd_ws     the workspace of the staged mok_moe_forward call on this plan
+ *              with opts.save_for_backward = 1 (it holds the gathered rows,
+ *              h, the gate and up pre-activations a and b, and the fp32
+ *              slot outputs o); not modified
+ *   dx_shards  HOST array of R device pointers, shard r = [S_r, H] bf16
+ *   dw_gate, dw_up [E, H, I] bf16; dw_down [E, I, H] bf16; dlogits [T, E] fp32
+ *   ws         backward workspace (>= mok_backward_workspace_bytes)
+ * H % 128 == 0, I % 128 == 0.  Device-side failures go to ws's status word
+ * (mok_get_status).  Asynchronous on `stream`.
+ */
+int mok_moe_backward(const void* const* dy_shards, int H, int I,
+                     const void* w_gate, const void* w_up, const void* w_down,
+                     const mok_plan_t* plan, const void* fwd_ws, size_t fwd_ws_bytes,
+                     void* const* dx_shards, void* dw_gate, void* dw_up, void* dw_down,
+                     float* dlogits, void* ws, size_t ws_bytes, mok_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * MXFP8 (OCP MX v1.0: 32-element blocks, E8M0 scale byte = s + 127 with
