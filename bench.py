@@ -429,6 +429,61 @@ def time_router(wl: Workload, steps: int, warmup: int):
                     "in the same kernel, then the schedule kernels"}
 
 
+def backward_work(cfg):
+    """Algorithmic bytes / flops of one backward (bf16 path)."""
+    ns, H, I, E, T = cfg.slots, cfg.H, cfg.I, cfg.E, cfg.T
+    rc = T * H * 2 + ns * H * 4 + ns * H * 2 + T * E * 4            # dy, fp32 slots in; do rows, dlogits out
+    dh = E * I * H * 2 + ns * H * 2 + 2 * ns * I * 2 + 2 * ns * I * 2  # Wd, do; a, b in; da, db out
+    dx = 2 * E * H * I * 2 + 2 * ns * I * 2 + ns * H * 4            # Wg, Wu, da, db in; fp32 dx rows out
+    rd = ns * H * 4 + T * H * 2                                      # dx rows in, dx out
+    wg = 3 * E * H * I * 2 + ns * (2 * H + I + 2 * I + H) * 2        # bf16 dW out; x, h, do, da|db rows in
+    return {"flops": 12.0 * H * I * ns, "bytes": float(rc + dh + dx + rd + wg), "wgrad_bytes": float(wg)}
+
+
+def time_backward(wl: Workload, steps: int, warmup: int):
+    """mok_moe_backward on the workload after one staged forward that keeps
+    the gate/up pre-activations; dy synthetic N(0,1) bf16 resident in HBM;
+    CUDA events on the launching stream around the backward calls only."""
+    import combine_device_top_b200 as mok
+
+    cfg, device = wl.cfg, wl.device
+    opts = mok.fwd_opts(mode=mok.MOK_MODE_STAGED, save_for_backward=True)
+    fws = torch.empty(mok.forward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, 0, opts), dtype=torch.uint8,
+                      device=device)
+    mok.moe_forward(wl.x_shards, *wl.w, wl.plan, 0, opts, y_shards=wl.y_shards, ws=fws)
+    dy = mokgen.normal(cfg.seed, 99, (cfg.T, cfg.H), 1.0).to(device)
+    dys = mok.shards(dy, cfg.R)
+    dx = torch.empty_like(dy)
+    dxs = mok.shards(dx, cfg.R)
+    dw = (torch.empty((cfg.E, cfg.H, cfg.I), dtype=torch.bfloat16, device=device),
+          torch.empty((cfg.E, cfg.H, cfg.I), dtype=torch.bfloat16, device=device),
+          torch.empty((cfg.E, cfg.I, cfg.H), dtype=torch.bfloat16, device=device))
+    dl = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=device)
+    bws = torch.empty(mok.lib().mok_backward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k), dtype=torch.uint8,
+                      device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        mok.moe_backward(dys, *wl.w, wl.plan, fws, dx_shards=dxs, dw=dw, dlogits=dl, ws=bws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        mok.moe_backward(dys, *wl.w, wl.plan, fws, dx_shards=dxs, dw=dw, dlogits=dl, ws=bws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if mok.get_status(bws) != mok.MOK_OK or not torch.isfinite(dx.float()).all():
+        raise RuntimeError("backward failed: " + mok.last_error())
+    ms = e0.elapsed_time(e1) / steps
+    work = backward_work(cfg)
+    del fws, bws, dw, dl, dx, dy
+    torch.cuda.empty_cache()
+    return {"workload": f"{cfg.name}: {cfg.describe()}", "ms_per_call": ms, "tokens_per_s": cfg.T / (ms / 1e3),
+            "GBps": work["bytes"] / (ms / 1e3) / 1e9, "TFLOPs": work["flops"] / (ms / 1e3) / 1e12,
+            "algorithmic_GB": work["bytes"] / 1e9, "steps": steps,
+            "note": "mok_moe_backward: reverse combine, dh + SwiGLU backward, dx, reverse dispatch, weight "
+                    "gradients (bf16 dW)"}
+
+
 # ------------------------------------------------------------------ roofline
 def tensor_peaks(peaks, mxfp8: bool, region_s: float):
     """(peak TFLOP/s of the MMA's dtype for a region this long, its kind)."""
@@ -611,6 +666,9 @@ def main():
         r2 = time_steps(wl, other, args.steps, args.warmup, minibatch, args.dispatch_ctas)
         subs[f"{cfg.name}_{other}"] = sub_record(cfg, other, r2, peaks, peak_src, args.steps)
         subs[f"{cfg.name}_router_plan"] = time_router(wl, args.steps, args.warmup)
+        bw = time_backward(wl, max(3, args.steps // 4), 2)
+        bw["frac_of_hbm"] = bw["GBps"] / peaks["hbm_gbs"]
+        subs[f"{cfg.name}_backward"] = bw
         wl.free()
         del wl
         zcfg = mokgen.CONFIGS["zipf"]
