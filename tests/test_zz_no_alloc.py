@@ -74,3 +74,29 @@ def test_plan_noalloc_rejects_shapes_beyond_its_scratch():
     rc = mok.lib().mok_plan_noalloc(dummy, T, E, k, 8, *([dummy] * 8), None)
     assert rc == mok.MOK_ERR_UNSUPPORTED
     assert "MOK_PLAN_NOALLOC_SCRATCH_BYTES" in mok.last_error()
+
+
+def test_plan_noalloc_leaves_device_memory_untouched():
+    """The call allocates nothing: device free memory is the same before and
+    after its first call on a new shape.  One call on another shape comes
+    first: the first call in a process loads the code module that holds the
+    static scratch array (its fixed 2 MiB, held until exit, as documented).
+    mok_plan then runs on the new shape, so its kernels' code is loaded too
+    (lazy module loading takes device memory for code, which is not an
+    allocation of this entry point)."""
+    _noalloc_plan(mokgen.small_ints(11, 76, (64, 16), 5).cuda(), 2, 2)
+    logits = mokgen.small_ints(11, 77, (777, 96), 5).cuda()
+    k, R = 6, 7
+    mok.plan(logits, k, R)
+    T, E = logits.shape
+    outs = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (E, E + 1, T * k, T * k, T * k, T * k, T * k)]
+    gates = torch.empty(T * k, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    rc = mok.lib().mok_plan_noalloc(ctypes.c_void_p(logits.data_ptr()), T, E, k, R,
+                                    *(ctypes.c_void_p(t.data_ptr()) for t in outs), ctypes.c_void_p(gates.data_ptr()),
+                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == mok.MOK_OK, mok.last_error()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
