@@ -200,8 +200,8 @@ def algorithmic_work(cfg):
         # values; slot outputs bf16
         el, slot = 1.0 + 1.0 / 32, 2.0
     else:
-        # bf16 weights, rows and h; slot outputs fp32
-        el, slot = 2.0, 4.0
+        # bf16 weights, rows and h; slot outputs fp16 with one exponent byte per 128 values
+        el, slot = 2.0, 2.0 + 1.0 / 128
     w_bytes = cfg.E * 3 * cfg.H * cfg.I * el
     gemm_bytes = w_bytes + ns * cfg.H * el + 2 * ns * cfg.I * el + ns * cfg.H * slot  # weights, rows, h out+in, slots
     gather_bytes = cfg.T * cfg.H * 2 + ns * cfg.H * el
@@ -278,7 +278,9 @@ def time_steps(wl: Workload, mode: str, steps: int, warmup: int, minibatch: int,
             bufs["ffn_ws"] = torch.empty(mok.lib().mok_expert_ffn_mxfp8_workspace_bytes(cfg.slots, cfg.I, cfg.E),
                                          dtype=torch.uint8, device=device)
         else:
-            bufs["out"] = torch.empty((cfg.slots, cfg.H), dtype=torch.float32, device=device)
+            # slot rows as MOK_SLOTS_F16S: fp16 values plus one exponent per 128 features
+            bufs["out"] = torch.empty(mok.lib().mok_slot_bytes(cfg.slots, cfg.H, mok.MOK_SLOTS_F16S),
+                                      dtype=torch.uint8, device=device)
             bufs["rows"] = torch.empty((cfg.slots, cfg.H), dtype=torch.bfloat16, device=device)
             bufs["ffn_ws"] = torch.empty(mok.lib().mok_expert_ffn_workspace_bytes(cfg.slots, cfg.I, cfg.E),
                                          dtype=torch.uint8, device=device)
@@ -432,7 +434,7 @@ def time_router(wl: Workload, steps: int, warmup: int):
 def backward_work(cfg):
     """Algorithmic bytes / flops of one backward (bf16 path)."""
     ns, H, I, E, T = cfg.slots, cfg.H, cfg.I, cfg.E, cfg.T
-    rc = T * H * 2 + ns * H * 4 + ns * H * 2 + T * E * 4            # dy, fp32 slots in; do rows, dlogits out
+    rc = T * H * 2 + ns * H * (2 + 1 / 128) + ns * H * 2 + T * E * 4  # dy, slot rows in; do rows, dlogits out
     dh = E * I * H * 2 + ns * H * 2 + 2 * ns * I * 2 + 2 * ns * I * 2  # Wd, do; a, b in; da, db out
     dx = 2 * E * H * I * 2 + 2 * ns * I * 2 + ns * H * 4            # Wg, Wu, da, db in; fp32 dx rows out
     rd = ns * H * 4 + T * H * 2                                      # dx rows in, dx out
@@ -609,9 +611,11 @@ def main():
                     help="persistent mode: least rows per minibatch (0: the two-wave rule alone; "
                          "default: the configuration's)")
     ap.add_argument("--dispatch-ctas", type=int, default=0,
-                    help="persistent mode: CTAs on the dispatch side (0: the library default, 8 bf16 / 16 MXFP8)")
+                    help="persistent mode: CTAs on the dispatch side (0: the library default, 6 bf16 / 16 MXFP8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub-records", action="store_true", help="time only the main workload")
+    ap.add_argument("--backward", action="store_true",
+                    help="time only mok_moe_backward on the workload (after one staged forward that keeps a, b)")
     ap.add_argument("--cpu-steps", type=int, default=64, help="experts the CPU baseline samples")
     ap.add_argument("--scale-experts", type=int, default=0,
                     help="profiling case: E experts and T scaled by the same factor (same rows per expert)")
@@ -633,7 +637,7 @@ def main():
              else "bf16 weights [E,H,I]/[E,I,H]")
     config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
               "tokens_per_step_per_gpu": cfg.T, "mode": args.mode,
-              **({"minibatch": minibatch, "dispatch_ctas": args.dispatch_ctas or (16 if cfg.mxfp8 else 8)}
+              **({"minibatch": minibatch, "dispatch_ctas": args.dispatch_ctas or (16 if cfg.mxfp8 else 6)}
                  if args.mode == "persistent" else {}),
               "l2": f"inputs larger than L2 ({algorithmic_work(cfg)['weight_bytes'] / 1e9:.1f} GB of expert "
                     f"weights streamed per step)"}
@@ -657,6 +661,13 @@ def main():
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     wl = Workload(cfg, device)
+    if args.backward:
+        if rank == 0:
+            bw = time_backward(wl, args.steps, args.warmup)
+            peaks, _ = load_peaks()
+            bw["frac_of_hbm"] = bw["GBps"] / peaks["hbm_gbs"]
+            print(json.dumps(bw), flush=True)
+        return 0
     res = time_steps(wl, args.mode, args.steps, args.warmup, minibatch, args.dispatch_ctas, world)
     e2e = time_e2e(wl, args.mode, args.steps, minibatch, world)
     subs = {}

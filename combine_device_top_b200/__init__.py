@@ -32,6 +32,7 @@ MOK_MODE_STAGED = 1
 MOK_MAX_SHARDS = 64
 MOK_SLOTS_F32 = 0
 MOK_SLOTS_BF16 = 1
+MOK_SLOTS_F16S = 2
 
 # every entry point of include/mok.h
 EXPORTS = (
@@ -42,7 +43,7 @@ EXPORTS = (
     "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8_workspace_bytes", "mok_expert_ffn_mxfp8",
     "mok_two_wave_rows", "mok_minibatch_bounds", "mok_forward_host_batches_workspace_bytes",
     "mok_moe_forward_host_batches", "mok_router_weights_bytes", "mok_router_prepare", "mok_plan_router",
-    "mok_backward_workspace_bytes", "mok_moe_backward",
+    "mok_backward_workspace_bytes", "mok_moe_backward", "mok_slot_bytes", "mok_slot_exp_offset",
 )
 
 
@@ -100,6 +101,10 @@ def lib() -> ctypes.CDLL:
     L.mok_expert_ffn_mxfp8_workspace_bytes.restype = sz
     L.mok_expert_ffn_mxfp8.argtypes = [vp, vp, i32, i32, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp]
     L.mok_two_wave_rows.argtypes = [i32, i32, i32, i32]
+    L.mok_slot_bytes.argtypes = [i32, i32, i32]
+    L.mok_slot_bytes.restype = sz
+    L.mok_slot_exp_offset.argtypes = [i32, i32]
+    L.mok_slot_exp_offset.restype = sz
     L.mok_backward_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
     L.mok_backward_workspace_bytes.restype = sz
     L.mok_moe_backward.argtypes = [vp, i32, i32, vp, vp, vp, ctypes.POINTER(PlanT), vp, sz, vp, vp, vp, vp, vp, vp, sz,
@@ -441,14 +446,16 @@ def expert_ffn_mxfp8(rows_q, scales, pack, p: Plan, out: torch.Tensor | None = N
 
 
 def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = None, ws=None, stream=None):
-    """Grouped SwiGLU FFN over expert-major rows; returns (out [T*k, H] fp32 slot-indexed, ws)."""
+    """Grouped SwiGLU FFN over expert-major rows; returns (out, ws): ``out`` is
+    the slot-indexed MOK_SLOTS_F16S buffer (uint8, ``mok_slot_bytes`` bytes:
+    [T*k, H] fp16, then [T*k, H/128] int8 block exponents)."""
     H = rows.shape[1]
     I = w_gate.shape[-1]
     for w in (w_gate, w_up, w_down):
         assert w.dtype == torch.bfloat16, "the weights are bf16"
     if out is None:
-        out = torch.empty((p.ns, H), dtype=torch.float32, device=rows.device)
-    assert out.dtype == torch.float32
+        out = torch.empty(lib().mok_slot_bytes(p.ns, H, MOK_SLOTS_F16S), dtype=torch.uint8, device=rows.device)
+    assert out.dtype == torch.uint8 and out.numel() >= lib().mok_slot_bytes(p.ns, H, MOK_SLOTS_F16S)
     if ws is None:
         ws = _workspace(lib().mok_expert_ffn_workspace_bytes(p.ns, I, p.c.E), rows.device)
     _check(lib().mok_expert_ffn(ctypes.c_void_p(rows.data_ptr()), H, I, ctypes.c_void_p(w_gate.data_ptr()),
@@ -459,11 +466,11 @@ def expert_ffn(rows, w_gate, w_up, w_down, p: Plan, out: torch.Tensor | None = N
 
 
 def combine(out: torch.Tensor, p: Plan, y_shards, stream=None):
-    """y = fixed-order gate-weighted sum of the per-slot outputs (fp32, or bf16 on the MXFP8 path;
-    fp32 accumulation)."""
-    assert out.dtype in (torch.float32, torch.bfloat16) and len(y_shards) == p.c.R
-    H = out.shape[-1]
-    dt = MOK_SLOTS_F32 if out.dtype == torch.float32 else MOK_SLOTS_BF16
+    """y = fixed-order gate-weighted sum of the per-slot outputs, fp32 accumulation.  ``out``: fp32
+    or bf16 [T*k, H], or a uint8 MOK_SLOTS_F16S buffer (then ``H`` comes from the y shards)."""
+    assert out.dtype in (torch.float32, torch.bfloat16, torch.uint8) and len(y_shards) == p.c.R
+    H = y_shards[0].shape[-1]
+    dt = {torch.float32: MOK_SLOTS_F32, torch.bfloat16: MOK_SLOTS_BF16, torch.uint8: MOK_SLOTS_F16S}[out.dtype]
     _check(lib().mok_combine(ctypes.c_void_p(out.data_ptr()), dt, H, ctypes.byref(p.c), _ptr_array(y_shards),
                              _stream(stream)))
     return y_shards

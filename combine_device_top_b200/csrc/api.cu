@@ -169,10 +169,11 @@ struct FwdLayout {
 static const uint64_t kDefaultTimeoutNs = 2000000000ull;
 // Dispatch CTAs of the persistent kernel by default.  On the bf16 path one
 // thread per CTA streams rows with bulk copies (about 200 KB in flight, some
-// 30 GB/s per CTA measured); at the page shape 2, 4, 8 and 16 CTAs gave
-// 15.7, 9.7, 8.0 and 8.4 ms per forward on B200 (one session).  The MXFP8
-// path quantises with every warp of its CTAs (16 measured best).
-static const int kDefaultDispatchBf16 = 8;
+// 30 GB/s per CTA measured); at the page shape on B200, 2, 4, 8 and 16 CTAs
+// gave 15.7, 9.7, 8.0 and 8.4 ms per forward in one session, and 5, 6, 7
+// and 8 gave 8.61, 7.87, 7.90 and 7.93 ms in another.  The MXFP8 path
+// quantises with every warp of its CTAs (16 measured best).
+static const int kDefaultDispatchBf16 = 6;
 
 static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const mok_fwd_opts* o, FwdLayout* L) {
     if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return false;
@@ -219,7 +220,7 @@ static bool fwd_layout(int T, int H, int I, int E, int k, int minibatch, const m
         l.rows = take((size_t)l.buf_rows * H * 2);
         l.h = take((size_t)l.buf_rows * I * 2);
     }
-    l.out = take((size_t)ns * H * (l.mx ? 2 : 4));  // slot outputs: fp32, or bf16 on the MXFP8 path
+    l.out = take(slot_bytes((size_t)ns, H, l.mx ? MOK_SLOTS_BF16 : MOK_SLOTS_F16S));  // slot outputs
     // kept for the backward (staged bf16 path): gate and up pre-activations
     l.save = (o && o->save_for_backward) ? 1 : 0;
     if (l.save) {
@@ -292,8 +293,9 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
     MOK_CUDA(launch_gemm_phase(0, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
                                tune, stream, save),
              "gate/up GEMM launch");
+    int8_t* out_exp = mxw ? nullptr : reinterpret_cast<int8_t*>(out) + slot_exp_offset((size_t)n_rows_buf, H);
     MOK_CUDA(launch_gemm_phase(1, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
-                               tune, stream),
+                               tune, stream, nullptr, out_exp),
              "down GEMM launch");
     return MOK_OK;
 }
@@ -355,6 +357,18 @@ int mok_plan(const float* logits, int T, int E, int top_k, int R, void* ws, size
     if (device_sms(nullptr) <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     MOK_CUDA(launch_plan(logits, T, E, top_k, R, base, L, reinterpret_cast<cudaStream_t>(stream)), "plan launch");
     return MOK_OK;
+}
+
+size_t mok_slot_bytes(int n_slots, int H, int slot_type) {
+    if (n_slots < 0 || H <= 0 || (slot_type != MOK_SLOTS_F32 && slot_type != MOK_SLOTS_BF16 &&
+                                  slot_type != MOK_SLOTS_F16S))
+        return 0;
+    if (slot_type == MOK_SLOTS_F16S && H % 128) return 0;
+    return slot_bytes((size_t)n_slots, H, slot_type);
+}
+
+size_t mok_slot_exp_offset(int n_slots, int H) {
+    return (n_slots < 0 || H <= 0) ? 0 : slot_exp_offset((size_t)n_slots, H);
 }
 
 size_t mok_router_weights_bytes(int H, int E) {
@@ -658,7 +672,8 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
                         base + L.h, base + L.out, F.status, F.timeout, stream, mxw, mxw ? &mxs : nullptr,
                         L.save ? &save : nullptr);
     if (rc) return rc;
-    MOK_CUDA(launch_combine(base + L.out, mxw != nullptr, plan->gates, T, k, H, T / R, ys, sms, stream),
+    MOK_CUDA(launch_combine(base + L.out, mxw ? MOK_SLOTS_BF16 : MOK_SLOTS_F16S, plan->gates, T, k, H, T / R, ys,
+                            sms, stream),
              "combine launch");
     return MOK_OK;
 }
@@ -721,7 +736,9 @@ int mok_moe_backward(const void* const* dy_shards, int H, int I, const void* w_g
     MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
     // 1. pull reverse-combine: do rows, gate gradients, dlogits
     MOK_CUDA(launch_reverse_combine(dys, T / R, H, T, k, E, plan->pos, plan->gates, plan->topk_idx,
-                                    reinterpret_cast<const float*>(fb + FL.out), do_rows, dlogits, sms, stream),
+                                    reinterpret_cast<const uint16_t*>(fb + FL.out),
+                                    reinterpret_cast<const int8_t*>(fb + FL.out + slot_exp_offset(ns, H)), do_rows,
+                                    dlogits, sms, stream),
              "reverse combine launch");
     // 2. dh = do Wd^T with the SwiGLU backward -> [da | db]; 3. dx rows = da Wg^T + db Wu^T -> slots
     MOK_CUDA(gemm_configure(dev), "gemm configure");
@@ -749,7 +766,8 @@ int mok_moe_backward(const void* const* dy_shards, int H, int I, const void* w_g
                                status, kDefaultTimeoutNs, sms, tune, stream, &bb),
              "dx GEMM launch");
     // 4. push reverse-dispatch: dx_t = sum of its k rows (the combine with unit weights)
-    MOK_CUDA(launch_combine(dx_slots, false, nullptr, T, k, H, T / R, dxs, sms, stream), "reverse dispatch launch");
+    MOK_CUDA(launch_combine(dx_slots, MOK_SLOTS_F32, nullptr, T, k, H, T / R, dxs, sms, stream),
+             "reverse dispatch launch");
     // 5. weight gradients per expert over its rows
     cudaError_t e = launch_wgrad(fb + FL.rows, fb + FL.h, do_rows, dab, (int)ns, plan->offsets, H, I, E, dw_gate,
                                  dw_up, dw_down, status, kDefaultTimeoutNs, sms, &err, stream);
@@ -927,9 +945,10 @@ int mok_combine(const void* out, int out_dtype, int H, const mok_plan_t* plan, v
                 mok_stream_t stream) {
     int rc = check_plan(plan);
     if (rc) return rc;
-    if (out_dtype != MOK_SLOTS_F32 && out_dtype != MOK_SLOTS_BF16)
+    if (out_dtype != MOK_SLOTS_F32 && out_dtype != MOK_SLOTS_BF16 && out_dtype != MOK_SLOTS_F16S)
         return fail(MOK_ERR_INVALID_ARG, "unknown slot dtype %d", out_dtype);
     if (H <= 0 || H % 8) return fail(MOK_ERR_UNSUPPORTED, "H %% 8 != 0");
+    if (out_dtype == MOK_SLOTS_F16S && H % 128) return fail(MOK_ERR_UNSUPPORTED, "H %% 128 != 0 (fp16 slot rows)");
     if (plan->T == 0) return MOK_OK;
     if (!out || !all_nonnull(y_shards, plan->R)) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
     if (!all_aligned16(y_shards, plan->R) || (reinterpret_cast<uintptr_t>(out) & 15u))
@@ -938,8 +957,8 @@ int mok_combine(const void* out, int out_dtype, int H, const mok_plan_t* plan, v
     for (int r = 0; r < plan->R; ++r) ys.p[r] = y_shards[r];
     const int sms = device_sms(nullptr);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
-    MOK_CUDA(launch_combine(out, out_dtype == MOK_SLOTS_BF16, plan->gates, plan->T, plan->k, H, plan->T / plan->R,
-                            ys, sms, reinterpret_cast<cudaStream_t>(stream)),
+    MOK_CUDA(launch_combine(out, out_dtype, plan->gates, plan->T, plan->k, H, plan->T / plan->R, ys, sms,
+                            reinterpret_cast<cudaStream_t>(stream)),
              "combine launch");
     return MOK_OK;
 }

@@ -23,14 +23,15 @@ namespace mok {
 // One warp per token: dy_t is read once (16-byte vectors, 8 features per
 // lane); for each of its k slots the warp writes the bf16 row do = g dy_t to
 // the slot's expert-major row and accumulates <dy_t, o_slot> from the
-// forward's fp32 slot outputs; then the softmax backward over the k gates
+// forward's slot rows (fp16 with block exponents); then the softmax backward over the k gates
 // gives the token's dlogits row (zeros outside its selection).
 template <int KB>
 __global__ void __launch_bounds__(256) k_reverse_combine(ShardsIn dys, int S_r, int H, int T, int k, int E,
                                                          const int32_t* __restrict__ pos,
                                                          const float* __restrict__ gates,
                                                          const int32_t* __restrict__ topk_idx,
-                                                         const float* __restrict__ o_slots,
+                                                         const uint16_t* __restrict__ o_slots,
+                                                         const int8_t* __restrict__ o_exps,
                                                          uint4* __restrict__ do_rows, float* __restrict__ dlogits) {
     const int lane = threadIdx.x & 31;
     const int nvec = H >> 3;
@@ -61,10 +62,18 @@ __global__ void __launch_bounds__(256) k_reverse_combine(ShardsIn dys, int S_r, 
 #pragma unroll
             for (int j = 0; j < KB; ++j) {
                 if (j < k) {
-                    const float4* o = reinterpret_cast<const float4*>(o_slots + ((size_t)t * k + j) * H) + 2 * v;
-                    const float4 o0 = __ldcs(o), o1 = __ldcs(o + 1);
-                    dgp[j] += d[0] * o0.x + d[1] * o0.y + d[2] * o0.z + d[3] * o0.w + d[4] * o1.x + d[5] * o1.y +
-                              d[6] * o1.z + d[7] * o1.w;
+                    // the forward's slot row: fp16 values, one power-of-two exponent per 128 features
+                    const size_t slot = (size_t)t * k + j;
+                    const uint4 ov = __ldcs(reinterpret_cast<const uint4*>(o_slots + slot * H) + v);
+                    const float sc = __int_as_float(((int)__ldg(o_exps + slot * (H >> 7) + (v >> 4)) + 127) << 23);
+                    const __half2* oh = reinterpret_cast<const __half2*>(&ov);
+                    float acc = 0.f;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 of = __half22float2(oh[p]);
+                        acc += d[2 * p] * of.x + d[2 * p + 1] * of.y;
+                    }
+                    dgp[j] += acc * sc;
                     const float g = gs[j];
                     do_rows[(size_t)rows[j] * nvec + v] =
                         make_uint4(pack_bf16x2(g * d[0], g * d[1]), pack_bf16x2(g * d[2], g * d[3]),
@@ -92,19 +101,22 @@ __global__ void __launch_bounds__(256) k_reverse_combine(ShardsIn dys, int S_r, 
 }
 
 cudaError_t launch_reverse_combine(const ShardsIn& dys, int S_r, int H, int T, int k, int E, const int32_t* pos,
-                                   const float* gates, const int32_t* topk_idx, const float* o_slots, void* do_rows,
-                                   float* dlogits, int num_sms, cudaStream_t stream) {
+                                   const float* gates, const int32_t* topk_idx, const uint16_t* o_slots,
+                                   const int8_t* o_exps, void* do_rows, float* dlogits, int num_sms,
+                                   cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
     const int want = (T + 7) / 8;
     const int grid = want < num_sms * 8 ? want : num_sms * 8;
     uint4* d = reinterpret_cast<uint4*>(do_rows);
     if (k <= 2)
-        k_reverse_combine<2><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, d, dlogits);
+        k_reverse_combine<2><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, o_exps, d,
+                                                       dlogits);
     else if (k <= 8)
-        k_reverse_combine<8><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, d, dlogits);
+        k_reverse_combine<8><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, o_exps, d,
+                                                       dlogits);
     else
-        k_reverse_combine<32><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, d,
-                                                        dlogits);
+        k_reverse_combine<32><<<grid, 256, 0, stream>>>(dys, S_r, H, T, k, E, pos, gates, topk_idx, o_slots, o_exps,
+                                                        d, dlogits);
     return cudaGetLastError();
 }
 

@@ -99,15 +99,15 @@ cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, c
 }
 
 template <int KMAX, class S>
-__global__ void __launch_bounds__(DC_THREADS) k_combine(const void* __restrict__ out, const float* __restrict__ gates,
-                                                        int T, int k, int H, int S_r, ShardsOut ys) {
+__global__ void __launch_bounds__(DC_THREADS) k_combine(SlotSrc src, const float* __restrict__ gates, int T, int k,
+                                                        int H, int S_r, ShardsOut ys) {
     const int lane = threadIdx.x & 31;
     const int nvec = H >> 3;
     const int warps = gridDim.x * (DC_THREADS / 32);
     for (int t = blockIdx.x * (DC_THREADS / 32) + (threadIdx.x >> 5); t < T; t += warps) {
         const int r = t / S_r;
         uint4* dst = reinterpret_cast<uint4*>(ys.p[r]) + (size_t)(t - r * S_r) * nvec;
-        warp_combine_token<KMAX, S>(out, gates, t, k, nvec, dst, lane);
+        warp_combine_token<KMAX, S>(src, gates, t, k, nvec, dst, lane);
     }
 }
 
@@ -121,27 +121,32 @@ cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, cons
 }
 
 template <class S>
-static void launch_combine_t(const void* out, const float* gates, int T, int k, int H, int S_r, const ShardsOut& ys,
-                             int grid, cudaStream_t stream) {
-    // KB slots' loads in flight per lane: all of them up to 8 (fp32 slots:
-    // 2 x 16 bytes each); k > 8 takes several rounds
+static void launch_combine_t(const SlotSrc& src, const float* gates, int T, int k, int H, int S_r,
+                             const ShardsOut& ys, int grid, cudaStream_t stream) {
+    // KB slots' loads in flight per lane: all of them up to 8; k > 8 takes
+    // several rounds
     if (k <= 2)
-        k_combine<2, S><<<grid, DC_THREADS, 0, stream>>>(out, gates, T, k, H, S_r, ys);
+        k_combine<2, S><<<grid, DC_THREADS, 0, stream>>>(src, gates, T, k, H, S_r, ys);
     else if (k <= 4)
-        k_combine<4, S><<<grid, DC_THREADS, 0, stream>>>(out, gates, T, k, H, S_r, ys);
+        k_combine<4, S><<<grid, DC_THREADS, 0, stream>>>(src, gates, T, k, H, S_r, ys);
     else
-        k_combine<8, S><<<grid, DC_THREADS, 0, stream>>>(out, gates, T, k, H, S_r, ys);
+        k_combine<8, S><<<grid, DC_THREADS, 0, stream>>>(src, gates, T, k, H, S_r, ys);
 }
 
-cudaError_t launch_combine(const void* out, bool slots_bf16, const float* gates, int T, int k, int H, int S_r,
+cudaError_t launch_combine(const void* out, int slot_type, const float* gates, int T, int k, int H, int S_r,
                            const ShardsOut& ys, int num_sms, cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
     const int want = (T + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     const int grid = want < num_sms * 8 ? want : num_sms * 8;
-    if (slots_bf16)
-        launch_combine_t<SlotBf16>(out, gates, T, k, H, S_r, ys, grid, stream);
-    else
-        launch_combine_t<SlotF32>(out, gates, T, k, H, S_r, ys, grid, stream);
+    SlotSrc src{out, nullptr};
+    if (slot_type == MOK_SLOTS_F16S) {
+        src.exps = reinterpret_cast<const int8_t*>(out) + slot_exp_offset(T * k, H);
+        launch_combine_t<SlotF16S>(src, gates, T, k, H, S_r, ys, grid, stream);
+    } else if (slot_type == MOK_SLOTS_BF16) {
+        launch_combine_t<SlotBf16>(src, gates, T, k, H, S_r, ys, grid, stream);
+    } else {
+        launch_combine_t<SlotF32>(src, gates, T, k, H, S_r, ys, grid, stream);
+    }
     return cudaGetLastError();
 }
 

@@ -113,17 +113,22 @@ __device__ __forceinline__ void warp_mx_quant8(const uint4& raw, uint2& q, uint3
            (__shfl_sync(0xffffffffu, sb, h0 + 8) << 16) | (__shfl_sync(0xffffffffu, sb, h0 + 12) << 24);
 }
 
-// Slot outputs as the grouped GEMM stores them: fp32 (bf16 path) or bf16
-// (MXFP8 path).  A lane owns 8 consecutive features of a slot row (v = index
-// of the 8-feature group): load() issues the raw 16-byte loads, widen()
-// turns them into 8 floats.  The combine issues every load of a round
-// before it widens any, so all of them are in flight together.
+// Slot outputs as the grouped GEMM stores them: fp16 with one exponent per
+// 128-feature block of a row (bf16 path, SlotF16S), bf16 (MXFP8 path) or
+// fp32 (the backward's dx rows).  A lane owns 8 consecutive features of a
+// slot row (v = index of the 8-feature group, block v / 16): load() issues
+// the raw loads, widen() turns them into 8 floats.  The combine issues every
+// load of a round before it widens any, so all of them are in flight.
+struct SlotSrc {
+    const void* out;     // [N_s, H] slot rows
+    const int8_t* exps;  // SlotF16S: [N_s, H/128] block exponents
+};
 struct SlotF32 {
     struct Raw {
         float4 a, b;
     };
-    __device__ static __forceinline__ Raw load(const void* out, size_t row, int nvec, int v) {
-        const float4* p = reinterpret_cast<const float4*>(out) + (row * nvec + v) * 2;
+    __device__ static __forceinline__ Raw load(const SlotSrc& s, size_t row, int nvec, int v) {
+        const float4* p = reinterpret_cast<const float4*>(s.out) + (row * nvec + v) * 2;
         return Raw{__ldcs(p), __ldcs(p + 1)};
     }
     __device__ static __forceinline__ void widen(const Raw& r, float (&f)[8]) {
@@ -133,8 +138,8 @@ struct SlotF32 {
 };
 struct SlotBf16 {
     using Raw = uint4;
-    __device__ static __forceinline__ Raw load(const void* out, size_t row, int nvec, int v) {
-        return __ldcs(reinterpret_cast<const uint4*>(out) + row * nvec + v);
+    __device__ static __forceinline__ Raw load(const SlotSrc& s, size_t row, int nvec, int v) {
+        return __ldcs(reinterpret_cast<const uint4*>(s.out) + row * nvec + v);
     }
     __device__ static __forceinline__ void widen(const Raw& r, float (&f)[8]) {
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&r);
@@ -146,6 +151,26 @@ struct SlotBf16 {
         }
     }
 };
+struct SlotF16S {
+    struct Raw {
+        uint4 v;
+        int e;
+    };
+    __device__ static __forceinline__ Raw load(const SlotSrc& s, size_t row, int nvec, int v) {
+        return Raw{__ldcs(reinterpret_cast<const uint4*>(s.out) + row * nvec + v),
+                   (int)__ldg(s.exps + row * (size_t)(nvec >> 4) + (v >> 4))};
+    }
+    __device__ static __forceinline__ void widen(const Raw& r, float (&f)[8]) {
+        const __half2* h2 = reinterpret_cast<const __half2*>(&r.v);
+        const float sc = __int_as_float((r.e + 127) << 23);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 x = __half22float2(h2[p]);
+            f[2 * p] = x.x * sc;
+            f[2 * p + 1] = x.y * sc;
+        }
+    }
+};
 
 // One warp: y[t] = bf16(sum_{j<k} g[t,j] * out[t,j,:]) in fp32, j ascending
 // (gates == nullptr: every g = 1, the backward's reverse-dispatch sum).
@@ -154,8 +179,8 @@ struct SlotBf16 {
 // (KB loads in flight), then accumulated in order; k > KB takes several
 // rounds of KB.
 template <int KB, class S>
-__device__ __forceinline__ void warp_combine_token(const void* __restrict__ out, const float* __restrict__ gates,
-                                                   int t, int k, int nvec, uint4* __restrict__ dst, int lane) {
+__device__ __forceinline__ void warp_combine_token(const SlotSrc& src, const float* __restrict__ gates, int t, int k,
+                                                   int nvec, uint4* __restrict__ dst, int lane) {
     const size_t row0 = (size_t)t * k;
     const float* gt = gates ? gates + row0 : nullptr;
     // lanes may run different numbers of iterations (nvec % 32 != 0): no
@@ -170,7 +195,7 @@ __device__ __forceinline__ void warp_combine_token(const void* __restrict__ out,
                 const int j = j0 + jj;
                 if (j < k) {
                     g[jj] = gates ? __ldg(gt + j) : 1.f;
-                    raw[jj] = S::load(out, row0 + j, nvec, v);
+                    raw[jj] = S::load(src, row0 + j, nvec, v);
                 }
             }
 #pragma unroll

@@ -72,9 +72,15 @@ constexpr int MT_D_FEATURES = 128;                // down unit: 128 output colum
 // bf16 path, pairs of M tiles sharing the token tile: [A0 16 KB][A1 16 KB]
 // [B 32 KB] x 3.  MXFP8 path: [A bf16, converted 16 KB][B 32 KB][A E4M3
 // bytes 8 KB][scales 1 KB] x 3.
-template <int SUB_, int NST_>
+// EXT_: the instantiation that also runs the backward phases (2, 3) and
+// keeps the forward's gate/up pre-activations; the plain forward
+// instantiations compile none of that code (measured: folding it into
+// the forward kernels cost 12 % of the page-shape GEMM, in the
+// single-thread TMA and MMA issue loops).
+template <int SUB_, int NST_, bool EXT_ = false>
 struct Bf16CfgT {
     static constexpr bool MX = false;
+    static constexpr bool EXT = EXT_;
     static constexpr int SUB = SUB_;  // M tiles per unit
     static constexpr int THREADS = 320;  // warps: 0 TMA, 1 MMA, 2-9 two epilogue groups
     static constexpr int NST = NST_;
@@ -87,6 +93,8 @@ struct Bf16CfgT {
 };
 using Bf16Cfg = Bf16CfgT<1, 4>;
 using Bf16PairCfg = Bf16CfgT<2, 3>;
+using Bf16ExtCfg = Bf16CfgT<1, 4, true>;
+using Bf16ExtPairCfg = Bf16CfgT<2, 3, true>;
 static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share the barrier offset");
 // MXFP8 path (block-scaled tcgen05 MMA, K = 128 per stage), SUB weight
 // tiles per unit: [A E4M3 SUB x 16 KB][B E4M3 <= 224 rows x 128 B][A scales
@@ -95,6 +103,7 @@ static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share
 template <int SUB_, int NST_>
 struct MxCfgT {
     static constexpr bool MX = true;
+    static constexpr bool EXT = false;
     static constexpr int SUB = SUB_;
     static constexpr int THREADS = 352;  // warps: 0 TMA, 1 MMA, 2-9 epilogue, 10 scale-factor layout
     static constexpr int NST = NST_;
@@ -133,7 +142,9 @@ struct Unit {
 struct CoreArgs {
     int H, I;
     void* h;                  // [buffer rows, I]: bf16 (bf16 path) or E4M3 (MXFP8 path)
-    void* out;                // [N_s, H] slot-indexed: fp32 (bf16 path) or bf16 (MXFP8 path)
+    void* out;                // [N_s, H] slot-indexed: fp16 + block exponents (bf16 path), bf16
+                              // (MXFP8 path), fp32 (backward dx rows)
+    int8_t* out_exp;          // bf16 path: [N_s, H/128] exponents of the fp16 slot rows
     const int32_t* row_slot;  // [N_s]
     DevStatus* st;
     uint64_t timeout_ns;
@@ -196,16 +207,24 @@ struct StagedSched {
 // Backward phases (bf16 path): 2 = dh = do Wd^T with the SwiGLU backward
 // in the epilogue (M = I features), 3 = dx rows = da Wg^T + db Wu^T pushed
 // to the token slots (M = H features); both read A K-major.
+template <class C>
 __device__ __forceinline__ int phase_tiles(const CoreArgs& a, int phase) {
-    return phase == 0 ? a.I / MT_G_FEATURES : phase == 2 ? a.I / MT_D_FEATURES : a.H / MT_D_FEATURES;
+    if constexpr (C::EXT)
+        return phase == 0 ? a.I / MT_G_FEATURES : phase == 2 ? a.I / MT_D_FEATURES : a.H / MT_D_FEATURES;
+    else
+        return phase == 0 ? a.I / MT_G_FEATURES : a.H / MT_D_FEATURES;
 }
 // Contraction length of a phase.
+template <class C>
 __device__ __forceinline__ int phase_k(const CoreArgs& a, int phase) {
-    return phase == 0 || phase == 2 ? a.H : phase == 1 ? a.I : 2 * a.I;
+    if constexpr (C::EXT)
+        return phase == 0 || phase == 2 ? a.H : phase == 1 ? a.I : 2 * a.I;
+    else
+        return phase == 0 ? a.H : a.I;
 }
 template <class C>
 __device__ __forceinline__ int unit_subs(const CoreArgs& a, const Unit& u) {
-    return min(C::SUB, phase_tiles(a, u.phase) - u.m * C::SUB);
+    return min(C::SUB, phase_tiles<C>(a, u.phase) - u.m * C::SUB);
 }
 
 // Token tile of a unit: one box of the 16-rounded row count.  Returns the
@@ -225,9 +244,9 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
         if (!s.wait_inputs(u, a.st, a.timeout_ns)) break;
-        const int K = phase_k(a, u.phase);
+        const int K = phase_k<C>(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
-        const BMaps& bm = (u.phase == 0 || u.phase == 2) ? maps.rows : maps.h;
+        const BMaps& bm = (u.phase == 0 || (C::EXT && u.phase == 2)) ? maps.rows : maps.h;
         const int bx = token_box(u.rows);
         const int nsub = unit_subs<C>(a, u);
         uint32_t bytes = (uint32_t)(16 * (bx + 1)) * B_ROW_BYTES;
@@ -275,11 +294,11 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
                         tma_load_2d_hint(sa, &maps.wg, &full[stage], mt * MT_G_FEATURES, ky, evict_first);
                         tma_load_2d_hint(sa + A_BYTES / 2, &maps.wu, &full[stage], mt * MT_G_FEATURES, ky,
                                          evict_first);
-                    } else if (u.phase == 2) {
+                    } else if (C::EXT && u.phase == 2) {
                         // Wd [E*I, H] K-major: 128 feature rows x 64 K in one box
                         tma_load_2d_hint(sa, &maps.wd, &full[stage], kb * BK, u.expert * a.I + mt * MT_D_FEATURES,
                                          evict_first);
-                    } else if (u.phase == 3) {
+                    } else if (C::EXT && u.phase == 3) {
                         // Wg then Wu [E*H, I] K-major: K runs over I twice
                         const int KI = a.I / BK;
                         const bool up = kb >= KI;
@@ -330,7 +349,7 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
     uint32_t phase = 0;
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
-        const int K = phase_k(a, u.phase);
+        const int K = phase_k<C>(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
         const int nsub = unit_subs<C>(a, u);
         const int lead = u.brow0 & 3;
@@ -407,14 +426,14 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
     uint32_t tk = 0;  // next accumulator ticket
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
-        const int K = phase_k(a, u.phase);
+        const int K = phase_k<C>(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
         const int N = (u.rows + 15) & ~15;
         const int nsub = unit_subs<C>(a, u);
         const int nt = unit_tickets<C>(nsub, N);
         const bool wide = nt == 2;
         // bf16 path: every phase bf16 x bf16; A MN-major (forward) or K-major (backward)
-        const bool a_kmaj = u.phase >= 2;
+        const bool a_kmaj = C::EXT && u.phase >= 2;
         const uint32_t idesc = umma_idesc_f16(128, N, a_kmaj ? 0 : 1, /*B K-major*/ 0, /*bf16*/ 1);
         bool ok = true;
         for (int t = 0; t < nt && ok; ++t) {
@@ -559,7 +578,7 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                     const size_t at = row * a.I + mt * MT_G_FEATURES + j0;
                     if (live) {
                         *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.h) + at) = pk;
-                        if (a.save_a) {
+                        if (C::EXT && a.save_a) {
                             *reinterpret_cast<uint4*>(a.save_a + at) =
                                 make_uint4(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]),
                                            pack_bf16x2(gv[4], gv[5]), pack_bf16x2(gv[6], gv[7]));
@@ -570,7 +589,7 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                     }
                 }
             }
-        } else if (u.phase == 2) {
+        } else if (C::EXT && u.phase == 2) {
             // dh of features mt*128 + 4*lane .. +3, a warp per token: the SwiGLU backward with the
             // row's saved a, b (bf16); da and db rows pushed as bf16 into dab [rows, 2I]
 #pragma unroll 2
@@ -609,15 +628,27 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
             for (int it = 0; it < 8; ++it) {
                 const int t = it * 4 + q;
                 const int col = cc * 32 + t;
-                if (col < u.rows) {
+                if (col < u.rows) {  // warp-uniform: t depends on the warp only
                     const int slot = __ldg(a.row_slot + u.grow0 + col);
                     const float4 o4 = *reinterpret_cast<const float4*>(epi + t * EPI_TLD + 4 * lane);
                     const size_t at = (size_t)slot * a.H + mt * MT_D_FEATURES;
-                    if constexpr (C::MX)
+                    if constexpr (C::MX) {
                         reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + at)[lane] =
                             make_uint2(pack_bf16x2(o4.x, o4.y), pack_bf16x2(o4.z, o4.w));
-                    else
+                    } else if constexpr (C::EXT) {
+                        // backward dx rows (phase 3): fp32
                         reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + at)[lane] = o4;
+                    } else {
+                        // fp16 with one exponent for the row's 128 features of this tile
+                        float m = fmaxf(fmaxf(fabsf(o4.x), fabsf(o4.y)), fmaxf(fabsf(o4.z), fabsf(o4.w)));
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                        const int sx = slot_block_exponent(m);
+                        const float inv = pow2f(-sx);
+                        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + at)[lane] =
+                            make_uint2(pack_half2(o4.x * inv, o4.y * inv), pack_half2(o4.z * inv, o4.w * inv));
+                        if (lane == 0) a.out_exp[(size_t)slot * (a.H / MT_D_FEATURES) + mt] = (int8_t)sx;
+                    }
                 }
             }
         }

@@ -48,6 +48,12 @@ cudaError_t gemm_configure(int dev) {
                                  Bf16PairCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm<MxCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, MxCfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm<Bf16ExtCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Bf16ExtCfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm<Bf16ExtPairCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Bf16ExtPairCfg::SMEM);
 
     if (e == cudaSuccess) done[dev] = true;
     return e;
@@ -56,7 +62,7 @@ cudaError_t gemm_configure(int dev) {
 cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const MxTokenScales* mxs,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd) {
+                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd, int8_t* out_exp) {
     if (mx && !mxs) return cudaErrorInvalidValue;
     if (phase >= 2 && (mx || !bwd || !bwd->save_a || !bwd->save_b || !bwd->dab)) return cudaErrorInvalidValue;
     CoreArgs a{};
@@ -74,6 +80,8 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.I = sh.I;
     a.h = h_out;
     a.out = out;
+    a.out_exp = out_exp;
+    if (phase == 1 && !mx && !out_exp) return cudaErrorInvalidValue;  // fp16 slot rows need their exponents
     a.row_slot = row_slot;
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
@@ -93,7 +101,16 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     } else {
         MxMaps none;
         memset(&none, 0, sizeof none);
-        if (pair)
+        // the backward phases and the forward that keeps a, b run the
+        // instantiations with that code; the plain forward runs without it
+        const bool ext = bwd != nullptr;
+        if (pair && ext)
+            k_grouped_gemm<Bf16ExtPairCfg><<<grid, Bf16ExtPairCfg::THREADS, Bf16ExtPairCfg::SMEM, stream>>>(
+                maps, none, a, chunks, counts2, phase, MT, GC);
+        else if (ext)
+            k_grouped_gemm<Bf16ExtCfg><<<grid, Bf16ExtCfg::THREADS, Bf16ExtCfg::SMEM, stream>>>(
+                maps, none, a, chunks, counts2, phase, MT, GC);
+        else if (pair)
             k_grouped_gemm<Bf16PairCfg><<<grid, Bf16PairCfg::THREADS, Bf16PairCfg::SMEM, stream>>>(
                 maps, none, a, chunks, counts2, phase, MT, GC);
         else

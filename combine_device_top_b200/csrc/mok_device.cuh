@@ -332,6 +332,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Slot rows of the bf16 path: fp16 values with one power-of-two exponent s
+// per 128-feature block of a row (value = half * 2^s).  s puts the block's
+// largest magnitude m in [2^14, 2^15): s = floor(log2 m) - 14, clamped to
+// [-126, 126] so that 2^s and 2^-s are normal floats (0 for m = 0 or a
+// non-finite m, which then stays inf / NaN).  Exact power-of-two scaling, one
+// fp16 rounding: fp16's 11 significant bits with fp32's exponent range.
+__device__ __forceinline__ int slot_block_exponent(float m) {
+    const uint32_t bits = __float_as_uint(m);
+    const int e = (int)((bits >> 23) & 0xffu);
+    if (m == 0.f || e == 0xff) return 0;
+    const int s = e - 127 - 14;
+    return s < -126 ? -126 : (s > 126 ? 126 : s);
+}
+__device__ __forceinline__ float pow2f(int s) { return __int_as_float((s + 127) << 23); }  // s in [-126, 127]
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -47,9 +47,16 @@ cudaError_t launch_gather(const ShardsIn& xs, int S_r, int H, int T, int k, cons
 // E4M3, block scales in planes [H/128][sc_rows][4] (see mx_sc_rows)
 cudaError_t launch_gather_mx(const ShardsIn& xs, int S_r, int H, int T, int k, const int32_t* pos, void* rows,
                              void* xsc, int sc_rows, int num_sms, cudaStream_t stream);
-// y = fixed-order weighted sum of the slot outputs out [T*k, H]: fp32, or
-// bf16 when slots_bf16 (the MXFP8 path)
-cudaError_t launch_combine(const void* out, bool slots_bf16, const float* gates, int T, int k, int H, int S_r,
+// Slot rows in MOK_SLOTS_F16S form: [n_slots, H] fp16, then, at this byte
+// offset, [n_slots, H/128] int8 block exponents.
+inline size_t slot_exp_offset(size_t n_slots, int H) { return (n_slots * (size_t)H * 2 + 255) & ~(size_t)255; }
+inline size_t slot_bytes(size_t n_slots, int H, int slot_type) {
+    if (slot_type == MOK_SLOTS_F16S) return slot_exp_offset(n_slots, H) + n_slots * (size_t)(H / 128);
+    return n_slots * (size_t)H * (slot_type == MOK_SLOTS_BF16 ? 2 : 4);
+}
+// y = fixed-order weighted sum of the slot outputs out [T*k, H] of type
+// slot_type (MOK_SLOTS_*); gates == nullptr: unit weights
+cudaError_t launch_combine(const void* out, int slot_type, const float* gates, int T, int k, int H, int S_r,
                            const ShardsOut& ys, int num_sms, cudaStream_t stream);
 
 // ---- work decomposition of the grouped GEMM
@@ -152,7 +159,8 @@ struct BwdBuffers {
 cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const MxTokenScales* mxs,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd = nullptr);
+                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd = nullptr,
+                              int8_t* out_exp = nullptr);
 
 // ---- the persistent SM-partitioned forward (persistent.cu)
 struct PersistLaunch {
@@ -165,7 +173,7 @@ struct PersistLaunch {
     void* h;                       // [2*cap, I] bf16, or E4M3 (MXFP8)
     uint8_t *ring_sc, *h_sc;       // MXFP8: scale planes of ring and h rows (sc_rows = mx_sc_rows(2*cap))
     int sc_rows;
-    void* out;                     // [T*k, H] fp32, or bf16 (MXFP8)
+    void* out;                     // [T*k, H] slot rows: MOK_SLOTS_F16S (bf16 path) or bf16 (MXFP8)
     const Chunk* chunks;
     const Minibatch* mbs;
     const int* counts2;
@@ -190,8 +198,9 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uin
 // ---- the backward (bwd.cu)
 // do rows (bf16, expert-major) = g dy_t; dlogits [T, E] by the softmax backward
 cudaError_t launch_reverse_combine(const ShardsIn& dys, int S_r, int H, int T, int k, int E, const int32_t* pos,
-                                   const float* gates, const int32_t* topk_idx, const float* o_slots, void* do_rows,
-                                   float* dlogits, int num_sms, cudaStream_t stream);
+                                   const float* gates, const int32_t* topk_idx, const uint16_t* o_slots,
+                                   const int8_t* o_exps, void* do_rows, float* dlogits, int num_sms,
+                                   cudaStream_t stream);
 // dWd = h^T do, dWg = x^T da, dWu = x^T db per expert (bf16 outputs)
 cudaError_t launch_wgrad(const void* x_rows, const void* h_rows, const void* do_rows, const void* dab, int n_rows,
                          const int32_t* offsets, int H, int I, int E, void* dwg, void* dwu, void* dwd, void* status,

@@ -289,10 +289,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int t = ld_acquire_gpu(&p.ready_q[at]) - 1;
         const int r = t / p.S_r;
         uint4* dst = reinterpret_cast<uint4*>(p.ys.p[r]) + (size_t)(t - r * p.S_r) * nvec;
+        const SlotSrc src{a.out, a.out_exp};
         if constexpr (C::MX)
-            warp_combine_token<KMAX, SlotBf16>(a.out, p.gates, t, p.k, nvec, dst, lane);
+            warp_combine_token<KMAX, SlotBf16>(src, p.gates, t, p.k, nvec, dst, lane);
         else
-            warp_combine_token<KMAX, SlotF32>(a.out, p.gates, t, p.k, nvec, dst, lane);
+            warp_combine_token<KMAX, SlotF16S>(src, p.gates, t, p.k, nvec, dst, lane);
     }
 }
 
@@ -340,6 +341,7 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     a.I = L.I;
     a.h = L.h;
     a.out = L.out;
+    if (!L.mxw) a.out_exp = reinterpret_cast<int8_t*>(L.out) + slot_exp_offset((size_t)L.T * L.k, L.H);
     a.row_slot = L.row_slot;
     a.st = reinterpret_cast<DevStatus*>(L.status);
     a.timeout_ns = L.timeout_ns;

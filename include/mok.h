@@ -64,10 +64,23 @@ enum {
 
 enum { MOK_MAX_SHARDS = 64, MOK_MAX_EXPERTS = 1024, MOK_MAX_TOPK = 32 };
 
-/* Element type of the per-slot expert outputs out [T, k, H] that the
- * grouped GEMM pushes and the combine reads: fp32 on the bf16 path, bf16 on
- * the MXFP8 path. */
-enum { MOK_SLOTS_F32 = 0, MOK_SLOTS_BF16 = 1 };
+/* Form of the per-slot expert outputs out [T, k, H] that the grouped GEMM
+ * pushes and the combine reads:
+ *   MOK_SLOTS_F16S  the bf16 path: [N_s, H] fp16 values v and, at byte
+ *                   offset mok_slot_exp_offset(N_s, H) of the same buffer,
+ *                   [N_s, H/128] int8 exponents s, one per 128-feature block
+ *                   of a row; the element is v * 2^s.  s puts the block's
+ *                   largest magnitude in [2^14, 2^15) (clamped to
+ *                   [-126, 126]), so a slot row keeps fp16's 11 significant
+ *                   bits with fp32's exponent range;
+ *   MOK_SLOTS_BF16  the MXFP8 path: [N_s, H] bf16;
+ *   MOK_SLOTS_F32   [N_s, H] fp32 (accepted by mok_combine). */
+enum { MOK_SLOTS_F32 = 0, MOK_SLOTS_BF16 = 1, MOK_SLOTS_F16S = 2 };
+
+/* Bytes of a slot buffer of n_slots rows in the given form, and the byte
+ * offset of the exponents of the MOK_SLOTS_F16S form (a multiple of 256). */
+size_t mok_slot_bytes(int n_slots, int H, int slot_type);
+size_t mok_slot_exp_offset(int n_slots, int H);
 
 /* ------------------------------------------------------------------------
  * Step 1 + 2: the plan.
@@ -212,7 +225,7 @@ typedef struct mok_fwd_opts {
     int32_t ring_slots;    /* rows of the ring token buffer (persistent mode);  */
                            /* 0 = 2 * max(minibatch, 4096) rows                 */
     int32_t dispatch_ctas; /* CTAs doing the dispatch in persistent mode;       */
-                           /* 0 = default (8 bf16: bulk copies; 16 MXFP8:      */
+                           /* 0 = default (6 bf16: bulk copies; 16 MXFP8:      */
                            /* quantising warps).  Every CTA combines once its  */
                            /* own role is done                                 */
     int32_t gemm_ctas;     /* GEMM CTAs; 0 = all remaining SMs                  */

@@ -73,6 +73,36 @@ def assert_bf16_close(got: torch.Tensor, want: torch.Tensor, what: str = ""):
     return rf, ma
 
 
+def decode_slots(buf: torch.Tensor, n: int, H: int) -> torch.Tensor:
+    """fp32 values [n, H] of a MOK_SLOTS_F16S slot buffer (uint8): fp16 values
+    times 2^s, one int8 exponent s per 128-feature block of a row."""
+    import combine_device_top_b200 as mok
+
+    b = buf.cpu()
+    off = mok.lib().mok_slot_exp_offset(n, H)
+    v = b[: n * H * 2].view(torch.float16).view(n, H).double()
+    e = b[off: off + n * (H // 128)].view(torch.int8).view(n, H // 128).double()
+    return v * torch.exp2(e).repeat_interleave(128, dim=1)
+
+
+def encode_slots(x: torch.Tensor) -> torch.Tensor:
+    """MOK_SLOTS_F16S buffer (uint8) of x [n, H]: per 128-feature block of a
+    row, s = floor(log2 max|x|) - 14 clamped to [-126, 126] (0 for an
+    all-zero block), values fp16(x * 2^-s)."""
+    import combine_device_top_b200 as mok
+
+    n, H = x.shape
+    xb = x.double().view(n, H // 128, 128)
+    m = xb.abs().amax(dim=2)
+    s = torch.where(m > 0, torch.floor(torch.log2(m.clamp_min(1e-300))) - 14, torch.zeros_like(m)).clamp(-126, 126)
+    v = (xb * torch.exp2(-s)[..., None]).view(n, H).to(torch.float16)
+    off = mok.lib().mok_slot_exp_offset(n, H)
+    buf = torch.zeros(mok.lib().mok_slot_bytes(n, H, mok.MOK_SLOTS_F16S), dtype=torch.uint8)
+    buf[: n * H * 2] = v.view(-1).view(torch.uint8)
+    buf[off: off + n * (H // 128)] = s.to(torch.int8).view(-1).view(torch.uint8)
+    return buf
+
+
 class Case:
     """Inputs of one configuration, on the host and on the device."""
 

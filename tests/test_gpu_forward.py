@@ -6,7 +6,7 @@ import torch
 import combine_device_top_b200 as mok
 import mokgen
 import oracle
-from helpers import Case, assert_bf16_close, sample_tokens
+from helpers import Case, assert_bf16_close, decode_slots, encode_slots, sample_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -57,21 +57,30 @@ def test_gather_bit_exact(name):
     assert torch.equal(rows.cpu(), want)
 
 
-@pytest.mark.parametrize("slot_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("slot_dtype", ["f16s", torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("name", ["many_experts", "k16", "k32"])
 def test_combine_matches_oracle(name, slot_dtype):
-    """The fixed-order combine over slot outputs of either type (fp32: the
-    bf16 path, bf16: the MXFP8 path); k = 16 and 32 take several rounds of
-    the combine's 8 slots in flight."""
+    """The fixed-order combine over slot outputs of every form (fp16 with
+    block exponents: the bf16 path, bf16: the MXFP8 path, fp32); k = 16 and
+    32 take several rounds of the combine's 8 slots in flight.  The fp16
+    rows span many binades (block exponents far apart)."""
     case = Case(FFN_CASES[name])
     cfg = case.cfg
     p = mok.plan(case.dlogits, cfg.k, cfg.R)
-    out = mokgen.normal(5, 77, (cfg.T * cfg.k, cfg.H), 1.0, dtype=torch.float32).to(slot_dtype)
+    vals = mokgen.normal(5, 77, (cfg.T * cfg.k, cfg.H), 1.0, dtype=torch.float32)
+    if slot_dtype == "f16s":
+        vals = vals * torch.exp2(torch.randint(-40, 40, (cfg.T * cfg.k, 1),
+                                               generator=torch.Generator().manual_seed(3)).float())
+        out = encode_slots(vals)
+        vals = decode_slots(out, cfg.T * cfg.k, cfg.H)
+    else:
+        out = vals.to(slot_dtype)
+        vals = out.double()
     ys = [torch.empty((cfg.S_r, cfg.H), dtype=torch.bfloat16, device="cuda") for _ in range(cfg.R)]
     mok.combine(out.cuda(), p, ys)
     torch.cuda.synchronize()
     g = oracle.plan(case.logits, cfg.k, cfg.R)["gates"]
-    want = oracle.combine(out.double().view(cfg.T, cfg.k, cfg.H), g)
+    want = oracle.combine(vals.view(cfg.T, cfg.k, cfg.H), g)
     got = torch.cat([y.cpu() for y in ys])
     # fp32 accumulation, one bf16 rounding: within a bf16 half-ulp (2^-8
     # relative) of the exact value, plus fp32 accumulation slack
@@ -88,7 +97,7 @@ def test_grouped_gemm_swiglu_matches_oracle(name):
     out, ws = mok.expert_ffn(rows, case.dwg, case.dwu, case.dwd, p)
     torch.cuda.synchronize()
     want, _, _ = _oracle_slots(case, p)
-    assert_bf16_close(out.cpu(), want, name)
+    assert_bf16_close(decode_slots(out, p.ns, cfg.H), want, name)
 
 
 @pytest.mark.parametrize("name", ["multi_chunk", "many_experts", "tiny"])
@@ -109,7 +118,7 @@ def test_grouped_gemm_m_tile_pairing_is_exact(name, monkeypatch):
         got[pair] = out.cpu()
     assert torch.equal(got["0"], got["1"])
     want, _, _ = _oracle_slots(case, p)
-    assert_bf16_close(got["1"], want, name)
+    assert_bf16_close(decode_slots(got["1"], p.ns, cfg.H), want, name)
 
 
 def test_grouped_gemm_single_expert_vs_torch_fp32():
@@ -126,8 +135,7 @@ def test_grouped_gemm_single_expert_vs_torch_fp32():
     h = (torch.nn.functional.silu(a) * b).to(torch.bfloat16).float()
     ref = h @ case.dwd[0].float()
     torch.cuda.synchronize()
-    assert out.dtype == torch.float32
-    assert_bf16_close(out, ref, "dense")
+    assert_bf16_close(decode_slots(out, p.ns, cfg.H), ref.cpu(), "dense")
 
 
 @pytest.mark.parametrize("name", list(FFN_CASES))
@@ -229,4 +237,4 @@ def test_forward_large_magnitudes_keep_range(scale):
     out, _ = mok.expert_ffn(rows, case.dwg, case.dwu, case.dwd, p)
     want_slots, _, _ = _oracle_slots(case, p)
     assert want_slots.abs().max().item() > 65504.0
-    assert_bf16_close(out.cpu(), want_slots, f"slots x * {scale}")
+    assert_bf16_close(decode_slots(out, p.ns, cfg.H), want_slots, f"slots x * {scale}")
