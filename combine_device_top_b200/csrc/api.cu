@@ -95,6 +95,30 @@ bool encode_bmaps(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, 
     return true;
 }
 
+// {64, rows, cols / 64} view of a row-major [rows, cols] bf16 array (strides
+// {cols * 2, 128} bytes): a {64, box_rows, box_blocks} box is box_blocks
+// consecutive 64-column blocks of box_rows rows, 128-byte swizzle, each block
+// the MN-major operand layout of the MMA.
+bool encode_cols3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                        uint32_t box_blocks, const char** err) {
+    auto enc = get_encode();
+    if (!enc) {
+        *err = "cuTensorMapEncodeTiled unavailable";
+        return false;
+    }
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, box_blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        *err = "cuTensorMapEncodeTiled failed (3D column blocks)";
+        return false;
+    }
+    return true;
+}
+
 // Wd viewed as {64 (columns inside a 64-wide block), E*I (rows), H/64 (column
 // blocks)} with strides {H*2, 128} bytes: a {64, 64, 2} box is the MMA's
 // two-atom MN-major tile of a 128-column down unit, in one TMA op.

@@ -127,28 +127,37 @@ cudaError_t launch_reverse_combine(const ShardsIn& dys, int S_r, int H, int T, i
 //   dWd[e] [I, H] = h^T do:   M = i, N = h, A = h rows, B = do rows
 //   dWg[e] [H, I] = x^T da:   M = h, N = i, A = x rows, B = da (dab cols 0..I)
 //   dWu[e] [H, I] = x^T db:   M = h, N = i, A = x rows, B = db (dab cols I..2I)
-// K = the expert's rows, 64 per stage; both operands are MN-major tiles of
-// {64 columns, 64 rows} boxes (128-byte swizzle).  Rows of the last stage
-// past the expert belong to the next expert (or are TMA zero fill): the MMA
-// warp zeroes them in shared memory before the MMAs.  Accumulators: two of
-// NB columns in TMEM, so one unit's epilogue overlaps the next's MMAs.
-// Output bf16 rows, 2 NB bytes per TMEM lane.
-constexpr int WG_THREADS = 192;  // warp 0 TMA, warp 1 zeroing + MMA, warps 2-5 epilogue
-constexpr int WG_NST = 4;
+// K = the expert's rows, 64 per stage; both operands are MN-major tiles
+// (128-byte swizzle), each loaded as ONE 3D box of its 64-column blocks
+// ({64 columns, 64 rows, blocks}).  Rows of the last stage past the expert
+// belong to the next expert (or are TMA zero fill): a warp zeroes them in
+// the A tile (x or h rows; then every product with those rows is 0) while
+// the MMA works on the stage before.  Accumulators: two of NB columns in
+// TMEM, so one unit's epilogue overlaps the next's MMAs.  The epilogue
+// writes the bf16 tile into a 128-byte-swizzled staging tile and stores it
+// with TMA (one op per 64 columns).
+constexpr int WG_THREADS = 224;  // warp 0 TMA, 1 MMA, 2 tail zeroing, 3-6 epilogue
+constexpr int WG_NST = 3;
 constexpr int WG_A_BYTES = 128 * 64 * 2;  // 16 KB
+constexpr int WG_NB_MAX = 256;
+constexpr int WG_STAGE_MAX = WG_A_BYTES + WG_NB_MAX * 128;  // 48 KB
+constexpr int WG_OUT_BYTES = 128 * WG_NB_MAX * 2;            // 64 KB staging tile
+constexpr int WG_SMEM = WG_NST * WG_STAGE_MAX + WG_OUT_BYTES + 256 + 1024;
 // bound of the waits that drain this CTA's own loads and MMAs before it leaves
 constexpr uint64_t DRAIN_NS_WG = 1000000000ull;
 
 struct WgradMaps {
-    CUtensorMap x, h, dor, dab;  // {64, 64} boxes of rows [N_s, H], [N_s, I], [N_s, H], [N_s, 2I]
+    // operands: {64, rows, blocks} views of x [N_s, H], h [N_s, I], do [N_s, H], dab [N_s, 2I]
+    CUtensorMap x, h, dor, dab;
+    // outputs: {64, 128} boxes of dWd [E*I, H], dWg / dWu [E*H, I]
+    CUtensorMap owd, owg, owu;
 };
 
 struct WgradArgs {
-    int H, I, E, nb;           // nb: N tile (256 or 128)
+    int H, I, E, nb;             // nb: N tile (256 or 128)
     int dm_t, dn_t, gm_t, gn_t;  // M / N tiles of dWd and of dWg (= dWu)
-    int upe;                   // units per expert
-    const int32_t* offsets;    // [E+1]
-    uint16_t *dwg, *dwu, *dwd;
+    int upe;                     // units per expert
+    const int32_t* offsets;      // [E+1]
     DevStatus* st;
     uint64_t timeout_ns;
 };
@@ -185,17 +194,21 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                                                            ~uintptr_t(1023));
     const int b_bytes = a.nb * 64 * 2;
     const int stage_bytes = WG_A_BYTES + b_bytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + WG_NST * stage_bytes);
-    uint64_t* empty = full + WG_NST;
+    unsigned char* otile = smem + WG_NST * WG_STAGE_MAX;                  // [nb/64][128 rows][128 B], swizzled
+    uint64_t* full = reinterpret_cast<uint64_t*>(otile + WG_OUT_BYTES);  // TMA bytes landed
+    uint64_t* ready = full + WG_NST;                                     // tail rows zeroed
+    uint64_t* empty = ready + WG_NST;                                    // stage consumed (MMA commit)
     uint64_t* tfull = empty + WG_NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* fin = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+    volatile int* ok_flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // one per epilogue warp
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < WG_NST; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&ready[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -210,6 +223,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         tma_prefetch_desc(&maps.h);
         tma_prefetch_desc(&maps.dor);
         tma_prefetch_desc(&maps.dab);
+        tma_prefetch_desc(&maps.owd);
+        tma_prefetch_desc(&maps.owg);
+        tma_prefetch_desc(&maps.owu);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -230,19 +246,17 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                 const int KB = (w.rows + 63) / 64;
                 const CUtensorMap* am = w.g == 0 ? &maps.h : &maps.x;
                 const CUtensorMap* bm = w.g == 0 ? &maps.dor : &maps.dab;
-                const int bx0 = w.n0 + (w.g == 2 ? a.I : 0);
+                const int bz0 = (w.n0 + (w.g == 2 ? a.I : 0)) / 64;  // first 64-column block of B
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 100)) {
                         ok = false;
                         break;
                     }
-                    unsigned char* st = smem + stage * stage_bytes;
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(WG_A_BYTES + b_bytes));
+                    unsigned char* st = smem + stage * WG_STAGE_MAX;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
                     const int y = w.r0 + kb * 64;
-                    tma_load_2d(st, am, &full[stage], w.m0, y);
-                    tma_load_2d(st + 8192, am, &full[stage], w.m0 + 64, y);
-                    for (int c = 0; c < a.nb / 64; ++c)
-                        tma_load_2d(st + WG_A_BYTES + c * 8192, bm, &full[stage], bx0 + c * 64, y);
+                    tma_load_3d(st, am, &full[stage], 0, y, w.m0 / 64);
+                    tma_load_3d(st + WG_A_BYTES, bm, &full[stage], 0, y, bz0);
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == WG_NST) {
@@ -254,42 +268,58 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
             for (int s = 0; s < WG_NST; ++s)
                 if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, nullptr, DRAIN_NS_WG, 101);
         }
-    } else if (warp == 1) {
+    } else if (warp == 2) {
+        // ---- tail rows of the A tile zeroed, every stage passed on to the MMA
         int stage = 0;
-        uint32_t phase = 0, tk = 0;
-        const uint32_t idesc = umma_idesc_f16(128, a.nb, /*A MN-major*/ 1, /*B MN-major*/ 1, /*bf16*/ 1);
+        uint32_t phase = 0;
         bool ok = true;
         for (int i = 0; ok && wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
-            if (w.rows == 0) continue;  // the epilogue writes zeros; no accumulator is used
             const int KB = (w.rows + 63) / 64;
-            if (lane == 0) ok = mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 102);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            tc_fence_after();
             for (int kb = 0; kb < KB; ++kb) {
                 int got = 0;
-                if (lane == 0) got = mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 103) ? 1 : 0;
+                if (lane == 0) got = mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 106) ? 1 : 0;
                 if (__shfl_sync(0xffffffffu, got, 0) == 0) {
                     ok = false;
                     break;
                 }
-                unsigned char* st = smem + stage * stage_bytes;
                 const int valid = min(64, w.rows - kb * 64);
                 if (valid < 64) {
-                    // rows past the expert: zero their 128-byte K lines in every 64-wide block of A and B
-                    const int nblk = 2 + a.nb / 64;
+                    // a K row is one 128-byte line of each 64-column block (8 KB)
+                    unsigned char* st = smem + stage * WG_STAGE_MAX;
                     const int lines = 64 - valid;
-                    for (int i2 = lane; i2 < nblk * lines * 8; i2 += 32) {
+                    for (int i2 = lane; i2 < 2 * lines * 8; i2 += 32) {
                         const int blk = i2 / (lines * 8), rem = i2 - blk * lines * 8;
-                        const int line = valid + rem / 8, chunk = rem % 8;
-                        *reinterpret_cast<uint4*>(st + blk * 8192 + line * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(st + blk * 8192 + (valid + rem / 8) * 128 + (rem % 8) * 16) =
+                            make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async_shared();
-                    __syncwarp();
                 }
-                if (lane == 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ready[stage]);
+                if (++stage == WG_NST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, tk = 0;
+            const uint32_t idesc = umma_idesc_f16(128, a.nb, /*A MN-major*/ 1, /*B MN-major*/ 1, /*bf16*/ 1);
+            bool ok = true;
+            for (int i = 0; ok && wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
+                if (w.rows == 0) continue;  // the epilogue writes zeros; no accumulator is used
+                const int KB = (w.rows + 63) / 64;
+                if (!mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 102)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&ready[stage], phase, a.st, a.timeout_ns, 103)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(st), sb = sa + WG_A_BYTES;
+                    const uint32_t sa = smem_u32(smem + stage * WG_STAGE_MAX), sb = sa + WG_A_BYTES;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         // both MN-major SW128: 16 K rows = 2 atoms of 1 KB; 64-wide blocks 8 KB apart
@@ -298,52 +328,70 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                         umma_bf16(tmem + (tk & 1u) * 256u, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty[stage]);
+                    if (++stage == WG_NST) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
-                __syncwarp();
-                if (++stage == WG_NST) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                if (!ok) break;
+                umma_commit(&tfull[tk & 1u]);
+                ++tk;
             }
-            if (!ok) break;
-            if (lane == 0) umma_commit(&tfull[tk & 1u]);
-            ++tk;
-        }
-        if (lane == 0) {
             umma_commit(fin);
             mbar_wait(fin, 0, nullptr, DRAIN_NS_WG, 104);
         }
-        __syncwarp();
     } else {
-        // ---- epilogue: TMEM lane = output row m0 + 32 q + lane, NB bf16 columns
+        // ---- epilogue: TMEM lane = output row m0 + 32 q + lane; bf16 into the
+        // swizzled staging tile, then TMA stores of its 64-column blocks
         const int q = warp & 3;
+        const int r = q * 32 + lane;  // row inside the tile
+        const bool leader = warp == 3 && lane == 0;
         uint32_t tk = 0;
         for (int i = 0; wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
-            uint16_t* out = w.g == 0 ? a.dwd + (size_t)w.e * a.I * a.H : (w.g == 1 ? a.dwg : a.dwu) + (size_t)w.e * a.H * a.I;
-            const int ldo = w.g == 0 ? a.H : a.I;
-            uint16_t* orow = out + (size_t)(w.m0 + q * 32 + lane) * ldo + w.n0;
-            if (w.rows == 0) {
-                for (int c = 0; c < a.nb; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-                continue;
-            }
-            int got = 0;
-            if (lane == 0) got = mbar_wait(&tfull[tk & 1u], (tk >> 1) & 1u, a.st, a.timeout_ns, 105) ? 1 : 0;
-            if (__shfl_sync(0xffffffffu, got, 0) == 0) break;
-            tc_fence_after();
+            int ok = 1;
+            if (w.rows > 0 && lane == 0) ok = mbar_wait(&tfull[tk & 1u], (tk >> 1) & 1u, a.st, a.timeout_ns, 105) ? 1 : 0;
+            if (lane == 0) ok_flags[q] = ok;
+            // the previous unit's stores have read the staging tile
+            if (leader) bulk_wait_read<0>();
+            named_bar_sync(1, 128);
+            // the four warps leave or go on together
+            const int all_ok = ok_flags[0] & ok_flags[1] & ok_flags[2] & ok_flags[3];
+            named_bar_sync(1, 128);  // the flags are written again at the next unit
+            if (!all_ok) break;
+            if (w.rows > 0) tc_fence_after();
             for (int c = 0; c < a.nb; c += 32) {
                 float v[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (tk & 1u) * 256u + (uint32_t)c, v);
+                if (w.rows > 0) {
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (tk & 1u) * 256u + (uint32_t)c, v);
+                } else {
 #pragma unroll
-                for (int p = 0; p < 32; p += 8)
-                    *reinterpret_cast<uint4*>(orow + c + p) =
-                        make_uint4(pack_bf16x2(v[p], v[p + 1]), pack_bf16x2(v[p + 2], v[p + 3]),
-                                   pack_bf16x2(v[p + 4], v[p + 5]), pack_bf16x2(v[p + 6], v[p + 7]));
+                    for (int p = 0; p < 32; ++p) v[p] = 0.f;
+                }
+                unsigned char* blk = otile + (c / 64) * (128 * 128) + r * 128;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int chunk = ((c % 64) / 8) + p;  // 16-byte chunk of the row's 128-byte line
+                    *reinterpret_cast<uint4*>(blk + ((chunk ^ (r & 7)) << 4)) =
+                        make_uint4(pack_bf16x2(v[8 * p], v[8 * p + 1]), pack_bf16x2(v[8 * p + 2], v[8 * p + 3]),
+                                   pack_bf16x2(v[8 * p + 4], v[8 * p + 5]), pack_bf16x2(v[8 * p + 6], v[8 * p + 7]));
+                }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[tk & 1u]);
-            ++tk;
+            if (w.rows > 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[tk & 1u]);
+                ++tk;
+            }
+            fence_proxy_async_shared();  // generic writes of the tile -> the TMA store reads them
+            named_bar_sync(1, 128);
+            if (leader) {
+                const CUtensorMap* om = w.g == 0 ? &maps.owd : (w.g == 1 ? &maps.owg : &maps.owu);
+                const int y0 = w.e * (w.g == 0 ? a.I : a.H) + w.m0;
+                for (int b = 0; b < a.nb / 64; ++b) tma_store_2d(om, otile + b * (128 * 128), w.n0 + b * 64, y0);
+                bulk_commit();
+            }
         }
+        if (leader) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -353,44 +401,38 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     }
 }
 
-static bool encode_rows64(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, const char** err) {
-    return encode_tmap_2d_bf16(m, base, inner, rows, 64, 64, err);
-}
-
 cudaError_t launch_wgrad(const void* x_rows, const void* h_rows, const void* do_rows, const void* dab, int n_rows,
                          const int32_t* offsets, int H, int I, int E, void* dwg, void* dwu, void* dwd, void* status,
                          uint64_t timeout_ns, int num_sms, const char** err, cudaStream_t stream) {
-    WgradMaps maps;
-    if (!encode_rows64(&maps.x, x_rows, (uint64_t)H, (uint64_t)n_rows, err) ||
-        !encode_rows64(&maps.h, h_rows, (uint64_t)I, (uint64_t)n_rows, err) ||
-        !encode_rows64(&maps.dor, do_rows, (uint64_t)H, (uint64_t)n_rows, err) ||
-        !encode_rows64(&maps.dab, dab, (uint64_t)2 * I, (uint64_t)n_rows, err))
-        return cudaErrorInvalidValue;
     WgradArgs a{};
     a.H = H;
     a.I = I;
     a.E = E;
     a.nb = (H % 256 == 0 && I % 256 == 0) ? 256 : 128;
+    WgradMaps maps;
+    if (!encode_cols3d_bf16(&maps.x, x_rows, (uint64_t)H, (uint64_t)n_rows, 64, 2, err) ||
+        !encode_cols3d_bf16(&maps.h, h_rows, (uint64_t)I, (uint64_t)n_rows, 64, 2, err) ||
+        !encode_cols3d_bf16(&maps.dor, do_rows, (uint64_t)H, (uint64_t)n_rows, 64, a.nb / 64, err) ||
+        !encode_cols3d_bf16(&maps.dab, dab, (uint64_t)2 * I, (uint64_t)n_rows, 64, a.nb / 64, err) ||
+        !encode_tmap_2d_bf16(&maps.owd, dwd, (uint64_t)H, (uint64_t)E * I, 64, 128, err) ||
+        !encode_tmap_2d_bf16(&maps.owg, dwg, (uint64_t)I, (uint64_t)E * H, 64, 128, err) ||
+        !encode_tmap_2d_bf16(&maps.owu, dwu, (uint64_t)I, (uint64_t)E * H, 64, 128, err))
+        return cudaErrorInvalidValue;
     a.dm_t = I / 128;
     a.dn_t = H / a.nb;
     a.gm_t = H / 128;
     a.gn_t = I / a.nb;
     a.upe = a.dm_t * a.dn_t + 2 * a.gm_t * a.gn_t;
     a.offsets = offsets;
-    a.dwg = reinterpret_cast<uint16_t*>(dwg);
-    a.dwu = reinterpret_cast<uint16_t*>(dwu);
-    a.dwd = reinterpret_cast<uint16_t*>(dwd);
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;
-    const int smem = WG_NST * (WG_A_BYTES + a.nb * 128) + 256 + 1024;
     static bool attr[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr[dev]) {
-        e = cudaFuncSetAttribute(k_wgrad, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 WG_NST * (WG_A_BYTES + 256 * 128) + 256 + 1024);
+        e = cudaFuncSetAttribute(k_wgrad, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
         if (e != cudaSuccess) return e;
         attr[dev] = true;
     }
@@ -398,7 +440,7 @@ cudaError_t launch_wgrad(const void* x_rows, const void* h_rows, const void* do_
     const int grid = (int)(units < num_sms ? units : num_sms);
     *err = "weight-gradient launch";
     if (grid <= 0) return cudaSuccess;
-    k_wgrad<<<grid, WG_THREADS, smem, stream>>>(maps, a);
+    k_wgrad<<<grid, WG_THREADS, WG_SMEM, stream>>>(maps, a);
     return cudaGetLastError();
 }
 

@@ -194,6 +194,10 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
 // 128-byte swizzle, zero fill out of bounds.
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                          uint32_t box_outer, const char** err);
+// {64, rows, cols / 64} view of a row-major [rows, cols] bf16 array, boxes of
+// box_blocks 64-column blocks x box_rows rows (128-byte swizzle)
+bool encode_cols3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                        uint32_t box_blocks, const char** err);
 
 // ---- the backward (bwd.cu)
 // do rows (bf16, expert-major) = g dy_t; dlogits [T, E] by the softmax backward
