@@ -257,7 +257,7 @@ def _gpu_index():
 
 
 def time_steps(wl: Workload, mode: str, steps: int, warmup: int, minibatch: int, dispatch_ctas: int = 0,
-               world: int = 1):
+               world: int = 1, dispatch_warps: int = 0):
     """Time `steps` steps after `warmup` untimed ones; staged mode goes through
     the per-step ABI calls (the same kernels as mok_moe_forward's staged
     mode) so that events on the launching stream time each phase."""
@@ -266,7 +266,8 @@ def time_steps(wl: Workload, mode: str, steps: int, warmup: int, minibatch: int,
     cfg, device = wl.cfg, wl.device
     staged = mode == "staged"
     opts = mok.fwd_opts(mode=mok.MOK_MODE_STAGED if staged else mok.MOK_MODE_PERSISTENT,
-                        ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8, dispatch_ctas=dispatch_ctas)
+                        ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8, dispatch_ctas=dispatch_ctas,
+                        dispatch_warps=dispatch_warps)
     p = wl.plan
     bufs = {}
     if staged:
@@ -367,7 +368,8 @@ def _mx_ptr(pack):
     return ctypes.cast(ctypes.byref(_mx_ptr.keep), ctypes.c_void_p)
 
 
-def time_e2e(wl: Workload, mode: str, steps: int, minibatch: int, world: int):
+def time_e2e(wl: Workload, mode: str, steps: int, minibatch: int, world: int, dispatch_ctas: int = 0,
+             dispatch_warps: int = 0):
     """End to end from pinned host memory through mok_moe_forward_host_batches:
     every step uploads its x and logits and reads its y back; the library
     overlaps step i+1's upload and step i-1's download with step i's compute."""
@@ -375,7 +377,8 @@ def time_e2e(wl: Workload, mode: str, steps: int, minibatch: int, world: int):
 
     cfg, device = wl.cfg, wl.device
     opts = mok.fwd_opts(mode=mok.MOK_MODE_STAGED if mode == "staged" else mok.MOK_MODE_PERSISTENT,
-                        ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8)
+                        ring_slots=cfg.ring_slots, mxfp8=cfg.mxfp8, dispatch_ctas=dispatch_ctas,
+                        dispatch_warps=dispatch_warps)
     hx, hl = wl.x.pin_memory(), wl.logits.pin_memory()
     hy = torch.empty_like(wl.x).pin_memory()
     wts = (wl.pack, None, None) if wl.pack is not None else wl.w
@@ -612,6 +615,8 @@ def main():
                          "default: the configuration's)")
     ap.add_argument("--dispatch-ctas", type=int, default=0,
                     help="persistent mode: CTAs on the dispatch side (0: the library default, 6 bf16 / 16 MXFP8)")
+    ap.add_argument("--dispatch-warps", type=int, default=0,
+                    help="persistent mode: 1 or 2 dispatch warps in every CTA instead of dispatch CTAs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub-records", action="store_true", help="time only the main workload")
     ap.add_argument("--backward", action="store_true",
@@ -637,7 +642,8 @@ def main():
              else "bf16 weights [E,H,I]/[E,I,H]")
     config = {"workload": f"{cfg.name}: {cfg.describe()}, {wdesc}",
               "tokens_per_step_per_gpu": cfg.T, "mode": args.mode,
-              **({"minibatch": minibatch, "dispatch_ctas": args.dispatch_ctas or (16 if cfg.mxfp8 else 6)}
+              **(({"minibatch": minibatch, "dispatch_warps_per_cta": args.dispatch_warps} if args.dispatch_warps
+                  else {"minibatch": minibatch, "dispatch_ctas": args.dispatch_ctas or (16 if cfg.mxfp8 else 6)})
                  if args.mode == "persistent" else {}),
               "l2": f"inputs larger than L2 ({algorithmic_work(cfg)['weight_bytes'] / 1e9:.1f} GB of expert "
                     f"weights streamed per step)"}
@@ -668,13 +674,14 @@ def main():
             bw["frac_of_hbm"] = bw["GBps"] / peaks["hbm_gbs"]
             print(json.dumps(bw), flush=True)
         return 0
-    res = time_steps(wl, args.mode, args.steps, args.warmup, minibatch, args.dispatch_ctas, world)
-    e2e = time_e2e(wl, args.mode, args.steps, minibatch, world)
+    res = time_steps(wl, args.mode, args.steps, args.warmup, minibatch, args.dispatch_ctas, world,
+                     args.dispatch_warps)
+    e2e = time_e2e(wl, args.mode, args.steps, minibatch, world, args.dispatch_ctas, args.dispatch_warps)
     subs = {}
     if not args.no_sub_records and not args.scale_experts and world == 1 and args.config == "page":
         peaks, peak_src = load_peaks()
         other = "persistent" if args.mode == "staged" else "staged"
-        r2 = time_steps(wl, other, args.steps, args.warmup, minibatch, args.dispatch_ctas)
+        r2 = time_steps(wl, other, args.steps, args.warmup, minibatch, args.dispatch_ctas, 1, args.dispatch_warps)
         subs[f"{cfg.name}_{other}"] = sub_record(cfg, other, r2, peaks, peak_src, args.steps)
         subs[f"{cfg.name}_router_plan"] = time_router(wl, args.steps, args.warmup)
         bw = time_backward(wl, max(3, args.steps // 4), 2)

@@ -64,7 +64,7 @@ class PlanT(ctypes.Structure):
 class FwdOpts(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("dispatch_ctas", ctypes.c_int32),
                 ("gemm_ctas", ctypes.c_int32), ("mxfp8", ctypes.c_int32), ("min_waves", ctypes.c_int32),
-                ("save_for_backward", ctypes.c_int32), ("reserved", ctypes.c_int32), ("timeout_ns", ctypes.c_uint64)]
+                ("save_for_backward", ctypes.c_int32), ("dispatch_warps", ctypes.c_int32), ("timeout_ns", ctypes.c_uint64)]
 
 
 @lru_cache(maxsize=1)
@@ -264,9 +264,10 @@ def quantize_weights_mxfp8(w: torch.Tensor, stream=None):
 
 
 def fwd_opts(mode: int = MOK_MODE_PERSISTENT, ring_slots: int = 0, dispatch_ctas: int = 0, gemm_ctas: int = 0,
-             mxfp8: bool = False, timeout_ns: int = 0, min_waves: int = 0, save_for_backward: bool = False) -> FwdOpts:
-    return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), min_waves, int(save_for_backward), 0,
-                   timeout_ns)
+             mxfp8: bool = False, timeout_ns: int = 0, min_waves: int = 0, save_for_backward: bool = False,
+             dispatch_warps: int = 0) -> FwdOpts:
+    return FwdOpts(mode, ring_slots, dispatch_ctas, gemm_ctas, int(mxfp8), min_waves, int(save_for_backward),
+                   dispatch_warps, timeout_ns)
 
 
 def forward_workspace_bytes(T, H, I, E, k, minibatch, opts: FwdOpts | None = None) -> int:

@@ -484,7 +484,7 @@ namespace mok {
 // and chunks) in the workspace.
 struct FwdSetup {
     FwdLayout L;
-    int sms, dispatch, gemm, upc, min_units;
+    int sms, dispatch, dwarps, gemm, upc, min_units;
     bool pair;
     uint64_t timeout;
     const mok_mxfp8_weights* mxw;
@@ -509,7 +509,10 @@ static int setup_forward(int H, int I, const void* w_gate, const mok_plan_t* pla
         if (!m || !m->gate || !m->gate_scales || !m->up || !m->up_scales || !m->down || !m->down_scales)
             return fail(MOK_ERR_INVALID_ARG, "MXFP8 weight pack with NULL members");
     }
-    if (opts && opts->reserved != 0) return fail(MOK_ERR_INVALID_ARG, "opts.reserved must be 0");
+    const int dwarps = opts ? opts->dispatch_warps : 0;
+    if (dwarps < 0 || dwarps > 2) return fail(MOK_ERR_INVALID_ARG, "dispatch_warps must be in [0, 2]");
+    if (dwarps > 0 && opts->dispatch_ctas > 0)
+        return fail(MOK_ERR_INVALID_ARG, "dispatch_warps and dispatch_ctas exclude each other");
     if (opts && opts->save_for_backward && (mode != MOK_MODE_STAGED || (opts->mxfp8 != 0)))
         return fail(MOK_ERR_UNSUPPORTED, "save_for_backward needs the staged bf16 path");
     if (mode == MOK_MODE_PERSISTENT && minibatch != 0 && minibatch < 16)
@@ -523,8 +526,14 @@ static int setup_forward(int H, int I, const void* w_gate, const mok_plan_t* pla
     F->sms = device_sms(nullptr);
     if (F->sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     F->dispatch = 0;
+    F->dwarps = 0;
     F->gemm = F->sms;
-    if (mode == MOK_MODE_PERSISTENT) {
+    if (mode == MOK_MODE_PERSISTENT && dwarps > 0) {
+        // warp layout: every CTA runs the GEMM and dispatch warps
+        F->dwarps = dwarps;
+        F->gemm = (opts->gemm_ctas > 0) ? opts->gemm_ctas : F->sms;
+        if (F->gemm > F->sms) return fail(MOK_ERR_INVALID_ARG, "gemm_ctas must be at most the %d SMs", F->sms);
+    } else if (mode == MOK_MODE_PERSISTENT) {
         F->dispatch = (opts && opts->dispatch_ctas > 0) ? opts->dispatch_ctas : (F->mxw ? 16 : kDefaultDispatchBf16);
         F->gemm = (opts && opts->gemm_ctas > 0) ? opts->gemm_ctas : F->sms - F->dispatch;
         if (F->dispatch >= F->sms || F->gemm < 1 || F->dispatch + F->gemm > F->sms)
@@ -631,6 +640,7 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         PersistLaunch P{};
         P.grid = F.dispatch + F.gemm;
         P.dispatch_ctas = F.dispatch;
+        P.dispatch_warps = F.dwarps;
         P.pair = F.pair;
         P.cap = L.cap;
         P.H = H;
@@ -662,6 +672,7 @@ int mok_moe_forward(const void* const* x_shards, int H, int I, const void* w_gat
         P.ready_q = P.tok_cnt + T;
         P.q_tail = P.ready_q + T;
         P.q_claim = P.q_tail + 1;
+        P.d_claim = P.q_claim + 1;
         P.xs = xs;
         P.ys = ys;
         P.src_rank = plan->sched_src_rank;

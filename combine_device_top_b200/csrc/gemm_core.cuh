@@ -726,8 +726,10 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
 }
 
 // ------------------------------------------------------------------ one GEMM CTA
-// Runs every unit the schedule gives this CTA.  All C::THREADS threads must
-// call it; it returns after TMEM is released.  mx: MXFP8 maps (C::MX only).
+// Runs every unit the schedule gives this CTA.  Threads [0, C::THREADS) must
+// call it; any further warps of the block take part in its first barrier
+// (a __syncthreads of their own) and in nothing else.  It returns after TMEM
+// is released.  mx: MXFP8 maps (C::MX only).
 template <class S, class C>
 __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx, const CoreArgs& a, const S& s,
                                          unsigned char* smem) {
@@ -796,8 +798,10 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
         gemm_sf_layout<S, C>(a, s, smem, full, sfready);
     }
 
+    // the GEMM roles' threads only: a persistent kernel may run other warps
+    // beside them (barrier 3; the epilogue groups use 1 and 2)
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(3, C::THREADS);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);

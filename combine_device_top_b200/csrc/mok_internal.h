@@ -165,6 +165,7 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
 // ---- the persistent SM-partitioned forward (persistent.cu)
 struct PersistLaunch {
     int grid, dispatch_ctas, cap;  // CTAs, of which the first dispatch_ctas gather; ring half rows
+    int dispatch_warps;            // > 0: no dispatch CTAs, this many dispatch warps in every CTA
     bool pair;                     // bf16 GEMM units of two M tiles (the work list counted units this way)
     int H, I, E, T, k, S_r;
     const void *wg, *wu, *wd;      // bf16 weights; unused on the MXFP8 path
@@ -178,8 +179,8 @@ struct PersistLaunch {
     const Minibatch* mbs;
     const int* counts2;
     // zeroed counters: chunk_ready, g_done, d_chunk [max_chunks]; d_done
-    // [max_mb]; tok_cnt, ready_q [T]; q_tail, q_claim [1]
-    int *chunk_ready, *g_done, *d_chunk, *d_done, *tok_cnt, *ready_q, *q_tail, *q_claim;
+    // [max_mb]; tok_cnt, ready_q [T]; q_tail, q_claim, d_claim [1]
+    int *chunk_ready, *g_done, *d_chunk, *d_done, *tok_cnt, *ready_q, *q_tail, *q_claim, *d_claim;
     ShardsIn xs;
     ShardsOut ys;
     const int32_t *src_rank, *src_index, *row_slot;

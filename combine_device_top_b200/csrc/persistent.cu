@@ -29,6 +29,13 @@
 //                queue order (a warp per token): the combine of early
 //                tokens overlaps the GEMM of later experts (macrobatch
 //                overlap), and the rest runs on every SM at the end.
+// Warp layout (dispatch_warps > 0): no dispatch CTAs.  Every CTA runs the
+// GEMM roles and, beside them, dispatch_warps warps that claim the
+// expert-major rows in pieces of PIECE_ROWS from one device counter, in
+// row order, copy (MXFP8: quantise) them into the ring and add the rows
+// they wrote to chunk_ready[c]; a gate/up unit then waits for all of its
+// chunk's rows.  The GEMM keeps every SM, and the dispatch warps join the
+// combine as soon as the last piece is claimed.
 // Dependencies only point to lower unit indices (or to the dispatch side,
 // which waits only on lower indices), and the combine waits only on the GEMM
 // side, so the lowest unfinished unit can always proceed: no deadlock
@@ -59,6 +66,7 @@ struct PersistParams {
     int cap;             // rows per ring half
     int MTG, MTD;        // units (groups of C::SUB M tiles) per chunk of the gate/up and down phases
     int dispatch_ctas;
+    int dispatch_warps;  // per CTA, warp layout (then dispatch_ctas == 0); 0: dispatch CTAs
     // counters (zeroed before the launch)
     int* chunk_ready;  // [max_chunks] 1 once the chunk's rows are in the ring
     int* g_done;       // [max_chunks] gate/up units done for chunk c
@@ -68,6 +76,7 @@ struct PersistParams {
     int* ready_q;      // [T] 1 + token, in the order tokens became complete (0: not yet)
     int* q_tail;       // tokens appended to ready_q
     int* q_claim;      // queue positions claimed by combining warps
+    int* d_claim;      // warp layout: pieces of rows claimed by dispatch warps
     // token data
     ShardsIn xs;
     ShardsOut ys;
@@ -121,7 +130,9 @@ struct PersistSched {
     }
 
     __device__ bool wait_inputs(const Unit& u, DevStatus* st, uint64_t timeout_ns) const {
-        const bool ok = u.phase == 0 ? flag_wait_geq(&p->chunk_ready[u.chunk], 1, st, timeout_ns, 40)
+        // chunk_ready counts rows in the warp layout, whole chunks otherwise
+        const int need = p->dispatch_warps > 0 ? u.rows : 1;
+        const bool ok = u.phase == 0 ? flag_wait_geq(&p->chunk_ready[u.chunk], need, st, timeout_ns, 40)
                                      : flag_wait_geq(&p->g_done[u.chunk], p->MTG, st, timeout_ns, 41);
         fence_proxy_async_global();
         return ok;
@@ -152,10 +163,130 @@ struct PersistSched {
     }
 };
 
+// Rows a dispatch warp claims at a time (warp layout).
+constexpr int PIECE_ROWS = 16;
+constexpr int MAX_DISPATCH_WARPS = 2;  // 12 bf16 warps keep 168 registers a thread (3 warps per SM sub-partition)
+
+// MXFP8: one warp quantises source row src into E4M3 ring row brow and its
+// H/32 block scales into the scale planes; four 256-element steps' loads in
+// flight per lane.
+__device__ __forceinline__ void mx_dispatch_row(const PersistParams& p, const CoreArgs& a, const uint4* src,
+                                                int brow, int lane) {
+    uint32_t* planes = reinterpret_cast<uint32_t*>(p.ring_sc);
+    uint8_t* dst = reinterpret_cast<uint8_t*>(p.ring) + (size_t)brow * a.H;
+    for (int c0 = 0; c0 < a.H; c0 += 1024) {
+        uint4 raw[4];
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+            const int cc = c0 + 256 * s4 + lane * 8;
+            raw[s4] = cc < a.H ? __ldg(src + (cc >> 3)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+            const int cs = c0 + 256 * s4;
+            if (cs < a.H) {  // warp-uniform
+                uint2 q;
+                uint32_t word;
+                warp_mx_quant8(raw[s4], q, word, lane);
+                const int cc = cs + lane * 8;
+                if (cc < a.H) {
+                    *reinterpret_cast<uint2*>(dst + cc) = q;
+                    if ((lane & 15) == 0) planes[(size_t)((cs >> 7) + (lane >> 4)) * a.sc_rows + brow] = word;
+                }
+            }
+        }
+    }
+}
+
+// bf16: one warp copies a row of nvec 16-byte vectors, eight per lane in
+// flight (4 KB per warp).
+__device__ __forceinline__ void warp_copy_row_deep(const uint4* __restrict__ src, uint4* __restrict__ dst, int nvec,
+                                                   int lane) {
+    for (int v0 = 0; v0 < nvec; v0 += 256) {
+        uint4 t[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int v = v0 + 32 * j + lane;
+            if (v < nvec) t[j] = __ldg(src + v);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int v = v0 + 32 * j + lane;
+            if (v < nvec) dst[v] = t[j];
+        }
+    }
+}
+
+// Warp layout: a dispatch warp claims pieces of PIECE_ROWS expert-major
+// rows in order, and for each chunk a piece touches waits (once per
+// minibatch, lane 0, bounded) for the ring half to be free, writes the rows
+// and publishes them: every lane fences its own stores (generic -> async
+// proxy, then GPU scope), the warp converges, and lane 0 adds the row count
+// to chunk_ready[c] with release semantics.  Pieces are claimed in order, so
+// every piece below a claimed one is already claimed by a running warp:
+// the lowest unfinished piece waits only on the GEMM of minibatch b - 2,
+// which waits only on lower pieces.
+template <class C>
+__device__ __forceinline__ void warp_dispatch(const PersistParams& p, const CoreArgs& a, int nch, int nmb, int lane) {
+    if (nmb <= 0 || nch <= 0) return;
+    const int total = p.mbs[nmb - 1].row1;
+    const int nvec = a.H >> 3;
+    int ready_b = 1;  // ring halves of minibatches 0 and 1 start free
+    while (true) {
+        int piece = 0;
+        if (lane == 0) piece = atomicAdd(p.d_claim, 1);
+        piece = __shfl_sync(0xffffffffu, piece, 0);
+        const int r0 = piece * PIECE_ROWS;
+        if (r0 >= total || failed(a.st)) return;
+        const int r1 = min(r0 + PIECE_ROWS, total);
+        // the chunk holding row r0: chunks are in row order
+        int lo = 0, hi = nch - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.chunks[mid].row0 <= r0) lo = mid; else hi = mid - 1;
+        }
+        int c = lo;
+        int r = r0;
+        while (r < r1 && c < nch) {
+            const Chunk ck = p.chunks[c];
+            const int e1 = min(r1, ck.row0 + ck.rows);
+            const int b = ck.mb;
+            if (b > ready_b) {
+                int ok = 1;
+                if (lane == 0) {
+                    const Minibatch old = p.mbs[b - 2];
+                    ok = flag_wait_geq(&p.d_done[b - 2], (old.chunk1 - old.chunk0) * p.MTD, a.st, a.timeout_ns, 51)
+                             ? 1 : 0;
+                }
+                if (__shfl_sync(0xffffffffu, ok, 0) == 0) return;
+                ready_b = b;
+            }
+            const Minibatch mb = p.mbs[b];
+            for (int rr = r; rr < e1; ++rr) {
+                const int sr = __ldg(p.src_rank + rr), si = __ldg(p.src_index + rr);
+                const uint4* src = reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec;
+                const int brow = (b & 1) * p.cap + (rr - mb.row0);
+                if constexpr (C::MX)
+                    mx_dispatch_row(p, a, src, brow, lane);
+                else
+                    warp_copy_row_deep(src, reinterpret_cast<uint4*>(p.ring) + (size_t)brow * nvec, nvec, lane);
+            }
+            // the rows are read next by TMA in the GEMM CTAs
+            fence_proxy_async_global();
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) red_release_gpu_add(&p.chunk_ready[c], e1 - r);
+            r = e1;
+            ++c;
+        }
+    }
+}
+
 // C: the GEMM CTAs' configuration (bf16 with one M tile per unit or pairs,
-// or MXFP8); the dispatch CTAs run with the same block shape.
+// or MXFP8); the dispatch CTAs run with the same block shape.  In the warp
+// layout the block has C::THREADS + 32 * dispatch_warps threads.
 template <int KMAX, class C>
-__global__ void __launch_bounds__(C::THREADS, 1)
+__global__ void __launch_bounds__(C::THREADS + 32 * MAX_DISPATCH_WARPS, 1)
     k_moe_persistent(const __grid_constant__ GemmMaps maps, const __grid_constant__ MxMaps mx, const CoreArgs a,
                      const __grid_constant__ PersistParams p) {
     extern __shared__ unsigned char smem_raw[];
@@ -167,7 +298,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nvec = a.H >> 3;  // 16-byte vectors per token row
 
-    if ((int)blockIdx.x < D) {
+    if (p.dispatch_warps > 0) {
+        // ---------------------------------------- warp layout
+        if (warp >= C::THREADS / 32) {
+            __syncthreads();  // the GEMM roles' set-up barrier (barrier 0 counts every thread)
+            warp_dispatch<C>(p, a, nch, nmb, lane);
+        } else {
+            PersistSched s;
+            s.p = &p;
+            s.nch = nch;
+            s.nmb = nmb;
+            s.gidx = blockIdx.x;
+            s.gctas = gridDim.x;
+            s.total = nch * (p.MTG + p.MTD);
+            gemm_cta<PersistSched, C>(maps, &mx, a, s, smem);
+        }
+    } else if ((int)blockIdx.x < D) {
         // ---------------------------------------- dispatch side: fill the ring
         // bf16: one thread streams rows through the CTA's otherwise idle
         // shared memory with bulk async copies (about 200 KB in flight per
@@ -203,37 +349,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const Chunk ck = p.chunks[c];
                 const int r0 = ck.row0, r1 = ck.row0 + ck.rows;
                 if constexpr (C::MX) {
-                    // E4M3 row at ring row brow, its H/32 block scales in the planes;
-                    // four 256-element steps' loads in flight per lane
-                    uint32_t* planes = reinterpret_cast<uint32_t*>(p.ring_sc);
                     for (int r = r0 + warp; r < r1; r += C::THREADS / 32) {
                         const int sr = __ldg(p.src_rank + r), si = __ldg(p.src_index + r);
-                        const uint4* src = reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec;
-                        const int brow = (b & 1) * p.cap + (r - mb.row0);
-                        uint8_t* dst = reinterpret_cast<uint8_t*>(p.ring) + (size_t)brow * a.H;
-                        for (int c0 = 0; c0 < a.H; c0 += 1024) {
-                            uint4 raw[4];
-#pragma unroll
-                            for (int s4 = 0; s4 < 4; ++s4) {
-                                const int cc = c0 + 256 * s4 + lane * 8;
-                                raw[s4] = cc < a.H ? __ldg(src + (cc >> 3)) : make_uint4(0, 0, 0, 0);
-                            }
-#pragma unroll
-                            for (int s4 = 0; s4 < 4; ++s4) {
-                                const int cs = c0 + 256 * s4;
-                                if (cs < a.H) {  // warp-uniform
-                                    uint2 q;
-                                    uint32_t word;
-                                    warp_mx_quant8(raw[s4], q, word, lane);
-                                    const int cc = cs + lane * 8;
-                                    if (cc < a.H) {
-                                        *reinterpret_cast<uint2*>(dst + cc) = q;
-                                        if ((lane & 15) == 0)
-                                            planes[(size_t)((cs >> 7) + (lane >> 4)) * a.sc_rows + brow] = word;
-                                    }
-                                }
-                            }
-                        }
+                        mx_dispatch_row(p, a, reinterpret_cast<const uint4*>(p.xs.p[sr]) + (size_t)si * nvec,
+                                        (b & 1) * p.cap + (r - mb.row0), lane);
                     }
                 } else if (bulk) {
                     if (threadIdx.x == 0) {
@@ -300,6 +419,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 template <int KMAX, class C>
 static cudaError_t launch_persistent_k(int grid, const GemmMaps& maps, const MxMaps& mx, const CoreArgs& a,
                                        const PersistParams& p, cudaStream_t stream) {
+    const int threads = C::THREADS + 32 * p.dispatch_warps;
     static bool attr[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -311,7 +431,7 @@ static cudaError_t launch_persistent_k(int grid, const GemmMaps& maps, const MxM
         attr[dev] = true;
     }
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_moe_persistent<KMAX, C>, C::THREADS, C::SMEM);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_moe_persistent<KMAX, C>, threads, C::SMEM);
     if (e != cudaSuccess) return e;
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -320,7 +440,7 @@ static cudaError_t launch_persistent_k(int grid, const GemmMaps& maps, const MxM
     void* args[] = {const_cast<GemmMaps*>(&maps), const_cast<MxMaps*>(&mx), const_cast<CoreArgs*>(&a),
                     const_cast<PersistParams*>(&p)};
     return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_moe_persistent<KMAX, C>), dim3(grid),
-                                       dim3(C::THREADS), args, C::SMEM, stream);
+                                       dim3(threads), args, C::SMEM, stream);
 }
 
 cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, cudaStream_t stream) {
@@ -364,6 +484,9 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.MTG = (L.I / MT_G_FEATURES + sub - 1) / sub;
     p.MTD = (L.H / MT_D_FEATURES + sub - 1) / sub;
     p.dispatch_ctas = L.dispatch_ctas;
+    p.dispatch_warps = L.dispatch_warps;
+    if (p.dispatch_warps < 0 || p.dispatch_warps > MAX_DISPATCH_WARPS || (p.dispatch_warps > 0 && p.dispatch_ctas != 0))
+        return cudaErrorInvalidValue;
     p.chunk_ready = L.chunk_ready;
     p.g_done = L.g_done;
     p.d_chunk = L.d_chunk;
@@ -372,6 +495,7 @@ cudaError_t launch_forward_persistent(const PersistLaunch& L, const char** err, 
     p.ready_q = L.ready_q;
     p.q_tail = L.q_tail;
     p.q_claim = L.q_claim;
+    p.d_claim = L.d_claim;
     p.xs = L.xs;
     p.ys = L.ys;
     p.S_r = L.S_r;

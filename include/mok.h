@@ -227,7 +227,7 @@ typedef struct mok_fwd_opts {
     int32_t dispatch_ctas; /* CTAs doing the dispatch in persistent mode;       */
                            /* 0 = default (6 bf16: bulk copies; 16 MXFP8:      */
                            /* quantising warps).  Every CTA combines once its  */
-                           /* own role is done                                 */
+                           /* own role is done.  Must be 0 with dispatch_warps */
     int32_t gemm_ctas;     /* GEMM CTAs; 0 = all remaining SMs                  */
     int32_t mxfp8;         /* 1 = MXFP8 path (weights from                      */
                            /* mok_quantize_weights_mxfp8; either mode);         */
@@ -238,7 +238,12 @@ typedef struct mok_fwd_opts {
     int32_t save_for_backward; /* staged bf16 path: 1 = keep the gate and up    */
                            /* pre-activations (bf16) in the workspace for      */
                            /* mok_moe_backward                                 */
-    int32_t reserved;      /* must be 0                                         */
+    int32_t dispatch_warps; /* persistent mode, 1 or 2: no dispatch CTAs; every */
+                           /* CTA runs the GEMM and this many dispatch warps,  */
+                           /* which claim the expert-major rows 16 at a time   */
+                           /* and copy (MXFP8: quantise) them into the ring;   */
+                           /* they combine once the rows are all claimed.      */
+                           /* 0 = dispatch CTAs (dispatch_ctas)                */
     uint64_t timeout_ns;   /* bound on every device-side wait; 0 = 2 s          */
 } mok_fwd_opts;
 

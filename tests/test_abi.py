@@ -266,3 +266,18 @@ def test_router_entry_points_check_arguments():
     assert call(lo=8200) == mok.MOK_ERR_UNSUPPORTED
     assert call(xs=(ctypes.c_void_p * 2)(4096, 8200)) == mok.MOK_ERR_UNSUPPORTED
     assert call(ws=4096, nbytes=need - 1) == mok.MOK_ERR_WORKSPACE
+
+
+def test_forward_dispatch_warps_rules():
+    """The warp layout of the persistent kernel takes 1 or 2 dispatch warps
+    per CTA and no dispatch CTAs; both are checked before anything else is
+    touched (the pointers here are not device memory)."""
+    p = _filled_plan(16, 8, 2, 2)
+    L = mok.lib()
+    arr = (ctypes.c_void_p * 2)(4096, 8192)
+    for o, what in ((mok.fwd_opts(dispatch_warps=3), "dispatch_warps"),
+                    (mok.fwd_opts(dispatch_warps=-1), "dispatch_warps"),
+                    (mok.fwd_opts(dispatch_warps=1, dispatch_ctas=4), "exclude")):
+        rc = L.mok_moe_forward(arr, 128, 128, 4096, 4096, 4096, ctypes.byref(p), 256, ctypes.byref(o), 256,
+                               1 << 30, arr, None)
+        assert rc == mok.MOK_ERR_INVALID_ARG and what in mok.last_error(), mok.last_error()

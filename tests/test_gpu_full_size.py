@@ -2,7 +2,8 @@
 
 bf16 path (Mixtral-shaped, page and zipf shapes): every token of y is
 checked against the oracle, and the persistent SM-partitioned kernel (the
-configuration's minibatch and ring) must produce the staged path's bits.
+configuration's minibatch and ring; dispatch CTAs, and dispatch warps in
+every CTA) must produce the staged path's bits.
 MXFP8 page shape: every row is computed on the GPU, the persistent kernel
 is bit-identical to staged, and a token set that covers every expert (each
 expert's rows are checked through at least one of its tokens) is compared
@@ -23,11 +24,11 @@ PERSIST = mok.MOK_MODE_PERSISTENT
 REL_FRO_MX = 2e-2
 
 
-def _forward(case: Case, mode, minibatch, ring_slots=0):
+def _forward(case: Case, mode, minibatch, ring_slots=0, dispatch_warps=0):
     cfg = case.cfg
     p = mok.plan(case.dlogits, cfg.k, cfg.R)
     ys, ws = mok.moe_forward(case.x_shards(), case.dwg, case.dwu, case.dwd, p, minibatch,
-                             mok.fwd_opts(mode=mode, ring_slots=ring_slots))
+                             mok.fwd_opts(mode=mode, ring_slots=ring_slots, dispatch_warps=dispatch_warps))
     code = mok.get_status(ws)
     y = torch.cat([s.cpu() for s in ys])
     del ws, ys
@@ -57,6 +58,9 @@ def test_forward_full_size_every_token(name):
     y_p, code_p = _forward(case, PERSIST, cfg.minibatch, cfg.ring_slots)
     assert code_p == mok.MOK_OK
     assert torch.equal(y_p, y)
+    y_w, code_w = _forward(case, PERSIST, cfg.minibatch, cfg.ring_slots, dispatch_warps=2)
+    assert code_w == mok.MOK_OK
+    assert torch.equal(y_w, y)
     want = _oracle_all_tokens(case)
     assert_bf16_close(y, want, name)
 

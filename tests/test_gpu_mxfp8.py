@@ -128,7 +128,8 @@ def test_mxfp8_steps_one_at_a_time_equal_forward(name):
 
 
 @pytest.mark.parametrize("name,minibatch,ring,dispatch", [("tiny", 64, 0, 16), ("page_like", 256, 0, 4),
-                                                          ("page_like", 16, 0, 2), ("ragged", 600, 1300, 8)])
+                                                          ("page_like", 16, 0, 2), ("ragged", 600, 1300, 8),
+                                                          ("page_like", 256, 0, -2), ("ragged", 600, 1300, -1)])
 def test_mxfp8_persistent_equals_staged(name, minibatch, ring, dispatch):
     """The persistent SM-partitioned kernel on the MXFP8 path (its dispatch
     CTAs quantise the rows into the ring) computes the staged path's bits at
@@ -143,7 +144,9 @@ def test_mxfp8_persistent_equals_staged(name, minibatch, ring, dispatch):
     p = mok.plan(logits.cuda(), cfg.k, cfg.R)
     xs = mok.shards(x.cuda(), cfg.R)
     ys_s, ws_s = mok.moe_forward_mxfp8(xs, pack, p)
-    opts = mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT, mxfp8=True, ring_slots=ring, dispatch_ctas=dispatch)
+    # dispatch < 0: the warp layout (quantising dispatch warps in every CTA)
+    split = dict(dispatch_ctas=dispatch) if dispatch > 0 else dict(dispatch_warps=-dispatch)
+    opts = mok.fwd_opts(mode=mok.MOK_MODE_PERSISTENT, mxfp8=True, ring_slots=ring, **split)
     ys_p, ws_p = mok.moe_forward_mxfp8(xs, pack, p, minibatch=minibatch, opts=opts)
     assert mok.get_status(ws_s) == mok.MOK_OK and mok.get_status(ws_p) == mok.MOK_OK
     y_s = torch.cat([s.cpu() for s in ys_s])

@@ -46,6 +46,20 @@ def test_persistent_invariant_to_minibatch_ring_and_split(minibatch, ring, dispa
     assert torch.equal(y_p, y_s)
 
 
+@pytest.mark.parametrize("minibatch,ring,dwarps,gemm", [(16, 0, 1, 0), (256, 0, 2, 0), (600, 1300, 2, 0),
+                                                        (2560, 0, 2, 0), (128, 0, 1, 5), (4096, 8192, 1, 0)])
+def test_persistent_warp_layout_equals_staged(minibatch, ring, dwarps, gemm):
+    """The warp layout (no dispatch CTAs: every CTA runs the GEMM roles and
+    1 or 2 dispatch warps that claim rows 16 at a time) computes the staged
+    path's bits at every minibatch size, ring size and grid."""
+    cfg = mokgen.scaled(mokgen.CONFIGS["page"], E=48, T=1024)
+    case = Case(cfg)
+    y_s, _, _ = _run(case, STAGED, 0)
+    y_p, code, _ = _run(case, PERSIST, minibatch, ring_slots=ring, dispatch_warps=dwarps, gemm_ctas=gemm)
+    assert code == mok.MOK_OK, mok.last_error()
+    assert torch.equal(y_p, y_s)
+
+
 def test_persistent_small_gemm_grid():
     case = Case(FFN_CASES["multi_chunk"])
     y_s, _, _ = _run(case, STAGED, 0)
@@ -61,18 +75,20 @@ def test_persistent_wait_timeout_reports_status_and_recovers():
     case = Case(FFN_CASES["tiny"])
     cfg = case.cfg
     p = mok.plan(case.dlogits, cfg.k, cfg.R)
-    bad = mok.fwd_opts(mode=PERSIST, timeout_ns=1)
-    ys, ws = mok.moe_forward(case.x_shards(), case.dwg, case.dwu, case.dwd, p, 64, bad)
-    assert mok.get_status(ws) == mok.MOK_ERR_TIMEOUT
-    assert "status" in mok.last_error()
-    good = mok.fwd_opts(mode=PERSIST)
-    ys, ws = mok.moe_forward(case.x_shards(), case.dwg, case.dwu, case.dwd, p, 64, good, ws=ws)
-    assert mok.get_status(ws) == mok.MOK_OK
     y_s, _, _ = _run(case, STAGED, 0)
-    assert torch.equal(torch.cat(ys), y_s)
+    for dwarps in (0, 2):  # dispatch CTAs, then the warp layout
+        bad = mok.fwd_opts(mode=PERSIST, timeout_ns=1, dispatch_warps=dwarps)
+        ys, ws = mok.moe_forward(case.x_shards(), case.dwg, case.dwu, case.dwd, p, 64, bad)
+        assert mok.get_status(ws) == mok.MOK_ERR_TIMEOUT
+        assert "status" in mok.last_error()
+        good = mok.fwd_opts(mode=PERSIST, dispatch_warps=dwarps)
+        ys, ws = mok.moe_forward(case.x_shards(), case.dwg, case.dwu, case.dwd, p, 64, good, ws=ws)
+        assert mok.get_status(ws) == mok.MOK_OK
+        assert torch.equal(torch.cat(ys), y_s)
 
 
-@pytest.mark.parametrize("minibatch,ring,dispatch", [(64, 256, 4), (100, 320, 2), (16, 256, 8)])
+@pytest.mark.parametrize("minibatch,ring,dispatch", [(64, 256, 4), (100, 320, 2), (16, 256, 8), (64, 256, -1),
+                                                     (16, 256, -2)])
 def test_persistent_ring_wraps_on_a_small_shape(minibatch, ring, dispatch):
     """Experts far taller than the ring half (one takes most tokens): every
     expert is split across minibatches, the ring wraps many times and the
@@ -84,7 +100,9 @@ def test_persistent_ring_wraps_on_a_small_shape(minibatch, ring, dispatch):
     logits[:, 2] += 4.0                          # expert 2 is in almost every token's top-2
     case.logits, case.dlogits = logits, logits.cuda()
     y_s, code_s, _ = _run(case, STAGED, 0)
-    y_p, code_p, _ = _run(case, PERSIST, minibatch, ring_slots=ring, dispatch_ctas=dispatch)
+    # dispatch < 0: the warp layout with -dispatch dispatch warps per CTA
+    split = dict(dispatch_ctas=dispatch) if dispatch > 0 else dict(dispatch_warps=-dispatch)
+    y_p, code_p, _ = _run(case, PERSIST, minibatch, ring_slots=ring, **split)
     assert code_s == mok.MOK_OK and code_p == mok.MOK_OK
     counts = mok.plan(case.dlogits, cfg.k, cfg.R).counts().cpu()
     assert counts.max().item() > 4 * (ring // 2)  # the tallest expert spans several ring halves
