@@ -88,9 +88,9 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uin
     return true;
 }
 
-bool encode_bmaps(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err) {
+bool encode_bmaps(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err, int step) {
     for (int i = 0; i < B_MAPS; ++i)
-        if (!encode_tmap_2d_bf16(&maps->m[i], base, inner, rows, 64, (uint32_t)(16 * (i + 1)), err))
+        if (!encode_tmap_2d_bf16(&maps->m[i], base, inner, rows, 64, (uint32_t)(step * (i + 1)), err))
             return false;
     return true;
 }
@@ -141,7 +141,9 @@ bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* w
            encode_tmap_2d_bf16(&m->wu, wu, (uint64_t)I, (uint64_t)E * H, 64, 64, err) &&
            encode_tmap_2d_bf16(&m->wd, wd, (uint64_t)H, (uint64_t)E * I, 64, 64, err) &&
            encode_bmaps(&m->rows, rows, (uint64_t)H, (uint64_t)buf_rows, err) &&
-           encode_bmaps(&m->h, h, (uint64_t)I, (uint64_t)buf_rows, err);
+           encode_bmaps(&m->h, h, (uint64_t)I, (uint64_t)buf_rows, err) &&
+           encode_bmaps(&m->rows2, rows, (uint64_t)H, (uint64_t)buf_rows, err, 8) &&
+           encode_bmaps(&m->h2, h, (uint64_t)I, (uint64_t)buf_rows, err, 8);
 }
 
 // 2D map of a row-major [outer, inner] byte array.

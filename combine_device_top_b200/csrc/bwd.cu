@@ -130,19 +130,21 @@ cudaError_t launch_reverse_combine(const ShardsIn& dys, int S_r, int H, int T, i
 // K = the expert's rows, 64 per stage; both operands are MN-major tiles
 // (128-byte swizzle), each loaded as ONE 3D box of its 64-column blocks
 // ({64 columns, 64 rows, blocks}).  Rows of the last stage past the expert
-// belong to the next expert (or are TMA zero fill): a warp zeroes them in
-// the A tile (x or h rows; then every product with those rows is 0) while
-// the MMA works on the stage before.  Accumulators: two of NB columns in
-// TMEM, so one unit's epilogue overlaps the next's MMAs.  The epilogue
-// writes the bf16 tile into a 128-byte-swizzled staging tile and stores it
-// with TMA (one op per 64 columns).
-constexpr int WG_THREADS = 224;  // warp 0 TMA, 1 MMA, 2 tail zeroing, 3-6 epilogue
-constexpr int WG_NST = 3;
+// belong to the next expert (or are TMA zero fill): the MMA warp zeroes
+// them in the A tile (x or h rows; then every product with those rows is
+// 0) before it issues that stage.  Accumulators: two of NB columns in TMEM,
+// so one unit's epilogue overlaps the next's MMAs.  The epilogue writes the
+// bf16 tile 64 columns at a time into a ring of two 128-byte-swizzled
+// staging blocks and stores each block with one TMA op.
+constexpr int WG_THREADS = 192;  // warp 0 TMA, 1 MMA (and tail zeroing), 2-5 epilogue
+constexpr int WG_NST = 4;
 constexpr int WG_A_BYTES = 128 * 64 * 2;  // 16 KB
 constexpr int WG_NB_MAX = 256;
 constexpr int WG_STAGE_MAX = WG_A_BYTES + WG_NB_MAX * 128;  // 48 KB
-constexpr int WG_OUT_BYTES = 128 * WG_NB_MAX * 2;            // 64 KB staging tile
+constexpr int WG_OUT_BLOCK = 128 * 64 * 2;                   // one 64-column block of the tile, 16 KB
+constexpr int WG_OUT_BYTES = 2 * WG_OUT_BLOCK;               // ring of two blocks
 constexpr int WG_SMEM = WG_NST * WG_STAGE_MAX + WG_OUT_BYTES + 256 + 1024;
+static_assert(WG_SMEM <= 232448, "weight-gradient layout exceeds shared memory");
 // bound of the waits that drain this CTA's own loads and MMAs before it leaves
 constexpr uint64_t DRAIN_NS_WG = 1000000000ull;
 
@@ -194,10 +196,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                                                            ~uintptr_t(1023));
     const int b_bytes = a.nb * 64 * 2;
     const int stage_bytes = WG_A_BYTES + b_bytes;
-    unsigned char* otile = smem + WG_NST * WG_STAGE_MAX;                  // [nb/64][128 rows][128 B], swizzled
+    unsigned char* otile = smem + WG_NST * WG_STAGE_MAX;                  // 2 x [128 rows][128 B], swizzled
     uint64_t* full = reinterpret_cast<uint64_t*>(otile + WG_OUT_BYTES);  // TMA bytes landed
-    uint64_t* ready = full + WG_NST;                                     // tail rows zeroed
-    uint64_t* empty = ready + WG_NST;                                    // stage consumed (MMA commit)
+    uint64_t* empty = full + WG_NST;                                     // stage consumed (MMA commit)
     uint64_t* tfull = empty + WG_NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* fin = tempty + 2;
@@ -208,7 +209,6 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < WG_NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&ready[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -268,127 +268,126 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
             for (int s = 0; s < WG_NST; ++s)
                 if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, nullptr, DRAIN_NS_WG, 101);
         }
-    } else if (warp == 2) {
-        // ---- tail rows of the A tile zeroed, every stage passed on to the MMA
+    } else if (warp == 1) {
+        // ---- MMA (lane 0 waits and issues); the whole warp zeroes the A
+        // tile's rows past the expert in the unit's last stage first
         int stage = 0;
-        uint32_t phase = 0;
+        uint32_t phase = 0, tk = 0;
+        const uint32_t idesc = umma_idesc_f16(128, a.nb, /*A MN-major*/ 1, /*B MN-major*/ 1, /*bf16*/ 1);
         bool ok = true;
         for (int i = 0; ok && wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
+            if (w.rows == 0) continue;  // the epilogue writes zeros; no accumulator is used
             const int KB = (w.rows + 63) / 64;
+            int got = 0;
+            if (lane == 0) got = mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 102) ? 1 : 0;
+            if (__shfl_sync(0xffffffffu, got, 0) == 0) break;
+            tc_fence_after();
             for (int kb = 0; kb < KB; ++kb) {
-                int got = 0;
-                if (lane == 0) got = mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 106) ? 1 : 0;
+                if (lane == 0) got = mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 103) ? 1 : 0;
                 if (__shfl_sync(0xffffffffu, got, 0) == 0) {
                     ok = false;
                     break;
                 }
                 const int valid = min(64, w.rows - kb * 64);
-                if (valid < 64) {
-                    // a K row is one 128-byte line of each 64-column block (8 KB)
+                const int nks = (valid + 15) >> 4;  // MMAs of 16 K rows that hold any of the expert's rows
+                if (valid < nks * 16) {
+                    // a K row is one 128-byte line of each 64-column block (8 KB); only the
+                    // rows of the last MMA's 16 need zeros, the MMAs past it are not issued
                     unsigned char* st = smem + stage * WG_STAGE_MAX;
-                    const int lines = 64 - valid;
+                    const int lines = nks * 16 - valid;
                     for (int i2 = lane; i2 < 2 * lines * 8; i2 += 32) {
                         const int blk = i2 / (lines * 8), rem = i2 - blk * lines * 8;
                         *reinterpret_cast<uint4*>(st + blk * 8192 + (valid + rem / 8) * 128 + (rem % 8) * 16) =
                             make_uint4(0, 0, 0, 0);
                     }
-                    fence_proxy_async_shared();
+                    fence_proxy_async_shared();  // generic writes -> the MMA reads them
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ready[stage]);
-                if (++stage == WG_NST) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0, tk = 0;
-            const uint32_t idesc = umma_idesc_f16(128, a.nb, /*A MN-major*/ 1, /*B MN-major*/ 1, /*bf16*/ 1);
-            bool ok = true;
-            for (int i = 0; ok && wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
-                if (w.rows == 0) continue;  // the epilogue writes zeros; no accumulator is used
-                const int KB = (w.rows + 63) / 64;
-                if (!mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 102)) break;
-                tc_fence_after();
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&ready[stage], phase, a.st, a.timeout_ns, 103)) {
-                        ok = false;
-                        break;
-                    }
+                if (lane == 0) {
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + stage * WG_STAGE_MAX), sb = sa + WG_A_BYTES;
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
+                    for (int ks = 0; ks < nks; ++ks) {
                         // both MN-major SW128: 16 K rows = 2 atoms of 1 KB; 64-wide blocks 8 KB apart
                         const uint64_t ad = umma_desc_sw128(sa + ks * 2048, 8192, 1024);
                         const uint64_t bd = umma_desc_sw128(sb + ks * 2048, 8192, 1024);
                         umma_bf16(tmem + (tk & 1u) * 256u, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty[stage]);
-                    if (++stage == WG_NST) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
                 }
-                if (!ok) break;
-                umma_commit(&tfull[tk & 1u]);
-                ++tk;
+                __syncwarp();
+                if (++stage == WG_NST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
+            if (!ok) break;
+            if (lane == 0) umma_commit(&tfull[tk & 1u]);
+            ++tk;
+        }
+        if (lane == 0) {
             umma_commit(fin);
             mbar_wait(fin, 0, nullptr, DRAIN_NS_WG, 104);
         }
     } else {
-        // ---- epilogue: TMEM lane = output row m0 + 32 q + lane; bf16 into the
-        // swizzled staging tile, then TMA stores of its 64-column blocks
+        // ---- epilogue (warps 2-5; a warp reads TMEM lanes 32 (warp % 4) + 0..31):
+        // TMEM lane = output row m0 + 32 q + lane; bf16 into the swizzled
+        // staging blocks, one TMA store (and one bulk group) per 64-column
+        // block as soon as it is written.  A block buffer is written again
+        // two blocks later, once its store has read it (the one younger
+        // group may still be reading the other buffer).
         const int q = warp & 3;
         const int r = q * 32 + lane;  // row inside the tile
         const bool leader = warp == 3 && lane == 0;
-        uint32_t tk = 0;
+        const int nblk = a.nb / 64;
+        uint32_t tk = 0, gb = 0;
         for (int i = 0; wg_unit(a, blockIdx.x + i * gridDim.x, w); ++i) {
             int ok = 1;
             if (w.rows > 0 && lane == 0) ok = mbar_wait(&tfull[tk & 1u], (tk >> 1) & 1u, a.st, a.timeout_ns, 105) ? 1 : 0;
             if (lane == 0) ok_flags[q] = ok;
-            // the previous unit's stores have read the staging tile
-            if (leader) bulk_wait_read<0>();
             named_bar_sync(1, 128);
             // the four warps leave or go on together
             const int all_ok = ok_flags[0] & ok_flags[1] & ok_flags[2] & ok_flags[3];
             named_bar_sync(1, 128);  // the flags are written again at the next unit
             if (!all_ok) break;
             if (w.rows > 0) tc_fence_after();
-            for (int c = 0; c < a.nb; c += 32) {
-                float v[32];
-                if (w.rows > 0) {
-                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (tk & 1u) * 256u + (uint32_t)c, v);
-                } else {
+            const CUtensorMap* om = w.g == 0 ? &maps.owd : (w.g == 1 ? &maps.owg : &maps.owu);
+            const int y0 = w.e * (w.g == 0 ? a.I : a.H) + w.m0;
+            for (int b = 0; b < nblk; ++b, ++gb) {
+                unsigned char* buf = otile + (gb & 1u) * WG_OUT_BLOCK;
+                if (leader) bulk_wait_read<1>();
+                named_bar_sync(1, 128);  // the buffer is free
+                unsigned char* blk = buf + r * 128;
 #pragma unroll
-                    for (int p = 0; p < 32; ++p) v[p] = 0.f;
-                }
-                unsigned char* blk = otile + (c / 64) * (128 * 128) + r * 128;
+                for (int c2 = 0; c2 < 64; c2 += 32) {
+                    float v[32];
+                    if (w.rows > 0) {
+                        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (tk & 1u) * 256u + (uint32_t)(b * 64 + c2),
+                                           v);
+                    } else {
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const int chunk = ((c % 64) / 8) + p;  // 16-byte chunk of the row's 128-byte line
-                    *reinterpret_cast<uint4*>(blk + ((chunk ^ (r & 7)) << 4)) =
-                        make_uint4(pack_bf16x2(v[8 * p], v[8 * p + 1]), pack_bf16x2(v[8 * p + 2], v[8 * p + 3]),
-                                   pack_bf16x2(v[8 * p + 4], v[8 * p + 5]), pack_bf16x2(v[8 * p + 6], v[8 * p + 7]));
+                        for (int p = 0; p < 32; ++p) v[p] = 0.f;
+                    }
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const int chunk = c2 / 8 + p;  // 16-byte chunk of the row's 128-byte line
+                        *reinterpret_cast<uint4*>(blk + ((chunk ^ (r & 7)) << 4)) =
+                            make_uint4(pack_bf16x2(v[8 * p], v[8 * p + 1]), pack_bf16x2(v[8 * p + 2], v[8 * p + 3]),
+                                       pack_bf16x2(v[8 * p + 4], v[8 * p + 5]), pack_bf16x2(v[8 * p + 6], v[8 * p + 7]));
+                    }
                 }
-            }
-            if (w.rows > 0) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[tk & 1u]);
-                ++tk;
-            }
-            fence_proxy_async_shared();  // generic writes of the tile -> the TMA store reads them
-            named_bar_sync(1, 128);
-            if (leader) {
-                const CUtensorMap* om = w.g == 0 ? &maps.owd : (w.g == 1 ? &maps.owg : &maps.owu);
-                const int y0 = w.e * (w.g == 0 ? a.I : a.H) + w.m0;
-                for (int b = 0; b < a.nb / 64; ++b) tma_store_2d(om, otile + b * (128 * 128), w.n0 + b * 64, y0);
-                bulk_commit();
+                if (b == nblk - 1 && w.rows > 0) {
+                    // every column of the accumulator has been read
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[tk & 1u]);
+                    ++tk;
+                }
+                fence_proxy_async_shared();  // generic writes of the block -> the TMA store reads them
+                named_bar_sync(1, 128);
+                if (leader) {
+                    tma_store_2d(om, buf, w.n0 + b * 64, y0);
+                    bulk_commit();
+                }
             }
         }
         if (leader) bulk_wait_all();

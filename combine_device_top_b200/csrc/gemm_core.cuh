@@ -81,6 +81,7 @@ template <int SUB_, int NST_, bool EXT_ = false>
 struct Bf16CfgT {
     static constexpr bool MX = false;
     static constexpr bool EXT = EXT_;
+    static constexpr bool CG2 = false;
     static constexpr int SUB = SUB_;  // M tiles per unit
     static constexpr int THREADS = 320;  // warps: 0 TMA, 1 MMA, 2-9 two epilogue groups
     static constexpr int NST = NST_;
@@ -96,6 +97,29 @@ using Bf16PairCfg = Bf16CfgT<2, 3>;
 using Bf16ExtCfg = Bf16CfgT<1, 4, true>;
 using Bf16ExtPairCfg = Bf16CfgT<2, 3, true>;
 static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share the barrier offset");
+// bf16 forward on CTA pairs (tcgen05 cta_group::2): a cluster of two CTAs
+// runs each unit as one M = 256 MMA, CTA r holding M tile 2 m + r and half
+// of the token tile: [A 16 KB][B half <= 128 rows x 128 B] x 6.  Per SM a
+// stage carries 32 KB for the work a single-tile stage does with 48 KB,
+// like a pair of M tiles in one CTA, while each CTA keeps two 256-column
+// accumulators, so the epilogue still overlaps the next unit's MMAs.
+template <int NST_>
+struct Bf16Cta2CfgT {
+    static constexpr bool MX = false;
+    static constexpr bool EXT = false;
+    static constexpr bool CG2 = true;
+    static constexpr int SUB = 1;
+    static constexpr int THREADS = 320;  // warps: 0 TMA, 1 MMA (first CTA of the pair), 2-9 epilogue
+    static constexpr int NST = NST_;
+    static constexpr int BKX = BK;
+    static constexpr int STAGE = A_BYTES + B_BYTES / 2;
+    static constexpr int A_OFF = 0, B_OFF = A_BYTES;
+    static constexpr int EPI_OFF = NST * STAGE;
+    static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static_assert(SMEM <= 232448, "CTA-pair layout exceeds shared memory");
+};
+using Bf16Cta2Cfg = Bf16Cta2CfgT<6>;
 // MXFP8 path (block-scaled tcgen05 MMA, K = 128 per stage), SUB weight
 // tiles per unit: [A E4M3 SUB x 16 KB][B E4M3 <= 224 rows x 128 B][A scales
 // as loaded SUB x 512 B][B scales as loaded <= 1 KB][A scales, MMA layout
@@ -104,6 +128,7 @@ template <int SUB_, int NST_>
 struct MxCfgT {
     static constexpr bool MX = true;
     static constexpr bool EXT = false;
+    static constexpr bool CG2 = false;
     static constexpr int SUB = SUB_;
     static constexpr int THREADS = 352;  // warps: 0 TMA, 1 MMA, 2-9 epilogue, 10 scale-factor layout
     static constexpr int NST = NST_;
@@ -192,6 +217,36 @@ struct StagedSched {
         u.brow0 = ck.row0;
         u.rows = ck.rows;
         u.m = m;
+        u.grow0 = ck.row0;
+        u.chunk = c;
+        u.mb = ck.mb;
+        return true;
+    }
+    __device__ bool wait_inputs(const Unit&, DevStatus*, uint64_t) const { return true; }
+    __device__ bool unit_done(const Unit&) const { return false; }
+    __device__ void chunk_done(const Unit&, int, int) const {}
+};
+
+// CTA-pair schedule: units are (chunk, pair of M tiles), dealt round-robin
+// to the clusters; both CTAs of a cluster walk the same units, CTA r taking
+// M tile 2 m + r (u.m is that tile).  MT counts pairs.
+struct StagedSched2 {
+    static constexpr bool kSignals = false;
+    int phase, nch, MT, GC;
+    uint32_t rank;
+    const Chunk* chunks;
+
+    __device__ bool get(int i, Unit& u) const {
+        const int idx = (int)(blockIdx.x >> 1) + i * (int)(gridDim.x >> 1);
+        if (idx >= nch * MT) return false;
+        int c, m;
+        unit_map(idx, nch, MT, GC, c, m);
+        const Chunk ck = chunks[c];
+        u.phase = phase;
+        u.expert = ck.expert;
+        u.brow0 = ck.row0;
+        u.rows = ck.rows;
+        u.m = 2 * m + (int)rank;
         u.grow0 = ck.row0;
         u.chunk = c;
         u.mb = ck.mb;
@@ -327,6 +382,66 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const MxMaps
     // never leave with a load in flight into this CTA's shared memory
     for (int st = 0; st < C::NST; ++st)
         if ((issued >> st) & 1u) mbar_wait(&full[st], (issued_phase >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 11);
+}
+
+// ------------------------------------------------------------------ producer, CTA pairs
+// Each CTA of the pair loads its own M tile of weights and its half of the
+// token tile (rows [r N/2, (r + 1) N/2) of the chunk, N the 16-rounded row
+// count) into its own stage; both loads count their bytes on the FIRST
+// CTA's full[stage], whose producer expects the pair's total.  A stage is
+// reused once the MMA's commit has arrived on this CTA's empty[stage].
+template <class S, class C>
+__device__ __forceinline__ void gemm_producer_pair(const GemmMaps& maps, const CoreArgs& a, const S& s,
+                                                   unsigned char* smem, uint64_t* full, uint64_t* empty,
+                                                   uint32_t rank) {
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, issued_phase = 0;
+    const uint64_t evict_first = l2_policy_evict_first();
+    const uint64_t evict_normal = l2_policy_evict_normal();
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        const int K = phase_k<C>(a, u.phase);
+        const int KB = (K + C::BKX - 1) / C::BKX;
+        const BMaps& bm = u.phase == 0 ? maps.rows2 : maps.h2;
+        const int hb = ((u.rows + 15) >> 4) - 1;  // half tile of 8 (hb + 1) rows: map hb of the 8-row set
+        const int brow = u.brow0 + (int)rank * 8 * (hb + 1);
+        const uint32_t bytes = 2u * ((uint32_t)A_BYTES + (uint32_t)(8 * (hb + 1)) * B_ROW_BYTES);
+        const int mt = u.m;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 12)) {
+                ok = false;
+                break;
+            }
+            unsigned char* st = smem + stage * C::STAGE;
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], bytes);
+            const uint32_t full0 = smem_in_rank(&full[stage], 0);  // the first CTA's full[stage]
+            const int ky = u.expert * K + kb * C::BKX;
+            if (u.phase == 0) {
+                tma_load_2d_pair(st + C::A_OFF, &maps.wg, full0, mt * MT_G_FEATURES, ky, evict_first);
+                tma_load_2d_pair(st + C::A_OFF + A_BYTES / 2, &maps.wu, full0, mt * MT_G_FEATURES, ky, evict_first);
+            } else if (maps.has_wd3) {
+                tma_load_3d_pair(st + C::A_OFF, &maps.wd3, full0, 0, ky, mt * 2, evict_first);
+            } else {
+                tma_load_2d_pair(st + C::A_OFF, &maps.wd, full0, mt * MT_D_FEATURES, ky, evict_first);
+                tma_load_2d_pair(st + C::A_OFF + A_BYTES / 2, &maps.wd, full0, mt * MT_D_FEATURES + 64, ky,
+                                 evict_first);
+            }
+            tma_load_2d_pair(st + C::B_OFF, &bm.m[hb], full0, kb * C::BKX, brow, evict_normal);
+            issued |= 1u << stage;
+            issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == C::NST) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (!ok) break;
+    }
+    // never leave with a load in flight into this CTA's shared memory: the
+    // MMA's commit on empty[stage] follows the stage's loads (both CTAs')
+    for (int st = 0; st < C::NST; ++st)
+        if ((issued >> st) & 1u) mbar_wait(&empty[st], (issued_phase >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 13);
 }
 
 // ------------------------------------------------------------------ MXFP8 scale-factor layout (warp 10)
@@ -507,6 +622,59 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
     // wait for every MMA this thread issued before TMEM is released
     umma_commit(fin);
     mbar_wait(fin, 0, nullptr, DRAIN_TIMEOUT_NS, 22);
+}
+
+// ------------------------------------------------------------------ MMA issuer, CTA pairs
+// One thread of the pair's first CTA: per stage (both CTAs' loads counted
+// on full[stage]) 4 MMAs of M = 256, N = the 16-rounded rows, K = 16 into
+// both CTAs' accumulators; the stage's commit arrives on empty[stage] of
+// both CTAs, the unit's on tfull[] of both.  tempty[] (this CTA's) counts
+// the epilogue warps of both CTAs.
+template <class S, class C>
+__device__ __forceinline__ void gemm_mma_pair(const CoreArgs& a, const S& s, unsigned char* smem, uint64_t* full,
+                                              uint64_t* empty, uint64_t* tfull, uint64_t* tempty, uint64_t* fin,
+                                              uint32_t tmem_base) {
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t tk = 0;
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        const int K = phase_k<C>(a, u.phase);
+        const int KB = (K + C::BKX - 1) / C::BKX;
+        const int N = (u.rows + 15) & ~15;
+        const uint32_t idesc = umma_idesc_f16(256, N, /*A MN-major*/ 1, /*B K-major*/ 0, /*bf16*/ 1);
+        if (!mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 23)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 24)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + stage * C::STAGE + C::A_OFF);
+            const uint32_t sb = smem_u32(smem + stage * C::STAGE + C::B_OFF);
+#pragma unroll
+            for (int ks = 0; ks < BK / 16; ++ks) {
+                // same descriptors as one CTA's: A MN-major SW128 (halves 8 KB apart), B K-major SW128;
+                // the second CTA's rows sit at the same offsets in its shared memory
+                const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
+                const uint64_t ad = umma_desc_sw128(sa + ks * 2048, A_BYTES / 2, 1024);
+                umma_bf16_pair(tmem_base + (tk & 1u) * ACC_COLS, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair_both(&empty[stage], 0x3);
+            if (++stage == C::NST) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(&tfull[tk & 1u], 0x3);
+        ++tk;
+    }
+    // wait for every MMA this thread issued before TMEM is released
+    umma_commit_pair_local(fin);
+    mbar_wait(fin, 0, nullptr, DRAIN_TIMEOUT_NS, 25);
 }
 
 // ------------------------------------------------------------------ epilogue (warps 2..9)
@@ -691,11 +859,16 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
             epi_drain_tile<C>(a, u, u.m * C::SUB + sub, acc_col(tk, sub, wide), epi, tmem_base,
                               nsub == 2 ? 0 : g, nsub == 2 ? 1 : 2, bar);
         }
-        // this group is done with every buffer of the unit
+        // this group is done with every buffer of the unit (CTA pairs: on
+        // the first CTA's tempty, where the MMA issuer waits)
         tc_fence_before();
         __syncwarp();
-        if (lane == 0)
-            for (int t = 0; t < nt; ++t) mbar_arrive(&tempty[(tk + (uint32_t)t) & 1u]);
+        if (lane == 0) {
+            if constexpr (C::CG2)
+                mbar_arrive_cluster(smem_in_rank(&tempty[tk & 1u], 0));
+            else
+                for (int t = 0; t < nt; ++t) mbar_arrive(&tempty[(tk + (uint32_t)t) & 1u]);
+        }
         tk += (uint32_t)nt;
         if (S::kSignals) {
             // h rows are read next by TMA (async proxy) in some CTA: make this
@@ -755,7 +928,7 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 8);  // 4 warps of each epilogue group
+            mbar_init(&tempty[b], C::CG2 ? 16 : 8);  // 4 warps of each epilogue group (of both CTAs of a pair)
         }
         mbar_init(fin, 1);
         fence_mbar_init();
@@ -780,18 +953,35 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
         }
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (C::CG2) {
+            tmem_alloc_pair(tmem_slot, TMEM_COLS);  // both CTAs of the pair, same columns
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (C::CG2) cluster_sync_all();  // both CTAs' barriers and TMEM are set up
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    uint32_t rank = 0;
+    if constexpr (C::CG2) rank = cluster_ctarank();
 
     if (warp == 0) {
-        if (lane == 0) gemm_producer<S, C>(maps, mx, a, s, smem, full, empty);
+        if (lane == 0) {
+            if constexpr (C::CG2)
+                gemm_producer_pair<S, C>(maps, a, s, smem, full, empty, rank);
+            else
+                gemm_producer<S, C>(maps, mx, a, s, smem, full, empty);
+        }
     } else if (warp == 1) {
-        if (lane == 0) gemm_mma<S, C>(a, s, smem, C::MX ? sfready : full, empty, tfull, tempty, fin, tmem_base);
+        if constexpr (C::CG2) {
+            if (lane == 0 && rank == 0) gemm_mma_pair<S, C>(a, s, smem, full, empty, tfull, tempty, fin, tmem_base);
+        } else {
+            if (lane == 0) gemm_mma<S, C>(a, s, smem, C::MX ? sfready : full, empty, tfull, tempty, fin, tmem_base);
+        }
     } else if (warp < 10) {
         gemm_epilogue<S, C>(a, s, smem, tfull, tempty, ok_flags, done_cnt, tmem_base);
     } else if constexpr (C::MX) {
@@ -802,7 +992,15 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
     // beside them (barrier 3; the epilogue groups use 1 and 2)
     tc_fence_before();
     named_bar_sync(3, C::THREADS);
-    if (warp == 1) {
+    if constexpr (C::CG2) {
+        // the first CTA's MMAs (which read this CTA's shared memory and write
+        // its TMEM) have completed, and no epilogue still reads TMEM
+        cluster_sync_all();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        }
+    } else if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }

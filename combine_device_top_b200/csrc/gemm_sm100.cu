@@ -23,6 +23,49 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     gemm_cta<StagedSched, C>(maps, &mx, a, s, smem);
 }
 
+// The bf16 forward phases on CTA pairs (clusters of two): MT counts pairs of
+// M tiles.
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    k_grouped_gemm_pair(const __grid_constant__ GemmMaps maps, const CoreArgs a, const Chunk* __restrict__ chunks,
+                        const int* __restrict__ counts2, int phase, int MT, int GC) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = align_smem_1024(smem_raw);
+    StagedSched2 s;
+    s.phase = phase;
+    s.nch = *reinterpret_cast<volatile const int*>(counts2);
+    s.MT = MT;
+    s.GC = GC;
+    s.rank = cluster_ctarank();
+    s.chunks = chunks;
+    gemm_cta<StagedSched2, C>(maps, nullptr, a, s, smem);
+}
+
+template <class C>
+static cudaError_t launch_pair_phase(int grid, const GemmMaps& maps, const CoreArgs& a, const Chunk* chunks,
+                                     const int* counts2, int phase, int MT, int GC, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)(grid & ~1));
+    // as many pairs as can be resident at once (the grid walks its units)
+    int clusters = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, k_grouped_gemm_pair<C>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    if (2 * clusters < grid) grid = 2 * clusters;
+    cfg.gridDim = dim3((unsigned)(grid & ~1));
+    return cudaLaunchKernelEx(&cfg, k_grouped_gemm_pair<C>, maps, a, chunks, counts2, phase, MT, GC);
+}
+
 // Defaults measured on B200 (page shape and a 512-rows-per-expert case):
 // small raster groups paid.  Pairs of M tiles halve the token-tile bytes
 // each SM takes in per weight byte, but a pair of chunks taller than 128 rows
@@ -31,9 +74,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // used when the mean rows per expert is at most 192.  MOK_GEMM_GROUP and
 // MOK_GEMM_PAIR (0/1) override (tuning knobs only: results do not change).
 GemmTuning gemm_tuning(int rows, int E) {
-    GemmTuning v{2, rows <= 192 * E ? 1 : 0};
+    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 0};
     if (const char* s = getenv("MOK_GEMM_GROUP")) v.group_chunks = atoi(s) < 1 ? 1 : atoi(s);
     if (const char* s = getenv("MOK_GEMM_PAIR")) v.pair = atoi(s) != 0;
+    if (const char* s = getenv("MOK_GEMM_CTA_PAIR")) v.cta_pair = atoi(s) != 0;
     return v;
 }
 
@@ -54,6 +98,9 @@ cudaError_t gemm_configure(int dev) {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm<Bf16ExtPairCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Bf16ExtPairCfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm_pair<Bf16Cta2Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Bf16Cta2Cfg::SMEM);
 
     if (e == cudaSuccess) done[dev] = true;
     return e;
@@ -95,6 +142,9 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     const int sub = pair ? 2 : 1;
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
+    // CTA pairs: the bf16 forward phases, an even number of M tiles, an even grid
+    if (tune.cta_pair && !mx && !bwd && phase <= 1 && tiles % 2 == 0 && grid >= 2)
+        return launch_pair_phase<Bf16Cta2Cfg>(grid, maps, a, chunks, counts2, phase, tiles / 2, GC, stream);
     if (mx) {
         k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,
                                                                             MT, GC);

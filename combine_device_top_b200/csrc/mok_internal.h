@@ -94,9 +94,10 @@ struct GemmShape {
 struct GemmTuning {
     int group_chunks;  // raster group size in chunks
     int pair;          // 1: units of two M tiles sharing each token tile (bf16 path)
+    int cta_pair;      // 1: the bf16 forward launches run on CTA pairs (tcgen05 cta_group::2)
 };
 // defaults for `rows` expert-major rows over E experts, overridable by
-// MOK_GEMM_GROUP / MOK_GEMM_PAIR
+// MOK_GEMM_GROUP / MOK_GEMM_PAIR / MOK_GEMM_CTA_PAIR
 GemmTuning gemm_tuning(int rows, int E);
 cudaError_t gemm_configure(int dev);
 // Token-side (B operand) tensor maps of one buffer with box heights 16, 32,
@@ -107,7 +108,9 @@ constexpr int B_MAX_BOX = 256;
 struct BMaps {
     CUtensorMap m[B_MAPS];
 };
-bool encode_bmaps(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err);
+// box heights step, 2 step, ..., 16 step rows (step 16: a whole chunk's token
+// tile; step 8: one CTA's half of it in a CTA pair)
+bool encode_bmaps(BMaps* maps, const void* base, uint64_t inner, uint64_t rows, const char** err, int step = 16);
 
 // Every tensor map the GEMM core reads.
 struct GemmMaps {
@@ -115,6 +118,7 @@ struct GemmMaps {
     CUtensorMap wd3;         // Wd as {64, E*I, H/64}: one op loads both 64-column halves of a down tile
     BMaps rows;              // token rows (bf16) of the row buffer
     BMaps h;                 // h rows (bf16) of the h buffer
+    BMaps rows2, h2;         // the same with heights 8 .. 128 (half a token tile, CTA pairs)
     int has_wd3;             // wd3 could be encoded (else two 2D ops per down stage)
 };
 bool encode_gemm_maps(GemmMaps* m, const void* wg, const void* wu, const void* wd, const void* rows, const void* h,
