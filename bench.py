@@ -524,6 +524,10 @@ def staged_roofline(cfg, res, peaks, peak_src, mode, steps):
         "tensor_frac_of_measured_bf16": tflops / bf16_peak,
         "tensor_frac_of_dtype_peak": tflops / tc_peak,
         "tensor_frac_of_nominal_dense": tflops / nominal,
+        # both measured bf16 figures, whichever the region length picked: a
+        # power-capped run (clocks in `clocks`) is closer to the sustained one
+        "tensor_frac_of_bf16_burst": tflops / (peaks["bf16_tflops"] * (2.0 if cfg.mxfp8 else 1.0)),
+        "tensor_frac_of_bf16_sustained": tflops / (peaks["bf16_tflops_sustained"] * (2.0 if cfg.mxfp8 else 1.0)),
     })
     rates = {"gather_GBps": work["gather_bytes"] / (t_gather / 1e3) / 1e9,
              "combine_GBps": work["combine_bytes"] / (t_comb / 1e3) / 1e9,

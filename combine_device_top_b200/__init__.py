@@ -206,7 +206,7 @@ def plan(logits: torch.Tensor, top_k: int, R: int, ws: torch.Tensor | None = Non
 
 def router_prepare(w_r: torch.Tensor, stream=None):
     """``mok_router_prepare``: W_r [H, E] fp32 (device) -> (w_hi, w_lo), each
-    [E rounded up to 128, H] bf16."""
+    [E rounded up to 64, H] bf16."""
     assert w_r.is_cuda and w_r.dtype == torch.float32 and w_r.is_contiguous()
     H, E = w_r.shape
     nbytes = lib().mok_router_weights_bytes(H, E)

@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens(ShardsIn xs, int S
 // byte b: block 4g + b), the operand form of the block-scaled MMA.
 // Each lane owns 8 consecutive elements, 4 lanes a block, a half-warp one
 // 4-block scale word (warp_mx_quant8); the step loop is warp-uniform (lanes
-// past the end join the shuffles with zeros).
+// past the end join the shuffles with zeros).  Four 256-element steps'
+// loads are in flight per lane before the first is quantised.
 __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens_mx(ShardsIn xs, int S_r, int H, int T, int k,
                                                                  const int32_t* __restrict__ pos,
                                                                  uint8_t* __restrict__ rows, uint8_t* __restrict__ xsc,
@@ -69,19 +70,29 @@ __global__ void __launch_bounds__(DC_THREADS) k_gather_tokens_mx(ShardsIn xs, in
         const int r = t / S_r;
         const uint4* src = reinterpret_cast<const uint4*>(xs.p[r]) + (size_t)(t - r * S_r) * nvec;
         const int my_row = lane < k ? __ldg(pos + (size_t)t * k + lane) : 0;
-        for (int c0 = 0; c0 < H; c0 += 256) {
-            const int c = c0 + lane * 8;
-            const bool live = c < H;
-            const uint4 raw = live ? __ldg(src + (c >> 3)) : make_uint4(0, 0, 0, 0);
-            uint2 q;
-            uint32_t word;
-            warp_mx_quant8(raw, q, word, lane);
-            uint32_t* plane = reinterpret_cast<uint32_t*>(xsc) + (size_t)((c0 >> 7) + (lane >> 4)) * sc_rows;
-            for (int j = 0; j < k; ++j) {
-                const int row = __shfl_sync(0xffffffffu, my_row, j);
-                if (live) {
-                    *reinterpret_cast<uint2*>(rows + (size_t)row * H + c) = q;
-                    if ((lane & 15) == 0) plane[row] = word;
+        for (int c00 = 0; c00 < H; c00 += 1024) {
+            uint4 raw[4];
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                const int c = c00 + 256 * s4 + lane * 8;
+                raw[s4] = c < H ? __ldg(src + (c >> 3)) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                const int c0 = c00 + 256 * s4;
+                if (c0 >= H) break;  // warp-uniform
+                const int c = c0 + lane * 8;
+                const bool live = c < H;
+                uint2 q;
+                uint32_t word;
+                warp_mx_quant8(raw[s4], q, word, lane);
+                uint32_t* plane = reinterpret_cast<uint32_t*>(xsc) + (size_t)((c0 >> 7) + (lane >> 4)) * sc_rows;
+                for (int j = 0; j < k; ++j) {
+                    const int row = __shfl_sync(0xffffffffu, my_row, j);
+                    if (live) {
+                        *reinterpret_cast<uint2*>(rows + (size_t)row * H + c) = q;
+                        if ((lane & 15) == 0) plane[row] = word;
+                    }
                 }
             }
         }

@@ -137,7 +137,9 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     // measured, pairs were 6-10 % slower there (a tall pair fills TMEM, and
     // its quantising epilogue then stalls the next unit's MMAs).  The down
     // launch's units are short (K = I), so that stall weighs more there:
-    // pairs for gate/up only measured 3 % faster than pairs for both.
+    // pairs for gate/up only measured 3 % faster than pairs for both.  In
+    // the backward's dh and dx launches pairs measured 2 % slower (two runs
+    // each, one session).
     const bool pair = tune.pair && !mx && phase == 0;
     const int sub = pair ? 2 : 1;
     const int MT = (tiles + sub - 1) / sub;  // units along M

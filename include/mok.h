@@ -131,13 +131,13 @@ int mok_plan(const float* logits, int T, int E, int top_k, int R,
 enum { MOK_ROUTER_MAX_EXPERTS = 384 };
 
 /* Bytes of EACH of the two router weight parts made by mok_router_prepare:
- * [E rounded up to 128, H] bf16.  0 for an unsupported shape. */
+ * [E rounded up to 64, H] bf16.  0 for an unsupported shape. */
 size_t mok_router_weights_bytes(int H, int E);
 
 /*
  * mok_router_prepare -- one-time split of the router weights W_r [H, E]
  * fp32 (device) into two bf16 parts [E_pad, H] (expert-major, H
- * contiguous; E_pad = E rounded up to 128, padding rows zero):
+ * contiguous; E_pad = E rounded up to 64, padding rows zero):
  * w_hi = bf16(W_r), w_lo = bf16(W_r - w_hi), so w_hi + w_lo carries about
  * 16 significant bits of W_r with fp32's exponent range.  H % 64 == 0,
  * E <= MOK_ROUTER_MAX_EXPERTS; w_hi and w_lo (device, caller-owned,

@@ -246,7 +246,7 @@ def test_host_batches_reject_null_host_pointers_before_any_copy():
 def test_router_entry_points_check_arguments():
     L = mok.lib()
     assert L.mok_router_weights_bytes(7168, 384) == 384 * 7168 * 2
-    assert L.mok_router_weights_bytes(512, 8) == 128 * 512 * 2          # experts padded to 128 rows
+    assert L.mok_router_weights_bytes(512, 8) == 64 * 512 * 2           # experts padded to 64 rows (two halves)
     assert L.mok_router_weights_bytes(512, 385) == 0                      # above MOK_ROUTER_MAX_EXPERTS
     assert L.mok_router_prepare(4096, 512, 385, 4096, 8192, None) == mok.MOK_ERR_UNSUPPORTED
     assert L.mok_router_prepare(4096, 500, 8, 4096, 8192, None) == mok.MOK_ERR_UNSUPPORTED   # H % 64

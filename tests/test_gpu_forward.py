@@ -121,6 +121,27 @@ def test_grouped_gemm_m_tile_pairing_is_exact(name, monkeypatch):
     assert_bf16_close(decode_slots(got["1"], p.ns, cfg.H), want, name)
 
 
+@pytest.mark.parametrize("name", ["tiny", "many_experts", "wide", "k16"])
+def test_grouped_gemm_cta_pairs_are_exact(name, monkeypatch):
+    """The same phases on CTA pairs (clusters of two CTAs, one M = 256 MMA
+    over both CTAs' weight tiles, each CTA holding half of the token tile)
+    accumulate every output in the same K order: results are bit-identical
+    to one-CTA units, and match the oracle."""
+    case = Case(FFN_CASES[name])
+    cfg = case.cfg
+    p = mok.plan(case.dlogits, cfg.k, cfg.R)
+    rows = mok.gather(case.x_shards(), p)
+    got = {}
+    for cta_pair in ("0", "1"):
+        monkeypatch.setenv("MOK_GEMM_CTA_PAIR", cta_pair)
+        out, ws = mok.expert_ffn(rows, case.dwg, case.dwu, case.dwd, p)
+        assert mok.get_status(ws) == mok.MOK_OK, mok.last_error()
+        got[cta_pair] = out.cpu()
+    assert torch.equal(got["0"], got["1"])
+    want, _, _ = _oracle_slots(case, p)
+    assert_bf16_close(decode_slots(got["1"], p.ns, cfg.H), want, name)
+
+
 def test_grouped_gemm_single_expert_vs_torch_fp32():
     """E = 1, k = 1: the grouped GEMM is a dense SwiGLU FFN; compare with a
     plain PyTorch fp32 reference of the same op on the GPU (h rounded to
