@@ -38,6 +38,8 @@
 // Every wait is bounded; a wait that gives up records MOK_ERR_TIMEOUT in
 // the status word and the CTA skips to the end after draining its own loads
 // and MMAs (both CTAs still meet at the cluster barrier).
+#include <cstring>
+
 #include "mok_device.cuh"
 #include "mok_internal.h"
 #include "topk.cuh"
@@ -53,9 +55,16 @@ constexpr int RT_BAR_BYTES = 256;
 constexpr int RT_STAGE_BUDGET = RT_SMEM_MAX - 1024 - RT_BAR_BYTES;  // minus alignment slack and barriers
 constexpr uint64_t RT_DRAIN_NS = 1000000000ull;
 
+// x tiles by TMA when no 128-token tile straddles two shards (S_r % 128 == 0):
+// one {64 K, 128 tokens} box per shard map and stage
+struct RouterXMaps {
+    CUtensorMap m[MOK_MAX_SHARDS];
+};
+
 struct RouterArgs {
     ShardsIn xs;
     int S_r, T, H, E, k;
+    int x_tma;    // 1: x tiles by TMA (maps in RouterXMaps), else by the copy warps
     int eh;       // experts per CTA (a multiple of 32, <= 256)
     int nst;      // stages
     int stage;    // bytes per stage: A + the hi and lo B tiles
@@ -90,7 +99,7 @@ __device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t v) {
 template <int NC>
 __global__ void __launch_bounds__(RT_THREADS, 1)
     k_router(const __grid_constant__ CUtensorMap map_hi, const __grid_constant__ CUtensorMap map_lo,
-             const RouterArgs a) {
+             const __grid_constant__ RouterXMaps xmaps, const RouterArgs a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                            ~uintptr_t(1023));
@@ -132,14 +141,16 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---- W tiles of this CTA's experts
-            const uint32_t bytes = (uint32_t)(2 * a.eh * RT_BK * 2);
+            // ---- W tiles of this CTA's experts (and the x tile, by TMA)
+            const uint32_t bytes = (uint32_t)(2 * a.eh * RT_BK * 2 + (a.x_tma ? RT_A_BYTES : 0));
+            const int shard = t0 / a.S_r, srow = t0 - shard * a.S_r;
             int issued = 0;
             for (int kb = 0; kb < KB; ++kb) {
                 const int s = kb % a.nst;
                 if (!mbar_wait(&empty[s], ((kb / a.nst) & 1u) ^ 1u, a.st, a.timeout_ns, 90)) break;
                 unsigned char* b = smem + s * a.stage + RT_A_BYTES;
                 mbar_arrive_expect_tx(&full[s], bytes);
+                if (a.x_tma) tma_load_2d(smem + s * a.stage, &xmaps.m[shard], &full[s], kb * RT_BK, srow);
                 tma_load_2d(b, &map_hi, &full[s], kb * RT_BK, e_base);
                 tma_load_2d(b + a.eh * RT_BK * 2, &map_lo, &full[s], kb * RT_BK, e_base);
                 issued = kb + 1;
@@ -156,7 +167,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
                 const int s = kb % a.nst;
                 const uint32_t par = (kb / a.nst) & 1u;
                 if (!mbar_wait(&full[s], par, a.st, a.timeout_ns, 92)) break;
-                if (!mbar_wait(&afull[s], par, a.st, a.timeout_ns, 93)) break;
+                if (!a.x_tma && !mbar_wait(&afull[s], par, a.st, a.timeout_ns, 93)) break;
                 tc_fence_after();
                 const uint32_t sa = smem_u32(smem + s * a.stage);
                 const uint32_t sb = sa + RT_A_BYTES;
@@ -174,7 +185,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
             // the accumulator is final once every MMA issued has completed
             umma_commit(done);
         }
-    } else {
+    } else if (!a.x_tma) {
         // ---- x tile: thread et copies token t0 + et's 128 bytes of each K step
         // into its row of the stage's A tile (K-major, 128-byte swizzle: 16-byte
         // chunk c at slot c ^ (et & 7)) with asynchronous copies, the steps of
@@ -325,8 +336,8 @@ cudaError_t launch_router_split(const float* w, int H, int E, void* hi, void* lo
 }
 
 template <int NC>
-static cudaError_t launch_router_nc(const CUtensorMap& mh, const CUtensorMap& ml, const RouterArgs& a, int smem,
-                                   cudaStream_t stream) {
+static cudaError_t launch_router_nc(const CUtensorMap& mh, const CUtensorMap& ml, const RouterXMaps& xm,
+                                   const RouterArgs& a, int smem, cudaStream_t stream) {
     static bool attr[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -350,7 +361,7 @@ static cudaError_t launch_router_nc(const CUtensorMap& mh, const CUtensorMap& ml
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_router<NC>, mh, ml, a);
+    return cudaLaunchKernelEx(&cfg, k_router<NC>, mh, ml, xm, a);
 }
 
 cudaError_t launch_router(const ShardsIn& xs, int S_r, int T, int H, int E, int k, const void* w_hi,
@@ -389,12 +400,19 @@ cudaError_t launch_router(const ShardsIn& xs, int S_r, int T, int H, int E, int 
     if (!encode_tmap_2d_bf16(&mh, w_hi, (uint64_t)H, (uint64_t)ep, RT_BK, (uint32_t)a.eh, err) ||
         !encode_tmap_2d_bf16(&ml, w_lo, (uint64_t)H, (uint64_t)ep, RT_BK, (uint32_t)a.eh, err))
         return cudaErrorInvalidValue;
+    RouterXMaps xm;  // the kernel parameter (only the first R maps are read)
+    memset(&xm, 0, sizeof xm);
+    const int R = T / S_r;
+    a.x_tma = S_r % 128 == 0 ? 1 : 0;
+    if (a.x_tma)
+        for (int r = 0; r < R && a.x_tma; ++r)
+            if (!encode_tmap_2d_bf16(&xm.m[r], xs.p[r], (uint64_t)H, (uint64_t)S_r, RT_BK, 128, err)) a.x_tma = 0;
     const int smem = a.nst * a.stage + RT_BAR_BYTES + 1024;
     const int nc = a.eh / 32;
     *err = "router launch";
-    if (nc <= 2) return launch_router_nc<2>(mh, ml, a, smem, stream);
-    if (nc <= 4) return launch_router_nc<4>(mh, ml, a, smem, stream);
-    return launch_router_nc<8>(mh, ml, a, smem, stream);
+    if (nc <= 2) return launch_router_nc<2>(mh, ml, xm, a, smem, stream);
+    if (nc <= 4) return launch_router_nc<4>(mh, ml, xm, a, smem, stream);
+    return launch_router_nc<8>(mh, ml, xm, a, smem, stream);
 }
 
 }  // namespace mok
