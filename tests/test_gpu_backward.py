@@ -25,6 +25,9 @@ CASES = {
     "ragged": mokgen.scaled(mokgen.CONFIGS["tiny"], T=300, H=256, I=256, E=6, k=3, R=3, seed=402),
     "many_experts": mokgen.scaled(mokgen.CONFIGS["tiny"], T=192, H=384, I=128, E=24, k=4, R=2, seed=403),
     "wide": mokgen.scaled(mokgen.CONFIGS["tiny"], T=64, H=1024, I=512, E=4, k=2, R=2, seed=404),
+    # experts of about 640 rows: the weight-gradient kernel reloads the A
+    # tile for every N tile (more K stages than its resident slots)
+    "tall": mokgen.scaled(mokgen.CONFIGS["tiny"], T=640, H=256, I=256, E=2, k=2, R=2, seed=406),
 }
 
 
