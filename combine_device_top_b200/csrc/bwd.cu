@@ -59,13 +59,28 @@ __global__ void __launch_bounds__(256) k_reverse_combine(ShardsIn dys, int S_r, 
                 d[2 * p] = __uint_as_float(w[p] << 16);
                 d[2 * p + 1] = __uint_as_float(w[p] & 0xffff0000u);
             }
+            // the forward's slot rows: fp16 values, one power-of-two exponent per
+            // 128 features; the loads of up to 8 slots are issued before any is used
+            constexpr int C = KB < 8 ? KB : 8;
 #pragma unroll
-            for (int j = 0; j < KB; ++j) {
+            for (int j0 = 0; j0 < KB; j0 += C) {
+                if (j0 >= k) break;
+                uint4 ovs[C];
+                int exs[C];
+#pragma unroll
+                for (int c = 0; c < C; ++c) {
+                    if (j0 + c < k) {
+                        const size_t slot = (size_t)t * k + j0 + c;
+                        ovs[c] = __ldcs(reinterpret_cast<const uint4*>(o_slots + slot * H) + v);
+                        exs[c] = __ldg(o_exps + slot * (H >> 7) + (v >> 4));
+                    }
+                }
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const int j = j0 + c;
                 if (j < k) {
-                    // the forward's slot row: fp16 values, one power-of-two exponent per 128 features
-                    const size_t slot = (size_t)t * k + j;
-                    const uint4 ov = __ldcs(reinterpret_cast<const uint4*>(o_slots + slot * H) + v);
-                    const float sc = __int_as_float(((int)__ldg(o_exps + slot * (H >> 7) + (v >> 4)) + 127) << 23);
+                    const uint4 ov = ovs[c];
+                    const float sc = __int_as_float((exs[c] + 127) << 23);
                     const __half2* oh = reinterpret_cast<const __half2*>(&ov);
                     float acc = 0.f;
 #pragma unroll
@@ -79,6 +94,7 @@ __global__ void __launch_bounds__(256) k_reverse_combine(ShardsIn dys, int S_r, 
                         make_uint4(pack_bf16x2(g * d[0], g * d[1]), pack_bf16x2(g * d[2], g * d[3]),
                                    pack_bf16x2(g * d[4], g * d[5]), pack_bf16x2(g * d[6], g * d[7]));
                 }
+            }
             }
         }
         // dg_j over the warp; every lane ends with every sum
