@@ -439,8 +439,8 @@ def backward_work(cfg):
     ns, H, I, E, T = cfg.slots, cfg.H, cfg.I, cfg.E, cfg.T
     rc = T * H * 2 + ns * H * (2 + 1 / 128) + ns * H * 2 + T * E * 4  # dy, slot rows in; do rows, dlogits out
     dh = E * I * H * 2 + ns * H * 2 + 2 * ns * I * 2 + 2 * ns * I * 2  # Wd, do; a, b in; da, db out
-    dx = 2 * E * H * I * 2 + 2 * ns * I * 2 + ns * H * 4            # Wg, Wu, da, db in; fp32 dx rows out
-    rd = ns * H * 4 + T * H * 2                                      # dx rows in, dx out
+    dx = 2 * E * H * I * 2 + 2 * ns * I * 2 + ns * H * (2 + 1 / 128)  # Wg, Wu, da, db in; dx rows out (fp16 + exps)
+    rd = ns * H * (2 + 1 / 128) + T * H * 2                            # dx rows in, dx out
     wg = 3 * E * H * I * 2 + ns * (2 * H + I + 2 * I + H) * 2        # bf16 dW out; x, h, do, da|db rows in
     return {"flops": 12.0 * H * I * ns, "bytes": float(rc + dh + dx + rd + wg), "wgrad_bytes": float(wg)}
 

@@ -719,7 +719,7 @@ size_t mok_backward_workspace_bytes(int T, int H, int I, int E, int k) {
     if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return 0;
     const size_t ns = (size_t)T * k;
     return align256(sizeof(DevStatus)) + align256(ns * H * 2) + align256(ns * (size_t)I * 4) +
-           align256(ns * H * 4);
+           align256(slot_bytes(ns, H, MOK_SLOTS_F16S));
 }
 
 int mok_moe_backward(const void* const* dy_shards, int H, int I, const void* w_gate, const void* w_up,
@@ -763,7 +763,8 @@ int mok_moe_backward(const void* const* dy_shards, int H, int I, const void* w_g
     off += align256(ns * H * 2);
     uint16_t* dab = reinterpret_cast<uint16_t*>(base + off);
     off += align256(ns * (size_t)I * 4);
-    float* dx_slots = reinterpret_cast<float*>(base + off);
+    unsigned char* dx_slots = base + off;  // fp16 rows with one exponent per 128 features (MOK_SLOTS_F16S)
+    int8_t* dx_exps = reinterpret_cast<int8_t*>(dx_slots + slot_exp_offset(ns, H));
     ShardsIn dys{};
     ShardsOut dxs{};
     for (int r = 0; r < R; ++r) {
@@ -800,10 +801,10 @@ int mok_moe_backward(const void* const* dy_shards, int H, int I, const void* w_g
                                kDefaultTimeoutNs, sms, tune, stream, &bb),
              "dh GEMM launch");
     MOK_CUDA(launch_gemm_phase(3, maps, nullptr, nullptr, sh, chunks, counts2, nullptr, dx_slots, plan->row_slot,
-                               status, kDefaultTimeoutNs, sms, tune, stream, &bb),
+                               status, kDefaultTimeoutNs, sms, tune, stream, &bb, dx_exps),
              "dx GEMM launch");
     // 4. push reverse-dispatch: dx_t = sum of its k rows (the combine with unit weights)
-    MOK_CUDA(launch_combine(dx_slots, MOK_SLOTS_F32, nullptr, T, k, H, T / R, dxs, sms, stream),
+    MOK_CUDA(launch_combine(dx_slots, MOK_SLOTS_F16S, nullptr, T, k, H, T / R, dxs, sms, stream),
              "reverse dispatch launch");
     // 5. weight gradients per expert over its rows
     cudaError_t e = launch_wgrad(fb + FL.rows, fb + FL.h, do_rows, dab, (int)ns, plan->offsets, H, I, E, dw_gate,

@@ -167,8 +167,8 @@ struct Unit {
 struct CoreArgs {
     int H, I;
     void* h;                  // [buffer rows, I]: bf16 (bf16 path) or E4M3 (MXFP8 path)
-    void* out;                // [N_s, H] slot-indexed: fp16 + block exponents (bf16 path), bf16
-                              // (MXFP8 path), fp32 (backward dx rows)
+    void* out;                // [N_s, H] slot-indexed: fp16 + block exponents (bf16 path and the
+                              // backward's dx rows), bf16 (MXFP8 path)
     int8_t* out_exp;          // bf16 path: [N_s, H/128] exponents of the fp16 slot rows
     const int32_t* row_slot;  // [N_s]
     DevStatus* st;
@@ -790,8 +790,9 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 }
             }
         } else {
-            // push to the token's slot, one row per warp store (fp32: 512 bytes, MXFP8 path bf16: 256
-            // bytes); the combine rounds y once.  Phase 3 (dx rows) pushes the same way.
+            // push to the token's slot, one row per warp store (fp16 with the row's exponent for
+            // these 128 features, or bf16 on the MXFP8 path: 256 bytes); the combine rounds y
+            // once.  Phase 3 (the backward's dx rows) pushes the same way.
 #pragma unroll 4
             for (int it = 0; it < 8; ++it) {
                 const int t = it * 4 + q;
@@ -803,9 +804,6 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                     if constexpr (C::MX) {
                         reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + at)[lane] =
                             make_uint2(pack_bf16x2(o4.x, o4.y), pack_bf16x2(o4.z, o4.w));
-                    } else if constexpr (C::EXT) {
-                        // backward dx rows (phase 3): fp32
-                        reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + at)[lane] = o4;
                     } else {
                         // fp16 with one exponent for the row's 128 features of this tile
                         float m = fmaxf(fmaxf(fabsf(o4.x), fabsf(o4.y)), fmaxf(fabsf(o4.z), fabsf(o4.w)));

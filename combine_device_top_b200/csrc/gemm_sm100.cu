@@ -128,7 +128,7 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.h = h_out;
     a.out = out;
     a.out_exp = out_exp;
-    if (phase == 1 && !mx && !out_exp) return cudaErrorInvalidValue;  // fp16 slot rows need their exponents
+    if ((phase == 1 || phase == 3) && !mx && !out_exp) return cudaErrorInvalidValue;  // fp16 slot rows need their exponents
     a.row_slot = row_slot;
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;

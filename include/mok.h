@@ -342,7 +342,8 @@ int mok_minibatch_bounds(const mok_plan_t* plan, int H, int I, const void* w_gat
  * ---------------------------------------------------------------------- */
 
 /* Bytes of backward workspace: do rows [N_s, H] bf16, [da | db] rows
- * [N_s, 2I] bf16, dx rows [N_s, H] fp32 and a status word. */
+ * [N_s, 2I] bf16, dx rows [N_s, H] as MOK_SLOTS_F16S (fp16 values, one
+ * exponent per 128 features) and a status word. */
 size_t mok_backward_workspace_bytes(int T, int H, int I, int E, int k);
 
 /*
@@ -354,7 +355,8 @@ size_t mok_backward_workspace_bytes(int T, int H, int I, int E, int k);
  *      bf16 row in the expert-major layout, dg[t,j] = <dy_t, o[t,j]>;
  *   2. dh = do Wd^T (fp32 accumulation); da = dh b silu'(a),
  *      db = dh silu(a), rounded to bf16;
- *   3. dx rows = da Wg^T + db Wu^T (fp32), pushed to their token's slot;
+ *   3. dx rows = da Wg^T + db Wu^T (fp32 accumulation), pushed to their
+ *      token's slot as fp16 with one power-of-two exponent per 128 features;
  *   4. push reverse-dispatch: dx_t = bf16(sum_j dx rows of t), j ascending;
  *   5. dWd[e] = h^T do, dWg[e] = x^T da, dWu[e] = x^T db over the expert's
  *      rows (fp32 accumulation, bf16 results; an expert with no rows gets
