@@ -625,6 +625,9 @@ def main():
     ap.add_argument("--no-sub-records", action="store_true", help="time only the main workload")
     ap.add_argument("--backward", action="store_true",
                     help="time only mok_moe_backward on the workload (after one staged forward that keeps a, b)")
+    ap.add_argument("--router", action="store_true",
+                    help="time only mok_plan_router (the router projection, top-k and schedule) on the workload's "
+                         "tokens; no expert weights are built")
     ap.add_argument("--cpu-steps", type=int, default=64, help="experts the CPU baseline samples")
     ap.add_argument("--scale-experts", type=int, default=0,
                     help="profiling case: E experts and T scaled by the same factor (same rows per expert)")
@@ -670,6 +673,15 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    if args.router:
+        if rank == 0:
+            import types
+            import combine_device_top_b200 as mok
+
+            x = mokgen.tokens(cfg).to(device)
+            lite = types.SimpleNamespace(cfg=cfg, device=device, x_shards=mok.shards(x, cfg.R))
+            print(json.dumps(time_router(lite, args.steps, args.warmup)), flush=True)
+        return 0
     wl = Workload(cfg, device)
     if args.backward:
         if rank == 0:
