@@ -429,9 +429,10 @@ def time_router(wl: Workload, steps: int, warmup: int):
     flops = 2.0 * cfg.T * cfg.H * cfg.E            # useful: one projection
     return {"workload": f"{cfg.name}: {cfg.describe()}", "ms_per_call": ms, "tokens_per_s": cfg.T / (ms / 1e3),
             "useful_TFLOPs": flops / (ms / 1e3) / 1e12, "mma_TFLOPs": 2 * flops / (ms / 1e3) / 1e12,
-            "x_GBps": cfg.T * cfg.H * 2 / (ms / 1e3) / 1e9, "ctas": (cfg.T + 127) // 128, "steps": steps,
-            "note": "mok_plan_router: x (w_hi + w_lo) on tcgen05 (two bf16 MMAs per product), top-k and gates "
-                    "in the same kernel, then the schedule kernels"}
+            "x_GBps": cfg.T * cfg.H * 2 / (ms / 1e3) / 1e9, "ctas": 2 * ((cfg.T + 127) // 128), "steps": steps,
+            "note": "mok_plan_router: x (w_hi + w_lo) on tcgen05 (two bf16 MMAs per product), a CTA pair per "
+                    "128 tokens (half of the experts each), top-k and gates in the same kernel, then the schedule "
+                    "kernels"}
 
 
 def backward_work(cfg):
