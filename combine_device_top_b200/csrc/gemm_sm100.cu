@@ -74,10 +74,10 @@ static cudaError_t launch_pair_phase(int grid, const GemmMaps& maps, const CoreA
 // used when the mean rows per expert is at most 192.  MOK_GEMM_GROUP and
 // MOK_GEMM_PAIR (0/1) override (tuning knobs only: results do not change).
 GemmTuning gemm_tuning(int rows, int E) {
-    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 0};
+    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 1};
     if (const char* s = getenv("MOK_GEMM_GROUP")) v.group_chunks = atoi(s) < 1 ? 1 : atoi(s);
     if (const char* s = getenv("MOK_GEMM_PAIR")) v.pair = atoi(s) != 0;
-    if (const char* s = getenv("MOK_GEMM_CTA_PAIR")) v.cta_pair = atoi(s) != 0;
+    if (const char* s = getenv("MOK_GEMM_CTA_PAIR")) v.cta_pair = atoi(s) < 0 ? 0 : atoi(s);
     return v;
 }
 
@@ -144,8 +144,13 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     const int sub = pair ? 2 : 1;
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
-    // CTA pairs: the bf16 forward phases, an even number of M tiles, an even grid
-    if (tune.cta_pair && !mx && !bwd && phase <= 1 && tiles % 2 == 0 && grid >= 2)
+    // CTA pairs: the bf16 forward phases (by default the down phase only), an
+    // even number of M tiles, an even grid.  Measured on B200 (ncu launch
+    // times, one session): down on CTA pairs 5 % faster than single tiles at
+    // the page shape and 1 % at the zipf shape; gate/up on CTA pairs 4 %
+    // slower than M-tile pairs (page) and 5 % slower than single tiles (zipf).
+    const bool cta2 = tune.cta_pair >= 2 || (tune.cta_pair == 1 && phase == 1);
+    if (cta2 && !mx && !bwd && phase <= 1 && tiles % 2 == 0 && grid >= 2)
         return launch_pair_phase<Bf16Cta2Cfg>(grid, maps, a, chunks, counts2, phase, tiles / 2, GC, stream);
     if (mx) {
         k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,
