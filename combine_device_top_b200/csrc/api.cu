@@ -787,7 +787,9 @@ int mok_moe_backward(const void* const* dy_shards, int H, int I, const void* w_g
         !encode_tmap_2d_bf16(&maps.wg, w_gate, (uint64_t)I, (uint64_t)E * H, 64, 128, &err) ||
         !encode_tmap_2d_bf16(&maps.wu, w_up, (uint64_t)I, (uint64_t)E * H, 64, 128, &err) ||
         !encode_bmaps(&maps.rows, do_rows, (uint64_t)H, (uint64_t)ns, &err) ||
-        !encode_bmaps(&maps.h, dab, (uint64_t)2 * I, (uint64_t)ns, &err))
+        !encode_bmaps(&maps.h, dab, (uint64_t)2 * I, (uint64_t)ns, &err) ||
+        !encode_bmaps(&maps.rows2, do_rows, (uint64_t)H, (uint64_t)ns, &err, 8) ||
+        !encode_bmaps(&maps.h2, dab, (uint64_t)2 * I, (uint64_t)ns, &err, 8))
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
     BwdBuffers bb{};
     bb.save_a = reinterpret_cast<uint16_t*>(const_cast<unsigned char*>(fb) + FL.save_a);

@@ -103,10 +103,10 @@ static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share
 // stage carries 32 KB for the work a single-tile stage does with 48 KB,
 // like a pair of M tiles in one CTA, while each CTA keeps two 256-column
 // accumulators, so the epilogue still overlaps the next unit's MMAs.
-template <int NST_>
+template <int NST_, bool EXT_ = false>
 struct Bf16Cta2CfgT {
     static constexpr bool MX = false;
-    static constexpr bool EXT = false;
+    static constexpr bool EXT = EXT_;  // also the backward's dh and dx phases (2, 3)
     static constexpr bool CG2 = true;
     static constexpr int SUB = 1;
     static constexpr int THREADS = 320;  // warps: 0 TMA, 1 MMA (first CTA of the pair), 2-9 epilogue
@@ -120,6 +120,7 @@ struct Bf16Cta2CfgT {
     static_assert(SMEM <= 232448, "CTA-pair layout exceeds shared memory");
 };
 using Bf16Cta2Cfg = Bf16Cta2CfgT<6>;
+using Bf16Cta2ExtCfg = Bf16Cta2CfgT<6, true>;
 // MXFP8 path (block-scaled tcgen05 MMA, K = 128 per stage), SUB weight
 // tiles per unit: [A E4M3 SUB x 16 KB][B E4M3 <= 224 rows x 128 B][A scales
 // as loaded SUB x 512 B][B scales as loaded <= 1 KB][A scales, MMA layout
@@ -403,7 +404,7 @@ __device__ __forceinline__ void gemm_producer_pair(const GemmMaps& maps, const C
     for (int i = 0; s.get(i, u); ++i) {
         const int K = phase_k<C>(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
-        const BMaps& bm = u.phase == 0 ? maps.rows2 : maps.h2;
+        const BMaps& bm = (u.phase == 0 || (C::EXT && u.phase == 2)) ? maps.rows2 : maps.h2;
         const int hb = ((u.rows + 15) >> 4) - 1;  // half tile of 8 (hb + 1) rows: map hb of the 8-row set
         const int brow = u.brow0 + (int)rank * 8 * (hb + 1);
         const uint32_t bytes = 2u * ((uint32_t)A_BYTES + (uint32_t)(8 * (hb + 1)) * B_ROW_BYTES);
@@ -421,6 +422,16 @@ __device__ __forceinline__ void gemm_producer_pair(const GemmMaps& maps, const C
             if (u.phase == 0) {
                 tma_load_2d_pair(st + C::A_OFF, &maps.wg, full0, mt * MT_G_FEATURES, ky, evict_first);
                 tma_load_2d_pair(st + C::A_OFF + A_BYTES / 2, &maps.wu, full0, mt * MT_G_FEATURES, ky, evict_first);
+            } else if (C::EXT && u.phase == 2) {
+                // Wd [E*I, H] K-major: 128 feature rows x 64 K in one box
+                tma_load_2d_pair(st + C::A_OFF, &maps.wd, full0, kb * BK, u.expert * a.I + mt * MT_D_FEATURES,
+                                 evict_first);
+            } else if (C::EXT && u.phase == 3) {
+                // Wg then Wu [E*H, I] K-major: K runs over I twice
+                const int KI = a.I / BK;
+                const bool up = kb >= KI;
+                tma_load_2d_pair(st + C::A_OFF, up ? &maps.wu : &maps.wg, full0, (kb - (up ? KI : 0)) * BK,
+                                 u.expert * a.H + mt * MT_D_FEATURES, evict_first);
             } else if (maps.has_wd3) {
                 tma_load_3d_pair(st + C::A_OFF, &maps.wd3, full0, 0, ky, mt * 2, evict_first);
             } else {
@@ -642,7 +653,8 @@ __device__ __forceinline__ void gemm_mma_pair(const CoreArgs& a, const S& s, uns
         const int K = phase_k<C>(a, u.phase);
         const int KB = (K + C::BKX - 1) / C::BKX;
         const int N = (u.rows + 15) & ~15;
-        const uint32_t idesc = umma_idesc_f16(256, N, /*A MN-major*/ 1, /*B K-major*/ 0, /*bf16*/ 1);
+        const bool a_kmaj = C::EXT && u.phase >= 2;  // the backward reads the weights K-major
+        const uint32_t idesc = umma_idesc_f16(256, N, a_kmaj ? 0 : 1, /*B K-major*/ 0, /*bf16*/ 1);
         if (!mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 23)) break;
         tc_fence_after();
         bool ok = true;
@@ -659,7 +671,8 @@ __device__ __forceinline__ void gemm_mma_pair(const CoreArgs& a, const S& s, uns
                 // same descriptors as one CTA's: A MN-major SW128 (halves 8 KB apart), B K-major SW128;
                 // the second CTA's rows sit at the same offsets in its shared memory
                 const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
-                const uint64_t ad = umma_desc_sw128(sa + ks * 2048, A_BYTES / 2, 1024);
+                const uint64_t ad = a_kmaj ? umma_desc_sw128(sa + ks * 32, 16, 1024)
+                                           : umma_desc_sw128(sa + ks * 2048, A_BYTES / 2, 1024);
                 umma_bf16_pair(tmem_base + (tk & 1u) * ACC_COLS, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
             }
             umma_commit_pair_both(&empty[stage], 0x3);

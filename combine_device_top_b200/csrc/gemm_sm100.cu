@@ -101,6 +101,9 @@ cudaError_t gemm_configure(int dev) {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm_pair<Bf16Cta2Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Bf16Cta2Cfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm_pair<Bf16Cta2ExtCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Bf16Cta2ExtCfg::SMEM);
 
     if (e == cudaSuccess) done[dev] = true;
     return e;
@@ -144,14 +147,18 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     const int sub = pair ? 2 : 1;
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
-    // CTA pairs: the bf16 forward phases (by default the down phase only), an
-    // even number of M tiles, an even grid.  Measured on B200 (ncu launch
+    // CTA pairs: the bf16 phases (by default all but gate/up), an even number
+    // of M tiles, an even grid.  Measured on B200 (ncu launch
     // times, one session): down on CTA pairs 5 % faster than single tiles at
     // the page shape and 1 % at the zipf shape; gate/up on CTA pairs 4 %
     // slower than M-tile pairs (page) and 5 % slower than single tiles (zipf).
-    const bool cta2 = tune.cta_pair >= 2 || (tune.cta_pair == 1 && phase == 1);
-    if (cta2 && !mx && !bwd && phase <= 1 && tiles % 2 == 0 && grid >= 2)
-        return launch_pair_phase<Bf16Cta2Cfg>(grid, maps, a, chunks, counts2, phase, tiles / 2, GC, stream);
+    const bool cta2 = tune.cta_pair >= 2 || (tune.cta_pair == 1 && phase != 0);
+    if (cta2 && !mx && tiles % 2 == 0 && grid >= 2) {
+        if (phase >= 2)  // the backward's dh and dx phases
+            return launch_pair_phase<Bf16Cta2ExtCfg>(grid, maps, a, chunks, counts2, phase, tiles / 2, GC, stream);
+        if (!bwd)
+            return launch_pair_phase<Bf16Cta2Cfg>(grid, maps, a, chunks, counts2, phase, tiles / 2, GC, stream);
+    }
     if (mx) {
         k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,
                                                                             MT, GC);

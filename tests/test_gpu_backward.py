@@ -86,3 +86,16 @@ def test_save_for_backward_keeps_the_forward_bits():
     y1, _ = mok.moe_forward(xs, *w, p, 0, mok.fwd_opts(mode=mok.MOK_MODE_STAGED))
     y2, _ = mok.moe_forward(xs, *w, p, 0, mok.fwd_opts(mode=mok.MOK_MODE_STAGED, save_for_backward=True))
     assert torch.equal(torch.cat(y1), torch.cat(y2))
+
+
+@pytest.mark.parametrize("name", ["wide", "tall"])
+def test_backward_cta_pairs_are_exact(name, monkeypatch):
+    """The dh and dx phases on CTA pairs (one M = 256 MMA over two SMs) give
+    the same bits as on single CTAs; the weight gradients do not depend on
+    the setting at all."""
+    got = {}
+    for cta_pair in ("0", "1"):
+        monkeypatch.setenv("MOK_GEMM_CTA_PAIR", cta_pair)
+        got[cta_pair], _, _, _ = _run(CASES[name])
+    for key in ("dx", "dwg", "dwu", "dwd", "dlogits"):
+        assert torch.equal(got["0"][key], got["1"][key]), key
