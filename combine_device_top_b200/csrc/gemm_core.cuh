@@ -103,17 +103,19 @@ static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share
 // stage carries 32 KB for the work a single-tile stage does with 48 KB,
 // like a pair of M tiles in one CTA, while each CTA keeps two 256-column
 // accumulators, so the epilogue still overlaps the next unit's MMAs.
-template <int NST_, bool EXT_ = false>
+// SUB_ = 2: each CTA holds two M tiles (a cluster covers four), sharing its
+// half of the token tile: [A0 16 KB][A1 16 KB][B half] x 4.
+template <int NST_, bool EXT_ = false, int SUB_ = 1>
 struct Bf16Cta2CfgT {
     static constexpr bool MX = false;
     static constexpr bool EXT = EXT_;  // also the backward's dh and dx phases (2, 3)
     static constexpr bool CG2 = true;
-    static constexpr int SUB = 1;
+    static constexpr int SUB = SUB_;  // M tiles per CTA and unit
     static constexpr int THREADS = 320;  // warps: 0 TMA, 1 MMA (first CTA of the pair), 2-9 epilogue
     static constexpr int NST = NST_;
     static constexpr int BKX = BK;
-    static constexpr int STAGE = A_BYTES + B_BYTES / 2;
-    static constexpr int A_OFF = 0, B_OFF = A_BYTES;
+    static constexpr int STAGE = SUB * A_BYTES + B_BYTES / 2;
+    static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
     static constexpr int EPI_OFF = NST * STAGE;
     static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
@@ -121,6 +123,7 @@ struct Bf16Cta2CfgT {
 };
 using Bf16Cta2Cfg = Bf16Cta2CfgT<6>;
 using Bf16Cta2ExtCfg = Bf16Cta2CfgT<6, true>;
+using Bf16Cta2PairCfg = Bf16Cta2CfgT<4, false, 2>;
 // MXFP8 path (block-scaled tcgen05 MMA, K = 128 per stage), SUB weight
 // tiles per unit: [A E4M3 SUB x 16 KB][B E4M3 <= 224 rows x 128 B][A scales
 // as loaded SUB x 512 B][B scales as loaded <= 1 KB][A scales, MMA layout
@@ -228,9 +231,10 @@ struct StagedSched {
     __device__ void chunk_done(const Unit&, int, int) const {}
 };
 
-// CTA-pair schedule: units are (chunk, pair of M tiles), dealt round-robin
+// CTA-pair schedule: units are (chunk, 2 C::SUB M tiles), dealt round-robin
 // to the clusters; both CTAs of a cluster walk the same units, CTA r taking
-// M tile 2 m + r (u.m is that tile).  MT counts pairs.
+// M tiles (2 m + r) C::SUB + s (u.m = 2 m + r, in units of C::SUB tiles).
+// MT counts cluster units.
 struct StagedSched2 {
     static constexpr bool kSignals = false;
     int phase, nch, MT, GC;
@@ -407,8 +411,8 @@ __device__ __forceinline__ void gemm_producer_pair(const GemmMaps& maps, const C
         const BMaps& bm = (u.phase == 0 || (C::EXT && u.phase == 2)) ? maps.rows2 : maps.h2;
         const int hb = ((u.rows + 15) >> 4) - 1;  // half tile of 8 (hb + 1) rows: map hb of the 8-row set
         const int brow = u.brow0 + (int)rank * 8 * (hb + 1);
-        const uint32_t bytes = 2u * ((uint32_t)A_BYTES + (uint32_t)(8 * (hb + 1)) * B_ROW_BYTES);
-        const int mt = u.m;
+        const int nsub = unit_subs<C>(a, u);  // the same in both CTAs (whole cluster units)
+        const uint32_t bytes = 2u * ((uint32_t)(nsub * A_BYTES) + (uint32_t)(8 * (hb + 1)) * B_ROW_BYTES);
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, a.st, a.timeout_ns, 12)) {
@@ -419,25 +423,27 @@ __device__ __forceinline__ void gemm_producer_pair(const GemmMaps& maps, const C
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], bytes);
             const uint32_t full0 = smem_in_rank(&full[stage], 0);  // the first CTA's full[stage]
             const int ky = u.expert * K + kb * C::BKX;
-            if (u.phase == 0) {
-                tma_load_2d_pair(st + C::A_OFF, &maps.wg, full0, mt * MT_G_FEATURES, ky, evict_first);
-                tma_load_2d_pair(st + C::A_OFF + A_BYTES / 2, &maps.wu, full0, mt * MT_G_FEATURES, ky, evict_first);
-            } else if (C::EXT && u.phase == 2) {
-                // Wd [E*I, H] K-major: 128 feature rows x 64 K in one box
-                tma_load_2d_pair(st + C::A_OFF, &maps.wd, full0, kb * BK, u.expert * a.I + mt * MT_D_FEATURES,
-                                 evict_first);
-            } else if (C::EXT && u.phase == 3) {
-                // Wg then Wu [E*H, I] K-major: K runs over I twice
-                const int KI = a.I / BK;
-                const bool up = kb >= KI;
-                tma_load_2d_pair(st + C::A_OFF, up ? &maps.wu : &maps.wg, full0, (kb - (up ? KI : 0)) * BK,
-                                 u.expert * a.H + mt * MT_D_FEATURES, evict_first);
-            } else if (maps.has_wd3) {
-                tma_load_3d_pair(st + C::A_OFF, &maps.wd3, full0, 0, ky, mt * 2, evict_first);
-            } else {
-                tma_load_2d_pair(st + C::A_OFF, &maps.wd, full0, mt * MT_D_FEATURES, ky, evict_first);
-                tma_load_2d_pair(st + C::A_OFF + A_BYTES / 2, &maps.wd, full0, mt * MT_D_FEATURES + 64, ky,
-                                 evict_first);
+            for (int sub = 0; sub < nsub; ++sub) {
+                unsigned char* sa = st + C::A_OFF + sub * A_BYTES;
+                const int mt = u.m * C::SUB + sub;
+                if (u.phase == 0) {
+                    tma_load_2d_pair(sa, &maps.wg, full0, mt * MT_G_FEATURES, ky, evict_first);
+                    tma_load_2d_pair(sa + A_BYTES / 2, &maps.wu, full0, mt * MT_G_FEATURES, ky, evict_first);
+                } else if (C::EXT && u.phase == 2) {
+                    // Wd [E*I, H] K-major: 128 feature rows x 64 K in one box
+                    tma_load_2d_pair(sa, &maps.wd, full0, kb * BK, u.expert * a.I + mt * MT_D_FEATURES, evict_first);
+                } else if (C::EXT && u.phase == 3) {
+                    // Wg then Wu [E*H, I] K-major: K runs over I twice
+                    const int KI = a.I / BK;
+                    const bool up = kb >= KI;
+                    tma_load_2d_pair(sa, up ? &maps.wu : &maps.wg, full0, (kb - (up ? KI : 0)) * BK,
+                                     u.expert * a.H + mt * MT_D_FEATURES, evict_first);
+                } else if (maps.has_wd3) {
+                    tma_load_3d_pair(sa, &maps.wd3, full0, 0, ky, mt * 2, evict_first);
+                } else {
+                    tma_load_2d_pair(sa, &maps.wd, full0, mt * MT_D_FEATURES, ky, evict_first);
+                    tma_load_2d_pair(sa + A_BYTES / 2, &maps.wd, full0, mt * MT_D_FEATURES + 64, ky, evict_first);
+                }
             }
             tma_load_2d_pair(st + C::B_OFF, &bm.m[hb], full0, kb * C::BKX, brow, evict_normal);
             issued |= 1u << stage;
@@ -655,9 +661,16 @@ __device__ __forceinline__ void gemm_mma_pair(const CoreArgs& a, const S& s, uns
         const int N = (u.rows + 15) & ~15;
         const bool a_kmaj = C::EXT && u.phase >= 2;  // the backward reads the weights K-major
         const uint32_t idesc = umma_idesc_f16(256, N, a_kmaj ? 0 : 1, /*B K-major*/ 0, /*bf16*/ 1);
-        if (!mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 23)) break;
-        tc_fence_after();
+        const int nsub = unit_subs<C>(a, u);
+        const int nt = unit_tickets<C>(nsub, N);
+        const bool wide = nt == 2;
         bool ok = true;
+        for (int t = 0; t < nt && ok; ++t) {
+            const uint32_t tkt = tk + (uint32_t)t;
+            ok = mbar_wait(&tempty[tkt & 1u], ((tkt >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 23);
+        }
+        if (!ok) break;
+        tc_fence_after();
         for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 24)) {
                 ok = false;
@@ -671,9 +684,15 @@ __device__ __forceinline__ void gemm_mma_pair(const CoreArgs& a, const S& s, uns
                 // same descriptors as one CTA's: A MN-major SW128 (halves 8 KB apart), B K-major SW128;
                 // the second CTA's rows sit at the same offsets in its shared memory
                 const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
-                const uint64_t ad = a_kmaj ? umma_desc_sw128(sa + ks * 32, 16, 1024)
-                                           : umma_desc_sw128(sa + ks * 2048, A_BYTES / 2, 1024);
-                umma_bf16_pair(tmem_base + (tk & 1u) * ACC_COLS, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+#pragma unroll
+                for (int sub = 0; sub < C::SUB; ++sub) {
+                    if (sub < nsub) {
+                        const uint32_t s0 = sa + sub * A_BYTES;
+                        const uint64_t ad = a_kmaj ? umma_desc_sw128(s0 + ks * 32, 16, 1024)
+                                                   : umma_desc_sw128(s0 + ks * 2048, A_BYTES / 2, 1024);
+                        umma_bf16_pair(tmem_base + acc_col(tk, sub, wide), ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                    }
+                }
             }
             umma_commit_pair_both(&empty[stage], 0x3);
             if (++stage == C::NST) {
@@ -682,8 +701,8 @@ __device__ __forceinline__ void gemm_mma_pair(const CoreArgs& a, const S& s, uns
             }
         }
         if (!ok) break;
-        umma_commit_pair_both(&tfull[tk & 1u], 0x3);
-        ++tk;
+        for (int t = 0; t < nt; ++t) umma_commit_pair_both(&tfull[(tk + (uint32_t)t) & 1u], 0x3);
+        tk += (uint32_t)nt;
     }
     // wait for every MMA this thread issued before TMEM is released
     umma_commit_pair_local(fin);
@@ -875,10 +894,12 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-            if constexpr (C::CG2)
-                mbar_arrive_cluster(smem_in_rank(&tempty[tk & 1u], 0));
-            else
-                for (int t = 0; t < nt; ++t) mbar_arrive(&tempty[(tk + (uint32_t)t) & 1u]);
+            for (int t = 0; t < nt; ++t) {
+                if constexpr (C::CG2)
+                    mbar_arrive_cluster(smem_in_rank(&tempty[(tk + (uint32_t)t) & 1u], 0));
+                else
+                    mbar_arrive(&tempty[(tk + (uint32_t)t) & 1u]);
+            }
         }
         tk += (uint32_t)nt;
         if (S::kSignals) {

@@ -104,6 +104,9 @@ cudaError_t gemm_configure(int dev) {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm_pair<Bf16Cta2ExtCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Bf16Cta2ExtCfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm_pair<Bf16Cta2PairCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Bf16Cta2PairCfg::SMEM);
 
     if (e == cudaSuccess) done[dev] = true;
     return e;
@@ -152,7 +155,10 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     // times, one session): down on CTA pairs 5 % faster than single tiles at
     // the page shape and 1 % at the zipf shape; gate/up on CTA pairs 4 %
     // slower than M-tile pairs (page) and 5 % slower than single tiles (zipf).
-    const bool cta2 = tune.cta_pair >= 2 || (tune.cta_pair == 1 && phase != 0);
+    // 3: as 1, with the gate/up phase on CTA pairs of two M tiles each
+    if (tune.cta_pair == 3 && phase == 0 && pair && !mx && !bwd && tiles % 4 == 0 && grid >= 2)
+        return launch_pair_phase<Bf16Cta2PairCfg>(grid, maps, a, chunks, counts2, phase, tiles / 4, GC, stream);
+    const bool cta2 = tune.cta_pair == 2 || ((tune.cta_pair == 1 || tune.cta_pair == 3) && phase != 0);
     if (cta2 && !mx && tiles % 2 == 0 && grid >= 2) {
         if (phase >= 2)  // the backward's dh and dx phases
             return launch_pair_phase<Bf16Cta2ExtCfg>(grid, maps, a, chunks, counts2, phase, tiles / 2, GC, stream);

@@ -132,12 +132,14 @@ def test_grouped_gemm_cta_pairs_are_exact(name, monkeypatch):
     p = mok.plan(case.dlogits, cfg.k, cfg.R)
     rows = mok.gather(case.x_shards(), p)
     got = {}
-    for cta_pair in ("0", "1", "2"):  # none, the down phase, both phases
+    # none; the down phase; both phases; gate/up on pairs of CTAs holding two M tiles each
+    for cta_pair in ("0", "1", "2", "3"):
         monkeypatch.setenv("MOK_GEMM_CTA_PAIR", cta_pair)
         out, ws = mok.expert_ffn(rows, case.dwg, case.dwu, case.dwd, p)
         assert mok.get_status(ws) == mok.MOK_OK, mok.last_error()
         got[cta_pair] = out.cpu()
-    assert torch.equal(got["0"], got["1"]) and torch.equal(got["0"], got["2"])
+    for mode in ("1", "2", "3"):
+        assert torch.equal(got["0"], got[mode]), mode
     want, _, _ = _oracle_slots(case, p)
     assert_bf16_close(decode_slots(got["2"], p.ns, cfg.H), want, name)
 
