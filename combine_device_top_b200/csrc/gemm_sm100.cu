@@ -23,8 +23,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     gemm_cta<StagedSched, C>(maps, &mx, a, s, smem);
 }
 
-// The bf16 forward phases on CTA pairs (clusters of two): MT counts pairs of
-// M tiles.
+// The bf16 phases on CTA pairs (clusters of two): MT counts cluster units
+// (2 C::SUB M tiles each).
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     k_grouped_gemm_pair(const __grid_constant__ GemmMaps maps, const CoreArgs a, const Chunk* __restrict__ chunks,
@@ -74,7 +74,7 @@ static cudaError_t launch_pair_phase(int grid, const GemmMaps& maps, const CoreA
 // used when the mean rows per expert is at most 192.  MOK_GEMM_GROUP and
 // MOK_GEMM_PAIR (0/1) override (tuning knobs only: results do not change).
 GemmTuning gemm_tuning(int rows, int E) {
-    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 1};
+    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 3};
     if (const char* s = getenv("MOK_GEMM_GROUP")) v.group_chunks = atoi(s) < 1 ? 1 : atoi(s);
     if (const char* s = getenv("MOK_GEMM_PAIR")) v.pair = atoi(s) != 0;
     if (const char* s = getenv("MOK_GEMM_CTA_PAIR")) v.cta_pair = atoi(s) < 0 ? 0 : atoi(s);
@@ -150,12 +150,15 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     const int sub = pair ? 2 : 1;
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
-    // CTA pairs: the bf16 phases (by default all but gate/up), an even number
-    // of M tiles, an even grid.  Measured on B200 (ncu launch
-    // times, one session): down on CTA pairs 5 % faster than single tiles at
-    // the page shape and 1 % at the zipf shape; gate/up on CTA pairs 4 %
-    // slower than M-tile pairs (page) and 5 % slower than single tiles (zipf).
-    // 3: as 1, with the gate/up phase on CTA pairs of two M tiles each
+    // CTA pairs (MOK_GEMM_CTA_PAIR): 0 none; 1 every bf16 launch but gate/up;
+    // 2 all, one M tile per CTA; 3 (default) as 1, and gate/up, where the
+    // M-tile pairing rule holds, on CTA pairs of two M tiles per CTA.  Needs
+    // an even number of M tiles (a multiple of 4 for two per CTA) and an
+    // even grid.  Measured on B200 (ncu launch times, one session each): down
+    // on CTA pairs 5 % faster than single tiles at the page shape and 1 % at
+    // the zipf shape; gate/up on CTA pairs of one tile 4 % slower than M-tile
+    // pairs (page) and 5 % slower than single tiles (zipf); gate/up on CTA
+    // pairs of two tiles 3 % faster than M-tile pairs (page).
     if (tune.cta_pair == 3 && phase == 0 && pair && !mx && !bwd && tiles % 4 == 0 && grid >= 2)
         return launch_pair_phase<Bf16Cta2PairCfg>(grid, maps, a, chunks, counts2, phase, tiles / 4, GC, stream);
     const bool cta2 = tune.cta_pair == 2 || ((tune.cta_pair == 1 || tune.cta_pair == 3) && phase != 0);

@@ -94,7 +94,8 @@ struct GemmShape {
 struct GemmTuning {
     int group_chunks;  // raster group size in chunks
     int pair;          // 1: units of two M tiles sharing each token tile (bf16 path)
-    int cta_pair;      // bf16 launches on CTA pairs (tcgen05 cta_group::2): 0 none, 1 all but gate/up, 2 all
+    int cta_pair;      // bf16 launches on CTA pairs (tcgen05 cta_group::2): 0 none, 1 all but gate/up,
+                       // 2 all, 3 as 1 plus gate/up with two M tiles per CTA when pairing
 };
 // defaults for `rows` expert-major rows over E experts, overridable by
 // MOK_GEMM_GROUP / MOK_GEMM_PAIR / MOK_GEMM_CTA_PAIR
