@@ -158,7 +158,8 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     // on CTA pairs 5 % faster than single tiles at the page shape and 1 % at
     // the zipf shape; gate/up on CTA pairs of one tile 4 % slower than M-tile
     // pairs (page) and 5 % slower than single tiles (zipf); gate/up on CTA
-    // pairs of two tiles 3 % faster than M-tile pairs (page).
+    // pairs of two tiles 3 % faster than M-tile pairs (page); down on CTA
+    // pairs of two tiles slower than on CTA pairs of one (page).
     if (tune.cta_pair == 3 && phase == 0 && pair && !mx && !bwd && tiles % 4 == 0 && grid >= 2)
         return launch_pair_phase<Bf16Cta2PairCfg>(grid, maps, a, chunks, counts2, phase, tiles / 4, GC, stream);
     const bool cta2 = tune.cta_pair == 2 || ((tune.cta_pair == 1 || tune.cta_pair == 3) && phase != 0);
