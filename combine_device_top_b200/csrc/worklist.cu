@@ -32,14 +32,17 @@ __global__ void __launch_bounds__(1024) k_build_chunks(const int32_t* __restrict
                                                        int* __restrict__ counts2, DevStatus* st) {
     __shared__ int s_nmb;
     __shared__ int warp_sums[32];
+    __shared__ int s_off[1025];  // offsets[0..E] (E <= 1024): the serial walk below reads shared memory
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = offsets[i];
+    __syncthreads();
     if (threadIdx.x == 0) {
         int b0 = 0, n = 0, e = 0;
         while (b0 < n_slots) {
-            while (e < E - 1 && offsets[e + 1] <= b0) ++e;  // expert holding row b0
+            while (e < E - 1 && s_off[e + 1] <= b0) ++e;  // expert holding row b0
             const int limit = min(n_slots, b0 + cap);
             int b = b0, units = 0, ee = e;
             while (true) {
-                const int end = min(offsets[ee + 1], limit);
+                const int end = min(s_off[ee + 1], limit);
                 units += piece_chunks(end - b, maxr) * upc;
                 b = end;
                 if (b >= limit || (b >= b0 + M && units >= min_units) || ee == E - 1) break;
