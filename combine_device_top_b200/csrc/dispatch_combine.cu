@@ -5,9 +5,9 @@
 // Both kernels are HBM-bound streams of 16-byte vectors: one warp per token,
 // a grid of a few CTAs per SM looping over the tokens.  The gather reads each
 // token once and writes it to its k rows (T*H*2 bytes in, N_s*H*2 out); the
-// combine reads the per-slot outputs (N_s*H*4 bytes of fp32 on the bf16
-// path, N_s*H*2 of bf16 on the MXFP8 path) and writes T*H*2 bytes of bf16 y,
-// rounding once.
+// combine reads the per-slot outputs (N_s*H*2 bytes of fp16 plus N_s*H/128
+// exponents on the bf16 path, N_s*H*2 of bf16 on the MXFP8 path) and writes
+// T*H*2 bytes of bf16 y, rounding once.
 #include "dispatch_combine.cuh"
 #include "mok_internal.h"
 #include "mxfp8.cuh"

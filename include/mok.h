@@ -443,10 +443,13 @@ size_t mok_expert_ffn_workspace_bytes(int n_rows, int I, int E);
 
 /* Grouped SwiGLU FFN over the expert-major rows of `plan`:
  *   h[row]   = bf16(silu(rows[row] Wg[e]) * (rows[row] Wu[e]))   [N_s, I]
- *   out[row_slot[row]] = h[row] Wd[e]  (fp32 accumulation and result) [N_s, H]
+ *   out[row_slot[row]] = h[row] Wd[e]  (fp32 accumulation)       [N_s, H]
  * (e = expert of the row; all weights bf16).  h stays in the workspace;
- * `out` is fp32 (MOK_SLOTS_F32) and slot-indexed, i.e. [T, k, H].  Source:
- * MoK article, routing paragraph (grouped GEMM over contiguous per-expert
+ * `out` is slot-indexed ([T, k, H]) in the MOK_SLOTS_F16S form: a buffer of
+ * mok_slot_bytes(N_s, H, MOK_SLOTS_F16S) bytes, 256-byte aligned, whose
+ * fp32 results are stored as fp16 values with one exponent per 128
+ * features (the form mok_moe_forward's bf16 path pushes).  Source: MoK
+ * article, routing paragraph (grouped GEMM over contiguous per-expert
  * tokens) and push-combine paragraph. */
 int mok_expert_ffn(const void* rows, int H, int I,
                    const void* w_gate, const void* w_up, const void* w_down,
@@ -467,8 +470,9 @@ int mok_expert_ffn_mxfp8(const void* rows_q, const void* scales, int H, int I,
                          void* ws, size_t ws_bytes, void* out, mok_stream_t stream);
 
 /* y[t] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]), fp32, j ascending,
- * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] of out_dtype
- * (MOK_SLOTS_F32 or MOK_SLOTS_BF16), 16-byte aligned.
+ * written to y_shard[t / S_r][t % S_r].  out: [T, k, H] in the form
+ * out_dtype names (MOK_SLOTS_F32, MOK_SLOTS_BF16, or MOK_SLOTS_F16S with
+ * H % 128 == 0), 16-byte aligned.
  * Source: MoK article, benchmark paragraph (final weighted merge). */
 int mok_combine(const void* out, int out_dtype, int H, const mok_plan_t* plan,
                 void* const* y_shards, mok_stream_t stream);
