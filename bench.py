@@ -490,6 +490,63 @@ def time_backward(wl: Workload, steps: int, warmup: int):
                     "gradients (bf16 dW)"}
 
 
+def time_ep(cfg, device, steps: int, warmup: int, wl: Workload | None = None):
+    """The expert-parallel forward (EpGroup: logits all-gather, plan, pull
+    dispatch + FFN + push, combine, device barriers) with this process as one
+    rank of the torch.distributed group (or a group of one): the layer's T
+    tokens and E experts split over the ranks.  Each rank's tokens and its
+    experts' weights resident in HBM; CUDA events on the launching stream;
+    max over ranks."""
+    import combine_device_top_b200 as mok
+
+    dist = torch.distributed
+    world = dist.get_world_size() if dist.is_initialized() else 1
+    rank = dist.get_rank() if dist.is_initialized() else 0
+    grp = mok.EpGroup(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, device=device)
+    S_r = grp.S_r
+    if wl is not None and world == 1:
+        x, logits_local, w = wl.dx, wl.dlogits, wl.w
+    else:
+        x_all = mokgen.tokens(cfg)
+        logits_all = mokgen.router_logits(cfg, x_all)
+        x = x_all[rank * S_r:(rank + 1) * S_r].to(device)
+        logits_local = logits_all[rank * S_r:(rank + 1) * S_r].contiguous().to(device)
+        w = (torch.empty((grp.e_loc, cfg.H, cfg.I), dtype=torch.bfloat16, device=device),
+             torch.empty((grp.e_loc, cfg.H, cfg.I), dtype=torch.bfloat16, device=device),
+             torch.empty((grp.e_loc, cfg.I, cfg.H), dtype=torch.bfloat16, device=device))
+        for i, e in enumerate(range(grp.e0, grp.e0 + grp.e_loc)):
+            for dst, src in zip(w, mokgen.expert_weights(cfg, e)):
+                dst[i].copy_(src)
+    grp.x.copy_(x)
+    y = torch.empty((S_r, cfg.H), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        grp.forward(logits_local, *w, y=y)
+    torch.cuda.synchronize()
+    if dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        grp.forward(logits_local, *w, y=y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if grp.status() != mok.MOK_OK:
+        raise RuntimeError("EP status " + mok.last_error())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, device)
+    if dist.is_initialized():
+        dist.barrier()
+    grp.close()
+    return {"workload": f"{cfg.name}: {cfg.describe()}", "ranks": world, "ms_per_step": ms,
+            "tokens_per_s": cfg.T / (ms / 1e3), "steps": steps,
+            "note": "EpGroup.forward per step: all-gather of the logits, mok_plan, mok_ep_dispatch_ffn (barrier, "
+                    "pull dispatch of this rank's experts' rows from the ranks' x, grouped SwiGLU FFN, push of "
+                    "every slot row into its token's rank's slot buffer), mok_ep_combine (barrier, combine); "
+                    + ("one rank: the pull and the push stay in this GPU's HBM" if world == 1 else
+                       "peer pointers over NVLink")}
+
+
 # ------------------------------------------------------------------ roofline
 def tensor_peaks(peaks, mxfp8: bool, region_s: float):
     """(peak TFLOP/s of the MMA's dtype for a region this long, its kind)."""
@@ -626,6 +683,8 @@ def main():
     ap.add_argument("--no-sub-records", action="store_true", help="time only the main workload")
     ap.add_argument("--backward", action="store_true",
                     help="time only mok_moe_backward on the workload (after one staged forward that keeps a, b)")
+    ap.add_argument("--ep", action="store_true",
+                    help="time the expert-parallel forward alone, the layer split over the torchrun ranks")
     ap.add_argument("--router", action="store_true",
                     help="time only mok_plan_router (the router projection, top-k and schedule) on the workload's "
                          "tokens; no expert weights are built")
@@ -683,6 +742,13 @@ def main():
             lite = types.SimpleNamespace(cfg=cfg, device=device, x_shards=mok.shards(x, cfg.R))
             print(json.dumps(time_router(lite, args.steps, args.warmup)), flush=True)
         return 0
+    if args.ep:
+        r = time_ep(cfg, device, args.steps, args.warmup, Workload(cfg, device) if world == 1 else None)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(r), flush=True)
+        return 0
     wl = Workload(cfg, device)
     if args.backward:
         if rank == 0:
@@ -704,6 +770,7 @@ def main():
         bw = time_backward(wl, max(3, args.steps // 4), 2)
         bw["frac_of_hbm"] = bw["GBps"] / peaks["hbm_gbs"]
         subs[f"{cfg.name}_backward"] = bw
+        subs[f"{cfg.name}_expert_parallel_1rank"] = time_ep(cfg, device, args.steps, args.warmup, wl)
         wl.free()
         del wl
         zcfg = mokgen.CONFIGS["zipf"]

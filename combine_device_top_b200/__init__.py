@@ -33,6 +33,9 @@ MOK_MAX_SHARDS = 64
 MOK_SLOTS_F32 = 0
 MOK_SLOTS_BF16 = 1
 MOK_SLOTS_F16S = 2
+MOK_EP_SYNC_CALLER = 0
+MOK_EP_SYNC_DEVICE = 1
+MOK_IPC_HANDLE_BYTES = 64
 
 # every entry point of include/mok.h
 EXPORTS = (
@@ -44,6 +47,8 @@ EXPORTS = (
     "mok_two_wave_rows", "mok_minibatch_bounds", "mok_forward_host_batches_workspace_bytes",
     "mok_moe_forward_host_batches", "mok_router_weights_bytes", "mok_router_prepare", "mok_plan_router",
     "mok_backward_workspace_bytes", "mok_moe_backward", "mok_slot_bytes", "mok_slot_exp_offset",
+    "mok_ep_slot_bytes", "mok_ep_workspace_bytes", "mok_ep_dispatch_ffn", "mok_ep_combine",
+    "mok_ipc_export", "mok_ipc_import", "mok_ipc_close",
 )
 
 
@@ -65,6 +70,13 @@ class FwdOpts(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("ring_slots", ctypes.c_int32), ("dispatch_ctas", ctypes.c_int32),
                 ("gemm_ctas", ctypes.c_int32), ("mxfp8", ctypes.c_int32), ("min_waves", ctypes.c_int32),
                 ("save_for_backward", ctypes.c_int32), ("dispatch_warps", ctypes.c_int32), ("timeout_ns", ctypes.c_uint64)]
+
+
+class EpT(ctypes.Structure):
+    """``mok_ep_t``: one rank's view of an expert-parallel group."""
+    _fields_ = [("G", ctypes.c_int32), ("g", ctypes.c_int32), ("e0", ctypes.c_int32), ("e_loc", ctypes.c_int32),
+                ("sync", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("x", ctypes.c_void_p * MOK_MAX_SHARDS), ("slots", ctypes.c_void_p * MOK_MAX_SHARDS)]
 
 
 @lru_cache(maxsize=1)
@@ -119,6 +131,19 @@ def lib() -> ctypes.CDLL:
                                                ctypes.POINTER(FwdOpts), vp, sz, vp]
     L.mok_minibatch_bounds.argtypes = [ctypes.POINTER(PlanT), i32, i32, vp, i32, ctypes.POINTER(FwdOpts), vp, sz,
                                        vp, vp, i32, ctypes.POINTER(ctypes.c_int), vp]
+    u32, u64 = ctypes.c_uint32, ctypes.c_uint64
+    L.mok_ep_slot_bytes.argtypes = [i32, i32, i32]
+    L.mok_ep_slot_bytes.restype = sz
+    L.mok_ep_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    L.mok_ep_workspace_bytes.restype = sz
+    L.mok_ep_dispatch_ffn.argtypes = [ctypes.POINTER(PlanT), ctypes.POINTER(EpT), i32, i32, vp, vp, vp, u32, u64, vp,
+                                      sz, vp]
+    L.mok_ep_combine.argtypes = [ctypes.POINTER(PlanT), ctypes.POINTER(EpT), i32, u32, u64, vp, vp, sz, vp]
+    L.mok_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_size_t)]
+    L.mok_ipc_import.argtypes = [vp, ctypes.POINTER(ctypes.c_void_p)]
+    L.mok_ipc_close.argtypes = [vp]
+    for n in ("mok_ep_dispatch_ffn", "mok_ep_combine", "mok_ipc_export", "mok_ipc_import", "mok_ipc_close"):
+        getattr(L, n).restype = ctypes.c_int
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
               "mok_moe_forward_host", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
               "mok_quantize_weights_mxfp8", "mok_mxfp8_scale_rows", "mok_gather_mxfp8", "mok_expert_ffn_mxfp8",
@@ -528,3 +553,159 @@ def moe_forward_host_batches(xs_host, logits_host, top_k: int, R: int, w_gate, w
                                               ws.numel(), _stream(stream)))
     del keep
     return ys_host
+
+
+# ---------------------------------------------------------------- expert parallelism
+def ep_partition(E: int, G: int, g: int) -> tuple[int, int]:
+    """Experts of rank g when E experts are split over G ranks in contiguous
+    blocks, the first E % G ranks holding one more: (e0, e_loc)."""
+    assert 0 <= g < G and E >= 0
+    base, extra = divmod(E, G)
+    e0 = g * base + min(g, extra)
+    return e0, base + (1 if g < extra else 0)
+
+
+def ep_slot_bytes(S_r: int, H: int, k: int) -> int:
+    return lib().mok_ep_slot_bytes(S_r, H, k)
+
+
+def ep_workspace_bytes(T: int, H: int, I: int, e_loc: int, k: int) -> int:
+    return lib().mok_ep_workspace_bytes(T, H, I, e_loc, k)
+
+
+def ep_desc(G: int, g: int, e0: int, e_loc: int, x_ptrs, slot_ptrs, sync: int = MOK_EP_SYNC_DEVICE) -> EpT:
+    """A ``mok_ep_t`` from the ranks' x and slot-buffer addresses (ints, as
+    this GPU addresses them)."""
+    assert len(x_ptrs) == G and len(slot_ptrs) == G and 1 <= G <= MOK_MAX_SHARDS
+    d = EpT()
+    d.G, d.g, d.e0, d.e_loc, d.sync = G, g, e0, e_loc, sync
+    for h in range(G):
+        d.x[h] = x_ptrs[h]
+        d.slots[h] = slot_ptrs[h]
+    return d
+
+
+def ep_dispatch_ffn(p: Plan, ep: EpT, w_gate, w_up, w_down, step: int, ws: torch.Tensor, timeout_ns: int = 0,
+                    stream=None) -> None:
+    """Rank ep.g's barrier, pull dispatch, grouped SwiGLU FFN and push of step
+    ``step``; w_* are this rank's experts' weights ([e_loc, H, I] and [e_loc, I, H] bf16)."""
+    H, I = w_gate.shape[-2], w_gate.shape[-1]
+    for w in (w_gate, w_up, w_down):
+        assert w.dtype == torch.bfloat16 and w.shape[0] == ep.e_loc, "the rank's bf16 weights"
+    _check(lib().mok_ep_dispatch_ffn(ctypes.byref(p.c), ctypes.byref(ep), H, I, ctypes.c_void_p(w_gate.data_ptr()),
+                                     ctypes.c_void_p(w_up.data_ptr()), ctypes.c_void_p(w_down.data_ptr()), step,
+                                     timeout_ns, ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)))
+
+
+def ep_combine(p: Plan, ep: EpT, y: torch.Tensor, step: int, ws: torch.Tensor, timeout_ns: int = 0,
+               stream=None) -> torch.Tensor:
+    """Rank ep.g's barrier and combine of step ``step`` into y [S_r, H] bf16."""
+    assert y.dtype == torch.bfloat16 and y.is_contiguous()
+    _check(lib().mok_ep_combine(ctypes.byref(p.c), ctypes.byref(ep), y.shape[-1], step, timeout_ns,
+                                ctypes.c_void_p(y.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                _stream(stream)))
+    return y
+
+
+def ipc_export(t: torch.Tensor) -> tuple[bytes, int]:
+    """(handle bytes, byte offset) of the cudaMalloc allocation holding ``t``."""
+    h = (ctypes.c_ubyte * MOK_IPC_HANDLE_BYTES)()
+    off = ctypes.c_size_t(0)
+    _check(lib().mok_ipc_export(ctypes.c_void_p(t.data_ptr()), h, ctypes.byref(off)))
+    return bytes(h), off.value
+
+
+def ipc_import(handle: bytes) -> int:
+    """Base address (an int) of another process's allocation, mapped here."""
+    assert len(handle) == MOK_IPC_HANDLE_BYTES
+    buf = (ctypes.c_ubyte * MOK_IPC_HANDLE_BYTES).from_buffer_copy(handle)
+    base = ctypes.c_void_p(0)
+    _check(lib().mok_ipc_import(buf, ctypes.byref(base)))
+    return base.value
+
+
+def ipc_close(base: int) -> None:
+    _check(lib().mok_ipc_close(ctypes.c_void_p(base)))
+
+
+class EpGroup:
+    """The expert-parallel forward on this process's GPU, one process per GPU
+    under ``torch.distributed`` (rank g of G): rank g holds tokens [g*S_r,
+    (g+1)*S_r) of a layer of T tokens and the experts ``ep_partition(E, G, g)``.
+
+    At construction every rank allocates its token buffer ``x`` [S_r, H] and
+    its slot buffer, exports both (CUDA IPC) and maps the other ranks' (an
+    all-gather of the handles: plumbing, once).  :meth:`forward` then runs a
+    step: an all-gather of the logits (so every rank builds the same plan),
+    the plan, and the library's two calls (pull dispatch + FFN + push, then
+    combine), with the group barriers on the device.  ``ipc`` replaces the
+    (export, import, close) functions, e.g. by fakes in host-only tests.
+    """
+
+    def __init__(self, T: int, H: int, I: int, E: int, k: int, device=None, group=None, ipc=None):
+        import torch.distributed as dist
+        self.dist = dist
+        self.group = group
+        self.G = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.g = dist.get_rank(group) if dist.is_initialized() else 0
+        assert T % self.G == 0, "T must split evenly over the ranks"
+        self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
+        self.S_r = T // self.G
+        self.e0, self.e_loc = ep_partition(E, self.G, self.g)
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.export, self.import_, self.close_ = ipc or (ipc_export, ipc_import, ipc_close)
+        self.step = 0
+        self._opened: list[int] = []
+        self.x = torch.empty((self.S_r, H), dtype=torch.bfloat16, device=self.device)
+        self.slots = torch.zeros(ep_slot_bytes(self.S_r, H, k), dtype=torch.uint8, device=self.device)
+        self.ws = _workspace(ep_workspace_bytes(T, H, I, self.e_loc, k), self.device)
+        xp, sp = self._exchange()
+        self.desc = ep_desc(self.G, self.g, self.e0, self.e_loc, xp, sp, MOK_EP_SYNC_DEVICE)
+
+    def _exchange(self):
+        """Every rank's x and slot addresses as this GPU addresses them."""
+        if self.G == 1:
+            return [self.x.data_ptr()], [self.slots.data_ptr()]
+        mine = (self.export(self.x), self.export(self.slots))
+        allv = [None] * self.G
+        self.dist.all_gather_object(allv, mine, group=self.group)
+        xp, sp = [], []
+        for h, ((xh, xo), (sh, so)) in enumerate(allv):
+            if h == self.g:
+                xp.append(self.x.data_ptr())
+                sp.append(self.slots.data_ptr())
+                continue
+            bx, bs = self.import_(xh), self.import_(sh)
+            self._opened += [bx, bs]
+            xp.append(bx + xo)
+            sp.append(bs + so)
+        return xp, sp
+
+    def gather_logits(self, logits_local: torch.Tensor) -> torch.Tensor:
+        """[T, E] fp32: the ranks' [S_r, E] logits in rank order."""
+        if self.G == 1:
+            return logits_local
+        out = torch.empty((self.T, self.E), dtype=logits_local.dtype, device=logits_local.device)
+        self.dist.all_gather_into_tensor(out, logits_local.contiguous(), group=self.group)
+        return out
+
+    def forward(self, logits_local: torch.Tensor, w_gate, w_up, w_down, y: torch.Tensor | None = None,
+                timeout_ns: int = 0, stream=None) -> torch.Tensor:
+        """One step over the tokens in ``self.x``: returns y [S_r, H] bf16.
+        w_*: this rank's experts' weights."""
+        self.step += 1
+        p = plan(self.gather_logits(logits_local), self.k, self.G, stream=stream)
+        ep_dispatch_ffn(p, self.desc, w_gate, w_up, w_down, self.step, self.ws, timeout_ns, stream)
+        if y is None:
+            y = torch.empty((self.S_r, self.H), dtype=torch.bfloat16, device=self.device)
+        return ep_combine(p, self.desc, y, self.step, self.ws, timeout_ns, stream)
+
+    def status(self, stream=None) -> int:
+        return get_status(self.ws, stream)
+
+    def close(self) -> None:
+        """Unmap the other ranks' buffers (after the last step has finished)."""
+        for b in self._opened:
+            self.close_(b)
+        self._opened = []
+

@@ -296,7 +296,8 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
                           const void* wd, int E, const int32_t* row_slot, const Chunk* chunks, const int* counts2,
                           void* h, void* out, DevStatus* status, uint64_t timeout_ns, cudaStream_t stream,
                           const mok_mxfp8_weights* mxw = nullptr, const MxTokenScales* mxs = nullptr,
-                          const BwdBuffers* save = nullptr) {
+                          const BwdBuffers* save = nullptr, const PushDest* push = nullptr, int push_slots = 0,
+                          int tune_rows = -1) {
     int dev = 0;
     const int sms = device_sms(&dev);
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
@@ -314,14 +315,15 @@ static int run_expert_ffn(const void* rows, int n_rows_buf, int H, int I, const 
         return fail(MOK_ERR_CUDA, "tensor map: %s", err);
     }
     GemmShape sh{H, I, E};
-    const GemmTuning tune = gemm_tuning(n_rows_buf, E);
+    const GemmTuning tune = gemm_tuning(tune_rows >= 0 ? tune_rows : n_rows_buf, E);
     const MxMaps* mxp = mxw ? &mx : nullptr;
     MOK_CUDA(launch_gemm_phase(0, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
                                tune, stream, save),
              "gate/up GEMM launch");
-    int8_t* out_exp = mxw ? nullptr : reinterpret_cast<int8_t*>(out) + slot_exp_offset((size_t)n_rows_buf, H);
+    int8_t* out_exp =
+        mxw || push ? nullptr : reinterpret_cast<int8_t*>(out) + slot_exp_offset((size_t)n_rows_buf, H);
     MOK_CUDA(launch_gemm_phase(1, maps, mxp, mxs, sh, chunks, counts2, h, out, row_slot, status, timeout_ns, sms,
-                               tune, stream, nullptr, out_exp),
+                               tune, stream, nullptr, out_exp, push, push_slots),
              "down GEMM launch");
     return MOK_OK;
 }
@@ -1197,6 +1199,217 @@ int mok_moe_forward_host_batches(int n, const void* const* x_host, const float* 
                                  const mok_fwd_opts* opts, void* ws, size_t ws_bytes, mok_stream_t stream) {
     return forward_host_batches(n, x_host, logits_host, y_host, T, H, I, E, top_k, R, w_gate, w_up, w_down, minibatch,
                                 opts, ws, ws_bytes, 2, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ expert parallelism
+namespace mok {
+
+// Byte offset of the barrier counter in a rank's slot buffer.
+static size_t ep_counter_offset(int S_r, int H, int k) {
+    return align256(slot_bytes((size_t)S_r * k, H, MOK_SLOTS_F16S));
+}
+
+struct EpLayout {
+    size_t status, push, offsets, row_slot, counts2, chunks, mbs, rows, h, total;
+    int max_chunks, max_mb;
+};
+
+static size_t ep_layout(int T, int H, int I, int e_loc, int k, EpLayout* L) {
+    const int ns = T * k;
+    L->max_mb = max_minibatches(ns, ns > 0 ? ns : 1);
+    L->max_chunks = max_chunks(ns, e_loc > 0 ? e_loc : 1, L->max_mb);
+    size_t off = 0;
+    L->status = off;
+    off += align256(sizeof(DevStatus));
+    L->push = off;
+    off += align256(sizeof(PushDest));
+    L->offsets = off;
+    off += align256(sizeof(int32_t) * ((size_t)e_loc + 1));
+    L->row_slot = off;
+    off += align256(sizeof(int32_t) * (size_t)ns);
+    L->counts2 = off;
+    off += align256(sizeof(int) * 4);
+    L->chunks = off;
+    off += align256(sizeof(Chunk) * (size_t)L->max_chunks);
+    L->mbs = off;
+    off += align256(sizeof(Minibatch) * (size_t)L->max_mb);
+    L->rows = off;
+    off += align256((size_t)ns * H * 2);
+    L->h = off;
+    off += align256((size_t)ns * I * 2);
+    L->total = off;
+    return off;
+}
+
+static int check_ep(const mok_plan_t* plan, const mok_ep_t* ep, int H) {
+    if (!ep) return fail(MOK_ERR_INVALID_ARG, "ep is NULL");
+    if (ep->G < 1 || ep->G > MOK_MAX_SHARDS || ep->g < 0 || ep->g >= ep->G)
+        return fail(MOK_ERR_INVALID_ARG, "EP rank %d of %d out of range", ep->g, ep->G);
+    if (plan->R != ep->G) return fail(MOK_ERR_INVALID_ARG, "plan R (%d) must equal the group size (%d)", plan->R, ep->G);
+    if (ep->e0 < 0 || ep->e_loc < 0 || ep->e0 + ep->e_loc > plan->E)
+        return fail(MOK_ERR_INVALID_ARG, "experts [%d, %d) outside 0 .. %d", ep->e0, ep->e0 + ep->e_loc, plan->E);
+    if (ep->sync != MOK_EP_SYNC_CALLER && ep->sync != MOK_EP_SYNC_DEVICE)
+        return fail(MOK_ERR_INVALID_ARG, "unknown EP sync mode %d", ep->sync);
+    if (H <= 0 || H % 128) return fail(MOK_ERR_UNSUPPORTED, "H %% 128 != 0 (H = %d)", H);
+    for (int r = 0; r < ep->G; ++r) {
+        if (!ep->x[r] || !ep->slots[r]) return fail(MOK_ERR_INVALID_ARG, "NULL pointer of rank %d", r);
+        if (reinterpret_cast<uintptr_t>(ep->x[r]) & 15u)
+            return fail(MOK_ERR_UNSUPPORTED, "x of rank %d is not 16-byte aligned", r);
+        if (reinterpret_cast<uintptr_t>(ep->slots[r]) & 255u)
+            return fail(MOK_ERR_UNSUPPORTED, "slot buffer of rank %d is not 256-byte aligned", r);
+    }
+    return MOK_OK;
+}
+
+// The group barrier of step `step`, half `half` (1: before the dispatch, 2:
+// before the combine): waits for arrival number 2 * (step - 1) + half of
+// every rank.
+static int ep_barrier(const mok_plan_t* plan, const mok_ep_t* ep, int H, uint32_t step, int half,
+                      uint64_t timeout_ns, void* status, cudaStream_t stream) {
+    if (ep->sync != MOK_EP_SYNC_DEVICE) return MOK_OK;
+    const int S_r = plan->T / plan->R;
+    ShardsOut counters{};
+    for (int r = 0; r < ep->G; ++r)
+        counters.p[r] = static_cast<unsigned char*>(ep->slots[r]) + ep_counter_offset(S_r, H, plan->k);
+    const uint32_t target = (2u * (step - 1u) + (uint32_t)half) * (uint32_t)ep->G;
+    MOK_CUDA(launch_ep_barrier(counters, ep->G, ep->g, target, status, timeout_ns ? timeout_ns : kDefaultTimeoutNs,
+                               stream),
+             "EP barrier launch");
+    return MOK_OK;
+}
+
+using AddrRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+static AddrRangeFn get_addr_range() {
+    static AddrRangeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<AddrRangeFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace mok
+
+extern "C" {
+
+size_t mok_ep_slot_bytes(int S_r, int H, int k) {
+    if (S_r < 0 || H <= 0 || H % 128 || k <= 0) return 0;
+    return ep_counter_offset(S_r, H, k) + 256;
+}
+
+size_t mok_ep_workspace_bytes(int T, int H, int I, int e_loc, int k) {
+    if (T < 0 || H <= 0 || I <= 0 || e_loc < 0 || k <= 0) return 0;
+    EpLayout L;
+    return ep_layout(T, H, I, e_loc, k, &L);
+}
+
+int mok_ep_dispatch_ffn(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I, const void* w_gate,
+                        const void* w_up, const void* w_down, uint32_t step, uint64_t timeout_ns, void* ws,
+                        size_t ws_bytes, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if ((rc = check_hi(H, I))) return rc;
+    if ((rc = check_ep(plan, ep, H))) return rc;
+    if (step < 1) return fail(MOK_ERR_INVALID_ARG, "step counts from 1");
+    EpLayout L;
+    if ((rc = check_ws(ws, ws_bytes, ep_layout(plan->T, H, I, ep->e_loc, plan->k, &L)))) return rc;
+    if (ep->e_loc > 0 && (!w_gate || !w_up || !w_down)) return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    DevStatus* status = reinterpret_cast<DevStatus*>(base + L.status);
+    MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
+    if ((rc = ep_barrier(plan, ep, H, step, 1, timeout_ns, status, stream))) return rc;
+    const int ns = plan->T * plan->k;
+    if (ns == 0 || ep->e_loc == 0) return MOK_OK;  // nothing to pull or compute on this rank
+    const int S_r = plan->T / plan->R;
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    PushDest pd{};
+    ShardsIn xs{};
+    for (int r = 0; r < ep->G; ++r) {
+        pd.out[r] = ep->slots[r];
+        pd.exp[r] = static_cast<int8_t*>(ep->slots[r]) + slot_exp_offset((size_t)S_r * plan->k, H);
+        xs.p[r] = ep->x[r];
+    }
+    PushDest* push_dev = reinterpret_cast<PushDest*>(base + L.push);
+    int32_t* offsets_loc = reinterpret_cast<int32_t*>(base + L.offsets);
+    int32_t* row_slot_loc = reinterpret_cast<int32_t*>(base + L.row_slot);
+    int* counts2 = reinterpret_cast<int*>(base + L.counts2);
+    Chunk* chunks = reinterpret_cast<Chunk*>(base + L.chunks);
+    Minibatch* mbs = reinterpret_cast<Minibatch*>(base + L.mbs);
+    MOK_CUDA(launch_ep_setup(pd, push_dev, plan->offsets, ep->e0, ep->e_loc, offsets_loc, stream), "EP setup launch");
+    MOK_CUDA(launch_build_chunks(offsets_loc, ep->e_loc, ns, ns, ns, CHUNK_MAX_ROWS, 0, 1, chunks, L.max_chunks, mbs,
+                                 L.max_mb, counts2, status, stream),
+             "work list launch");
+    MOK_CUDA(launch_ep_pull(xs, H, plan->offsets, ep->e0, ep->e_loc, plan->sched_src_rank, plan->sched_src_index,
+                            plan->row_slot, base + L.rows, row_slot_loc, ns, sms, stream),
+             "pull dispatch launch");
+    // the GEMM's tuning sees the rows this rank's experts hold on average
+    const int tune_rows = (int)((int64_t)ns * ep->e_loc / plan->E);
+    return run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, ep->e_loc, row_slot_loc, chunks, counts2,
+                          base + L.h, nullptr, status, kDefaultTimeoutNs, stream, nullptr, nullptr, nullptr, push_dev,
+                          S_r * plan->k, tune_rows);
+}
+
+int mok_ep_combine(const mok_plan_t* plan, const mok_ep_t* ep, int H, uint32_t step, uint64_t timeout_ns, void* y,
+                   void* ws, size_t ws_bytes, mok_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int rc = check_plan(plan);
+    if (rc) return rc;
+    if ((rc = check_ep(plan, ep, H))) return rc;
+    if (step < 1) return fail(MOK_ERR_INVALID_ARG, "step counts from 1");
+    if ((rc = check_ws(ws, ws_bytes, sizeof(DevStatus)))) return rc;
+    if (!y) return fail(MOK_ERR_INVALID_ARG, "y is NULL");
+    if (reinterpret_cast<uintptr_t>(y) & 15u) return fail(MOK_ERR_UNSUPPORTED, "y must be 16-byte aligned");
+    DevStatus* status = static_cast<DevStatus*>(ws);
+    if ((rc = ep_barrier(plan, ep, H, step, 2, timeout_ns, status, stream))) return rc;
+    const int S_r = plan->T / plan->R;
+    if (S_r == 0) return MOK_OK;
+    const int sms = device_sms(nullptr);
+    if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
+    ShardsOut ys{};
+    ys.p[0] = y;
+    MOK_CUDA(launch_combine(ep->slots[ep->g], MOK_SLOTS_F16S, plan->gates + (size_t)ep->g * S_r * plan->k, S_r,
+                            plan->k, H, S_r, ys, sms, stream),
+             "combine launch");
+    return MOK_OK;
+}
+
+int mok_ipc_export(const void* dptr, void* handle, size_t* offset) {
+    if (!dptr || !handle || !offset) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    static_assert(sizeof(cudaIpcMemHandle_t) == MOK_IPC_HANDLE_BYTES, "IPC handle size");
+    AddrRangeFn range = get_addr_range();
+    if (!range) return fail(MOK_ERR_CUDA, "cuMemGetAddressRange unavailable");
+    CUdeviceptr b = 0;
+    size_t size = 0;
+    if (range(&b, &size, reinterpret_cast<CUdeviceptr>(dptr)) != CUDA_SUCCESS)
+        return fail(MOK_ERR_CUDA, "cuMemGetAddressRange failed (not device memory?)");
+    cudaIpcMemHandle_t h;
+    MOK_CUDA(cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(b)), "cudaIpcGetMemHandle");
+    memcpy(handle, &h, sizeof h);
+    *offset = (size_t)(reinterpret_cast<CUdeviceptr>(dptr) - b);
+    return MOK_OK;
+}
+
+int mok_ipc_import(const void* handle, void** base) {
+    if (!handle || !base) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof h);
+    MOK_CUDA(cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess), "cudaIpcOpenMemHandle");
+    return MOK_OK;
+}
+
+int mok_ipc_close(void* base) {
+    if (!base) return fail(MOK_ERR_INVALID_ARG, "NULL pointer");
+    MOK_CUDA(cudaIpcCloseMemHandle(base), "cudaIpcCloseMemHandle");
+    return MOK_OK;
 }
 
 }  // extern "C"

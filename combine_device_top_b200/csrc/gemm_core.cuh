@@ -19,12 +19,16 @@
 //     h = silu(gate) * up and stores h rows.
 //   down unit (phase 1): A = 128 columns of Wd (MN-major from [E, I, H]),
 //     B = the chunk's h rows.  The epilogue pushes each row's 128 outputs
-//     to out[row_slot[row]] (the push combine): fp32 on the bf16 path, bf16
-//     on the MXFP8 path.
+//     to out[row_slot[row]] (the push combine): fp16 with one power-of-two
+//     exponent per 128 features on the bf16 path, bf16 on the MXFP8 path.
+//     Under expert parallelism the slot's source rank owns the row: the
+//     store goes to that rank's slot buffer (a peer pointer) at the slot's
+//     index there.
 // Precision: the bf16 path runs both GEMMs as bf16 x bf16 with fp32
 // accumulation on the caller's bf16 weights; h = silu(gate) * up is rounded
-// once to bf16 (the range of fp32, no saturation) and the slot outputs stay
-// fp32, so the only roundings before y's own are h's.  The MXFP8 path runs
+// once to bf16 (the range of fp32, no saturation) and the slot outputs keep
+// 11 significant bits with fp32's exponent range, so the roundings before
+// y's own are h's and the slot rows'.  The MXFP8 path runs
 // the block-scaled tensor-core MMA (kind::mxf8f6f4): E4M3 weights and E4M3
 // token rows / h rows, each with one E8M0 scale per 32 K values, which the
 // MMA reads from TMEM; the products are exact and accumulate in fp32.  The
@@ -175,6 +179,11 @@ struct CoreArgs {
                               // backward's dx rows), bf16 (MXFP8 path)
     int8_t* out_exp;          // bf16 path: [N_s, H/128] exponents of the fp16 slot rows
     const int32_t* row_slot;  // [N_s]
+    // Expert parallelism (nullptr: every slot goes to out / out_exp): slot s
+    // belongs to rank d = s / push_slots and is stored at s - d * push_slots
+    // of push->out[d] (fp16 rows) and push->exp[d] (their exponents).
+    const PushDest* push;
+    int push_slots;
     DevStatus* st;
     uint64_t timeout_ns;
     // MXFP8 path: E8M0 scales of the token side as planes [K/128][sc_rows][4]
@@ -714,8 +723,9 @@ __device__ __forceinline__ void gemm_mma_pair(const CoreArgs& a, const S& s, uns
 // tokens at a time, through a token-major staging tile in shared memory
 // (epi[token][feature], pitch EPI_TLD), so that every global store is a
 // row-contiguous run: gate/up writes h rows (8 lanes per 64-feature row),
-// down pushes a row's 128 outputs (a warp per row: 512 bytes of fp32, or
-// 256 bytes of bf16 on the MXFP8 path) to the tokens' slots.
+// down pushes a row's 128 outputs (a warp per row: 256 bytes of fp16 and one
+// exponent byte, or 256 bytes of bf16 on the MXFP8 path) to the tokens'
+// slots.
 // Chunks cc0, cc0 + ccstep, ... of the tile are drained by this warpgroup
 // (named barrier `bar`, staging tile `epi`).
 template <class C>
@@ -830,11 +840,19 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                 const int t = it * 4 + q;
                 const int col = cc * 32 + t;
                 if (col < u.rows) {  // warp-uniform: t depends on the warp only
-                    const int slot = __ldg(a.row_slot + u.grow0 + col);
+                    int slot = __ldg(a.row_slot + u.grow0 + col);
+                    void* out = a.out;
+                    int8_t* out_exp = a.out_exp;
+                    if (a.push) {  // the slot's source rank
+                        const int d = slot / a.push_slots;
+                        slot -= d * a.push_slots;
+                        out = a.push->out[d];
+                        out_exp = a.push->exp[d];
+                    }
                     const float4 o4 = *reinterpret_cast<const float4*>(epi + t * EPI_TLD + 4 * lane);
                     const size_t at = (size_t)slot * a.H + mt * MT_D_FEATURES;
                     if constexpr (C::MX) {
-                        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + at)[lane] =
+                        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + at)[lane] =
                             make_uint2(pack_bf16x2(o4.x, o4.y), pack_bf16x2(o4.z, o4.w));
                     } else {
                         // fp16 with one exponent for the row's 128 features of this tile
@@ -843,9 +861,9 @@ __device__ __forceinline__ void epi_drain_tile(const CoreArgs& a, const Unit& u,
                         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
                         const int sx = slot_block_exponent(m);
                         const float inv = pow2f(-sx);
-                        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + at)[lane] =
+                        reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + at)[lane] =
                             make_uint2(pack_half2(o4.x * inv, o4.y * inv), pack_half2(o4.z * inv, o4.w * inv));
-                        if (lane == 0) a.out_exp[(size_t)slot * (a.H / MT_D_FEATURES) + mt] = (int8_t)sx;
+                        if (lane == 0) out_exp[(size_t)slot * (a.H / MT_D_FEATURES) + mt] = (int8_t)sx;
                     }
                 }
             }

@@ -115,8 +115,10 @@ cudaError_t gemm_configure(int dev) {
 cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx, const MxTokenScales* mxs,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
-                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd, int8_t* out_exp) {
+                              const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd, int8_t* out_exp,
+                              const PushDest* push, int push_slots) {
     if (mx && !mxs) return cudaErrorInvalidValue;
+    if (push && push_slots <= 0) return cudaErrorInvalidValue;
     if (phase >= 2 && (mx || !bwd || !bwd->save_a || !bwd->save_b || !bwd->dab)) return cudaErrorInvalidValue;
     CoreArgs a{};
     if (bwd) {
@@ -134,7 +136,10 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     a.h = h_out;
     a.out = out;
     a.out_exp = out_exp;
-    if ((phase == 1 || phase == 3) && !mx && !out_exp) return cudaErrorInvalidValue;  // fp16 slot rows need their exponents
+    if ((phase == 1 || phase == 3) && !mx && !out_exp && !push)
+        return cudaErrorInvalidValue;  // fp16 slot rows need their exponents
+    a.push = push;
+    a.push_slots = push_slots;
     a.row_slot = row_slot;
     a.st = reinterpret_cast<DevStatus*>(status);
     a.timeout_ns = timeout_ns;

@@ -88,6 +88,12 @@ cudaError_t launch_build_chunks(const int32_t* offsets, int E, int n_slots, int 
                                 int max_mb, int* counts2, void* status, cudaStream_t stream);
 
 // ---- the grouped GEMM (tcgen05)
+// Slot buffers of the ranks of an expert-parallel group, as this GPU
+// addresses them (peer pointers): fp16 slot rows and their exponents.
+struct PushDest {
+    void* out[MOK_MAX_SHARDS];
+    int8_t* exp[MOK_MAX_SHARDS];
+};
 struct GemmShape {
     int H, I, E;
 };
@@ -148,7 +154,9 @@ struct MxTokenScales {
 };
 
 // Staged grouped GEMM over every chunk: phase 0 = gate/up + SwiGLU -> h,
-// phase 1 = down -> out[row_slot] (fp32 slots; bf16 on the MXFP8 path).
+// phase 1 = down -> out[row_slot] (fp16 slot rows with exponents; bf16 on
+// the MXFP8 path), or, with `push` (a device array), to the slot's rank:
+// push->out[d] / push->exp[d] at slot - d * push_slots, d = slot / push_slots.
 struct MxMaps;
 // mx: MXFP8 weight maps (MXFP8 path: rows and h are E4M3 with the scale
 // planes of mxs), or nullptr (bf16 path).
@@ -165,7 +173,21 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
                               const GemmShape& sh, const Chunk* chunks, const int* counts2, void* h_out, void* out,
                               const int32_t* row_slot, void* status, uint64_t timeout_ns, int grid,
                               const GemmTuning& tune, cudaStream_t stream, const BwdBuffers* bwd = nullptr,
-                              int8_t* out_exp = nullptr);
+                              int8_t* out_exp = nullptr, const PushDest* push = nullptr, int push_slots = 0);
+
+// ---- expert parallelism (ep.cu)
+// offsets_loc[i] = offsets[e0 + i] - offsets[e0] (i <= e_loc); *push_dev = push
+cudaError_t launch_ep_setup(const PushDest& push, PushDest* push_dev, const int32_t* offsets, int e0, int e_loc,
+                            int32_t* offsets_loc, cudaStream_t stream);
+// rows[i] = x[src_rank[row]][src_index[row]], row_slot_loc[i] = row_slot[row]
+// for row = offsets[e0] + i < offsets[e0 + e_loc]; max_rows bounds the count
+cudaError_t launch_ep_pull(const ShardsIn& xs, int H, const int32_t* offsets, int e0, int e_loc,
+                           const int32_t* src_rank, const int32_t* src_index, const int32_t* row_slot, void* rows,
+                           int32_t* row_slot_loc, int max_rows, int num_sms, cudaStream_t stream);
+// one arrival on every rank's counter, then a bounded wait for this rank's
+// counter (counters.p[g]) to reach target
+cudaError_t launch_ep_barrier(const ShardsOut& counters, int G, int g, uint32_t target, void* status,
+                              uint64_t timeout_ns, cudaStream_t stream);
 
 // ---- the persistent SM-partitioned forward (persistent.cu)
 struct PersistLaunch {

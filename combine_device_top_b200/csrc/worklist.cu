@@ -36,10 +36,13 @@ __global__ void __launch_bounds__(1024) k_build_chunks(const int32_t* __restrict
     for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = offsets[i];
     __syncthreads();
     if (threadIdx.x == 0) {
+        // the rows end at offsets[E]; n_slots bounds it (under expert
+        // parallelism a rank's share of the rows is known on the device only)
+        const int n_end = min(n_slots, s_off[E]);
         int b0 = 0, n = 0, e = 0;
-        while (b0 < n_slots) {
+        while (b0 < n_end) {
             while (e < E - 1 && s_off[e + 1] <= b0) ++e;  // expert holding row b0
-            const int limit = min(n_slots, b0 + cap);
+            const int limit = min(n_end, b0 + cap);
             int b = b0, units = 0, ee = e;
             while (true) {
                 const int end = min(s_off[ee + 1], limit);

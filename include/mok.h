@@ -526,6 +526,113 @@ int mok_moe_forward_host_batches(int n, const void* const* x_host, const float* 
                                  int minibatch, const mok_fwd_opts* opts,
                                  void* ws, size_t ws_bytes, mok_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Expert parallelism over G GPUs, one process per GPU.
+ * Source: MoK article, pull-dispatch paragraph (the rank that owns an expert
+ * pulls that expert's tokens from the source ranks' memory by
+ * {src_rank, src_index}) and push-combine paragraph (each expert output goes
+ * back to its token's rank, which merges its k results); MoK wiki summary,
+ * key points (NVLink loads and stores from inside the kernels, no
+ * collective library on the data path).
+ *
+ * Rank g holds tokens [g*S_r, (g+1)*S_r) of the layer (S_r = T / G) in its
+ * x buffer and the experts [e0, e0 + e_loc) (the weights of those experts
+ * only).  Every rank builds the same plan with mok_plan over the
+ * all-gathered logits [T, E] with R = G, so the plan's source shard of a
+ * token is its rank.  A step s = 1, 2, ... on every rank:
+ *   mok_ep_dispatch_ffn(step s)  group barrier (every rank's x is ready and
+ *                                every rank has finished reading its slot
+ *                                buffer in step s-1), pull dispatch of this
+ *                                rank's rows from the ranks' x over NVLink,
+ *                                the grouped SwiGLU FFN, and the push of
+ *                                every slot row into its token's rank's slot
+ *                                buffer from the down GEMM's epilogue;
+ *   mok_ep_combine(step s)       group barrier (every push of step s has
+ *                                landed), then the fixed-order weighted
+ *                                combine of this rank's tokens.
+ * The results equal mok_moe_forward's staged bf16 path over the same plan,
+ * bit for bit.
+ * ---------------------------------------------------------------------- */
+
+/* How the ranks of a group are ordered between the two calls of a step:
+ *   MOK_EP_SYNC_DEVICE  each call starts with a device-side barrier over the
+ *                       counters in the ranks' slot buffers (the multi-GPU
+ *                       mode: one process per GPU, every wait bounded);
+ *   MOK_EP_SYNC_CALLER  no barrier: the caller orders the ranks' calls (one
+ *                       process driving every rank's buffers, e.g. all on
+ *                       one GPU; all ranks' mok_ep_dispatch_ffn, then all
+ *                       ranks' mok_ep_combine). */
+enum { MOK_EP_SYNC_CALLER = 0, MOK_EP_SYNC_DEVICE = 1 };
+
+typedef struct mok_ep_t {
+    int32_t G;     /* ranks in the group, 1 .. MOK_MAX_SHARDS (the plan's R)  */
+    int32_t g;     /* this rank, 0 .. G-1                                     */
+    int32_t e0;    /* this rank's experts: e0 .. e0 + e_loc - 1 of the plan's */
+    int32_t e_loc; /* E (e_loc may be 0)                                      */
+    int32_t sync;  /* MOK_EP_SYNC_DEVICE or MOK_EP_SYNC_CALLER                */
+    int32_t reserved;
+    /* x[h]: rank h's tokens [S_r, H] bf16, as THIS GPU addresses them (a
+     * peer pointer from mok_ipc_import, or a local pointer), 16-byte
+     * aligned; h < G. */
+    const void* x[MOK_MAX_SHARDS];
+    /* slots[h]: rank h's slot buffer of mok_ep_slot_bytes(S_r, H, k) bytes,
+     * as THIS GPU addresses it, 256-byte aligned; zero-filled once before
+     * the group's first step (it holds the barrier counter). */
+    void* slots[MOK_MAX_SHARDS];
+} mok_ep_t;
+
+/* Bytes of one rank's slot buffer: [S_r*k, H] fp16 slot rows with their
+ * block exponents (the MOK_SLOTS_F16S form of mok_slot_bytes), then the
+ * 256-byte barrier counter region.  H % 128 == 0; 0 if the shape is invalid. */
+size_t mok_ep_slot_bytes(int S_r, int H, int k);
+
+/* Bytes of the per-rank workspace for (T, H, I, e_loc, k): status word, the
+ * local expert offsets, the work list, and room for every slot's row and h
+ * row (a rank may receive all T*k rows). */
+size_t mok_ep_workspace_bytes(int T, int H, int I, int e_loc, int k);
+
+/*
+ * mok_ep_dispatch_ffn -- the first half of an expert-parallel step on rank
+ * ep->g: barrier (MOK_EP_SYNC_DEVICE), pull dispatch, grouped SwiGLU FFN and
+ * push.
+ *   plan      the group's plan (R == ep->G), identical on every rank
+ *   w_gate    [e_loc, H, I] bf16, w_up [e_loc, H, I], w_down [e_loc, I, H]:
+ *             the weights of experts e0 .. e0 + e_loc - 1 on this GPU
+ *   step      1, 2, 3, ... (the same on every rank; the barrier waits for
+ *             every rank's arrival number 2*step - 1)
+ *   timeout_ns  bound of the barrier's wait (0: 2 s); a wait that gives up
+ *             writes MOK_ERR_TIMEOUT to the workspace's status word
+ *   ws        this rank's workspace (>= mok_ep_workspace_bytes(T, H, I,
+ *             e_loc, k)); its status word is cleared at the start
+ * H % 128 == 0, I % 64 == 0.  Asynchronous on `stream`.
+ */
+int mok_ep_dispatch_ffn(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I,
+                        const void* w_gate, const void* w_up, const void* w_down,
+                        uint32_t step, uint64_t timeout_ns, void* ws, size_t ws_bytes,
+                        mok_stream_t stream);
+
+/*
+ * mok_ep_combine -- the second half of step `step` on rank ep->g: barrier
+ * (MOK_EP_SYNC_DEVICE; arrival number 2*step), then
+ *   y[i] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]),  t = g*S_r + i,
+ * over the slot rows in this rank's slot buffer (ep->slots[ep->g]), fp32,
+ * j ascending.  y: [S_r, H] bf16, 16-byte aligned.  ws: the workspace given
+ * to mok_ep_dispatch_ffn (its status word).  Asynchronous on `stream`.
+ */
+int mok_ep_combine(const mok_plan_t* plan, const mok_ep_t* ep, int H, uint32_t step,
+                   uint64_t timeout_ns, void* y, void* ws, size_t ws_bytes, mok_stream_t stream);
+
+/* CUDA IPC for the peer pointers of mok_ep_t.  mok_ipc_export writes the
+ * MOK_IPC_HANDLE_BYTES-byte handle of the cudaMalloc allocation holding
+ * `dptr` and dptr's byte offset in it; another process opens it with
+ * mok_ipc_import (peer access enabled on demand; the allocation is then
+ * addressed as *base + offset) and releases it with mok_ipc_close(base).
+ * Memory from cudaMalloc (PyTorch's default allocator) only. */
+#define MOK_IPC_HANDLE_BYTES 64
+int mok_ipc_export(const void* dptr, void* handle, size_t* offset);
+int mok_ipc_import(const void* handle, void** base);
+int mok_ipc_close(void* base);
+
 #ifdef __cplusplus
 }
 #endif
