@@ -83,6 +83,7 @@ constexpr int MT_D_FEATURES = 128;                // down unit: 128 output colum
 // single-thread TMA and MMA issue loops).
 template <int SUB_, int NST_, bool EXT_ = false>
 struct Bf16CfgT {
+    static constexpr bool SPLIT = false;  // one ring of [weights | tokens] stages
     static constexpr bool MX = false;
     static constexpr bool EXT = EXT_;
     static constexpr bool CG2 = false;
@@ -111,6 +112,7 @@ static_assert(Bf16Cfg::BAR_OFF == Bf16PairCfg::BAR_OFF, "both bf16 layouts share
 // half of the token tile: [A0 16 KB][A1 16 KB][B half] x 4.
 template <int NST_, bool EXT_ = false, int SUB_ = 1>
 struct Bf16Cta2CfgT {
+    static constexpr bool SPLIT = false;  // one ring of [weights | tokens] stages
     static constexpr bool MX = false;
     static constexpr bool EXT = EXT_;  // also the backward's dh and dx phases (2, 3)
     static constexpr bool CG2 = true;
@@ -134,6 +136,7 @@ using Bf16Cta2PairCfg = Bf16Cta2CfgT<4, false, 2>;
 // SUB x 512 B][B scales, MMA layout 1 KB] x NST.
 template <int SUB_, int NST_>
 struct MxCfgT {
+    static constexpr bool SPLIT = false;  // one ring of [weights | tokens] stages
     static constexpr bool MX = true;
     static constexpr bool EXT = false;
     static constexpr bool CG2 = false;
@@ -157,7 +160,42 @@ struct MxCfgT {
     static_assert(SMEM <= 232448, "MXFP8 layout exceeds shared memory");
     static_assert(TM_SFB + 8 <= 512, "scale factors must fit in TMEM");
 };
-using MxCfg = MxCfgT<1, 4>;
+using MxOneRingCfg = MxCfgT<1, 4>;
+// MXFP8 path with two stage rings: a deep ring of weight tiles (E4M3 16 KB
+// and their scales) streamed from HBM and a shallower ring of token tiles
+// (<= 224 rows and their scales) mostly served by L2.  One ring of [weights
+// | tokens] stages holds 4 stages, i.e. 64 KB of weights in flight per SM,
+// which at HBM latency under load keeps the stream well below the HBM
+// rate; NW = 6 weight slots keep 96 KB in flight with NT = 3 token slots.
+// K step i of the CTA's unit sequence uses weight slot i % NW and token slot
+// i % NT.  Warps: 0 loads the weight tiles, 11 the token tiles, 10 lays both
+// scale sets out for the TMEM copy, 1 issues the MMAs, 2-9 drain.
+template <int NW_, int NT_>
+struct MxSplitCfgT {
+    static constexpr bool SPLIT = true;
+    static constexpr bool MX = true;
+    static constexpr bool EXT = false;
+    static constexpr bool CG2 = false;
+    static constexpr int SUB = 1;
+    static constexpr int THREADS = 384;  // warps: 0 weight TMA, 1 MMA, 2-9 epilogue, 10 scale layout, 11 token TMA
+    static constexpr int NW = NW_, NT = NT_;
+    static constexpr int NST = NT_;
+    static constexpr int BKX = 128;  // K per stage
+    // weight slot: [A E4M3 16 KB][A scales as loaded 512 B][A scales, MMA layout 512 B]
+    static constexpr int A_OFF = 0, SFA_RAW_OFF = 16384, SFA_OFF = 16384 + 512, WSTAGE = 17408;
+    // token slot: [B E4M3 <= 224 rows x 128 B][B scales as loaded 1 KB][B scales, MMA layout 1 KB]
+    static constexpr int B_OFF = 0, SFB_RAW_OFF = CHUNK_MAX_ROWS_MX * 128, SFB_OFF = SFB_RAW_OFF + 1024;
+    static constexpr int TSTAGE = SFB_OFF + 1024;
+    static constexpr int T_BASE = NW * WSTAGE;
+    static constexpr int EPI_OFF = T_BASE + NT * TSTAGE;  // one staging tile per epilogue group
+    static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static constexpr uint32_t TM_SFA = 480, TM_SFB = 484;
+    static_assert(WSTAGE % 1024 == 0 && TSTAGE % 1024 == 0, "MXFP8 slots must keep 1024-byte alignment");
+    static_assert(SMEM <= 232448, "MXFP8 two-ring layout exceeds shared memory");
+};
+using MxSplitCfg = MxSplitCfgT<6, 3>;
+using MxCfg = MxSplitCfg;
 
 // One unit of work: C::SUB consecutive M tiles (fewer at the end of the M
 // range) of one phase over one chunk; the tiles share every token tile.
@@ -539,6 +577,164 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
     }
 }
 
+// ------------------------------------------------------------------ MXFP8, two rings
+// Weight tiles of every K step of every unit into the weight ring (warp 0).
+// Weights are read-only, so this producer does not wait for a unit's inputs
+// (in the persistent kernel it runs ahead of the dispatch, bounded by the
+// ring).
+template <class S, class C>
+__device__ __forceinline__ void mx_producer_w(const MxMaps* mx, const CoreArgs& a, const S& s, unsigned char* smem,
+                                              uint64_t* wfull, uint64_t* wempty) {
+    int slot = 0;
+    uint32_t ph = 0;
+    uint32_t issued = 0, issued_ph = 0;
+    const uint64_t evict_first = l2_policy_evict_first();
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        if (failed(a.st)) break;
+        const int K = phase_k<C>(a, u.phase);
+        const int KB = (K + C::BKX - 1) / C::BKX;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&wempty[slot], ph ^ 1u, a.st, a.timeout_ns, 14)) {
+                ok = false;
+                break;
+            }
+            unsigned char* w = smem + slot * C::WSTAGE;
+            mbar_arrive_expect_tx(&wfull[slot], 16384u + 512u);
+            const int ky = u.expert * K + kb * C::BKX;
+            const int kys = ky / 32;  // scale row of the stage's first K block
+            if (u.phase == 0) {
+                // gate and up columns of the M tile: two 64-byte-swizzled 64-column boxes
+                tma_load_2d_hint(w + C::A_OFF, &mx->gq, &wfull[slot], u.m * MT_G_FEATURES, ky, evict_first);
+                tma_load_2d_hint(w + C::A_OFF + 8192, &mx->uq, &wfull[slot], u.m * MT_G_FEATURES, ky, evict_first);
+                tma_load_2d(w + C::SFA_RAW_OFF, &mx->gs, &wfull[slot], u.m * MT_G_FEATURES, kys);
+                tma_load_2d(w + C::SFA_RAW_OFF + 256, &mx->us, &wfull[slot], u.m * MT_G_FEATURES, kys);
+            } else {
+                tma_load_2d_hint(w + C::A_OFF, &mx->dq, &wfull[slot], u.m * MT_D_FEATURES, ky, evict_first);
+                tma_load_2d(w + C::SFA_RAW_OFF, &mx->ds, &wfull[slot], u.m * MT_D_FEATURES, kys);
+            }
+            issued |= 1u << slot;
+            issued_ph = (issued_ph & ~(1u << slot)) | (ph << slot);
+            if (++slot == C::NW) {
+                slot = 0;
+                ph ^= 1u;
+            }
+        }
+        if (!ok) break;
+    }
+    // never leave with a load in flight into this CTA's shared memory
+    for (int st = 0; st < C::NW; ++st)
+        if ((issued >> st) & 1u) mbar_wait(&wfull[st], (issued_ph >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 15);
+}
+
+// Token tiles (E4M3 rows, one box of the 16-rounded row count) and their
+// scales of every K step into the token ring (warp 11), after the unit's
+// inputs are ready.
+template <class S, class C>
+__device__ __forceinline__ void mx_producer_t(const GemmMaps& maps, const CoreArgs& a, const S& s,
+                                              unsigned char* smem, uint64_t* tkfull, uint64_t* tkempty) {
+    int slot = 0;
+    uint32_t ph = 0;
+    uint32_t issued = 0, issued_ph = 0;
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        if (!s.wait_inputs(u, a.st, a.timeout_ns)) break;
+        const int K = phase_k<C>(a, u.phase);
+        const int KB = (K + C::BKX - 1) / C::BKX;
+        const BMaps& bm = u.phase == 0 ? maps.rows : maps.h;
+        const int bx = token_box(u.rows);
+        // the stage's token scales: one 16-byte aligned run of the plane,
+        // starting up to 3 rows before the chunk
+        const int sc_lead = u.brow0 & 3;
+        const uint32_t sc_bytes = (uint32_t)(4 * (sc_lead + u.rows) + 15) & ~15u;
+        const uint32_t bytes = (uint32_t)(16 * (bx + 1)) * B_ROW_BYTES + sc_bytes;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&tkempty[slot], ph ^ 1u, a.st, a.timeout_ns, 16)) {
+                ok = false;
+                break;
+            }
+            unsigned char* t = smem + C::T_BASE + slot * C::TSTAGE;
+            mbar_arrive_expect_tx(&tkfull[slot], bytes);
+            const uint8_t* plane = (u.phase == 0 ? a.xsc : a.hsc) + (size_t)kb * a.sc_rows * 4;
+            bulk_load(t + C::SFB_RAW_OFF, plane + (size_t)(u.brow0 - sc_lead) * 4, sc_bytes, &tkfull[slot]);
+            tma_load_2d(t + C::B_OFF, &bm.m[bx], &tkfull[slot], kb * C::BKX, u.brow0);
+            issued |= 1u << slot;
+            issued_ph = (issued_ph & ~(1u << slot)) | (ph << slot);
+            if (++slot == C::NT) {
+                slot = 0;
+                ph ^= 1u;
+            }
+        }
+        if (!ok) break;
+    }
+    for (int st = 0; st < C::NT; ++st)
+        if ((issued >> st) & 1u) mbar_wait(&tkfull[st], (issued_ph >> st) & 1u, nullptr, DRAIN_TIMEOUT_NS, 17);
+}
+
+// Scale layout of the two-ring path (warp 10): as gemm_sf_layout, with the
+// weight scales in the weight slot and the token scales in the token slot;
+// arrives on sfready[token slot] once both slots' loads have landed.
+template <class S, class C>
+__device__ __forceinline__ void mx_sf_layout_split(const CoreArgs& a, const S& s, unsigned char* smem,
+                                                   uint64_t* wfull, uint64_t* tkfull, uint64_t* sfready) {
+    const int lane = threadIdx.x & 31;
+    int ws = 0, ts = 0;
+    uint32_t wph = 0, tph = 0;
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        const int K = phase_k<C>(a, u.phase);
+        const int KB = (K + C::BKX - 1) / C::BKX;
+        const int lead = u.brow0 & 3;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&wfull[ws], wph, a.st, a.timeout_ns, 81) ||
+                !mbar_wait(&tkfull[ts], tph, a.st, a.timeout_ns, 82)) {
+                ok = false;
+                break;
+            }
+            unsigned char* w = smem + ws * C::WSTAGE;
+            unsigned char* t = smem + C::T_BASE + ts * C::TSTAGE;
+            const uint8_t* ra = w + C::SFA_RAW_OFF;
+            uint32_t wa[4];
+#pragma unroll
+            for (int r1 = 0; r1 < 4; ++r1) {
+                const int r = lane + 32 * r1;
+                // feature r of the tile: gate/up keeps 64 gate then 64 up rows of 64 bytes
+                const uint8_t* col = u.phase == 0 ? ra + (r >> 6) * 256 + (r & 63) : ra + r;
+                const int pitch = u.phase == 0 ? 64 : 128;
+                wa[r1] = (uint32_t)col[0] | ((uint32_t)col[pitch] << 8) | ((uint32_t)col[2 * pitch] << 16) |
+                         ((uint32_t)col[3 * pitch] << 24);
+            }
+            *reinterpret_cast<uint4*>(w + C::SFA_OFF + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            const uint32_t* rb = reinterpret_cast<const uint32_t*>(t + C::SFB_RAW_OFF) + lead;
+#pragma unroll
+            for (int r2 = 0; r2 < 2; ++r2) {
+                uint32_t wb[4];
+#pragma unroll
+                for (int r1 = 0; r1 < 4; ++r1) {
+                    const int r = lane + 32 * r1 + 128 * r2;
+                    wb[r1] = r < u.rows ? rb[r] : 0u;
+                }
+                *reinterpret_cast<uint4*>(t + C::SFB_OFF + 512 * r2 + 16 * lane) =
+                    make_uint4(wb[0], wb[1], wb[2], wb[3]);
+            }
+            fence_proxy_async_shared();  // generic writes -> the TMEM copy (async proxy) reads
+            mbar_arrive(&sfready[ts]);
+            if (++ws == C::NW) {
+                ws = 0;
+                wph ^= 1u;
+            }
+            if (++ts == C::NT) {
+                ts = 0;
+                tph ^= 1u;
+            }
+        }
+        if (!ok) break;
+    }
+}
+
 // ------------------------------------------------------------------ TMEM placement
 // TMEM holds two 256-column accumulator buffers used in ring order; each use
 // is a "ticket" (buffer = ticket & 1, barrier parity = (ticket >> 1) & 1).
@@ -648,6 +844,71 @@ __device__ __forceinline__ void gemm_mma(const CoreArgs& a, const S& s, unsigned
     // wait for every MMA this thread issued before TMEM is released
     umma_commit(fin);
     mbar_wait(fin, 0, nullptr, DRAIN_TIMEOUT_NS, 22);
+}
+
+// ------------------------------------------------------------------ MMA issuer, MXFP8 two rings
+// As gemm_mma's MXFP8 branch: per K step the scales of the weight slot and
+// the token slot into TMEM, then 4 block-scaled MMAs (K = 32 each); the
+// step's commits free both slots.
+template <class S, class C>
+__device__ __forceinline__ void gemm_mma_mx_split(const CoreArgs& a, const S& s, unsigned char* smem,
+                                                  uint64_t* sfready, uint64_t* wempty, uint64_t* tkempty,
+                                                  uint64_t* tfull, uint64_t* tempty, uint64_t* fin,
+                                                  uint32_t tmem_base) {
+    int ws = 0, ts = 0;
+    uint32_t tph = 0;
+    uint32_t tk = 0;  // next accumulator ticket
+    Unit u;
+    for (int i = 0; s.get(i, u); ++i) {
+        const int K = phase_k<C>(a, u.phase);
+        const int KB = (K + C::BKX - 1) / C::BKX;
+        const int N = (u.rows + 15) & ~15;
+        bool ok = mbar_wait(&tempty[tk & 1u], ((tk >> 1) & 1u) ^ 1u, a.st, a.timeout_ns, 26);
+        if (!ok) break;
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&sfready[ts], tph, a.st, a.timeout_ns, 27)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            unsigned char* w = smem + ws * C::WSTAGE;
+            unsigned char* t = smem + C::T_BASE + ts * C::TSTAGE;
+            const uint32_t sa = smem_u32(w + C::A_OFF);
+            const uint32_t sb = smem_u32(t + C::B_OFF);
+            // scale factors of this stage into TMEM (executed in order with the MMAs)
+            tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFA, w + C::SFA_OFF);
+            tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFB, t + C::SFB_OFF);
+            if (N > 128) tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFB + 4, t + C::SFB_OFF + 512);
+            const int nks = min(4, (K - kb * C::BKX) / 32);  // 32 K values per MMA
+            for (int ks = 0; ks < nks; ++ks) {
+                // B: K-major E4M3 SW128, 32 K = 32 bytes inside the atom
+                const uint64_t bd = umma_desc_sw128(sb + ks * 32, 16, 1024);
+                const uint32_t sel = (uint32_t)ks << 30;  // scale byte of these 32 K values
+                const uint32_t idx = umma_idesc_mxf8(128, N, 1, 0, (uint32_t)ks);
+                // A: MN-major E4M3; gate/up = two 64-byte-swizzled 64-column halves 8 KB apart
+                // (8-row K groups 512 bytes apart), down = one 128-byte-swizzled 128-column tile
+                // (K groups 1 KB apart); 32 K rows per MMA.
+                const uint64_t ad = u.phase == 0 ? umma_desc(sa + ks * 2048, 8192, 512, UMMA_LAYOUT_SW64)
+                                                 : umma_desc(sa + ks * 4096, 0, 1024, UMMA_LAYOUT_SW128);
+                umma_mxf8(tmem_base + acc_col(tk, 0, false), ad, bd, idx, tmem_base + C::TM_SFA + sel,
+                          tmem_base + C::TM_SFB + sel, (kb | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit(&wempty[ws]);
+            umma_commit(&tkempty[ts]);
+            if (++ws == C::NW) ws = 0;
+            if (++ts == C::NT) {
+                ts = 0;
+                tph ^= 1u;
+            }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[tk & 1u]);
+        ++tk;
+    }
+    // wait for every MMA this thread issued before TMEM is released
+    umma_commit(fin);
+    mbar_wait(fin, 0, nullptr, DRAIN_TIMEOUT_NS, 28);
 }
 
 // ------------------------------------------------------------------ MMA issuer, CTA pairs
@@ -953,28 +1214,56 @@ __device__ __forceinline__ void gemm_epilogue(const CoreArgs& a, const S& s, uns
 // call it; any further warps of the block take part in its first barrier
 // (a __syncthreads of their own) and in nothing else.  It returns after TMEM
 // is released.  mx: MXFP8 maps (C::MX only).
+// Depth of the ring that `full` / `empty` index: the weight ring of the
+// two-ring MXFP8 layout, else the one ring.
+template <class C>
+constexpr int ring_w() {
+    if constexpr (C::SPLIT)
+        return C::NW;
+    else
+        return C::NST;
+}
+
 template <class S, class C>
 __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx, const CoreArgs& a, const S& s,
                                          unsigned char* smem) {
+    // one ring: full, empty, sfready [NST] each; two rings (MXFP8): the
+    // weight ring's full and empty [NW], the token ring's tkfull and tkempty
+    // [NT = NST], and sfready [NT]
+    constexpr int NWR = ring_w<C>();
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-    uint64_t* empty = full + C::NST;
-    uint64_t* sfready = empty + C::NST;  // MXFP8 only: stage scales in the MMA layout
+    uint64_t* empty = full + NWR;
+    uint64_t* tkfull = empty + NWR;
+    uint64_t* tkempty = tkfull + (C::SPLIT ? C::NST : 0);
+    uint64_t* sfready = C::SPLIT ? tkempty + C::NST : empty + C::NST;  // MXFP8: stage scales in the MMA layout
     uint64_t* tfull = sfready + C::NST;
     uint64_t* tempty = tfull + 2;
     uint64_t* fin = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     volatile int* ok_flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // one per epilogue group
     int* done_cnt = const_cast<int*>(ok_flags) + 2;                            // two, by unit parity
-    static_assert((3 * C::NST + 5) * 8 + 4 * 5 <= 256, "barrier region");
+    static_assert(((C::SPLIT ? 2 * NWR + 3 * C::NST : 3 * C::NST) + 5) * 8 + 4 * 5 <= 256, "barrier region");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         done_cnt[0] = 0;
         done_cnt[1] = 0;
-        for (int st = 0; st < C::NST; ++st) {
-            mbar_init(&full[st], 1);
-            mbar_init(&empty[st], 1);
-            mbar_init(&sfready[st], 32);
+        if constexpr (C::SPLIT) {
+            for (int st = 0; st < NWR; ++st) {
+                mbar_init(&full[st], 1);
+                mbar_init(&empty[st], 1);
+            }
+            for (int st = 0; st < C::NST; ++st) {
+                mbar_init(&tkfull[st], 1);
+                mbar_init(&tkempty[st], 1);
+                mbar_init(&sfready[st], 32);
+            }
+        } else {
+            for (int st = 0; st < C::NST; ++st) {
+                mbar_init(&full[st], 1);
+                mbar_init(&empty[st], 1);
+                mbar_init(&sfready[st], 32);
+            }
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
@@ -1023,17 +1312,27 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
         if (lane == 0) {
             if constexpr (C::CG2)
                 gemm_producer_pair<S, C>(maps, a, s, smem, full, empty, rank);
+            else if constexpr (C::SPLIT)
+                mx_producer_w<S, C>(mx, a, s, smem, full, empty);
             else
                 gemm_producer<S, C>(maps, mx, a, s, smem, full, empty);
         }
     } else if (warp == 1) {
         if constexpr (C::CG2) {
             if (lane == 0 && rank == 0) gemm_mma_pair<S, C>(a, s, smem, full, empty, tfull, tempty, fin, tmem_base);
+        } else if constexpr (C::SPLIT) {
+            if (lane == 0)
+                gemm_mma_mx_split<S, C>(a, s, smem, sfready, empty, tkempty, tfull, tempty, fin, tmem_base);
         } else {
             if (lane == 0) gemm_mma<S, C>(a, s, smem, C::MX ? sfready : full, empty, tfull, tempty, fin, tmem_base);
         }
     } else if (warp < 10) {
         gemm_epilogue<S, C>(a, s, smem, tfull, tempty, ok_flags, done_cnt, tmem_base);
+    } else if constexpr (C::SPLIT) {
+        if (warp == 10)
+            mx_sf_layout_split<S, C>(a, s, smem, full, tkfull, sfready);
+        else if (lane == 0)
+            mx_producer_t<S, C>(maps, a, s, smem, tkfull, tkempty);
     } else if constexpr (C::MX) {
         gemm_sf_layout<S, C>(a, s, smem, full, sfready);
     }

@@ -74,10 +74,11 @@ static cudaError_t launch_pair_phase(int grid, const GemmMaps& maps, const CoreA
 // used when the mean rows per expert is at most 192.  MOK_GEMM_GROUP and
 // MOK_GEMM_PAIR (0/1) override (tuning knobs only: results do not change).
 GemmTuning gemm_tuning(int rows, int E) {
-    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 3};
+    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 3, 2};
     if (const char* s = getenv("MOK_GEMM_GROUP")) v.group_chunks = atoi(s) < 1 ? 1 : atoi(s);
     if (const char* s = getenv("MOK_GEMM_PAIR")) v.pair = atoi(s) != 0;
     if (const char* s = getenv("MOK_GEMM_CTA_PAIR")) v.cta_pair = atoi(s) < 0 ? 0 : atoi(s);
+    if (const char* s = getenv("MOK_MX_RINGS")) v.mx_rings = atoi(s) == 1 ? 1 : 2;
     return v;
 }
 
@@ -92,6 +93,9 @@ cudaError_t gemm_configure(int dev) {
                                  Bf16PairCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm<MxCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize, MxCfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_grouped_gemm<MxOneRingCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 MxOneRingCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_grouped_gemm<Bf16ExtCfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Bf16ExtCfg::SMEM);
@@ -175,8 +179,12 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
             return launch_pair_phase<Bf16Cta2Cfg>(grid, maps, a, chunks, counts2, phase, tiles / 2, GC, stream);
     }
     if (mx) {
-        k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,
-                                                                            MT, GC);
+        if (tune.mx_rings == 1)
+            k_grouped_gemm<MxOneRingCfg><<<grid, MxOneRingCfg::THREADS, MxOneRingCfg::SMEM, stream>>>(
+                maps, *mx, a, chunks, counts2, phase, MT, GC);
+        else
+            k_grouped_gemm<MxCfg><<<grid, MxCfg::THREADS, MxCfg::SMEM, stream>>>(maps, *mx, a, chunks, counts2, phase,
+                                                                                MT, GC);
     } else {
         MxMaps none;
         memset(&none, 0, sizeof none);

@@ -102,9 +102,10 @@ struct GemmTuning {
     int pair;          // 1: units of two M tiles sharing each token tile (bf16 path)
     int cta_pair;      // bf16 launches on CTA pairs (tcgen05 cta_group::2): 0 none, 1 all but gate/up,
                        // 2 all, 3 as 1 plus gate/up with two M tiles per CTA when pairing
+    int mx_rings;      // MXFP8 staged launches: 2 = weight and token rings, 1 = one ring of stages
 };
 // defaults for `rows` expert-major rows over E experts, overridable by
-// MOK_GEMM_GROUP / MOK_GEMM_PAIR / MOK_GEMM_CTA_PAIR
+// MOK_GEMM_GROUP / MOK_GEMM_PAIR / MOK_GEMM_CTA_PAIR / MOK_MX_RINGS
 GemmTuning gemm_tuning(int rows, int E);
 cudaError_t gemm_configure(int dev);
 // Token-side (B operand) tensor maps of one buffer with box heights 16, 32,
