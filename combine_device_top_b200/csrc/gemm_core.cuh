@@ -95,7 +95,8 @@ struct Bf16CfgT {
     static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
     static constexpr int EPI_OFF = NST * STAGE;           // one staging tile per epilogue group
     static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + slack for 1024-byte alignment
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + slack for 1024-byte alignment
 };
 using Bf16Cfg = Bf16CfgT<1, 4>;
 using Bf16PairCfg = Bf16CfgT<2, 3>;
@@ -124,7 +125,8 @@ struct Bf16Cta2CfgT {
     static constexpr int A_OFF = 0, B_OFF = SUB * A_BYTES;
     static constexpr int EPI_OFF = NST * STAGE;
     static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;
     static_assert(SMEM <= 232448, "CTA-pair layout exceeds shared memory");
 };
 using Bf16Cta2Cfg = Bf16Cta2CfgT<6>;
@@ -152,7 +154,8 @@ struct MxCfgT {
     static constexpr int STAGE = SFB_OFF + 1024;
     static constexpr int EPI_OFF = NST * STAGE;           // one staging tile per epilogue group
     static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;
     // TMEM: accumulators in columns [0, 480) (N <= 224), then the scale
     // factors of the SUB weight tiles (4 columns each) and of the tokens (8)
     static constexpr uint32_t TM_SFA = 480, TM_SFB = 480 + 4 * SUB;
@@ -189,8 +192,14 @@ struct MxSplitCfgT {
     static constexpr int T_BASE = NW * WSTAGE;
     static constexpr int EPI_OFF = T_BASE + NT * TSTAGE;  // one staging tile per epilogue group
     static constexpr int BAR_OFF = EPI_OFF + 2 * EPI_BYTES;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;
-    static constexpr uint32_t TM_SFA = 480, TM_SFB = 484;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;
+    // TMEM: accumulators in columns [0, 480) (N <= 224); two sets of scale
+    // factors (the weight tile's 4 columns, the tokens' 8), used by
+    // alternate K steps, so that the copy of step i + 1's scales does not
+    // overwrite columns step i's MMAs still read
+    static constexpr uint32_t TM_SFA = 480, TM_SFB = 484, TM_SF_SET = 12;
+    static_assert(TM_SFB + TM_SF_SET + 8 <= 512, "scale factors must fit in TMEM");
     static_assert(WSTAGE % 1024 == 0 && TSTAGE % 1024 == 0, "MXFP8 slots must keep 1024-byte alignment");
     static_assert(SMEM <= 232448, "MXFP8 two-ring layout exceeds shared memory");
 };
@@ -534,7 +543,8 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
         const int lead = u.brow0 & 3;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
-            if (!mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 80)) {
+            // the warp leaves or goes on as one (it synchronises below)
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, a.st, a.timeout_ns, 80))) {
                 ok = false;
                 break;
             }
@@ -567,7 +577,8 @@ __device__ __forceinline__ void gemm_sf_layout(const CoreArgs& a, const S& s, un
                     make_uint4(wb[0], wb[1], wb[2], wb[3]);
             }
             fence_proxy_async_shared();  // generic writes -> the TMEM copy (async proxy) reads
-            mbar_arrive(&sfready[stage]);
+            __syncwarp();                // every lane's writes and fence precede the one arrival
+            if (lane == 0) mbar_arrive(&sfready[stage]);
             if (++stage == C::NST) {
                 stage = 0;
                 phase ^= 1u;
@@ -689,8 +700,10 @@ __device__ __forceinline__ void mx_sf_layout_split(const CoreArgs& a, const S& s
         const int lead = u.brow0 & 3;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
-            if (!mbar_wait(&wfull[ws], wph, a.st, a.timeout_ns, 81) ||
-                !mbar_wait(&tkfull[ts], tph, a.st, a.timeout_ns, 82)) {
+            // the warp leaves or goes on as one (it synchronises below)
+            const bool landed = mbar_wait(&wfull[ws], wph, a.st, a.timeout_ns, 81) &&
+                                mbar_wait(&tkfull[ts], tph, a.st, a.timeout_ns, 82);
+            if (!__all_sync(0xffffffffu, landed)) {
                 ok = false;
                 break;
             }
@@ -721,7 +734,8 @@ __device__ __forceinline__ void mx_sf_layout_split(const CoreArgs& a, const S& s
                     make_uint4(wb[0], wb[1], wb[2], wb[3]);
             }
             fence_proxy_async_shared();  // generic writes -> the TMEM copy (async proxy) reads
-            mbar_arrive(&sfready[ts]);
+            __syncwarp();                // every lane's writes and fence precede the one arrival
+            if (lane == 0) mbar_arrive(&sfready[ts]);
             if (++ws == C::NW) {
                 ws = 0;
                 wph ^= 1u;
@@ -858,6 +872,7 @@ __device__ __forceinline__ void gemm_mma_mx_split(const CoreArgs& a, const S& s,
     int ws = 0, ts = 0;
     uint32_t tph = 0;
     uint32_t tk = 0;  // next accumulator ticket
+    uint32_t set = 0;  // scale-factor set of the next K step
     Unit u;
     for (int i = 0; s.get(i, u); ++i) {
         const int K = phase_k<C>(a, u.phase);
@@ -877,9 +892,12 @@ __device__ __forceinline__ void gemm_mma_mx_split(const CoreArgs& a, const S& s,
             const uint32_t sa = smem_u32(w + C::A_OFF);
             const uint32_t sb = smem_u32(t + C::B_OFF);
             // scale factors of this stage into TMEM (executed in order with the MMAs)
-            tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFA, w + C::SFA_OFF);
-            tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFB, t + C::SFB_OFF);
-            if (N > 128) tmem_cp_32x128b_warpx4(tmem_base + C::TM_SFB + 4, t + C::SFB_OFF + 512);
+            const uint32_t sfa = tmem_base + C::TM_SFA + set * C::TM_SF_SET;
+            const uint32_t sfb = tmem_base + C::TM_SFB + set * C::TM_SF_SET;
+            set ^= 1u;
+            tmem_cp_32x128b_warpx4(sfa, w + C::SFA_OFF);
+            tmem_cp_32x128b_warpx4(sfb, t + C::SFB_OFF);
+            if (N > 128) tmem_cp_32x128b_warpx4(sfb + 4, t + C::SFB_OFF + 512);
             const int nks = min(4, (K - kb * C::BKX) / 32);  // 32 K values per MMA
             for (int ks = 0; ks < nks; ++ks) {
                 // B: K-major E4M3 SW128, 32 K = 32 bytes inside the atom
@@ -891,8 +909,8 @@ __device__ __forceinline__ void gemm_mma_mx_split(const CoreArgs& a, const S& s,
                 // (K groups 1 KB apart); 32 K rows per MMA.
                 const uint64_t ad = u.phase == 0 ? umma_desc(sa + ks * 2048, 8192, 512, UMMA_LAYOUT_SW64)
                                                  : umma_desc(sa + ks * 4096, 0, 1024, UMMA_LAYOUT_SW128);
-                umma_mxf8(tmem_base + acc_col(tk, 0, false), ad, bd, idx, tmem_base + C::TM_SFA + sel,
-                          tmem_base + C::TM_SFB + sel, (kb | ks) != 0 ? 1u : 0u);
+                umma_mxf8(tmem_base + acc_col(tk, 0, false), ad, bd, idx, sfa + sel, sfb + sel,
+                          (kb | ks) != 0 ? 1u : 0u);
             }
             umma_commit(&wempty[ws]);
             umma_commit(&tkempty[ts]);
@@ -1242,7 +1260,7 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
     volatile int* ok_flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // one per epilogue group
     int* done_cnt = const_cast<int*>(ok_flags) + 2;                            // two, by unit parity
-    static_assert(((C::SPLIT ? 2 * NWR + 3 * C::NST : 3 * C::NST) + 5) * 8 + 4 * 5 <= 256, "barrier region");
+    static_assert(((C::SPLIT ? 2 * NWR + 3 * C::NST : 3 * C::NST) + 5) * 8 + 4 * 5 <= C::BAR_BYTES, "barrier region");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -1256,13 +1274,13 @@ __device__ __forceinline__ void gemm_cta(const GemmMaps& maps, const MxMaps* mx,
             for (int st = 0; st < C::NST; ++st) {
                 mbar_init(&tkfull[st], 1);
                 mbar_init(&tkempty[st], 1);
-                mbar_init(&sfready[st], 32);
+                mbar_init(&sfready[st], 1);
             }
         } else {
             for (int st = 0; st < C::NST; ++st) {
                 mbar_init(&full[st], 1);
                 mbar_init(&empty[st], 1);
-                mbar_init(&sfready[st], 32);
+                mbar_init(&sfready[st], 1);
             }
         }
         for (int b = 0; b < 2; ++b) {
