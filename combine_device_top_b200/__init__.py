@@ -692,19 +692,24 @@ class EpGroup:
     def forward(self, logits_local: torch.Tensor, w_gate, w_up, w_down, y: torch.Tensor | None = None,
                 timeout_ns: int = 0, stream=None) -> torch.Tensor:
         """One step over the tokens in ``self.x``: returns y [S_r, H] bf16.
-        w_*: this rank's experts' weights."""
-        self.step += 1
-        p = plan(self.gather_logits(logits_local), self.k, self.G, stream=stream)
-        ep_dispatch_ffn(p, self.desc, w_gate, w_up, w_down, self.step, self.ws, timeout_ns, stream)
-        if y is None:
-            y = torch.empty((self.S_r, self.H), dtype=torch.bfloat16, device=self.device)
-        return ep_combine(p, self.desc, y, self.step, self.ws, timeout_ns, stream)
+        w_*: this rank's experts' weights.  Everything, the all-gather of the
+        logits included, is ordered on ``stream`` (default: the current
+        stream), after whatever wrote ``self.x`` there."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            self.step += 1
+            p = plan(self.gather_logits(logits_local), self.k, self.G, stream=s)
+            ep_dispatch_ffn(p, self.desc, w_gate, w_up, w_down, self.step, self.ws, timeout_ns, s)
+            if y is None:
+                y = torch.empty((self.S_r, self.H), dtype=torch.bfloat16, device=self.device)
+            return ep_combine(p, self.desc, y, self.step, self.ws, timeout_ns, s)
 
     def status(self, stream=None) -> int:
         return get_status(self.ws, stream)
 
     def close(self) -> None:
-        """Unmap the other ranks' buffers (after the last step has finished)."""
+        """Unmap the other ranks' buffers.  Call it once every rank's last
+        step has finished (synchronise, then a barrier of the group)."""
         for b in self._opened:
             self.close_(b)
         self._opened = []
