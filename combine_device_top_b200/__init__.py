@@ -47,7 +47,8 @@ EXPORTS = (
     "mok_two_wave_rows", "mok_minibatch_bounds", "mok_forward_host_batches_workspace_bytes",
     "mok_moe_forward_host_batches", "mok_router_weights_bytes", "mok_router_prepare", "mok_plan_router",
     "mok_backward_workspace_bytes", "mok_moe_backward", "mok_slot_bytes", "mok_slot_exp_offset",
-    "mok_ep_slot_bytes", "mok_ep_workspace_bytes", "mok_ep_dispatch_ffn", "mok_ep_combine",
+    "mok_ep_slot_bytes", "mok_ep_workspace_bytes", "mok_ep_dispatch_ffn", "mok_ep_dispatch_ffn_mxfp8",
+    "mok_ep_combine",
     "mok_ipc_export", "mok_ipc_import", "mok_ipc_close",
 )
 
@@ -75,7 +76,7 @@ class FwdOpts(ctypes.Structure):
 class EpT(ctypes.Structure):
     """``mok_ep_t``: one rank's view of an expert-parallel group."""
     _fields_ = [("G", ctypes.c_int32), ("g", ctypes.c_int32), ("e0", ctypes.c_int32), ("e_loc", ctypes.c_int32),
-                ("sync", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("sync", ctypes.c_int32), ("mxfp8", ctypes.c_int32),
                 ("x", ctypes.c_void_p * MOK_MAX_SHARDS), ("slots", ctypes.c_void_p * MOK_MAX_SHARDS)]
 
 
@@ -138,11 +139,14 @@ def lib() -> ctypes.CDLL:
     L.mok_ep_workspace_bytes.restype = sz
     L.mok_ep_dispatch_ffn.argtypes = [ctypes.POINTER(PlanT), ctypes.POINTER(EpT), i32, i32, vp, vp, vp, u32, u64, vp,
                                       sz, vp]
+    L.mok_ep_dispatch_ffn_mxfp8.argtypes = [ctypes.POINTER(PlanT), ctypes.POINTER(EpT), i32, i32, vp, u32, u64, vp,
+                                            sz, vp]
     L.mok_ep_combine.argtypes = [ctypes.POINTER(PlanT), ctypes.POINTER(EpT), i32, u32, u64, vp, vp, sz, vp]
     L.mok_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_size_t)]
     L.mok_ipc_import.argtypes = [vp, ctypes.POINTER(ctypes.c_void_p)]
     L.mok_ipc_close.argtypes = [vp]
-    for n in ("mok_ep_dispatch_ffn", "mok_ep_combine", "mok_ipc_export", "mok_ipc_import", "mok_ipc_close"):
+    for n in ("mok_ep_dispatch_ffn", "mok_ep_dispatch_ffn_mxfp8", "mok_ep_combine", "mok_ipc_export",
+              "mok_ipc_import", "mok_ipc_close"):
         getattr(L, n).restype = ctypes.c_int
     for n in ("mok_plan", "mok_moe_forward", "mok_get_status", "mok_gather", "mok_expert_ffn", "mok_combine",
               "mok_moe_forward_host", "mok_plan_noalloc", "mok_mxfp8_quantize_rows",
@@ -573,12 +577,13 @@ def ep_workspace_bytes(T: int, H: int, I: int, e_loc: int, k: int) -> int:
     return lib().mok_ep_workspace_bytes(T, H, I, e_loc, k)
 
 
-def ep_desc(G: int, g: int, e0: int, e_loc: int, x_ptrs, slot_ptrs, sync: int = MOK_EP_SYNC_DEVICE) -> EpT:
+def ep_desc(G: int, g: int, e0: int, e_loc: int, x_ptrs, slot_ptrs, sync: int = MOK_EP_SYNC_DEVICE,
+            mxfp8: bool = False) -> EpT:
     """A ``mok_ep_t`` from the ranks' x and slot-buffer addresses (ints, as
     this GPU addresses them)."""
     assert len(x_ptrs) == G and len(slot_ptrs) == G and 1 <= G <= MOK_MAX_SHARDS
     d = EpT()
-    d.G, d.g, d.e0, d.e_loc, d.sync = G, g, e0, e_loc, sync
+    d.G, d.g, d.e0, d.e_loc, d.sync, d.mxfp8 = G, g, e0, e_loc, sync, int(bool(mxfp8))
     for h in range(G):
         d.x[h] = x_ptrs[h]
         d.slots[h] = slot_ptrs[h]
@@ -595,6 +600,19 @@ def ep_dispatch_ffn(p: Plan, ep: EpT, w_gate, w_up, w_down, step: int, ws: torch
     _check(lib().mok_ep_dispatch_ffn(ctypes.byref(p.c), ctypes.byref(ep), H, I, ctypes.c_void_p(w_gate.data_ptr()),
                                      ctypes.c_void_p(w_up.data_ptr()), ctypes.c_void_p(w_down.data_ptr()), step,
                                      timeout_ns, ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)))
+
+
+def ep_dispatch_ffn_mxfp8(p: Plan, ep: EpT, pack, H: int, step: int, ws: torch.Tensor, timeout_ns: int = 0,
+                          stream=None) -> None:
+    """The MXFP8 path of :func:`ep_dispatch_ffn`; pack = (qg, sg, qu, su, qd,
+    sd) of this rank's experts (:func:`quantize_weights_mxfp8`)."""
+    qg, sg, qu, su, qd, sd = pack
+    I = qg.shape[-1]
+    assert qg.shape[0] == ep.e_loc and ep.mxfp8 == 1
+    w = MxWeights(qg.data_ptr(), sg.data_ptr(), qu.data_ptr(), su.data_ptr(), qd.data_ptr(), sd.data_ptr())
+    _check(lib().mok_ep_dispatch_ffn_mxfp8(ctypes.byref(p.c), ctypes.byref(ep), H, I,
+                                           ctypes.cast(ctypes.byref(w), ctypes.c_void_p), step, timeout_ns,
+                                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)))
 
 
 def ep_combine(p: Plan, ep: EpT, y: torch.Tensor, step: int, ws: torch.Tensor, timeout_ns: int = 0,
@@ -642,7 +660,8 @@ class EpGroup:
     (export, import, close) functions, e.g. by fakes in host-only tests.
     """
 
-    def __init__(self, T: int, H: int, I: int, E: int, k: int, device=None, group=None, ipc=None):
+    def __init__(self, T: int, H: int, I: int, E: int, k: int, device=None, group=None, ipc=None,
+                 mxfp8: bool = False):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -650,6 +669,7 @@ class EpGroup:
         self.g = dist.get_rank(group) if dist.is_initialized() else 0
         assert T % self.G == 0, "T must split evenly over the ranks"
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
+        self.mxfp8 = bool(mxfp8)
         self.S_r = T // self.G
         self.e0, self.e_loc = ep_partition(E, self.G, self.g)
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
@@ -660,7 +680,7 @@ class EpGroup:
         self.slots = torch.zeros(ep_slot_bytes(self.S_r, H, k), dtype=torch.uint8, device=self.device)
         self.ws = _workspace(ep_workspace_bytes(T, H, I, self.e_loc, k), self.device)
         xp, sp = self._exchange()
-        self.desc = ep_desc(self.G, self.g, self.e0, self.e_loc, xp, sp, MOK_EP_SYNC_DEVICE)
+        self.desc = ep_desc(self.G, self.g, self.e0, self.e_loc, xp, sp, MOK_EP_SYNC_DEVICE, self.mxfp8)
 
     def _exchange(self):
         """Every rank's x and slot addresses as this GPU addresses them."""
@@ -692,14 +712,18 @@ class EpGroup:
     def forward(self, logits_local: torch.Tensor, w_gate, w_up, w_down, y: torch.Tensor | None = None,
                 timeout_ns: int = 0, stream=None) -> torch.Tensor:
         """One step over the tokens in ``self.x``: returns y [S_r, H] bf16.
-        w_*: this rank's experts' weights.  Everything, the all-gather of the
-        logits included, is ordered on ``stream`` (default: the current
-        stream), after whatever wrote ``self.x`` there."""
+        w_*: this rank's experts' weights (MXFP8 group: w_gate is the pack of
+        :func:`quantize_weights_mxfp8`, w_up and w_down None).  Everything,
+        the all-gather of the logits included, is ordered on ``stream``
+        (default: the current stream), after whatever wrote ``self.x`` there."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         with torch.cuda.stream(s):
             self.step += 1
             p = plan(self.gather_logits(logits_local), self.k, self.G, stream=s)
-            ep_dispatch_ffn(p, self.desc, w_gate, w_up, w_down, self.step, self.ws, timeout_ns, s)
+            if self.mxfp8:
+                ep_dispatch_ffn_mxfp8(p, self.desc, w_gate, self.H, self.step, self.ws, timeout_ns, s)
+            else:
+                ep_dispatch_ffn(p, self.desc, w_gate, w_up, w_down, self.step, self.ws, timeout_ns, s)
             if y is None:
                 y = torch.empty((self.S_r, self.H), dtype=torch.bfloat16, device=self.device)
             return ep_combine(p, self.desc, y, self.step, self.ws, timeout_ns, s)

@@ -4,6 +4,7 @@
 // workspace.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -1235,10 +1236,11 @@ static size_t ep_layout(int T, int H, int I, int e_loc, int k, EpLayout* L) {
     off += align256(sizeof(Chunk) * (size_t)L->max_chunks);
     L->mbs = off;
     off += align256(sizeof(Minibatch) * (size_t)L->max_mb);
+    // rows and h: bf16, or (MXFP8 path) E4M3 bytes followed by their scale planes
     L->rows = off;
-    off += align256((size_t)ns * H * 2);
+    off += std::max(align256((size_t)ns * H * 2), align256((size_t)ns * H) + align256(mx_sc_bytes(ns, H)));
     L->h = off;
-    off += align256((size_t)ns * I * 2);
+    off += std::max(align256((size_t)ns * I * 2), align256((size_t)ns * I) + align256(mx_sc_bytes(ns, I)));
     L->total = off;
     return off;
 }
@@ -1252,6 +1254,7 @@ static int check_ep(const mok_plan_t* plan, const mok_ep_t* ep, int H) {
         return fail(MOK_ERR_INVALID_ARG, "experts [%d, %d) outside 0 .. %d", ep->e0, ep->e0 + ep->e_loc, plan->E);
     if (ep->sync != MOK_EP_SYNC_CALLER && ep->sync != MOK_EP_SYNC_DEVICE)
         return fail(MOK_ERR_INVALID_ARG, "unknown EP sync mode %d", ep->sync);
+    if (ep->mxfp8 != 0 && ep->mxfp8 != 1) return fail(MOK_ERR_INVALID_ARG, "ep mxfp8 must be 0 or 1");
     if (H <= 0 || H % 128) return fail(MOK_ERR_UNSUPPORTED, "H %% 128 != 0 (H = %d)", H);
     for (int r = 0; r < ep->G; ++r) {
         if (!ep->x[r] || !ep->slots[r]) return fail(MOK_ERR_INVALID_ARG, "NULL pointer of rank %d", r);
@@ -1310,18 +1313,30 @@ size_t mok_ep_workspace_bytes(int T, int H, int I, int e_loc, int k) {
     return ep_layout(T, H, I, e_loc, k, &L);
 }
 
-int mok_ep_dispatch_ffn(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I, const void* w_gate,
-                        const void* w_up, const void* w_down, uint32_t step, uint64_t timeout_ns, void* ws,
-                        size_t ws_bytes, mok_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+}  // extern "C"
+
+namespace mok {
+
+// The body of both dispatch calls: barrier, set-up, work list, pull (bf16 or
+// quantising) and the grouped FFN with push destinations.
+static int ep_dispatch(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I, const void* w_gate,
+                       const void* w_up, const void* w_down, const mok_mxfp8_weights* mxw, uint32_t step,
+                       uint64_t timeout_ns, void* ws, size_t ws_bytes, cudaStream_t stream) {
     int rc = check_plan(plan);
     if (rc) return rc;
     if ((rc = check_hi(H, I))) return rc;
     if ((rc = check_ep(plan, ep, H))) return rc;
     if (step < 1) return fail(MOK_ERR_INVALID_ARG, "step counts from 1");
+    if ((ep->mxfp8 != 0) != (mxw != nullptr))
+        return fail(MOK_ERR_INVALID_ARG, "ep->mxfp8 does not match the call (bf16 or MXFP8 weights)");
     EpLayout L;
     if ((rc = check_ws(ws, ws_bytes, ep_layout(plan->T, H, I, ep->e_loc, plan->k, &L)))) return rc;
-    if (ep->e_loc > 0 && (!w_gate || !w_up || !w_down)) return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
+    if (ep->e_loc > 0) {
+        if (mxw ? (!mxw->gate || !mxw->gate_scales || !mxw->up || !mxw->up_scales || !mxw->down ||
+                   !mxw->down_scales)
+                : (!w_gate || !w_up || !w_down))
+            return fail(MOK_ERR_INVALID_ARG, "NULL weight pointer");
+    }
     unsigned char* base = static_cast<unsigned char*>(ws);
     DevStatus* status = reinterpret_cast<DevStatus*>(base + L.status);
     MOK_CUDA(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream), "status reset");
@@ -1345,17 +1360,48 @@ int mok_ep_dispatch_ffn(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I
     Chunk* chunks = reinterpret_cast<Chunk*>(base + L.chunks);
     Minibatch* mbs = reinterpret_cast<Minibatch*>(base + L.mbs);
     MOK_CUDA(launch_ep_setup(pd, push_dev, plan->offsets, ep->e0, ep->e_loc, offsets_loc, stream), "EP setup launch");
-    MOK_CUDA(launch_build_chunks(offsets_loc, ep->e_loc, ns, ns, ns, CHUNK_MAX_ROWS, 0, 1, chunks, L.max_chunks, mbs,
-                                 L.max_mb, counts2, status, stream),
+    MOK_CUDA(launch_build_chunks(offsets_loc, ep->e_loc, ns, ns, ns, mxw ? CHUNK_MAX_ROWS_MX : CHUNK_MAX_ROWS, 0, 1,
+                                 chunks, L.max_chunks, mbs, L.max_mb, counts2, status, stream),
              "work list launch");
+    // the GEMM's tuning sees the rows this rank's experts hold on average
+    const int tune_rows = (int)((int64_t)ns * ep->e_loc / plan->E);
+    if (mxw) {
+        MxTokenScales mxs;
+        mxs.sc_rows = mx_sc_rows(ns);
+        mxs.xsc = base + L.rows + align256((size_t)ns * H);
+        mxs.hsc = base + L.h + align256((size_t)ns * I);
+        MOK_CUDA(launch_ep_pull_mx(xs, H, plan->offsets, ep->e0, ep->e_loc, plan->sched_src_rank,
+                                   plan->sched_src_index, plan->row_slot, base + L.rows,
+                                   const_cast<uint8_t*>(mxs.xsc), mxs.sc_rows, row_slot_loc, ns, sms, stream),
+                 "pull dispatch launch");
+        return run_expert_ffn(base + L.rows, ns, H, I, nullptr, nullptr, nullptr, ep->e_loc, row_slot_loc, chunks,
+                              counts2, base + L.h, nullptr, status, kDefaultTimeoutNs, stream, mxw, &mxs, nullptr,
+                              push_dev, S_r * plan->k, tune_rows);
+    }
     MOK_CUDA(launch_ep_pull(xs, H, plan->offsets, ep->e0, ep->e_loc, plan->sched_src_rank, plan->sched_src_index,
                             plan->row_slot, base + L.rows, row_slot_loc, ns, sms, stream),
              "pull dispatch launch");
-    // the GEMM's tuning sees the rows this rank's experts hold on average
-    const int tune_rows = (int)((int64_t)ns * ep->e_loc / plan->E);
     return run_expert_ffn(base + L.rows, ns, H, I, w_gate, w_up, w_down, ep->e_loc, row_slot_loc, chunks, counts2,
                           base + L.h, nullptr, status, kDefaultTimeoutNs, stream, nullptr, nullptr, nullptr, push_dev,
                           S_r * plan->k, tune_rows);
+}
+
+}  // namespace mok
+
+extern "C" {
+
+int mok_ep_dispatch_ffn(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I, const void* w_gate,
+                        const void* w_up, const void* w_down, uint32_t step, uint64_t timeout_ns, void* ws,
+                        size_t ws_bytes, mok_stream_t stream) {
+    return ep_dispatch(plan, ep, H, I, w_gate, w_up, w_down, nullptr, step, timeout_ns, ws, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mok_ep_dispatch_ffn_mxfp8(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I, const mok_mxfp8_weights* w,
+                              uint32_t step, uint64_t timeout_ns, void* ws, size_t ws_bytes, mok_stream_t stream) {
+    if (!w) return fail(MOK_ERR_INVALID_ARG, "NULL MXFP8 weights");
+    return ep_dispatch(plan, ep, H, I, nullptr, nullptr, nullptr, w, step, timeout_ns, ws, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 int mok_ep_combine(const mok_plan_t* plan, const mok_ep_t* ep, int H, uint32_t step, uint64_t timeout_ns, void* y,
@@ -1376,8 +1422,8 @@ int mok_ep_combine(const mok_plan_t* plan, const mok_ep_t* ep, int H, uint32_t s
     if (sms <= 0) return fail(MOK_ERR_CUDA, "no CUDA device");
     ShardsOut ys{};
     ys.p[0] = y;
-    MOK_CUDA(launch_combine(ep->slots[ep->g], MOK_SLOTS_F16S, plan->gates + (size_t)ep->g * S_r * plan->k, S_r,
-                            plan->k, H, S_r, ys, sms, stream),
+    MOK_CUDA(launch_combine(ep->slots[ep->g], ep->mxfp8 ? MOK_SLOTS_BF16 : MOK_SLOTS_F16S,
+                            plan->gates + (size_t)ep->g * S_r * plan->k, S_r, plan->k, H, S_r, ys, sms, stream),
              "combine launch");
     return MOK_OK;
 }

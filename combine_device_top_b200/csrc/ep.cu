@@ -16,12 +16,14 @@
 //                 row) and the device copy of the slot-buffer pointers;
 //   k_ep_pull     pull dispatch: its experts' rows, each read from the
 //                 source rank's x (16-byte loads over NVLink) into a local
-//                 expert-major buffer;
+//                 expert-major buffer (k_ep_pull_mx on the MXFP8 path:
+//                 quantised to E4M3 rows and block scales on the way);
 //   the grouped GEMM of the single-GPU path over those rows, whose down
 //                 epilogue stores every slot row into the source rank's slot
 //                 buffer (the push);
 //   k_ep_barrier  every rank's pushes have landed;
 //   the combine   over its own tokens' slot rows, from local memory.
+#include "dispatch_combine.cuh"
 #include "mok_device.cuh"
 #include "mok_internal.h"
 
@@ -77,6 +79,50 @@ __global__ void __launch_bounds__(EP_THREADS, 4)
     }
 }
 
+// The MXFP8 pull: as k_ep_pull, each row quantised on the way (32-element
+// blocks, OCP MX): rows_q[i] the E4M3 bytes, the scale planes [H/128]
+// [sc_rows][4] at row i.  A warp per row, four 256-element steps' loads in
+// flight per lane.  H % 128 == 0.
+__global__ void __launch_bounds__(EP_THREADS, 4)
+    k_ep_pull_mx(const __grid_constant__ ShardsIn xs, int H, const int32_t* __restrict__ offsets, int e0, int e_loc,
+                 const int32_t* __restrict__ src_rank, const int32_t* __restrict__ src_index,
+                 const int32_t* __restrict__ row_slot, uint8_t* __restrict__ rows_q, uint8_t* __restrict__ xsc,
+                 int sc_rows, int32_t* __restrict__ row_slot_loc) {
+    const int r0 = __ldg(offsets + e0);
+    const int n = __ldg(offsets + e0 + e_loc) - r0;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (EP_THREADS / 32);
+    uint32_t* planes = reinterpret_cast<uint32_t*>(xsc);
+    for (int i = blockIdx.x * (EP_THREADS / 32) + (threadIdx.x >> 5); i < n; i += warps) {
+        const int row = r0 + i;
+        const uint4* src = reinterpret_cast<const uint4*>(xs.p[__ldg(src_rank + row)]) +
+                           (size_t)__ldg(src_index + row) * (H >> 3);
+        uint8_t* dst = rows_q + (size_t)i * H;
+        if (lane == 0) row_slot_loc[i] = __ldg(row_slot + row);
+        for (int c0 = 0; c0 < H; c0 += 1024) {
+            uint4 raw[4];
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                const int c = c0 + 256 * s4 + lane * 8;
+                raw[s4] = c < H ? __ldg(src + (c >> 3)) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                const int cs = c0 + 256 * s4;
+                if (cs >= H) break;  // warp-uniform
+                uint2 q;
+                uint32_t word;
+                warp_mx_quant8(raw[s4], q, word, lane);
+                const int c = cs + lane * 8;
+                if (c < H) {
+                    *reinterpret_cast<uint2*>(dst + c) = q;
+                    if ((lane & 15) == 0) planes[(size_t)((cs >> 7) + (lane >> 4)) * sc_rows + i] = word;
+                }
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ void red_add_release_sys(uint32_t* p, uint32_t v) {
     asm volatile("red.release.sys.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -125,6 +171,19 @@ cudaError_t launch_ep_pull(const ShardsIn& xs, int H, const int32_t* offsets, in
     const int grid = want < num_sms * 4 ? want : num_sms * 4;
     k_ep_pull<<<grid, EP_THREADS, 0, stream>>>(xs, H, offsets, e0, e_loc, src_rank, src_index, row_slot,
                                                reinterpret_cast<uint4*>(rows), row_slot_loc);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_pull_mx(const ShardsIn& xs, int H, const int32_t* offsets, int e0, int e_loc,
+                              const int32_t* src_rank, const int32_t* src_index, const int32_t* row_slot,
+                              void* rows_q, void* xsc, int sc_rows, int32_t* row_slot_loc, int max_rows, int num_sms,
+                              cudaStream_t stream) {
+    if (max_rows <= 0) return cudaSuccess;
+    const int want = (max_rows + (EP_THREADS / 32) - 1) / (EP_THREADS / 32);
+    const int grid = want < num_sms * 4 ? want : num_sms * 4;
+    k_ep_pull_mx<<<grid, EP_THREADS, 0, stream>>>(xs, H, offsets, e0, e_loc, src_rank, src_index, row_slot,
+                                                  reinterpret_cast<uint8_t*>(rows_q), reinterpret_cast<uint8_t*>(xsc),
+                                                  sc_rows, row_slot_loc);
     return cudaGetLastError();
 }
 

@@ -185,6 +185,12 @@ cudaError_t launch_ep_setup(const PushDest& push, PushDest* push_dev, const int3
 cudaError_t launch_ep_pull(const ShardsIn& xs, int H, const int32_t* offsets, int e0, int e_loc,
                            const int32_t* src_rank, const int32_t* src_index, const int32_t* row_slot, void* rows,
                            int32_t* row_slot_loc, int max_rows, int num_sms, cudaStream_t stream);
+// the same pull quantised to MXFP8: rows_q [*, H] E4M3, scale planes
+// [H/128][sc_rows][4] indexed by local row
+cudaError_t launch_ep_pull_mx(const ShardsIn& xs, int H, const int32_t* offsets, int e0, int e_loc,
+                              const int32_t* src_rank, const int32_t* src_index, const int32_t* row_slot,
+                              void* rows_q, void* xsc, int sc_rows, int32_t* row_slot_loc, int max_rows, int num_sms,
+                              cudaStream_t stream);
 // one arrival on every rank's counter, then a bounded wait for this rank's
 // counter (counters.p[g]) to reach target
 cudaError_t launch_ep_barrier(const ShardsOut& counters, int G, int g, uint32_t target, void* status,

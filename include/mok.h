@@ -570,7 +570,9 @@ typedef struct mok_ep_t {
     int32_t e0;    /* this rank's experts: e0 .. e0 + e_loc - 1 of the plan's */
     int32_t e_loc; /* E (e_loc may be 0)                                      */
     int32_t sync;  /* MOK_EP_SYNC_DEVICE or MOK_EP_SYNC_CALLER                */
-    int32_t reserved;
+    int32_t mxfp8; /* 0: bf16 path (mok_ep_dispatch_ffn, fp16 slot rows with  */
+                   /* exponents); 1: MXFP8 path (mok_ep_dispatch_ffn_mxfp8,   */
+                   /* bf16 slot rows)                                          */
     /* x[h]: rank h's tokens [S_r, H] bf16, as THIS GPU addresses them (a
      * peer pointer from mok_ipc_import, or a local pointer), 16-byte
      * aligned; h < G. */
@@ -582,13 +584,14 @@ typedef struct mok_ep_t {
 } mok_ep_t;
 
 /* Bytes of one rank's slot buffer: [S_r*k, H] fp16 slot rows with their
- * block exponents (the MOK_SLOTS_F16S form of mok_slot_bytes), then the
- * 256-byte barrier counter region.  H % 128 == 0; 0 if the shape is invalid. */
+ * block exponents (the MOK_SLOTS_F16S form of mok_slot_bytes; the MXFP8
+ * path stores bf16 rows [S_r*k, H] at its start), then the 256-byte barrier
+ * counter region.  H % 128 == 0; 0 if the shape is invalid. */
 size_t mok_ep_slot_bytes(int S_r, int H, int k);
 
-/* Bytes of the per-rank workspace for (T, H, I, e_loc, k): status word, the
- * local expert offsets, the work list, and room for every slot's row and h
- * row (a rank may receive all T*k rows). */
+/* Bytes of the per-rank workspace for (T, H, I, e_loc, k), either path:
+ * status word, the local expert offsets, the work list, and room for every
+ * slot's row and h row (a rank may receive all T*k rows). */
 size_t mok_ep_workspace_bytes(int T, int H, int I, int e_loc, int k);
 
 /*
@@ -612,11 +615,24 @@ int mok_ep_dispatch_ffn(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I
                         mok_stream_t stream);
 
 /*
+ * mok_ep_dispatch_ffn_mxfp8 -- the same on the MXFP8 path (ep->mxfp8 == 1):
+ * the pull quantises each row to E4M3 with its block scales (as
+ * mok_gather_mxfp8), the grouped FFN runs on the block-scaled MMA (as
+ * mok_expert_ffn_mxfp8) with `w`, the pack of mok_quantize_weights_mxfp8
+ * for this rank's e_loc experts (host struct, device arrays), and the down
+ * epilogue pushes bf16 slot rows.  The results equal mok_moe_forward's
+ * staged MXFP8 path over the same plan, bit for bit.
+ */
+int mok_ep_dispatch_ffn_mxfp8(const mok_plan_t* plan, const mok_ep_t* ep, int H, int I,
+                              const mok_mxfp8_weights* w, uint32_t step, uint64_t timeout_ns,
+                              void* ws, size_t ws_bytes, mok_stream_t stream);
+
+/*
  * mok_ep_combine -- the second half of step `step` on rank ep->g: barrier
  * (MOK_EP_SYNC_DEVICE; arrival number 2*step), then
  *   y[i] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]),  t = g*S_r + i,
- * over the slot rows in this rank's slot buffer (ep->slots[ep->g]), fp32,
- * j ascending.  y: [S_r, H] bf16, 16-byte aligned.  ws: the workspace given
+ * over the slot rows in this rank's slot buffer (ep->slots[ep->g]; fp16
+ * with exponents, or bf16 when ep->mxfp8), fp32, j ascending.  y: [S_r, H] bf16, 16-byte aligned.  ws: the workspace given
  * to mok_ep_dispatch_ffn (its status word).  Asynchronous on `stream`.
  */
 int mok_ep_combine(const mok_plan_t* plan, const mok_ep_t* ep, int H, uint32_t step,

@@ -97,6 +97,35 @@ def test_ep_dispatch_rejects_bad_buffers_and_steps():
     assert rc == mok.MOK_ERR_WORKSPACE and "small" in msg
 
 
+def test_ep_dispatch_checks_the_path():
+    L = mok.lib()
+    p = _fake_plan()
+    ep = _fake_ep()
+    ep.mxfp8 = 1                                               # bf16 call on an MXFP8 group
+    rc, msg = _dispatch(p, ep)
+    assert rc == mok.MOK_ERR_INVALID_ARG and "mxfp8" in msg
+    ep.mxfp8 = 2
+    assert _dispatch(p, ep)[0] == mok.MOK_ERR_INVALID_ARG
+    ep = _fake_ep()
+    rc = L.mok_ep_dispatch_ffn_mxfp8(ctypes.byref(p), ctypes.byref(ep), 256, 128, None, 1, 0,
+                                     ctypes.c_void_p(0x800000), 1 << 40, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG                       # no weights
+    w = mok.MxWeights(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000)
+    rc = L.mok_ep_dispatch_ffn_mxfp8(ctypes.byref(p), ctypes.byref(ep), 256, 128,
+                                     ctypes.cast(ctypes.byref(w), ctypes.c_void_p), 1, 0,
+                                     ctypes.c_void_p(0x800000), 1 << 40, None)
+    assert rc == mok.MOK_ERR_INVALID_ARG                       # MXFP8 call on a bf16 group
+    assert "mxfp8" in L.mok_last_error_string().decode()
+
+
+def test_ep_workspace_holds_either_path():
+    T, H, I, k = 512, 7168, 2048, 8
+    ns = T * k
+    ws = mok.ep_workspace_bytes(T, H, I, 48, k)
+    sc = lambda K: (K // 128) * (((ns + 3) & ~3) + 4) * 4
+    assert ws >= ns * (H + I) * 2 and ws >= ns * (H + I) + sc(H) + sc(I)
+
+
 def test_ep_combine_rejects_bad_arguments():
     L = mok.lib()
     p = _fake_plan()

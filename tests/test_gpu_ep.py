@@ -208,3 +208,60 @@ def test_ipc_export_import_between_processes():
     proc.join(timeout=120)
     assert status == "ok", detail
     assert proc.exitcode == 0
+
+
+# ---------------------------------------------------------------- the MXFP8 path
+def _mx_pack(wg, wu, wd):
+    if wg.shape[0] == 0:  # a rank without experts: no weights to quantise
+        H, I = wg.shape[1], wg.shape[2]
+        shapes = [(0, H, I), (0, H // 32, I), (0, H, I), (0, H // 32, I), (0, I, H), (0, I // 32, H)]
+        return tuple(torch.empty(sh, dtype=torch.uint8, device="cuda") for sh in shapes)
+    return (*mok.quantize_weights_mxfp8(wg), *mok.quantize_weights_mxfp8(wu), *mok.quantize_weights_mxfp8(wd))
+
+
+MX_CASES = {
+    "ragged": small(T=384, H=256, I=128, E=10, k=3, R=1, seed=741),
+    "few_experts": small(T=256, H=384, I=256, E=3, k=2, R=1, seed=742),
+}
+
+
+@pytest.mark.parametrize("name", list(MX_CASES))
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_ep_mxfp8_ranks_match_the_single_gpu_forward(name, G):
+    """The MXFP8 path (quantising pull, block-scaled FFN, bf16 slot rows
+    pushed to the token's rank) over G emulated ranks equals the staged
+    MXFP8 forward bit for bit; each rank quantises only its own experts."""
+    case = Case(MX_CASES[name])
+    cfg = case.cfg
+    p = mok.plan(case.dlogits, cfg.k, G)
+    ys, _ = mok.moe_forward_mxfp8(mok.shards(case.dx, G), _mx_pack(case.dwg, case.dwu, case.dwd), p)
+    want = torch.cat(ys)
+    ranks = Ranks(case, G)
+    for d in ranks.desc:
+        d.mxfp8 = 1
+    packs = [_mx_pack(*ranks.w[h]) for h in range(G)]
+    y = [torch.empty((ranks.S_r, cfg.H), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    for h in range(G):
+        mok.ep_dispatch_ffn_mxfp8(p, ranks.desc[h], packs[h], cfg.H, 1, ranks.ws[h])
+    for h in range(G):
+        mok.ep_combine(p, ranks.desc[h], y[h], 1, ranks.ws[h])
+    for h in range(G):
+        assert mok.get_status(ranks.ws[h]) == mok.MOK_OK
+    assert torch.equal(torch.cat(y), want)
+
+
+def test_ep_group_driver_mxfp8_with_one_rank():
+    """EpGroup(mxfp8=True) on one rank, device barriers, two steps."""
+    case = Case(MX_CASES["ragged"])
+    cfg = case.cfg
+    pack = _mx_pack(case.dwg, case.dwu, case.dwd)
+    p = mok.plan(case.dlogits, cfg.k, 1)
+    ys, _ = mok.moe_forward_mxfp8([case.dx], pack, p)
+    grp = mok.EpGroup(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, mxfp8=True)
+    grp.x.copy_(case.dx)
+    for _ in range(2):
+        y = grp.forward(case.dlogits, pack, None, None)
+        assert grp.status() == mok.MOK_OK
+        assert torch.equal(y, ys[0])
+    grp.close()
+
