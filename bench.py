@@ -502,10 +502,11 @@ def time_ep(cfg, device, steps: int, warmup: int, wl: Workload | None = None):
     dist = torch.distributed
     world = dist.get_world_size() if dist.is_initialized() else 1
     rank = dist.get_rank() if dist.is_initialized() else 0
-    grp = mok.EpGroup(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, device=device)
+    grp = mok.EpGroup(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, device=device, mxfp8=cfg.mxfp8)
     S_r = grp.S_r
     if wl is not None and world == 1:
-        x, logits_local, w = wl.dx, wl.dlogits, wl.w
+        x, logits_local = wl.dx, wl.dlogits
+        w = (wl.pack, None, None) if cfg.mxfp8 else wl.w
     else:
         x_all = mokgen.tokens(cfg)
         logits_all = mokgen.router_logits(cfg, x_all)
@@ -517,6 +518,13 @@ def time_ep(cfg, device, steps: int, warmup: int, wl: Workload | None = None):
         for i, e in enumerate(range(grp.e0, grp.e0 + grp.e_loc)):
             for dst, src in zip(w, mokgen.expert_weights(cfg, e)):
                 dst[i].copy_(src)
+        if cfg.mxfp8:
+            if grp.e_loc:
+                pack = tuple(t for wt in w for t in mok.quantize_weights_mxfp8(wt))
+            else:
+                shapes = [(0, cfg.H, cfg.I), (0, cfg.H // 32, cfg.I)] * 2 + [(0, cfg.I, cfg.H), (0, cfg.I // 32, cfg.H)]
+                pack = tuple(torch.empty(sh, dtype=torch.uint8, device=device) for sh in shapes)
+            w = (pack, None, None)
     grp.x.copy_(x)
     y = torch.empty((S_r, cfg.H), dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream()
@@ -539,6 +547,7 @@ def time_ep(cfg, device, steps: int, warmup: int, wl: Workload | None = None):
         dist.barrier()
     grp.close()
     return {"workload": f"{cfg.name}: {cfg.describe()}", "ranks": world, "ms_per_step": ms,
+            "dtype": "mxfp8-e4m3" if cfg.mxfp8 else "bf16",
             "tokens_per_s": cfg.T / (ms / 1e3), "steps": steps,
             "note": "EpGroup.forward per step: all-gather of the logits, mok_plan, mok_ep_dispatch_ffn (barrier, "
                     "pull dispatch of this rank's experts' rows from the ranks' x, grouped SwiGLU FFN, push of "
