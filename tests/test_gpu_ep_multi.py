@@ -24,7 +24,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, q):
+def _rank_main(rank, world, port, q, mxfp8=False):
     import datetime
 
     import torch.distributed as dist
@@ -40,18 +40,24 @@ def _rank_main(rank, world, port, q):
         x = mokgen.tokens(cfg)
         logits = mokgen.router_logits(cfg, x)
         wg, wu, wd = mokgen.all_expert_weights(cfg)
-        grp = mok.EpGroup(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
+        grp = mok.EpGroup(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, mxfp8=mxfp8)
         S_r, e0, n = grp.S_r, grp.e0, grp.e_loc
         grp.x.copy_(x[rank * S_r:(rank + 1) * S_r].cuda())
         w = [t[e0:e0 + n].contiguous().cuda() for t in (wg, wu, wd)]
+        pack = lambda ws: tuple(t for wt in ws for t in mok.quantize_weights_mxfp8(wt))
+        if mxfp8:  # every rank holds at least one of the 10 experts
+            w = [pack(w), None, None]
         ok = True
         for _ in range(3):
             y = grp.forward(logits[rank * S_r:(rank + 1) * S_r].contiguous().cuda(), *w)
             ok &= grp.status() == mok.MOK_OK
         # the single-GPU staged forward of the whole layer, on this GPU
         p = mok.plan(logits.cuda(), cfg.k, world)
-        ys, _ = mok.moe_forward(mok.shards(x.cuda(), world), wg.cuda(), wu.cuda(), wd.cuda(), p, 0,
-                                mok.fwd_opts(mode=mok.MOK_MODE_STAGED))
+        full = [wg.cuda(), wu.cuda(), wd.cuda()]
+        if mxfp8:
+            ys, _ = mok.moe_forward_mxfp8(mok.shards(x.cuda(), world), pack(full), p)
+        else:
+            ys, _ = mok.moe_forward(mok.shards(x.cuda(), world), *full, p, 0, mok.fwd_opts(mode=mok.MOK_MODE_STAGED))
         torch.cuda.synchronize()
         ok &= torch.equal(y, ys[rank])
         dist.barrier()
@@ -64,11 +70,12 @@ def _rank_main(rank, world, port, q):
 
 
 @pytest.mark.skipif(torch.cuda.device_count() < WORLD, reason="needs two GPUs")
-def test_ep_forward_over_two_gpus_matches_single_gpu():
+@pytest.mark.parametrize("mxfp8", [False, True])
+def test_ep_forward_over_two_gpus_matches_single_gpu(mxfp8):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, WORLD, port, q)) for r in range(WORLD)]
+    procs = [ctx.Process(target=_rank_main, args=(r, WORLD, port, q, mxfp8)) for r in range(WORLD)]
     for p in procs:
         p.start()
     got = dict(q.get(timeout=300) for _ in range(WORLD))
