@@ -550,8 +550,8 @@ int mok_moe_forward_host_batches(int n, const void* const* x_host, const float* 
  *   mok_ep_combine(step s)       group barrier (every push of step s has
  *                                landed), then the fixed-order weighted
  *                                combine of this rank's tokens.
- * The results equal mok_moe_forward's staged bf16 path over the same plan,
- * bit for bit.
+ * The results equal mok_moe_forward's staged path (bf16 or MXFP8) over the
+ * same plan, bit for bit.
  * ---------------------------------------------------------------------- */
 
 /* How the ranks of a group are ordered between the two calls of a step:
@@ -632,8 +632,9 @@ int mok_ep_dispatch_ffn_mxfp8(const mok_plan_t* plan, const mok_ep_t* ep, int H,
  * (MOK_EP_SYNC_DEVICE; arrival number 2*step), then
  *   y[i] = bf16(sum_{j<k} gates[t,j] * out[t,j,:]),  t = g*S_r + i,
  * over the slot rows in this rank's slot buffer (ep->slots[ep->g]; fp16
- * with exponents, or bf16 when ep->mxfp8), fp32, j ascending.  y: [S_r, H] bf16, 16-byte aligned.  ws: the workspace given
- * to mok_ep_dispatch_ffn (its status word).  Asynchronous on `stream`.
+ * with exponents, or bf16 when ep->mxfp8), fp32, j ascending.
+ * y: [S_r, H] bf16, 16-byte aligned.  ws: the workspace given to the
+ * dispatch call (its status word).  Asynchronous on `stream`.
  */
 int mok_ep_combine(const mok_plan_t* plan, const mok_ep_t* ep, int H, uint32_t step,
                    uint64_t timeout_ns, void* y, void* ws, size_t ws_bytes, mok_stream_t stream);
