@@ -74,9 +74,12 @@ static cudaError_t launch_pair_phase(int grid, const GemmMaps& maps, const CoreA
 // used when the mean rows per expert is at most 192.  MOK_GEMM_GROUP and
 // MOK_GEMM_PAIR (0/1) override (tuning knobs only: results do not change).
 GemmTuning gemm_tuning(int rows, int E) {
-    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 3, 2};
+    GemmTuning v{2, rows <= 192 * E ? 1 : 0, 3, 2, 1};
     if (const char* s = getenv("MOK_GEMM_GROUP")) v.group_chunks = atoi(s) < 1 ? 1 : atoi(s);
-    if (const char* s = getenv("MOK_GEMM_PAIR")) v.pair = atoi(s) != 0;
+    if (const char* s = getenv("MOK_GEMM_PAIR")) {
+        v.pair = atoi(s) != 0;
+        v.gate_up_pair2 = 0;  // the explicit setting decides the gate/up unit shape too
+    }
     if (const char* s = getenv("MOK_GEMM_CTA_PAIR")) v.cta_pair = atoi(s) < 0 ? 0 : atoi(s);
     if (const char* s = getenv("MOK_MX_RINGS")) v.mx_rings = atoi(s) == 1 ? 1 : 2;
     return v;
@@ -160,16 +163,20 @@ cudaError_t launch_gemm_phase(int phase, const GemmMaps& maps, const MxMaps* mx,
     const int MT = (tiles + sub - 1) / sub;  // units along M
     const int GC = tune.group_chunks > 0 ? tune.group_chunks : 1;
     // CTA pairs (MOK_GEMM_CTA_PAIR): 0 none; 1 every bf16 launch but gate/up;
-    // 2 all, one M tile per CTA; 3 (default) as 1, and gate/up, where the
-    // M-tile pairing rule holds, on CTA pairs of two M tiles per CTA.  Needs
-    // an even number of M tiles (a multiple of 4 for two per CTA) and an
-    // even grid.  Measured on B200 (ncu launch times, one session each): down
-    // on CTA pairs 5 % faster than single tiles at the page shape and 1 % at
-    // the zipf shape; gate/up on CTA pairs of one tile 4 % slower than M-tile
+    // 2 all, one M tile per CTA; 3 (default) as 1, and gate/up on CTA pairs
+    // of two M tiles per CTA (MOK_GEMM_PAIR=0 keeps gate/up on single CTAs
+    // where the M-tile pairing rule does not hold).  Needs an even number of
+    // M tiles (a multiple of 4 for two per CTA) and an even grid.  Measured
+    // on B200 (ncu launch times or bench A/Bs, one session each): down on CTA
+    // pairs 5 % faster than single tiles at the page shape and 1 % at the
+    // zipf shape; gate/up on CTA pairs of one tile 4 % slower than M-tile
     // pairs (page) and 5 % slower than single tiles (zipf); gate/up on CTA
-    // pairs of two tiles 3 % faster than M-tile pairs (page); down on CTA
-    // pairs of two tiles slower than on CTA pairs of one (page).
-    if (tune.cta_pair == 3 && phase == 0 && pair && !mx && !bwd && tiles % 4 == 0 && grid >= 2)
+    // pairs of two tiles 3 % faster than M-tile pairs (page), 1-3 % faster
+    // than single tiles at the zipf shape (512 rows per expert) and 1.5 % at
+    // the Mixtral-shaped config (1024); down on CTA pairs of two tiles slower
+    // than on CTA pairs of one (page).
+    if (tune.cta_pair == 3 && phase == 0 && (pair || tune.gate_up_pair2) && !mx && !bwd && tiles % 4 == 0 &&
+        grid >= 2)
         return launch_pair_phase<Bf16Cta2PairCfg>(grid, maps, a, chunks, counts2, phase, tiles / 4, GC, stream);
     const bool cta2 = tune.cta_pair == 2 || ((tune.cta_pair == 1 || tune.cta_pair == 3) && phase != 0);
     if (cta2 && !mx && tiles % 2 == 0 && grid >= 2) {

@@ -103,6 +103,7 @@ struct GemmTuning {
     int cta_pair;      // bf16 launches on CTA pairs (tcgen05 cta_group::2): 0 none, 1 all but gate/up,
                        // 2 all, 3 as 1 plus gate/up with two M tiles per CTA when pairing
     int mx_rings;      // MXFP8 staged launches: 2 = weight and token rings, 1 = one ring of stages
+    int gate_up_pair2; // bf16 gate/up on CTA pairs of two M tiles at every shape (else where `pair` holds)
 };
 // defaults for `rows` expert-major rows over E experts, overridable by
 // MOK_GEMM_GROUP / MOK_GEMM_PAIR / MOK_GEMM_CTA_PAIR / MOK_MX_RINGS

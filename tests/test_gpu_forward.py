@@ -121,7 +121,7 @@ def test_grouped_gemm_m_tile_pairing_is_exact(name, monkeypatch):
     assert_bf16_close(decode_slots(got["1"], p.ns, cfg.H), want, name)
 
 
-@pytest.mark.parametrize("name", ["tiny", "many_experts", "wide", "k16"])
+@pytest.mark.parametrize("name", ["tiny", "many_experts", "wide", "k16", "multi_chunk"])
 def test_grouped_gemm_cta_pairs_are_exact(name, monkeypatch):
     """The same phases on CTA pairs (clusters of two CTAs, one M = 256 MMA
     over both CTAs' weight tiles, each CTA holding half of the token tile)
