@@ -213,3 +213,39 @@ def test_ep_group_exchanges_handles_and_logits_over_gloo(world):
         # the logits are gathered in rank order: rank h's rows carry h
         assert d["rows"] == list(range(world)) and d["shape"] == (8 * world, 10)
     assert e_next == 10
+
+
+def _rank_dies(rank, world, port, q):
+    """Rank 1 leaves before the group's handle exchange; rank 0's exchange
+    must end with an error (the process group's timeout or the broken
+    connection), not wait for ever."""
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    def leave(msg):
+        q.put((rank, msg))
+        q.close()
+        q.join_thread()  # the message is out before the process ends
+        os._exit(0)
+    if rank == 1:
+        leave("left")  # between steps, with nothing in flight
+    try:
+        mok.EpGroup(16, 128, 64, 4, 2, device="cpu", ipc=_fake_ipc([]))
+        msg = "no error"
+    except Exception as e:  # the failure seen on the host
+        msg = type(e).__name__
+    leave(msg)
+
+
+def test_ep_group_reports_a_rank_that_left():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+    assert got[1] == "left"
+    assert got[0] not in ("no error",), got
